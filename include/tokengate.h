@@ -1,0 +1,232 @@
+/*
+ * tokengate.h -- C ABI of libtokengate, a B200 (sm_100a) implementation of
+ * the data-parallel hot path of TokenGate's gated prefill.
+ *
+ * Sources (web pages about the TokenGate paper), cited below by tag:
+ *   [TC] Tencent Cloud developer article "TokenGate：端到端可训练的 Token 剪枝机制，
+ *        让大模型 Prefill 提速 11.3 倍"
+ *   [FW] farwalk.ai item "Researchers from Stanford and Berkeley propose
+ *        TokenGate, using learnable pruning to speed up long-context Prefill
+ *        by up to about 11x", section "论文的方法"
+ *   [AI] ai.866data.com article "让大模型学会"略读"：TokenGate如何破解长上下文推理
+ *        的效率困局", section "可学习剪枝的机制设计"
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - The caller owns all memory. Tensor arguments are DEVICE pointers unless
+ *    a comment says otherwise; the library allocates nothing. Scratch space
+ *    is passed as (ws, ws_bytes); tg_workspace_size() gives the size.
+ *  - Layouts are row-major and token-major. Weight matrices are stored
+ *    [out_features, in_features] (the nn.Linear layout).
+ *  - Activations and weight matrices use the call's tg_dtype (bf16 or fp32).
+ *    One-dimensional parameters (norm weights, scorer bias/w2, gain, tau) and
+ *    scores are always fp32. Indices and positions are int32.
+ *  - Calls are asynchronous on the given stream and never synchronise with
+ *    the host. Arguments are validated on the host before any launch; a bad
+ *    argument returns an error and launches nothing.
+ *  - Results are deterministic: the same inputs give the same bits.
+ *  - Device code never traps. Every wait inside a kernel is bounded; a wait
+ *    that runs out sets a sticky device error word, read by
+ *    tg_device_error().
+ */
+#ifndef TOKENGATE_H
+#define TOKENGATE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st* tg_stream;
+
+typedef enum {
+  TG_OK = 0,
+  TG_ERR_INVALID_ARG = 1, /* null pointer, bad size or unaligned pointer */
+  TG_ERR_UNSUPPORTED = 2, /* dtype / head_dim / width not built for     */
+  TG_ERR_BUDGET = 3,      /* k < 1 or k > n                              */
+  TG_ERR_WORKSPACE = 4,   /* ws_bytes smaller than tg_workspace_size()   */
+  TG_ERR_CUDA = 5         /* a CUDA call failed; see tg_last_cuda_error  */
+} tg_status;
+
+typedef enum { TG_F32 = 0, TG_BF16 = 1 } tg_dtype;
+
+typedef enum {
+  TG_OP_SCORE = 0,
+  TG_OP_TOPK_SELECT = 1,
+  TG_OP_COMPACT = 2,
+  TG_OP_GATED_ATTN = 3,
+  TG_OP_PREFILL = 4
+} tg_op;
+
+/* Sizes used to size a workspace; fields an op does not use are ignored. */
+typedef struct {
+  int64_t n;        /* tokens entering the gate                        */
+  int64_t k;        /* tokens kept (rows of the gated attention)        */
+  int32_t d_model;
+  int32_t n_heads_q;
+  int32_t n_heads_kv;
+  int32_t head_dim;
+  int32_t d_score;  /* scorer hidden width F                           */
+  int32_t d_ffn;    /* SwiGLU intermediate width I (0: no FFN)          */
+  int32_t n_layers;
+  int32_t gate_layer;
+  tg_dtype dtype;
+} tg_shape;
+
+/* Bytes of scratch the op needs for these sizes (0 if none). */
+size_t tg_workspace_size(tg_op op, const tg_shape* shape);
+
+/*
+ * tg_score -- importance score of every token.
+ *   s_t = w2 . SiLU(W1 . RMSNorm(x_t; norm_w, eps) + b1) + b2
+ * A small MLP reads each token's post-attention residual at the gate layer
+ * and emits one scalar ([TC] "TokenGate 提前筛选 Token"; [AI]). The pages do
+ * not fix the MLP's inner form; this library uses RMSNorm -> Linear(d->f) ->
+ * SiLU -> Linear(f->1).
+ *   x       [n, d] dtype       norm_w [d] fp32     w1 [f, d] dtype
+ *   b1      [f] fp32 or NULL   w2 [f] fp32         b2 [1] fp32 or NULL
+ *   scores  [n] fp32 (out)
+ * bf16 needs f % 16 == 0, f <= 256, d % 8 == 0; fp32 any f <= 1024.
+ */
+tg_status tg_score(const void* x, int64_t n, int32_t d, int32_t f, const float* norm_w, float eps,
+                   const void* w1, const float* b1, const float* w2, const float* b2, tg_dtype dtype,
+                   float* scores, void* ws, size_t ws_bytes, tg_stream stream);
+
+/*
+ * tg_topk_select -- the kept set.
+ * Keeps exactly k tokens: every protected token (protect[i] != 0) plus the
+ * k - P best unprotected tokens ranked by (score descending, index
+ * ascending); -0.0 ranks equal to +0.0 and NaN below -inf. kept_idx is
+ * written ascending. The top-K selector and the un-prunable question span
+ * are from [TC] "TokenGate 提前筛选 Token" and [AI]; the tie order is this
+ * library's choice (deterministic).
+ *   scores  [n] fp32           protect [n] uint8 or NULL (none protected)
+ *   kept_idx [k] int32 (out)
+ * If more than k tokens are protected (known only on the device), kept_idx
+ * is filled with -1 and the workspace's first int32 is set to TG_ERR_BUDGET
+ * (it is TG_OK otherwise).
+ */
+tg_status tg_topk_select(const float* scores, const uint8_t* protect, int64_t n, int64_t k,
+                         int32_t* kept_idx, void* ws, size_t ws_bytes, tg_stream stream);
+
+/*
+ * tg_compact -- gather of the kept rows.
+ *   x_out[r] = x[kept_idx[r]], pos_out[r] = pos_in[kept_idx[r]] (or
+ *   kept_idx[r] when pos_in is NULL), scores_out[r] = scores[kept_idx[r]].
+ * Only the kept tokens continue into the layers above the gate, carrying
+ * their original positions ([TC] "TokenGate 提前筛选 Token"; [FW]).
+ *   x [n, d] dtype, pos_in [n] int32 or NULL, scores [n] fp32 or NULL,
+ *   kept_idx [k] int32 with every entry in [0, n) (checked on the device:
+ *   an entry out of range writes a zero row and sets the device error word).
+ *   x_out [k, d], pos_out [k], scores_out [k] or NULL.
+ * x and x_out rows must be 16-byte aligned (d * elem % 16 == 0).
+ */
+tg_status tg_compact(const void* x, const int32_t* pos_in, const float* scores,
+                     const int32_t* kept_idx, int64_t n, int64_t k, int32_t d, tg_dtype dtype,
+                     void* x_out, int32_t* pos_out, float* scores_out, tg_stream stream);
+
+/*
+ * tg_gated_attn_prefill -- token-gated causal GQA attention over the kept rows.
+ *   l_ij = (q_i . k_j) / (sqrt(dh) * tau_h) + gain_h * logsigmoid(s_j),
+ *   for pos_j <= pos_i; o_i = sum_j softmax_j(l_ij) v_j.
+ * The kept tokens' scores enter the attention logits of the layers above the
+ * gate as a bias, with a learnable per-head gain and temperature ([TC]
+ * "门控机制为评分网络建立梯度路径"; [AI]). The pages state the bias only in
+ * words; the formula above is this library's reading. q and kk are rotated
+ * here by RoPE (rotate-half, theta_i = rope_base^(-2i/dh)) at the original
+ * positions pos. Query head h reads KV head h / (hq / hkv).
+ *   q [k, hq, dh], kk [k, hkv, dh], v [k, hkv, dh] dtype (un-rotated)
+ *   pos [k] int32 strictly ascending; s [k] fp32 or NULL (no bias)
+ *   gain [hq] fp32 or NULL (0); tau [hq] fp32 > 0 or NULL (1)
+ *   out [k, hq, dh] dtype
+ * bf16 needs dh == 128; fp32 needs dh in {64, 128}. hq % hkv == 0.
+ */
+tg_status tg_gated_attn_prefill(const void* q, const void* kk, const void* v, const int32_t* pos,
+                                const float* s, const float* gain, const float* tau, int64_t k,
+                                int32_t hq, int32_t hkv, int32_t dh, float rope_base,
+                                tg_dtype dtype, void* out, void* ws, size_t ws_bytes,
+                                tg_stream stream);
+
+/* ---- the full stack ---------------------------------------------------- */
+
+typedef struct {
+  const float* attn_norm; /* [d]                                               */
+  const void* wqkv;       /* [(hq + 2 hkv) dh, d]: rows of Wq, then Wk, then Wv */
+  const float* q_norm;    /* [dh] per-head RMSNorm weight of q; NULL = off      */
+  const float* k_norm;    /* [dh] same for k (both or neither)                  */
+  const void* wo;         /* [d, hq dh]                                        */
+  const float* ffn_norm;  /* [d]                                               */
+  const void* w_gate_up;  /* [2 I, d]: rows of W_gate, then W_up; NULL = no FFN */
+  const void* w_down;     /* [d, I]                                            */
+  const float* gain;      /* [hq] gate-bias gain, layers above the gate; NULL=0 */
+  const float* tau;       /* [hq] temperature, layers above the gate; NULL = 1  */
+} tg_layer;
+
+typedef struct {
+  tg_dtype dtype;
+  int32_t n_layers, d_model, n_heads_q, n_heads_kv, head_dim, d_ffn, d_score;
+  float norm_eps, rope_base;
+  const tg_layer* layers;   /* HOST array of n_layers entries (device pointers inside) */
+  const float* final_norm;  /* [d] or NULL (no final norm)                    */
+  const float* score_norm;  /* [d]                                           */
+  const void* score_w1;     /* [F, d]                                        */
+  const float* score_b1;    /* [F] or NULL                                   */
+  const float* score_w2;    /* [F]                                           */
+  const float* score_b2;    /* [1] or NULL                                   */
+} tg_model;
+
+/* Per-layer KV outputs (post-RoPE keys, values), each [rows, hkv, dh] dtype.
+ * rows = n for layers <= gate_layer, k above it. NULL pointers skip a layer. */
+typedef struct {
+  void* k;
+  void* v;
+} tg_kv;
+
+/*
+ * tg_prefill -- the gated prefill of a decoder stack ([TC] "TokenGate 提前筛选
+ * Token"; [FW]; [AI]).
+ * Layers below gate_layer L run over all n tokens. Layer L runs attention
+ * over all n tokens; the scorer reads its post-attention residual; the
+ * selector keeps k tokens (protected ones always); layer L's FFN and every
+ * layer above run over the k kept rows only, with token-gated attention at
+ * the kept tokens' original positions, and make KV for those rows only.
+ * Layers at and below L keep n-row KV ([TC] "TokenGate 的工程验证仍有限").
+ * gate_layer = -1 puts the gate before layer 0 (the scorer reads x itself).
+ * With k == n and every gain NULL/0 and tau NULL/1 the call is a dense
+ * prefill.
+ *   x [n, d] dtype (input hidden states); protect [n] uint8 or NULL
+ *   out [k, d] dtype: final-normed hidden states of the kept rows
+ *   kept_idx [k] int32 (out, ascending); scores [n] fp32 (out) or NULL
+ *   kv: HOST array of n_layers tg_kv, or NULL
+ */
+tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protect, int64_t n,
+                     int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx, float* scores,
+                     const tg_kv* kv, void* ws, size_t ws_bytes, tg_stream stream);
+
+/* ---- diagnostics -------------------------------------------------------- */
+
+/* Static description of a status code. */
+const char* tg_status_string(tg_status status);
+
+/* The CUDA error behind the last TG_ERR_CUDA on this host thread (0 if none). */
+int tg_last_cuda_error(void);
+
+/*
+ * Reads (and with clear != 0, resets) the sticky device error word of the
+ * current device: 0 when no kernel has reported a problem. Nonzero bits:
+ * 1 = a bounded wait ran out, 2 = an index out of range was skipped.
+ * This call synchronises the current device (a diagnostic, not for hot loops).
+ */
+tg_status tg_device_error(uint32_t* word, int clear);
+
+/* Library version string. */
+const char* tg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TOKENGATE_H */

@@ -1,0 +1,289 @@
+"""Python binding of libtokengate, the B200 (sm_100a) gated-prefill library.
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+PyTorch supplies device memory (tensors, workspaces) and streams. The names
+mirror the C ABI in include/tokengate.h.
+
+The shared library is built in-tree (``python -m
+learned_token_pruning_score_b200._build``); importing this package without
+it raises ImportError -- there is no fallback path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Dict, List, Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtokengate.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is not built; run `python -m learned_token_pruning_score_b200._build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+# ----------------------------------------------------------------- ABI types
+
+TG_OK, TG_ERR_INVALID_ARG, TG_ERR_UNSUPPORTED, TG_ERR_BUDGET, TG_ERR_WORKSPACE, TG_ERR_CUDA = range(6)
+TG_F32, TG_BF16 = 0, 1
+TG_OP_SCORE, TG_OP_TOPK_SELECT, TG_OP_COMPACT, TG_OP_GATED_ATTN, TG_OP_PREFILL = range(5)
+
+_c_i32, _c_i64, _c_f32, _c_p, _c_sz = (ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                                       ctypes.c_void_p, ctypes.c_size_t)
+
+
+class TgShape(ctypes.Structure):
+    _fields_ = [("n", _c_i64), ("k", _c_i64), ("d_model", _c_i32), ("n_heads_q", _c_i32),
+                ("n_heads_kv", _c_i32), ("head_dim", _c_i32), ("d_score", _c_i32),
+                ("d_ffn", _c_i32), ("n_layers", _c_i32), ("gate_layer", _c_i32),
+                ("dtype", ctypes.c_int)]
+
+
+class TgLayer(ctypes.Structure):
+    _fields_ = [(n, _c_p) for n in ("attn_norm", "wqkv", "q_norm", "k_norm", "wo", "ffn_norm",
+                                    "w_gate_up", "w_down", "gain", "tau")]
+
+
+class TgModel(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("n_layers", _c_i32), ("d_model", _c_i32),
+                ("n_heads_q", _c_i32), ("n_heads_kv", _c_i32), ("head_dim", _c_i32),
+                ("d_ffn", _c_i32), ("d_score", _c_i32), ("norm_eps", _c_f32),
+                ("rope_base", _c_f32), ("layers", ctypes.POINTER(TgLayer)),
+                ("final_norm", _c_p), ("score_norm", _c_p), ("score_w1", _c_p),
+                ("score_b1", _c_p), ("score_w2", _c_p), ("score_b2", _c_p)]
+
+
+class TgKV(ctypes.Structure):
+    _fields_ = [("k", _c_p), ("v", _c_p)]
+
+
+def _sig(name, res, *args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = list(args)
+    return f
+
+
+_ci = ctypes.c_int
+_workspace_size = _sig("tg_workspace_size", _c_sz, _ci, ctypes.POINTER(TgShape))
+_score = _sig("tg_score", _ci, _c_p, _c_i64, _c_i32, _c_i32, _c_p, _c_f32, _c_p, _c_p, _c_p, _c_p,
+              _ci, _c_p, _c_p, _c_sz, _c_p)
+_topk = _sig("tg_topk_select", _ci, _c_p, _c_p, _c_i64, _c_i64, _c_p, _c_p, _c_sz, _c_p)
+_compact = _sig("tg_compact", _ci, _c_p, _c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i32, _ci, _c_p,
+                _c_p, _c_p, _c_p)
+_attn = _sig("tg_gated_attn_prefill", _ci, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i64,
+             _c_i32, _c_i32, _c_i32, _c_f32, _ci, _c_p, _c_p, _c_sz, _c_p)
+_prefill = _sig("tg_prefill", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64, _c_i64, _c_i32,
+                _c_p, _c_p, _c_p, ctypes.POINTER(TgKV), _c_p, _c_sz, _c_p)
+_status_string = _sig("tg_status_string", ctypes.c_char_p, _ci)
+_last_cuda_error = _sig("tg_last_cuda_error", _ci)
+_device_error = _sig("tg_device_error", _ci, ctypes.POINTER(ctypes.c_uint32), _ci)
+_version = _sig("tg_version", ctypes.c_char_p)
+
+
+class TokenGateError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = f"{where}: {tg_status_string(status)}"
+        if status == TG_ERR_CUDA:
+            msg += f" (cudaError {_last_cuda_error()})"
+        super().__init__(msg)
+        self.status = status
+
+
+def _check(status: int, where: str) -> None:
+    if status != TG_OK:
+        raise TokenGateError(status, where)
+
+
+# ----------------------------------------------------------------- helpers
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return TG_BF16
+    if t.dtype == torch.float32:
+        return TG_F32
+    raise ValueError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libtokengate must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream, device) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ws(nbytes: int, device, ws: Optional[torch.Tensor]) -> torch.Tensor:
+    if ws is None:
+        return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+    if ws.numel() * ws.element_size() < nbytes:
+        raise ValueError(f"workspace too small: {ws.numel() * ws.element_size()} < {nbytes}")
+    return ws
+
+
+def tg_status_string(status: int) -> str:
+    return _status_string(status).decode()
+
+
+def tg_version() -> str:
+    return _version().decode()
+
+
+def tg_workspace_size(op: int, n=0, k=0, d_model=0, n_heads_q=0, n_heads_kv=0, head_dim=0,
+                      d_score=0, d_ffn=0, n_layers=0, gate_layer=0, dtype=TG_BF16) -> int:
+    s = TgShape(n, k, d_model, n_heads_q, n_heads_kv, head_dim, d_score, d_ffn, n_layers,
+                gate_layer, dtype)
+    return int(_workspace_size(op, ctypes.byref(s)))
+
+
+def tg_device_error(clear: bool = False) -> int:
+    w = ctypes.c_uint32(0)
+    _check(_device_error(ctypes.byref(w), int(clear)), "tg_device_error")
+    return int(w.value)
+
+
+# ----------------------------------------------------------------- the calls
+
+
+def tg_score(x, norm_w, w1, w2, b1=None, b2=None, eps: float = 1e-6, scores=None, ws=None,
+             stream=None) -> torch.Tensor:
+    n, d = x.shape
+    f = w1.shape[0]
+    if scores is None:
+        scores = torch.empty(n, dtype=torch.float32, device=x.device)
+    dt = _dt(x)
+    need = tg_workspace_size(TG_OP_SCORE, n=n, d_model=d, d_score=f, dtype=dt)
+    ws = _ws(need, x.device, ws)
+    _check(_score(_ptr(x), n, d, f, _ptr(norm_w), eps, _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), dt,
+                  _ptr(scores), _ptr(ws), ws.numel(), _stream(stream, x.device)), "tg_score")
+    return scores
+
+
+def tg_topk_select(scores, protect, k: int, kept_idx=None, ws=None, stream=None) -> torch.Tensor:
+    n = scores.shape[0]
+    if kept_idx is None:
+        kept_idx = torch.empty(k, dtype=torch.int32, device=scores.device)
+    need = tg_workspace_size(TG_OP_TOPK_SELECT, n=n)
+    ws = _ws(need, scores.device, ws)
+    _check(_topk(_ptr(scores), _ptr(protect), n, k, _ptr(kept_idx), _ptr(ws), ws.numel(),
+                 _stream(stream, scores.device)), "tg_topk_select")
+    return kept_idx
+
+
+def tg_compact(x, kept_idx, pos_in=None, scores=None, x_out=None, pos_out=None, scores_out=None,
+               stream=None):
+    n, d = x.shape
+    k = kept_idx.shape[0]
+    if x_out is None:
+        x_out = torch.empty(k, d, dtype=x.dtype, device=x.device)
+    if pos_out is None:
+        pos_out = torch.empty(k, dtype=torch.int32, device=x.device)
+    if scores is not None and scores_out is None:
+        scores_out = torch.empty(k, dtype=torch.float32, device=x.device)
+    _check(_compact(_ptr(x), _ptr(pos_in), _ptr(scores), _ptr(kept_idx), n, k, d, _dt(x),
+                    _ptr(x_out), _ptr(pos_out), _ptr(scores_out), _stream(stream, x.device)),
+           "tg_compact")
+    return x_out, pos_out, scores_out
+
+
+def tg_gated_attn_prefill(q, k, v, pos, s=None, gain=None, tau=None, rope_base: float = 1e6,
+                          out=None, ws=None, stream=None) -> torch.Tensor:
+    t, hq, dh = q.shape
+    hkv = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    dt = _dt(q)
+    need = tg_workspace_size(TG_OP_GATED_ATTN, k=t, n_heads_q=hq, n_heads_kv=hkv, head_dim=dh,
+                             dtype=dt)
+    ws = _ws(need, q.device, ws)
+    _check(_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), _ptr(s), _ptr(gain), _ptr(tau), t, hq, hkv,
+                 dh, rope_base, dt, _ptr(out), _ptr(ws), ws.numel(), _stream(stream, q.device)),
+           "tg_gated_attn_prefill")
+    return out
+
+
+@dataclass
+class Model:
+    """Device tensors of a decoder stack plus the ctypes view tg_prefill takes.
+
+    layers: one dict per layer with keys attn_norm, wqkv, wo, ffn_norm,
+    w_gate_up, w_down (optional), q_norm/k_norm (optional), gain/tau
+    (optional; used above the gate). Matrices in the model dtype, vectors fp32.
+    """
+
+    n_heads_q: int
+    n_heads_kv: int
+    head_dim: int
+    layers: List[Dict[str, torch.Tensor]]
+    score: Dict[str, torch.Tensor]  # score_norm, score_w1, score_w2, score_b1?, score_b2?
+    final_norm: Optional[torch.Tensor] = None
+    eps: float = 1e-6
+    rope_base: float = 1e6
+
+    def __post_init__(self):
+        w = self.layers[0]["wqkv"]
+        self.dtype = _dt(w)
+        self.d_model = w.shape[1]
+        gu = self.layers[0].get("w_gate_up")
+        self.d_ffn = 0 if gu is None else gu.shape[0] // 2
+        self.d_score = self.score["score_w1"].shape[0]
+        arr = (TgLayer * len(self.layers))()
+        for i, lw in enumerate(self.layers):
+            for name, _ in TgLayer._fields_:
+                setattr(arr[i], name, _ptr(lw.get(name)))
+        self._layers_c = arr
+        self.c = TgModel(self.dtype, len(self.layers), self.d_model, self.n_heads_q,
+                         self.n_heads_kv, self.head_dim, self.d_ffn, self.d_score, self.eps,
+                         self.rope_base, arr, _ptr(self.final_norm),
+                         _ptr(self.score["score_norm"]), _ptr(self.score["score_w1"]),
+                         _ptr(self.score.get("score_b1")), _ptr(self.score["score_w2"]),
+                         _ptr(self.score.get("score_b2")))
+
+    def workspace_size(self, n: int, k: int, gate_layer: int) -> int:
+        return tg_workspace_size(TG_OP_PREFILL, n=n, k=k, d_model=self.d_model,
+                                 n_heads_q=self.n_heads_q, n_heads_kv=self.n_heads_kv,
+                                 head_dim=self.head_dim, d_score=self.d_score, d_ffn=self.d_ffn,
+                                 n_layers=len(self.layers), gate_layer=gate_layer,
+                                 dtype=self.dtype)
+
+
+def tg_prefill(model: Model, x, protect, k: int, gate_layer: int, out=None, kept_idx=None,
+               scores=None, kv: Optional[Sequence] = None, ws=None, stream=None):
+    """Returns (out [k, d], kept_idx [k], scores [n] or None)."""
+    n, d = x.shape
+    if out is None:
+        out = torch.empty(k, d, dtype=x.dtype, device=x.device)
+    if kept_idx is None:
+        kept_idx = torch.empty(k, dtype=torch.int32, device=x.device)
+    ws = _ws(model.workspace_size(n, k, gate_layer), x.device, ws)
+    kv_c = None
+    if kv is not None:
+        kv_c = (TgKV * len(model.layers))()
+        for i, pair in enumerate(kv):
+            if pair is not None:
+                kv_c[i].k, kv_c[i].v = _ptr(pair[0]), _ptr(pair[1])
+    _check(_prefill(ctypes.byref(model.c), _ptr(x), _ptr(protect), n, k, gate_layer, _ptr(out),
+                    _ptr(kept_idx), _ptr(scores), kv_c, _ptr(ws), ws.numel(),
+                    _stream(stream, x.device)), "tg_prefill")
+    return out, kept_idx, scores
+
+
+__all__ = [
+    "tg_score", "tg_topk_select", "tg_compact", "tg_gated_attn_prefill", "tg_prefill",
+    "tg_workspace_size", "tg_status_string", "tg_device_error", "tg_version", "Model",
+    "TokenGateError", "LIB_PATH", "TG_OK", "TG_ERR_INVALID_ARG", "TG_ERR_UNSUPPORTED",
+    "TG_ERR_BUDGET", "TG_ERR_WORKSPACE", "TG_ERR_CUDA", "TG_F32", "TG_BF16", "TG_OP_SCORE",
+    "TG_OP_TOPK_SELECT", "TG_OP_COMPACT", "TG_OP_GATED_ATTN", "TG_OP_PREFILL",
+]

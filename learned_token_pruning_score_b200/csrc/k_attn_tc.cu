@@ -1,0 +1,322 @@
+// k_attn_tc.cu -- token-gated causal GQA attention on the 5th-generation
+// tensor cores (sm_100a), bf16 operands, fp32 accumulation and softmax.
+//
+// For the kept rows i, j (compacted order; positions ascend with the row):
+//   l_ij = (q_i . k_j) / (sqrt(dh) * tau_h) + gain_h * logsigmoid(s_j),  j <= i
+//   o_i  = sum_j softmax_j(l_ij) v_j
+// The kept tokens' gate scores enter the logits of the upper layers' attention
+// as a bias, with a learnable per-head gain and a per-head temperature that
+// compensates the sharper softmax over fewer keys (Tencent Cloud article
+// "TokenGate：端到端可训练的 Token 剪枝机制，让大模型 Prefill 提速 11.3 倍", section
+// "门控机制为评分网络建立梯度路径"; ai.866data.com article "让大模型学会"略读"…",
+// section "可学习剪枝的机制设计"). The pages' own kernel was a FlashAttention-2
+// variant with a per-key bias (section "TokenGate 的工程验证仍有限"); this is a
+// new design for sm_100a. With gain = 0 and tau = 1 it is plain causal
+// attention (the dense layers below the gate use it that way).
+//
+// One CTA per (128-row query tile, query head); heavy (late) tiles first.
+//   warp 0     TMA: Q tile once; K and V^T tiles (128 keys) into a 2-deep ring.
+//   warp 1     MMA: S_j = Q K_j^T into one of two TMEM S buffers (issued one
+//              tile ahead), then O += P_j V_j into a TMEM O accumulator.
+//   warps 4-7  softmax, one thread per query row: tcgen05.ld of its S row,
+//              scale + gate bias (log2 domain), causal mask, running max with
+//              lazy rescaling (O and l are rescaled only when the max grows
+//              by more than 2^8), P = exp2(...) written bf16 to shared memory
+//              in the 128-byte-swizzled K-major layout the MMA reads.
+//   end        O / l read from TMEM, written bf16.
+// TMEM: S0 = cols [0,128), S1 = [128,256), O = [256,384) of 512.
+#include "tg_device.cuh"
+#include "tg_internal.h"
+
+namespace tg {
+namespace {
+
+constexpr int kBlk = 128;         // query rows per tile = keys per KV tile
+constexpr int kDh = 128;
+constexpr int kThreads = 256;
+constexpr int kSub = 128 * 128;   // bytes of one [128 rows x 64 bf16] swizzled sub-tile
+constexpr int kTile = 2 * kSub;   // [128 x 128] bf16 tile
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kTile;          // 2 stages
+constexpr int kOffV = kOffK + 2 * kTile;      // 2 stages
+constexpr int kOffP = kOffV + 2 * kTile;      // 2 buffers
+constexpr int kOffBar = kOffP + 2 * kTile;
+constexpr size_t kSmem = 1024 + kOffBar + 256;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThresh = 8.0f;  // log2 units
+
+struct Params {
+  int64_t T;
+  int hq, hkv;
+  int n_qtiles;
+  const float* lsig;
+  const float* gain;
+  const float* tau;
+  __nv_bfloat16* out;
+  unsigned int* err;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+            const __grid_constant__ CUtensorMap tmV, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* p_full = bars + 7;    // [2]
+  uint64_t* pv_done = bars + 9;   // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x / p.hq);  // heavy first
+  const int head = static_cast<int>(blockIdx.x % p.hq);
+  const int g = head / (p.hq / p.hkv);
+  const int q0 = qt * kBlk;
+  const int n_kv = qt + 1;  // causal: KV tiles 0..qt
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&pv_done[i], 1);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 2) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------- TMA producer
+    mbar_arrive_expect_tx(q_full, kTile);
+    tma_load_3d(&tmQ, q_full, smem + kOffQ, 0, head, q0);
+    tma_load_3d(&tmQ, q_full, smem + kOffQ + kSub, 64, head, q0);
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j & 1;
+      if (!mbar_wait(&kv_empty[s], ((j >> 1) & 1) ^ 1, p.err)) break;
+      mbar_arrive_expect_tx(&kv_full[s], 2 * kTile);
+      uint8_t* kd = smem + kOffK + s * kTile;
+      uint8_t* vd = smem + kOffV + s * kTile;
+      tma_load_3d(&tmK, &kv_full[s], kd, 0, g, j * kBlk);
+      tma_load_3d(&tmK, &kv_full[s], kd + kSub, 64, g, j * kBlk);
+      tma_load_3d(&tmV, &kv_full[s], vd, j * kBlk, 0, g);
+      tma_load_3d(&tmV, &kv_full[s], vd + kSub, j * kBlk + 64, 0, g);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+    const uint32_t q_addr = smem_addr(smem + kOffQ);
+    auto issue_qk = [&](int j) {
+      const int s = j & 1;
+      const uint32_t k_addr = smem_addr(smem + kOffK + s * kTile);
+      const uint32_t d = tmem + static_cast<uint32_t>(s * 128);
+#pragma unroll
+      for (int kk = 0; kk < kDh / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
+        umma_f16_ss(d, sdesc_kmajor_sw128(q_addr + off), sdesc_kmajor_sw128(k_addr + off), idesc,
+                    kk > 0 ? 1u : 0u);
+      }
+      umma_commit(&s_full[s]);
+    };
+    bool ok = mbar_wait(q_full, 0, p.err) && mbar_wait(&kv_full[0], 0, p.err);
+    if (ok) {
+      tc_fence_after();
+      issue_qk(0);
+    }
+    for (int j = 0; j < n_kv && ok; ++j) {
+      if (j + 1 < n_kv) {
+        if (!mbar_wait(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1, p.err)) break;
+        tc_fence_after();
+        issue_qk(j + 1);
+      }
+      const int b = j & 1;
+      if (!mbar_wait(&p_full[b], (j >> 1) & 1, p.err)) break;
+      tc_fence_after();
+      const uint32_t p_addr = smem_addr(smem + kOffP + b * kTile);
+      const uint32_t v_addr = smem_addr(smem + kOffV + b * kTile);
+#pragma unroll
+      for (int kk = 0; kk < kBlk / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
+        umma_f16_ss(tmem + 256, sdesc_kmajor_sw128(p_addr + off),
+                    sdesc_kmajor_sw128(v_addr + off), idesc, (j > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(&kv_empty[b]);
+      umma_commit(&pv_done[b]);
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------- softmax
+    const int r = threadIdx.x - 128;  // row within the tile = TMEM lane
+    const int64_t q_row = static_cast<int64_t>(q0) + r;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float tau = p.tau ? __ldg(p.tau + head) : 1.0f;
+    const float scale2 = kLog2e / (sqrtf(static_cast<float>(kDh)) * tau);
+    const float gb2 = (p.gain && p.lsig) ? __ldg(p.gain + head) * kLog2e : 0.0f;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int b = j & 1;
+      if (!mbar_wait_warp(&s_full[b], (j >> 1) & 1, p.err)) { ok = false; break; }
+      tc_fence_after();
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float t[32];
+        tmem_ld32_wait(tmem + lane_off + static_cast<uint32_t>(b * 128 + c * 32), t);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[c * 32 + i] = t[i];
+      }
+      const int kv0 = j * kBlk;
+      float rmax = -INFINITY;
+      const bool diag = (j == n_kv - 1);
+      if (gb2 != 0.0f) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          const int col = kv0 + i;
+          const float bias = col < p.T ? __ldg(p.lsig + col) : 0.0f;
+          x[i] = fmaf(x[i], scale2, gb2 * bias);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) x[i] *= scale2;
+      }
+      if (diag) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (kv0 + i > q_row) x[i] = -INFINITY;
+      }
+#pragma unroll
+      for (int i = 0; i < 128; ++i) rmax = fmaxf(rmax, x[i]);
+      float alpha = 1.0f;
+      if (rmax > m + kRescaleThresh || m == -INFINITY) {
+        alpha = ex2(m - rmax);  // 0 on the first tile
+        l *= alpha;
+        m = rmax;
+      }
+      // TMEM loads/stores are warp-collective: the warp rescales its 32 O
+      // rows together (alpha = 1 for rows whose max did not move).
+      const bool rescale_o = j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f);
+      float rsum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        x[i] = ex2(x[i] - m);
+        rsum += x[i];
+      }
+      l += rsum;
+      // P buffer b is free once PV_{j-2} has completed; when O must be
+      // rescaled, PV_{j-1} must have completed too (it implies PV_{j-2}).
+      if (rescale_o) {
+        if (!mbar_wait_warp(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.err)) { ok = false; break; }
+      } else if (j >= 2) {
+        if (!mbar_wait_warp(&pv_done[b], ((j - 2) >> 1) & 1, p.err)) { ok = false; break; }
+      }
+      tc_fence_after();
+      uint8_t* pb = smem + kOffP + b * kTile;
+#pragma unroll
+      for (int cidx = 0; cidx < 16; ++cidx) {
+        const int hs = cidx >> 3, c = cidx & 7;
+        uint4 u;
+        u.x = pack_bf16x2(x[cidx * 8 + 0], x[cidx * 8 + 1]);
+        u.y = pack_bf16x2(x[cidx * 8 + 2], x[cidx * 8 + 3]);
+        u.z = pack_bf16x2(x[cidx * 8 + 4], x[cidx * 8 + 5]);
+        u.w = pack_bf16x2(x[cidx * 8 + 6], x[cidx * 8 + 7]);
+        *reinterpret_cast<uint4*>(pb + hs * kSub + r * 128 + ((c ^ (r & 7)) << 4)) = u;
+      }
+      if (rescale_o) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          const uint32_t ta = tmem + lane_off + 256u + static_cast<uint32_t>(c * 32);
+          tmem_ld32_wait(ta, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32_wait(ta, o);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[b]);
+    }
+    if (ok && mbar_wait_warp(&pv_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, p.err)) {
+      tc_fence_after();
+      const float inv = 1.0f / l;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        tmem_ld32_wait(tmem + lane_off + 256u + static_cast<uint32_t>(c * 32), o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] *= inv;
+        if (q_row < p.T) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (q_row * p.hq + head) * kDh + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 u;
+            u.x = pack_bf16x2(o[8 * v + 0], o[8 * v + 1]);
+            u.y = pack_bf16x2(o[8 * v + 2], o[8 * v + 3]);
+            u.z = pack_bf16x2(o[8 * v + 4], o[8 * v + 5]);
+            u.w = pack_bf16x2(o[8 * v + 6], o[8 * v + 7]);
+            dst[v] = u;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+bool attn_tc_supported(const AttnArgs& a) {
+  auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+  return a.dh == kDh && a.hq % a.hkv == 0 && a.t_pad % 64 == 0 && a.t_pad >= a.T && al16(a.q) &&
+         al16(a.k) && al16(a.v) && al16(a.out) && a.T < (int64_t(1) << 31) - kBlk;
+}
+
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
+  if (a.T <= 0) return cudaSuccess;
+  CUtensorMap tq, tk, tv;
+  const int64_t e = 2;
+  if (!make_tmap_3d_bf16(&tq, a.q, kDh, a.hq, a.T, kDh * e, int64_t(a.hq) * kDh * e, 1, kBlk))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_3d_bf16(&tk, a.k, kDh, a.hkv, a.T, kDh * e, int64_t(a.hkv) * kDh * e, 1, kBlk))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_3d_bf16(&tv, a.v, a.t_pad, kDh, a.hkv, a.t_pad * e, a.t_pad * kDh * e, kDh, 1))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.T = a.T;
+  p.hq = a.hq;
+  p.hkv = a.hkv;
+  p.n_qtiles = static_cast<int>((a.T + kBlk - 1) / kBlk);
+  p.lsig = a.lsig;
+  p.gain = a.gain;
+  p.tau = a.tau;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.err = device_error_word();
+  cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(attn_tc), int(kSmem));
+  if (err != cudaSuccess) return err;
+  const unsigned grid = static_cast<unsigned>(p.n_qtiles) * static_cast<unsigned>(a.hq);
+  attn_tc<<<grid, kThreads, kSmem, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace tg

@@ -1,0 +1,298 @@
+// k_gemm_tc.cu -- bf16 GEMM on the 5th-generation tensor cores (sm_100a).
+//
+//   C[M, N] = A[M, K] . B[N, K]^T   (both operands K-major, fp32 accumulate)
+//
+// Used for every dense contraction of the path: the scorer's first layer,
+// QKV, the output projection, SwiGLU gate/up and down. Epilogues fused into
+// the TMEM read-out: plain store, residual add (x + W.o), SwiGLU
+// (SiLU(gate) * up, with gate and up tiles side by side in one 256-wide
+// accumulator), and the scorer's tail s = w2 . SiLU(h + b1) + b2 (all F <= 256
+// hidden units of a row sit in one accumulator row, so the dot is
+// thread-local).
+//
+// Structure: persistent CTAs (one per SM), 8 warps.
+//   warp 0    TMA producer: A tile [128 x 64] + B tile [BN x 64] per stage,
+//             128-byte swizzle, STAGES-deep ring of full/empty mbarriers.
+//   warp 1    MMA issuer: one thread issues tcgen05.mma (M=128, N=BN, K=16)
+//             x4 per stage into a TMEM accumulator, commits to free the stage.
+//   warp 2    TMEM allocation (2 x BN columns: double-buffered accumulator).
+//   warps 4-7 epilogue: tcgen05.ld of their 32-lane quarter, fused op, store.
+// The epilogue of tile t overlaps the MMAs of tile t+1.
+#include "tg_device.cuh"
+#include "tg_internal.h"
+
+namespace tg {
+namespace {
+
+constexpr int kBM = 128, kBK = 64;
+constexpr int kThreads = 256;
+
+template <int kBN>
+struct Cfg {
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = kBN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = kBN == 256 ? 4 : 6;
+  static constexpr int kTmemCols = 2 * kBN;
+  static constexpr size_t kSmem = 1024 /*align slack*/ + size_t(kStages) * kStageBytes + 256;
+};
+
+struct EpiParams {
+  int64_t M;
+  int N, K, inter;
+  void* C;
+  int64_t ldc;
+  const void* R;
+  int64_t ldr;
+  const float* b1;
+  const float* w2;
+  const float* b2;
+  float* scores;
+  int tiles_m, tiles_n;
+  unsigned int* err;
+};
+
+__device__ __forceinline__ void store32_bf16(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 u;
+    u.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    u.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    u.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d[q] = u;
+  }
+}
+
+__device__ __forceinline__ void add32_bf16(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = s[q];
+    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[8 * q + j] += __bfloat162float(e[j]);
+  }
+}
+
+template <int kBN, int kEpi>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            EpiParams p) {
+  using C = Cfg<kBN>;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned base for the swizzled tiles.
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  uint8_t* tiles = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(C::kStages) * C::kStageBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::kStages;
+  uint64_t* acc_full = bars + 2 * C::kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 2) tmem_alloc(tmem_slot, C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = p.tiles_m * p.tiles_n;
+  const int num_kb = (p.K + kBK - 1) / kBK;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------- producer
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
+      const int b_row0 = kEpi == EPI_SWIGLU ? nb * 128 : nb * kBN;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&empty[s], ph ^ 1u, p.err)) { ok = false; break; }
+        uint8_t* a_dst = tiles + size_t(s) * C::kStageBytes;
+        uint8_t* b_dst = a_dst + C::kABytes;
+        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+        tma_load_2d(&tmA, &full[s], a_dst, kb * kBK, mb * kBM);
+#pragma unroll
+        for (int h = 0; h < kBN / 128; ++h) {
+          const int row = (kEpi == EPI_SWIGLU && h == 1) ? p.inter + b_row0 : b_row0 + h * 128;
+          tma_load_2d(&tmB, &full[s], b_dst + h * 128 * 128, kb * kBK, row);
+        }
+        if (++s == C::kStages) { s = 0; ph ^= 1u; }
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN);
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      const int a = it & 1;
+      const uint32_t use = static_cast<uint32_t>(it >> 1);
+      if (!mbar_wait(&acc_empty[a], (use & 1u) ^ 1u, p.err)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * kBN);
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&full[s], ph, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_addr(tiles + size_t(s) * C::kStageBytes);
+        const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) {
+          umma_f16_ss(d_tmem, sdesc_kmajor_sw128(a_addr + k * 32), sdesc_kmajor_sw128(b_addr + k * 32),
+                      idesc, (kb | k) != 0 ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+        if (++s == C::kStages) { s = 0; ph ^= 1u; }
+      }
+      if (ok) umma_commit(&acc_full[a]);
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------- epilogue
+    const int quarter = warp & 3;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
+      const int a = it & 1;
+      const uint32_t use = static_cast<uint32_t>(it >> 1);
+      if (!mbar_wait_warp(&acc_full[a], use & 1u, p.err)) break;
+      tc_fence_after();
+      const int64_t row = static_cast<int64_t>(mb) * kBM + quarter * 32 + lane;
+      const bool row_ok = row < p.M;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(a * kBN);
+      if constexpr (kEpi == EPI_STORE || kEpi == EPI_RESIDUAL) {
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+          float v[32];
+          tmem_ld32_wait(t_row + c * 32, v);
+          const int col = nb * kBN + c * 32;
+          if (row_ok && col < p.N) {
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) + row * p.ldc + col;
+            if (kEpi == EPI_RESIDUAL)
+              add32_bf16(static_cast<const __nv_bfloat16*>(p.R) + row * p.ldr + col, v);
+            store32_bf16(dst, v);
+          }
+        }
+      } else if constexpr (kEpi == EPI_SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float g[32], u[32];
+          tmem_ld32_wait(t_row + c * 32, g);
+          tmem_ld32_wait(t_row + 128 + c * 32, u);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) g[j] = silu_f(g[j]) * u[j];
+          if (row_ok)
+            store32_bf16(static_cast<__nv_bfloat16*>(p.C) + row * p.ldc + nb * 128 + c * 32, g);
+        }
+      } else {  // EPI_SCORE
+        float acc = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+          float v[32];
+          tmem_ld32_wait(t_row + c * 32, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int f = c * 32 + j;
+            if (f < p.N) {
+              const float h = v[j] + (p.b1 ? __ldg(p.b1 + f) : 0.f);
+              acc = fmaf(__ldg(p.w2 + f), silu_f(h), acc);
+            }
+          }
+        }
+        if (row_ok) p.scores[row] = acc + (p.b2 ? __ldg(p.b2) : 0.f);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[a]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+template <int kBN, int kEpi>
+cudaError_t run(const GemmArgs& g, cudaStream_t st) {
+  using C = Cfg<kBN>;
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d_bf16(&ta, g.A, g.M, g.K, g.lda, kBM)) return cudaErrorInvalidValue;
+  const int64_t b_rows = g.N;
+  if (!make_tmap_2d_bf16(&tb, g.B, b_rows, g.K, g.ldb, 128)) return cudaErrorInvalidValue;
+  EpiParams p;
+  p.M = g.M;
+  p.N = kEpi == EPI_SWIGLU ? g.inter : g.N;
+  p.K = g.K;
+  p.inter = g.inter;
+  p.C = g.C;
+  p.ldc = g.ldc;
+  p.R = g.R;
+  p.ldr = g.ldr;
+  p.b1 = g.b1;
+  p.w2 = g.w2;
+  p.b2 = g.b2;
+  p.scores = g.scores;
+  p.tiles_m = static_cast<int>((g.M + kBM - 1) / kBM);
+  p.tiles_n = kEpi == EPI_SWIGLU ? g.inter / 128 : (g.N + kBN - 1) / kBN;
+  p.err = device_error_word();
+  const int tiles = p.tiles_m * p.tiles_n;
+  if (tiles == 0) return cudaSuccess;
+  auto kern = gemm_tc<kBN, kEpi>;
+  cudaError_t e = set_smem_attr_once(reinterpret_cast<const void*>(kern), static_cast<int>(C::kSmem));
+  if (e != cudaSuccess) return e;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  kern<<<grid, kThreads, C::kSmem, st>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemm_tc_supported(const GemmArgs& g) {
+  // TMA: 16-byte aligned bases and row strides.
+  auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+  if (!al16(g.A) || !al16(g.B) || (g.lda % 8) || (g.ldb % 8) || g.K % 8 || g.K <= 0) return false;
+  switch (g.epi) {
+    case EPI_STORE:
+    case EPI_RESIDUAL:
+      return g.N % 32 == 0 && al16(g.C) && g.ldc % 8 == 0 &&
+             (g.epi == EPI_STORE || (al16(g.R) && g.ldr % 8 == 0));
+    case EPI_SWIGLU:
+      return g.inter % 128 == 0 && g.N == 2 * g.inter && al16(g.C) && g.ldc % 8 == 0;
+    case EPI_SCORE:
+      return g.N >= 1 && g.N <= 256 && g.scores != nullptr && g.w2 != nullptr;
+  }
+  return false;
+}
+
+cudaError_t launch_gemm_tc(const GemmArgs& g, cudaStream_t st) {
+  if (g.M <= 0) return cudaSuccess;
+  switch (g.epi) {
+    case EPI_STORE: return run<256, EPI_STORE>(g, st);
+    case EPI_RESIDUAL: return run<256, EPI_RESIDUAL>(g, st);
+    case EPI_SWIGLU: return run<256, EPI_SWIGLU>(g, st);
+    case EPI_SCORE: return run<256, EPI_SCORE>(g, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace tg

@@ -1,0 +1,277 @@
+// k_rowwise.cu -- row-wise kernels around the GEMMs and the attention:
+// RMSNorm, RoPE (with optional per-head qk-norm) at original positions, the
+// V-tile transpose feeding the tensor-core attention, the per-key gate bias
+// logsigmoid(s_j), and two fp32 helpers of the SIMT path.
+//
+// RoPE at the kept tokens' original positions keeps the relative geometry of
+// the pruned context (the pages state that kept tokens continue with their
+// positions: Tencent Cloud article "TokenGate：端到端可训练的 Token 剪枝机制，
+// 让大模型 Prefill 提速 11.3 倍", section "TokenGate 提前筛选 Token"). The
+// rotate-half pairing and theta_i = base^(-2i/dh) follow the Qwen3 backbone
+// the pages evaluate. The angle pos * theta_i is formed and reduced modulo
+// 2*pi in double precision before the fp32 sine/cosine: at pos ~1.3e5 an
+// fp32 angle would be off by ~1e-2 rad.
+#include <algorithm>
+
+#include "tg_device.cuh"
+#include "tg_internal.h"
+
+namespace tg {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ float ld_f(const T* p);
+template <>
+__device__ __forceinline__ float ld_f<float>(const float* p) { return __ldg(p); }
+template <>
+__device__ __forceinline__ float ld_f<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(__ldg(p));
+}
+template <typename T>
+__device__ __forceinline__ T to_t(float v);
+template <>
+__device__ __forceinline__ float to_t<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 to_t<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ float to_float(float v) { return v; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// ---------------------------------------------------------------- RMSNorm
+// One warp per row: y = x * rsqrt(mean(x^2) + eps) * gamma.
+template <typename T>
+__global__ void __launch_bounds__(256) rmsnorm_rows(const T* __restrict__ x,
+                                                    const float* __restrict__ g, float eps,
+                                                    int64_t rows, int d, T* __restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const T* xr = x + row * d;
+  T* yr = y + row * d;
+  constexpr int kVec = 16 / sizeof(T);
+  float ss = 0.f;
+  const bool vec = (d % kVec) == 0;
+  if (vec) {
+    for (int c = lane * kVec; c < d; c += 32 * kVec) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(xr + c));
+      const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int j = 0; j < kVec; ++j) {
+        const float f = to_float(e[j]);
+        ss += f * f;
+      }
+    }
+  } else {
+    for (int c = lane; c < d; c += 32) {
+      const float f = ld_f(xr + c);
+      ss += f * f;
+    }
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / static_cast<float>(d) + eps);
+  if (vec) {
+    for (int c = lane * kVec; c < d; c += 32 * kVec) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(xr + c));
+      const T* e = reinterpret_cast<const T*>(&u);
+      uint4 o;
+      T* oe = reinterpret_cast<T*>(&o);
+#pragma unroll
+      for (int j = 0; j < kVec; ++j) oe[j] = to_t<T>(to_float(e[j]) * r * __ldg(g + c + j));
+      *reinterpret_cast<uint4*>(yr + c) = o;
+    }
+  } else {
+    for (int c = lane; c < d; c += 32) yr[c] = to_t<T>(ld_f(xr + c) * r * __ldg(g + c));
+  }
+}
+
+// ---------------------------------------------------------------- RoPE + qk-norm
+// One CTA (4 warps) per token; cos/sin of this token's position in shared
+// memory, then each warp rotates whole heads. Thread 0 also writes the
+// token's gate bias logsigmoid(s_t).
+template <typename T, int kDh>
+__global__ void __launch_bounds__(128) rope_qk(RopePrepArgs a) {
+  constexpr int kHalf = kDh / 2;
+  constexpr int kPairs = kHalf / 32;  // pairs per lane
+  __shared__ float s_cos[kHalf], s_sin[kHalf];
+  const int64_t t = blockIdx.x;
+  const int pos = a.pos ? __ldg(a.pos + t) : static_cast<int>(t);
+  if (threadIdx.x < kHalf) {
+    const int i = threadIdx.x;
+    const double theta = exp2(-(2.0 * i / kDh) * log2(static_cast<double>(a.rope_base)));
+    const double ang = static_cast<double>(pos) * theta;
+    const double two_pi = 6.283185307179586476925286766559;
+    const double red = ang - two_pi * rint(ang * (1.0 / two_pi));
+    float sv, cv;
+    sincosf(static_cast<float>(red), &sv, &cv);
+    s_cos[i] = cv;
+    s_sin[i] = sv;
+  }
+  if (threadIdx.x == 0 && a.s != nullptr) a.lsig_out[t] = logsigmoid_f(__ldg(a.s + t));
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int heads = a.hq + a.hkv;
+  for (int h = warp; h < heads; h += 4) {
+    const bool is_q = h < a.hq;
+    const int hh = is_q ? h : h - a.hq;
+    const T* src = static_cast<const T*>(is_q ? a.q_src : a.k_src) +
+                   t * (is_q ? a.q_stride : a.k_stride) + hh * kDh;
+    T* dst = static_cast<T*>(is_q ? a.q_out : a.k_out) +
+             (t * (is_q ? a.hq : a.hkv) + hh) * kDh;
+    const float* nw = is_q ? a.q_norm : a.k_norm;
+    float lo[kPairs], hi[kPairs];
+    float ss = 0.f;
+#pragma unroll
+    for (int p = 0; p < kPairs; ++p) {
+      lo[p] = ld_f(src + lane + 32 * p);
+      hi[p] = ld_f(src + lane + 32 * p + kHalf);
+      ss += lo[p] * lo[p] + hi[p] * hi[p];
+    }
+    if (nw != nullptr) {
+      const float r = rsqrtf(warp_sum(ss) / static_cast<float>(kDh) + a.eps);
+#pragma unroll
+      for (int p = 0; p < kPairs; ++p) {
+        lo[p] = lo[p] * r * __ldg(nw + lane + 32 * p);
+        hi[p] = hi[p] * r * __ldg(nw + lane + 32 * p + kHalf);
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < kPairs; ++p) {
+      const int i = lane + 32 * p;
+      const float c = s_cos[i], s = s_sin[i];
+      dst[i] = to_t<T>(lo[p] * c - hi[p] * s);
+      dst[i + kHalf] = to_t<T>(hi[p] * c + lo[p] * s);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- V transpose
+// One CTA per (64-token tile, KV head): vT[g][e][t] = v[t][g][e] (zero for
+// t >= T), so that the attention's P.V product reads V K-major. Also copies
+// v into a [T, hkv, dh] KV-cache buffer when asked.
+template <int kDh>
+__global__ void __launch_bounds__(256) v_transpose(RopePrepArgs a) {
+  constexpr int kTile = 64;
+  constexpr int kLd = kDh + 8;  // padded row (bf16 elements)
+  __shared__ __align__(16) __nv_bfloat16 tile[kTile * kLd];
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTile;
+  const int g = blockIdx.y;
+  const __nv_bfloat16* v = static_cast<const __nv_bfloat16*>(a.v_src);
+  __nv_bfloat16* kvv = static_cast<__nv_bfloat16*>(a.kv_v_out);
+  constexpr int kVecRow = kDh / 8;  // uint4 per row
+  for (int i = threadIdx.x; i < kTile * kVecRow; i += 256) {
+    const int r = i / kVecRow, c = i % kVecRow;
+    const int64_t t = t0 + r;
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (t < a.T) {
+      u = __ldg(reinterpret_cast<const uint4*>(v + t * a.v_stride + g * kDh) + c);
+      if (kvv) reinterpret_cast<uint4*>(kvv + (t * a.hkv + g) * kDh)[c] = u;
+    }
+    *reinterpret_cast<uint4*>(&tile[r * kLd + c * 8]) = u;
+  }
+  __syncthreads();
+  __nv_bfloat16* vt = static_cast<__nv_bfloat16*>(a.vT_out) + static_cast<int64_t>(g) * kDh * a.t_pad;
+  for (int i = threadIdx.x; i < kDh * (kTile / 8); i += 256) {
+    const int e = i / (kTile / 8), c = i % (kTile / 8);
+    uint4 o;
+    __nv_bfloat16* oe = reinterpret_cast<__nv_bfloat16*>(&o);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) oe[j] = tile[(c * 8 + j) * kLd + e];
+    *reinterpret_cast<uint4*>(vt + static_cast<int64_t>(e) * a.t_pad + t0 + c * 8) = o;
+  }
+}
+
+// fp32 path: plain copy of v into a KV-cache buffer.
+__global__ void copy_v_f32(RopePrepArgs a) {
+  const int64_t t = blockIdx.x;
+  const float* v = static_cast<const float*>(a.v_src) + t * a.v_stride;
+  float* o = static_cast<float*>(a.kv_v_out) + t * a.hkv * a.dh;
+  for (int i = threadIdx.x; i < a.hkv * a.dh; i += blockDim.x) o[i] = __ldg(v + i);
+}
+
+// ---------------------------------------------------------------- fp32 helpers
+__global__ void swiglu_f32(const float* __restrict__ gu, int64_t rows, int inter,
+                           float* __restrict__ h) {
+  const int64_t total = rows * inter;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / inter;
+    const int j = static_cast<int>(i % inter);
+    const float g = gu[r * 2 * inter + j], u = gu[r * 2 * inter + inter + j];
+    h[i] = silu_f(g) * u;
+  }
+}
+
+__global__ void score_dot_f32(const float* __restrict__ hpre, int64_t rows, int f,
+                              const float* __restrict__ b1, const float* __restrict__ w2,
+                              const float* __restrict__ b2, float* __restrict__ scores) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  float acc = 0.f;
+  for (int j = lane; j < f; j += 32) {
+    const float h = hpre[row * f + j] + (b1 ? __ldg(b1 + j) : 0.f);
+    acc += __ldg(w2 + j) * silu_f(h);
+  }
+  acc = warp_sum(acc);
+  if (lane == 0) scores[row] = acc + (b2 ? __ldg(b2) : 0.f);
+}
+
+}  // namespace
+
+cudaError_t launch_rmsnorm(const void* x, const float* gamma, float eps, int64_t rows, int d,
+                           bool bf16, void* y, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
+  if (bf16)
+    rmsnorm_rows<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), gamma, eps, rows, d, static_cast<__nv_bfloat16*>(y));
+  else
+    rmsnorm_rows<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(x), gamma, eps, rows, d,
+                                                static_cast<float*>(y));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_prep(const RopePrepArgs& a, cudaStream_t st) {
+  if (a.T <= 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>(a.T);
+  if (a.bf16) {
+    if (a.dh == 128) rope_qk<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(a);
+    else rope_qk<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(a);
+    if (a.vT_out) {
+      const dim3 g2(static_cast<unsigned>(a.t_pad / 64), static_cast<unsigned>(a.hkv));
+      if (a.dh == 128) v_transpose<128><<<g2, 256, 0, st>>>(a);
+      else v_transpose<64><<<g2, 256, 0, st>>>(a);
+    }
+  } else {
+    if (a.dh == 128) rope_qk<float, 128><<<grid, 128, 0, st>>>(a);
+    else rope_qk<float, 64><<<grid, 128, 0, st>>>(a);
+    if (a.kv_v_out) copy_v_f32<<<grid, 128, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu_f32(const float* gu, int64_t rows, int inter, float* h, cudaStream_t st) {
+  const int64_t total = rows * inter;
+  if (total <= 0) return cudaSuccess;
+  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((total + 255) / 256, 148 * 16));
+  swiglu_f32<<<blocks, 256, 0, st>>>(gu, rows, inter, h);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_score_dot_f32(const float* hpre, int64_t rows, int f, const float* b1,
+                                 const float* w2, const float* b2, float* scores, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  score_dot_f32<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(hpre, rows, f, b1, w2, b2,
+                                                                       scores);
+  return cudaGetLastError();
+}
+
+}  // namespace tg

@@ -1,0 +1,391 @@
+// k_select.cu -- deterministic top-K selection with protected tokens.
+//
+// The top-K selector keeps the K best-scoring tokens and never drops the
+// protected (question) span (Tencent Cloud article "TokenGate：端到端可训练的
+// Token 剪枝机制，让大模型 Prefill 提速 11.3 倍", section "TokenGate 提前筛选
+// Token"; ai.866data.com article "让大模型学会"略读"…", section
+// "可学习剪枝的机制设计"). Ranking is (score descending, index ascending),
+// with -0.0 == +0.0 and NaN lowest.
+//
+// Method: radix select over the 32-bit order-preserving key of each fp32
+// score, in three digits (11, 11, 10 bits). Each pass histograms the next
+// digit of the keys that still match the prefix found so far; every CTA
+// finds the threshold bin from the finished histogram of the previous pass
+// (identical work, identical result), so no CTA waits on another. The last
+// two kernels count, per chunk, the tokens kept for sure and the tokens tied
+// at the threshold key, then write the kept indices in index order: the tied
+// tokens taken are the lowest-index ones. Integer atomics only, so the
+// result is bit-reproducible.
+#include "tg_device.cuh"
+#include "tg_internal.h"
+
+namespace tg {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kPerThread = 8;
+constexpr int kChunk = kThreads * kPerThread;  // tokens per CTA
+
+// Workspace layout (32-bit words).
+struct SelState {
+  int32_t status;    // 0 = ok, 3 = more protected tokens than k
+  uint32_t n_prot;   // protected count (atomic sum)
+  uint32_t prefix;   // key bits found so far
+  uint32_t need;     // unprotected tokens still to take at/below prefix
+  uint32_t thresh;   // final threshold key
+  uint32_t ties;     // tokens with key == thresh to take (lowest indices)
+  uint32_t pad[2];
+};
+constexpr int kHist0 = 2048, kHist1 = 2048, kHist2 = 1024;
+constexpr size_t kOffHist0 = sizeof(SelState);
+constexpr size_t kOffHist1 = kOffHist0 + kHist0 * 4;
+constexpr size_t kOffHist2 = kOffHist1 + kHist1 * 4;
+constexpr size_t kOffCounts = kOffHist2 + kHist2 * 4;  // then 2 x C words
+constexpr size_t kZeroBytes = kOffCounts;
+
+struct Ws {
+  SelState* st;
+  uint32_t* h0;
+  uint32_t* h1;
+  uint32_t* h2;
+  uint32_t* n_def;  // [C] tokens kept for sure in chunk c
+  uint32_t* n_tie;  // [C] unprotected tokens with key == thresh in chunk c
+};
+
+__host__ __device__ inline Ws ws_view(void* base, int64_t chunks) {
+  char* b = static_cast<char*>(base);
+  Ws w;
+  w.st = reinterpret_cast<SelState*>(b);
+  w.h0 = reinterpret_cast<uint32_t*>(b + kOffHist0);
+  w.h1 = reinterpret_cast<uint32_t*>(b + kOffHist1);
+  w.h2 = reinterpret_cast<uint32_t*>(b + kOffHist2);
+  w.n_def = reinterpret_cast<uint32_t*>(b + kOffCounts);
+  w.n_tie = w.n_def + chunks;
+  return w;
+}
+
+// Loads this thread's 8 tokens: keys (protected tokens flagged separately).
+template <bool kVec>
+__device__ __forceinline__ int load_tokens(const float* __restrict__ scores,
+                                           const uint8_t* __restrict__ protect, int64_t n,
+                                           int64_t first, uint32_t (&key)[kPerThread],
+                                           bool (&prot)[kPerThread]) {
+  int valid = 0;
+  if (kVec && first + kPerThread <= n) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(scores + first));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(scores + first) + 1);
+    const float s[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint2 pm = make_uint2(0u, 0u);
+    if (protect) pm = __ldg(reinterpret_cast<const uint2*>(protect + first));
+#pragma unroll
+    for (int j = 0; j < kPerThread; ++j) {
+      key[j] = score_key(s[j]);
+      const uint32_t word = j < 4 ? pm.x : pm.y;
+      prot[j] = ((word >> (8 * (j & 3))) & 0xFFu) != 0u;
+    }
+    valid = kPerThread;
+  } else {
+#pragma unroll
+    for (int j = 0; j < kPerThread; ++j) {
+      const int64_t i = first + j;
+      if (i < n) {
+        key[j] = score_key(__ldg(scores + i));
+        prot[j] = protect ? (__ldg(protect + i) != 0) : false;
+        ++valid;
+      } else {
+        key[j] = 0u;
+        prot[j] = false;
+      }
+    }
+  }
+  return valid;
+}
+
+// Exclusive prefix sum over the CTA (thread order). Returns this thread's
+// exclusive prefix; *total receives the CTA sum.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* total) {
+  __shared__ uint32_t warp_sums[kThreads / 32];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    uint32_t w = lane < kThreads / 32 ? warp_sums[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kThreads / 32) warp_sums[lane] = w;  // inclusive
+  }
+  __syncthreads();
+  const uint32_t before_warp = wid ? warp_sums[wid - 1] : 0u;
+  if (total) *total = warp_sums[kThreads / 32 - 1];
+  const uint32_t r = before_warp + x - v;
+  __syncthreads();
+  return r;
+}
+
+// Finds, scanning bins from the highest, the bin b* where the running count
+// of higher bins is < need and reaches need inside b*. Returns b* and the
+// rank left inside it (need - count above). Every thread gets the result.
+template <int kBins>
+__device__ __forceinline__ void find_bin(const uint32_t* __restrict__ hist, uint32_t need,
+                                         uint32_t* bin_out, uint32_t* need_out) {
+  constexpr int kPer = kBins / kThreads;
+  __shared__ uint32_t s_bin, s_need;
+  uint32_t h[kPer];
+  uint32_t local = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    h[j] = hist[kBins - 1 - (threadIdx.x * kPer + j)];  // descending bins
+    local += h[j];
+  }
+  if (threadIdx.x == 0) {
+    s_bin = 0u;
+    s_need = need;
+  }
+  uint32_t total;
+  const uint32_t before = block_excl_scan(local, &total);
+  if (before < need && need <= before + local) {
+    uint32_t run = before;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if (run + h[j] >= need) {
+        s_bin = static_cast<uint32_t>(kBins - 1 - (threadIdx.x * kPer + j));
+        s_need = need - run;
+        break;
+      }
+      run += h[j];
+    }
+  }
+  __syncthreads();
+  *bin_out = s_bin;
+  *need_out = s_need;
+}
+
+// Pass 0: protected count and the top-digit histogram.
+template <bool kVec>
+__global__ void __launch_bounds__(kThreads) sel_hist0(const float* __restrict__ scores,
+                                                      const uint8_t* __restrict__ protect,
+                                                      int64_t n, Ws w) {
+  __shared__ uint32_t hist[kHist0];
+  for (int i = threadIdx.x; i < kHist0; i += kThreads) hist[i] = 0u;
+  __syncthreads();
+  uint32_t key[kPerThread];
+  bool prot[kPerThread];
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * kChunk + threadIdx.x * kPerThread;
+  const int valid = load_tokens<kVec>(scores, protect, n, first, key, prot);
+  uint32_t np = 0;
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j) {
+    if (j < valid) {
+      if (prot[j]) ++np;
+      else atomicAdd(&hist[key[j] >> 21], 1u);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) np += __shfl_xor_sync(0xFFFFFFFFu, np, o);
+  if ((threadIdx.x & 31) == 0 && np) atomicAdd(&w.st->n_prot, np);
+  __syncthreads();
+  for (int i = threadIdx.x; i < kHist0; i += kThreads)
+    if (hist[i]) atomicAdd(&w.h0[i], hist[i]);
+}
+
+// Pass 1 / 2: find the previous digit, histogram the next one.
+template <bool kVec, int kPass>
+__global__ void __launch_bounds__(kThreads) sel_hist_next(const float* __restrict__ scores,
+                                                          const uint8_t* __restrict__ protect,
+                                                          int64_t n, int64_t k, Ws w) {
+  constexpr int kBinsPrev = kPass == 1 ? kHist0 : kHist1;
+  constexpr int kBinsNext = kPass == 1 ? kHist1 : kHist2;
+  __shared__ uint32_t hist[kBinsNext];
+  uint32_t need, prefix;
+  if (kPass == 1) {
+    const int64_t np = w.st->n_prot;
+    if (np > k) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) w.st->status = 3;
+      return;
+    }
+    need = static_cast<uint32_t>(k - np);
+    prefix = 0u;
+  } else {
+    if (w.st->status != 0) return;
+    need = w.st->need;
+    prefix = w.st->prefix;
+  }
+  if (need == 0u) return;  // nothing unprotected to keep
+  uint32_t bin, rest;
+  find_bin<kBinsPrev>(kPass == 1 ? w.h0 : w.h1, need, &bin, &rest);
+  const uint32_t new_prefix = kPass == 1 ? bin : ((prefix << 11) | bin);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    w.st->prefix = new_prefix;
+    w.st->need = rest;
+  }
+  for (int i = threadIdx.x; i < kBinsNext; i += kThreads) hist[i] = 0u;
+  __syncthreads();
+  uint32_t key[kPerThread];
+  bool prot[kPerThread];
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * kChunk + threadIdx.x * kPerThread;
+  const int valid = load_tokens<kVec>(scores, protect, n, first, key, prot);
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j) {
+    if (j < valid && !prot[j]) {
+      if (kPass == 1) {
+        if ((key[j] >> 21) == new_prefix) atomicAdd(&hist[(key[j] >> 10) & 0x7FFu], 1u);
+      } else {
+        if ((key[j] >> 10) == new_prefix) atomicAdd(&hist[key[j] & 0x3FFu], 1u);
+      }
+    }
+  }
+  __syncthreads();
+  uint32_t* gh = kPass == 1 ? w.h1 : w.h2;
+  for (int i = threadIdx.x; i < kBinsNext; i += kThreads)
+    if (hist[i]) atomicAdd(&gh[i], hist[i]);
+}
+
+// Final digit, then per-chunk counts of sure keeps and threshold ties.
+template <bool kVec>
+__global__ void __launch_bounds__(kThreads) sel_count(const float* __restrict__ scores,
+                                                      const uint8_t* __restrict__ protect,
+                                                      int64_t n, int64_t k, Ws w) {
+  if (w.st->status != 0) return;
+  const int64_t np = w.st->n_prot;
+  uint32_t thresh, ties;
+  if (static_cast<int64_t>(np) == k) {
+    thresh = 0xFFFFFFFFu;  // no unprotected token is kept
+    ties = 0u;
+  } else {
+    uint32_t bin, rest;
+    find_bin<kHist2>(w.h2, w.st->need, &bin, &rest);
+    thresh = (w.st->prefix << 10) | bin;
+    ties = rest;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    w.st->thresh = thresh;
+    w.st->ties = ties;
+  }
+  uint32_t key[kPerThread];
+  bool prot[kPerThread];
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * kChunk + threadIdx.x * kPerThread;
+  const int valid = load_tokens<kVec>(scores, protect, n, first, key, prot);
+  uint32_t nd = 0, nt = 0;
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j) {
+    if (j < valid) {
+      if (prot[j] || key[j] > thresh) ++nd;
+      else if (key[j] == thresh) ++nt;
+    }
+  }
+  uint32_t td, tt;
+  block_excl_scan(nd, &td);
+  block_excl_scan(nt, &tt);
+  if (threadIdx.x == 0) {
+    w.n_def[blockIdx.x] = td;
+    w.n_tie[blockIdx.x] = tt;
+  }
+}
+
+// Writes the kept indices of this chunk, in index order, at their global rank.
+template <bool kVec>
+__global__ void __launch_bounds__(kThreads) sel_write(const float* __restrict__ scores,
+                                                      const uint8_t* __restrict__ protect,
+                                                      int64_t n, int64_t k,
+                                                      int32_t* __restrict__ kept_idx, Ws w) {
+  if (w.st->status != 0) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < k;
+         i += static_cast<int64_t>(gridDim.x) * kThreads)
+      kept_idx[i] = -1;
+    return;
+  }
+  const uint32_t thresh = w.st->thresh, ties = w.st->ties;
+  // Bases from the chunks before this one: ties seen before this chunk, and
+  // kept tokens before it, where chunk c keeps n_def[c] plus
+  // clamp(ties - ties_before(c), 0, n_tie[c]) of its tied tokens.
+  uint32_t tie_base = 0, out_base = 0;
+  for (uint32_t g = 0; g < blockIdx.x; g += kThreads) {
+    const uint32_t c = g + threadIdx.x;
+    const bool in = c < blockIdx.x;
+    const uint32_t nt = in ? w.n_tie[c] : 0u;
+    uint32_t group_ties, group_out;
+    const uint32_t before = tie_base + block_excl_scan(nt, &group_ties);
+    uint32_t take = 0;
+    if (in && before < ties) take = min(nt, ties - before);
+    const uint32_t contrib = in ? w.n_def[c] + take : 0u;
+    block_excl_scan(contrib, &group_out);
+    tie_base += group_ties;
+    out_base += group_out;
+  }
+  uint32_t key[kPerThread];
+  bool prot[kPerThread];
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * kChunk + threadIdx.x * kPerThread;
+  const int valid = load_tokens<kVec>(scores, protect, n, first, key, prot);
+  uint32_t lt = 0;
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j)
+    if (j < valid && !prot[j] && key[j] == thresh) ++lt;
+  uint32_t dummy;
+  const uint32_t tie_before = tie_base + block_excl_scan(lt, &dummy);
+  bool keep[kPerThread];
+  uint32_t lk = 0, run = tie_before;
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j) {
+    bool kp = false;
+    if (j < valid) {
+      if (prot[j] || key[j] > thresh) {
+        kp = true;
+      } else if (key[j] == thresh) {
+        kp = run < ties;
+        ++run;
+      }
+    }
+    keep[j] = kp;
+    lk += kp ? 1u : 0u;
+  }
+  uint32_t pos = out_base + block_excl_scan(lk, &dummy);
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j) {
+    if (keep[j]) {
+      if (pos < static_cast<uint64_t>(k)) kept_idx[pos] = static_cast<int32_t>(first + j);
+      ++pos;
+    }
+  }
+}
+
+template <bool kVec>
+cudaError_t run_select(const float* scores, const uint8_t* protect, int64_t n, int64_t k,
+                       int32_t* kept_idx, void* ws, cudaStream_t st) {
+  const int64_t chunks = (n + kChunk - 1) / kChunk;
+  Ws w = ws_view(ws, chunks);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kZeroBytes, st);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(static_cast<unsigned>(chunks));
+  sel_hist0<kVec><<<grid, kThreads, 0, st>>>(scores, protect, n, w);
+  sel_hist_next<kVec, 1><<<grid, kThreads, 0, st>>>(scores, protect, n, k, w);
+  sel_hist_next<kVec, 2><<<grid, kThreads, 0, st>>>(scores, protect, n, k, w);
+  sel_count<kVec><<<grid, kThreads, 0, st>>>(scores, protect, n, k, w);
+  sel_write<kVec><<<grid, kThreads, 0, st>>>(scores, protect, n, k, kept_idx, w);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t select_ws_bytes(int64_t n) {
+  const int64_t chunks = (n + kChunk - 1) / kChunk;
+  return kOffCounts + static_cast<size_t>(chunks) * 2 * 4;
+}
+
+cudaError_t launch_topk_select(const float* scores, const uint8_t* protect, int64_t n, int64_t k,
+                               int32_t* kept_idx, void* ws, cudaStream_t st) {
+  const bool vec = (reinterpret_cast<uintptr_t>(scores) % 16 == 0) &&
+                   (protect == nullptr || reinterpret_cast<uintptr_t>(protect) % 8 == 0);
+  return vec ? run_select<true>(scores, protect, n, k, kept_idx, ws, st)
+             : run_select<false>(scores, protect, n, k, kept_idx, ws, st);
+}
+
+}  // namespace tg

@@ -1,0 +1,514 @@
+// tg_api.cu -- the C ABI of libtokengate (declared in include/tokengate.h).
+//
+// Host-side argument validation, workspace planning and the orchestration of
+// the gated prefill. Every call validates on the host, then only enqueues
+// kernels on the caller's stream: no allocation, no host synchronisation.
+//
+// The gated forward runs in three stages (Tencent Cloud article
+// "TokenGate：端到端可训练的 Token 剪枝机制，让大模型 Prefill 提速 11.3 倍", section
+// "TokenGate 提前筛选 Token"; farwalk.ai item on TokenGate, section "论文的方法";
+// ai.866data.com article "让大模型学会"略读"…", section "可学习剪枝的机制设计"):
+// layers below the gate over all N tokens; at the gate layer, attention over
+// all N tokens, then the scorer on the post-attention residual, the top-K
+// selector and compaction; the gate layer's FFN and all layers above over
+// the K kept rows, with token-gated attention, writing K-row KV only.
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "../../include/tokengate.h"
+#include "tg_internal.h"
+
+__device__ unsigned int g_tg_error_word;
+
+namespace tg {
+
+namespace {
+thread_local int t_last_cuda_error = 0;
+constexpr int kMaxDevices = 64;
+
+int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev;
+}
+}  // namespace
+
+int num_sms() {
+  static int cache[kMaxDevices] = {0};
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+unsigned int* device_error_word() {
+  static unsigned int* cache[kMaxDevices] = {nullptr};
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (cache[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_tg_error_word) == cudaSuccess)
+      cache[dev] = static_cast<unsigned int*>(ptr);
+  }
+  return cache[dev];
+}
+
+cudaError_t set_smem_attr_once(const void* fn, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({fn, dev})) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert({fn, dev});
+  return e;
+}
+
+namespace {
+
+tg_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return TG_OK;
+  t_last_cuda_error = static_cast<int>(e);
+  return TG_ERR_CUDA;
+}
+
+#define TG_TRY(expr)                                  \
+  do {                                                \
+    const cudaError_t tg_e_ = (expr);                 \
+    if (tg_e_ != cudaSuccess) return cuda_status(tg_e_); \
+  } while (0)
+
+#define TG_CHECK(cond, code) \
+  do {                       \
+    if (!(cond)) return (code); \
+  } while (0)
+
+size_t elem_size(tg_dtype dt) { return dt == TG_BF16 ? 2 : 4; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ plans
+// Each plan carves its buffers from an Arena; with a null base it only
+// measures, so sizing and use can never disagree.
+
+struct ScorePlan {
+  void* y = nullptr;     // [n, d] normed rows (dtype)
+  float* hpre = nullptr; // fp32 path: [n, f] pre-activation
+  size_t bytes = 0;
+  ScorePlan(void* ws, int64_t n, int d, int f, tg_dtype dt) {
+    Arena a(ws);
+    y = a.carve(size_t(n) * d * elem_size(dt));
+    if (dt == TG_F32) hpre = static_cast<float*>(a.carve(size_t(n) * f * 4));
+    bytes = a.used;
+  }
+};
+
+struct AttnPlan {
+  void* q_rot = nullptr;  // [k, hq, dh]
+  void* k_rot = nullptr;  // [k, hkv, dh]
+  void* vT = nullptr;     // bf16: [hkv, dh, t_pad]
+  float* lsig = nullptr;  // [k]
+  int64_t t_pad = 0;
+  size_t bytes = 0;
+  AttnPlan(void* ws, int64_t k, int hq, int hkv, int dh, tg_dtype dt, bool need_k) {
+    Arena a(ws);
+    const size_t e = elem_size(dt);
+    t_pad = static_cast<int64_t>(align_up(static_cast<size_t>(k), 64));
+    q_rot = a.carve(size_t(k) * hq * dh * e);
+    if (need_k) k_rot = a.carve(size_t(k) * hkv * dh * e);
+    if (dt == TG_BF16) vT = a.carve(size_t(hkv) * dh * t_pad * e);
+    lsig = static_cast<float*>(a.carve(size_t(k) * 4 + 16));
+    bytes = a.used;
+  }
+};
+
+struct PrefillPlan {
+  void* h = nullptr;       // [n, d] residual stream (all-token stage)
+  void* hk = nullptr;      // [k, d] residual stream (kept rows)
+  void* y = nullptr;       // [n, d] normed rows
+  void* qkv = nullptr;     // [n, (hq + 2 hkv) dh]
+  void* attn_o = nullptr;  // [n, hq dh]
+  void* mlp = nullptr;     // [n, I] (fp32: + [n, 2I] gate/up product)
+  void* gu = nullptr;
+  float* scores = nullptr; // [n]
+  float* hpre = nullptr;   // fp32 scorer pre-activation [n, F]
+  int32_t* pos_k = nullptr;
+  float* s_k = nullptr;
+  float* lsig_k = nullptr;
+  void* sel_ws = nullptr;
+  AttnPlan attn;           // sized for n rows, reused by every layer
+  size_t bytes = 0;
+  PrefillPlan(void* ws, const tg_model& m, int64_t n, int64_t k)
+      : attn(nullptr, n, m.n_heads_q, m.n_heads_kv, m.head_dim, m.dtype, true) {
+    Arena a(ws);
+    const size_t e = elem_size(m.dtype);
+    const int d = m.d_model, hq = m.n_heads_q, hkv = m.n_heads_kv, dh = m.head_dim;
+    h = a.carve(size_t(n) * d * e);
+    hk = a.carve(size_t(k) * d * e);
+    y = a.carve(size_t(n) * d * e);
+    qkv = a.carve(size_t(n) * (hq + 2 * hkv) * dh * e);
+    attn_o = a.carve(size_t(n) * hq * dh * e);
+    if (m.d_ffn > 0) {
+      mlp = a.carve(size_t(n) * m.d_ffn * e);
+      if (m.dtype == TG_F32) gu = a.carve(size_t(n) * 2 * m.d_ffn * 4);
+    }
+    scores = static_cast<float*>(a.carve(size_t(n) * 4));
+    if (m.dtype == TG_F32) hpre = static_cast<float*>(a.carve(size_t(n) * m.d_score * 4));
+    pos_k = static_cast<int32_t*>(a.carve(size_t(k) * 4));
+    s_k = static_cast<float*>(a.carve(size_t(k) * 4));
+    lsig_k = static_cast<float*>(a.carve(size_t(k) * 4));
+    sel_ws = a.carve(select_ws_bytes(n));
+    void* attn_base = a.carve(attn.bytes);
+    attn = AttnPlan(attn_base, n, hq, hkv, dh, m.dtype, true);
+    bytes = a.used;
+  }
+};
+
+// ------------------------------------------------------------------ pieces
+
+cudaError_t gemm(const GemmArgs& g, tg_dtype dt, cudaStream_t st) {
+  if (dt == TG_BF16) {
+    if (!gemm_tc_supported(g)) return cudaErrorInvalidValue;
+    return launch_gemm_tc(g, st);
+  }
+  return launch_gemm_simt_f32(g, st);
+}
+
+GemmArgs gemm_args(const void* A, int64_t lda, const void* B, int64_t ldb, void* C, int64_t ldc,
+                   int64_t M, int N, int K, EpiKind epi) {
+  GemmArgs g{};
+  g.A = A; g.lda = lda; g.B = B; g.ldb = ldb; g.C = C; g.ldc = ldc;
+  g.M = M; g.N = N; g.K = K; g.epi = epi;
+  return g;
+}
+
+// Scorer over `rows` rows of x (dtype dt) into scores[rows].
+cudaError_t run_score(const void* x, int64_t rows, int d, int f, const float* norm_w, float eps,
+                      const void* w1, const float* b1, const float* w2, const float* b2,
+                      tg_dtype dt, float* scores, void* y, float* hpre, cudaStream_t st) {
+  cudaError_t e = launch_rmsnorm(x, norm_w, eps, rows, d, dt == TG_BF16, y, st);
+  if (e != cudaSuccess) return e;
+  if (dt == TG_BF16) {
+    GemmArgs g = gemm_args(y, d, w1, d, nullptr, 0, rows, f, d, EPI_SCORE);
+    g.b1 = b1; g.w2 = w2; g.b2 = b2; g.scores = scores;
+    return gemm(g, dt, st);
+  }
+  GemmArgs g = gemm_args(y, d, w1, d, hpre, f, rows, f, d, EPI_STORE);
+  e = gemm(g, dt, st);
+  if (e != cudaSuccess) return e;
+  return launch_score_dot_f32(hpre, rows, f, b1, w2, b2, scores, st);
+}
+
+// RoPE/qk-norm prep + attention, q/k/v taken from rows with the given strides.
+cudaError_t run_attention(const void* q, int64_t q_stride, const void* kk, int64_t k_stride,
+                          const void* v, int64_t v_stride, const int32_t* pos, const float* s,
+                          const float* lsig_ready, const float* gain, const float* tau,
+                          const float* q_norm, const float* k_norm, float eps, int64_t rows,
+                          int hq, int hkv, int dh, float rope_base, tg_dtype dt,
+                          const AttnPlan& plan, void* k_out, void* v_out, void* out,
+                          cudaStream_t st) {
+  RopePrepArgs r{};
+  r.q_src = q; r.k_src = kk; r.v_src = v;
+  r.q_stride = q_stride; r.k_stride = k_stride; r.v_stride = v_stride;
+  r.pos = pos; r.q_norm = q_norm; r.k_norm = k_norm; r.eps = eps;
+  r.T = rows; r.hq = hq; r.hkv = hkv; r.dh = dh; r.rope_base = rope_base;
+  r.bf16 = dt == TG_BF16;
+  r.q_out = plan.q_rot;
+  r.k_out = k_out ? k_out : plan.k_rot;
+  r.vT_out = dt == TG_BF16 ? plan.vT : nullptr;
+  r.t_pad = plan.t_pad;
+  r.kv_v_out = v_out;
+  r.s = lsig_ready ? nullptr : s;
+  r.lsig_out = plan.lsig;
+  cudaError_t e = launch_rope_prep(r, st);
+  if (e != cudaSuccess) return e;
+  AttnArgs a{};
+  a.q = plan.q_rot;
+  a.k = r.k_out;
+  a.lsig = (s || lsig_ready) ? (lsig_ready ? lsig_ready : plan.lsig) : nullptr;
+  a.gain = gain; a.tau = tau;
+  a.T = rows; a.hq = hq; a.hkv = hkv; a.dh = dh;
+  a.out = out;
+  if (dt == TG_BF16) {
+    a.v = plan.vT;
+    a.t_pad = plan.t_pad;
+    if (!attn_tc_supported(a)) return cudaErrorInvalidValue;
+    return launch_attn_tc(a, st);
+  }
+  a.v = v;
+  a.t_pad = v_stride;
+  return launch_attn_simt_f32(a, st);
+}
+
+// ---- the decoder-layer pieces used by tg_prefill
+
+struct Dims {
+  int d, hq, hkv, dh, inter, qkv;
+};
+
+cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
+                               const PrefillPlan& P, void* h, int64_t rows, const int32_t* pos,
+                               const float* lsig, const float* gain, const float* tau,
+                               const tg_kv* kv, cudaStream_t st) {
+  const tg_dtype dt = m.dtype;
+  const size_t e = elem_size(dt);
+  cudaError_t err = launch_rmsnorm(h, lw.attn_norm, m.norm_eps, rows, D.d, dt == TG_BF16, P.y, st);
+  if (err != cudaSuccess) return err;
+  err = gemm(gemm_args(P.y, D.d, lw.wqkv, D.d, P.qkv, D.qkv, rows, D.qkv, D.d, EPI_STORE), dt, st);
+  if (err != cudaSuccess) return err;
+  const char* qkv = static_cast<const char*>(P.qkv);
+  err = run_attention(qkv, D.qkv, qkv + size_t(D.hq) * D.dh * e, D.qkv,
+                      qkv + size_t(D.hq + D.hkv) * D.dh * e, D.qkv, pos, nullptr, lsig, gain, tau,
+                      lw.q_norm, lw.k_norm, m.norm_eps, rows, D.hq, D.hkv, D.dh, m.rope_base, dt,
+                      P.attn, kv ? kv->k : nullptr, kv ? kv->v : nullptr, P.attn_o, st);
+  if (err != cudaSuccess) return err;
+  GemmArgs g = gemm_args(P.attn_o, int64_t(D.hq) * D.dh, lw.wo, int64_t(D.hq) * D.dh, h, D.d, rows,
+                         D.d, D.hq * D.dh, EPI_RESIDUAL);
+  g.R = h;
+  g.ldr = D.d;
+  return gemm(g, dt, st);
+}
+
+cudaError_t ffn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
+                         const PrefillPlan& P, void* h, int64_t rows, cudaStream_t st) {
+  if (lw.w_gate_up == nullptr) return cudaSuccess;
+  const tg_dtype dt = m.dtype;
+  cudaError_t err = launch_rmsnorm(h, lw.ffn_norm, m.norm_eps, rows, D.d, dt == TG_BF16, P.y, st);
+  if (err != cudaSuccess) return err;
+  if (dt == TG_BF16) {
+    GemmArgs g = gemm_args(P.y, D.d, lw.w_gate_up, D.d, P.mlp, D.inter, rows, 2 * D.inter, D.d,
+                           EPI_SWIGLU);
+    g.inter = D.inter;
+    err = gemm(g, dt, st);
+  } else {
+    err = gemm(gemm_args(P.y, D.d, lw.w_gate_up, D.d, P.gu, 2 * D.inter, rows, 2 * D.inter, D.d,
+                         EPI_STORE), dt, st);
+    if (err == cudaSuccess)
+      err = launch_swiglu_f32(static_cast<const float*>(P.gu), rows, D.inter,
+                              static_cast<float*>(P.mlp), st);
+  }
+  if (err != cudaSuccess) return err;
+  GemmArgs g = gemm_args(P.mlp, D.inter, lw.w_down, D.inter, h, D.d, rows, D.d, D.inter,
+                         EPI_RESIDUAL);
+  g.R = h;
+  g.ldr = D.d;
+  return gemm(g, dt, st);
+}
+
+tg_status validate_model(const tg_model* m, int64_t n, int64_t k, int gate_layer) {
+  TG_CHECK(m != nullptr && m->layers != nullptr, TG_ERR_INVALID_ARG);
+  TG_CHECK(m->dtype == TG_BF16 || m->dtype == TG_F32, TG_ERR_UNSUPPORTED);
+  TG_CHECK(m->n_layers >= 1 && m->d_model > 0 && m->n_heads_q > 0 && m->n_heads_kv > 0,
+           TG_ERR_INVALID_ARG);
+  TG_CHECK(m->n_heads_q % m->n_heads_kv == 0, TG_ERR_INVALID_ARG);
+  TG_CHECK(gate_layer >= -1 && gate_layer < m->n_layers, TG_ERR_INVALID_ARG);
+  TG_CHECK(n >= 1 && n < (int64_t(1) << 31) - 256, TG_ERR_INVALID_ARG);
+  TG_CHECK(k >= 1 && k <= n, TG_ERR_BUDGET);
+  TG_CHECK(m->score_norm && m->score_w1 && m->score_w2 && m->d_score >= 1, TG_ERR_INVALID_ARG);
+  TG_CHECK(std::isfinite(m->norm_eps) && m->norm_eps >= 0.f && m->rope_base > 1.f,
+           TG_ERR_INVALID_ARG);
+  const int d = m->d_model, dh = m->head_dim, qkv = (m->n_heads_q + 2 * m->n_heads_kv) * dh;
+  for (int l = 0; l < m->n_layers; ++l) {
+    const tg_layer& L = m->layers[l];
+    TG_CHECK(L.attn_norm && L.wqkv && L.wo, TG_ERR_INVALID_ARG);
+    TG_CHECK((L.q_norm == nullptr) == (L.k_norm == nullptr), TG_ERR_INVALID_ARG);
+    if (L.w_gate_up) TG_CHECK(L.w_down && L.ffn_norm && m->d_ffn > 0, TG_ERR_INVALID_ARG);
+  }
+  bool any_ffn = false;
+  for (int l = 0; l < m->n_layers; ++l) any_ffn |= m->layers[l].w_gate_up != nullptr;
+  if (m->dtype == TG_BF16) {
+    TG_CHECK(dh == 128, TG_ERR_UNSUPPORTED);
+    TG_CHECK(d % 32 == 0 && qkv % 32 == 0, TG_ERR_UNSUPPORTED);
+    TG_CHECK(m->d_score <= 256, TG_ERR_UNSUPPORTED);
+    if (any_ffn) TG_CHECK(m->d_ffn % 128 == 0, TG_ERR_UNSUPPORTED);
+  } else {
+    TG_CHECK(dh == 64 || dh == 128, TG_ERR_UNSUPPORTED);
+  }
+  return TG_OK;
+}
+
+}  // namespace
+}  // namespace tg
+
+using namespace tg;
+
+extern "C" {
+
+size_t tg_workspace_size(tg_op op, const tg_shape* s) {
+  if (s == nullptr) return 0;
+  switch (op) {
+    case TG_OP_SCORE:
+      return ScorePlan(nullptr, s->n, s->d_model, s->d_score, s->dtype).bytes;
+    case TG_OP_TOPK_SELECT:
+      return select_ws_bytes(s->n);
+    case TG_OP_COMPACT:
+      return 0;
+    case TG_OP_GATED_ATTN:
+      return AttnPlan(nullptr, s->k, s->n_heads_q, s->n_heads_kv, s->head_dim, s->dtype, true).bytes;
+    case TG_OP_PREFILL: {
+      tg_model m{};
+      m.dtype = s->dtype;
+      m.d_model = s->d_model;
+      m.n_heads_q = s->n_heads_q;
+      m.n_heads_kv = s->n_heads_kv;
+      m.head_dim = s->head_dim;
+      m.d_ffn = s->d_ffn;
+      m.d_score = s->d_score;
+      return PrefillPlan(nullptr, m, s->n, s->k).bytes;
+    }
+  }
+  return 0;
+}
+
+tg_status tg_score(const void* x, int64_t n, int32_t d, int32_t f, const float* norm_w, float eps,
+                   const void* w1, const float* b1, const float* w2, const float* b2, tg_dtype dt,
+                   float* scores, void* ws, size_t ws_bytes, tg_stream stream) {
+  TG_CHECK(dt == TG_BF16 || dt == TG_F32, TG_ERR_UNSUPPORTED);
+  TG_CHECK(x && norm_w && w1 && w2 && scores && n >= 1 && d >= 1 && f >= 1, TG_ERR_INVALID_ARG);
+  if (dt == TG_BF16) {
+    TG_CHECK(f <= 256 && d % 8 == 0, TG_ERR_UNSUPPORTED);
+    TG_CHECK(aligned16(x) && aligned16(w1), TG_ERR_INVALID_ARG);
+  } else {
+    TG_CHECK(f <= 1024, TG_ERR_UNSUPPORTED);
+  }
+  ScorePlan plan(nullptr, n, d, f, dt);
+  TG_CHECK(ws != nullptr && ws_bytes >= plan.bytes, TG_ERR_WORKSPACE);
+  plan = ScorePlan(ws, n, d, f, dt);
+  return cuda_status(run_score(x, n, d, f, norm_w, eps, w1, b1, w2, b2, dt, scores, plan.y,
+                               plan.hpre, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tg_status tg_topk_select(const float* scores, const uint8_t* protect, int64_t n, int64_t k,
+                         int32_t* kept_idx, void* ws, size_t ws_bytes, tg_stream stream) {
+  TG_CHECK(scores && kept_idx && n >= 1 && n < (int64_t(1) << 31) - 4096, TG_ERR_INVALID_ARG);
+  TG_CHECK(k >= 1 && k <= n, TG_ERR_BUDGET);
+  TG_CHECK(ws != nullptr && ws_bytes >= select_ws_bytes(n), TG_ERR_WORKSPACE);
+  TG_CHECK((reinterpret_cast<uintptr_t>(ws) & 15u) == 0, TG_ERR_INVALID_ARG);
+  return cuda_status(launch_topk_select(scores, protect, n, k, kept_idx, ws,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tg_status tg_compact(const void* x, const int32_t* pos_in, const float* scores,
+                     const int32_t* kept_idx, int64_t n, int64_t k, int32_t d, tg_dtype dt,
+                     void* x_out, int32_t* pos_out, float* scores_out, tg_stream stream) {
+  TG_CHECK(dt == TG_BF16 || dt == TG_F32, TG_ERR_UNSUPPORTED);
+  TG_CHECK(x && kept_idx && x_out && pos_out && n >= 1 && d >= 1, TG_ERR_INVALID_ARG);
+  TG_CHECK(k >= 1 && k <= n, TG_ERR_BUDGET);
+  TG_CHECK(scores_out == nullptr || scores != nullptr, TG_ERR_INVALID_ARG);
+  const int64_t row_bytes = int64_t(d) * int64_t(elem_size(dt));
+  TG_CHECK(row_bytes % 16 == 0 && row_bytes < (int64_t(1) << 30), TG_ERR_UNSUPPORTED);
+  TG_CHECK(aligned16(x) && aligned16(x_out), TG_ERR_INVALID_ARG);
+  return cuda_status(launch_compact(x, pos_in, scores, kept_idx, n, k, static_cast<int>(row_bytes),
+                                    x_out, pos_out, scores_out, nullptr,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tg_status tg_gated_attn_prefill(const void* q, const void* kk, const void* v, const int32_t* pos,
+                                const float* s, const float* gain, const float* tau, int64_t k,
+                                int32_t hq, int32_t hkv, int32_t dh, float rope_base,
+                                tg_dtype dt, void* out, void* ws, size_t ws_bytes,
+                                tg_stream stream) {
+  TG_CHECK(dt == TG_BF16 || dt == TG_F32, TG_ERR_UNSUPPORTED);
+  TG_CHECK(q && kk && v && pos && out && k >= 1 && hq >= 1 && hkv >= 1, TG_ERR_INVALID_ARG);
+  TG_CHECK(k < (int64_t(1) << 31) - 256, TG_ERR_INVALID_ARG);
+  TG_CHECK(hq % hkv == 0 && rope_base > 1.f, TG_ERR_INVALID_ARG);
+  if (dt == TG_BF16) {
+    TG_CHECK(dh == 128, TG_ERR_UNSUPPORTED);
+    TG_CHECK(aligned16(q) && aligned16(kk) && aligned16(v) && aligned16(out), TG_ERR_INVALID_ARG);
+  } else {
+    TG_CHECK(dh == 64 || dh == 128, TG_ERR_UNSUPPORTED);
+  }
+  AttnPlan plan(nullptr, k, hq, hkv, dh, dt, true);
+  TG_CHECK(ws != nullptr && ws_bytes >= plan.bytes, TG_ERR_WORKSPACE);
+  plan = AttnPlan(ws, k, hq, hkv, dh, dt, true);
+  return cuda_status(run_attention(q, int64_t(hq) * dh, kk, int64_t(hkv) * dh, v,
+                                   int64_t(hkv) * dh, pos, s, nullptr, gain, tau, nullptr, nullptr,
+                                   0.f, k, hq, hkv, dh, rope_base, dt, plan, nullptr, nullptr, out,
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protect, int64_t n,
+                     int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx, float* scores,
+                     const tg_kv* kv, void* ws, size_t ws_bytes, tg_stream stream) {
+  const tg_status vs = validate_model(model, n, k, gate_layer);
+  if (vs != TG_OK) return vs;
+  TG_CHECK(x && out && kept_idx, TG_ERR_INVALID_ARG);
+  const tg_model& m = *model;
+  if (m.dtype == TG_BF16) TG_CHECK(aligned16(x) && aligned16(out), TG_ERR_INVALID_ARG);
+  PrefillPlan P(nullptr, m, n, k);
+  TG_CHECK(ws != nullptr && ws_bytes >= P.bytes, TG_ERR_WORKSPACE);
+  P = PrefillPlan(ws, m, n, k);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t e = elem_size(m.dtype);
+  Dims D{m.d_model, m.n_heads_q, m.n_heads_kv, m.head_dim, m.d_ffn,
+         (m.n_heads_q + 2 * m.n_heads_kv) * m.head_dim};
+  float* sc = scores ? scores : P.scores;
+
+  TG_TRY(cudaMemcpyAsync(P.h, x, size_t(n) * D.d * e, cudaMemcpyDeviceToDevice, st));
+  // Stage 1: layers below the gate, and the gate layer's attention, over n rows.
+  for (int l = 0; l < gate_layer; ++l) {
+    TG_TRY(attention_sublayer(m, m.layers[l], D, P, P.h, n, nullptr, nullptr, nullptr, nullptr,
+                              kv ? &kv[l] : nullptr, st));
+    TG_TRY(ffn_sublayer(m, m.layers[l], D, P, P.h, n, st));
+  }
+  if (gate_layer >= 0)
+    TG_TRY(attention_sublayer(m, m.layers[gate_layer], D, P, P.h, n, nullptr, nullptr, nullptr,
+                              nullptr, kv ? &kv[gate_layer] : nullptr, st));
+  // Stage 2: score the post-attention residual, select, compact.
+  TG_TRY(run_score(P.h, n, D.d, m.d_score, m.score_norm, m.norm_eps, m.score_w1, m.score_b1,
+                   m.score_w2, m.score_b2, m.dtype, sc, P.y, P.hpre, st));
+  TG_TRY(launch_topk_select(sc, protect, n, k, kept_idx, P.sel_ws, st));
+  TG_TRY(launch_compact(P.h, nullptr, sc, kept_idx, n, k, static_cast<int>(D.d * e), P.hk, P.pos_k,
+                        P.s_k, P.lsig_k, st));
+  // Stage 3: the gate layer's FFN and the layers above, over the k kept rows.
+  if (gate_layer >= 0) TG_TRY(ffn_sublayer(m, m.layers[gate_layer], D, P, P.hk, k, st));
+  for (int l = gate_layer + 1; l < m.n_layers; ++l) {
+    const tg_layer& L = m.layers[l];
+    TG_TRY(attention_sublayer(m, L, D, P, P.hk, k, P.pos_k, P.lsig_k, L.gain, L.tau,
+                              kv ? &kv[l] : nullptr, st));
+    TG_TRY(ffn_sublayer(m, L, D, P, P.hk, k, st));
+  }
+  if (m.final_norm)
+    TG_TRY(launch_rmsnorm(P.hk, m.final_norm, m.norm_eps, k, D.d, m.dtype == TG_BF16, out, st));
+  else
+    TG_TRY(cudaMemcpyAsync(out, P.hk, size_t(k) * D.d * e, cudaMemcpyDeviceToDevice, st));
+  return TG_OK;
+}
+
+const char* tg_status_string(tg_status s) {
+  switch (s) {
+    case TG_OK: return "ok";
+    case TG_ERR_INVALID_ARG: return "invalid argument";
+    case TG_ERR_UNSUPPORTED: return "unsupported dtype or shape";
+    case TG_ERR_BUDGET: return "invalid budget (k < 1, k > n, or more protected tokens than k)";
+    case TG_ERR_WORKSPACE: return "workspace too small";
+    case TG_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+int tg_last_cuda_error(void) { return t_last_cuda_error; }
+
+tg_status tg_device_error(uint32_t* word, int clear) {
+  TG_CHECK(word != nullptr, TG_ERR_INVALID_ARG);
+  unsigned int v = 0;
+  TG_TRY(cudaMemcpyFromSymbol(&v, g_tg_error_word, sizeof(v)));
+  *word = v;
+  if (clear) {
+    const unsigned int z = 0;
+    TG_TRY(cudaMemcpyToSymbol(g_tg_error_word, &z, sizeof(z)));
+  }
+  return TG_OK;
+}
+
+const char* tg_version(void) { return "tokengate-b200 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

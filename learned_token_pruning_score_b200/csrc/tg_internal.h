@@ -1,0 +1,115 @@
+// tg_internal.h -- launchers shared between the kernel files and the C ABI.
+// Host code only. Each launcher enqueues work on `st` and returns the launch
+// status (cudaSuccess or the CUDA error); argument checks are the caller's.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace tg {
+
+// Rounds `x` up to a multiple of `a` (a power of two).
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) & ~(a - 1); }
+
+// Bump allocator over a caller-provided workspace. carve() returns nullptr
+// in size-only mode (base == nullptr) so the same code computes sizes.
+struct Arena {
+  char* base;
+  size_t used;
+  explicit Arena(void* b) : base(static_cast<char*>(b)), used(0) {}
+  void* carve(size_t bytes) {
+    used = align_up(used, 256);
+    void* p = base ? base + used : nullptr;
+    used += bytes;
+    return p;
+  }
+};
+
+int num_sms();
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device).
+cudaError_t set_smem_attr_once(const void* fn, int bytes);
+unsigned int* device_error_word();  // device address of the sticky error word
+
+// ---- selection (k_select.cu)
+size_t select_ws_bytes(int64_t n);
+cudaError_t launch_topk_select(const float* scores, const uint8_t* protect, int64_t n, int64_t k,
+                               int32_t* kept_idx, void* ws, cudaStream_t st);
+
+// ---- compaction (k_compact.cu). Optional lsig_out[r] = logsigmoid(scores[idx[r]]).
+cudaError_t launch_compact(const void* x, const int32_t* pos_in, const float* scores,
+                           const int32_t* kept_idx, int64_t n, int64_t k, int row_bytes,
+                           void* x_out, int32_t* pos_out, float* scores_out, float* lsig_out,
+                           cudaStream_t st);
+
+// ---- row-wise kernels (k_rowwise.cu)
+cudaError_t launch_rmsnorm(const void* x, const float* gamma, float eps, int64_t rows, int d,
+                           bool bf16, void* y, cudaStream_t st);
+
+// RoPE/qk-norm preparation of one attention call.
+//  src rows: q at q_src + t*q_stride, k at k_src + t*k_stride, v at v_src + t*v_stride
+//  (element strides, dtype elements). Writes:
+//   q_out [T, hq, dh], k_out [T, hkv, dh] (rotated, optional qk-norm),
+//   bf16 only: vT_out [hkv, dh, t_pad] (zero in columns >= T)
+//   fp32 only: v_out [T, hkv, dh] (plain copy) when v_out != nullptr
+//   kv_v_out [T, hkv, dh] (copy of v) when non-null
+//   lsig_out [T] = logsigmoid(s) when s != nullptr
+struct RopePrepArgs {
+  const void* q_src; const void* k_src; const void* v_src;
+  int64_t q_stride, k_stride, v_stride;
+  const int32_t* pos;  // nullptr: position = row index
+  const float* q_norm; const float* k_norm; float eps;
+  int64_t T; int hq, hkv, dh; float rope_base; bool bf16;
+  void* q_out; void* k_out; void* vT_out; int64_t t_pad; void* v_out; void* kv_v_out;
+  const float* s; float* lsig_out;
+};
+cudaError_t launch_rope_prep(const RopePrepArgs& a, cudaStream_t st);
+
+// fp32 helpers used by the SIMT path
+cudaError_t launch_swiglu_f32(const float* gu, int64_t rows, int inter, float* h, cudaStream_t st);
+cudaError_t launch_score_dot_f32(const float* hpre, int64_t rows, int f, const float* b1,
+                                 const float* w2, const float* b2, float* scores, cudaStream_t st);
+
+// ---- GEMMs. C[M,N] = A[M,K] . B[N,K]^T with an epilogue.
+enum EpiKind { EPI_STORE = 0, EPI_RESIDUAL = 1, EPI_SWIGLU = 2, EPI_SCORE = 3 };
+struct GemmArgs {
+  const void* A; int64_t lda;      // [M, K] elements, row stride lda
+  const void* B; int64_t ldb;      // [N, K]
+  void* C; int64_t ldc;            // [M, N] (SWIGLU: [M, N/2]); unused for SCORE
+  const void* R; int64_t ldr;      // residual [M, N] (EPI_RESIDUAL), may equal C
+  int64_t M; int N; int K;
+  EpiKind epi;
+  int inter;                       // SWIGLU: I (B rows [0,I) gate, [I,2I) up), N = 2I
+  const float* b1; const float* w2; const float* b2; float* scores;  // SCORE
+};
+// bf16 on the 5th-generation tensor cores (k_gemm_tc.cu)
+bool gemm_tc_supported(const GemmArgs& g);
+cudaError_t launch_gemm_tc(const GemmArgs& g, cudaStream_t st);
+// fp32 SIMT (k_gemm_simt.cu); SWIGLU and SCORE are not handled here (the
+// caller stores the product and runs the fp32 helpers above).
+cudaError_t launch_gemm_simt_f32(const GemmArgs& g, cudaStream_t st);
+
+// ---- attention. q [T,hq,dh] rotated, k [T,hkv,dh] rotated, lsig [T] or null.
+struct AttnArgs {
+  const void* q; const void* k; const void* v;  // v: bf16 -> vT [hkv, dh, t_pad]; fp32 -> [T,hkv,dh]
+  int64_t t_pad;  // bf16: padded token count of vT; fp32: row stride of v in elements (0 = hkv*dh)
+  const float* lsig; const float* gain; const float* tau;
+  int64_t T; int hq, hkv, dh;
+  void* out;                                    // [T, hq, dh]
+};
+bool attn_tc_supported(const AttnArgs& a);
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st);      // bf16, tcgen05
+cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t st); // fp32 SIMT
+
+// ---- tensor maps (tg_tmap.cu)
+// 2-D bf16 tensor map, row-major [rows, cols] with row stride ld (elements),
+// box [box_rows, 64 cols], 128-byte swizzle. Returns false on failure.
+bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                       int box_rows);
+// 3-D bf16 tensor map over dims (x fastest): sizes {d0, d1, d2}, byte strides
+// {s1, s2} of dims 1 and 2, box {64, b1, b2}, 128-byte swizzle.
+bool make_tmap_3d_bf16(CUtensorMap* m, const void* base, int64_t d0, int64_t d1, int64_t d2,
+                       int64_t s1_bytes, int64_t s2_bytes, int b1, int b2);
+
+}  // namespace tg

@@ -1,0 +1,149 @@
+"""The C ABI on the host: the library loads, exports every declared symbol,
+sizes workspaces, and rejects bad arguments before launching anything.
+
+None of these calls reaches a kernel: each one fails host-side validation,
+so they run on a machine without a GPU.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import learned_token_pruning_score_b200 as tg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tokengate.h")
+BOGUS = ctypes.c_void_p(4096)  # never dereferenced: every call below fails validation first
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tg_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_functions()
+    assert {"tg_score", "tg_topk_select", "tg_compact", "tg_gated_attn_prefill",
+            "tg_prefill", "tg_workspace_size", "tg_status_string"} <= set(names)
+    lib = ctypes.CDLL(tg.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_version():
+    assert tg.tg_status_string(tg.TG_OK) == "ok"
+    for s in range(1, 6):
+        assert len(tg.tg_status_string(s)) > 3
+    assert "sm_100a" in tg.tg_version()
+
+
+def test_workspace_sizes():
+    a = tg.tg_workspace_size(tg.TG_OP_TOPK_SELECT, n=8192)
+    b = tg.tg_workspace_size(tg.TG_OP_TOPK_SELECT, n=131072)
+    assert 0 < a < b
+    assert tg.tg_workspace_size(tg.TG_OP_COMPACT, n=10, k=5) == 0
+    s1 = tg.tg_workspace_size(tg.TG_OP_GATED_ATTN, k=2048, n_heads_q=16, n_heads_kv=8,
+                              head_dim=128, dtype=tg.TG_BF16)
+    # q, k, V^T (bf16) and the per-key bias
+    assert s1 >= 2048 * 16 * 128 * 2 + 2048 * 8 * 128 * 2 * 2 + 2048 * 4
+    p = dict(d_model=2048, n_heads_q=16, n_heads_kv=8, head_dim=128, d_score=256, d_ffn=6144,
+             n_layers=28, gate_layer=1, dtype=tg.TG_BF16)
+    assert tg.tg_workspace_size(tg.TG_OP_PREFILL, n=32768, k=4096, **p) > \
+        tg.tg_workspace_size(tg.TG_OP_PREFILL, n=16384, k=4096, **p)
+
+
+def test_select_validation():
+    f = tg._topk
+    assert f(None, None, 10, 5, BOGUS, BOGUS, 1 << 20, None) == tg.TG_ERR_INVALID_ARG
+    assert f(BOGUS, None, 10, 0, BOGUS, BOGUS, 1 << 20, None) == tg.TG_ERR_BUDGET
+    assert f(BOGUS, None, 10, 11, BOGUS, BOGUS, 1 << 20, None) == tg.TG_ERR_BUDGET
+    assert f(BOGUS, None, 10, 5, BOGUS, BOGUS, 4, None) == tg.TG_ERR_WORKSPACE
+    assert f(BOGUS, None, 10, 5, BOGUS, None, 1 << 20, None) == tg.TG_ERR_WORKSPACE
+
+
+def test_compact_validation():
+    f = tg._compact
+    assert f(BOGUS, None, None, BOGUS, 10, 11, 64, tg.TG_BF16, BOGUS, BOGUS, None, None) == \
+        tg.TG_ERR_BUDGET
+    # 6 bf16 = 12-byte rows cannot be copied in 16-byte vectors
+    assert f(BOGUS, None, None, BOGUS, 10, 5, 6, tg.TG_BF16, BOGUS, BOGUS, None, None) == \
+        tg.TG_ERR_UNSUPPORTED
+    assert f(BOGUS, None, None, BOGUS, 10, 5, 64, 7, BOGUS, BOGUS, None, None) == \
+        tg.TG_ERR_UNSUPPORTED
+    # scores_out requested without scores
+    assert f(BOGUS, None, None, BOGUS, 10, 5, 64, tg.TG_BF16, BOGUS, BOGUS, BOGUS, None) == \
+        tg.TG_ERR_INVALID_ARG
+    unaligned = ctypes.c_void_p(4096 + 2)
+    assert f(unaligned, None, None, BOGUS, 10, 5, 64, tg.TG_BF16, BOGUS, BOGUS, None, None) == \
+        tg.TG_ERR_INVALID_ARG
+
+
+def test_score_validation():
+    f = tg._score
+    args = [BOGUS, 100, 2048, 256, BOGUS, 1e-6, BOGUS, None, BOGUS, None]
+    assert f(*args, tg.TG_BF16, BOGUS, BOGUS, 16, None) == tg.TG_ERR_WORKSPACE
+    a2 = list(args)
+    a2[3] = 512  # F > 256 is not built for bf16
+    assert f(*a2, tg.TG_BF16, BOGUS, BOGUS, 1 << 30, None) == tg.TG_ERR_UNSUPPORTED
+    a3 = list(args)
+    a3[0] = None
+    assert f(*a3, tg.TG_BF16, BOGUS, BOGUS, 1 << 30, None) == tg.TG_ERR_INVALID_ARG
+
+
+def test_attention_validation():
+    f = tg._attn
+    base = [BOGUS, BOGUS, BOGUS, BOGUS, None, None, None, 128]
+    assert f(*base, 4, 2, 64, 1e6, tg.TG_BF16, BOGUS, BOGUS, 1 << 30, None) == \
+        tg.TG_ERR_UNSUPPORTED  # bf16 head_dim 64 is not built
+    assert f(*base, 4, 3, 128, 1e6, tg.TG_BF16, BOGUS, BOGUS, 1 << 30, None) == \
+        tg.TG_ERR_INVALID_ARG  # hq % hkv != 0
+    assert f(*base, 4, 2, 128, 1e6, tg.TG_BF16, BOGUS, BOGUS, 64, None) == tg.TG_ERR_WORKSPACE
+    assert f(*base, 4, 2, 96, 1e6, tg.TG_F32, BOGUS, BOGUS, 1 << 30, None) == \
+        tg.TG_ERR_UNSUPPORTED
+
+
+def _bogus_model(**over):
+    layers = (tg.TgLayer * 2)()
+    for i in range(2):
+        for name, _ in tg.TgLayer._fields_:
+            setattr(layers[i], name, 4096)
+        layers[i].q_norm = None
+        layers[i].k_norm = None
+    m = tg.TgModel(tg.TG_BF16, 2, 2048, 16, 8, 128, 6144, 256, 1e-6, 1e6, layers, 4096, 4096,
+                   4096, None, 4096, None)
+    for k, v in over.items():
+        setattr(m, k, v)
+    return m, layers
+
+
+def test_prefill_validation():
+    f = tg._prefill
+    m, keep = _bogus_model()
+    assert f(ctypes.byref(m), BOGUS, None, 1000, 0, 1, BOGUS, BOGUS, None, None, BOGUS, 1 << 40,
+             None) == tg.TG_ERR_BUDGET
+    assert f(ctypes.byref(m), BOGUS, None, 1000, 100, 2, BOGUS, BOGUS, None, None, BOGUS, 1 << 40,
+             None) == tg.TG_ERR_INVALID_ARG  # gate layer past the stack
+    assert f(ctypes.byref(m), BOGUS, None, 1000, 100, 1, BOGUS, BOGUS, None, None, BOGUS, 16,
+             None) == tg.TG_ERR_WORKSPACE
+    m2, keep2 = _bogus_model(head_dim=64)
+    assert f(ctypes.byref(m2), BOGUS, None, 1000, 100, 1, BOGUS, BOGUS, None, None, BOGUS,
+             1 << 40, None) == tg.TG_ERR_UNSUPPORTED
+    m3, keep3 = _bogus_model(d_ffn=6100)  # SwiGLU width must be a multiple of 128 in bf16
+    assert f(ctypes.byref(m3), BOGUS, None, 1000, 100, 1, BOGUS, BOGUS, None, None, BOGUS,
+             1 << 40, None) == tg.TG_ERR_UNSUPPORTED
+    assert f(None, BOGUS, None, 1000, 100, 1, BOGUS, BOGUS, None, None, BOGUS, 1 << 40, None) == \
+        tg.TG_ERR_INVALID_ARG
+    keep[0].k_norm = 4096  # q_norm and k_norm come together
+    assert f(ctypes.byref(m), BOGUS, None, 1000, 100, 1, BOGUS, BOGUS, None, None, BOGUS,
+             1 << 40, None) == tg.TG_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="exercises the no-device error path")
+def test_device_error_without_a_device_is_a_cuda_error():
+    with pytest.raises(tg.TokenGateError) as ei:
+        tg.tg_device_error()
+    assert ei.value.status == tg.TG_ERR_CUDA
