@@ -1,0 +1,627 @@
+#!/usr/bin/env python
+"""Benchmark of the gated prefill on B200.
+
+Default workload: the 28-layer Qwen3-1.7B-shaped gated prefill in bf16 at
+batch 1 -- N = 32768 tokens, gate at layer 1, K = 4096 kept tokens, the last
+128 protected, qk-norm on, seeded random weights and N(0,1) hidden states in
+place of the embedding lookup. One step = one tg_prefill call: every stage
+of the path (dense layers over N, scorer, select, compact, gated layers over
+K, final norm).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python bench.py --sweep      # select+compact sweep and the 128K gated layer
+
+Prints one JSON line (rank 0). `value` = tokens/s (N / TTFT) summed over the
+ranks; ranks run independent replicas (the path has no exchange step).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "gated-prefill tokens/s (N/TTFT) at N=32K"
+UNIT = "tokens/s"
+WORKLOAD = synth.QWEN_PREFILL_32K
+HEADLINE_K = 4096
+SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+LAUNCHES_PER_RECORD = {"select": 5, "rope_prep": 2, "copy": 0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"],
+                    bf16_sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ----------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    def __init__(self, gpu_index: int):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={SMI_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, reasons, mx = [], set(), None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- helpers
+
+
+def kernel_source_hash(name: str) -> str:
+    files = {"attention_tc": "k_attn_tc.cu", "gemm_tc": "k_gemm_tc.cu"}
+    key = "gemm_tc" if name.startswith("gemm_tc") else name
+    f = files.get(key)
+    if f is None:
+        return ""
+    with open(os.path.join(ROOT, "learned_token_pruning_score_b200", "csrc", f), "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:12]
+
+
+def traffic_from_profiles(kernel: str, workload: str):
+    """dram bytes per launch of `kernel` from the committed ncu summary, or
+    None if absent or taken on another revision of the kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash(kernel)
+    with open(path) as fh:
+        for line in fh:
+            if line.startswith("#") or not line.strip():
+                continue
+            kv = dict(tok.split("=", 1) for tok in line.split() if "=" in tok)
+            if kv.get("kernel") == kernel and kv.get("workload") == workload and \
+                    kv.get("src") == want:
+                return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+def build_model(tg, torch, w, device):
+    p = synth.torch_model_params(w, seed=w.seed, device=device)
+    score = {k: p[k] for k in ("score_norm", "score_w1", "score_b1", "score_w2", "score_b2")}
+    return tg.Model(n_heads_q=w.hq, n_heads_kv=w.hkv, head_dim=w.dh, layers=p["layers"],
+                    score=score, final_norm=p["final_norm"], eps=w.eps, rope_base=w.rope_base)
+
+
+def dense_model(tg, model):
+    layers = [{k: v for k, v in lw.items() if k not in ("gain", "tau")} for lw in model.layers]
+    return tg.Model(n_heads_q=model.n_heads_q, n_heads_kv=model.n_heads_kv,
+                    head_dim=model.head_dim, layers=layers, score=model.score,
+                    final_norm=model.final_norm, eps=model.eps, rope_base=model.rope_base)
+
+
+# ----------------------------------------------------------------- oracle CPU leg
+
+
+def oracle_sample(seconds: float, rows: int = 2048):
+    """Times the oracle on a bounded sample of the workload: one gated upper
+    layer (attention + SwiGLU, the workload's shapes) over `rows` kept rows,
+    repeated until `seconds` elapse. Returns (FLOP/s, sample description,
+    threads used)."""
+    from oracle import tokengate_oracle as ref
+
+    w = WORKLOAD
+    rng = synth.rng_for(w.seed)
+    lp = synth.layer_params(w, rng, upper=True)
+    lw = ref.Layer(attn_norm=lp["attn_norm"], wqkv=ref.round_bf16(lp["wqkv"]),
+                   wo=ref.round_bf16(lp["wo"]), ffn_norm=lp["ffn_norm"],
+                   w_gate_up=ref.round_bf16(lp["w_gate_up"]), w_down=ref.round_bf16(lp["w_down"]),
+                   q_norm=lp["q_norm"], k_norm=lp["k_norm"], gain=lp["gain"], tau=lp["tau"])
+    m = ref.Model(d_model=w.d, n_heads_q=w.hq, n_heads_kv=w.hkv, head_dim=w.dh, layers=[lw],
+                  final_norm=None, score_norm=np.ones(w.d), score_w1=np.zeros((1, w.d)),
+                  score_b1=None, score_w2=np.zeros(1), score_b2=None)
+    x = ref.round_bf16(rng.standard_normal((rows, w.d)))
+    pos = np.sort(rng.choice(w.n, rows, replace=False)).astype(np.int32)
+    s = rng.standard_normal(rows).astype(np.float32)
+    flops_one = layer_flops(w, rows)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        ref.gated_layer_forward(x, pos, s, lw, m)
+        reps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count() or 1
+    desc = (f"oracle gated upper layer (Qwen3-1.7B shapes, {rows} rows) x{reps} in {dt:.1f} s; "
+            f"TTFT extrapolated by algorithmic FLOPs of the full workload")
+    return flops_one * reps / dt, desc, threads, dt
+
+
+def layer_flops(w, t, with_ffn=True):
+    qkv = (w.hq + 2 * w.hkv) * w.dh
+    f = 2.0 * t * w.d * qkv + 4.0 * w.dh * w.hq * t * (t + 1) / 2 + 2.0 * t * w.hq * w.dh * w.d
+    if with_ffn:
+        f += 2.0 * t * w.d * 2 * w.inter + 2.0 * t * w.inter * w.d
+    return f
+
+
+def workload_flops(w, k):
+    n, L = w.n, w.gate_layer
+    f = L * layer_flops(w, n) + layer_flops(w, n, with_ffn=False)
+    f += 2.0 * n * w.d * w.f  # scorer
+    f += 2.0 * k * w.d * 3 * w.inter  # gate layer's FFN on K
+    f += (w.n_layers - L - 1) * layer_flops(w, k)
+    return f
+
+
+# ----------------------------------------------------------------- reference arm
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    w = WORKLOAD
+    per_step = []
+    desc = ""
+    threads = 1
+    for i in range(args.warmup + args.steps):
+        rate, desc, threads, dt = oracle_sample(seconds=0.0, rows=1024)
+        if i >= args.warmup:
+            per_step.append(w.n / (workload_flops(w, HEADLINE_K) / rate))
+    value = statistics.mean(per_step)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * w.n / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "n": w.n, "k": HEADLINE_K, "layers": w.n_layers,
+                   "gate_layer": w.gate_layer, "d_model": w.d, "heads": f"{w.hq}/{w.hkv}x{w.dh}",
+                   "protected": w.n_protect},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- our arm
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import learned_token_pruning_score_b200 as tg
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist  # noqa: F811
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    w = WORKLOAD
+    k = args.budget
+    pk = peaks()
+    model = build_model(tg, torch, w, device)
+    x = synth.torch_hidden_states(w, seed=w.seed + 1000 + rank, device=str(device))
+    prot = torch.zeros(w.n, dtype=torch.uint8, device=device)
+    prot[w.n - w.n_protect:] = 1
+    out = torch.empty(k, w.d, dtype=torch.bfloat16, device=device)
+    kept = torch.empty(k, dtype=torch.int32, device=device)
+    scores = torch.empty(w.n, dtype=torch.float32, device=device)
+    ws = torch.empty(model.workspace_size(w.n, k, w.gate_layer), dtype=torch.uint8, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
+    stream = torch.cuda.current_stream(device)
+    tg.tg_device_error(clear=True)
+
+    def step():
+        tg.tg_prefill(model, x, prot, k, w.gate_layer, out=out, kept_idx=kept, scores=scores,
+                      ws=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # ---- timed region: device time of each step with events; L2 flushed
+    # between steps (outside the events); launches traced for the roofline.
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    t_wall = time.perf_counter()
+    tg.tg_trace_start(1 << 16)
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        torch.cuda.nvtx.range_push("tg_step")
+        step()
+        torch.cuda.nvtx.range_pop()
+        stops[i].record(stream)
+    torch.cuda.synchronize()
+    trace = tg.tg_trace_stop()
+    barrier()
+    wall = time.perf_counter() - t_wall
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
+    total_ms = sum(step_ms)
+    if dist is not None:
+        t = torch.tensor([total_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * w.n * args.steps / (total_ms / 1000.0)
+    err_word = tg.tg_device_error()
+
+    # ---- per-kernel breakdown from the trace (timed steps only)
+    per = {}
+    for r in trace:
+        key = r["kernel"]
+        if r["kernel"] == "attention_tc":
+            key = "attention_tc_dense" if r["layer"] <= w.gate_layer else "attention_tc_gated"
+        e = per.setdefault(key, {"ms": 0.0, "flops": 0.0, "bytes": 0.0, "launches": 0})
+        e["ms"] += r["ms"]
+        e["flops"] += r["flops"]
+        e["bytes"] += r["bytes"]
+        e["launches"] += LAUNCHES_PER_RECORD.get(r["kernel"], 1)
+    traced_ms = sum(e["ms"] for e in per.values())
+    by_kernel = {}
+    for key, e in sorted(per.items(), key=lambda kv: -kv[1]["ms"]):
+        d = {"ms_per_step": e["ms"] / args.steps, "share": e["ms"] / traced_ms,
+             "launches_per_step": e["launches"] / args.steps}
+        if e["flops"] > 0:
+            d["tflops"] = e["flops"] / (e["ms"] / 1e3) / 1e12
+        else:
+            d["gbs"] = e["bytes"] / (e["ms"] / 1e3) / 1e9
+        by_kernel[key] = d
+    # dominant kernel = largest total device time among traced kernels
+    kern_tot = {}
+    for r in trace:
+        kern_tot.setdefault(r["kernel"], [0.0, 0.0, 0.0, 0])
+        kt = kern_tot[r["kernel"]]
+        kt[0] += r["ms"]
+        kt[1] += r["flops"]
+        kt[2] += r["bytes"]
+        kt[3] += 1
+    dom = max(kern_tot, key=lambda n: kern_tot[n][0])
+    dms, dfl, dby, dn = kern_tot[dom]
+    tensor_bound = dfl > 0
+    if tensor_bound:
+        achieved = dfl / (dms / 1e3) / 1e12
+        peak = pk["bf16_sustained"]
+        unit = "TFLOP/s"
+    else:
+        achieved = dby / (dms / 1e3) / 1e9
+        peak = pk["hbm"]
+        unit = "GB/s"
+    traffic = traffic_from_profiles(dom, w.name)
+    roofline = {"bound": "tensor" if tensor_bound else "hbm", "kernel": dom,
+                "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                "peak_source": f"{pk['source']} ({'bf16_tflops_sustained' if tensor_bound else 'hbm_gbs'})",
+                "traffic": traffic, "algorithmic_per_launch": (dfl if tensor_bound else dby) / dn,
+                "launches": dn}
+    att_g = per.get("attention_tc_gated", {})
+    att_d = per.get("attention_tc_dense", {})
+    sel = per.get("select", {"ms": 0, "bytes": 0})
+    cmp_ = per.get("compact", {"ms": 0, "bytes": 0})
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_host = x.cpu().pin_memory()
+        prot_host = prot.cpu().pin_memory()
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        kept_host = torch.empty(kept.shape, dtype=kept.dtype).pin_memory()
+        x_dev = torch.empty_like(x)
+        prot_dev = torch.empty_like(prot)
+
+        def e2e_step():
+            x_dev.copy_(x_host, non_blocking=True)
+            prot_dev.copy_(prot_host, non_blocking=True)
+            tg.tg_prefill(model, x_dev, prot_dev, k, w.gate_layer, out=out, kept_idx=kept,
+                          scores=scores, ws=ws, stream=stream)
+            out_host.copy_(out, non_blocking=True)
+            kept_host.copy_(kept, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([e_ms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = x.numel() * x.element_size() + prot.numel()
+        d2h = out.numel() * out.element_size() + kept.numel() * 4
+        e2e = {"value": world * w.n * args.steps / (e_ms / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e_ms / args.steps}
+
+    # ---- other budgets, dense baseline and peak memory (not timed region)
+    extras = {}
+    if not args.quick:
+        def ttft(mdl, kk, reps=3):
+            o = torch.empty(kk, w.d, dtype=torch.bfloat16, device=device)
+            ki = torch.empty(kk, dtype=torch.int32, device=device)
+            wsz = torch.empty(mdl.workspace_size(w.n, kk, w.gate_layer), dtype=torch.uint8,
+                              device=device)
+            tg.tg_prefill(mdl, x, prot, kk, w.gate_layer, out=o, kept_idx=ki, ws=wsz)
+            torch.cuda.synchronize()
+            torch.cuda.reset_peak_memory_stats(device)
+            ms = []
+            for _ in range(reps):
+                flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                tg.tg_prefill(mdl, x, prot, kk, w.gate_layer, out=o, kept_idx=ki, ws=wsz)
+                b.record(stream)
+                torch.cuda.synchronize()
+                ms.append(a.elapsed_time(b))
+            mem = torch.cuda.max_memory_allocated(device)
+            del o, ki, wsz
+            return statistics.median(ms), mem
+
+        del ws
+        torch.cuda.empty_cache()
+        for kk in synth.PREFILL_32K_BUDGETS:
+            t_ms, mem = ttft(model, kk)
+            extras[f"gated_k{kk}"] = {"ttft_ms": t_ms, "tokens_per_s": w.n / (t_ms / 1e3),
+                                      "tflop": workload_flops(w, kk) / 1e12,
+                                      "peak_mem_gb": mem / 1e9}
+        t_ms, mem = ttft(dense_model(tg, model), w.n)
+        extras["dense"] = {"ttft_ms": t_ms, "tokens_per_s": w.n / (t_ms / 1e3),
+                           "tflop": workload_flops(w, w.n) / 1e12, "peak_mem_gb": mem / 1e9}
+        for kk in synth.PREFILL_32K_BUDGETS:
+            g = extras[f"gated_k{kk}"]
+            g["ttft_speedup_vs_dense"] = extras["dense"]["ttft_ms"] / g["ttft_ms"]
+            g["peak_mem_reduction_vs_dense"] = extras["dense"]["peak_mem_gb"] / g["peak_mem_gb"]
+
+    # ---- CPU baseline: the oracle, rank 0 only, N = 1
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        rate, desc, threads, _ = oracle_sample(seconds=args.cpu_seconds)
+        cpu_tps = w.n / (workload_flops(w, k) / rate)
+        cpu = {"value": cpu_tps, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": desc, "extrapolated": True}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded random weights and N(0,1) hidden states)",
+            "config": {"workload": w.name, "n": w.n, "k": k, "layers": w.n_layers,
+                       "gate_layer": w.gate_layer, "d_model": w.d,
+                       "heads": f"{w.hq}/{w.hkv}x{w.dh}", "ffn": w.inter, "scorer": w.f,
+                       "protected": w.n_protect, "qk_norm": w.qk_norm,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "flushed between timed steps (256 MB write); inputs > L2"},
+            "ttft_ms": ms_per_step,
+            "tflop_per_step": workload_flops(w, k) / 1e12,
+            "model_tflops": workload_flops(w, k) / (ms_per_step / 1e3) / 1e12,
+            "roofline": roofline,
+            "attn_gated_tflops": att_g and att_g["flops"] / (att_g["ms"] / 1e3) / 1e12,
+            "attn_dense_tflops": att_d and att_d["flops"] / (att_d["ms"] / 1e3) / 1e12,
+            "attn_gated_frac_of_peak": att_g and
+            att_g["flops"] / (att_g["ms"] / 1e3) / 1e12 / pk["bf16_sustained"],
+            "select_compact_gbs": (sel["bytes"] + cmp_["bytes"]) /
+            max(1e-9, (sel["ms"] + cmp_["ms"]) / 1e3) / 1e9,
+            "by_kernel": by_kernel,
+            "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(sum(e["launches"] for e in per.values())),
+            "clocks": clk, "wall_s_timed": wall, "device_error_word": err_word,
+            "extras": extras,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- sweep mode
+
+
+def run_sweep(args):
+    """Select+compact over the sweep points (HBM roofline) and the 128K
+    long-context gated layer; one JSON line per point."""
+    import torch
+
+    import learned_token_pruning_score_b200 as tg
+    from oracle import tokengate_oracle as ref
+
+    device = torch.device("cuda", 0)
+    pk = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    for n, k in synth.sweep_points():
+        rng = synth.rng_for(synth.SWEEP_SEED)
+        s = torch.from_numpy(synth.sweep_scores(n, rng)).to(device)
+        prot = torch.from_numpy(synth.protect_tail(n, synth.SWEEP_PROTECT)).to(device)
+        x = torch.randn(n, synth.SWEEP_D, device=device, dtype=torch.bfloat16)
+        idx = torch.empty(k, dtype=torch.int32, device=device)
+        xo = torch.empty(k, synth.SWEEP_D, device=device, dtype=torch.bfloat16)
+        po = torch.empty(k, dtype=torch.int32, device=device)
+        so = torch.empty(k, dtype=torch.float32, device=device)
+        ws = torch.empty(tg.tg_workspace_size(tg.TG_OP_TOPK_SELECT, n=n), dtype=torch.uint8,
+                         device=device)
+
+        def once():
+            tg.tg_topk_select(s, prot, k, kept_idx=idx, ws=ws)
+            tg.tg_compact(x, idx, scores=s, x_out=xo, pos_out=po, scores_out=so)
+
+        for _ in range(3):
+            once()
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            once()
+            b.record()
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        t = statistics.median(ms)
+        byt = ref.select_compact_bytes(n, k, synth.SWEEP_D)
+        gbs = byt / (t / 1e3) / 1e9
+        print(json.dumps({"sweep": "select+compact", "n": n, "k": k, "us": t * 1e3,
+                          "bytes": byt, "gbs": gbs, "frac_hbm": gbs / pk["hbm"]}), flush=True)
+
+
+# ----------------------------------------------------------------- profiling cases
+
+
+def run_case(args):
+    """Small, repeatable invocations of one kernel family for ncu captures.
+
+    attn:  tg_gated_attn_prefill over `rows` rows, Qwen3-1.7B heads (16/8 x 128),
+           gate bias on -- the attention kernel (plus its RoPE prep).
+    layer: tg_prefill of a 2-layer Qwen3-1.7B-shaped model, gate at layer 0,
+           N = rows, K = rows / 8 -- every GEMM epilogue, select and compact.
+    """
+    import torch
+
+    import learned_token_pruning_score_b200 as tg
+
+    device = torch.device("cuda", 0)
+    torch.manual_seed(0)
+    w = WORKLOAD
+    t = args.rows
+    if args.case == "attn":
+        q = torch.randn(t, w.hq, w.dh, device=device, dtype=torch.bfloat16)
+        kk = torch.randn(t, w.hkv, w.dh, device=device, dtype=torch.bfloat16)
+        v = torch.randn(t, w.hkv, w.dh, device=device, dtype=torch.bfloat16)
+        pos = torch.arange(t, dtype=torch.int32, device=device)
+        s = torch.randn(t, device=device)
+        gain = torch.rand(w.hq, device=device) * 2
+        tau = torch.rand(w.hq, device=device) + 0.5
+        out = torch.empty_like(q)
+        ws = torch.empty(tg.tg_workspace_size(tg.TG_OP_GATED_ATTN, k=t, n_heads_q=w.hq,
+                                              n_heads_kv=w.hkv, head_dim=w.dh),
+                         dtype=torch.uint8, device=device)
+        run = lambda: tg.tg_gated_attn_prefill(q, kk, v, pos, s, gain, tau, out=out, ws=ws)  # noqa: E731
+    else:
+        wl = synth.shrink(w, n=t, k=max(128, t // 8), n_layers=2, gate_layer=0)
+        model = build_model(tg, torch, wl, device)
+        x = synth.torch_hidden_states(wl, seed=1, device=str(device))
+        ws = torch.empty(model.workspace_size(wl.n, wl.k, 0), dtype=torch.uint8, device=device)
+        out = torch.empty(wl.k, wl.d, dtype=torch.bfloat16, device=device)
+        kept = torch.empty(wl.k, dtype=torch.int32, device=device)
+        run = lambda: tg.tg_prefill(model, x, None, wl.k, 0, out=out, kept_idx=kept, ws=ws)  # noqa: E731
+    for _ in range(args.steps):
+        run()
+    torch.cuda.synchronize()
+    assert tg.tg_device_error() == 0
+    print(json.dumps({"case": args.case, "rows": t, "reps": args.steps}))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--budget", type=int, default=HEADLINE_K)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--quick", action="store_true", help="skip the other budgets / dense run")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--case", choices=["attn", "layer"], default=None)
+    ap.add_argument("--rows", type=int, default=32768)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if args.sweep:
+        return run_sweep(args)
+    if args.case:
+        return run_case(args)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

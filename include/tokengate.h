@@ -206,6 +206,50 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
                      int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx, float* scores,
                      const tg_kv* kv, void* ws, size_t ws_bytes, tg_stream stream);
 
+/* ---- launch tracing (optional) --------------------------------------------
+ * Measurement aid with no counterpart on the pages (they report only
+ * end-to-end prefill latency and memory). While tracing is on for a host
+ * thread, every kernel the library launches from that thread is bracketed by
+ * a pair of CUDA events on its stream, and the launch's algorithmic work
+ * (FLOPs of the contraction, or bytes an ideal kernel must move) is noted.
+ * Events are host-side driver objects created on first use; no device
+ * memory is allocated. */
+
+typedef enum {
+  TG_K_COPY = 0,          /* device-to-device copy                          */
+  TG_K_RMSNORM = 1,
+  TG_K_GEMM_STORE = 2,    /* tcgen05 GEMM, plain store epilogue             */
+  TG_K_GEMM_RESIDUAL = 3, /* tcgen05 GEMM, residual-add epilogue            */
+  TG_K_GEMM_SWIGLU = 4,   /* tcgen05 GEMM, SiLU(gate)*up epilogue           */
+  TG_K_GEMM_SCORE = 5,    /* tcgen05 GEMM, scorer-tail epilogue             */
+  TG_K_ROPE_PREP = 6,     /* RoPE + qk-norm + V transpose + gate bias        */
+  TG_K_ATTENTION = 7,     /* tcgen05 gated attention                        */
+  TG_K_SELECT = 8,        /* the radix-select kernels of one top-K           */
+  TG_K_COMPACT = 9,
+  TG_K_GEMM_F32 = 10,     /* SIMT fp32 GEMM                                 */
+  TG_K_ATTENTION_F32 = 11,
+  TG_K_F32_HELPER = 12,   /* fp32 SwiGLU / scorer tail                      */
+  TG_K_COUNT = 13
+} tg_kernel;
+
+typedef struct {
+  int32_t kernel;  /* tg_kernel                                           */
+  int32_t layer;   /* decoder layer of a tg_prefill launch, else -1        */
+  int64_t rows;    /* rows (tokens) the launch processed                    */
+  float ms;        /* device time between the bracketing events             */
+  double flops;    /* algorithmic FLOPs of the launch (0 if memory-bound)   */
+  double bytes;    /* algorithmic bytes of the launch                       */
+} tg_trace_record;
+
+/* Starts tracing on this host thread, for at most `capacity` launches. */
+tg_status tg_trace_start(int32_t capacity);
+/* Stops tracing, waits for the recorded events, and copies up to `cap`
+ * records into `out` (HOST array). Returns the record count, or a negative
+ * tg_status on failure. */
+int32_t tg_trace_stop(tg_trace_record* out, int32_t cap);
+/* Static name of a tg_kernel. */
+const char* tg_kernel_name(int32_t kernel);
+
 /* ---- diagnostics -------------------------------------------------------- */
 
 /* Static description of a status code. */

@@ -4,8 +4,8 @@ Argument marshalling only: every step runs in the library's CUDA kernels.
 PyTorch supplies device memory (tensors, workspaces) and streams. The names
 mirror the C ABI in include/tokengate.h.
 
-The shared library is built in-tree (``python -m
-learned_token_pruning_score_b200._build``); importing this package without
+The shared library is built in-tree (``python
+learned_token_pruning_score_b200/_build.py``); importing this package without
 it raises ImportError -- there is no fallback path.
 """
 
@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libtokengate.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is not built; run `python -m learned_token_pruning_score_b200._build`")
+        f"{LIB_PATH} is not built; run `python learned_token_pruning_score_b200/_build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -62,6 +62,11 @@ class TgKV(ctypes.Structure):
     _fields_ = [("k", _c_p), ("v", _c_p)]
 
 
+class TgTraceRecord(ctypes.Structure):
+    _fields_ = [("kernel", _c_i32), ("layer", _c_i32), ("rows", _c_i64), ("ms", _c_f32),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
 def _sig(name, res, *args):
     f = getattr(_lib, name)
     f.restype = res
@@ -84,6 +89,9 @@ _status_string = _sig("tg_status_string", ctypes.c_char_p, _ci)
 _last_cuda_error = _sig("tg_last_cuda_error", _ci)
 _device_error = _sig("tg_device_error", _ci, ctypes.POINTER(ctypes.c_uint32), _ci)
 _version = _sig("tg_version", ctypes.c_char_p)
+_trace_start = _sig("tg_trace_start", _ci, _c_i32)
+_trace_stop = _sig("tg_trace_stop", _c_i32, ctypes.POINTER(TgTraceRecord), _c_i32)
+_kernel_name = _sig("tg_kernel_name", ctypes.c_char_p, _c_i32)
 
 
 class TokenGateError(RuntimeError):
@@ -152,6 +160,23 @@ def tg_device_error(clear: bool = False) -> int:
     w = ctypes.c_uint32(0)
     _check(_device_error(ctypes.byref(w), int(clear)), "tg_device_error")
     return int(w.value)
+
+
+def tg_trace_start(capacity: int = 65536) -> None:
+    """Bracket every library kernel launched from this thread with CUDA events."""
+    _check(_trace_start(capacity), "tg_trace_start")
+
+
+def tg_trace_stop() -> List[dict]:
+    """Stop tracing; one dict per traced launch: kernel, layer, rows, ms,
+    flops, bytes (algorithmic work of the launch)."""
+    cap = 1 << 20
+    buf = (TgTraceRecord * cap)()
+    n = _trace_stop(buf, cap)
+    if n < 0:
+        raise TokenGateError(-n, "tg_trace_stop")
+    return [dict(kernel=_kernel_name(r.kernel).decode(), layer=r.layer, rows=r.rows, ms=r.ms,
+                 flops=r.flops, bytes=r.bytes) for r in buf[:n]]
 
 
 # ----------------------------------------------------------------- the calls
@@ -283,7 +308,7 @@ def tg_prefill(model: Model, x, protect, k: int, gate_layer: int, out=None, kept
 __all__ = [
     "tg_score", "tg_topk_select", "tg_compact", "tg_gated_attn_prefill", "tg_prefill",
     "tg_workspace_size", "tg_status_string", "tg_device_error", "tg_version", "Model",
-    "TokenGateError", "LIB_PATH", "TG_OK", "TG_ERR_INVALID_ARG", "TG_ERR_UNSUPPORTED",
+    "TokenGateError", "LIB_PATH", "tg_trace_start", "tg_trace_stop", "TG_OK", "TG_ERR_INVALID_ARG", "TG_ERR_UNSUPPORTED",
     "TG_ERR_BUDGET", "TG_ERR_WORKSPACE", "TG_ERR_CUDA", "TG_F32", "TG_BF16", "TG_OP_SCORE",
     "TG_OP_TOPK_SELECT", "TG_OP_COMPACT", "TG_OP_GATED_ATTN", "TG_OP_PREFILL",
 ]

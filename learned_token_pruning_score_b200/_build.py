@@ -1,6 +1,6 @@
 """Builds libtokengate.so in-tree with nvcc for sm_100a.
 
-    python -m learned_token_pruning_score_b200._build
+    python learned_token_pruning_score_b200/_build.py   (or __graft_entry__.build())
 
 Each .cu under csrc/ is compiled to an object under _build/ (in parallel,
 skipped when up to date), then linked into a shared library next to this

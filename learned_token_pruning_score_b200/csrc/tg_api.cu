@@ -18,6 +18,7 @@
 #include <mutex>
 #include <set>
 #include <utility>
+#include <vector>
 
 #include "../../include/tokengate.h"
 #include "tg_internal.h"
@@ -74,6 +75,31 @@ cudaError_t set_smem_attr_once(const void* fn, int bytes) {
 }
 
 namespace {
+
+// ------------------------------------------------------------------ tracing
+struct Tracer {
+  bool on = false;
+  int cap = 0;
+  int layer = -1;
+  std::vector<cudaEvent_t> ev;  // 2 per record
+  std::vector<tg_trace_record> recs;
+};
+thread_local Tracer t_trace;
+
+// Runs `launch` (which enqueues one kernel, or one fixed group of kernels)
+// and, while tracing is on, brackets it with a pair of events.
+template <class F>
+cudaError_t traced(tg_kernel kernel, int64_t rows, double flops, double bytes, cudaStream_t st,
+                   F&& launch) {
+  Tracer& T = t_trace;
+  if (!T.on || static_cast<int>(T.recs.size()) >= T.cap) return launch();
+  const size_t i = T.recs.size();
+  cudaEventRecord(T.ev[2 * i], st);
+  const cudaError_t e = launch();
+  cudaEventRecord(T.ev[2 * i + 1], st);
+  T.recs.push_back(tg_trace_record{static_cast<int32_t>(kernel), T.layer, rows, 0.f, flops, bytes});
+  return e;
+}
 
 tg_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return TG_OK;
@@ -175,11 +201,54 @@ struct PrefillPlan {
 // ------------------------------------------------------------------ pieces
 
 cudaError_t gemm(const GemmArgs& g, tg_dtype dt, cudaStream_t st) {
+  const double e = static_cast<double>(elem_size(dt));
+  const double flops = 2.0 * double(g.M) * g.N * g.K;
+  double out_bytes = 0.0;
+  tg_kernel kid = TG_K_GEMM_F32;
+  switch (g.epi) {
+    case EPI_STORE: out_bytes = double(g.M) * g.N * e; kid = TG_K_GEMM_STORE; break;
+    case EPI_RESIDUAL: out_bytes = 2.0 * double(g.M) * g.N * e; kid = TG_K_GEMM_RESIDUAL; break;
+    case EPI_SWIGLU: out_bytes = double(g.M) * g.inter * e; kid = TG_K_GEMM_SWIGLU; break;
+    case EPI_SCORE: out_bytes = double(g.M) * 4.0; kid = TG_K_GEMM_SCORE; break;
+  }
+  const double bytes = (double(g.M) + g.N) * g.K * e + out_bytes;
   if (dt == TG_BF16) {
     if (!gemm_tc_supported(g)) return cudaErrorInvalidValue;
-    return launch_gemm_tc(g, st);
+    return traced(kid, g.M, flops, bytes, st, [&] { return launch_gemm_tc(g, st); });
   }
-  return launch_gemm_simt_f32(g, st);
+  return traced(TG_K_GEMM_F32, g.M, flops, bytes, st, [&] { return launch_gemm_simt_f32(g, st); });
+}
+
+cudaError_t rmsnorm(const void* x, const float* gamma, float eps, int64_t rows, int d, tg_dtype dt,
+                    void* y, cudaStream_t st) {
+  const double bytes = 2.0 * double(rows) * d * elem_size(dt) + 4.0 * d;
+  return traced(TG_K_RMSNORM, rows, 0.0, bytes, st,
+                [&] { return launch_rmsnorm(x, gamma, eps, rows, d, dt == TG_BF16, y, st); });
+}
+
+cudaError_t copy_rows(void* dst, const void* src, size_t bytes, int64_t rows, cudaStream_t st) {
+  return traced(TG_K_COPY, rows, 0.0, 2.0 * double(bytes), st, [&] {
+    return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st);
+  });
+}
+
+cudaError_t select_topk(const float* scores, const uint8_t* protect, int64_t n, int64_t k,
+                        int32_t* kept, void* ws, cudaStream_t st) {
+  const double bytes = 4.0 * n + (protect ? double(n) : 0.0) + 4.0 * k;
+  return traced(TG_K_SELECT, n, 0.0, bytes, st,
+                [&] { return launch_topk_select(scores, protect, n, k, kept, ws, st); });
+}
+
+cudaError_t compact(const void* x, const int32_t* pos_in, const float* scores, const int32_t* idx,
+                    int64_t n, int64_t k, int row_bytes, void* x_out, int32_t* pos_out,
+                    float* s_out, float* lsig_out, cudaStream_t st) {
+  const double bytes = 2.0 * double(k) * row_bytes + 4.0 * k /*idx*/ + 4.0 * k /*pos*/ +
+                       (scores ? 4.0 * k : 0.0) + (s_out ? 4.0 * k : 0.0) +
+                       (lsig_out ? 4.0 * k : 0.0);
+  return traced(TG_K_COMPACT, k, 0.0, bytes, st, [&] {
+    return launch_compact(x, pos_in, scores, idx, n, k, row_bytes, x_out, pos_out, s_out,
+                          lsig_out, st);
+  });
 }
 
 GemmArgs gemm_args(const void* A, int64_t lda, const void* B, int64_t ldb, void* C, int64_t ldc,
@@ -194,7 +263,7 @@ GemmArgs gemm_args(const void* A, int64_t lda, const void* B, int64_t ldb, void*
 cudaError_t run_score(const void* x, int64_t rows, int d, int f, const float* norm_w, float eps,
                       const void* w1, const float* b1, const float* w2, const float* b2,
                       tg_dtype dt, float* scores, void* y, float* hpre, cudaStream_t st) {
-  cudaError_t e = launch_rmsnorm(x, norm_w, eps, rows, d, dt == TG_BF16, y, st);
+  cudaError_t e = rmsnorm(x, norm_w, eps, rows, d, dt, y, st);
   if (e != cudaSuccess) return e;
   if (dt == TG_BF16) {
     GemmArgs g = gemm_args(y, d, w1, d, nullptr, 0, rows, f, d, EPI_SCORE);
@@ -204,7 +273,9 @@ cudaError_t run_score(const void* x, int64_t rows, int d, int f, const float* no
   GemmArgs g = gemm_args(y, d, w1, d, hpre, f, rows, f, d, EPI_STORE);
   e = gemm(g, dt, st);
   if (e != cudaSuccess) return e;
-  return launch_score_dot_f32(hpre, rows, f, b1, w2, b2, scores, st);
+  return traced(TG_K_F32_HELPER, rows, 0.0, double(rows) * f * 4.0, st, [&] {
+    return launch_score_dot_f32(hpre, rows, f, b1, w2, b2, scores, st);
+  });
 }
 
 // RoPE/qk-norm prep + attention, q/k/v taken from rows with the given strides.
@@ -228,8 +299,15 @@ cudaError_t run_attention(const void* q, int64_t q_stride, const void* kk, int64
   r.kv_v_out = v_out;
   r.s = lsig_ready ? nullptr : s;
   r.lsig_out = plan.lsig;
-  cudaError_t e = launch_rope_prep(r, st);
+  const size_t es = elem_size(dt);
+  const double prep_bytes = double(rows) * (hq + hkv) * dh * es * 2.0 +
+                            (dt == TG_BF16 ? double(rows) * hkv * dh * es * 2.0 : 0.0) +
+                            (v_out ? double(rows) * hkv * dh * es : 0.0) + (r.s ? 8.0 * rows : 0.0);
+  cudaError_t e = traced(TG_K_ROPE_PREP, rows, 0.0, prep_bytes, st,
+                         [&] { return launch_rope_prep(r, st); });
   if (e != cudaSuccess) return e;
+  const double attn_flops = 4.0 * dh * hq * double(rows) * double(rows + 1) / 2.0;
+  const double attn_bytes = double(rows) * (2 * hq + 2 * hkv) * dh * es;
   AttnArgs a{};
   a.q = plan.q_rot;
   a.k = r.k_out;
@@ -241,11 +319,13 @@ cudaError_t run_attention(const void* q, int64_t q_stride, const void* kk, int64
     a.v = plan.vT;
     a.t_pad = plan.t_pad;
     if (!attn_tc_supported(a)) return cudaErrorInvalidValue;
-    return launch_attn_tc(a, st);
+    return traced(TG_K_ATTENTION, rows, attn_flops, attn_bytes, st,
+                  [&] { return launch_attn_tc(a, st); });
   }
   a.v = v;
   a.t_pad = v_stride;
-  return launch_attn_simt_f32(a, st);
+  return traced(TG_K_ATTENTION_F32, rows, attn_flops, attn_bytes, st,
+                [&] { return launch_attn_simt_f32(a, st); });
 }
 
 // ---- the decoder-layer pieces used by tg_prefill
@@ -260,7 +340,7 @@ cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims
                                const tg_kv* kv, cudaStream_t st) {
   const tg_dtype dt = m.dtype;
   const size_t e = elem_size(dt);
-  cudaError_t err = launch_rmsnorm(h, lw.attn_norm, m.norm_eps, rows, D.d, dt == TG_BF16, P.y, st);
+  cudaError_t err = rmsnorm(h, lw.attn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
   if (err != cudaSuccess) return err;
   err = gemm(gemm_args(P.y, D.d, lw.wqkv, D.d, P.qkv, D.qkv, rows, D.qkv, D.d, EPI_STORE), dt, st);
   if (err != cudaSuccess) return err;
@@ -281,7 +361,7 @@ cudaError_t ffn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
                          const PrefillPlan& P, void* h, int64_t rows, cudaStream_t st) {
   if (lw.w_gate_up == nullptr) return cudaSuccess;
   const tg_dtype dt = m.dtype;
-  cudaError_t err = launch_rmsnorm(h, lw.ffn_norm, m.norm_eps, rows, D.d, dt == TG_BF16, P.y, st);
+  cudaError_t err = rmsnorm(h, lw.ffn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
   if (err != cudaSuccess) return err;
   if (dt == TG_BF16) {
     GemmArgs g = gemm_args(P.y, D.d, lw.w_gate_up, D.d, P.mlp, D.inter, rows, 2 * D.inter, D.d,
@@ -292,8 +372,10 @@ cudaError_t ffn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
     err = gemm(gemm_args(P.y, D.d, lw.w_gate_up, D.d, P.gu, 2 * D.inter, rows, 2 * D.inter, D.d,
                          EPI_STORE), dt, st);
     if (err == cudaSuccess)
-      err = launch_swiglu_f32(static_cast<const float*>(P.gu), rows, D.inter,
-                              static_cast<float*>(P.mlp), st);
+      err = traced(TG_K_F32_HELPER, rows, 0.0, double(rows) * D.inter * 12.0, st, [&] {
+        return launch_swiglu_f32(static_cast<const float*>(P.gu), rows, D.inter,
+                                 static_cast<float*>(P.mlp), st);
+      });
   }
   if (err != cudaSuccess) return err;
   GemmArgs g = gemm_args(P.mlp, D.inter, lw.w_down, D.inter, h, D.d, rows, D.d, D.inter,
@@ -392,8 +474,8 @@ tg_status tg_topk_select(const float* scores, const uint8_t* protect, int64_t n,
   TG_CHECK(k >= 1 && k <= n, TG_ERR_BUDGET);
   TG_CHECK(ws != nullptr && ws_bytes >= select_ws_bytes(n), TG_ERR_WORKSPACE);
   TG_CHECK((reinterpret_cast<uintptr_t>(ws) & 15u) == 0, TG_ERR_INVALID_ARG);
-  return cuda_status(launch_topk_select(scores, protect, n, k, kept_idx, ws,
-                                        reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(select_topk(scores, protect, n, k, kept_idx, ws,
+                                 reinterpret_cast<cudaStream_t>(stream)));
 }
 
 tg_status tg_compact(const void* x, const int32_t* pos_in, const float* scores,
@@ -406,9 +488,8 @@ tg_status tg_compact(const void* x, const int32_t* pos_in, const float* scores,
   const int64_t row_bytes = int64_t(d) * int64_t(elem_size(dt));
   TG_CHECK(row_bytes % 16 == 0 && row_bytes < (int64_t(1) << 30), TG_ERR_UNSUPPORTED);
   TG_CHECK(aligned16(x) && aligned16(x_out), TG_ERR_INVALID_ARG);
-  return cuda_status(launch_compact(x, pos_in, scores, kept_idx, n, k, static_cast<int>(row_bytes),
-                                    x_out, pos_out, scores_out, nullptr,
-                                    reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(compact(x, pos_in, scores, kept_idx, n, k, static_cast<int>(row_bytes), x_out,
+                             pos_out, scores_out, nullptr, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 tg_status tg_gated_attn_prefill(const void* q, const void* kk, const void* v, const int32_t* pos,
@@ -452,34 +533,45 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
          (m.n_heads_q + 2 * m.n_heads_kv) * m.head_dim};
   float* sc = scores ? scores : P.scores;
 
-  TG_TRY(cudaMemcpyAsync(P.h, x, size_t(n) * D.d * e, cudaMemcpyDeviceToDevice, st));
+  struct LayerTag {  // annotates traced launches with their decoder layer
+    explicit LayerTag(int l) { t_trace.layer = l; }
+    ~LayerTag() { t_trace.layer = -1; }
+  };
+  TG_TRY(copy_rows(P.h, x, size_t(n) * D.d * e, n, st));
   // Stage 1: layers below the gate, and the gate layer's attention, over n rows.
   for (int l = 0; l < gate_layer; ++l) {
+    LayerTag tag(l);
     TG_TRY(attention_sublayer(m, m.layers[l], D, P, P.h, n, nullptr, nullptr, nullptr, nullptr,
                               kv ? &kv[l] : nullptr, st));
     TG_TRY(ffn_sublayer(m, m.layers[l], D, P, P.h, n, st));
   }
-  if (gate_layer >= 0)
+  if (gate_layer >= 0) {
+    LayerTag tag(gate_layer);
     TG_TRY(attention_sublayer(m, m.layers[gate_layer], D, P, P.h, n, nullptr, nullptr, nullptr,
                               nullptr, kv ? &kv[gate_layer] : nullptr, st));
+  }
   // Stage 2: score the post-attention residual, select, compact.
   TG_TRY(run_score(P.h, n, D.d, m.d_score, m.score_norm, m.norm_eps, m.score_w1, m.score_b1,
                    m.score_w2, m.score_b2, m.dtype, sc, P.y, P.hpre, st));
-  TG_TRY(launch_topk_select(sc, protect, n, k, kept_idx, P.sel_ws, st));
-  TG_TRY(launch_compact(P.h, nullptr, sc, kept_idx, n, k, static_cast<int>(D.d * e), P.hk, P.pos_k,
-                        P.s_k, P.lsig_k, st));
+  TG_TRY(select_topk(sc, protect, n, k, kept_idx, P.sel_ws, st));
+  TG_TRY(compact(P.h, nullptr, sc, kept_idx, n, k, static_cast<int>(D.d * e), P.hk, P.pos_k, P.s_k,
+                 P.lsig_k, st));
   // Stage 3: the gate layer's FFN and the layers above, over the k kept rows.
-  if (gate_layer >= 0) TG_TRY(ffn_sublayer(m, m.layers[gate_layer], D, P, P.hk, k, st));
+  if (gate_layer >= 0) {
+    LayerTag tag(gate_layer);
+    TG_TRY(ffn_sublayer(m, m.layers[gate_layer], D, P, P.hk, k, st));
+  }
   for (int l = gate_layer + 1; l < m.n_layers; ++l) {
+    LayerTag tag(l);
     const tg_layer& L = m.layers[l];
     TG_TRY(attention_sublayer(m, L, D, P, P.hk, k, P.pos_k, P.lsig_k, L.gain, L.tau,
                               kv ? &kv[l] : nullptr, st));
     TG_TRY(ffn_sublayer(m, L, D, P, P.hk, k, st));
   }
   if (m.final_norm)
-    TG_TRY(launch_rmsnorm(P.hk, m.final_norm, m.norm_eps, k, D.d, m.dtype == TG_BF16, out, st));
+    TG_TRY(rmsnorm(P.hk, m.final_norm, m.norm_eps, k, D.d, m.dtype, out, st));
   else
-    TG_TRY(cudaMemcpyAsync(out, P.hk, size_t(k) * D.d * e, cudaMemcpyDeviceToDevice, st));
+    TG_TRY(copy_rows(out, P.hk, size_t(k) * D.d * e, k, st));
   return TG_OK;
 }
 
@@ -510,5 +602,47 @@ tg_status tg_device_error(uint32_t* word, int clear) {
 }
 
 const char* tg_version(void) { return "tokengate-b200 0.1.0 (sm_100a)"; }
+
+tg_status tg_trace_start(int32_t capacity) {
+  TG_CHECK(capacity >= 1 && capacity <= (1 << 20), TG_ERR_INVALID_ARG);
+  Tracer& T = t_trace;
+  while (T.ev.size() < size_t(2) * capacity) {
+    cudaEvent_t ev;
+    TG_TRY(cudaEventCreate(&ev));
+    T.ev.push_back(ev);
+  }
+  T.cap = capacity;
+  T.recs.clear();
+  T.layer = -1;
+  T.on = true;
+  return TG_OK;
+}
+
+int32_t tg_trace_stop(tg_trace_record* out, int32_t cap) {
+  Tracer& T = t_trace;
+  T.on = false;
+  const int n = static_cast<int>(T.recs.size());
+  if (n == 0) return 0;
+  cudaError_t e = cudaEventSynchronize(T.ev[2 * (n - 1) + 1]);
+  if (e != cudaSuccess) return -static_cast<int32_t>(cuda_status(e));
+  int count = 0;
+  for (int i = 0; i < n && i < cap; ++i) {
+    float ms = 0.f;
+    e = cudaEventElapsedTime(&ms, T.ev[2 * i], T.ev[2 * i + 1]);
+    if (e != cudaSuccess) return -static_cast<int32_t>(cuda_status(e));
+    T.recs[i].ms = ms;
+    if (out) out[i] = T.recs[i];
+    ++count;
+  }
+  T.recs.clear();
+  return count;
+}
+
+const char* tg_kernel_name(int32_t kernel) {
+  static const char* names[TG_K_COUNT] = {
+      "copy", "rmsnorm", "gemm_tc_store", "gemm_tc_residual", "gemm_tc_swiglu", "gemm_tc_score",
+      "rope_prep", "attention_tc", "select", "compact", "gemm_f32", "attention_f32", "f32_helper"};
+  return (kernel >= 0 && kernel < TG_K_COUNT) ? names[kernel] : "unknown";
+}
 
 }  // extern "C"
