@@ -113,6 +113,31 @@ tg_status tg_topk_select(const float* scores, const uint8_t* protect, int64_t n,
                          int32_t* kept_idx, void* ws, size_t ws_bytes, tg_stream stream);
 
 /*
+ * tg_topk_select_noalloc -- tg_topk_select without a workspace argument.
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot hand the library scratch device memory: code that only receives
+ * input and output buffers from a host application which keeps the GPU's
+ * memory in its own pool, or a latency-critical loop that must not call
+ * cudaMalloc/cudaFree because those calls can synchronise the device.
+ * The selection is the same as tg_topk_select (same kernels, same result).
+ * Its scratch (about 24 KB) is a static array in device memory that every
+ * GPU loading the library holds until the process exits.
+ *  - n must not exceed TG_SELECT_NOALLOC_MAX_N; larger n returns
+ *    TG_ERR_UNSUPPORTED before any launch (use tg_topk_select instead).
+ *  - The first call on a device looks up the array's device address (one
+ *    runtime call, with that device current); make that first call before
+ *    any stream capture.
+ *  - Every call on a device shares the one array, and each call clears what
+ *    it needs. Calls whose kernels overlap on the GPU (e.g. on two streams)
+ *    race on it: keep them ordered on one stream.
+ *  - If more than k tokens are protected, kept_idx is filled with -1.
+ * The call itself allocates nothing.
+ */
+#define TG_SELECT_NOALLOC_MAX_N 1048576
+tg_status tg_topk_select_noalloc(const float* scores, const uint8_t* protect, int64_t n,
+                                 int64_t k, int32_t* kept_idx, tg_stream stream);
+
+/*
  * tg_compact -- gather of the kept rows.
  *   x_out[r] = x[kept_idx[r]], pos_out[r] = pos_in[kept_idx[r]] (or
  *   kept_idx[r] when pos_in is NULL), scores_out[r] = scores[kept_idx[r]].

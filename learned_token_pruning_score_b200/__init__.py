@@ -79,6 +79,7 @@ _workspace_size = _sig("tg_workspace_size", _c_sz, _ci, ctypes.POINTER(TgShape))
 _score = _sig("tg_score", _ci, _c_p, _c_i64, _c_i32, _c_i32, _c_p, _c_f32, _c_p, _c_p, _c_p, _c_p,
               _ci, _c_p, _c_p, _c_sz, _c_p)
 _topk = _sig("tg_topk_select", _ci, _c_p, _c_p, _c_i64, _c_i64, _c_p, _c_p, _c_sz, _c_p)
+_topk_noalloc = _sig("tg_topk_select_noalloc", _ci, _c_p, _c_p, _c_i64, _c_i64, _c_p, _c_p)
 _compact = _sig("tg_compact", _ci, _c_p, _c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i32, _ci, _c_p,
                 _c_p, _c_p, _c_p)
 _attn = _sig("tg_gated_attn_prefill", _ci, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i64,
@@ -207,6 +208,25 @@ def tg_topk_select(scores, protect, k: int, kept_idx=None, ws=None, stream=None)
     return kept_idx
 
 
+SELECT_NOALLOC_MAX_N = 1 << 20
+
+
+def tg_topk_select_noalloc(scores, protect, k: int, kept_idx=None, stream=None) -> torch.Tensor:
+    """tg_topk_select with no workspace: the library keeps this call's scratch
+    in a static device array (n <= SELECT_NOALLOC_MAX_N). For callers that can
+    pass only inputs and outputs. Calls that overlap on the GPU share that
+    array and race; the first call on a device should precede stream capture."""
+    n = scores.shape[0]
+    if n > SELECT_NOALLOC_MAX_N:
+        raise ValueError(f"n={n} exceeds the allocation-free limit {SELECT_NOALLOC_MAX_N}; "
+                         "use tg_topk_select with a workspace")
+    if kept_idx is None:
+        kept_idx = torch.empty(k, dtype=torch.int32, device=scores.device)
+    _check(_topk_noalloc(_ptr(scores), _ptr(protect), n, k, _ptr(kept_idx),
+                         _stream(stream, scores.device)), "tg_topk_select_noalloc")
+    return kept_idx
+
+
 def tg_compact(x, kept_idx, pos_in=None, scores=None, x_out=None, pos_out=None, scores_out=None,
                stream=None):
     n, d = x.shape
@@ -306,7 +326,7 @@ def tg_prefill(model: Model, x, protect, k: int, gate_layer: int, out=None, kept
 
 
 __all__ = [
-    "tg_score", "tg_topk_select", "tg_compact", "tg_gated_attn_prefill", "tg_prefill",
+    "tg_score", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_prefill",
     "tg_workspace_size", "tg_status_string", "tg_device_error", "tg_version", "Model",
     "TokenGateError", "LIB_PATH", "tg_trace_start", "tg_trace_stop", "TG_OK", "TG_ERR_INVALID_ARG", "TG_ERR_UNSUPPORTED",
     "TG_ERR_BUDGET", "TG_ERR_WORKSPACE", "TG_ERR_CUDA", "TG_F32", "TG_BF16", "TG_OP_SCORE",

@@ -16,6 +16,8 @@
 // at the threshold key, then write the kept indices in index order: the tied
 // tokens taken are the lowest-index ones. Integer atomics only, so the
 // result is bit-reproducible.
+#include <mutex>
+
 #include "tg_device.cuh"
 #include "tg_internal.h"
 
@@ -373,7 +375,42 @@ cudaError_t run_select(const float* scores, const uint8_t* protect, int64_t n, i
   return cudaGetLastError();
 }
 
+// Scratch of the allocation-free variant: one array per device, sized for
+// the largest n it accepts, shared by every call on that device.
+constexpr int64_t kNoAllocMaxN = int64_t(1) << 20;
+constexpr size_t kNoAllocBytes = kOffCounts + size_t(kNoAllocMaxN / kChunk) * 2 * 4;
+static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[64] = {};
+
 }  // namespace
+
+int64_t select_noalloc_max_n() { return kNoAllocMaxN; }
+
+// Host code cannot use g_select_scratch's name as a device address: the
+// symbol's device address is looked up once per device (with that device
+// current) and cached; kernels then get that pointer.
+cudaError_t launch_topk_select_noalloc(const float* scores, const uint8_t* protect, int64_t n,
+                                       int64_t k, int32_t* kept_idx, cudaStream_t st) {
+  if (n > kNoAllocMaxN) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_select_scratch);
+      if (e != cudaSuccess) return e;
+      g_scratch_ptr[dev] = p;
+    }
+    scratch = g_scratch_ptr[dev];
+  }
+  return launch_topk_select(scores, protect, n, k, kept_idx, scratch, st);
+}
 
 size_t select_ws_bytes(int64_t n) {
   const int64_t chunks = (n + kChunk - 1) / kChunk;

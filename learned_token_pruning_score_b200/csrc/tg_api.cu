@@ -478,6 +478,18 @@ tg_status tg_topk_select(const float* scores, const uint8_t* protect, int64_t n,
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+tg_status tg_topk_select_noalloc(const float* scores, const uint8_t* protect, int64_t n,
+                                 int64_t k, int32_t* kept_idx, tg_stream stream) {
+  TG_CHECK(scores && kept_idx && n >= 1, TG_ERR_INVALID_ARG);
+  TG_CHECK(n <= select_noalloc_max_n(), TG_ERR_UNSUPPORTED);
+  TG_CHECK(k >= 1 && k <= n, TG_ERR_BUDGET);
+  const double bytes = 4.0 * n + (protect ? double(n) : 0.0) + 4.0 * k;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return cuda_status(traced(TG_K_SELECT, n, 0.0, bytes, st, [&] {
+    return launch_topk_select_noalloc(scores, protect, n, k, kept_idx, st);
+  }));
+}
+
 tg_status tg_compact(const void* x, const int32_t* pos_in, const float* scores,
                      const int32_t* kept_idx, int64_t n, int64_t k, int32_t d, tg_dtype dt,
                      void* x_out, int32_t* pos_out, float* scores_out, tg_stream stream) {

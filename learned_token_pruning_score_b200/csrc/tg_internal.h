@@ -36,6 +36,10 @@ unsigned int* device_error_word();  // device address of the sticky error word
 size_t select_ws_bytes(int64_t n);
 cudaError_t launch_topk_select(const float* scores, const uint8_t* protect, int64_t n, int64_t k,
                                int32_t* kept_idx, void* ws, cudaStream_t st);
+// Same selection with its scratch in a static device array (no workspace).
+int64_t select_noalloc_max_n();
+cudaError_t launch_topk_select_noalloc(const float* scores, const uint8_t* protect, int64_t n,
+                                       int64_t k, int32_t* kept_idx, cudaStream_t st);
 
 // ---- compaction (k_compact.cu). Optional lsig_out[r] = logsigmoid(scores[idx[r]]).
 cudaError_t launch_compact(const void* x, const int32_t* pos_in, const float* scores,
