@@ -284,6 +284,306 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 2) tmem_dealloc(tmem, 512);
 }
 
+
+// ============================================================================
+// Paired-head design: one CTA per (128-row query tile, pair of query heads
+// sharing one KV head). The K/V tiles are loaded once for both heads.
+//   warp 0      TMA: both Q tiles once; K and V^T tiles in 2-deep rings.
+//   warp 1      MMA (one thread), per KV tile j:
+//                 O_A += P_A V_j  (P_A read from TMEM), S_A = Q_A K_{j+1}^T,
+//                 O_B += P_B V_j,                      S_B = Q_B K_{j+1}^T
+//               so while one softmax warpgroup works, the tensor pipe serves
+//               the other head (ping-pong).
+//   warps 4-7   softmax of head A, warps 8-11 softmax of head B; one thread
+//               per query row. S is read from TMEM, the per-key gate bias
+//               (pre-scaled by the head's gain) comes from a shared-memory
+//               ring staged by the same warpgroup, P is written back to TMEM
+//               as packed bf16 over the first half of S's columns.
+// TMEM columns: S_A [0,128) (P_A [0,64)), S_B [128,256) (P_B [128,192)),
+//               O_A [256,384), O_B [384,512).
+// Ordering: the commit that signals S_h(j+1) is issued after O_h += P_h(j) V_j,
+// so when a softmax thread sees S_h(j+1) the previous P.V of its head has
+// finished: O_h may be rescaled and P_h overwritten without another wait.
+// ============================================================================
+namespace pair {
+
+constexpr int kThreads = 384;
+constexpr int kOffQA = 0;
+constexpr int kOffQB = kOffQA + kTile;
+constexpr int kOffK = kOffQB + kTile;        // 2 stages
+constexpr int kOffV = kOffK + 2 * kTile;     // 2 stages
+constexpr int kOffBias = kOffV + 2 * kTile;  // [2 heads][2 slots][128] fp32
+constexpr int kOffBar = kOffBias + 2 * 2 * 128 * 4;
+constexpr size_t kSmem = 1024 + kOffBar + 256;
+
+struct Params {
+  int64_t T;
+  int hq, hkv;
+  int n_qtiles;
+  const float* lsig;
+  const float* gain;
+  const float* tau;
+  __nv_bfloat16* out;
+  unsigned int* err;
+};
+
+template <bool kBias>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* k_empty = bars + 3;   // [2]
+  uint64_t* v_full = bars + 5;    // [2]
+  uint64_t* v_empty = bars + 7;   // [2]
+  uint64_t* s_full = bars + 9;    // [2 heads]
+  uint64_t* p_full = bars + 11;   // [2 heads]
+  uint64_t* o_full = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // KV-head-major order (the CTAs running together share one KV head's K/V
+  // in L2), heavy (late) query tiles first within a KV head.
+  const int pairs_per_kv = (p.hq / p.hkv) / 2;
+  const int per_kv = p.n_qtiles * pairs_per_kv;
+  const int g = static_cast<int>(blockIdx.x) / per_kv;
+  const int rem = static_cast<int>(blockIdx.x) % per_kv;
+  const int qt = p.n_qtiles - 1 - rem / pairs_per_kv;
+  const int head0 = g * (p.hq / p.hkv) + 2 * (rem % pairs_per_kv);
+  const int q0 = qt * kBlk;
+  const int n_kv = qt + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+    }
+    mbar_init(o_full, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 2) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------- TMA producer
+    mbar_arrive_expect_tx(q_full, 2 * kTile);
+    tma_load_3d(&tmQ, q_full, smem + kOffQA, 0, head0, q0);
+    tma_load_3d(&tmQ, q_full, smem + kOffQA + kSub, 64, head0, q0);
+    tma_load_3d(&tmQ, q_full, smem + kOffQB, 0, head0 + 1, q0);
+    tma_load_3d(&tmQ, q_full, smem + kOffQB + kSub, 64, head0 + 1, q0);
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j & 1;
+      const uint32_t ph = ((j >> 1) & 1) ^ 1;
+      if (!mbar_wait(&k_empty[s], ph, p.err)) break;
+      uint8_t* kd = smem + kOffK + s * kTile;
+      mbar_arrive_expect_tx(&k_full[s], kTile);
+      tma_load_3d(&tmK, &k_full[s], kd, 0, g, j * kBlk);
+      tma_load_3d(&tmK, &k_full[s], kd + kSub, 64, g, j * kBlk);
+      if (!mbar_wait(&v_empty[s], ph, p.err)) break;
+      uint8_t* vd = smem + kOffV + s * kTile;
+      mbar_arrive_expect_tx(&v_full[s], kTile);
+      tma_load_3d(&tmV, &v_full[s], vd, j * kBlk, 0, g);
+      tma_load_3d(&tmV, &v_full[s], vd + kSub, j * kBlk + 64, 0, g);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+    auto issue_qk = [&](int h, int j) {
+      const uint32_t q_addr = smem_addr(smem + (h ? kOffQB : kOffQA));
+      const uint32_t k_addr = smem_addr(smem + kOffK + (j & 1) * kTile);
+      const uint32_t d = tmem + static_cast<uint32_t>(h * 128);
+#pragma unroll
+      for (int kk = 0; kk < kDh / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
+        umma_f16_ss(d, sdesc_kmajor_sw128(q_addr + off), sdesc_kmajor_sw128(k_addr + off), idesc,
+                    kk > 0 ? 1u : 0u);
+      }
+      umma_commit(&s_full[h]);
+    };
+    auto issue_pv = [&](int h, int j) {
+      const uint32_t v_addr = smem_addr(smem + kOffV + (j & 1) * kTile);
+      const uint32_t a = tmem + static_cast<uint32_t>(h * 128);        // P_h
+      const uint32_t d = tmem + 256u + static_cast<uint32_t>(h * 128);  // O_h
+#pragma unroll
+      for (int kk = 0; kk < kBlk / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
+        umma_f16_ts(d, a + static_cast<uint32_t>(kk * 8), sdesc_kmajor_sw128(v_addr + off), idesc,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+      }
+    };
+    bool ok = mbar_wait(q_full, 0, p.err) && mbar_wait(&k_full[0], 0, p.err);
+    if (ok) {
+      tc_fence_after();
+      issue_qk(0, 0);
+      issue_qk(1, 0);
+      umma_commit(&k_empty[0]);
+    }
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int s = j & 1;
+      const uint32_t ph = (j >> 1) & 1;
+      const bool more = j + 1 < n_kv;
+      if (!mbar_wait(&v_full[s], ph, p.err)) break;
+      if (!mbar_wait(&p_full[0], j & 1, p.err)) break;
+      tc_fence_after();
+      issue_pv(0, j);
+      if (more) {
+        if (!mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, p.err)) break;
+        tc_fence_after();
+        issue_qk(0, j + 1);
+      }
+      if (!mbar_wait(&p_full[1], j & 1, p.err)) break;
+      tc_fence_after();
+      issue_pv(1, j);
+      umma_commit(&v_empty[s]);
+      if (more) {
+        issue_qk(1, j + 1);
+        umma_commit(&k_empty[(j + 1) & 1]);
+      }
+    }
+    if (ok) umma_commit(o_full);
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------- softmax
+    const int h = (warp - 4) >> 2;  // 0: head A (warps 4-7), 1: head B (warps 8-11)
+    const int head = head0 + h;
+    const int r = (threadIdx.x - 128) & 127;  // row within the tile = TMEM lane
+    const int64_t q_row = static_cast<int64_t>(q0) + r;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_col = static_cast<uint32_t>(h * 128);
+    const uint32_t o_col = 256u + static_cast<uint32_t>(h * 128);
+    const float tau = p.tau ? __ldg(p.tau + head) : 1.0f;
+    const float scale2 = kLog2e / (sqrtf(static_cast<float>(kDh)) * tau);
+    // bias in units of S: l2 = (S + cmul * lsig) * scale2
+    const float cmul = kBias ? __ldg(p.gain + head) * sqrtf(static_cast<float>(kDh)) * tau : 0.f;
+    float* bias_ring = reinterpret_cast<float*>(smem + kOffBias) + h * 256;
+    float bnext = 0.f;
+    if (kBias) bnext = r < p.T ? __ldg(p.lsig + r) : 0.f;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    // Every thread runs all n_kv iterations: the bias staging's named barrier
+    // has no timeout, so after a failed (timed-out) wait a warp keeps joining
+    // it and skips everything else.
+    for (int j = 0; j < n_kv; ++j) {
+      const int kv0 = j * kBlk;
+      const float4* cb = reinterpret_cast<const float4*>(bias_ring + (j & 1) * 128);
+      if (kBias) {
+        bias_ring[(j & 1) * 128 + r] = cmul * bnext;
+        const int64_t nc = static_cast<int64_t>(kv0) + kBlk + r;
+        bnext = (j + 1 < n_kv && nc < p.T) ? __ldg(p.lsig + nc) : 0.f;
+        named_bar_sync(1 + h, 128);
+      }
+      if (!ok) continue;
+      if (!mbar_wait_warp(&s_full[h], j & 1, p.err)) { ok = false; continue; }
+      tc_fence_after();
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float t[32];
+        tmem_ld32_wait(tmem + lane_off + s_col + static_cast<uint32_t>(c * 32), t);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[c * 32 + i] = t[i];
+      }
+      if (kBias) {
+#pragma unroll
+        for (int i4 = 0; i4 < 32; ++i4) {
+          const float4 b = cb[i4];
+          x[4 * i4 + 0] += b.x;
+          x[4 * i4 + 1] += b.y;
+          x[4 * i4 + 2] += b.z;
+          x[4 * i4 + 3] += b.w;
+        }
+      }
+      if (j == n_kv - 1) {  // diagonal tile: causal mask
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (kv0 + i > q_row) x[i] = -INFINITY;
+      }
+      float rmax = x[0];
+#pragma unroll
+      for (int i = 1; i < 128; ++i) rmax = fmaxf(rmax, x[i]);
+      const float mx = rmax * scale2;
+      float alpha = 1.0f;
+      if (mx > m + kRescaleThresh || m == -INFINITY) {
+        alpha = ex2(m - mx);  // 0 on the first tile
+        l *= alpha;
+        m = mx;
+      }
+      const bool rescale_o = j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f);
+      float rsum = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float a0 = ex2(fmaf(x[64 * half + 2 * i], scale2, -m));
+          const float a1 = ex2(fmaf(x[64 * half + 2 * i + 1], scale2, -m));
+          rsum += a0 + a1;
+          pk[i] = pack_bf16x2(a0, a1);
+        }
+        tmem_st32(tmem + lane_off + s_col + static_cast<uint32_t>(32 * half), pk);
+        tmem_wait_st();
+      }
+      l += rsum;
+      if (rescale_o) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          const uint32_t ta = tmem + lane_off + o_col + static_cast<uint32_t>(c * 32);
+          tmem_ld32_wait(ta, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32_wait(ta, o);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&p_full[h]);
+    }
+    if (ok && mbar_wait_warp(o_full, 0, p.err)) {
+      tc_fence_after();
+      const float inv = 1.0f / l;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        tmem_ld32_wait(tmem + lane_off + o_col + static_cast<uint32_t>(c * 32), o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] *= inv;
+        if (q_row < p.T) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (q_row * p.hq + head) * kDh + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 u;
+            u.x = pack_bf16x2(o[8 * v + 0], o[8 * v + 1]);
+            u.y = pack_bf16x2(o[8 * v + 2], o[8 * v + 3]);
+            u.z = pack_bf16x2(o[8 * v + 4], o[8 * v + 5]);
+            u.w = pack_bf16x2(o[8 * v + 6], o[8 * v + 7]);
+            dst[v] = u;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace pair
+
 }  // namespace
 
 bool attn_tc_supported(const AttnArgs& a) {
@@ -312,6 +612,26 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   p.tau = a.tau;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.err = device_error_word();
+  if ((a.hq / a.hkv) % 2 == 0) {
+    // paired-head kernel (the two query heads of a pair share a KV head)
+    pair::Params pp;
+    pp.T = p.T;
+    pp.hq = p.hq;
+    pp.hkv = p.hkv;
+    pp.n_qtiles = p.n_qtiles;
+    pp.lsig = p.lsig;
+    pp.gain = p.gain;
+    pp.tau = p.tau;
+    pp.out = p.out;
+    pp.err = p.err;
+    const bool bias = a.lsig != nullptr && a.gain != nullptr;
+    auto kern = bias ? pair::attn_tc_pair<true> : pair::attn_tc_pair<false>;
+    cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(kern), int(pair::kSmem));
+    if (err != cudaSuccess) return err;
+    const unsigned grid = static_cast<unsigned>(p.n_qtiles) * static_cast<unsigned>(a.hq / 2);
+    kern<<<grid, pair::kThreads, pair::kSmem, st>>>(tq, tk, tv, pp);
+    return cudaGetLastError();
+  }
   cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(attn_tc), int(kSmem));
   if (err != cudaSuccess) return err;
   const unsigned grid = static_cast<unsigned>(p.n_qtiles) * static_cast<unsigned>(a.hq);
