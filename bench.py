@@ -141,6 +141,16 @@ def build_model(tg, torch, w, device):
                     score=score, final_norm=p["final_norm"], eps=w.eps, rope_base=w.rope_base)
 
 
+def kv_buffers(torch, w, k, device):
+    """Per-layer KV-cache outputs: n rows at/below the gate, k rows above."""
+    out = []
+    for li in range(w.n_layers):
+        rows = w.n if li <= w.gate_layer else k
+        out.append((torch.empty(rows, w.hkv, w.dh, dtype=torch.bfloat16, device=device),
+                    torch.empty(rows, w.hkv, w.dh, dtype=torch.bfloat16, device=device)))
+    return out
+
+
 def dense_model(tg, model):
     layers = [{k: v for k, v in lw.items() if k not in ("gain", "tau")} for lw in model.layers]
     return tg.Model(n_heads_q=model.n_heads_q, n_heads_kv=model.n_heads_kv,
@@ -263,13 +273,14 @@ def run_ours(args, rank, world, local_rank):
     kept = torch.empty(k, dtype=torch.int32, device=device)
     scores = torch.empty(w.n, dtype=torch.float32, device=device)
     ws = torch.empty(model.workspace_size(w.n, k, w.gate_layer), dtype=torch.uint8, device=device)
+    kv = None if args.no_kv else kv_buffers(torch, w, k, device)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
     stream = torch.cuda.current_stream(device)
     tg.tg_device_error(clear=True)
 
     def step():
         tg.tg_prefill(model, x, prot, k, w.gate_layer, out=out, kept_idx=kept, scores=scores,
-                      ws=ws, stream=stream)
+                      kv=kv, ws=ws, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -376,7 +387,7 @@ def run_ours(args, rank, world, local_rank):
             x_dev.copy_(x_host, non_blocking=True)
             prot_dev.copy_(prot_host, non_blocking=True)
             tg.tg_prefill(model, x_dev, prot_dev, k, w.gate_layer, out=out, kept_idx=kept,
-                          scores=scores, ws=ws, stream=stream)
+                          scores=scores, kv=kv, ws=ws, stream=stream)
             out_host.copy_(out, non_blocking=True)
             kept_host.copy_(kept, non_blocking=True)
 
@@ -406,28 +417,32 @@ def run_ours(args, rank, world, local_rank):
     extras = {}
     if not args.quick:
         def ttft(mdl, kk, reps=3):
-            o = torch.empty(kk, w.d, dtype=torch.bfloat16, device=device)
-            ki = torch.empty(kk, dtype=torch.int32, device=device)
-            wsz = torch.empty(mdl.workspace_size(w.n, kk, w.gate_layer), dtype=torch.uint8,
-                              device=device)
-            tg.tg_prefill(mdl, x, prot, kk, w.gate_layer, out=o, kept_idx=ki, ws=wsz)
+            # peak memory of one prefill: weights + input + outputs (incl. KV
+            # cache) + workspace, all allocated by the caller
             torch.cuda.synchronize()
             torch.cuda.reset_peak_memory_stats(device)
+            o = torch.empty(kk, w.d, dtype=torch.bfloat16, device=device)
+            ki = torch.empty(kk, dtype=torch.int32, device=device)
+            kvb = None if args.no_kv else kv_buffers(torch, w, kk, device)
+            wsz = torch.empty(mdl.workspace_size(w.n, kk, w.gate_layer), dtype=torch.uint8,
+                              device=device)
+            tg.tg_prefill(mdl, x, prot, kk, w.gate_layer, out=o, kept_idx=ki, kv=kvb, ws=wsz)
+            torch.cuda.synchronize()
             ms = []
             for _ in range(reps):
                 flush.zero_()
                 a = torch.cuda.Event(enable_timing=True)
                 b = torch.cuda.Event(enable_timing=True)
                 a.record(stream)
-                tg.tg_prefill(mdl, x, prot, kk, w.gate_layer, out=o, kept_idx=ki, ws=wsz)
+                tg.tg_prefill(mdl, x, prot, kk, w.gate_layer, out=o, kept_idx=ki, kv=kvb, ws=wsz)
                 b.record(stream)
                 torch.cuda.synchronize()
                 ms.append(a.elapsed_time(b))
             mem = torch.cuda.max_memory_allocated(device)
-            del o, ki, wsz
+            del o, ki, wsz, kvb
             return statistics.median(ms), mem
 
-        del ws
+        del ws, kv
         torch.cuda.empty_cache()
         for kk in synth.PREFILL_32K_BUDGETS:
             t_ms, mem = ttft(model, kk)
@@ -460,6 +475,7 @@ def run_ours(args, rank, world, local_rank):
                        "gate_layer": w.gate_layer, "d_model": w.d,
                        "heads": f"{w.hq}/{w.hkv}x{w.dh}", "ffn": w.inter, "scorer": w.f,
                        "protected": w.n_protect, "qk_norm": w.qk_norm,
+                       "kv_cache_out": not args.no_kv,
                        "parallelism": f"replicas x{world}",
                        "l2": "flushed between timed steps (256 MB write); inputs > L2"},
             "ttft_ms": ms_per_step,
@@ -587,6 +603,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--budget", type=int, default=HEADLINE_K)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-kv", action="store_true", help="do not write the KV cache outputs")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the other budgets / dense run")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

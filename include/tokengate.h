@@ -254,7 +254,9 @@ typedef enum {
   TG_K_GEMM_F32 = 10,     /* SIMT fp32 GEMM                                 */
   TG_K_ATTENTION_F32 = 11,
   TG_K_F32_HELPER = 12,   /* fp32 SwiGLU / scorer tail                      */
-  TG_K_COUNT = 13
+  TG_K_GEMM_QKV = 13,     /* tcgen05 GEMM, fused qk-norm + RoPE + V^T epilogue */
+  TG_K_ROPE_TABLE = 14,   /* cos/sin table of one set of positions           */
+  TG_K_COUNT = 15
 } tg_kernel;
 
 typedef struct {

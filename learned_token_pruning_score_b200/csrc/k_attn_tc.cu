@@ -320,6 +320,7 @@ struct Params {
   int64_t T;
   int hq, hkv;
   int n_qtiles;
+  int kv_major;  // 1: CTAs ordered KV-head-major (large T), 0: heaviest tiles first
   const float* lsig;
   const float* gain;
   const float* tau;
@@ -346,14 +347,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // KV-head-major order (the CTAs running together share one KV head's K/V
-  // in L2), heavy (late) query tiles first within a KV head.
+  // CTA order. When all K/V fits in L2 easily, the heaviest (latest) query
+  // tiles of every head go first (longest-first list scheduling). Otherwise
+  // KV-head-major, so that the CTAs running together share one KV head's
+  // K/V in L2, heaviest first within each KV head.
   const int pairs_per_kv = (p.hq / p.hkv) / 2;
-  const int per_kv = p.n_qtiles * pairs_per_kv;
-  const int g = static_cast<int>(blockIdx.x) / per_kv;
-  const int rem = static_cast<int>(blockIdx.x) % per_kv;
-  const int qt = p.n_qtiles - 1 - rem / pairs_per_kv;
-  const int head0 = g * (p.hq / p.hkv) + 2 * (rem % pairs_per_kv);
+  const int n_pairs = p.hq / 2;
+  int qt, head0;
+  if (p.kv_major) {
+    const int per_kv = p.n_qtiles * pairs_per_kv;
+    const int g0 = static_cast<int>(blockIdx.x) / per_kv;
+    const int rem = static_cast<int>(blockIdx.x) % per_kv;
+    qt = p.n_qtiles - 1 - rem / pairs_per_kv;
+    head0 = g0 * (p.hq / p.hkv) + 2 * (rem % pairs_per_kv);
+  } else {
+    qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x) / n_pairs;
+    head0 = 2 * (static_cast<int>(blockIdx.x) % n_pairs);
+  }
+  const int g = head0 / (p.hq / p.hkv);
   const int q0 = qt * kBlk;
   const int n_kv = qt + 1;
 
@@ -600,7 +611,9 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
     return cudaErrorInvalidValue;
   if (!make_tmap_3d_bf16(&tk, a.k, kDh, a.hkv, a.T, kDh * e, int64_t(a.hkv) * kDh * e, 1, kBlk))
     return cudaErrorInvalidValue;
-  if (!make_tmap_3d_bf16(&tv, a.v, a.t_pad, kDh, a.hkv, a.t_pad * e, a.t_pad * kDh * e, kDh, 1))
+  // V^T: the inner extent is T (not the padded row length), so key columns
+  // past T read as zeros whatever the padding holds.
+  if (!make_tmap_3d_bf16(&tv, a.v, a.T, kDh, a.hkv, a.t_pad * e, a.t_pad * kDh * e, kDh, 1))
     return cudaErrorInvalidValue;
   Params p;
   p.T = a.T;
@@ -619,6 +632,9 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
     pp.hq = p.hq;
     pp.hkv = p.hkv;
     pp.n_qtiles = p.n_qtiles;
+    // K and V of all KV heads: above ~48 MB the working set would not stay
+    // in the 126 MB L2 across a wave of CTAs spread over every head.
+    pp.kv_major = (double(a.T) * a.hkv * kDh * 4.0 > 48.0e6) ? 1 : 0;
     pp.lsig = p.lsig;
     pp.gain = p.gain;
     pp.tau = p.tau;

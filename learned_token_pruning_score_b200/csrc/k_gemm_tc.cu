@@ -50,7 +50,22 @@ struct EpiParams {
   float* scores;
   int tiles_m, tiles_n;
   unsigned int* err;
+  // EPI_QKV
+  int hq, hkv;
+  const float2* rope_cs;
+  const float* q_norm;
+  const float* k_norm;
+  float eps;
+  __nv_bfloat16* q_out;
+  __nv_bfloat16* k_out;
+  __nv_bfloat16* vT_out;
+  int64_t t_pad;
+  __nv_bfloat16* v_out;
 };
+
+__device__ __forceinline__ float round_bf16_f(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
 
 __device__ __forceinline__ void store32_bf16(__nv_bfloat16* dst, const float (&v)[32]) {
   uint4* d = reinterpret_cast<uint4*>(dst);
@@ -204,6 +219,74 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (row_ok)
             store32_bf16(static_cast<__nv_bfloat16*>(p.C) + row * p.ldc + nb * 128 + c * 32, g);
         }
+      } else if constexpr (kEpi == EPI_QKV) {
+        // Two whole heads per tile (head dim 128). The accumulator is rounded
+        // to bf16 first (the stored-q/k/v value), then q/k get the optional
+        // per-head RMSNorm and RoPE; v is written transposed (and as cache).
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          const int hg = nb * 2 + hh;  // head index across the q | k | v columns
+          const uint32_t t_head = t_row + static_cast<uint32_t>(hh * 128);
+          if (hg < p.hq + p.hkv) {
+            const bool is_q = hg < p.hq;
+            const float* nw = is_q ? p.q_norm : p.k_norm;
+            float rstd = 1.0f;
+            if (nw != nullptr) {
+              float ss = 0.f;
+#pragma unroll 1
+              for (int c = 0; c < 4; ++c) {
+                float v[32];
+                tmem_ld32_wait(t_head + c * 32, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  const float f = round_bf16_f(v[i]);
+                  ss = fmaf(f, f, ss);
+                }
+              }
+              rstd = rsqrtf(ss * (1.0f / 128.0f) + p.eps);
+            }
+            __nv_bfloat16* dst =
+                is_q ? p.q_out + (row * p.hq + hg) * 128
+                     : p.k_out + (row * p.hkv + (hg - p.hq)) * 128;
+            const float2* cs = p.rope_cs + row * 64;
+#pragma unroll 1
+            for (int c = 0; c < 2; ++c) {
+              float lo[32], hi[32];
+              tmem_ld32_wait(t_head + c * 32, lo);
+              tmem_ld32_wait(t_head + 64 + c * 32, hi);
+              if (row_ok) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  const int pi = c * 32 + i;
+                  float a = round_bf16_f(lo[i]) * rstd;
+                  float b = round_bf16_f(hi[i]) * rstd;
+                  if (nw != nullptr) {
+                    a *= __ldg(nw + pi);
+                    b *= __ldg(nw + pi + 64);
+                  }
+                  const float2 t = __ldg(cs + pi);
+                  lo[i] = a * t.x - b * t.y;
+                  hi[i] = b * t.x + a * t.y;
+                }
+                store32_bf16(dst + c * 32, lo);
+                store32_bf16(dst + 64 + c * 32, hi);
+              }
+            }
+          } else {
+            const int g = hg - p.hq - p.hkv;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              float v[32];
+              tmem_ld32_wait(t_head + c * 32, v);
+              if (row_ok) {
+                if (p.v_out) store32_bf16(p.v_out + (row * p.hkv + g) * 128 + c * 32, v);
+                __nv_bfloat16* vt = p.vT_out + (static_cast<int64_t>(g) * 128 + c * 32) * p.t_pad + row;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) vt[static_cast<int64_t>(i) * p.t_pad] = __float2bfloat16_rn(v[i]);
+              }
+            }
+          }
+        }
       } else {  // EPI_SCORE
         float acc = 0.f;
 #pragma unroll 1
@@ -252,6 +335,17 @@ cudaError_t run(const GemmArgs& g, cudaStream_t st) {
   p.w2 = g.w2;
   p.b2 = g.b2;
   p.scores = g.scores;
+  p.hq = g.hq;
+  p.hkv = g.hkv;
+  p.rope_cs = g.rope_cs;
+  p.q_norm = g.q_norm;
+  p.k_norm = g.k_norm;
+  p.eps = g.eps;
+  p.q_out = static_cast<__nv_bfloat16*>(g.q_out);
+  p.k_out = static_cast<__nv_bfloat16*>(g.k_out);
+  p.vT_out = static_cast<__nv_bfloat16*>(g.vT_out);
+  p.t_pad = g.t_pad;
+  p.v_out = static_cast<__nv_bfloat16*>(g.v_out);
   p.tiles_m = static_cast<int>((g.M + kBM - 1) / kBM);
   p.tiles_n = kEpi == EPI_SWIGLU ? g.inter / 128 : (g.N + kBN - 1) / kBN;
   p.err = device_error_word();
@@ -280,6 +374,10 @@ bool gemm_tc_supported(const GemmArgs& g) {
       return g.inter % 128 == 0 && g.N == 2 * g.inter && al16(g.C) && g.ldc % 8 == 0;
     case EPI_SCORE:
       return g.N >= 1 && g.N <= 256 && g.scores != nullptr && g.w2 != nullptr;
+    case EPI_QKV:
+      return g.hq > 0 && g.hkv > 0 && g.hq % 2 == 0 && g.N == (g.hq + 2 * g.hkv) * 128 &&
+             g.rope_cs != nullptr && al16(g.q_out) && al16(g.k_out) && g.vT_out != nullptr &&
+             g.t_pad >= g.M && (g.v_out == nullptr || al16(g.v_out));
   }
   return false;
 }
@@ -291,6 +389,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, cudaStream_t st) {
     case EPI_RESIDUAL: return run<256, EPI_RESIDUAL>(g, st);
     case EPI_SWIGLU: return run<256, EPI_SWIGLU>(g, st);
     case EPI_SCORE: return run<256, EPI_SCORE>(g, st);
+    case EPI_QKV: return run<256, EPI_QKV>(g, st);
   }
   return cudaErrorInvalidValue;
 }

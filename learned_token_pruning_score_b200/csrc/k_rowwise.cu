@@ -92,6 +92,52 @@ __global__ void __launch_bounds__(256) rmsnorm_rows(const T* __restrict__ x,
   }
 }
 
+// bf16 rows of width kVPL * 256: one warp per row, the row held in registers
+// (kVPL 16-byte vectors per lane), so it is read from HBM once and all loads
+// of a lane are independent.
+template <int kVPL>
+__global__ void __launch_bounds__(256) rmsnorm_rows_bf16_reg(const __nv_bfloat16* __restrict__ x,
+                                                            const float* __restrict__ g, float eps,
+                                                            int64_t rows,
+                                                            __nv_bfloat16* __restrict__ y) {
+  constexpr int kD = kVPL * 256;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * kD);
+  uint4 v[kVPL];
+#pragma unroll
+  for (int i = 0; i < kVPL; ++i) v[i] = __ldcs(xr + lane + 32 * i);
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < kVPL; ++i) {
+    const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&v[i]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(e[j]);
+      ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+    }
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / static_cast<float>(kD) + eps);
+  uint4* yr = reinterpret_cast<uint4*>(y + row * kD);
+#pragma unroll
+  for (int i = 0; i < kVPL; ++i) {
+    const int c = (lane + 32 * i) * 8;  // first element of this vector
+    const float4 g0 = __ldg(reinterpret_cast<const float4*>(g + c));
+    const float4 g1 = __ldg(reinterpret_cast<const float4*>(g + c) + 1);
+    const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&v[i]);
+    const float2 f0 = __bfloat1622float2(e[0]), f1 = __bfloat1622float2(e[1]);
+    const float2 f2 = __bfloat1622float2(e[2]), f3 = __bfloat1622float2(e[3]);
+    uint4 o;
+    o.x = pack_bf16x2(f0.x * r * g0.x, f0.y * r * g0.y);
+    o.y = pack_bf16x2(f1.x * r * g0.z, f1.y * r * g0.w);
+    o.z = pack_bf16x2(f2.x * r * g1.x, f2.y * r * g1.y);
+    o.w = pack_bf16x2(f3.x * r * g1.z, f3.y * r * g1.w);
+    yr[lane + 32 * i] = o;
+  }
+}
+
 // ---------------------------------------------------------------- RoPE + qk-norm
 // One CTA (4 warps) per token; cos/sin of this token's position in shared
 // memory, then each warp rotates whole heads. Thread 0 also writes the
@@ -150,6 +196,24 @@ __global__ void __launch_bounds__(128) rope_qk(RopePrepArgs a) {
       dst[i + kHalf] = to_t<T>(hi[p] * c + lo[p] * s);
     }
   }
+}
+
+// cos/sin of every (position, frequency) pair, built once per set of
+// positions and read by the QKV GEMM epilogue of every layer.
+__global__ void rope_table_kernel(const int32_t* __restrict__ pos, int64_t T, int half, int dh,
+                                  float rope_base, float2* __restrict__ cs) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= T * half) return;
+  const int64_t t = idx / half;
+  const int i = static_cast<int>(idx % half);
+  const int p = pos ? __ldg(pos + t) : static_cast<int>(t);
+  const double theta = exp2(-(2.0 * i / dh) * log2(static_cast<double>(rope_base)));
+  const double ang = static_cast<double>(p) * theta;
+  const double two_pi = 6.283185307179586476925286766559;
+  const double red = ang - two_pi * rint(ang * (1.0 / two_pi));
+  float sv, cv;
+  sincosf(static_cast<float>(red), &sv, &cv);
+  cs[idx] = make_float2(cv, sv);
 }
 
 // ---------------------------------------------------------------- V transpose
@@ -230,6 +294,22 @@ cudaError_t launch_rmsnorm(const void* x, const float* gamma, float eps, int64_t
                            bool bf16, void* y, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
+  const bool g_al = (reinterpret_cast<uintptr_t>(gamma) & 15u) == 0;
+  const bool xy_al = ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 15u) == 0;
+  if (bf16 && g_al && xy_al && d % 256 == 0 && d <= 16 * 256) {
+    const auto* xb = static_cast<const __nv_bfloat16*>(x);
+    auto* yb = static_cast<__nv_bfloat16*>(y);
+    switch (d / 256) {
+      case 1: rmsnorm_rows_bf16_reg<1><<<blocks, 256, 0, st>>>(xb, gamma, eps, rows, yb); break;
+      case 2: rmsnorm_rows_bf16_reg<2><<<blocks, 256, 0, st>>>(xb, gamma, eps, rows, yb); break;
+      case 4: rmsnorm_rows_bf16_reg<4><<<blocks, 256, 0, st>>>(xb, gamma, eps, rows, yb); break;
+      case 8: rmsnorm_rows_bf16_reg<8><<<blocks, 256, 0, st>>>(xb, gamma, eps, rows, yb); break;
+      case 16: rmsnorm_rows_bf16_reg<16><<<blocks, 256, 0, st>>>(xb, gamma, eps, rows, yb); break;
+      default:
+        rmsnorm_rows<__nv_bfloat16><<<blocks, 256, 0, st>>>(xb, gamma, eps, rows, d, yb);
+    }
+    return cudaGetLastError();
+  }
   if (bf16)
     rmsnorm_rows<__nv_bfloat16><<<blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), gamma, eps, rows, d, static_cast<__nv_bfloat16*>(y));
@@ -255,6 +335,16 @@ cudaError_t launch_rope_prep(const RopePrepArgs& a, cudaStream_t st) {
     else rope_qk<float, 64><<<grid, 128, 0, st>>>(a);
     if (a.kv_v_out) copy_v_f32<<<grid, 128, 0, st>>>(a);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_table(const int32_t* pos, int64_t T, int dh, float rope_base, float2* cs,
+                              cudaStream_t st) {
+  const int half = dh / 2;
+  const int64_t total = T * half;
+  if (total <= 0) return cudaSuccess;
+  rope_table_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(pos, T, half, dh,
+                                                                                rope_base, cs);
   return cudaGetLastError();
 }
 

@@ -170,6 +170,8 @@ struct PrefillPlan {
   float* s_k = nullptr;
   float* lsig_k = nullptr;
   void* sel_ws = nullptr;
+  float2* cs_n = nullptr;  // [n][dh/2] cos/sin of positions 0..n-1 (dense stage)
+  float2* cs_k = nullptr;  // [k][dh/2] cos/sin of the kept positions
   AttnPlan attn;           // sized for n rows, reused by every layer
   size_t bytes = 0;
   PrefillPlan(void* ws, const tg_model& m, int64_t n, int64_t k)
@@ -192,6 +194,8 @@ struct PrefillPlan {
     s_k = static_cast<float*>(a.carve(size_t(k) * 4));
     lsig_k = static_cast<float*>(a.carve(size_t(k) * 4));
     sel_ws = a.carve(select_ws_bytes(n));
+    cs_n = static_cast<float2*>(a.carve(size_t(n) * (dh / 2) * sizeof(float2)));
+    cs_k = static_cast<float2*>(a.carve(size_t(k) * (dh / 2) * sizeof(float2)));
     void* attn_base = a.carve(attn.bytes);
     attn = AttnPlan(attn_base, n, hq, hkv, dh, m.dtype, true);
     bytes = a.used;
@@ -210,6 +214,8 @@ cudaError_t gemm(const GemmArgs& g, tg_dtype dt, cudaStream_t st) {
     case EPI_RESIDUAL: out_bytes = 2.0 * double(g.M) * g.N * e; kid = TG_K_GEMM_RESIDUAL; break;
     case EPI_SWIGLU: out_bytes = double(g.M) * g.inter * e; kid = TG_K_GEMM_SWIGLU; break;
     case EPI_SCORE: out_bytes = double(g.M) * 4.0; kid = TG_K_GEMM_SCORE; break;
+    case EPI_QKV: out_bytes = double(g.M) * g.N * e + (g.v_out ? double(g.M) * g.hkv * 128 * e : 0.0);
+      kid = TG_K_GEMM_QKV; break;
   }
   const double bytes = (double(g.M) + g.N) * g.K * e + out_bytes;
   if (dt == TG_BF16) {
@@ -278,6 +284,33 @@ cudaError_t run_score(const void* x, int64_t rows, int d, int f, const float* no
   });
 }
 
+// Attention over prepared (rotated) q/k and prepared V (bf16: V^T [hkv, dh, t_pad]).
+cudaError_t attn_core(const AttnPlan& plan, const void* k_rot, const void* v, int64_t v_stride,
+                      const float* lsig, const float* gain, const float* tau, int64_t rows, int hq,
+                      int hkv, int dh, tg_dtype dt, void* out, cudaStream_t st) {
+  const size_t es = elem_size(dt);
+  const double attn_flops = 4.0 * dh * hq * double(rows) * double(rows + 1) / 2.0;
+  const double attn_bytes = double(rows) * (2 * hq + 2 * hkv) * dh * es;
+  AttnArgs a{};
+  a.q = plan.q_rot;
+  a.k = k_rot;
+  a.lsig = lsig;
+  a.gain = gain; a.tau = tau;
+  a.T = rows; a.hq = hq; a.hkv = hkv; a.dh = dh;
+  a.out = out;
+  if (dt == TG_BF16) {
+    a.v = plan.vT;
+    a.t_pad = plan.t_pad;
+    if (!attn_tc_supported(a)) return cudaErrorInvalidValue;
+    return traced(TG_K_ATTENTION, rows, attn_flops, attn_bytes, st,
+                  [&] { return launch_attn_tc(a, st); });
+  }
+  a.v = v;
+  a.t_pad = v_stride;
+  return traced(TG_K_ATTENTION_F32, rows, attn_flops, attn_bytes, st,
+                [&] { return launch_attn_simt_f32(a, st); });
+}
+
 // RoPE/qk-norm prep + attention, q/k/v taken from rows with the given strides.
 cudaError_t run_attention(const void* q, int64_t q_stride, const void* kk, int64_t k_stride,
                           const void* v, int64_t v_stride, const int32_t* pos, const float* s,
@@ -306,26 +339,8 @@ cudaError_t run_attention(const void* q, int64_t q_stride, const void* kk, int64
   cudaError_t e = traced(TG_K_ROPE_PREP, rows, 0.0, prep_bytes, st,
                          [&] { return launch_rope_prep(r, st); });
   if (e != cudaSuccess) return e;
-  const double attn_flops = 4.0 * dh * hq * double(rows) * double(rows + 1) / 2.0;
-  const double attn_bytes = double(rows) * (2 * hq + 2 * hkv) * dh * es;
-  AttnArgs a{};
-  a.q = plan.q_rot;
-  a.k = r.k_out;
-  a.lsig = (s || lsig_ready) ? (lsig_ready ? lsig_ready : plan.lsig) : nullptr;
-  a.gain = gain; a.tau = tau;
-  a.T = rows; a.hq = hq; a.hkv = hkv; a.dh = dh;
-  a.out = out;
-  if (dt == TG_BF16) {
-    a.v = plan.vT;
-    a.t_pad = plan.t_pad;
-    if (!attn_tc_supported(a)) return cudaErrorInvalidValue;
-    return traced(TG_K_ATTENTION, rows, attn_flops, attn_bytes, st,
-                  [&] { return launch_attn_tc(a, st); });
-  }
-  a.v = v;
-  a.t_pad = v_stride;
-  return traced(TG_K_ATTENTION_F32, rows, attn_flops, attn_bytes, st,
-                [&] { return launch_attn_simt_f32(a, st); });
+  return attn_core(plan, r.k_out, v, v_stride, (s || lsig_ready) ? (lsig_ready ? lsig_ready : plan.lsig) : nullptr,
+                   gain, tau, rows, hq, hkv, dh, dt, out, st);
 }
 
 // ---- the decoder-layer pieces used by tg_prefill
@@ -336,19 +351,34 @@ struct Dims {
 
 cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
                                const PrefillPlan& P, void* h, int64_t rows, const int32_t* pos,
-                               const float* lsig, const float* gain, const float* tau,
-                               const tg_kv* kv, cudaStream_t st) {
+                               const float2* cs, const float* lsig, const float* gain,
+                               const float* tau, const tg_kv* kv, cudaStream_t st) {
   const tg_dtype dt = m.dtype;
   const size_t e = elem_size(dt);
   cudaError_t err = rmsnorm(h, lw.attn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
   if (err != cudaSuccess) return err;
-  err = gemm(gemm_args(P.y, D.d, lw.wqkv, D.d, P.qkv, D.qkv, rows, D.qkv, D.d, EPI_STORE), dt, st);
-  if (err != cudaSuccess) return err;
-  const char* qkv = static_cast<const char*>(P.qkv);
-  err = run_attention(qkv, D.qkv, qkv + size_t(D.hq) * D.dh * e, D.qkv,
-                      qkv + size_t(D.hq + D.hkv) * D.dh * e, D.qkv, pos, nullptr, lsig, gain, tau,
-                      lw.q_norm, lw.k_norm, m.norm_eps, rows, D.hq, D.hkv, D.dh, m.rope_base, dt,
-                      P.attn, kv ? kv->k : nullptr, kv ? kv->v : nullptr, P.attn_o, st);
+  void* k_dst = (kv && kv->k) ? kv->k : P.attn.k_rot;
+  GemmArgs gq = gemm_args(P.y, D.d, lw.wqkv, D.d, nullptr, 0, rows, D.qkv, D.d, EPI_QKV);
+  gq.hq = D.hq; gq.hkv = D.hkv; gq.rope_cs = cs; gq.q_norm = lw.q_norm; gq.k_norm = lw.k_norm;
+  gq.eps = m.norm_eps; gq.q_out = P.attn.q_rot; gq.k_out = k_dst; gq.vT_out = P.attn.vT;
+  gq.t_pad = P.attn.t_pad; gq.v_out = kv ? kv->v : nullptr;
+  if (dt == TG_BF16 && D.dh == 128 && cs != nullptr && gemm_tc_supported(gq)) {
+    // fused: projection + qk-norm + RoPE + V^T in the GEMM epilogue
+    err = gemm(gq, dt, st);
+    if (err != cudaSuccess) return err;
+    err = attn_core(P.attn, k_dst, nullptr, 0, lsig, gain, tau, rows, D.hq, D.hkv, D.dh, dt,
+                    P.attn_o, st);
+  } else {
+    err = gemm(gemm_args(P.y, D.d, lw.wqkv, D.d, P.qkv, D.qkv, rows, D.qkv, D.d, EPI_STORE), dt,
+               st);
+    if (err != cudaSuccess) return err;
+    const char* qkv = static_cast<const char*>(P.qkv);
+    err = run_attention(qkv, D.qkv, qkv + size_t(D.hq) * D.dh * e, D.qkv,
+                        qkv + size_t(D.hq + D.hkv) * D.dh * e, D.qkv, pos, nullptr, lsig, gain,
+                        tau, lw.q_norm, lw.k_norm, m.norm_eps, rows, D.hq, D.hkv, D.dh,
+                        m.rope_base, dt, P.attn, kv ? kv->k : nullptr, kv ? kv->v : nullptr,
+                        P.attn_o, st);
+  }
   if (err != cudaSuccess) return err;
   GemmArgs g = gemm_args(P.attn_o, int64_t(D.hq) * D.dh, lw.wo, int64_t(D.hq) * D.dh, h, D.d, rows,
                          D.d, D.hq * D.dh, EPI_RESIDUAL);
@@ -550,17 +580,23 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
     ~LayerTag() { t_trace.layer = -1; }
   };
   TG_TRY(copy_rows(P.h, x, size_t(n) * D.d * e, n, st));
+  const bool tables = m.dtype == TG_BF16 && D.dh == 128;
+  const double cs_bytes = 8.0 * (D.dh / 2);
+  if (tables && gate_layer >= 0)
+    TG_TRY(traced(TG_K_ROPE_TABLE, n, 0.0, cs_bytes * n, st, [&] {
+      return launch_rope_table(nullptr, n, D.dh, m.rope_base, P.cs_n, st);
+    }));
   // Stage 1: layers below the gate, and the gate layer's attention, over n rows.
   for (int l = 0; l < gate_layer; ++l) {
     LayerTag tag(l);
-    TG_TRY(attention_sublayer(m, m.layers[l], D, P, P.h, n, nullptr, nullptr, nullptr, nullptr,
-                              kv ? &kv[l] : nullptr, st));
+    TG_TRY(attention_sublayer(m, m.layers[l], D, P, P.h, n, nullptr, P.cs_n, nullptr, nullptr,
+                              nullptr, kv ? &kv[l] : nullptr, st));
     TG_TRY(ffn_sublayer(m, m.layers[l], D, P, P.h, n, st));
   }
   if (gate_layer >= 0) {
     LayerTag tag(gate_layer);
-    TG_TRY(attention_sublayer(m, m.layers[gate_layer], D, P, P.h, n, nullptr, nullptr, nullptr,
-                              nullptr, kv ? &kv[gate_layer] : nullptr, st));
+    TG_TRY(attention_sublayer(m, m.layers[gate_layer], D, P, P.h, n, nullptr, P.cs_n, nullptr,
+                              nullptr, nullptr, kv ? &kv[gate_layer] : nullptr, st));
   }
   // Stage 2: score the post-attention residual, select, compact.
   TG_TRY(run_score(P.h, n, D.d, m.d_score, m.score_norm, m.norm_eps, m.score_w1, m.score_b1,
@@ -568,6 +604,10 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
   TG_TRY(select_topk(sc, protect, n, k, kept_idx, P.sel_ws, st));
   TG_TRY(compact(P.h, nullptr, sc, kept_idx, n, k, static_cast<int>(D.d * e), P.hk, P.pos_k, P.s_k,
                  P.lsig_k, st));
+  if (tables)
+    TG_TRY(traced(TG_K_ROPE_TABLE, k, 0.0, cs_bytes * k + 4.0 * k, st, [&] {
+      return launch_rope_table(P.pos_k, k, D.dh, m.rope_base, P.cs_k, st);
+    }));
   // Stage 3: the gate layer's FFN and the layers above, over the k kept rows.
   if (gate_layer >= 0) {
     LayerTag tag(gate_layer);
@@ -576,7 +616,7 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
   for (int l = gate_layer + 1; l < m.n_layers; ++l) {
     LayerTag tag(l);
     const tg_layer& L = m.layers[l];
-    TG_TRY(attention_sublayer(m, L, D, P, P.hk, k, P.pos_k, P.lsig_k, L.gain, L.tau,
+    TG_TRY(attention_sublayer(m, L, D, P, P.hk, k, P.pos_k, P.cs_k, P.lsig_k, L.gain, L.tau,
                               kv ? &kv[l] : nullptr, st));
     TG_TRY(ffn_sublayer(m, L, D, P, P.hk, k, st));
   }
@@ -653,7 +693,8 @@ int32_t tg_trace_stop(tg_trace_record* out, int32_t cap) {
 const char* tg_kernel_name(int32_t kernel) {
   static const char* names[TG_K_COUNT] = {
       "copy", "rmsnorm", "gemm_tc_store", "gemm_tc_residual", "gemm_tc_swiglu", "gemm_tc_score",
-      "rope_prep", "attention_tc", "select", "compact", "gemm_f32", "attention_f32", "f32_helper"};
+      "rope_prep", "attention_tc", "select", "compact", "gemm_f32", "attention_f32", "f32_helper",
+      "gemm_tc_qkv", "rope_table"};
   return (kernel >= 0 && kernel < TG_K_COUNT) ? names[kernel] : "unknown";
 }
 

@@ -69,6 +69,9 @@ struct RopePrepArgs {
   const float* s; float* lsig_out;
 };
 cudaError_t launch_rope_prep(const RopePrepArgs& a, cudaStream_t st);
+// cs[t][i] = (cos, sin)(pos[t] * base^(-2i/dh)), i < dh/2; pos null = row index.
+cudaError_t launch_rope_table(const int32_t* pos, int64_t T, int dh, float rope_base, float2* cs,
+                              cudaStream_t st);
 
 // fp32 helpers used by the SIMT path
 cudaError_t launch_swiglu_f32(const float* gu, int64_t rows, int inter, float* h, cudaStream_t st);
@@ -76,7 +79,7 @@ cudaError_t launch_score_dot_f32(const float* hpre, int64_t rows, int f, const f
                                  const float* w2, const float* b2, float* scores, cudaStream_t st);
 
 // ---- GEMMs. C[M,N] = A[M,K] . B[N,K]^T with an epilogue.
-enum EpiKind { EPI_STORE = 0, EPI_RESIDUAL = 1, EPI_SWIGLU = 2, EPI_SCORE = 3 };
+enum EpiKind { EPI_STORE = 0, EPI_RESIDUAL = 1, EPI_SWIGLU = 2, EPI_SCORE = 3, EPI_QKV = 4 };
 struct GemmArgs {
   const void* A; int64_t lda;      // [M, K] elements, row stride lda
   const void* B; int64_t ldb;      // [N, K]
@@ -86,6 +89,13 @@ struct GemmArgs {
   EpiKind epi;
   int inter;                       // SWIGLU: I (B rows [0,I) gate, [I,2I) up), N = 2I
   const float* b1; const float* w2; const float* b2; float* scores;  // SCORE
+  // QKV (head dim 128): columns [0, hq*128) are q heads, then hkv k heads,
+  // then hkv v heads. Writes q_out [M, hq, 128] and k_out [M, hkv, 128]
+  // (optional per-head RMSNorm, then RoPE from rope_cs [M][64] (cos, sin)),
+  // vT_out [hkv, 128, t_pad] and, if set, v_out [M, hkv, 128].
+  int hq, hkv;
+  const float2* rope_cs; const float* q_norm; const float* k_norm; float eps;
+  void* q_out; void* k_out; void* vT_out; int64_t t_pad; void* v_out;
 };
 // bf16 on the 5th-generation tensor cores (k_gemm_tc.cu)
 bool gemm_tc_supported(const GemmArgs& g);
