@@ -523,10 +523,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 128; ++i)
           if (kv0 + i > q_row) x[i] = -INFINITY;
       }
-      float rmax = x[0];
+      // Row max and row sum as 8-way trees: a single running max/sum would
+      // be a 128-long chain of dependent instructions per tile.
+      float mx8[8];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) rmax = fmaxf(rmax, x[i]);
-      const float mx = rmax * scale2;
+      for (int i = 0; i < 8; ++i) mx8[i] = x[i];
+#pragma unroll
+      for (int i = 8; i < 128; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], x[i]);
+#pragma unroll
+      for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + w]);
+      const float mx = mx8[0] * scale2;
       float alpha = 1.0f;
       if (mx > m + kRescaleThresh || m == -INFINITY) {
         alpha = ex2(m - mx);  // 0 on the first tile
@@ -534,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = mx;
       }
       const bool rescale_o = j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f);
-      float rsum = 0.f;
+      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
@@ -542,13 +550,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 32; ++i) {
           const float a0 = ex2(fmaf(x[64 * half + 2 * i], scale2, -m));
           const float a1 = ex2(fmaf(x[64 * half + 2 * i + 1], scale2, -m));
-          rsum += a0 + a1;
+          s8[(2 * i) & 7] += a0;
+          s8[(2 * i + 1) & 7] += a1;
           pk[i] = pack_bf16x2(a0, a1);
         }
         tmem_st32(tmem + lane_off + s_col + static_cast<uint32_t>(32 * half), pk);
         tmem_wait_st();
       }
-      l += rsum;
+#pragma unroll
+      for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) s8[i] += s8[i + w];
+      l += s8[0];
       if (rescale_o) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
