@@ -545,6 +545,51 @@ def run_sweep(args):
         gbs = byt / (t / 1e3) / 1e9
         print(json.dumps({"sweep": "select+compact", "n": n, "k": k, "us": t * 1e3,
                           "bytes": byt, "gbs": gbs, "frac_hbm": gbs / pk["hbm"]}), flush=True)
+        del s, prot, x, idx, xo, po, so, ws
+    torch.cuda.empty_cache()
+
+    # Long-context gated attention layer: N=131072 -> K=4096, one attention-only
+    # layer (Qwen3-1.7B heads), scorer + select + compact + gated attention, vs
+    # the same layer dense over all N tokens.
+    w = synth.LONG_128K
+    model = build_model(tg, torch, w, device)
+    x = synth.torch_hidden_states(w, seed=w.seed, device=str(device))
+    prot = torch.zeros(w.n, dtype=torch.uint8, device=device)
+    prot[w.n - w.n_protect:] = 1
+
+    def timed(kk, dense):
+        mdl = dense_model(tg, model) if dense else model
+        o = torch.empty(kk, w.d, dtype=torch.bfloat16, device=device)
+        ki = torch.empty(kk, dtype=torch.int32, device=device)
+        wsz = torch.empty(mdl.workspace_size(w.n, kk, -1), dtype=torch.uint8, device=device)
+        run = lambda: tg.tg_prefill(mdl, x, prot, kk, -1, out=o, kept_idx=ki, ws=wsz)  # noqa: E731
+        run()
+        torch.cuda.synchronize()
+        ms = []
+        tg.tg_trace_start(4096)
+        for _ in range(max(2, args.steps // 3)):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            run()
+            b.record()
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        tr = tg.tg_trace_stop()
+        att = [r for r in tr if r["kernel"] == "attention_tc"]
+        att_tf = sum(r["flops"] for r in att) / (sum(r["ms"] for r in att) / 1e3) / 1e12
+        del o, ki, wsz
+        return statistics.median(ms), att_tf
+
+    g_ms, g_tf = timed(w.k, False)
+    d_ms, d_tf = timed(w.n, True)
+    print(json.dumps({"workload": w.name, "n": w.n, "k": w.k, "gated_ms": g_ms,
+                      "gated_attention_tflops": g_tf, "dense_ms": d_ms,
+                      "dense_attention_tflops": d_tf, "speedup_vs_dense": d_ms / g_ms,
+                      "attn_frac_of_sustained_peak": {"gated": g_tf / pk["bf16_sustained"],
+                                                      "dense": d_tf / pk["bf16_sustained"]}}),
+          flush=True)
 
 
 # ----------------------------------------------------------------- profiling cases
@@ -566,6 +611,34 @@ def run_case(args):
     torch.manual_seed(0)
     w = WORKLOAD
     t = args.rows
+    if args.case == "gemm":
+        # the prefill's projection shapes: tg_linear (tcgen05) next to
+        # torch.matmul (cuBLAS) on the same operands, interleaved
+        shapes = [("qkv", 4096, 2048), ("o_proj", 2048, 2048), ("gate_up", 12288, 2048),
+                  ("down", 2048, 6144)]
+        for name, n, kdim in shapes:
+            x = torch.randn(t, kdim, device=device, dtype=torch.bfloat16)
+            wt = torch.randn(n, kdim, device=device, dtype=torch.bfloat16) * 0.02
+            y = torch.empty(t, n, device=device, dtype=torch.bfloat16)
+            res = {}
+            for _ in range(3):
+                for impl in ("tg_linear", "cublas"):
+                    f = (lambda: tg.tg_linear(x, wt, y=y)) if impl == "tg_linear" else \
+                        (lambda: torch.matmul(x, wt.t(), out=y))
+                    f()
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record()
+                    for _ in range(args.steps):
+                        f()
+                    b.record()
+                    torch.cuda.synchronize()
+                    res.setdefault(impl, []).append(a.elapsed_time(b) / args.steps)
+            fl = 2.0 * t * n * kdim
+            print(json.dumps({"case": "gemm", "shape": name, "m": t, "n": n, "k": kdim,
+                              **{f"{i}_tflops": fl / (statistics.median(v) / 1e3) / 1e12
+                                 for i, v in res.items()}}), flush=True)
+        return 0
     if args.case == "attn":
         q = torch.randn(t, w.hq, w.dh, device=device, dtype=torch.bfloat16)
         kk = torch.randn(t, w.hkv, w.dh, device=device, dtype=torch.bfloat16)
@@ -608,7 +681,7 @@ def main():
     ap.add_argument("--quick", action="store_true", help="skip the other budgets / dense run")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--sweep", action="store_true")
-    ap.add_argument("--case", choices=["attn", "layer"], default=None)
+    ap.add_argument("--case", choices=["attn", "layer", "gemm"], default=None)
     ap.add_argument("--rows", type=int, default=32768)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup

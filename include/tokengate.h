@@ -175,6 +175,19 @@ tg_status tg_gated_attn_prefill(const void* q, const void* kk, const void* v, co
                                 tg_dtype dtype, void* out, void* ws, size_t ws_bytes,
                                 tg_stream stream);
 
+/*
+ * tg_linear -- the backbone's projection GEMM, y = x . w^T (+ residual).
+ * The dense contraction of every QKV / output / FFN projection in the layers
+ * the gated stack runs ([TC] "TokenGate 提前筛选 Token": layers compute
+ * attention and feed-forward per token); exposed on its own for users and
+ * for measuring the kernel against a library GEMM.
+ *   x [m, k], w [n, k], residual [m, n] or NULL (may equal y), y [m, n]; dtype
+ * bf16: tcgen05 tensor cores, needs n % 32 == 0, k % 8 == 0, 16-byte aligned
+ * pointers; fp32: CUDA-core GEMM, any sizes.
+ */
+tg_status tg_linear(const void* x, const void* w, const void* residual, int64_t m, int32_t n,
+                    int32_t k, tg_dtype dtype, void* y, tg_stream stream);
+
 /* ---- the full stack ---------------------------------------------------- */
 
 typedef struct {
@@ -226,10 +239,16 @@ typedef struct {
  *   out [k, d] dtype: final-normed hidden states of the kept rows
  *   kept_idx [k] int32 (out, ascending); scores [n] fp32 (out) or NULL
  *   kv: HOST array of n_layers tg_kv, or NULL
+ *   hidden: HOST array of n_layers device pointers, or NULL. hidden[l], when
+ *     not NULL, receives layer l's output hidden states (after its FFN):
+ *     [n, d] for layers below the gate, [k, d] (kept rows, ascending) for the
+ *     gate layer and above. For inspection and per-layer checks; one copy
+ *     per requested layer.
  */
 tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protect, int64_t n,
                      int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx, float* scores,
-                     const tg_kv* kv, void* ws, size_t ws_bytes, tg_stream stream);
+                     const tg_kv* kv, void* const* hidden, void* ws, size_t ws_bytes,
+                     tg_stream stream);
 
 /* ---- launch tracing (optional) --------------------------------------------
  * Measurement aid with no counterpart on the pages (they report only

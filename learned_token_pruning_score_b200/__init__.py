@@ -79,13 +79,15 @@ _workspace_size = _sig("tg_workspace_size", _c_sz, _ci, ctypes.POINTER(TgShape))
 _score = _sig("tg_score", _ci, _c_p, _c_i64, _c_i32, _c_i32, _c_p, _c_f32, _c_p, _c_p, _c_p, _c_p,
               _ci, _c_p, _c_p, _c_sz, _c_p)
 _topk = _sig("tg_topk_select", _ci, _c_p, _c_p, _c_i64, _c_i64, _c_p, _c_p, _c_sz, _c_p)
+_linear = _sig("tg_linear", _ci, _c_p, _c_p, _c_p, _c_i64, _c_i32, _c_i32, _ci, _c_p, _c_p)
 _topk_noalloc = _sig("tg_topk_select_noalloc", _ci, _c_p, _c_p, _c_i64, _c_i64, _c_p, _c_p)
 _compact = _sig("tg_compact", _ci, _c_p, _c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i32, _ci, _c_p,
                 _c_p, _c_p, _c_p)
 _attn = _sig("tg_gated_attn_prefill", _ci, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i64,
              _c_i32, _c_i32, _c_i32, _c_f32, _ci, _c_p, _c_p, _c_sz, _c_p)
 _prefill = _sig("tg_prefill", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64, _c_i64, _c_i32,
-                _c_p, _c_p, _c_p, ctypes.POINTER(TgKV), _c_p, _c_sz, _c_p)
+                _c_p, _c_p, _c_p, ctypes.POINTER(TgKV), ctypes.POINTER(_c_p), _c_p, _c_sz,
+                _c_p)
 _status_string = _sig("tg_status_string", ctypes.c_char_p, _ci)
 _last_cuda_error = _sig("tg_last_cuda_error", _ci)
 _device_error = _sig("tg_device_error", _ci, ctypes.POINTER(ctypes.c_uint32), _ci)
@@ -208,6 +210,17 @@ def tg_topk_select(scores, protect, k: int, kept_idx=None, ws=None, stream=None)
     return kept_idx
 
 
+def tg_linear(x, w, residual=None, y=None, stream=None) -> torch.Tensor:
+    """y = x . w^T (+ residual): x [m, k], w [n, k] (nn.Linear layout)."""
+    m, k = x.shape
+    n = w.shape[0]
+    if y is None:
+        y = torch.empty(m, n, dtype=x.dtype, device=x.device)
+    _check(_linear(_ptr(x), _ptr(w), _ptr(residual), m, n, k, _dt(x), _ptr(y),
+                   _stream(stream, x.device)), "tg_linear")
+    return y
+
+
 SELECT_NOALLOC_MAX_N = 1 << 20
 
 
@@ -305,8 +318,13 @@ class Model:
 
 
 def tg_prefill(model: Model, x, protect, k: int, gate_layer: int, out=None, kept_idx=None,
-               scores=None, kv: Optional[Sequence] = None, ws=None, stream=None):
-    """Returns (out [k, d], kept_idx [k], scores [n] or None)."""
+               scores=None, kv: Optional[Sequence] = None, hidden: Optional[Sequence] = None,
+               ws=None, stream=None):
+    """Returns (out [k, d], kept_idx [k], scores [n] or None).
+
+    kv: per-layer (k_cache, v_cache) tensors or None entries; hidden:
+    per-layer output hidden-state tensors ([n, d] below the gate, [k, d] at
+    and above it) or None entries."""
     n, d = x.shape
     if out is None:
         out = torch.empty(k, d, dtype=x.dtype, device=x.device)
@@ -319,14 +337,19 @@ def tg_prefill(model: Model, x, protect, k: int, gate_layer: int, out=None, kept
         for i, pair in enumerate(kv):
             if pair is not None:
                 kv_c[i].k, kv_c[i].v = _ptr(pair[0]), _ptr(pair[1])
+    hid_c = None
+    if hidden is not None:
+        hid_c = (_c_p * len(model.layers))()
+        for i, t in enumerate(hidden):
+            hid_c[i] = _ptr(t)
     _check(_prefill(ctypes.byref(model.c), _ptr(x), _ptr(protect), n, k, gate_layer, _ptr(out),
-                    _ptr(kept_idx), _ptr(scores), kv_c, _ptr(ws), ws.numel(),
+                    _ptr(kept_idx), _ptr(scores), kv_c, hid_c, _ptr(ws), ws.numel(),
                     _stream(stream, x.device)), "tg_prefill")
     return out, kept_idx, scores
 
 
 __all__ = [
-    "tg_score", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_prefill",
+    "tg_score", "tg_linear", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_prefill",
     "tg_workspace_size", "tg_status_string", "tg_device_error", "tg_version", "Model",
     "TokenGateError", "LIB_PATH", "tg_trace_start", "tg_trace_stop", "TG_OK", "TG_ERR_INVALID_ARG", "TG_ERR_UNSUPPORTED",
     "TG_ERR_BUDGET", "TG_ERR_WORKSPACE", "TG_ERR_CUDA", "TG_F32", "TG_BF16", "TG_OP_SCORE",

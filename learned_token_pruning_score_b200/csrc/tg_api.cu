@@ -508,6 +508,20 @@ tg_status tg_topk_select(const float* scores, const uint8_t* protect, int64_t n,
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+tg_status tg_linear(const void* x, const void* w, const void* residual, int64_t m, int32_t n,
+                    int32_t k, tg_dtype dt, void* y, tg_stream stream) {
+  TG_CHECK(dt == TG_BF16 || dt == TG_F32, TG_ERR_UNSUPPORTED);
+  TG_CHECK(x && w && y && m >= 1 && n >= 1 && k >= 1, TG_ERR_INVALID_ARG);
+  GemmArgs g = gemm_args(x, k, w, k, y, n, m, n, k, residual ? EPI_RESIDUAL : EPI_STORE);
+  g.R = residual;
+  g.ldr = n;
+  if (dt == TG_BF16) {
+    TG_CHECK(n % 32 == 0 && k % 8 == 0, TG_ERR_UNSUPPORTED);
+    TG_CHECK(gemm_tc_supported(g), TG_ERR_INVALID_ARG);
+  }
+  return cuda_status(gemm(g, dt, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 tg_status tg_topk_select_noalloc(const float* scores, const uint8_t* protect, int64_t n,
                                  int64_t k, int32_t* kept_idx, tg_stream stream) {
   TG_CHECK(scores && kept_idx && n >= 1, TG_ERR_INVALID_ARG);
@@ -560,7 +574,8 @@ tg_status tg_gated_attn_prefill(const void* q, const void* kk, const void* v, co
 
 tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protect, int64_t n,
                      int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx, float* scores,
-                     const tg_kv* kv, void* ws, size_t ws_bytes, tg_stream stream) {
+                     const tg_kv* kv, void* const* hidden, void* ws, size_t ws_bytes,
+                     tg_stream stream) {
   const tg_status vs = validate_model(model, n, k, gate_layer);
   if (vs != TG_OK) return vs;
   TG_CHECK(x && out && kept_idx, TG_ERR_INVALID_ARG);
@@ -592,6 +607,7 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
     TG_TRY(attention_sublayer(m, m.layers[l], D, P, P.h, n, nullptr, P.cs_n, nullptr, nullptr,
                               nullptr, kv ? &kv[l] : nullptr, st));
     TG_TRY(ffn_sublayer(m, m.layers[l], D, P, P.h, n, st));
+    if (hidden && hidden[l]) TG_TRY(copy_rows(hidden[l], P.h, size_t(n) * D.d * e, n, st));
   }
   if (gate_layer >= 0) {
     LayerTag tag(gate_layer);
@@ -612,6 +628,8 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
   if (gate_layer >= 0) {
     LayerTag tag(gate_layer);
     TG_TRY(ffn_sublayer(m, m.layers[gate_layer], D, P, P.hk, k, st));
+    if (hidden && hidden[gate_layer])
+      TG_TRY(copy_rows(hidden[gate_layer], P.hk, size_t(k) * D.d * e, k, st));
   }
   for (int l = gate_layer + 1; l < m.n_layers; ++l) {
     LayerTag tag(l);
@@ -619,6 +637,7 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
     TG_TRY(attention_sublayer(m, L, D, P, P.hk, k, P.pos_k, P.cs_k, P.lsig_k, L.gain, L.tau,
                               kv ? &kv[l] : nullptr, st));
     TG_TRY(ffn_sublayer(m, L, D, P, P.hk, k, st));
+    if (hidden && hidden[l]) TG_TRY(copy_rows(hidden[l], P.hk, size_t(k) * D.d * e, k, st));
   }
   if (m.final_norm)
     TG_TRY(rmsnorm(P.hk, m.final_norm, m.norm_eps, k, D.d, m.dtype, out, st));

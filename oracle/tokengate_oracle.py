@@ -240,27 +240,28 @@ def rope(x, pos, base: float) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 
-def gated_attention(q, k, v, pos, s, gain, tau) -> np.ndarray:
-    """o_i = sum_j softmax_j(l_ij) v_j over kept keys with pos_j <= pos_i.
+def gated_attention_rows(q, pos_q, k, v, pos_k, s, gain, tau) -> np.ndarray:
+    """Token-gated attention of query rows q [Tq, Hq, dh] at positions pos_q
+    over keys k/v [Tk, Hkv, dh] at positions pos_k (R2, R5):
 
-    l_ij = (q_i . k_j) / (sqrt(dh) * tau_h) + gain_h * logsigmoid(s_j)
+    l_ij = (q_i . k_j) / (sqrt(dh) * tau_h) + gain_h * logsigmoid(s_j), pos_j <= pos_i
 
-    q: [T, Hq, dh] (already rotated), k/v: [T, Hkv, dh], pos: [T] original
-    positions, s: [T] gate scores or None (no bias), gain/tau: [Hq] or None
+    s: [Tk] gate scores of the keys or None (no bias); gain/tau: [Hq] or None
     (gain 0, tau 1). Pruned keys are simply absent from k/v.
     """
     q = np.asarray(q, dtype=F64)
     k = np.asarray(k, dtype=F64)
     v = np.asarray(v, dtype=F64)
-    t, hq, dh = q.shape
-    hkv = k.shape[1]
+    tq, hq, dh = q.shape
+    tk, hkv = k.shape[0], k.shape[1]
     group = hq // hkv
     gain = np.zeros(hq) if gain is None else np.asarray(gain, dtype=F64)
     tau = np.ones(hq) if tau is None else np.asarray(tau, dtype=F64)
-    key_bias = np.zeros(t) if s is None else logsigmoid(s)
-    p = np.asarray(pos, dtype=np.int64)
-    allowed = p[None, :] <= p[:, None]  # [query i, key j]
-    out = np.empty((t, hq, dh), dtype=F64)
+    key_bias = np.zeros(tk) if s is None else logsigmoid(s)
+    pq = np.asarray(pos_q, dtype=np.int64)
+    pk = np.asarray(pos_k, dtype=np.int64)
+    allowed = pk[None, :] <= pq[:, None]  # [query i, key j]
+    out = np.empty((tq, hq, dh), dtype=F64)
     for h in range(hq):
         g = h // group
         logits = (q[:, h, :] @ k[:, g, :].T) / (math.sqrt(dh) * tau[h])
@@ -271,6 +272,12 @@ def gated_attention(q, k, v, pos, s, gain, tau) -> np.ndarray:
         w = w / w.sum(axis=1, keepdims=True)
         out[:, h, :] = w @ v[:, g, :]
     return out
+
+
+def gated_attention(q, k, v, pos, s, gain, tau) -> np.ndarray:
+    """o_i = sum_j softmax_j(l_ij) v_j over kept keys with pos_j <= pos_i,
+    for the kept rows themselves as queries (q, k, v share positions pos)."""
+    return gated_attention_rows(q, pos, k, v, pos, s, gain, tau)
 
 
 def gated_attn_prefill(q, k, v, pos, s, gain, tau, rope_base, store=round_bf16):
@@ -431,7 +438,7 @@ def select_compact_bytes(n: int, k: int, d: int, elem: int = 2) -> int:
 __all__: Sequence[str] = [
     "round_bf16", "round_fp32", "identity", "STORE", "rmsnorm", "silu", "sigmoid",
     "logsigmoid", "score", "BudgetError", "topk_select", "compact", "rope",
-    "gated_attention", "gated_attn_prefill", "Layer", "Model", "attention_sublayer",
+    "gated_attention", "gated_attention_rows", "gated_attn_prefill", "Layer", "Model", "attention_sublayer",
     "ffn_sublayer", "prefill", "PrefillResult", "gated_layer_forward",
     "attention_flops", "select_compact_bytes",
 ]

@@ -120,26 +120,25 @@ def _bogus_model(**over):
     return m, layers
 
 
+def _prefill(model, n, k, gate, ws_bytes):
+    return tg._prefill(model, BOGUS, None, n, k, gate, BOGUS, BOGUS, None, None, None, BOGUS,
+                       ws_bytes, None)
+
+
 def test_prefill_validation():
-    f = tg._prefill
     m, keep = _bogus_model()
-    assert f(ctypes.byref(m), BOGUS, None, 1000, 0, 1, BOGUS, BOGUS, None, None, BOGUS, 1 << 40,
-             None) == tg.TG_ERR_BUDGET
-    assert f(ctypes.byref(m), BOGUS, None, 1000, 100, 2, BOGUS, BOGUS, None, None, BOGUS, 1 << 40,
-             None) == tg.TG_ERR_INVALID_ARG  # gate layer past the stack
-    assert f(ctypes.byref(m), BOGUS, None, 1000, 100, 1, BOGUS, BOGUS, None, None, BOGUS, 16,
-             None) == tg.TG_ERR_WORKSPACE
+    big = 1 << 40
+    assert _prefill(ctypes.byref(m), 1000, 0, 1, big) == tg.TG_ERR_BUDGET
+    assert _prefill(ctypes.byref(m), 1000, 1001, 1, big) == tg.TG_ERR_BUDGET
+    assert _prefill(ctypes.byref(m), 1000, 100, 2, big) == tg.TG_ERR_INVALID_ARG  # gate past stack
+    assert _prefill(ctypes.byref(m), 1000, 100, 1, 16) == tg.TG_ERR_WORKSPACE
     m2, keep2 = _bogus_model(head_dim=64)
-    assert f(ctypes.byref(m2), BOGUS, None, 1000, 100, 1, BOGUS, BOGUS, None, None, BOGUS,
-             1 << 40, None) == tg.TG_ERR_UNSUPPORTED
+    assert _prefill(ctypes.byref(m2), 1000, 100, 1, big) == tg.TG_ERR_UNSUPPORTED
     m3, keep3 = _bogus_model(d_ffn=6100)  # SwiGLU width must be a multiple of 128 in bf16
-    assert f(ctypes.byref(m3), BOGUS, None, 1000, 100, 1, BOGUS, BOGUS, None, None, BOGUS,
-             1 << 40, None) == tg.TG_ERR_UNSUPPORTED
-    assert f(None, BOGUS, None, 1000, 100, 1, BOGUS, BOGUS, None, None, BOGUS, 1 << 40, None) == \
-        tg.TG_ERR_INVALID_ARG
+    assert _prefill(ctypes.byref(m3), 1000, 100, 1, big) == tg.TG_ERR_UNSUPPORTED
+    assert _prefill(None, 1000, 100, 1, big) == tg.TG_ERR_INVALID_ARG
     keep[0].k_norm = 4096  # q_norm and k_norm come together
-    assert f(ctypes.byref(m), BOGUS, None, 1000, 100, 1, BOGUS, BOGUS, None, None, BOGUS,
-             1 << 40, None) == tg.TG_ERR_INVALID_ARG
+    assert _prefill(ctypes.byref(m), 1000, 100, 1, big) == tg.TG_ERR_INVALID_ARG
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="exercises the no-device error path")

@@ -130,3 +130,30 @@ def test_attn_reduces_to_causal_attention_when_gain_zero_tau_one():
     want = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True,
                                                             enable_gqa=True)
     assert_close(out, want[0].permute(1, 0, 2).numpy(), torch.bfloat16, "sdpa")
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 256, 64), (127, 2048, 2048), (1000, 4096, 2048),
+                                   (300, 2048, 6144), (4096, 288, 520)])
+@pytest.mark.parametrize("residual", [False, True])
+def test_linear_bf16(m, n, k, residual):
+    """The tcgen05 GEMM against a float64 product of the same bf16 values
+    (ragged m, k not a multiple of 64, n not a multiple of 256)."""
+    rng = np.random.default_rng(m + n + k)
+    x = dev(rng.standard_normal((m, k)), torch.bfloat16)
+    w = dev(rng.standard_normal((n, k)) * 0.02, torch.bfloat16)
+    r = dev(rng.standard_normal((m, n)), torch.bfloat16) if residual else None
+    y = tg.tg_linear(x, w, residual=r)
+    torch.cuda.synchronize()
+    want = host64(x) @ host64(w).T + (host64(r) if residual else 0.0)
+    assert_close(y, ref.round_bf16(want), torch.bfloat16, f"linear {m}x{n}x{k}")
+
+
+def test_linear_fp32_and_in_place_residual():
+    rng = np.random.default_rng(5)
+    x = dev(rng.standard_normal((77, 96)))
+    w = dev(rng.standard_normal((40, 96)))
+    y = dev(rng.standard_normal((77, 40)))
+    y0 = host64(y)
+    tg.tg_linear(x, w, residual=y, y=y)
+    torch.cuda.synchronize()
+    assert_close(y, host64(x) @ host64(w).T + y0, torch.float32, "fp32 linear")

@@ -1,0 +1,235 @@
+"""GPU parity at the benchmark workloads' sizes.
+
+* 28-layer Qwen3-1.7B-shaped gated prefill (qk-norm, gate at layer 1),
+  checked per layer and teacher-forced (hidden states with the bulk form of
+  the tolerance, see tests/_helpers.assert_close_bulk): the oracle runs each layer on the
+  GPU's own output of the layer before (tg_prefill's per-layer hidden-state
+  outputs), so bf16 rounding differences cannot accumulate over 28 layers;
+  the kept set is checked bit-exactly on the GPU's scores.
+  - at a reduced N=4096, K=512 (every other shape unchanged): every row;
+  - at the full N=32768, K=4096: sampled rows, attention keys and values
+    taken from the GPU's KV cache of the layer (its rows at the sampled
+    tokens checked too).
+* long-context gated attention layer: N=131072 -> K=4096, in full.
+
+Weights are drawn on the device (seeded), so host and device see the same
+bf16 values. Tolerance: |gpu - ref| <= 2e-2 + 1e-2 |ref|.
+"""
+
+from collections.abc import Sequence
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import tokengate_oracle as ref
+from tests._helpers import assert_close, assert_close_bulk, boundary_flips, host64
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+tg = pytest.importorskip("learned_token_pruning_score_b200")
+BF16 = torch.bfloat16
+rb = ref.round_bf16
+
+
+@pytest.fixture(autouse=True)
+def _no_device_errors():
+    tg.tg_device_error(clear=True)
+    yield
+    assert tg.tg_device_error() == 0
+
+
+class HostLayers(Sequence):
+    """The device layers as oracle Layers, converted to float64 on access
+    (one layer cached: the oracle walks them in order)."""
+
+    def __init__(self, layers):
+        self.layers = layers
+        self.cache = (None, None)
+
+    def __len__(self):
+        return len(self.layers)
+
+    def __getitem__(self, i):
+        if self.cache[0] != i:
+            lp = self.layers[i]
+            g = lambda k: host64(lp[k]) if k in lp else None  # noqa: E731
+            self.cache = (i, ref.Layer(attn_norm=g("attn_norm"), wqkv=g("wqkv"), wo=g("wo"),
+                                       ffn_norm=g("ffn_norm"), w_gate_up=g("w_gate_up"),
+                                       w_down=g("w_down"), q_norm=g("q_norm"), k_norm=g("k_norm"),
+                                       gain=g("gain"), tau=g("tau")))
+        return self.cache[1]
+
+
+def _models(w):
+    p = synth.torch_model_params(w, seed=w.seed, device="cuda")
+    score = {k: p[k] for k in ("score_norm", "score_w1", "score_b1", "score_w2", "score_b2")}
+    model = tg.Model(n_heads_q=w.hq, n_heads_kv=w.hkv, head_dim=w.dh, layers=p["layers"],
+                     score=score, final_norm=p["final_norm"], eps=w.eps, rope_base=w.rope_base)
+    om = ref.Model(d_model=w.d, n_heads_q=w.hq, n_heads_kv=w.hkv, head_dim=w.dh,
+                   layers=HostLayers(p["layers"]), final_norm=host64(p["final_norm"]),
+                   score_norm=host64(score["score_norm"]), score_w1=host64(score["score_w1"]),
+                   score_b1=host64(score["score_b1"]), score_w2=host64(score["score_w2"]),
+                   score_b2=host64(score["score_b2"]), eps=w.eps, rope_base=w.rope_base)
+    return model, om
+
+
+def _run_gpu(w, model, x, prot, with_hidden=False):
+    kv, hidden = [], []
+    for li in range(w.n_layers):
+        rows = w.n if li <= w.gate_layer else w.k
+        kv.append((torch.empty(rows, w.hkv, w.dh, device="cuda", dtype=BF16),
+                   torch.empty(rows, w.hkv, w.dh, device="cuda", dtype=BF16)))
+        hrows = w.n if li < w.gate_layer else w.k
+        hidden.append(torch.empty(hrows, w.d, device="cuda", dtype=BF16))
+    scores = torch.empty(w.n, device="cuda")
+    out, kept, _ = tg.tg_prefill(model, x, torch.from_numpy(prot).cuda(), w.k, w.gate_layer,
+                                 scores=scores, kv=kv, hidden=hidden if with_hidden else None)
+    torch.cuda.synchronize()
+    return out, kept.cpu().numpy(), scores.cpu().numpy(), kv, hidden
+
+
+def test_prefill_28_layers_reduced_n_per_layer():
+    w = synth.shrink(synth.QWEN_PREFILL_32K, n=4096, k=512)
+    model, om = _models(w)
+    x = synth.torch_hidden_states(w, seed=w.seed + 1000, device="cuda")
+    prot = synth.protect_tail(w.n, w.n_protect)
+    out, kept, scores, kv, hidden = _run_gpu(w, model, x, prot, with_hidden=True)
+    assert np.array_equal(kept, ref.topk_select(scores, prot, w.k))
+    pos_n = np.arange(w.n)
+    s_k = scores[kept].astype(np.float64)
+    h_in = host64(x)
+    for li in range(w.n_layers):
+        lw = om.layers[li]
+        dense = li <= w.gate_layer
+        pos = pos_n if dense else kept
+        r, (k_o, v_o) = ref.attention_sublayer(h_in, lw, om, pos, None if dense else s_k,
+                                               None if dense else lw.gain,
+                                               None if dense else lw.tau, rb)
+        assert_close(kv[li][0], k_o, BF16, f"k layer {li}")
+        assert_close(kv[li][1], v_o, BF16, f"v layer {li}")
+        if li == w.gate_layer:
+            s_ref = ref.round_fp32(ref.score(r, om.score_norm, om.eps, om.score_w1, om.score_b1,
+                                             om.score_w2, om.score_b2, rb))
+            assert_close(scores, s_ref, BF16, "scores")
+            flips, near = boundary_flips(s_ref.astype(np.float32), kept, prot, w.k, 2e-2, 1e-2)
+            assert near, flips
+            r = r[kept]
+        h_out = ref.ffn_sublayer(r, lw, om, rb)
+        assert_close_bulk(hidden[li], h_out, BF16, f"hidden layer {li}")
+        h_in = host64(hidden[li])  # teacher forcing: the next layer reads the GPU's output
+    assert_close(out, rb(ref.rmsnorm(h_in, om.final_norm, om.eps)), BF16, "out")
+
+
+def _attn_row(h, lw, m, pos_q, k_cache, v_cache, pos_k, s_k, gain, tau, want_k, want_v, what):
+    """One token through one layer's attention sub-layer, its keys/values
+    taken from the GPU's KV cache rows [0..its own row]; checks its own k/v."""
+    hq, hkv, dh = m.n_heads_q, m.n_heads_kv, m.head_dim
+    y = rb(ref.rmsnorm(h[None], lw.attn_norm, m.eps))
+    qkv = rb(y @ lw.wqkv.T)
+    q = qkv[:, : hq * dh].reshape(1, hq, dh)
+    k = qkv[:, hq * dh: (hq + hkv) * dh].reshape(1, hkv, dh)
+    v = qkv[:, (hq + hkv) * dh:].reshape(1, hkv, dh)
+    if lw.q_norm is not None:
+        q = ref.rmsnorm(q, lw.q_norm, m.eps)
+        k = ref.rmsnorm(k, lw.k_norm, m.eps)
+    q = rb(ref.rope(q, np.array([pos_q]), m.rope_base))
+    k = rb(ref.rope(k, np.array([pos_q]), m.rope_base))
+    assert_close(want_k, k[0], BF16, f"k {what}")
+    assert_close(want_v, v[0], BF16, f"v {what}")
+    o = rb(ref.gated_attention_rows(q, np.array([pos_q]), k_cache, v_cache, pos_k, s_k, gain, tau))
+    return rb(h[None] + o.reshape(1, hq * dh) @ lw.wo.T)[0]
+
+
+def test_prefill_28_layers_full_size_sampled_rows():
+    w = synth.QWEN_PREFILL_32K  # N=32768, K=4096, 28 layers, gate at layer 1
+    model, om = _models(w)
+    x = synth.torch_hidden_states(w, seed=w.seed + 1000, device="cuda")
+    prot = synth.protect_tail(w.n, w.n_protect)
+    out, kept, scores, kv, hidden = _run_gpu(w, model, x, prot, with_hidden=True)
+    # the kept set is exactly the selection of the GPU's scores
+    assert np.array_equal(kept, ref.topk_select(scores, prot, w.k))
+    rng = np.random.default_rng(11)
+    kept_set = set(kept.tolist())
+    pruned = np.array(sorted(set(range(w.n)) - kept_set))
+    sample_kept = sorted({int(kept[-1]), int(kept[0])} |
+                         set(rng.choice(kept[:-w.n_protect], 4, replace=False).tolist()) |
+                         {int(np.nonzero(prot)[0][3])})
+    sample_pruned = sorted(rng.choice(pruned, 3, replace=False).tolist())
+    tokens = sample_kept + sample_pruned
+    row_of = {int(t): r for r, t in enumerate(kept)}
+    s_kept = scores[kept].astype(np.float64)
+    rows = lambda t_, idx: host64(t_[torch.as_tensor(idx, device="cuda")])  # noqa: E731
+    xin = dict(zip(tokens, rows(x, tokens)))
+    for li in range(w.n_layers):
+        lw = om.layers[li]
+        if li <= w.gate_layer:  # every sampled token, keys 0..t
+            kc, vc = host64(kv[li][0]), host64(kv[li][1])
+            hin = xin if li == 0 else dict(zip(tokens, rows(hidden[li - 1], tokens)))
+            for t in tokens:
+                r = _attn_row(hin[t], lw, om, t, kc[: t + 1], vc[: t + 1], np.arange(t + 1),
+                              None, None, None, kc[t], vc[t], f"layer {li} token {t}")
+                if li < w.gate_layer:
+                    want = rows(hidden[li], [t])[0]
+                    assert_close_bulk(want, ref.ffn_sublayer(r[None], lw, om, rb)[0], BF16,
+                                      f"hidden layer {li} token {t}")
+                    continue
+                # the gate layer: score of the post-attention residual, then its
+                # FFN on the kept rows
+                s_ref = ref.round_fp32(ref.score(r[None], om.score_norm, om.eps, om.score_w1,
+                                                 om.score_b1, om.score_w2, om.score_b2, rb))
+                assert_close(scores[t:t + 1], s_ref, BF16, f"score token {t}")
+                if t in kept_set:
+                    want = rows(hidden[li], [row_of[t]])[0]
+                    assert_close_bulk(want, ref.ffn_sublayer(r[None], lw, om, rb)[0], BF16,
+                                      f"hidden layer {li} kept row {row_of[t]}")
+            del kc, vc
+            continue
+        rk_list = [row_of[t] for t in sample_kept]
+        hin = dict(zip(sample_kept, rows(hidden[li - 1], rk_list)))
+        want_out = dict(zip(sample_kept, rows(hidden[li], rk_list)))
+        kc_all, vc_all = host64(kv[li][0]), host64(kv[li][1])
+        for t in sample_kept:
+            rk = row_of[t]
+            kc, vc = kc_all[: rk + 1], vc_all[: rk + 1]
+            r = _attn_row(hin[t], lw, om, t, kc, vc, kept[: rk + 1], s_kept[: rk + 1], lw.gain,
+                          lw.tau, kc[rk], vc[rk], f"layer {li} kept row {rk}")
+            assert_close_bulk(want_out[t], ref.ffn_sublayer(r[None], lw, om, rb)[0], BF16,
+                              f"hidden layer {li} kept row {rk}")
+    last = rows(hidden[-1], [row_of[t] for t in sample_kept])
+    final = rb(ref.rmsnorm(last, om.final_norm, om.eps))
+    assert_close(rows(out, [row_of[t] for t in sample_kept]), final, BF16, "out sampled rows")
+
+
+def test_long_context_gated_layer_128k():
+    """N=131072 -> K=4096 (last 256 protected), one attention-only gated
+    layer with Qwen3-1.7B heads: scorer + select + compact + gated attention."""
+    w = synth.LONG_128K
+    rng = synth.rng_for(w.seed)
+    p = synth.model_params(w, rng)
+    dev = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to("cuda", dt)  # noqa: E731
+    lp = p["layers"][0]
+    layer_d = {k: dev(v, BF16 if v.ndim == 2 else torch.float32) for k, v in lp.items()}
+    score = {k: dev(p[k], BF16 if p[k].ndim == 2 else torch.float32)
+             for k in ("score_norm", "score_w1", "score_b1", "score_w2", "score_b2")}
+    model = tg.Model(n_heads_q=w.hq, n_heads_kv=w.hkv, head_dim=w.dh, layers=[layer_d],
+                     score=score, final_norm=dev(p["final_norm"], torch.float32))
+    g = lambda k: host64(layer_d[k]) if k in layer_d else None  # noqa: E731
+    om = ref.Model(d_model=w.d, n_heads_q=w.hq, n_heads_kv=w.hkv, head_dim=w.dh,
+                   layers=[ref.Layer(attn_norm=g("attn_norm"), wqkv=g("wqkv"), wo=g("wo"),
+                                     ffn_norm=g("ffn_norm"), w_gate_up=None, w_down=None,
+                                     gain=g("gain"), tau=g("tau"))],
+                   final_norm=host64(model.final_norm),
+                   score_norm=host64(score["score_norm"]), score_w1=host64(score["score_w1"]),
+                   score_b1=host64(score["score_b1"]), score_w2=host64(score["score_w2"]),
+                   score_b2=host64(score["score_b2"]))
+    x = dev(synth.hidden_states(w, rng), BF16)
+    prot = synth.protect_tail(w.n, w.n_protect)
+    out, kept, scores, kv, _ = _run_gpu(w, model, x, prot)
+    assert np.array_equal(kept, ref.topk_select(scores, prot, w.k))
+    res = ref.prefill(host64(x), prot, w.k, om, -1, store=rb, kept_idx=kept)
+    assert_close(scores, res.scores, BF16, "scores")
+    assert_close(kv[0][0], res.kv[0][0], BF16, "k")
+    assert_close(kv[0][1], res.kv[0][1], BF16, "v")
+    assert_close(out, res.out, BF16, "out")
