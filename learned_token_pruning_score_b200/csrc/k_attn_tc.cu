@@ -25,6 +25,8 @@
 //              in the 128-byte-swizzled K-major layout the MMA reads.
 //   end        O / l read from TMEM, written bf16.
 // TMEM: S0 = cols [0,128), S1 = [128,256), O = [256,384) of 512.
+#include <type_traits>
+
 #include "tg_device.cuh"
 #include "tg_internal.h"
 
@@ -295,10 +297,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 //               so while one softmax warpgroup works, the tensor pipe serves
 //               the other head (ping-pong).
 //   warps 4-7   softmax of head A, warps 8-11 softmax of head B; one thread
-//               per query row. S is read from TMEM, the per-key gate bias
-//               (pre-scaled by the head's gain) comes from a shared-memory
-//               ring staged by the same warpgroup, P is written back to TMEM
+//               per query row. S is read from TMEM, P is written back to TMEM
 //               as packed bf16 over the first half of S's columns.
+// The gate bias is added by the tensor core: S = Q K^T gets one more 16-wide
+// K-step whose A row is (g_hi, g_hi, g_lo, g_lo, 0...) for the head and
+// whose B row is (b_hi, b_lo, b_hi, b_lo, 0...) for the key, where
+// g = gain_h * sqrt(dh) * tau_h and b = logsigmoid(s_j), each split into two
+// bf16 parts; the step adds (g_hi + g_lo)(b_hi + b_lo) = g b to relative
+// 2^-17 (so (S + g b) / (sqrt(dh) tau_h) carries gain_h * logsigmoid(s_j)).
+// The softmax then needs no per-key loads.
 // TMEM columns: S_A [0,128) (P_A [0,64)), S_B [128,256) (P_B [128,192)),
 //               O_A [256,384), O_B [384,512).
 // Ordering: the commit that signals S_h(j+1) is issued after O_h += P_h(j) V_j,
@@ -308,20 +315,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 namespace pair {
 
 constexpr int kThreads = 384;
-constexpr int kOffQA = 0;
-constexpr int kOffQB = kOffQA + kTile;
-constexpr int kOffK = kOffQB + kTile;        // 2 stages
-constexpr int kOffV = kOffK + 2 * kTile;     // 2 stages
-constexpr int kOffBias = kOffV + 2 * kTile;  // [2 heads][2 slots][128] fp32
-constexpr int kOffBar = kOffBias + 2 * 2 * 128 * 4;
-constexpr size_t kSmem = 1024 + kOffBar + 256;
+// Shared-memory layout. With the gate bias, its 32-byte-swizzled tiles come
+// first (an addressing slip there cannot reach past the allocation), then
+// the 128-byte-swizzled operand tiles.
+constexpr int kAugTile = 128 * 32;  // [128 rows x 16 bf16]
+template <bool kBias>
+struct Layout {
+  static constexpr int kAug = kBias ? kAugTile : 0;
+  static constexpr int kOffQAugA = 0;
+  static constexpr int kOffQAugB = kOffQAugA + kAug;
+  static constexpr int kOffKAug = kOffQAugB + kAug;      // 2 stages
+  static constexpr int kOffQA = kOffKAug + 2 * kAug;     // 0 or 16 KB: 1024-aligned
+  static constexpr int kOffQB = kOffQA + kTile;
+  static constexpr int kOffK = kOffQB + kTile;           // 2 stages
+  static constexpr int kOffV = kOffK + 2 * kTile;        // 2 stages
+  static constexpr int kOffBar = kOffV + 2 * kTile;
+  static constexpr size_t kSmem = 1024 + kOffBar + 256;
+};
 
 struct Params {
   int64_t T;
   int hq, hkv;
   int n_qtiles;
   int kv_major;  // 1: CTAs ordered KV-head-major (large T), 0: heaviest tiles first
-  const float* lsig;
   const float* gain;
   const float* tau;
   __nv_bfloat16* out;
@@ -331,7 +347,12 @@ struct Params {
 template <bool kBias>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, Params p) {
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKAug,
+                 Params p) {
+  using Lay = Layout<kBias>;
+  constexpr int kOffQAugA = Lay::kOffQAugA, kOffQAugB = Lay::kOffQAugB, kOffKAug = Lay::kOffKAug;
+  constexpr int kOffQA = Lay::kOffQA, kOffQB = Lay::kOffQB, kOffK = Lay::kOffK, kOffV = Lay::kOffV;
+  constexpr int kOffBar = Lay::kOffBar;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
@@ -344,7 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = bars + 9;    // [2 heads]
   uint64_t* p_full = bars + 11;   // [2 heads]
   uint64_t* o_full = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* qaug_full = bars + 14;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // CTA order. When all K/V fits in L2 easily, the heaviest (latest) query
@@ -367,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int g = head0 / (p.hq / p.hkv);
   const int q0 = qt * kBlk;
   const int n_kv = qt + 1;
+  constexpr uint32_t kKBytes = kTile + (kBias ? kAugTile : 0);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -379,10 +402,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[i], 128);
     }
     mbar_init(o_full, 1);
+    mbar_init(qaug_full, 256);
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    if (kBias) tma_prefetch_desc(&tmKAug);
   }
   if (warp == 2) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -402,9 +427,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = ((j >> 1) & 1) ^ 1;
       if (!mbar_wait(&k_empty[s], ph, p.err)) break;
       uint8_t* kd = smem + kOffK + s * kTile;
-      mbar_arrive_expect_tx(&k_full[s], kTile);
+      mbar_arrive_expect_tx(&k_full[s], kKBytes);
       tma_load_3d(&tmK, &k_full[s], kd, 0, g, j * kBlk);
       tma_load_3d(&tmK, &k_full[s], kd + kSub, 64, g, j * kBlk);
+      if (kBias) tma_load_2d(&tmKAug, &k_full[s], smem + kOffKAug + s * kAugTile, 0, j * kBlk);
       if (!mbar_wait(&v_empty[s], ph, p.err)) break;
       uint8_t* vd = smem + kOffV + s * kTile;
       mbar_arrive_expect_tx(&v_full[s], kTile);
@@ -424,6 +450,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_f16_ss(d, sdesc_kmajor_sw128(q_addr + off), sdesc_kmajor_sw128(k_addr + off), idesc,
                     kk > 0 ? 1u : 0u);
       }
+      if (kBias) {  // the gate-bias K-step
+        umma_f16_ss(d, sdesc_kmajor_sw32(smem_addr(smem + (h ? kOffQAugB : kOffQAugA))),
+                    sdesc_kmajor_sw32(smem_addr(smem + kOffKAug + (j & 1) * kAugTile)), idesc, 1u);
+      }
       umma_commit(&s_full[h]);
     };
     auto issue_pv = [&](int h, int j) {
@@ -438,6 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     bool ok = mbar_wait(q_full, 0, p.err) && mbar_wait(&k_full[0], 0, p.err);
+    if (kBias) ok = ok && mbar_wait(qaug_full, 0, p.err);
     if (ok) {
       tc_fence_after();
       issue_qk(0, 0);
@@ -478,27 +509,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t o_col = 256u + static_cast<uint32_t>(h * 128);
     const float tau = p.tau ? __ldg(p.tau + head) : 1.0f;
     const float scale2 = kLog2e / (sqrtf(static_cast<float>(kDh)) * tau);
-    // bias in units of S: l2 = (S + cmul * lsig) * scale2
-    const float cmul = kBias ? __ldg(p.gain + head) * sqrtf(static_cast<float>(kDh)) * tau : 0.f;
-    float* bias_ring = reinterpret_cast<float*>(smem + kOffBias) + h * 256;
-    float bnext = 0.f;
-    if (kBias) bnext = r < p.T ? __ldg(p.lsig + r) : 0.f;
+    if (kBias) {
+      // this row of the head's gate-bias A tile: (g_hi, g_hi, g_lo, g_lo, 0 ...)
+      const float gs = __ldg(p.gain + head) * sqrtf(static_cast<float>(kDh)) * tau;
+      const __nv_bfloat16 ghi = __float2bfloat16_rn(gs);
+      const __nv_bfloat16 glo = __float2bfloat16_rn(gs - __bfloat162float(ghi));
+      __nv_bfloat162 hh, ll;
+      hh.x = ghi;
+      hh.y = ghi;
+      ll.x = glo;
+      ll.y = glo;
+      uint8_t* row = smem + (h ? kOffQAugB : kOffQAugA) + r * 32;
+      const int sw = (r >> 2) & 1;  // 32-byte swizzle: 16-byte chunk c sits at c ^ sw
+      *reinterpret_cast<uint4*>(row + ((0 ^ sw) << 4)) =
+          make_uint4(*reinterpret_cast<uint32_t*>(&hh), *reinterpret_cast<uint32_t*>(&ll), 0u, 0u);
+      *reinterpret_cast<uint4*>(row + ((1 ^ sw) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+      fence_async_smem();
+      mbar_arrive(qaug_full);
+    }
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    // Every thread runs all n_kv iterations: the bias staging's named barrier
-    // has no timeout, so after a failed (timed-out) wait a warp keeps joining
-    // it and skips everything else.
-    for (int j = 0; j < n_kv; ++j) {
+    for (int j = 0; j < n_kv && ok; ++j) {
       const int kv0 = j * kBlk;
-      const float4* cb = reinterpret_cast<const float4*>(bias_ring + (j & 1) * 128);
-      if (kBias) {
-        bias_ring[(j & 1) * 128 + r] = cmul * bnext;
-        const int64_t nc = static_cast<int64_t>(kv0) + kBlk + r;
-        bnext = (j + 1 < n_kv && nc < p.T) ? __ldg(p.lsig + nc) : 0.f;
-        named_bar_sync(1 + h, 128);
-      }
-      if (!ok) continue;
-      if (!mbar_wait_warp(&s_full[h], j & 1, p.err)) { ok = false; continue; }
+      if (!mbar_wait_warp(&s_full[h], j & 1, p.err)) { ok = false; break; }
       tc_fence_after();
       float x[128];
 #pragma unroll
@@ -507,16 +540,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32_wait(tmem + lane_off + s_col + static_cast<uint32_t>(c * 32), t);
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[c * 32 + i] = t[i];
-      }
-      if (kBias) {
-#pragma unroll
-        for (int i4 = 0; i4 < 32; ++i4) {
-          const float4 b = cb[i4];
-          x[4 * i4 + 0] += b.x;
-          x[4 * i4 + 1] += b.y;
-          x[4 * i4 + 2] += b.z;
-          x[4 * i4 + 3] += b.w;
-        }
       }
       if (j == n_kv - 1) {  // diagonal tile: causal mask
 #pragma unroll
@@ -608,6 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace pair
 
+
 }  // namespace
 
 bool attn_tc_supported(const AttnArgs& a) {
@@ -648,17 +672,24 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
     // K and V of all KV heads: above ~48 MB the working set would not stay
     // in the 126 MB L2 across a wave of CTAs spread over every head.
     pp.kv_major = (double(a.T) * a.hkv * kDh * 4.0 > 48.0e6) ? 1 : 0;
-    pp.lsig = p.lsig;
     pp.gain = p.gain;
     pp.tau = p.tau;
     pp.out = p.out;
     pp.err = p.err;
     const bool bias = a.lsig != nullptr && a.gain != nullptr;
+    CUtensorMap tka;
+    if (bias) {
+      if (a.kaug == nullptr || !make_tmap_2d_bf16_sw32(&tka, a.kaug, a.T, 16, kBlk))
+        return cudaErrorInvalidValue;
+    } else {
+      tka = tk;  // not read
+    }
     auto kern = bias ? pair::attn_tc_pair<true> : pair::attn_tc_pair<false>;
-    cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(kern), int(pair::kSmem));
+    const size_t smem = bias ? pair::Layout<true>::kSmem : pair::Layout<false>::kSmem;
+    cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(kern), int(smem));
     if (err != cudaSuccess) return err;
     const unsigned grid = static_cast<unsigned>(p.n_qtiles) * static_cast<unsigned>(a.hq / 2);
-    kern<<<grid, pair::kThreads, pair::kSmem, st>>>(tq, tk, tv, pp);
+    kern<<<grid, pair::kThreads, smem, st>>>(tq, tk, tv, tka, pp);
     return cudaGetLastError();
   }
   cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(attn_tc), int(kSmem));

@@ -216,6 +216,21 @@ __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int64_t T, in
   cs[idx] = make_float2(cv, sv);
 }
 
+// Gate-bias rows for the attention's extra K-step (see launch_bias_aug).
+__global__ void bias_aug_kernel(const float* __restrict__ lsig, int64_t T, uint4* __restrict__ kaug) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const float b = __ldg(lsig + t);
+  const __nv_bfloat16 hi = __float2bfloat16_rn(b);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(b - __bfloat162float(hi));
+  __nv_bfloat162 hl;
+  hl.x = hi;
+  hl.y = lo;
+  const uint32_t w = *reinterpret_cast<uint32_t*>(&hl);
+  kaug[2 * t] = make_uint4(w, w, 0u, 0u);
+  kaug[2 * t + 1] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // ---------------------------------------------------------------- V transpose
 // One CTA per (64-token tile, KV head): vT[g][e][t] = v[t][g][e] (zero for
 // t >= T), so that the attention's P.V product reads V K-major. Also copies
@@ -345,6 +360,13 @@ cudaError_t launch_rope_table(const int32_t* pos, int64_t T, int dh, float rope_
   if (total <= 0) return cudaSuccess;
   rope_table_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(pos, T, half, dh,
                                                                                 rope_base, cs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bias_aug(const float* lsig, int64_t T, void* kaug, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  bias_aug_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, st>>>(lsig, T,
+                                                                         static_cast<uint4*>(kaug));
   return cudaGetLastError();
 }
 

@@ -142,6 +142,7 @@ struct AttnPlan {
   void* k_rot = nullptr;  // [k, hkv, dh]
   void* vT = nullptr;     // bf16: [hkv, dh, t_pad]
   float* lsig = nullptr;  // [k]
+  void* kaug = nullptr;   // bf16 [k, 16] gate-bias rows (tensor-core path)
   int64_t t_pad = 0;
   size_t bytes = 0;
   AttnPlan(void* ws, int64_t k, int hq, int hkv, int dh, tg_dtype dt, bool need_k) {
@@ -152,6 +153,7 @@ struct AttnPlan {
     if (need_k) k_rot = a.carve(size_t(k) * hkv * dh * e);
     if (dt == TG_BF16) vT = a.carve(size_t(hkv) * dh * t_pad * e);
     lsig = static_cast<float*>(a.carve(size_t(k) * 4 + 16));
+    if (dt == TG_BF16) kaug = a.carve(size_t(k) * 32);
     bytes = a.used;
   }
 };
@@ -169,6 +171,7 @@ struct PrefillPlan {
   int32_t* pos_k = nullptr;
   float* s_k = nullptr;
   float* lsig_k = nullptr;
+  void* kaug_k = nullptr;  // bf16 [k, 16] gate-bias rows of the kept tokens
   void* sel_ws = nullptr;
   float2* cs_n = nullptr;  // [n][dh/2] cos/sin of positions 0..n-1 (dense stage)
   float2* cs_k = nullptr;  // [k][dh/2] cos/sin of the kept positions
@@ -193,6 +196,7 @@ struct PrefillPlan {
     pos_k = static_cast<int32_t*>(a.carve(size_t(k) * 4));
     s_k = static_cast<float*>(a.carve(size_t(k) * 4));
     lsig_k = static_cast<float*>(a.carve(size_t(k) * 4));
+    if (m.dtype == TG_BF16) kaug_k = a.carve(size_t(k) * 32);
     sel_ws = a.carve(select_ws_bytes(n));
     cs_n = static_cast<float2*>(a.carve(size_t(n) * (dh / 2) * sizeof(float2)));
     cs_k = static_cast<float2*>(a.carve(size_t(k) * (dh / 2) * sizeof(float2)));
@@ -286,8 +290,9 @@ cudaError_t run_score(const void* x, int64_t rows, int d, int f, const float* no
 
 // Attention over prepared (rotated) q/k and prepared V (bf16: V^T [hkv, dh, t_pad]).
 cudaError_t attn_core(const AttnPlan& plan, const void* k_rot, const void* v, int64_t v_stride,
-                      const float* lsig, const float* gain, const float* tau, int64_t rows, int hq,
-                      int hkv, int dh, tg_dtype dt, void* out, cudaStream_t st) {
+                      const float* lsig, const void* kaug, const float* gain, const float* tau,
+                      int64_t rows, int hq, int hkv, int dh, tg_dtype dt, void* out,
+                      cudaStream_t st) {
   const size_t es = elem_size(dt);
   const double attn_flops = 4.0 * dh * hq * double(rows) * double(rows + 1) / 2.0;
   const double attn_bytes = double(rows) * (2 * hq + 2 * hkv) * dh * es;
@@ -295,6 +300,7 @@ cudaError_t attn_core(const AttnPlan& plan, const void* k_rot, const void* v, in
   a.q = plan.q_rot;
   a.k = k_rot;
   a.lsig = lsig;
+  a.kaug = kaug;
   a.gain = gain; a.tau = tau;
   a.T = rows; a.hq = hq; a.hkv = hkv; a.dh = dh;
   a.out = out;
@@ -339,8 +345,14 @@ cudaError_t run_attention(const void* q, int64_t q_stride, const void* kk, int64
   cudaError_t e = traced(TG_K_ROPE_PREP, rows, 0.0, prep_bytes, st,
                          [&] { return launch_rope_prep(r, st); });
   if (e != cudaSuccess) return e;
-  return attn_core(plan, r.k_out, v, v_stride, (s || lsig_ready) ? (lsig_ready ? lsig_ready : plan.lsig) : nullptr,
-                   gain, tau, rows, hq, hkv, dh, dt, out, st);
+  const float* lsig = (s || lsig_ready) ? (lsig_ready ? lsig_ready : plan.lsig) : nullptr;
+  if (lsig && dt == TG_BF16) {
+    e = traced(TG_K_ROPE_PREP, rows, 0.0, 36.0 * rows, st,
+               [&] { return launch_bias_aug(lsig, rows, plan.kaug, st); });
+    if (e != cudaSuccess) return e;
+  }
+  return attn_core(plan, r.k_out, v, v_stride, lsig, dt == TG_BF16 ? plan.kaug : nullptr, gain,
+                   tau, rows, hq, hkv, dh, dt, out, st);
 }
 
 // ---- the decoder-layer pieces used by tg_prefill
@@ -351,8 +363,9 @@ struct Dims {
 
 cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
                                const PrefillPlan& P, void* h, int64_t rows, const int32_t* pos,
-                               const float2* cs, const float* lsig, const float* gain,
-                               const float* tau, const tg_kv* kv, cudaStream_t st) {
+                               const float2* cs, const float* lsig, const void* kaug,
+                               const float* gain, const float* tau, const tg_kv* kv,
+                               cudaStream_t st) {
   const tg_dtype dt = m.dtype;
   const size_t e = elem_size(dt);
   cudaError_t err = rmsnorm(h, lw.attn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
@@ -366,8 +379,8 @@ cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims
     // fused: projection + qk-norm + RoPE + V^T in the GEMM epilogue
     err = gemm(gq, dt, st);
     if (err != cudaSuccess) return err;
-    err = attn_core(P.attn, k_dst, nullptr, 0, lsig, gain, tau, rows, D.hq, D.hkv, D.dh, dt,
-                    P.attn_o, st);
+    err = attn_core(P.attn, k_dst, nullptr, 0, lsig, kaug, gain, tau, rows, D.hq, D.hkv, D.dh,
+                    dt, P.attn_o, st);
   } else {
     err = gemm(gemm_args(P.y, D.d, lw.wqkv, D.d, P.qkv, D.qkv, rows, D.qkv, D.d, EPI_STORE), dt,
                st);
@@ -605,14 +618,14 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
   for (int l = 0; l < gate_layer; ++l) {
     LayerTag tag(l);
     TG_TRY(attention_sublayer(m, m.layers[l], D, P, P.h, n, nullptr, P.cs_n, nullptr, nullptr,
-                              nullptr, kv ? &kv[l] : nullptr, st));
+                              nullptr, nullptr, kv ? &kv[l] : nullptr, st));
     TG_TRY(ffn_sublayer(m, m.layers[l], D, P, P.h, n, st));
     if (hidden && hidden[l]) TG_TRY(copy_rows(hidden[l], P.h, size_t(n) * D.d * e, n, st));
   }
   if (gate_layer >= 0) {
     LayerTag tag(gate_layer);
     TG_TRY(attention_sublayer(m, m.layers[gate_layer], D, P, P.h, n, nullptr, P.cs_n, nullptr,
-                              nullptr, nullptr, kv ? &kv[gate_layer] : nullptr, st));
+                              nullptr, nullptr, nullptr, kv ? &kv[gate_layer] : nullptr, st));
   }
   // Stage 2: score the post-attention residual, select, compact.
   TG_TRY(run_score(P.h, n, D.d, m.d_score, m.score_norm, m.norm_eps, m.score_w1, m.score_b1,
@@ -620,10 +633,14 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
   TG_TRY(select_topk(sc, protect, n, k, kept_idx, P.sel_ws, st));
   TG_TRY(compact(P.h, nullptr, sc, kept_idx, n, k, static_cast<int>(D.d * e), P.hk, P.pos_k, P.s_k,
                  P.lsig_k, st));
-  if (tables)
+  if (tables) {
     TG_TRY(traced(TG_K_ROPE_TABLE, k, 0.0, cs_bytes * k + 4.0 * k, st, [&] {
       return launch_rope_table(P.pos_k, k, D.dh, m.rope_base, P.cs_k, st);
     }));
+    // gate-bias rows of the kept tokens, shared by every gated layer
+    TG_TRY(traced(TG_K_ROPE_TABLE, k, 0.0, 36.0 * k, st,
+                  [&] { return launch_bias_aug(P.lsig_k, k, P.kaug_k, st); }));
+  }
   // Stage 3: the gate layer's FFN and the layers above, over the k kept rows.
   if (gate_layer >= 0) {
     LayerTag tag(gate_layer);
@@ -634,8 +651,8 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
   for (int l = gate_layer + 1; l < m.n_layers; ++l) {
     LayerTag tag(l);
     const tg_layer& L = m.layers[l];
-    TG_TRY(attention_sublayer(m, L, D, P, P.hk, k, P.pos_k, P.cs_k, P.lsig_k, L.gain, L.tau,
-                              kv ? &kv[l] : nullptr, st));
+    TG_TRY(attention_sublayer(m, L, D, P, P.hk, k, P.pos_k, P.cs_k, P.lsig_k, P.kaug_k, L.gain,
+                              L.tau, kv ? &kv[l] : nullptr, st));
     TG_TRY(ffn_sublayer(m, L, D, P, P.hk, k, st));
     if (hidden && hidden[l]) TG_TRY(copy_rows(hidden[l], P.hk, size_t(k) * D.d * e, k, st));
   }

@@ -274,6 +274,19 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t addr) {
   return d;
 }
 
+// Shared-memory matrix descriptor for a K-major tile with the 32-byte
+// swizzle: rows of 32 bytes (16 bf16, one MMA K-step), 8-row groups 256
+// bytes apart (tile base 256-aligned).
+__device__ __forceinline__ uint64_t sdesc_kmajor_sw32(uint32_t addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);          // start address
+  d |= static_cast<uint64_t>(1u) << 16;                        // leading byte offset (16 B)
+  d |= static_cast<uint64_t>(256u >> 4) << 32;                 // stride byte offset (256 B)
+  d |= static_cast<uint64_t>(1u) << 46;                        // descriptor version (sm_100)
+  d |= static_cast<uint64_t>(6u) << 61;                        // layout: 32-byte swizzle
+  return d;
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B (both
 // K-major), fp32 accumulator, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {

@@ -73,6 +73,11 @@ cudaError_t launch_rope_prep(const RopePrepArgs& a, cudaStream_t st);
 cudaError_t launch_rope_table(const int32_t* pos, int64_t T, int dh, float rope_base, float2* cs,
                               cudaStream_t st);
 
+// Gate-bias rows for the attention's extra K-step: kaug[t] = (b_hi, b_lo,
+// b_hi, b_lo, 0 x 12) in bf16 with b = lsig[t], b_hi = bf16(b),
+// b_lo = bf16(b - b_hi).
+cudaError_t launch_bias_aug(const float* lsig, int64_t T, void* kaug, cudaStream_t st);
+
 // fp32 helpers used by the SIMT path
 cudaError_t launch_swiglu_f32(const float* gu, int64_t rows, int inter, float* h, cudaStream_t st);
 cudaError_t launch_score_dot_f32(const float* hpre, int64_t rows, int f, const float* b1,
@@ -109,6 +114,7 @@ struct AttnArgs {
   const void* q; const void* k; const void* v;  // v: bf16 -> vT [hkv, dh, t_pad]; fp32 -> [T,hkv,dh]
   int64_t t_pad;  // bf16: padded token count of vT; fp32: row stride of v in elements (0 = hkv*dh)
   const float* lsig; const float* gain; const float* tau;
+  const void* kaug;  // bf16 [T, 16] gate-bias rows (launch_bias_aug of lsig), needed with lsig
   int64_t T; int hq, hkv, dh;
   void* out;                                    // [T, hq, dh]
 };
@@ -121,6 +127,10 @@ cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t st); // fp32 SI
 // box [box_rows, 64 cols], 128-byte swizzle. Returns false on failure.
 bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
                        int box_rows);
+// 2-D bf16 tensor map of 16-column rows (row stride ld elements), box
+// [box_rows, 16], 32-byte swizzle: one MMA K-step per row.
+bool make_tmap_2d_bf16_sw32(CUtensorMap* m, const void* base, int64_t rows, int64_t ld,
+                            int box_rows);
 // 3-D bf16 tensor map over dims (x fastest): sizes {d0, d1, d2}, byte strides
 // {s1, s2} of dims 1 and 2, box {64, b1, b2}, 128-byte swizzle.
 bool make_tmap_3d_bf16(CUtensorMap* m, const void* base, int64_t d0, int64_t d1, int64_t d2,
