@@ -59,14 +59,14 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    """nvidia-smi sampled every 100 ms while the timed region runs."""
 
     def __init__(self, gpu_index: int):
         self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={SMI_FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=self.file, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -429,6 +429,7 @@ def run_ours(args, rank, world, local_rank):
             tg.tg_prefill(mdl, x, prot, kk, w.gate_layer, out=o, kept_idx=ki, kv=kvb, ws=wsz)
             torch.cuda.synchronize()
             ms = []
+            tg.tg_trace_start(1 << 14)
             for _ in range(reps):
                 flush.zero_()
                 a = torch.cuda.Event(enable_timing=True)
@@ -438,20 +439,30 @@ def run_ours(args, rank, world, local_rank):
                 b.record(stream)
                 torch.cuda.synchronize()
                 ms.append(a.elapsed_time(b))
+            tr = tg.tg_trace_stop()
             mem = torch.cuda.max_memory_allocated(device)
             del o, ki, wsz, kvb
-            return statistics.median(ms), mem
+            att = {}
+            for name, sel in (("gated", lambda r: r["layer"] > w.gate_layer),
+                              ("dense", lambda r: r["layer"] <= w.gate_layer)):
+                rs = [r for r in tr if r["kernel"] == "attention_tc" and sel(r)]
+                if rs:
+                    tf = sum(r["flops"] for r in rs) / (sum(r["ms"] for r in rs) / 1e3) / 1e12
+                    att[f"attn_{name}_tflops"] = tf
+                    att[f"attn_{name}_frac_of_sustained_peak"] = tf / pk["bf16_sustained"]
+            return statistics.median(ms), mem, att
 
         del ws, kv
         torch.cuda.empty_cache()
         for kk in synth.PREFILL_32K_BUDGETS:
-            t_ms, mem = ttft(model, kk)
+            t_ms, mem, att = ttft(model, kk)
             extras[f"gated_k{kk}"] = {"ttft_ms": t_ms, "tokens_per_s": w.n / (t_ms / 1e3),
                                       "tflop": workload_flops(w, kk) / 1e12,
-                                      "peak_mem_gb": mem / 1e9}
-        t_ms, mem = ttft(dense_model(tg, model), w.n)
+                                      "peak_mem_gb": mem / 1e9, **att}
+        t_ms, mem, att = ttft(dense_model(tg, model), w.n)
         extras["dense"] = {"ttft_ms": t_ms, "tokens_per_s": w.n / (t_ms / 1e3),
-                           "tflop": workload_flops(w, w.n) / 1e12, "peak_mem_gb": mem / 1e9}
+                           "tflop": workload_flops(w, w.n) / 1e12, "peak_mem_gb": mem / 1e9,
+                           **att}
         for kk in synth.PREFILL_32K_BUDGETS:
             g = extras[f"gated_k{kk}"]
             g["ttft_speedup_vs_dense"] = extras["dense"]["ttft_ms"] / g["ttft_ms"]
@@ -644,9 +655,9 @@ def run_case(args):
         kk = torch.randn(t, w.hkv, w.dh, device=device, dtype=torch.bfloat16)
         v = torch.randn(t, w.hkv, w.dh, device=device, dtype=torch.bfloat16)
         pos = torch.arange(t, dtype=torch.int32, device=device)
-        s = torch.randn(t, device=device)
-        gain = torch.rand(w.hq, device=device) * 2
-        tau = torch.rand(w.hq, device=device) + 0.5
+        s = None if args.no_bias else torch.randn(t, device=device)
+        gain = None if args.no_bias else torch.rand(w.hq, device=device) * 2
+        tau = None if args.no_bias else torch.rand(w.hq, device=device) + 0.5
         out = torch.empty_like(q)
         ws = torch.empty(tg.tg_workspace_size(tg.TG_OP_GATED_ATTN, k=t, n_heads_q=w.hq,
                                               n_heads_kv=w.hkv, head_dim=w.dh),
@@ -671,7 +682,7 @@ def run_case(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--budget", type=int, default=HEADLINE_K)
@@ -683,6 +694,8 @@ def main():
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--case", choices=["attn", "layer", "gemm"], default=None)
     ap.add_argument("--rows", type=int, default=32768)
+    ap.add_argument("--no-bias", action="store_true",
+                    help="attn case: plain causal attention (as the layers below the gate)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
     rank = int(os.environ.get("RANK", "0"))
