@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __nv_bfloat16* dst =
                 is_q ? p.q_out + (row * p.hq + hg) * 128
                      : p.k_out + (row * p.hkv + (hg - p.hq)) * 128;
-            const float2* cs = p.rope_cs + row * 64;
+            const float2* cs = p.rope_cs + row;  // frequency-major: entry i at cs[i * M]
 #pragma unroll 1
             for (int c = 0; c < 2; ++c) {
               float lo[32], hi[32];
@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     a *= __ldg(nw + pi);
                     b *= __ldg(nw + pi + 64);
                   }
-                  const float2 t = __ldg(cs + pi);
+                  const float2 t = __ldg(cs + static_cast<int64_t>(pi) * p.M);
                   lo[i] = a * t.x - b * t.y;
                   hi[i] = b * t.x + a * t.y;
                 }

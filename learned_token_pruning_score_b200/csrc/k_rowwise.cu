@@ -199,13 +199,15 @@ __global__ void __launch_bounds__(128) rope_qk(RopePrepArgs a) {
 }
 
 // cos/sin of every (position, frequency) pair, built once per set of
-// positions and read by the QKV GEMM epilogue of every layer.
+// positions and read by the QKV GEMM epilogue of every layer. Frequency-major
+// ([half][T]): the epilogue's threads hold consecutive rows, so a warp reads
+// 32 consecutive entries of one frequency.
 __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int64_t T, int half, int dh,
                                   float rope_base, float2* __restrict__ cs) {
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= T * half) return;
-  const int64_t t = idx / half;
-  const int i = static_cast<int>(idx % half);
+  const int i = static_cast<int>(idx / T);
+  const int64_t t = idx % T;
   const int p = pos ? __ldg(pos + t) : static_cast<int>(t);
   const double theta = exp2(-(2.0 * i / dh) * log2(static_cast<double>(rope_base)));
   const double ang = static_cast<double>(p) * theta;

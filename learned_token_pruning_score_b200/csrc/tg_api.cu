@@ -173,8 +173,8 @@ struct PrefillPlan {
   float* lsig_k = nullptr;
   void* kaug_k = nullptr;  // bf16 [k, 16] gate-bias rows of the kept tokens
   void* sel_ws = nullptr;
-  float2* cs_n = nullptr;  // [n][dh/2] cos/sin of positions 0..n-1 (dense stage)
-  float2* cs_k = nullptr;  // [k][dh/2] cos/sin of the kept positions
+  float2* cs_n = nullptr;  // [dh/2][n] cos/sin of positions 0..n-1 (dense stage)
+  float2* cs_k = nullptr;  // [dh/2][k] cos/sin of the kept positions
   AttnPlan attn;           // sized for n rows, reused by every layer
   size_t bytes = 0;
   PrefillPlan(void* ws, const tg_model& m, int64_t n, int64_t k)

@@ -69,7 +69,8 @@ struct RopePrepArgs {
   const float* s; float* lsig_out;
 };
 cudaError_t launch_rope_prep(const RopePrepArgs& a, cudaStream_t st);
-// cs[t][i] = (cos, sin)(pos[t] * base^(-2i/dh)), i < dh/2; pos null = row index.
+// cs[i][t] = (cos, sin)(pos[t] * base^(-2i/dh)), i < dh/2 (frequency-major);
+// pos null = row index.
 cudaError_t launch_rope_table(const int32_t* pos, int64_t T, int dh, float rope_base, float2* cs,
                               cudaStream_t st);
 
@@ -96,7 +97,7 @@ struct GemmArgs {
   const float* b1; const float* w2; const float* b2; float* scores;  // SCORE
   // QKV (head dim 128): columns [0, hq*128) are q heads, then hkv k heads,
   // then hkv v heads. Writes q_out [M, hq, 128] and k_out [M, hkv, 128]
-  // (optional per-head RMSNorm, then RoPE from rope_cs [M][64] (cos, sin)),
+  // (optional per-head RMSNorm, then RoPE from rope_cs [64][M] (cos, sin)),
   // vT_out [hkv, 128, t_pad] and, if set, v_out [M, hkv, 128].
   int hq, hkv;
   const float2* rope_cs; const float* q_norm; const float* k_norm; float eps;
