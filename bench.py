@@ -249,6 +249,25 @@ def run_reference(args, rank, world):
     return 0
 
 
+def max_over_ranks(ms: float, dist=None, device=None) -> float:
+    """The slowest rank's device time. Every rank calls this at the same
+    point of the run (one all-reduce, MAX); without a process group it
+    returns `ms` unchanged."""
+    if dist is None:
+        return ms
+    import torch
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replicas_throughput(tokens_per_step: int, steps: int, world: int, total_ms: float) -> float:
+    """Whole-job tokens/s of `world` independent replicas, each running
+    `steps` steps of `tokens_per_step` tokens, over the slowest rank's time."""
+    return world * tokens_per_step * steps / (total_ms / 1000.0)
+
+
 # ----------------------------------------------------------------- our arm
 
 
@@ -312,13 +331,9 @@ def run_ours(args, rank, world, local_rank):
     wall = time.perf_counter() - t_wall
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
-    total_ms = sum(step_ms)
-    if dist is not None:
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, device)
     ms_per_step = total_ms / args.steps
-    value = world * w.n * args.steps / (total_ms / 1000.0)
+    value = replicas_throughput(w.n, args.steps, world, total_ms)
     err_word = tg.tg_device_error()
 
     # ---- per-kernel breakdown from the trace (timed steps only)
@@ -402,14 +417,10 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([e_ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
         h2d = x.numel() * x.element_size() + prot.numel()
         d2h = out.numel() * out.element_size() + kept.numel() * 4
-        e2e = {"value": world * w.n * args.steps / (e_ms / 1000.0), "unit": UNIT,
+        e2e = {"value": replicas_throughput(w.n, args.steps, world, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / args.steps}
 
