@@ -86,6 +86,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q0 = qt * kBlk;
   const int n_kv = qt + 1;  // causal: KV tiles 0..qt
 
+  pdl_trigger();
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
@@ -105,6 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // q, k, V^T and the bias rows come from the previous kernels
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------- TMA producer
@@ -391,6 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_kv = qt + 1;
   constexpr uint32_t kKBytes = kTile + (kBias ? kAugTile : 0);
 
+  pdl_trigger();
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
@@ -414,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // q, k, V^T and the bias rows come from the previous kernels
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------- TMA producer
@@ -689,14 +693,12 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
     cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(kern), int(smem));
     if (err != cudaSuccess) return err;
     const unsigned grid = static_cast<unsigned>(p.n_qtiles) * static_cast<unsigned>(a.hq / 2);
-    kern<<<grid, pair::kThreads, smem, st>>>(tq, tk, tv, tka, pp);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(pair::kThreads), smem, st, tq, tk, tv, tka, pp);
   }
   cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(attn_tc), int(kSmem));
   if (err != cudaSuccess) return err;
   const unsigned grid = static_cast<unsigned>(p.n_qtiles) * static_cast<unsigned>(a.hq);
-  attn_tc<<<grid, kThreads, kSmem, st>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  return launch_pdl(attn_tc, dim3(grid), dim3(kThreads), kSmem, st, tq, tk, tv, p);
 }
 
 }  // namespace tg

@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(kWarps * 32) compact_rows(
     const float* __restrict__ scores, const int32_t* __restrict__ idx, int64_t n, int64_t k,
     int vec_per_row, uint4* __restrict__ x_out, int32_t* __restrict__ pos_out,
     float* __restrict__ s_out, float* __restrict__ lsig_out, unsigned int* err) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
   if (row >= k) return;
@@ -57,9 +59,7 @@ cudaError_t launch_compact(const void* x, const int32_t* pos_in, const float* sc
                            cudaStream_t st) {
   if (k <= 0) return cudaSuccess;
   const int64_t blocks = (k + kWarps - 1) / kWarps;
-  compact_rows<<<static_cast<unsigned>(blocks), kWarps * 32, 0, st>>>(
-      static_cast<const uint4*>(x), pos_in, scores, kept_idx, n, k, row_bytes / 16,
-      static_cast<uint4*>(x_out), pos_out, scores_out, lsig_out, device_error_word());
+  TG_CUDA_TRY(launch_pdl(compact_rows, dim3(static_cast<unsigned>(blocks)), dim3(kWarps * 32), 0, st, static_cast<const uint4*>(x), pos_in, scores, kept_idx, n, k, row_bytes / 16, static_cast<uint4*>(x_out), pos_out, scores_out, lsig_out, device_error_word()));
   return cudaGetLastError();
 }
 

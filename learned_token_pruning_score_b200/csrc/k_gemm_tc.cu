@@ -6,36 +6,37 @@
 // QKV, the output projection, SwiGLU gate/up and down. Epilogues fused into
 // the TMEM read-out: plain store, residual add (x + W.o), SwiGLU
 // (SiLU(gate) * up, with gate and up tiles side by side in one 256-wide
-// accumulator), and the scorer's tail s = w2 . SiLU(h + b1) + b2 (all F <= 256
+// accumulator), the scorer's tail s = w2 . SiLU(h + b1) + b2 (all F <= 256
 // hidden units of a row sit in one accumulator row, so the dot is
-// thread-local).
+// thread-local), and QKV (qk-norm, RoPE, V transposed).
 //
-// Structure: persistent CTAs (one per SM), 8 warps.
-//   warp 0    TMA producer: A tile [128 x 64] + B tile [BN x 64] per stage,
-//             128-byte swizzle, STAGES-deep ring of full/empty mbarriers.
-//   warp 1    MMA issuer: one thread issues tcgen05.mma (M=128, N=BN, K=16)
-//             x4 per stage into a TMEM accumulator, commits to free the stage.
-//   warp 2    TMEM allocation (2 x BN columns: double-buffered accumulator).
-//   warps 4-7 epilogue: tcgen05.ld of their 32-lane quarter, fused op, store.
+// Structure: persistent clusters of two CTAs on two SMs (a CTA pair), 8
+// warps each. The pair computes 256 x 256 output tiles with one
+// tcgen05.mma.cta_group::2 (M=256, N=256, K=16) per K-step: each CTA stages
+// its 128 rows of A and its 128 rows of B, so per SM a K-step reads 32 KB of
+// operands from shared memory (a one-SM 128 x 256 tile reads 48 KB) and the
+// L2 traffic per FLOP is two thirds of the one-SM kernel's.
+//   warp 0    (both)   TMA producer, 6-stage ring of 32 KB stages, 128-byte
+//                      swizzle; the bytes of both CTAs count on rank 0's
+//                      full barrier.
+//   warp 1    (rank 0) MMA issuer: 4 MMAs per stage into a TMEM accumulator,
+//                      then commits that free the stage in both CTAs.
+//   warp 2    (both)   TMEM allocation: 2 x 256 columns (double-buffered
+//                      accumulator, cta_group::2).
+//   warps 4-7 (both)   epilogue: tcgen05.ld of their 32-lane quarter of the
+//                      CTA's 128 rows, fused op, store; then arrive on rank
+//                      0's accumulator-empty barrier.
 // The epilogue of tile t overlaps the MMAs of tile t+1.
+#include <atomic>
+
 #include "tg_device.cuh"
 #include "tg_internal.h"
 
 namespace tg {
 namespace {
 
-constexpr int kBM = 128, kBK = 64;
+constexpr int kBK = 64;
 constexpr int kThreads = 256;
-
-template <int kBN>
-struct Cfg {
-  static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = kBN * kBK * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = kBN == 256 ? 4 : 6;
-  static constexpr int kTmemCols = 2 * kBN;
-  static constexpr size_t kSmem = 1024 /*align slack*/ + size_t(kStages) * kStageBytes + 256;
-};
 
 struct EpiParams {
   int64_t M;
@@ -91,13 +92,145 @@ __device__ __forceinline__ void add32_bf16(const __nv_bfloat16* src, float (&v)[
   }
 }
 
+// The fused epilogue of one accumulator tile, run by one epilogue warp for
+// its 32 rows: this thread owns accumulator row `row` (global index), whose
+// kBN fp32 columns start at TMEM address `t_row`; `nb` is the tile's column
+// block.
 template <int kBN, int kEpi>
-__global__ void __launch_bounds__(kThreads, 1)
+__device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, uint32_t t_row,
+                                              int nb) {
+  const bool row_ok = row < p.M;
+  if constexpr (kEpi == EPI_STORE || kEpi == EPI_RESIDUAL) {
+#pragma unroll 1
+    for (int c = 0; c < kBN / 32; ++c) {
+      float v[32];
+      tmem_ld32_wait(t_row + c * 32, v);
+      const int col = nb * kBN + c * 32;
+      if (row_ok && col < p.N) {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) + row * p.ldc + col;
+        if (kEpi == EPI_RESIDUAL)
+          add32_bf16(static_cast<const __nv_bfloat16*>(p.R) + row * p.ldr + col, v);
+        store32_bf16(dst, v);
+      }
+    }
+  } else if constexpr (kEpi == EPI_SWIGLU) {
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float g[32], u[32];
+      tmem_ld32_wait(t_row + c * 32, g);
+      tmem_ld32_wait(t_row + 128 + c * 32, u);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) g[j] = silu_f(g[j]) * u[j];
+      if (row_ok)
+        store32_bf16(static_cast<__nv_bfloat16*>(p.C) + row * p.ldc + nb * 128 + c * 32, g);
+    }
+  } else if constexpr (kEpi == EPI_QKV) {
+    // Two whole heads per tile (head dim 128). The accumulator is rounded
+    // to bf16 first (the stored-q/k/v value), then q/k get the optional
+    // per-head RMSNorm and RoPE; v is written transposed (and as cache).
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {
+      const int hg = nb * 2 + hh;  // head index across the q | k | v columns
+      const uint32_t t_head = t_row + static_cast<uint32_t>(hh * 128);
+      if (hg < p.hq + p.hkv) {
+        const bool is_q = hg < p.hq;
+        const float* nw = is_q ? p.q_norm : p.k_norm;
+        float rstd = 1.0f;
+        if (nw != nullptr) {
+          float ss = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float v[32];
+            tmem_ld32_wait(t_head + c * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float f = round_bf16_f(v[i]);
+              ss = fmaf(f, f, ss);
+            }
+          }
+          rstd = rsqrtf(ss * (1.0f / 128.0f) + p.eps);
+        }
+        __nv_bfloat16* dst =
+            is_q ? p.q_out + (row * p.hq + hg) * 128
+                 : p.k_out + (row * p.hkv + (hg - p.hq)) * 128;
+        const float2* cs = p.rope_cs + row;  // frequency-major: entry i at cs[i * M]
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          float lo[32], hi[32];
+          tmem_ld32_wait(t_head + c * 32, lo);
+          tmem_ld32_wait(t_head + 64 + c * 32, hi);
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int pi = c * 32 + i;
+              float a = round_bf16_f(lo[i]) * rstd;
+              float b = round_bf16_f(hi[i]) * rstd;
+              if (nw != nullptr) {
+                a *= __ldg(nw + pi);
+                b *= __ldg(nw + pi + 64);
+              }
+              const float2 t = __ldg(cs + static_cast<int64_t>(pi) * p.M);
+              lo[i] = a * t.x - b * t.y;
+              hi[i] = b * t.x + a * t.y;
+            }
+            store32_bf16(dst + c * 32, lo);
+            store32_bf16(dst + 64 + c * 32, hi);
+          }
+        }
+      } else {
+        const int g = hg - p.hq - p.hkv;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32_wait(t_head + c * 32, v);
+          if (row_ok) {
+            if (p.v_out) store32_bf16(p.v_out + (row * p.hkv + g) * 128 + c * 32, v);
+            __nv_bfloat16* vt = p.vT_out + (static_cast<int64_t>(g) * 128 + c * 32) * p.t_pad + row;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) vt[static_cast<int64_t>(i) * p.t_pad] = __float2bfloat16_rn(v[i]);
+          }
+        }
+      }
+    }
+  } else {  // EPI_SCORE
+    float acc = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < kBN / 32; ++c) {
+      float v[32];
+      tmem_ld32_wait(t_row + c * 32, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int f = c * 32 + j;
+        if (f < p.N) {
+          const float h = v[j] + (p.b1 ? __ldg(p.b1 + f) : 0.f);
+          acc = fmaf(__ldg(p.w2 + f), silu_f(h), acc);
+        }
+      }
+    }
+    if (row_ok) p.scores[row] = acc + (p.b2 ? __ldg(p.b2) : 0.f);
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+// SWIGLU: rank 0 stages the 128 gate rows of B, rank 1 the matching 128 up
+// rows, so accumulator columns [0, 128) hold gate and [128, 256) hold up.
+struct PairCfg {
+  static constexpr int kHalfBytes = 128 * kBK * 2;       // 128 rows x 64 bf16
+  static constexpr int kStageBytes = 2 * kHalfBytes;     // A half + B half
+  static constexpr int kStages = 6;
+  static constexpr int kTmemCols = 512;                  // 2 x 256 fp32 accumulators
+  static constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes + 256;
+};
+
+template <int kEpi>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-            EpiParams p) {
-  using C = Cfg<kBN>;
+                 EpiParams p) {
+  using C = PairCfg;
+  constexpr int kBN = 256;
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte aligned base for the swizzled tiles.
+  // 1024-byte aligned base for the swizzled tiles; the offset is the same in
+  // both CTAs (same kernel, same static layout).
   const uint32_t raw_addr = smem_addr(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
   uint8_t* tiles = smem;
@@ -109,58 +242,67 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&full[s], 1);   // rank 0: its producer's arrive + both CTAs' bytes
+      mbar_init(&empty[s], 1);  // one commit from rank 0's MMA thread
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], 8);  // rank 0: 4 epilogue warps x 2 CTAs
     }
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
-  if (warp == 2) tmem_alloc(tmem_slot, C::kTmemCols);
+  if (warp == 2) tmem_alloc_pair(tmem_slot, C::kTmemCols);
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the previous kernel's outputs (A, the residual) are complete
 
   const int num_tiles = p.tiles_m * p.tiles_n;
   const int num_kb = (p.K + kBK - 1) / kBK;
+  const int pair = static_cast<int>(blockIdx.x >> 1), n_pairs = static_cast<int>(gridDim.x >> 1);
 
   if (warp == 0 && lane == 0) {
-    // ---------------------------------------------------------- producer
+    // ---------------------------------------------------------- producers
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
       const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
-      const int b_row0 = kEpi == EPI_SWIGLU ? nb * 128 : nb * kBN;
+      const int a_row = mb * 256 + static_cast<int>(rank) * 128;
+      const int b_row = kEpi == EPI_SWIGLU ? (rank ? p.inter : 0) + nb * 128
+                                           : nb * 256 + static_cast<int>(rank) * 128;
       for (int kb = 0; kb < num_kb; ++kb) {
         if (!mbar_wait(&empty[s], ph ^ 1u, p.err)) { ok = false; break; }
         uint8_t* a_dst = tiles + size_t(s) * C::kStageBytes;
-        uint8_t* b_dst = a_dst + C::kABytes;
-        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-        tma_load_2d(&tmA, &full[s], a_dst, kb * kBK, mb * kBM);
-#pragma unroll
-        for (int h = 0; h < kBN / 128; ++h) {
-          const int row = (kEpi == EPI_SWIGLU && h == 1) ? p.inter + b_row0 : b_row0 + h * 128;
-          tma_load_2d(&tmB, &full[s], b_dst + h * 128 * 128, kb * kBK, row);
-        }
+        uint8_t* b_dst = a_dst + C::kHalfBytes;
+        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::kStageBytes);
+        const uint32_t bar = mapa_shared(smem_addr(&full[s]), 0);
+        tma_load_2d_pair(&tmA, bar, a_dst, kb * kBK, a_row);
+        tma_load_2d_pair(&tmB, bar, b_dst, kb * kBK, b_row);
         if (++s == C::kStages) { s = 0; ph ^= 1u; }
       }
     }
-  } else if (warp == 1 && lane == 0) {
+    // Drain: every stage this CTA filled is released (by a commit that
+    // writes into this CTA's shared memory) before the CTA may exit.
+    for (int i = 0; i < C::kStages && ok; ++i) {
+      if (!mbar_wait(&empty[s], ph ^ 1u, p.err)) break;
+      if (++s == C::kStages) { s = 0; ph ^= 1u; }
+    }
+  } else if (warp == 1 && lane == 0 && rank == 0) {
     // ---------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN);
+    constexpr uint32_t idesc = idesc_bf16_f32(256, kBN);
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+    for (int tile = pair; tile < num_tiles && ok; tile += n_pairs, ++it) {
       const int a = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       if (!mbar_wait(&acc_empty[a], (use & 1u) ^ 1u, p.err)) break;
@@ -170,158 +312,63 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&full[s], ph, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_addr = smem_addr(tiles + size_t(s) * C::kStageBytes);
-        const uint32_t b_addr = a_addr + C::kABytes;
+        const uint32_t b_addr = a_addr + C::kHalfBytes;
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
-          umma_f16_ss(d_tmem, sdesc_kmajor_sw128(a_addr + k * 32), sdesc_kmajor_sw128(b_addr + k * 32),
-                      idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_f16_ss_pair(d_tmem, sdesc_kmajor_sw128(a_addr + k * 32),
+                           sdesc_kmajor_sw128(b_addr + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
         }
-        umma_commit(&empty[s]);
+        const uint32_t e = smem_addr(&empty[s]);
+        umma_commit_pair(e);
+        umma_commit_pair(mapa_shared(e, 1));
         if (++s == C::kStages) { s = 0; ph ^= 1u; }
       }
-      if (ok) umma_commit(&acc_full[a]);
+      if (ok) {
+        const uint32_t f = smem_addr(&acc_full[a]);
+        umma_commit_pair(f);
+        umma_commit_pair(mapa_shared(f, 1));
+      }
+    }
+    // Drain: both accumulators released by both CTAs' epilogues (their
+    // arrivals write into this CTA's shared memory) before exit.
+    for (int i = 0; i < 2 && ok; ++i, ++it) {
+      const int a = it & 1;
+      const uint32_t use = static_cast<uint32_t>(it >> 1);
+      if (!mbar_wait(&acc_empty[a], (use & 1u) ^ 1u, p.err)) break;
     }
   } else if (warp >= 4) {
     // ---------------------------------------------------------- epilogue
     const int quarter = warp & 3;
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+    for (int tile = pair; tile < num_tiles; tile += n_pairs, ++it) {
       const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
       const int a = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       if (!mbar_wait_warp(&acc_full[a], use & 1u, p.err)) break;
       tc_fence_after();
-      const int64_t row = static_cast<int64_t>(mb) * kBM + quarter * 32 + lane;
-      const bool row_ok = row < p.M;
+      const int64_t row =
+          static_cast<int64_t>(mb) * 256 + static_cast<int64_t>(rank) * 128 + quarter * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(a * kBN);
-      if constexpr (kEpi == EPI_STORE || kEpi == EPI_RESIDUAL) {
-#pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
-          float v[32];
-          tmem_ld32_wait(t_row + c * 32, v);
-          const int col = nb * kBN + c * 32;
-          if (row_ok && col < p.N) {
-            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) + row * p.ldc + col;
-            if (kEpi == EPI_RESIDUAL)
-              add32_bf16(static_cast<const __nv_bfloat16*>(p.R) + row * p.ldr + col, v);
-            store32_bf16(dst, v);
-          }
-        }
-      } else if constexpr (kEpi == EPI_SWIGLU) {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float g[32], u[32];
-          tmem_ld32_wait(t_row + c * 32, g);
-          tmem_ld32_wait(t_row + 128 + c * 32, u);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) g[j] = silu_f(g[j]) * u[j];
-          if (row_ok)
-            store32_bf16(static_cast<__nv_bfloat16*>(p.C) + row * p.ldc + nb * 128 + c * 32, g);
-        }
-      } else if constexpr (kEpi == EPI_QKV) {
-        // Two whole heads per tile (head dim 128). The accumulator is rounded
-        // to bf16 first (the stored-q/k/v value), then q/k get the optional
-        // per-head RMSNorm and RoPE; v is written transposed (and as cache).
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          const int hg = nb * 2 + hh;  // head index across the q | k | v columns
-          const uint32_t t_head = t_row + static_cast<uint32_t>(hh * 128);
-          if (hg < p.hq + p.hkv) {
-            const bool is_q = hg < p.hq;
-            const float* nw = is_q ? p.q_norm : p.k_norm;
-            float rstd = 1.0f;
-            if (nw != nullptr) {
-              float ss = 0.f;
-#pragma unroll 1
-              for (int c = 0; c < 4; ++c) {
-                float v[32];
-                tmem_ld32_wait(t_head + c * 32, v);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                  const float f = round_bf16_f(v[i]);
-                  ss = fmaf(f, f, ss);
-                }
-              }
-              rstd = rsqrtf(ss * (1.0f / 128.0f) + p.eps);
-            }
-            __nv_bfloat16* dst =
-                is_q ? p.q_out + (row * p.hq + hg) * 128
-                     : p.k_out + (row * p.hkv + (hg - p.hq)) * 128;
-            const float2* cs = p.rope_cs + row;  // frequency-major: entry i at cs[i * M]
-#pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-              float lo[32], hi[32];
-              tmem_ld32_wait(t_head + c * 32, lo);
-              tmem_ld32_wait(t_head + 64 + c * 32, hi);
-              if (row_ok) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                  const int pi = c * 32 + i;
-                  float a = round_bf16_f(lo[i]) * rstd;
-                  float b = round_bf16_f(hi[i]) * rstd;
-                  if (nw != nullptr) {
-                    a *= __ldg(nw + pi);
-                    b *= __ldg(nw + pi + 64);
-                  }
-                  const float2 t = __ldg(cs + static_cast<int64_t>(pi) * p.M);
-                  lo[i] = a * t.x - b * t.y;
-                  hi[i] = b * t.x + a * t.y;
-                }
-                store32_bf16(dst + c * 32, lo);
-                store32_bf16(dst + 64 + c * 32, hi);
-              }
-            }
-          } else {
-            const int g = hg - p.hq - p.hkv;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              float v[32];
-              tmem_ld32_wait(t_head + c * 32, v);
-              if (row_ok) {
-                if (p.v_out) store32_bf16(p.v_out + (row * p.hkv + g) * 128 + c * 32, v);
-                __nv_bfloat16* vt = p.vT_out + (static_cast<int64_t>(g) * 128 + c * 32) * p.t_pad + row;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) vt[static_cast<int64_t>(i) * p.t_pad] = __float2bfloat16_rn(v[i]);
-              }
-            }
-          }
-        }
-      } else {  // EPI_SCORE
-        float acc = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
-          float v[32];
-          tmem_ld32_wait(t_row + c * 32, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int f = c * 32 + j;
-            if (f < p.N) {
-              const float h = v[j] + (p.b1 ? __ldg(p.b1 + f) : 0.f);
-              acc = fmaf(__ldg(p.w2 + f), silu_f(h), acc);
-            }
-          }
-        }
-        if (row_ok) p.scores[row] = acc + (p.b2 ? __ldg(p.b2) : 0.f);
-      }
+      epilogue_tile<kBN, kEpi>(p, row, t_row, nb);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[a]);
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&acc_empty[a]), 0));
     }
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem_base, C::kTmemCols);
+  __syncwarp();
+  if (warp == 2) tmem_dealloc_pair(tmem_base, C::kTmemCols);
 }
 
-template <int kBN, int kEpi>
+template <int kEpi>
 cudaError_t run(const GemmArgs& g, cudaStream_t st) {
-  using C = Cfg<kBN>;
+  using C = PairCfg;
   CUtensorMap ta, tb;
-  if (!make_tmap_2d_bf16(&ta, g.A, g.M, g.K, g.lda, kBM)) return cudaErrorInvalidValue;
-  const int64_t b_rows = g.N;
-  if (!make_tmap_2d_bf16(&tb, g.B, b_rows, g.K, g.ldb, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d_bf16(&ta, g.A, g.M, g.K, g.lda, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d_bf16(&tb, g.B, g.N, g.K, g.ldb, 128)) return cudaErrorInvalidValue;
   EpiParams p;
   p.M = g.M;
   p.N = kEpi == EPI_SWIGLU ? g.inter : g.N;
@@ -346,17 +393,35 @@ cudaError_t run(const GemmArgs& g, cudaStream_t st) {
   p.vT_out = static_cast<__nv_bfloat16*>(g.vT_out);
   p.t_pad = g.t_pad;
   p.v_out = static_cast<__nv_bfloat16*>(g.v_out);
-  p.tiles_m = static_cast<int>((g.M + kBM - 1) / kBM);
-  p.tiles_n = kEpi == EPI_SWIGLU ? g.inter / 128 : (g.N + kBN - 1) / kBN;
+  p.tiles_m = static_cast<int>((g.M + 255) / 256);
+  p.tiles_n = kEpi == EPI_SWIGLU ? g.inter / 128 : (g.N + 255) / 256;
   p.err = device_error_word();
   const int tiles = p.tiles_m * p.tiles_n;
   if (tiles == 0) return cudaSuccess;
-  auto kern = gemm_tc<kBN, kEpi>;
+  auto kern = gemm_tc<kEpi>;
   cudaError_t e = set_smem_attr_once(reinterpret_cast<const void*>(kern), static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
-  const int grid = tiles < num_sms() ? tiles : num_sms();
-  kern<<<grid, kThreads, C::kSmem, st>>>(ta, tb, p);
-  return cudaGetLastError();
+  // Persistent grid: as many pairs as can be resident at once (the SMs of a
+  // pair must share a TPC, so this can be below num_sms() / 2).
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> resident[kMaxDevices];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int max_pairs = (dev >= 0 && dev < kMaxDevices) ? resident[dev].load() : 0;
+  if (max_pairs <= 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(num_sms() & ~1), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = st;
+    if (cudaOccupancyMaxActiveClusters(&max_pairs, kern, &cfg) != cudaSuccess || max_pairs <= 0) {
+      cudaGetLastError();
+      max_pairs = num_sms() / 2;
+    }
+    if (dev >= 0 && dev < kMaxDevices) resident[dev].store(max_pairs);
+  }
+  const int pairs = tiles < max_pairs ? tiles : max_pairs;
+  return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), C::kSmem, st, ta, tb, p);
 }
 
 }  // namespace
@@ -385,11 +450,11 @@ bool gemm_tc_supported(const GemmArgs& g) {
 cudaError_t launch_gemm_tc(const GemmArgs& g, cudaStream_t st) {
   if (g.M <= 0) return cudaSuccess;
   switch (g.epi) {
-    case EPI_STORE: return run<256, EPI_STORE>(g, st);
-    case EPI_RESIDUAL: return run<256, EPI_RESIDUAL>(g, st);
-    case EPI_SWIGLU: return run<256, EPI_SWIGLU>(g, st);
-    case EPI_SCORE: return run<256, EPI_SCORE>(g, st);
-    case EPI_QKV: return run<256, EPI_QKV>(g, st);
+    case EPI_STORE: return run<EPI_STORE>(g, st);
+    case EPI_RESIDUAL: return run<EPI_RESIDUAL>(g, st);
+    case EPI_SWIGLU: return run<EPI_SWIGLU>(g, st);
+    case EPI_SCORE: return run<EPI_SCORE>(g, st);
+    case EPI_QKV: return run<EPI_QKV>(g, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -51,6 +51,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) rmsnorm_rows(const T* __restrict__ x,
                                                     const float* __restrict__ g, float eps,
                                                     int64_t rows, int d, T* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -100,6 +102,8 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_bf16_reg(const __nv_bfloat16
                                                             const float* __restrict__ g, float eps,
                                                             int64_t rows,
                                                             __nv_bfloat16* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int kD = kVPL * 256;
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
@@ -144,6 +148,8 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_bf16_reg(const __nv_bfloat16
 // token's gate bias logsigmoid(s_t).
 template <typename T, int kDh>
 __global__ void __launch_bounds__(128) rope_qk(RopePrepArgs a) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int kHalf = kDh / 2;
   constexpr int kPairs = kHalf / 32;  // pairs per lane
   __shared__ float s_cos[kHalf], s_sin[kHalf];
@@ -204,6 +210,8 @@ __global__ void __launch_bounds__(128) rope_qk(RopePrepArgs a) {
 // 32 consecutive entries of one frequency.
 __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int64_t T, int half, int dh,
                                   float rope_base, float2* __restrict__ cs) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= T * half) return;
   const int i = static_cast<int>(idx / T);
@@ -220,6 +228,8 @@ __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int64_t T, in
 
 // Gate-bias rows for the attention's extra K-step (see launch_bias_aug).
 __global__ void bias_aug_kernel(const float* __restrict__ lsig, int64_t T, uint4* __restrict__ kaug) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= T) return;
   const float b = __ldg(lsig + t);
@@ -239,6 +249,8 @@ __global__ void bias_aug_kernel(const float* __restrict__ lsig, int64_t T, uint4
 // v into a [T, hkv, dh] KV-cache buffer when asked.
 template <int kDh>
 __global__ void __launch_bounds__(256) v_transpose(RopePrepArgs a) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int kTile = 64;
   constexpr int kLd = kDh + 8;  // padded row (bf16 elements)
   __shared__ __align__(16) __nv_bfloat16 tile[kTile * kLd];
@@ -271,6 +283,8 @@ __global__ void __launch_bounds__(256) v_transpose(RopePrepArgs a) {
 
 // fp32 path: plain copy of v into a KV-cache buffer.
 __global__ void copy_v_f32(RopePrepArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t t = blockIdx.x;
   const float* v = static_cast<const float*>(a.v_src) + t * a.v_stride;
   float* o = static_cast<float*>(a.kv_v_out) + t * a.hkv * a.dh;
@@ -280,6 +294,8 @@ __global__ void copy_v_f32(RopePrepArgs a) {
 // ---------------------------------------------------------------- fp32 helpers
 __global__ void swiglu_f32(const float* __restrict__ gu, int64_t rows, int inter,
                            float* __restrict__ h) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t total = rows * inter;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -293,6 +309,8 @@ __global__ void swiglu_f32(const float* __restrict__ gu, int64_t rows, int inter
 __global__ void score_dot_f32(const float* __restrict__ hpre, int64_t rows, int f,
                               const float* __restrict__ b1, const float* __restrict__ w2,
                               const float* __restrict__ b2, float* __restrict__ scores) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -317,22 +335,20 @@ cudaError_t launch_rmsnorm(const void* x, const float* gamma, float eps, int64_t
     const auto* xb = static_cast<const __nv_bfloat16*>(x);
     auto* yb = static_cast<__nv_bfloat16*>(y);
     switch (d / 256) {
-      case 1: rmsnorm_rows_bf16_reg<1><<<blocks, 256, 0, st>>>(xb, gamma, eps, rows, yb); break;
-      case 2: rmsnorm_rows_bf16_reg<2><<<blocks, 256, 0, st>>>(xb, gamma, eps, rows, yb); break;
-      case 4: rmsnorm_rows_bf16_reg<4><<<blocks, 256, 0, st>>>(xb, gamma, eps, rows, yb); break;
-      case 8: rmsnorm_rows_bf16_reg<8><<<blocks, 256, 0, st>>>(xb, gamma, eps, rows, yb); break;
-      case 16: rmsnorm_rows_bf16_reg<16><<<blocks, 256, 0, st>>>(xb, gamma, eps, rows, yb); break;
+      case 1: TG_CUDA_TRY(launch_pdl(rmsnorm_rows_bf16_reg<1>, dim3(blocks), dim3(256), 0, st, xb, gamma, eps, rows, yb)); break;
+      case 2: TG_CUDA_TRY(launch_pdl(rmsnorm_rows_bf16_reg<2>, dim3(blocks), dim3(256), 0, st, xb, gamma, eps, rows, yb)); break;
+      case 4: TG_CUDA_TRY(launch_pdl(rmsnorm_rows_bf16_reg<4>, dim3(blocks), dim3(256), 0, st, xb, gamma, eps, rows, yb)); break;
+      case 8: TG_CUDA_TRY(launch_pdl(rmsnorm_rows_bf16_reg<8>, dim3(blocks), dim3(256), 0, st, xb, gamma, eps, rows, yb)); break;
+      case 16: TG_CUDA_TRY(launch_pdl(rmsnorm_rows_bf16_reg<16>, dim3(blocks), dim3(256), 0, st, xb, gamma, eps, rows, yb)); break;
       default:
-        rmsnorm_rows<__nv_bfloat16><<<blocks, 256, 0, st>>>(xb, gamma, eps, rows, d, yb);
+        TG_CUDA_TRY(launch_pdl(rmsnorm_rows<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st, xb, gamma, eps, rows, d, yb));
     }
     return cudaGetLastError();
   }
   if (bf16)
-    rmsnorm_rows<__nv_bfloat16><<<blocks, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), gamma, eps, rows, d, static_cast<__nv_bfloat16*>(y));
+    TG_CUDA_TRY(launch_pdl(rmsnorm_rows<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x), gamma, eps, rows, d, static_cast<__nv_bfloat16*>(y)));
   else
-    rmsnorm_rows<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(x), gamma, eps, rows, d,
-                                                static_cast<float*>(y));
+    TG_CUDA_TRY(launch_pdl(rmsnorm_rows<float>, dim3(blocks), dim3(256), 0, st, static_cast<const float*>(x), gamma, eps, rows, d, static_cast<float*>(y)));
   return cudaGetLastError();
 }
 
@@ -340,17 +356,17 @@ cudaError_t launch_rope_prep(const RopePrepArgs& a, cudaStream_t st) {
   if (a.T <= 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>(a.T);
   if (a.bf16) {
-    if (a.dh == 128) rope_qk<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(a);
-    else rope_qk<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(a);
+    if (a.dh == 128) TG_CUDA_TRY(launch_pdl(rope_qk<__nv_bfloat16, 128>, dim3(grid), dim3(128), 0, st, a));
+    else TG_CUDA_TRY(launch_pdl(rope_qk<__nv_bfloat16, 64>, dim3(grid), dim3(128), 0, st, a));
     if (a.vT_out) {
       const dim3 g2(static_cast<unsigned>(a.t_pad / 64), static_cast<unsigned>(a.hkv));
-      if (a.dh == 128) v_transpose<128><<<g2, 256, 0, st>>>(a);
-      else v_transpose<64><<<g2, 256, 0, st>>>(a);
+      if (a.dh == 128) TG_CUDA_TRY(launch_pdl(v_transpose<128>, dim3(g2), dim3(256), 0, st, a));
+      else TG_CUDA_TRY(launch_pdl(v_transpose<64>, dim3(g2), dim3(256), 0, st, a));
     }
   } else {
-    if (a.dh == 128) rope_qk<float, 128><<<grid, 128, 0, st>>>(a);
-    else rope_qk<float, 64><<<grid, 128, 0, st>>>(a);
-    if (a.kv_v_out) copy_v_f32<<<grid, 128, 0, st>>>(a);
+    if (a.dh == 128) TG_CUDA_TRY(launch_pdl(rope_qk<float, 128>, dim3(grid), dim3(128), 0, st, a));
+    else TG_CUDA_TRY(launch_pdl(rope_qk<float, 64>, dim3(grid), dim3(128), 0, st, a));
+    if (a.kv_v_out) TG_CUDA_TRY(launch_pdl(copy_v_f32, dim3(grid), dim3(128), 0, st, a));
   }
   return cudaGetLastError();
 }
@@ -360,15 +376,13 @@ cudaError_t launch_rope_table(const int32_t* pos, int64_t T, int dh, float rope_
   const int half = dh / 2;
   const int64_t total = T * half;
   if (total <= 0) return cudaSuccess;
-  rope_table_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(pos, T, half, dh,
-                                                                                rope_base, cs);
+  TG_CUDA_TRY(launch_pdl(rope_table_kernel, dim3(static_cast<unsigned>((total + 255) / 256)), dim3(256), 0, st, pos, T, half, dh, rope_base, cs));
   return cudaGetLastError();
 }
 
 cudaError_t launch_bias_aug(const float* lsig, int64_t T, void* kaug, cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
-  bias_aug_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, st>>>(lsig, T,
-                                                                         static_cast<uint4*>(kaug));
+  TG_CUDA_TRY(launch_pdl(bias_aug_kernel, dim3(static_cast<unsigned>((T + 255) / 256)), dim3(256), 0, st, lsig, T, static_cast<uint4*>(kaug)));
   return cudaGetLastError();
 }
 
@@ -376,15 +390,14 @@ cudaError_t launch_swiglu_f32(const float* gu, int64_t rows, int inter, float* h
   const int64_t total = rows * inter;
   if (total <= 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((total + 255) / 256, 148 * 16));
-  swiglu_f32<<<blocks, 256, 0, st>>>(gu, rows, inter, h);
+  TG_CUDA_TRY(launch_pdl(swiglu_f32, dim3(blocks), dim3(256), 0, st, gu, rows, inter, h));
   return cudaGetLastError();
 }
 
 cudaError_t launch_score_dot_f32(const float* hpre, int64_t rows, int f, const float* b1,
                                  const float* w2, const float* b2, float* scores, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  score_dot_f32<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(hpre, rows, f, b1, w2, b2,
-                                                                       scores);
+  TG_CUDA_TRY(launch_pdl(score_dot_f32, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, st, hpre, rows, f, b1, w2, b2, scores));
   return cudaGetLastError();
 }
 

@@ -176,6 +176,8 @@ template <bool kVec>
 __global__ void __launch_bounds__(kThreads) sel_hist0(const float* __restrict__ scores,
                                                       const uint8_t* __restrict__ protect,
                                                       int64_t n, Ws w) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ uint32_t hist[kHist0];
   for (int i = threadIdx.x; i < kHist0; i += kThreads) hist[i] = 0u;
   __syncthreads();
@@ -204,6 +206,8 @@ template <bool kVec, int kPass>
 __global__ void __launch_bounds__(kThreads) sel_hist_next(const float* __restrict__ scores,
                                                           const uint8_t* __restrict__ protect,
                                                           int64_t n, int64_t k, Ws w) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int kBinsPrev = kPass == 1 ? kHist0 : kHist1;
   constexpr int kBinsNext = kPass == 1 ? kHist1 : kHist2;
   __shared__ uint32_t hist[kBinsNext];
@@ -256,6 +260,8 @@ template <bool kVec>
 __global__ void __launch_bounds__(kThreads) sel_count(const float* __restrict__ scores,
                                                       const uint8_t* __restrict__ protect,
                                                       int64_t n, int64_t k, Ws w) {
+  pdl_trigger();
+  pdl_wait();
   if (w.st->status != 0) return;
   const int64_t np = w.st->n_prot;
   uint32_t thresh, ties;
@@ -299,6 +305,8 @@ __global__ void __launch_bounds__(kThreads) sel_write(const float* __restrict__ 
                                                       const uint8_t* __restrict__ protect,
                                                       int64_t n, int64_t k,
                                                       int32_t* __restrict__ kept_idx, Ws w) {
+  pdl_trigger();
+  pdl_wait();
   if (w.st->status != 0) {
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < k;
          i += static_cast<int64_t>(gridDim.x) * kThreads)
@@ -367,11 +375,11 @@ cudaError_t run_select(const float* scores, const uint8_t* protect, int64_t n, i
   cudaError_t e = cudaMemsetAsync(ws, 0, kZeroBytes, st);
   if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>(chunks));
-  sel_hist0<kVec><<<grid, kThreads, 0, st>>>(scores, protect, n, w);
-  sel_hist_next<kVec, 1><<<grid, kThreads, 0, st>>>(scores, protect, n, k, w);
-  sel_hist_next<kVec, 2><<<grid, kThreads, 0, st>>>(scores, protect, n, k, w);
-  sel_count<kVec><<<grid, kThreads, 0, st>>>(scores, protect, n, k, w);
-  sel_write<kVec><<<grid, kThreads, 0, st>>>(scores, protect, n, k, kept_idx, w);
+  TG_CUDA_TRY(launch_pdl(sel_hist0<kVec>, dim3(grid), dim3(kThreads), 0, st, scores, protect, n, w));
+  TG_CUDA_TRY(launch_pdl(sel_hist_next<kVec, 1>, dim3(grid), dim3(kThreads), 0, st, scores, protect, n, k, w));
+  TG_CUDA_TRY(launch_pdl(sel_hist_next<kVec, 2>, dim3(grid), dim3(kThreads), 0, st, scores, protect, n, k, w));
+  TG_CUDA_TRY(launch_pdl(sel_count<kVec>, dim3(grid), dim3(kThreads), 0, st, scores, protect, n, k, w));
+  TG_CUDA_TRY(launch_pdl(sel_write<kVec>, dim3(grid), dim3(kThreads), 0, st, scores, protect, n, k, kept_idx, w));
   return cudaGetLastError();
 }
 

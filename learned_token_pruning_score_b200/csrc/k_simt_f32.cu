@@ -22,6 +22,8 @@ namespace {
 constexpr int kBM = 64, kBN = 64, kBK = 16;
 
 __global__ void __launch_bounds__(256) gemm_f32(GemmArgs g) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float As[kBK][kBM + 4];
   __shared__ float Bs[kBK][kBN + 4];
   const float* A = static_cast<const float*>(g.A);
@@ -75,6 +77,8 @@ __global__ void __launch_bounds__(256) gemm_f32(GemmArgs g) {
 // keys are visited in order with an online (running max) softmax.
 template <int kDh>
 __global__ void __launch_bounds__(256) attn_f32(AttnArgs a, int64_t v_stride) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int kPer = kDh / 32;
   const int lane = threadIdx.x & 31;
   const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
@@ -124,7 +128,7 @@ cudaError_t launch_gemm_simt_f32(const GemmArgs& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0) return cudaSuccess;
   const dim3 grid(static_cast<unsigned>((g.N + kBN - 1) / kBN),
                   static_cast<unsigned>((g.M + kBM - 1) / kBM));
-  gemm_f32<<<grid, 256, 0, st>>>(g);
+  TG_CUDA_TRY(launch_pdl(gemm_f32, dim3(grid), dim3(256), 0, st, g));
   return cudaGetLastError();
 }
 
@@ -134,8 +138,8 @@ cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t st) {
   const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
   // fp32 v is [T, hkv, dh] unless the caller passes a wider row in t_pad
   const int64_t v_stride = a.t_pad > 0 ? a.t_pad : static_cast<int64_t>(a.hkv) * a.dh;
-  if (a.dh == 128) attn_f32<128><<<blocks, 256, 0, st>>>(a, v_stride);
-  else attn_f32<64><<<blocks, 256, 0, st>>>(a, v_stride);
+  if (a.dh == 128) TG_CUDA_TRY(launch_pdl(attn_f32<128>, dim3(blocks), dim3(256), 0, st, a, v_stride));
+  else TG_CUDA_TRY(launch_pdl(attn_f32<64>, dim3(blocks), dim3(256), 0, st, a, v_stride));
   return cudaGetLastError();
 }
 

@@ -27,6 +27,34 @@ struct Arena {
   }
 };
 
+// Enqueues `kernel<<<grid, block, smem, st>>>(args...)` with programmatic
+// stream serialization allowed (see pdl_trigger / pdl_wait in
+// tg_device.cuh): the kernel may be scheduled, and run its prologue, while
+// the previous kernel of the stream drains. Every kernel launched this way
+// calls pdl_wait() before its first global-memory access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// Returns the CUDA error of `expr` from the enclosing launcher, if any.
+#define TG_CUDA_TRY(expr)                           \
+  do {                                              \
+    const cudaError_t tg_e_ = (expr);               \
+    if (tg_e_ != cudaSuccess) return tg_e_;         \
+  } while (0)
+
 int num_sms();
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device).
 cudaError_t set_smem_attr_once(const void* fn, int bytes);
