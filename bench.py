@@ -107,13 +107,18 @@ class ClockSampler:
 
 
 def kernel_source_hash(name: str) -> str:
+    """First 12 hex digits of the sha256 of the kernel's source file and the
+    device header it includes."""
     files = {"attention_tc": "k_attn_tc.cu", "gemm_tc": "k_gemm_tc.cu"}
     key = "gemm_tc" if name.startswith("gemm_tc") else name
     f = files.get(key)
     if f is None:
         return ""
-    with open(os.path.join(ROOT, "learned_token_pruning_score_b200", "csrc", f), "rb") as fh:
-        return hashlib.sha256(fh.read()).hexdigest()[:12]
+    h = hashlib.sha256()
+    for part in (f, "tg_device.cuh"):
+        with open(os.path.join(ROOT, "learned_token_pruning_score_b200", "csrc", part), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
 
 
 def traffic_from_profiles(kernel: str, workload: str):

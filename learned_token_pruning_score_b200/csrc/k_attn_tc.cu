@@ -25,6 +25,7 @@
 //              in the 128-byte-swizzled K-major layout the MMA reads.
 //   end        O / l read from TMEM, written bf16.
 // TMEM: S0 = cols [0,128), S1 = [128,256), O = [256,384) of 512.
+#include <atomic>
 #include <type_traits>
 
 #include "tg_device.cuh"
@@ -317,6 +318,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 namespace pair {
 
 constexpr int kThreads = 384;
+// Register split (setmaxnreg): the kernel launches with kRegsLaunch per
+// thread (the most that 384 threads may hold); warpgroup 0 drops to
+// kRegsLow and the softmax warpgroups rise to kRegsHigh. The split must use
+// exactly the registers the CTA launched with, or setmaxnreg.inc would wait
+// for registers that never come: the launcher checks the compiled count.
+constexpr uint32_t kRegsLaunch = 168, kRegsLow = 72, kRegsHigh = 216;
+static_assert(kRegsLow * 128 + kRegsHigh * 256 == kRegsLaunch * kThreads, "register split");
 // Shared-memory layout. With the gate bias, its 32-byte-swizzled tiles come
 // first (an addressing slip there cannot reach past the allocation), then
 // the 128-byte-swizzled operand tiles.
@@ -419,90 +427,96 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   pdl_wait();  // q, k, V^T and the bias rows come from the previous kernels
 
-  if (warp == 0 && lane == 0) {
-    // ---------------------------------------------------------- TMA producer
-    mbar_arrive_expect_tx(q_full, 2 * kTile);
-    tma_load_3d(&tmQ, q_full, smem + kOffQA, 0, head0, q0);
-    tma_load_3d(&tmQ, q_full, smem + kOffQA + kSub, 64, head0, q0);
-    tma_load_3d(&tmQ, q_full, smem + kOffQB, 0, head0 + 1, q0);
-    tma_load_3d(&tmQ, q_full, smem + kOffQB + kSub, 64, head0 + 1, q0);
-    for (int j = 0; j < n_kv; ++j) {
-      const int s = j & 1;
-      const uint32_t ph = ((j >> 1) & 1) ^ 1;
-      if (!mbar_wait(&k_empty[s], ph, p.err)) break;
-      uint8_t* kd = smem + kOffK + s * kTile;
-      mbar_arrive_expect_tx(&k_full[s], kKBytes);
-      tma_load_3d(&tmK, &k_full[s], kd, 0, g, j * kBlk);
-      tma_load_3d(&tmK, &k_full[s], kd + kSub, 64, g, j * kBlk);
-      if (kBias) tma_load_2d(&tmKAug, &k_full[s], smem + kOffKAug + s * kAugTile, 0, j * kBlk);
-      if (!mbar_wait(&v_empty[s], ph, p.err)) break;
-      uint8_t* vd = smem + kOffV + s * kTile;
-      mbar_arrive_expect_tx(&v_full[s], kTile);
-      tma_load_3d(&tmV, &v_full[s], vd, j * kBlk, 0, g);
-      tma_load_3d(&tmV, &v_full[s], vd + kSub, j * kBlk + 64, 0, g);
-    }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
-    auto issue_qk = [&](int h, int j) {
-      const uint32_t q_addr = smem_addr(smem + (h ? kOffQB : kOffQA));
-      const uint32_t k_addr = smem_addr(smem + kOffK + (j & 1) * kTile);
-      const uint32_t d = tmem + static_cast<uint32_t>(h * 128);
-#pragma unroll
-      for (int kk = 0; kk < kDh / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
-        umma_f16_ss(d, sdesc_kmajor_sw128(q_addr + off), sdesc_kmajor_sw128(k_addr + off), idesc,
-                    kk > 0 ? 1u : 0u);
+  if (warp < 4) {
+    // Warpgroup 0 (TMA, MMA, TMEM allocation) needs few registers: it hands
+    // them to the two softmax warpgroups.
+    setmaxnreg_dec<kRegsLow>();
+    if (warp == 0 && lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      mbar_arrive_expect_tx(q_full, 2 * kTile);
+      tma_load_3d(&tmQ, q_full, smem + kOffQA, 0, head0, q0);
+      tma_load_3d(&tmQ, q_full, smem + kOffQA + kSub, 64, head0, q0);
+      tma_load_3d(&tmQ, q_full, smem + kOffQB, 0, head0 + 1, q0);
+      tma_load_3d(&tmQ, q_full, smem + kOffQB + kSub, 64, head0 + 1, q0);
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j & 1;
+        const uint32_t ph = ((j >> 1) & 1) ^ 1;
+        if (!mbar_wait(&k_empty[s], ph, p.err)) break;
+        uint8_t* kd = smem + kOffK + s * kTile;
+        mbar_arrive_expect_tx(&k_full[s], kKBytes);
+        tma_load_3d(&tmK, &k_full[s], kd, 0, g, j * kBlk);
+        tma_load_3d(&tmK, &k_full[s], kd + kSub, 64, g, j * kBlk);
+        if (kBias) tma_load_2d(&tmKAug, &k_full[s], smem + kOffKAug + s * kAugTile, 0, j * kBlk);
+        if (!mbar_wait(&v_empty[s], ph, p.err)) break;
+        uint8_t* vd = smem + kOffV + s * kTile;
+        mbar_arrive_expect_tx(&v_full[s], kTile);
+        tma_load_3d(&tmV, &v_full[s], vd, j * kBlk, 0, g);
+        tma_load_3d(&tmV, &v_full[s], vd + kSub, j * kBlk + 64, 0, g);
       }
-      if (kBias) {  // the gate-bias K-step
-        umma_f16_ss(d, sdesc_kmajor_sw32(smem_addr(smem + (h ? kOffQAugB : kOffQAugA))),
-                    sdesc_kmajor_sw32(smem_addr(smem + kOffKAug + (j & 1) * kAugTile)), idesc, 1u);
-      }
-      umma_commit(&s_full[h]);
-    };
-    auto issue_pv = [&](int h, int j) {
-      const uint32_t v_addr = smem_addr(smem + kOffV + (j & 1) * kTile);
-      const uint32_t a = tmem + static_cast<uint32_t>(h * 128);        // P_h
-      const uint32_t d = tmem + 256u + static_cast<uint32_t>(h * 128);  // O_h
-#pragma unroll
-      for (int kk = 0; kk < kBlk / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
-        umma_f16_ts(d, a + static_cast<uint32_t>(kk * 8), sdesc_kmajor_sw128(v_addr + off), idesc,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-      }
-    };
-    bool ok = mbar_wait(q_full, 0, p.err) && mbar_wait(&k_full[0], 0, p.err);
-    if (kBias) ok = ok && mbar_wait(qaug_full, 0, p.err);
-    if (ok) {
-      tc_fence_after();
-      issue_qk(0, 0);
-      issue_qk(1, 0);
-      umma_commit(&k_empty[0]);
-    }
-    for (int j = 0; j < n_kv && ok; ++j) {
-      const int s = j & 1;
-      const uint32_t ph = (j >> 1) & 1;
-      const bool more = j + 1 < n_kv;
-      if (!mbar_wait(&v_full[s], ph, p.err)) break;
-      if (!mbar_wait(&p_full[0], j & 1, p.err)) break;
-      tc_fence_after();
-      issue_pv(0, j);
-      if (more) {
-        if (!mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, p.err)) break;
+    } else if (warp == 1 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+      auto issue_qk = [&](int h, int j) {
+        const uint32_t q_addr = smem_addr(smem + (h ? kOffQB : kOffQA));
+        const uint32_t k_addr = smem_addr(smem + kOffK + (j & 1) * kTile);
+        const uint32_t d = tmem + static_cast<uint32_t>(h * 128);
+  #pragma unroll
+        for (int kk = 0; kk < kDh / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
+          umma_f16_ss(d, sdesc_kmajor_sw128(q_addr + off), sdesc_kmajor_sw128(k_addr + off), idesc,
+                      kk > 0 ? 1u : 0u);
+        }
+        if (kBias) {  // the gate-bias K-step
+          umma_f16_ss(d, sdesc_kmajor_sw32(smem_addr(smem + (h ? kOffQAugB : kOffQAugA))),
+                      sdesc_kmajor_sw32(smem_addr(smem + kOffKAug + (j & 1) * kAugTile)), idesc, 1u);
+        }
+        umma_commit(&s_full[h]);
+      };
+      auto issue_pv = [&](int h, int j) {
+        const uint32_t v_addr = smem_addr(smem + kOffV + (j & 1) * kTile);
+        const uint32_t a = tmem + static_cast<uint32_t>(h * 128);        // P_h
+        const uint32_t d = tmem + 256u + static_cast<uint32_t>(h * 128);  // O_h
+  #pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
+          umma_f16_ts(d, a + static_cast<uint32_t>(kk * 8), sdesc_kmajor_sw128(v_addr + off), idesc,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(q_full, 0, p.err) && mbar_wait(&k_full[0], 0, p.err);
+      if (kBias) ok = ok && mbar_wait(qaug_full, 0, p.err);
+      if (ok) {
         tc_fence_after();
-        issue_qk(0, j + 1);
+        issue_qk(0, 0);
+        issue_qk(1, 0);
+        umma_commit(&k_empty[0]);
       }
-      if (!mbar_wait(&p_full[1], j & 1, p.err)) break;
-      tc_fence_after();
-      issue_pv(1, j);
-      umma_commit(&v_empty[s]);
-      if (more) {
-        issue_qk(1, j + 1);
-        umma_commit(&k_empty[(j + 1) & 1]);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        const bool more = j + 1 < n_kv;
+        if (!mbar_wait(&v_full[s], ph, p.err)) break;
+        if (!mbar_wait(&p_full[0], j & 1, p.err)) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (more) {
+          if (!mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, p.err)) break;
+          tc_fence_after();
+          issue_qk(0, j + 1);
+        }
+        if (!mbar_wait(&p_full[1], j & 1, p.err)) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        umma_commit(&v_empty[s]);
+        if (more) {
+          issue_qk(1, j + 1);
+          umma_commit(&k_empty[(j + 1) & 1]);
+        }
       }
+      if (ok) umma_commit(o_full);
     }
-    if (ok) umma_commit(o_full);
-  } else if (warp >= 4) {
+  } else {
+    setmaxnreg_inc<kRegsHigh>();
     // ---------------------------------------------------------- softmax
     const int h = (warp - 4) >> 2;  // 0: head A (warps 4-7), 1: head B (warps 8-11)
     const int head = head0 + h;
@@ -537,31 +551,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int kv0 = j * kBlk;
       if (!mbar_wait_warp(&s_full[h], j & 1, p.err)) { ok = false; break; }
       tc_fence_after();
+      // S row: four TMEM loads in flight, one wait.
       float x[128];
+      {
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        const uint32_t sa = tmem + lane_off + s_col;
+        tmem_ld32(sa, r0);
+        tmem_ld32(sa + 32, r1);
+        tmem_ld32(sa + 64, r2);
+        tmem_ld32(sa + 96, r3);
+        tmem_wait_ld_dep(r3);
+        tmem_ld_fence(r0);
+        tmem_ld_fence(r1);
+        tmem_ld_fence(r2);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float t[32];
-        tmem_ld32_wait(tmem + lane_off + s_col + static_cast<uint32_t>(c * 32), t);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[c * 32 + i] = t[i];
+        for (int i = 0; i < 32; ++i) {
+          x[i] = __uint_as_float(r0[i]);
+          x[32 + i] = __uint_as_float(r1[i]);
+          x[64 + i] = __uint_as_float(r2[i]);
+          x[96 + i] = __uint_as_float(r3[i]);
+        }
       }
-      if (j == n_kv - 1) {  // diagonal tile: causal mask
+      const bool diag = j == n_kv - 1;
+      if (diag) {  // diagonal tile: causal mask
 #pragma unroll
         for (int i = 0; i < 128; ++i)
           if (kv0 + i > q_row) x[i] = -INFINITY;
       }
-      // Row max and row sum as 8-way trees: a single running max/sum would
-      // be a 128-long chain of dependent instructions per tile.
+      // Row max: eight independent chains of 3-input max (a single running
+      // max would be a 128-long dependent chain).
       float mx8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = x[i];
+      for (int k = 0; k < 8; ++k) mx8[k] = fmax3f(x[k], x[8 + k], x[16 + k]);
 #pragma unroll
-      for (int i = 8; i < 128; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], x[i]);
+      for (int i = 24; i < 120; i += 16)
 #pragma unroll
-      for (int w = 4; w > 0; w >>= 1)
+        for (int k = 0; k < 8; ++k) mx8[k] = fmax3f(mx8[k], x[i + k], x[i + 8 + k]);
 #pragma unroll
-        for (int i = 0; i < w; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + w]);
-      const float mx = mx8[0] * scale2;
+      for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], x[120 + k]);
+      const float mx = fmax3f(fmax3f(mx8[0], mx8[1], mx8[2]), fmax3f(mx8[3], mx8[4], mx8[5]),
+                              fmaxf(mx8[6], mx8[7])) *
+                       scale2;
       float alpha = 1.0f;
       if (mx > m + kRescaleThresh || m == -INFINITY) {
         alpha = ex2(m - mx);  // 0 on the first tile
@@ -569,26 +599,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = mx;
       }
       const bool rescale_o = j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f);
-      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // P = 2^(S * scale2 - m) in packed pairs; the row sum in four packed
+      // partial sums. Off the diagonal tile (no masked logits) one pair in
+      // four goes through the FMA-pipe polynomial, which unloads the MUFU
+      // unit, the bottleneck of this loop.
+      float2 sp[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
+      const float2 sc2 = make_float2(scale2, scale2), nm2 = make_float2(-m, -m);
+      auto exp_tile = [&](auto poly) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float a0 = ex2(fmaf(x[64 * half + 2 * i], scale2, -m));
-          const float a1 = ex2(fmaf(x[64 * half + 2 * i + 1], scale2, -m));
-          s8[(2 * i) & 7] += a0;
-          s8[(2 * i + 1) & 7] += a1;
-          pk[i] = pack_bf16x2(a0, a1);
+          for (int i = 0; i < 32; ++i) {
+            const float2 y =
+                ffma2(make_float2(x[64 * half + 2 * i], x[64 * half + 2 * i + 1]), sc2, nm2);
+            float2 a;
+            if (decltype(poly)::value && (i & 3) == 3) {
+              a = exp2_poly3_x2(y);
+            } else {
+              a.x = ex2(y.x);
+              a.y = ex2(y.y);
+            }
+            sp[i & 3] = fadd2(sp[i & 3], a);
+            pk[i] = pack_bf16x2(a.x, a.y);
+          }
+          tmem_st32(tmem + lane_off + s_col + static_cast<uint32_t>(32 * half), pk);
+          tmem_wait_st();
         }
-        tmem_st32(tmem + lane_off + s_col + static_cast<uint32_t>(32 * half), pk);
-        tmem_wait_st();
-      }
-#pragma unroll
-      for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-        for (int i = 0; i < w; ++i) s8[i] += s8[i + w];
-      l += s8[0];
+      };
+      if (diag) exp_tile(std::false_type());
+      else exp_tile(std::true_type());
+      const float2 s2 = fadd2(fadd2(sp[0], sp[1]), fadd2(sp[2], sp[3]));
+      l += s2.x + s2.y;
       if (rescale_o) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -692,6 +735,17 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
     const size_t smem = bias ? pair::Layout<true>::kSmem : pair::Layout<false>::kSmem;
     cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(kern), int(smem));
     if (err != cudaSuccess) return err;
+    // The register split inside the kernel assumes the compiled per-thread
+    // count; with any other count setmaxnreg.inc could block, so refuse.
+    static std::atomic<int> regs_ok[2];
+    std::atomic<int>& ok = regs_ok[bias ? 1 : 0];
+    if (ok.load() == 0) {
+      cudaFuncAttributes fa;
+      err = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kern));
+      if (err != cudaSuccess) return err;
+      ok.store(fa.numRegs == int(pair::kRegsLaunch) ? 1 : -1);
+    }
+    if (ok.load() < 0) return cudaErrorInvalidConfiguration;
     const unsigned grid = static_cast<unsigned>(p.n_qtiles) * static_cast<unsigned>(a.hq / 2);
     return launch_pdl(kern, dim3(grid), dim3(pair::kThreads), smem, st, tq, tk, tv, tka, pp);
   }
