@@ -442,7 +442,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- other budgets, dense baseline and peak memory (not timed region)
     extras = {}
     if not args.quick:
-        def ttft(mdl, kk, reps=3):
+        def ttft(mdl, kk, reps=5):
             # peak memory of one prefill: weights + input + outputs (incl. KV
             # cache) + workspace, all allocated by the caller
             torch.cuda.synchronize()
@@ -454,16 +454,17 @@ def run_ours(args, rank, world, local_rank):
                               device=device)
             tg.tg_prefill(mdl, x, prot, kk, w.gate_layer, out=o, kept_idx=ki, kv=kvb, ws=wsz)
             torch.cuda.synchronize()
-            ms = []
-            for _ in range(reps):
+            # back to back like the headline steps (an idle gap before each
+            # step would let the clocks recover and flatter the number)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(reps)]
+            for a, b in evs:
                 flush.zero_()
-                a = torch.cuda.Event(enable_timing=True)
-                b = torch.cuda.Event(enable_timing=True)
                 a.record(stream)
                 tg.tg_prefill(mdl, x, prot, kk, w.gate_layer, out=o, kept_idx=ki, kv=kvb, ws=wsz)
                 b.record(stream)
-                torch.cuda.synchronize()
-                ms.append(a.elapsed_time(b))
+            torch.cuda.synchronize()
+            ms = [a.elapsed_time(b) for a, b in evs]
             # one more, traced: the attention kernels' own durations
             flush.zero_()
             tg.tg_trace_start(1 << 14)
