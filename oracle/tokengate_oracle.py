@@ -56,6 +56,10 @@ Readings where the pages are silent (each one is listed in the design notes):
       q/k after qk-norm + RoPE, the attention output, every residual-stream
       value, the SwiGLU product, and the final output. Everything between
       two rounding points is float64. Scores are stored as float32.
+  R8  Decode: the t-th generated token has position N + t; above the gate
+      its logits over the cached keys follow R2, with the kept prompt tokens'
+      scores as the bias and no bias (logsigmoid = 0) on generated tokens'
+      keys; tau applies to every key.
 """
 
 from __future__ import annotations
@@ -324,8 +328,9 @@ class Model:
     rope_base: float = 1e6
 
 
-def attention_sublayer(x, lw: Layer, m: Model, pos, s, gain, tau, store):
-    """r = x + Wo . attn(RoPE(qk-norm(W_qkv . RMSNorm(x)))) and the layer's KV."""
+def project_qkv(x, lw: Layer, m: Model, pos, store):
+    """Rows x [t, d] -> q [t, Hq, dh] and k [t, Hkv, dh] (qk-norm, then RoPE at
+    pos, stored) and v [t, Hkv, dh] (stored) (R4, R6, R7)."""
     t = x.shape[0]
     hq, hkv, dh = m.n_heads_q, m.n_heads_kv, m.head_dim
     y = store(rmsnorm(x, lw.attn_norm, m.eps))
@@ -336,10 +341,15 @@ def attention_sublayer(x, lw: Layer, m: Model, pos, s, gain, tau, store):
     if lw.q_norm is not None:
         q = rmsnorm(q, lw.q_norm, m.eps)
         k = rmsnorm(k, lw.k_norm, m.eps)
-    q = store(rope(q, pos, m.rope_base))
-    k = store(rope(k, pos, m.rope_base))
+    return store(rope(q, pos, m.rope_base)), store(rope(k, pos, m.rope_base)), v
+
+
+def attention_sublayer(x, lw: Layer, m: Model, pos, s, gain, tau, store):
+    """r = x + Wo . attn(RoPE(qk-norm(W_qkv . RMSNorm(x)))) and the layer's KV."""
+    t = x.shape[0]
+    q, k, v = project_qkv(x, lw, m, pos, store)
     o = store(gated_attention(q, k, v, pos, s, gain, tau))
-    r = store(x + o.reshape(t, hq * dh) @ np.asarray(lw.wo, dtype=F64).T)
+    r = store(x + o.reshape(t, m.n_heads_q * m.head_dim) @ np.asarray(lw.wo, dtype=F64).T)
     return r, (k, v)
 
 
@@ -410,6 +420,63 @@ def prefill(x, protect, k: int, m: Model, gate_layer: int, store=round_bf16,
     out = h if m.final_norm is None else store(rmsnorm(h, m.final_norm, m.eps))
     return PrefillResult(out=out, kept_idx=idx, scores=s.astype(np.float32), kv=kv,
                          gate_residual=r if gate_layer < 0 else None)
+
+
+def decode_step(x, pos: int, m: Model, gate_layer: int, cache, kept_scores=None,
+                store=round_bf16):
+    """One generated token through every layer, after a gated prefill.
+
+    Generated tokens are never pruned ([TC] "TokenGate 提前筛选 Token"), so
+    the token runs every layer and appends its k/v to every layer's cache.
+    Layers at and below the gate hold the full prompt's KV, layers above only
+    the kept tokens' KV ([TC] "TokenGate 的工程验证仍有限"). In decoding the
+    gate bias fixed at prefill is an additive mask over the cached keys (same
+    section), so an upper layer's logits are those of R2 with the kept prompt
+    tokens' scores; the generated tokens' keys carry no bias (R8).
+
+    x [d]: the token's input hidden state; pos: its position (the prompt is
+    0..N-1, so the t-th generated token has pos N + t).
+    cache: per layer (k [T_l, Hkv, dh] post-RoPE, v [T_l, Hkv, dh]): T_l =
+    N + t at or below the gate, K + t above, rows in position order, every one
+    earlier than pos. kept_scores [K]: gate scores of the kept prompt tokens,
+    which are rows 0..K-1 of every upper cache.
+    Returns (out [d] final-normed, [(k_new [Hkv, dh], v_new [Hkv, dh]) per layer]).
+    """
+    h = store(np.asarray(x, dtype=F64).reshape(1, -1))
+    p = np.array([pos], dtype=np.int64)
+    new_kv = []
+    for li, lw in enumerate(m.layers):
+        kc, vc = cache[li]
+        q, k, v = project_qkv(h, lw, m, p, store)
+        k_all = np.concatenate([np.asarray(kc, dtype=F64), k])
+        v_all = np.concatenate([np.asarray(vc, dtype=F64), v])
+        before = np.full(k_all.shape[0], pos, dtype=np.int64)  # every key is visible
+        if li > gate_layer:
+            ks = np.asarray(kept_scores, dtype=F64)
+            s_all = np.concatenate([ks, np.full(k_all.shape[0] - ks.size, np.inf)])  # logsig(inf) = 0
+            o = gated_attention_rows(q, p, k_all, v_all, before, s_all, lw.gain, lw.tau)
+        else:
+            o = gated_attention_rows(q, p, k_all, v_all, before, None, None, None)
+        o = store(o)
+        r = store(h + o.reshape(1, -1) @ np.asarray(lw.wo, dtype=F64).T)
+        h = ffn_sublayer(r, lw, m, store)
+        new_kv.append((k[0], v[0]))
+    out = h if m.final_norm is None else store(rmsnorm(h, m.final_norm, m.eps))
+    return out[0], new_kv
+
+
+def decode_bytes(m: Model, lens, elem: int = 2) -> int:
+    """Algorithmic HBM bytes of one decode step: every weight matrix read
+    once, every cached k/v row read once (lens[l] rows before the step), the
+    new k/v rows written."""
+    hkv, dh = m.n_heads_kv, m.head_dim
+    total = 0
+    for lw, t in zip(m.layers, lens):
+        for w in (lw.wqkv, lw.wo, lw.w_gate_up, lw.w_down):
+            if w is not None:
+                total += int(np.asarray(w).size) * elem
+        total += (2 * t + 2) * hkv * dh * elem
+    return total
 
 
 def gated_layer_forward(x_k, pos_k, s_k, lw: Layer, m: Model, store=round_bf16):

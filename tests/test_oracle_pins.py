@@ -496,3 +496,82 @@ def test_pruned_tokens_make_no_upper_kv_and_kept_set_drives_upper_layers():
 def test_work_counts():
     assert ref.attention_flops(2048, 16, 128) == pytest.approx(17.19e9, rel=1e-3)
     assert ref.select_compact_bytes(131072, 65536, 2048) == pytest.approx(538e6, rel=2e-3)
+
+
+# ---------------------------------------------------------------- decode step
+
+
+def _hf_cache(kv):
+    from transformers import DynamicCache
+
+    cache = DynamicCache()
+    for li, (k, v) in enumerate(kv):
+        cache.update(torch.from_numpy(np.ascontiguousarray(k)).permute(1, 0, 2)[None].contiguous(),
+                     torch.from_numpy(np.ascontiguousarray(v)).permute(1, 0, 2)[None].contiguous(),
+                     li)
+    return cache
+
+
+@pytest.mark.parametrize("store", [ref.identity, ref.round_bf16])
+def test_decode_step_equals_prefill_of_one_more_token(store):
+    """Incremental decoding is full recomputation: with every layer at or
+    below the gate (K = N), prefilling N tokens and decoding token N gives
+    token N's row of a prefill over N + 1 tokens, and the decoded k/v rows
+    are that prefill's last cache rows."""
+    m = _tiny_model(40, True, n_layers=3)
+    n, last = 17, 2
+    x = np.random.default_rng(7).standard_normal((n + 1, m.d_model))
+    res = ref.prefill(x[:n], ref_protect(n, 3), n, m, last, store=store)
+    out, new_kv = ref.decode_step(x[n], n, m, last, res.kv, None, store=store)
+    full = ref.prefill(x, ref_protect(n + 1, 3), n + 1, m, last, store=store)
+    tol = 1e-12 if store is ref.identity else 0.0
+    assert np.max(np.abs(out - full.out[-1])) <= tol
+    for (k_new, v_new), (k_full, v_full) in zip(new_kv, full.kv):
+        assert np.max(np.abs(k_new - k_full[-1])) <= tol
+        assert np.max(np.abs(v_new - v_full[-1])) <= tol
+
+
+@pytest.mark.parametrize("qk_norm", [True, False])
+def test_decode_step_matches_transformers_kv_cache(qk_norm):
+    """The oracle's decode over a prefill's cache against a Hugging Face
+    model stepping one token with the same cache (past_key_values)."""
+    m = _tiny_model(41 + qk_norm, qk_norm, n_layers=3)
+    n = 15
+    x = np.random.default_rng(8).standard_normal((n + 1, m.d_model))
+    res = ref.prefill(x[:n], ref_protect(n, 2), n, m, len(m.layers) - 1, store=ref.identity)
+    out, _ = ref.decode_step(x[n], n, m, len(m.layers) - 1, res.kv, None, store=ref.identity)
+    hf = _hf_model(m, qk_norm)
+    with torch.no_grad():
+        o = hf(inputs_embeds=torch.from_numpy(x[n:n + 1])[None], past_key_values=_hf_cache(res.kv),
+               position_ids=torch.tensor([[n]]), use_cache=True).last_hidden_state[0, -1].numpy()
+    assert np.allclose(out, o, rtol=0, atol=2e-6)  # float32-level, as the prefill pin
+
+
+def test_decode_gate_bias_matches_transformers_additive_mask():
+    """Above the gate, the kept prompt keys carry gain * logsigmoid(s_j) and
+    the generated token's own key carries none: with one gain for every head
+    and layer and tau = 1 that is an additive attention mask, which a Hugging
+    Face model applies to the logits as given."""
+    m = _tiny_model(43, True, n_layers=3)
+    rng = np.random.default_rng(9)
+    gain = 0.7
+    for lw in m.layers:
+        lw.gain = np.full(m.n_heads_q, gain)
+        lw.tau = np.ones(m.n_heads_q)
+    n, k = 15, 7
+    x = rng.standard_normal((n + 1, m.d_model))
+    res = ref.prefill(x[:n], ref_protect(n, 2), n, m, len(m.layers) - 1, store=ref.identity)
+    kept = np.sort(rng.choice(n, k, replace=False))
+    kv = [(kk[kept], vv[kept]) for kk, vv in res.kv]  # every layer above the gate
+    ks = rng.standard_normal(k) * 2
+    out, _ = ref.decode_step(x[n], n, m, -1, kv, ks, store=ref.identity)
+    mask = np.concatenate([gain * np.log(1.0 / (1.0 + np.exp(-ks))), [0.0]])
+    hf = _hf_model(m, True)
+    with torch.no_grad():
+        o = hf(inputs_embeds=torch.from_numpy(x[n:n + 1])[None], past_key_values=_hf_cache(kv),
+               position_ids=torch.tensor([[n]]), attention_mask=torch.from_numpy(mask)[None, None, None],
+               use_cache=True).last_hidden_state[0, -1].numpy()
+    assert np.allclose(out, o, rtol=0, atol=2e-6)
+    # and the bias matters: without it the output moves by O(0.1)
+    plain, _ = ref.decode_step(x[n], n, m, -1, kv, np.full(k, np.inf), store=ref.identity)
+    assert np.max(np.abs(plain - out)) > 1e-2
