@@ -58,7 +58,8 @@ typedef enum {
   TG_OP_TOPK_SELECT = 1,
   TG_OP_COMPACT = 2,
   TG_OP_GATED_ATTN = 3,
-  TG_OP_PREFILL = 4
+  TG_OP_PREFILL = 4,
+  TG_OP_DECODE = 5  /* shape: d_model, heads, head_dim, d_ffn, k = kept prompt tokens, dtype */
 } tg_op;
 
 /* Sizes used to size a workspace; fields an op does not use are ignored. */
@@ -250,6 +251,38 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
                      const tg_kv* kv, void* const* hidden, void* ws, size_t ws_bytes,
                      tg_stream stream);
 
+/* ---- decode over the pruned cache ---------------------------------------
+ *
+ * tg_decode_step -- one generated token through every layer after a gated
+ * prefill. Generated tokens are never pruned ([TC] "TokenGate 提前筛选
+ * Token"): the token runs every layer and appends its k and v to every
+ * layer's cache. Layers at and below the gate hold the whole prompt's KV,
+ * layers above it only the kept tokens' KV, and in decoding the gate bias
+ * fixed at prefill acts as an additive mask over the cached keys ([TC]
+ * "TokenGate 的工程验证仍有限"). Above the gate the logit of cache row j is
+ * (q.k_j) / (sqrt(dh) tau_h) + gain_h logsigmoid(s_j) for the kept prompt
+ * tokens (rows j < k_kept) and (q.k_j) / (sqrt(dh) tau_h) for generated ones.
+ *   x [1, d] bf16: the token's input hidden state; pos: its position (the
+ *     prompt is 0..n-1, the t-th generated token has pos n + t).
+ *   kv: HOST array of n_layers caches, each k and v [cap_l, hkv, dh] bf16
+ *     (keys after RoPE, as tg_prefill writes them), rows in position order.
+ *   lens: HOST array of n_layers row counts before this step: n + t at or
+ *     below the gate, k + t above. The token's k and v go to row lens[l];
+ *     the caller sizes every cache for the rows it appends and advances lens.
+ *   scores [n] fp32 and kept_idx [k_kept] int32: tg_prefill's outputs for
+ *     an n-token prompt; the bias of upper-layer row j < k_kept is
+ *     logsigmoid(scores[kept_idx[j]]). An index outside [0, n) gets no bias
+ *     and sets bit 2 of the device error word. scores NULL: no gate bias.
+ *   out [1, d] bf16: the token's final-normed hidden state.
+ * bf16 and head_dim 128 only (TG_ERR_UNSUPPORTED otherwise); GQA groups of 1,
+ * 2, 4 or 8 query heads. Workspace: tg_workspace_size(TG_OP_DECODE) with
+ * shape.k = k_kept. Asynchronous on the stream; validates on the host first.
+ */
+tg_status tg_decode_step(const tg_model* model, const void* x, int64_t pos, int32_t gate_layer,
+                         const tg_kv* kv, const int64_t* lens, const float* scores, int64_t n,
+                         const int32_t* kept_idx, int64_t k_kept, void* out, void* ws,
+                         size_t ws_bytes, tg_stream stream);
+
 /* ---- launch tracing (optional) --------------------------------------------
  * Measurement aid with no counterpart on the pages (they report only
  * end-to-end prefill latency and memory). While tracing is on for a host
@@ -275,7 +308,9 @@ typedef enum {
   TG_K_F32_HELPER = 12,   /* fp32 SwiGLU / scorer tail                      */
   TG_K_GEMM_QKV = 13,     /* tcgen05 GEMM, fused qk-norm + RoPE + V^T epilogue */
   TG_K_ROPE_TABLE = 14,   /* cos/sin table of one set of positions           */
-  TG_K_COUNT = 15
+  TG_K_DECODE_GEMV = 15,  /* decode: matrix-vector product (+ norm / epilogue) */
+  TG_K_DECODE_ATTN = 16,  /* decode: split attention over a layer's cache      */
+  TG_K_COUNT = 17
 } tg_kernel;
 
 typedef struct {

@@ -31,7 +31,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 TG_OK, TG_ERR_INVALID_ARG, TG_ERR_UNSUPPORTED, TG_ERR_BUDGET, TG_ERR_WORKSPACE, TG_ERR_CUDA = range(6)
 TG_F32, TG_BF16 = 0, 1
-TG_OP_SCORE, TG_OP_TOPK_SELECT, TG_OP_COMPACT, TG_OP_GATED_ATTN, TG_OP_PREFILL = range(5)
+TG_OP_SCORE, TG_OP_TOPK_SELECT, TG_OP_COMPACT, TG_OP_GATED_ATTN, TG_OP_PREFILL, TG_OP_DECODE = range(6)
 
 _c_i32, _c_i64, _c_f32, _c_p, _c_sz = (ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
                                        ctypes.c_void_p, ctypes.c_size_t)
@@ -88,6 +88,9 @@ _attn = _sig("tg_gated_attn_prefill", _ci, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _
 _prefill = _sig("tg_prefill", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64, _c_i64, _c_i32,
                 _c_p, _c_p, _c_p, ctypes.POINTER(TgKV), ctypes.POINTER(_c_p), _c_p, _c_sz,
                 _c_p)
+_decode = _sig("tg_decode_step", _ci, ctypes.POINTER(TgModel), _c_p, _c_i64, _c_i32,
+               ctypes.POINTER(TgKV), ctypes.POINTER(_c_i64), _c_p, _c_i64, _c_p, _c_i64, _c_p, _c_p,
+               _c_sz, _c_p)
 _status_string = _sig("tg_status_string", ctypes.c_char_p, _ci)
 _last_cuda_error = _sig("tg_last_cuda_error", _ci)
 _device_error = _sig("tg_device_error", _ci, ctypes.POINTER(ctypes.c_uint32), _ci)
@@ -309,12 +312,42 @@ class Model:
                          _ptr(self.score.get("score_b1")), _ptr(self.score["score_w2"]),
                          _ptr(self.score.get("score_b2")))
 
+    def decode_workspace_size(self, k_kept: int) -> int:
+        return tg_workspace_size(TG_OP_DECODE, k=k_kept, d_model=self.d_model,
+                                 n_heads_q=self.n_heads_q, n_heads_kv=self.n_heads_kv,
+                                 head_dim=self.head_dim, d_ffn=self.d_ffn, dtype=self.dtype)
+
     def workspace_size(self, n: int, k: int, gate_layer: int) -> int:
         return tg_workspace_size(TG_OP_PREFILL, n=n, k=k, d_model=self.d_model,
                                  n_heads_q=self.n_heads_q, n_heads_kv=self.n_heads_kv,
                                  head_dim=self.head_dim, d_score=self.d_score, d_ffn=self.d_ffn,
                                  n_layers=len(self.layers), gate_layer=gate_layer,
                                  dtype=self.dtype)
+
+
+def tg_decode_step(model: Model, x, pos: int, gate_layer: int, kv: Sequence, lens: Sequence[int],
+                   scores=None, kept_idx=None, out=None, ws=None, stream=None):
+    """One generated token through every layer after a gated prefill.
+
+    x [d] or [1, d] bf16; kv: per-layer (k_cache, v_cache) [cap, hkv, dh]
+    bf16 with room for the new row; lens: per-layer rows before this step (the
+    token's k/v go to row lens[l]; the caller advances lens). scores [n] /
+    kept_idx [k] from tg_prefill give the upper layers' gate bias (None: no
+    bias). Returns out [1, d]."""
+    d = x.shape[-1]
+    if out is None:
+        out = torch.empty(1, d, dtype=x.dtype, device=x.device)
+    k_kept = 0 if kept_idx is None else int(kept_idx.numel())
+    ws = _ws(model.decode_workspace_size(k_kept), x.device, ws)
+    kv_c = (TgKV * len(model.layers))()
+    for i, (kc, vc) in enumerate(kv):
+        kv_c[i].k, kv_c[i].v = _ptr(kc), _ptr(vc)
+    lens_c = (_c_i64 * len(model.layers))(*[int(t) for t in lens])
+    n_scores = 0 if scores is None else int(scores.numel())
+    _check(_decode(ctypes.byref(model.c), _ptr(x), int(pos), gate_layer, kv_c, lens_c,
+                   _ptr(scores), n_scores, _ptr(kept_idx), k_kept, _ptr(out), _ptr(ws),
+                   ws.numel(), _stream(stream, x.device)), "tg_decode_step")
+    return out
 
 
 def tg_prefill(model: Model, x, protect, k: int, gate_layer: int, out=None, kept_idx=None,
@@ -349,9 +382,9 @@ def tg_prefill(model: Model, x, protect, k: int, gate_layer: int, out=None, kept
 
 
 __all__ = [
-    "tg_score", "tg_linear", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_prefill",
+    "tg_score", "tg_linear", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_prefill", "tg_decode_step",
     "tg_workspace_size", "tg_status_string", "tg_device_error", "tg_version", "Model",
     "TokenGateError", "LIB_PATH", "tg_trace_start", "tg_trace_stop", "TG_OK", "TG_ERR_INVALID_ARG", "TG_ERR_UNSUPPORTED",
     "TG_ERR_BUDGET", "TG_ERR_WORKSPACE", "TG_ERR_CUDA", "TG_F32", "TG_BF16", "TG_OP_SCORE",
-    "TG_OP_TOPK_SELECT", "TG_OP_COMPACT", "TG_OP_GATED_ATTN", "TG_OP_PREFILL",
+    "TG_OP_TOPK_SELECT", "TG_OP_COMPACT", "TG_OP_GATED_ATTN", "TG_OP_PREFILL", "TG_OP_DECODE",
 ]

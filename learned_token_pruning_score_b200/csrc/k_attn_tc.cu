@@ -59,11 +59,6 @@ struct Params {
   unsigned int* err;
 };
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -211,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < 128; ++i) rmax = fmaxf(rmax, x[i]);
       float alpha = 1.0f;
       if (rmax > m + kRescaleThresh || m == -INFINITY) {
-        alpha = ex2(m - rmax);  // 0 on the first tile
+        alpha = ex2_approx(m - rmax);  // 0 on the first tile
         l *= alpha;
         m = rmax;
       }
@@ -221,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float rsum = 0.f;
 #pragma unroll
       for (int i = 0; i < 128; ++i) {
-        x[i] = ex2(x[i] - m);
+        x[i] = ex2_approx(x[i] - m);
         rsum += x[i];
       }
       l += rsum;
@@ -594,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        scale2;
       float alpha = 1.0f;
       if (mx > m + kRescaleThresh || m == -INFINITY) {
-        alpha = ex2(m - mx);  // 0 on the first tile
+        alpha = ex2_approx(m - mx);  // 0 on the first tile
         l *= alpha;
         m = mx;
       }
@@ -618,8 +613,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (decltype(poly)::value && (i & 3) == 3) {
               a = exp2_poly3_x2(y);
             } else {
-              a.x = ex2(y.x);
-              a.y = ex2(y.y);
+              a.x = ex2_approx(y.x);
+              a.y = ex2_approx(y.y);
             }
             sp[i & 3] = fadd2(sp[i & 3], a);
             pk[i] = pack_bf16x2(a.x, a.y);

@@ -157,14 +157,9 @@ __global__ void __launch_bounds__(128) rope_qk(RopePrepArgs a) {
   const int pos = a.pos ? __ldg(a.pos + t) : static_cast<int>(t);
   if (threadIdx.x < kHalf) {
     const int i = threadIdx.x;
-    const double theta = exp2(-(2.0 * i / kDh) * log2(static_cast<double>(a.rope_base)));
-    const double ang = static_cast<double>(pos) * theta;
-    const double two_pi = 6.283185307179586476925286766559;
-    const double red = ang - two_pi * rint(ang * (1.0 / two_pi));
-    float sv, cv;
-    sincosf(static_cast<float>(red), &sv, &cv);
-    s_cos[i] = cv;
-    s_sin[i] = sv;
+    const float2 cs = rope_cos_sin(pos, i, kDh, a.rope_base);
+    s_cos[i] = cs.x;
+    s_sin[i] = cs.y;
   }
   if (threadIdx.x == 0 && a.s != nullptr) a.lsig_out[t] = logsigmoid_f(__ldg(a.s + t));
   __syncthreads();
@@ -217,13 +212,7 @@ __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int64_t T, in
   const int i = static_cast<int>(idx / T);
   const int64_t t = idx % T;
   const int p = pos ? __ldg(pos + t) : static_cast<int>(t);
-  const double theta = exp2(-(2.0 * i / dh) * log2(static_cast<double>(rope_base)));
-  const double ang = static_cast<double>(p) * theta;
-  const double two_pi = 6.283185307179586476925286766559;
-  const double red = ang - two_pi * rint(ang * (1.0 / two_pi));
-  float sv, cv;
-  sincosf(static_cast<float>(red), &sv, &cv);
-  cs[idx] = make_float2(cv, sv);
+  cs[idx] = rope_cos_sin(p, i, dh, rope_base);
 }
 
 // Gate-bias rows for the attention's extra K-step (see launch_bias_aug).

@@ -428,6 +428,70 @@ cudaError_t ffn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
   return gemm(g, dt, st);
 }
 
+// Workspace of one decode step (batch 1, bf16).
+struct DecodePlan {
+  __nv_bfloat16* h = nullptr;    // [d] the token's residual stream
+  __nv_bfloat16* qkv = nullptr;  // [(hq + 2 hkv) dh] projected q | k | v
+  __nv_bfloat16* o = nullptr;    // [hq dh] attention output
+  __nv_bfloat16* act = nullptr;  // [I] SwiGLU product
+  float* lsig = nullptr;         // [k_kept] logsigmoid of the kept prompt scores
+  float* part = nullptr;         // split softmax states of the attention
+  unsigned int* cnt = nullptr;   // [hkv] split counters
+  size_t bytes = 0;
+  DecodePlan(void* base, const tg_model& m, int64_t k_kept) {
+    Arena a(base);
+    const int64_t dh = m.head_dim, hq = m.n_heads_q, hkv = m.n_heads_kv;
+    h = static_cast<__nv_bfloat16*>(a.carve(size_t(m.d_model) * 2));
+    qkv = static_cast<__nv_bfloat16*>(a.carve(size_t(hq + 2 * hkv) * dh * 2));
+    o = static_cast<__nv_bfloat16*>(a.carve(size_t(hq) * dh * 2));
+    act = static_cast<__nv_bfloat16*>(a.carve(size_t(m.d_ffn > 0 ? m.d_ffn : 1) * 2));
+    lsig = static_cast<float*>(a.carve(size_t(k_kept > 0 ? k_kept : 1) * 4));
+    part = static_cast<float*>(
+        a.carve(size_t(hkv) * kDecodeMaxSplits * size_t(hq / (hkv > 0 ? hkv : 1)) * (dh + 2) * 4));
+    cnt = static_cast<unsigned int*>(a.carve(size_t(hkv) * 4));
+    bytes = a.used;
+  }
+};
+
+tg_status validate_decode(const tg_model* m, const void* x, int64_t pos, int gate_layer,
+                          const tg_kv* kv, const int64_t* lens, const float* scores, int64_t n,
+                          const int32_t* kept_idx, int64_t k_kept, const void* out) {
+  TG_CHECK(m != nullptr && m->layers != nullptr && x && out && kv && lens, TG_ERR_INVALID_ARG);
+  TG_CHECK(m->dtype == TG_BF16 || m->dtype == TG_F32, TG_ERR_UNSUPPORTED);
+  TG_CHECK(m->dtype == TG_BF16 && m->head_dim == 128, TG_ERR_UNSUPPORTED);
+  TG_CHECK(m->n_layers >= 1 && m->d_model > 0 && m->n_heads_q > 0 && m->n_heads_kv > 0,
+           TG_ERR_INVALID_ARG);
+  TG_CHECK(m->n_heads_q % m->n_heads_kv == 0, TG_ERR_INVALID_ARG);
+  const int group = m->n_heads_q / m->n_heads_kv;
+  TG_CHECK(group == 1 || group == 2 || group == 4 || group == 8, TG_ERR_UNSUPPORTED);
+  TG_CHECK(m->d_model % 8 == 0 && (m->d_ffn <= 0 || m->d_ffn % 8 == 0), TG_ERR_UNSUPPORTED);
+  TG_CHECK(gate_layer >= -1 && gate_layer < m->n_layers, TG_ERR_INVALID_ARG);
+  TG_CHECK(pos >= 0 && pos < (int64_t(1) << 31), TG_ERR_INVALID_ARG);
+  TG_CHECK(std::isfinite(m->norm_eps) && m->norm_eps >= 0.f && m->rope_base > 1.f,
+           TG_ERR_INVALID_ARG);
+  TG_CHECK(aligned16(x) && aligned16(out), TG_ERR_INVALID_ARG);
+  if (scores != nullptr) {
+    TG_CHECK(kept_idx != nullptr && n >= 1, TG_ERR_INVALID_ARG);
+    TG_CHECK(k_kept >= 1 && k_kept <= n, TG_ERR_BUDGET);
+  }
+  for (int l = 0; l < m->n_layers; ++l) {
+    const tg_layer& L = m->layers[l];
+    TG_CHECK(L.attn_norm && L.wqkv && L.wo, TG_ERR_INVALID_ARG);
+    TG_CHECK((L.q_norm == nullptr) == (L.k_norm == nullptr), TG_ERR_INVALID_ARG);
+    if (L.w_gate_up) TG_CHECK(L.w_down && L.ffn_norm && m->d_ffn > 0, TG_ERR_INVALID_ARG);
+    TG_CHECK(aligned16(L.wqkv) && aligned16(L.wo) && aligned16(L.attn_norm), TG_ERR_INVALID_ARG);
+    if (L.w_gate_up)
+      TG_CHECK(aligned16(L.w_gate_up) && aligned16(L.w_down) && aligned16(L.ffn_norm),
+               TG_ERR_INVALID_ARG);
+    TG_CHECK(kv[l].k != nullptr && kv[l].v != nullptr, TG_ERR_INVALID_ARG);
+    TG_CHECK(aligned16(kv[l].k) && aligned16(kv[l].v), TG_ERR_INVALID_ARG);
+    TG_CHECK(lens[l] >= 0 && lens[l] < (int64_t(1) << 31) - 1, TG_ERR_INVALID_ARG);
+    // above the gate the kept prompt tokens are the first k_kept cache rows
+    if (l > gate_layer && scores != nullptr) TG_CHECK(lens[l] >= k_kept, TG_ERR_INVALID_ARG);
+  }
+  return TG_OK;
+}
+
 tg_status validate_model(const tg_model* m, int64_t n, int64_t k, int gate_layer) {
   TG_CHECK(m != nullptr && m->layers != nullptr, TG_ERR_INVALID_ARG);
   TG_CHECK(m->dtype == TG_BF16 || m->dtype == TG_F32, TG_ERR_UNSUPPORTED);
@@ -488,6 +552,16 @@ size_t tg_workspace_size(tg_op op, const tg_shape* s) {
       m.d_ffn = s->d_ffn;
       m.d_score = s->d_score;
       return PrefillPlan(nullptr, m, s->n, s->k).bytes;
+    }
+    case TG_OP_DECODE: {
+      tg_model m{};
+      m.dtype = s->dtype;
+      m.d_model = s->d_model;
+      m.n_heads_q = s->n_heads_q;
+      m.n_heads_kv = s->n_heads_kv;
+      m.head_dim = s->head_dim;
+      m.d_ffn = s->d_ffn;
+      return DecodePlan(nullptr, m, s->k).bytes;
     }
   }
   return 0;
@@ -726,11 +800,94 @@ int32_t tg_trace_stop(tg_trace_record* out, int32_t cap) {
   return count;
 }
 
+tg_status tg_decode_step(const tg_model* model, const void* x, int64_t pos, int32_t gate_layer,
+                         const tg_kv* kv, const int64_t* lens, const float* scores, int64_t n,
+                         const int32_t* kept_idx, int64_t k_kept, void* out, void* ws,
+                         size_t ws_bytes, tg_stream stream) {
+  const tg_status vs =
+      validate_decode(model, x, pos, gate_layer, kv, lens, scores, n, kept_idx, k_kept, out);
+  if (vs != TG_OK) return vs;
+  const tg_model& m = *model;
+  DecodePlan P(nullptr, m, scores ? k_kept : 0);
+  TG_CHECK(ws != nullptr && ws_bytes >= P.bytes, TG_ERR_WORKSPACE);
+  P = DecodePlan(ws, m, scores ? k_kept : 0);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int d = m.d_model, dh = m.head_dim, hq = m.n_heads_q, hkv = m.n_heads_kv;
+  const int nqkv = (hq + 2 * hkv) * dh;
+
+  auto gemv = [&](const void* w, const __nv_bfloat16* xin, const float* gamma, __nv_bfloat16* y,
+                  int n_out, int k, int epi, int inter) {
+    DecGemvArgs a;
+    a.w = static_cast<const __nv_bfloat16*>(w);
+    a.x = xin;
+    a.gamma = gamma;
+    a.eps = m.norm_eps;
+    a.y = y;
+    a.n_out = n_out;
+    a.k = k;
+    a.inter = inter;
+    const double rows_w = epi == DEC_EPI_SWIGLU ? 2.0 * n_out : double(n_out);
+    return traced(TG_K_DECODE_GEMV, 1, 0.0, rows_w * k * 2 + 2.0 * k + 2.0 * n_out, st,
+                  [&] { return launch_decode_gemv(a, epi, gamma != nullptr, st); });
+  };
+
+  struct LayerTag {
+    explicit LayerTag(int l) { t_trace.layer = l; }
+    ~LayerTag() { t_trace.layer = -1; }
+  };
+  TG_TRY(cudaMemsetAsync(P.cnt, 0, size_t(hkv) * 4, st));
+  TG_TRY(copy_rows(P.h, x, size_t(d) * 2, 1, st));
+  if (scores)
+    TG_TRY(traced(TG_K_DECODE_ATTN, k_kept, 0.0, 12.0 * k_kept, st, [&] {
+      return launch_decode_lsig(scores, n, kept_idx, k_kept, P.lsig, st);
+    }));
+  for (int l = 0; l < m.n_layers; ++l) {
+    LayerTag tag(l);
+    const tg_layer& L = m.layers[l];
+    const bool upper = l > gate_layer;
+    TG_TRY(gemv(L.wqkv, P.h, L.attn_norm, P.qkv, nqkv, d, DEC_EPI_STORE, 0));
+    DecAttnArgs a;
+    a.qkv = P.qkv;
+    a.q_norm = L.q_norm;
+    a.k_norm = L.k_norm;
+    a.eps = m.norm_eps;
+    a.rope_base = m.rope_base;
+    a.pos = pos;
+    a.k_cache = static_cast<__nv_bfloat16*>(kv[l].k);
+    a.v_cache = static_cast<__nv_bfloat16*>(kv[l].v);
+    a.len = lens[l];
+    a.gain = upper ? L.gain : nullptr;
+    a.tau = upper ? L.tau : nullptr;
+    a.lsig = (upper && scores) ? P.lsig : nullptr;
+    a.k_kept = scores ? k_kept : 0;
+    a.hq = hq;
+    a.hkv = hkv;
+    a.part = P.part;
+    a.counters = P.cnt;
+    a.max_split = kDecodeMaxSplits;
+    a.out = P.o;
+    const int splits = decode_splits(lens[l] + 1, hkv);
+    const double kv_bytes = (2.0 * lens[l] + 2.0) * hkv * dh * 2;
+    TG_TRY(traced(TG_K_DECODE_ATTN, lens[l] + 1, 0.0, kv_bytes, st,
+                  [&] { return launch_decode_attn(a, splits, st); }));
+    TG_TRY(gemv(L.wo, P.o, nullptr, P.h, d, hq * dh, DEC_EPI_RESIDUAL, 0));
+    if (L.w_gate_up) {
+      TG_TRY(gemv(L.w_gate_up, P.h, L.ffn_norm, P.act, m.d_ffn, d, DEC_EPI_SWIGLU, m.d_ffn));
+      TG_TRY(gemv(L.w_down, P.act, nullptr, P.h, d, m.d_ffn, DEC_EPI_RESIDUAL, 0));
+    }
+  }
+  if (m.final_norm)
+    TG_TRY(rmsnorm(P.h, m.final_norm, m.norm_eps, 1, d, TG_BF16, out, st));
+  else
+    TG_TRY(copy_rows(out, P.h, size_t(d) * 2, 1, st));
+  return TG_OK;
+}
+
 const char* tg_kernel_name(int32_t kernel) {
   static const char* names[TG_K_COUNT] = {
       "copy", "rmsnorm", "gemm_tc_store", "gemm_tc_residual", "gemm_tc_swiglu", "gemm_tc_score",
       "rope_prep", "attention_tc", "select", "compact", "gemm_f32", "attention_f32", "f32_helper",
-      "gemm_tc_qkv", "rope_table"};
+      "gemm_tc_qkv", "rope_table", "decode_gemv", "decode_attention"};
   return (kernel >= 0 && kernel < TG_K_COUNT) ? names[kernel] : "unknown";
 }
 

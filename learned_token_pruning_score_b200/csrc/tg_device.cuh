@@ -451,6 +451,27 @@ __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   return r;
 }
 
+// 2^x on the MUFU unit (ex2.approx: relative error ~2^-22; ex2(-inf) = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// (cos, sin) of RoPE frequency i (of dh/2) at position pos: theta_i =
+// base^(-2i/dh), the angle pos * theta_i formed in fp64 and reduced mod 2 pi
+// before the fp32 sin/cos, so large positions keep their accuracy. Every
+// kernel that rotates q or k takes its angles from here.
+__device__ __forceinline__ float2 rope_cos_sin(int64_t pos, int i, int dh, float base) {
+  const double theta = exp2(-(2.0 * i / dh) * log2(static_cast<double>(base)));
+  const double ang = static_cast<double>(pos) * theta;
+  const double two_pi = 6.283185307179586476925286766559;
+  const double red = ang - two_pi * rint(ang * (1.0 / two_pi));
+  float sv, cv;
+  sincosf(static_cast<float>(red), &sv, &cv);
+  return make_float2(cv, sv);
+}
+
 // 2^x for a pair, on the FMA pipe instead of the MUFU unit, for x <= 8:
 // x = j + f with j = round(x) and |f| <= 1/2 (adding 1.5 * 2^23 leaves
 // round(x) in the low mantissa bits), a degree-3 polynomial for 2^f

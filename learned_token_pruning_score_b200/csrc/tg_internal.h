@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -150,6 +151,44 @@ struct AttnArgs {
 bool attn_tc_supported(const AttnArgs& a);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st);      // bf16, tcgen05
 cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t st); // fp32 SIMT
+
+// ---- decode (k_decode.cu): one generated token, batch 1, bf16, head_dim 128
+enum DecEpi { DEC_EPI_STORE = 0, DEC_EPI_RESIDUAL = 1, DEC_EPI_SWIGLU = 2 };
+struct DecGemvArgs {
+  const __nv_bfloat16* w;  // [n_out, k] (SWIGLU: [2 inter, k], gate rows then up rows)
+  const __nv_bfloat16* x;  // [k]
+  const float* gamma;      // [k] RMSNorm weight when the launch normalises x
+  float eps;
+  __nv_bfloat16* y;        // [n_out]: STORE y = Wx; RESIDUAL y += Wx; SWIGLU y = SiLU(Wg x) (Wu x)
+  int n_out, k, inter;
+};
+cudaError_t launch_decode_gemv(const DecGemvArgs& a, int epi, bool norm, cudaStream_t st);
+
+constexpr int kDecodeMaxSplits = 64;
+struct DecAttnArgs {
+  const __nv_bfloat16* qkv;  // [(hq + 2 hkv) * 128]: the token's projected q | k | v
+  const float* q_norm;       // [128] or null
+  const float* k_norm;
+  float eps, rope_base;
+  int64_t pos;               // the token's position
+  __nv_bfloat16* k_cache;    // [>= len + 1, hkv, 128], post-RoPE keys; row len is written
+  __nv_bfloat16* v_cache;
+  int64_t len;               // cached rows before this token
+  const float* gain;         // [hq] or null (no gate bias)
+  const float* tau;          // [hq] or null (1)
+  const float* lsig;         // [k_kept] logsigmoid of the kept prompt tokens' scores, or null
+  int64_t k_kept;            // cache rows 0..k_kept-1 carry the bias
+  int hq, hkv;
+  float* part;               // [hkv][kDecodeMaxSplits][group][130] split softmax states
+  unsigned int* counters;    // [hkv], zero before the launch; left zero after it
+  int max_split;
+  __nv_bfloat16* out;        // [hq * 128]
+};
+// Key splits per KV head for a cache of `rows` rows (plus the new one).
+int decode_splits(int64_t rows, int hkv);
+cudaError_t launch_decode_attn(const DecAttnArgs& a, int n_split, cudaStream_t st);
+cudaError_t launch_decode_lsig(const float* scores, int64_t n, const int32_t* kept_idx, int64_t k,
+                               float* lsig, cudaStream_t st);
 
 // ---- tensor maps (tg_tmap.cu)
 // 2-D bf16 tensor map, row-major [rows, cols] with row stride ld (elements),

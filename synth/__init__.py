@@ -231,3 +231,22 @@ def torch_hidden_states(w: Workload, seed: int, device: str = "cuda"):
         rows = torch.randperm(w.n, generator=g, device=device)[:m]
         x[rows] *= w.salient_scale
     return x.to(torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+
+
+def decode_state(w: Workload, rng: np.random.Generator, generated: int = 0) -> Dict[str, object]:
+    """Inputs of one decode step after a prefill of w.n tokens that kept w.k,
+    with `generated` tokens decoded since: per-layer caches of N(0, 1)
+    float32 keys and values (w.n + generated rows at or below the gate,
+    w.k + generated above), gate scores [w.n] ~ N(0, 2^2), an ascending kept
+    set of w.k tokens that holds the protected tail, the new token's hidden
+    state [d] ~ N(0, 1), and its position w.n + generated."""
+    lens = [(w.n if li <= w.gate_layer else w.k) + generated for li in range(w.n_layers)]
+    caches = [(rng.standard_normal((t, w.hkv, w.dh), dtype=np.float32),
+               rng.standard_normal((t, w.hkv, w.dh), dtype=np.float32)) for t in lens]
+    scores = (rng.standard_normal(w.n) * 2.0).astype(np.float32)
+    tail = np.arange(w.n - w.n_protect, w.n)
+    rest = rng.choice(w.n - w.n_protect, size=w.k - w.n_protect, replace=False)
+    kept = np.sort(np.concatenate([rest, tail])).astype(np.int32)
+    x = rng.standard_normal(w.d, dtype=np.float32)
+    return {"lens": lens, "caches": caches, "scores": scores, "kept_idx": kept, "x": x,
+            "pos": w.n + generated}
