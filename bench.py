@@ -146,14 +146,82 @@ def build_model(tg, torch, w, device):
                     score=score, final_norm=p["final_norm"], eps=w.eps, rope_base=w.rope_base)
 
 
-def kv_buffers(torch, w, k, device):
-    """Per-layer KV-cache outputs: n rows at/below the gate, k rows above."""
+def kv_buffers(torch, w, k, device, extra_rows=0):
+    """Per-layer KV caches: n rows at/below the gate, k rows above, plus
+    `extra_rows` of room for generated tokens."""
     out = []
     for li in range(w.n_layers):
-        rows = w.n if li <= w.gate_layer else k
+        rows = (w.n if li <= w.gate_layer else k) + extra_rows
         out.append((torch.empty(rows, w.hkv, w.dh, dtype=torch.bfloat16, device=device),
                     torch.empty(rows, w.hkv, w.dh, dtype=torch.bfloat16, device=device)))
     return out
+
+
+def decode_step_bytes(w, lens):
+    """Algorithmic HBM bytes of one decode step: every weight matrix once,
+    every cached k/v row once, the new k/v rows written (bf16)."""
+    per_layer_w = 2 * ((w.hq + 2 * w.hkv) * w.dh * w.d + w.d * w.hq * w.dh +
+                       (3 * w.inter * w.d if w.inter else 0))
+    kv = sum((2 * t + 2) * w.hkv * w.dh * 2 for t in lens)
+    return w.n_layers * per_layer_w + kv
+
+
+def decode_bench(tg, torch, model, w, kk, dense, steps, warmup, device, stream, pk):
+    """Prefill the prompt (gated at budget kk, or dense), then decode
+    warmup + steps tokens back to back over the caches it wrote. Returns the
+    timed steps' ms per token and the per-kernel split of a traced step."""
+    extra = warmup + steps + 1
+    kvb = kv_buffers(torch, w, w.n if dense else kk, device, extra_rows=extra)
+    x = synth.torch_hidden_states(w, seed=w.seed + 2000, device=str(device))
+    prot = torch.zeros(w.n, dtype=torch.uint8, device=device)
+    prot[w.n - w.n_protect:] = 1
+    k = w.n if dense else kk
+    scores = torch.empty(w.n, dtype=torch.float32, device=device)
+    _, kept, _ = tg.tg_prefill(model, x, prot, k, w.gate_layer, scores=scores, kv=kvb, stream=stream)
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed + 3000)
+    toks = torch.randn(extra, w.d, device=device, generator=g).to(torch.bfloat16)
+    lens0 = [(w.n if (dense or li <= w.gate_layer) else kk) for li in range(w.n_layers)]
+    out = torch.empty(1, w.d, dtype=torch.bfloat16, device=device)
+    ws = torch.empty(model.decode_workspace_size(k), dtype=torch.uint8, device=device)
+    sc, ki = (None, None) if dense else (scores, kept)
+
+    def step(i):
+        tg.tg_decode_step(model, toks[i], w.n + i, w.gate_layer, kvb, [t + i for t in lens0],
+                          scores=sc, kept_idx=ki, out=out, ws=ws, stream=stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(warmup, warmup + steps):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    tg.tg_trace_start(1 << 12)
+    step(warmup + steps)
+    torch.cuda.synchronize()
+    tr = tg.tg_trace_stop()
+    by = {}
+    for r in tr:
+        e = by.setdefault(r["kernel"], {"ms": 0.0, "bytes": 0.0, "launches": 0})
+        e["ms"] += r["ms"]
+        e["bytes"] += r["bytes"]
+        e["launches"] += 1
+    for e in by.values():
+        e["gbs"] = e["bytes"] / (e["ms"] / 1e3) / 1e9 if e["ms"] > 0 else 0.0
+    mid = [t + warmup + steps // 2 for t in lens0]
+    nbytes = decode_step_bytes(w, mid)
+    res = {"ms_per_token": ms, "tokens_per_s": 1e3 / ms, "bytes_per_step": nbytes,
+           "gbs": nbytes / (ms / 1e3) / 1e9, "hbm_frac": nbytes / (ms / 1e3) / 1e9 / pk["hbm"],
+           "cache_rows": {"at_or_below_gate": lens0[0], "above_gate": lens0[-1]},
+           "steps": steps, "warmup": warmup, "launches_per_step": len(tr), "by_kernel": by}
+    del kvb, ws, x, toks
+    torch.cuda.empty_cache()
+    return res
 
 
 def dense_model(tg, model):
@@ -498,6 +566,15 @@ def run_ours(args, rank, world, local_rank):
             g = extras[f"gated_k{kk}"]
             g["ttft_speedup_vs_dense"] = extras["dense"]["ttft_ms"] / g["ttft_ms"]
             g["peak_mem_reduction_vs_dense"] = extras["dense"]["peak_mem_gb"] / g["peak_mem_gb"]
+        # decode over the pruned cache (next to the dense cache) after the prefill
+        dec = decode_bench(tg, torch, model, w, k, False, 64, 8, device, stream, pk)
+        dec_d = decode_bench(tg, torch, dense_model(tg, model), w, w.n, True, 64, 8, device,
+                             stream, pk)
+        dec["dense_ms_per_token"] = dec_d["ms_per_token"]
+        dec["dense_gbs"] = dec_d["gbs"]
+        dec["dense_hbm_frac"] = dec_d["hbm_frac"]
+        dec["speedup_vs_dense"] = dec_d["ms_per_token"] / dec["ms_per_token"]
+        extras["decode"] = {"workload": f"{w.name} + decode (K={k}, batch 1)", **dec}
 
     # ---- CPU baseline: the oracle, rank 0 only, N = 1
     cpu = None
@@ -682,6 +759,17 @@ def run_case(args):
                               **{f"{i}_tflops": fl / (statistics.median(v) / 1e3) / 1e12
                                  for i, v in res.items()}}), flush=True)
         return 0
+    if args.case == "decode":
+        # a 2-layer Qwen3-1.7B-shaped model, gate at layer 0: one layer with an
+        # N-row cache, one with a K-row cache; `steps` decode steps after the prefill
+        wl = synth.shrink(w, n=t, k=max(128, t // 8), n_layers=2, gate_layer=0)
+        model = build_model(tg, torch, wl, device)
+        res = decode_bench(tg, torch, model, wl, wl.k, False, args.steps, 3, device,
+                           torch.cuda.current_stream(device), peaks())
+        assert tg.tg_device_error() == 0
+        print(json.dumps({"case": "decode", "rows": t, "steps": args.steps,
+                          "ms_per_token": res["ms_per_token"], "gbs": res["gbs"]}))
+        return 0
     if args.case == "attn":
         q = torch.randn(t, w.hq, w.dh, device=device, dtype=torch.bfloat16)
         kk = torch.randn(t, w.hkv, w.dh, device=device, dtype=torch.bfloat16)
@@ -724,7 +812,7 @@ def main():
     ap.add_argument("--quick", action="store_true", help="skip the other budgets / dense run")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--sweep", action="store_true")
-    ap.add_argument("--case", choices=["attn", "layer", "gemm"], default=None)
+    ap.add_argument("--case", choices=["attn", "layer", "gemm", "decode"], default=None)
     ap.add_argument("--rows", type=int, default=32768)
     ap.add_argument("--no-bias", action="store_true",
                     help="attn case: plain causal attention (as the layers below the gate)")

@@ -308,9 +308,8 @@ typedef enum {
   TG_K_F32_HELPER = 12,   /* fp32 SwiGLU / scorer tail                      */
   TG_K_GEMM_QKV = 13,     /* tcgen05 GEMM, fused qk-norm + RoPE + V^T epilogue */
   TG_K_ROPE_TABLE = 14,   /* cos/sin table of one set of positions           */
-  TG_K_DECODE_GEMV = 15,  /* decode: matrix-vector product (+ norm / epilogue) */
-  TG_K_DECODE_ATTN = 16,  /* decode: split attention over a layer's cache      */
-  TG_K_COUNT = 17
+  TG_K_DECODE_STEP = 15,  /* decode: one token through every layer (one launch) */
+  TG_K_COUNT = 16
 } tg_kernel;
 
 typedef struct {

@@ -436,7 +436,8 @@ struct DecodePlan {
   __nv_bfloat16* act = nullptr;  // [I] SwiGLU product
   float* lsig = nullptr;         // [k_kept] logsigmoid of the kept prompt scores
   float* part = nullptr;         // split softmax states of the attention
-  unsigned int* cnt = nullptr;   // [hkv] split counters
+  unsigned int* cnt = nullptr;   // [hkv] split counters, then [2] grid-barrier words
+  size_t cnt_bytes = 0;
   size_t bytes = 0;
   DecodePlan(void* base, const tg_model& m, int64_t k_kept) {
     Arena a(base);
@@ -448,7 +449,8 @@ struct DecodePlan {
     lsig = static_cast<float*>(a.carve(size_t(k_kept > 0 ? k_kept : 1) * 4));
     part = static_cast<float*>(
         a.carve(size_t(hkv) * kDecodeMaxSplits * size_t(hq / (hkv > 0 ? hkv : 1)) * (dh + 2) * 4));
-    cnt = static_cast<unsigned int*>(a.carve(size_t(hkv) * 4));
+    cnt_bytes = size_t(hkv + 2) * 4;
+    cnt = static_cast<unsigned int*>(a.carve(cnt_bytes));
     bytes = a.used;
   }
 };
@@ -461,6 +463,7 @@ tg_status validate_decode(const tg_model* m, const void* x, int64_t pos, int gat
   TG_CHECK(m->dtype == TG_BF16 && m->head_dim == 128, TG_ERR_UNSUPPORTED);
   TG_CHECK(m->n_layers >= 1 && m->d_model > 0 && m->n_heads_q > 0 && m->n_heads_kv > 0,
            TG_ERR_INVALID_ARG);
+  TG_CHECK(m->n_layers <= kDecodeMaxLayers, TG_ERR_UNSUPPORTED);
   TG_CHECK(m->n_heads_q % m->n_heads_kv == 0, TG_ERR_INVALID_ARG);
   const int group = m->n_heads_q / m->n_heads_kv;
   TG_CHECK(group == 1 || group == 2 || group == 4 || group == 8, TG_ERR_UNSUPPORTED);
@@ -812,74 +815,63 @@ tg_status tg_decode_step(const tg_model* model, const void* x, int64_t pos, int3
   TG_CHECK(ws != nullptr && ws_bytes >= P.bytes, TG_ERR_WORKSPACE);
   P = DecodePlan(ws, m, scores ? k_kept : 0);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int d = m.d_model, dh = m.head_dim, hq = m.n_heads_q, hkv = m.n_heads_kv;
-  const int nqkv = (hq + 2 * hkv) * dh;
+  const int hkv = m.n_heads_kv;
 
-  auto gemv = [&](const void* w, const __nv_bfloat16* xin, const float* gamma, __nv_bfloat16* y,
-                  int n_out, int k, int epi, int inter) {
-    DecGemvArgs a;
-    a.w = static_cast<const __nv_bfloat16*>(w);
-    a.x = xin;
-    a.gamma = gamma;
-    a.eps = m.norm_eps;
-    a.y = y;
-    a.n_out = n_out;
-    a.k = k;
-    a.inter = inter;
-    const double rows_w = epi == DEC_EPI_SWIGLU ? 2.0 * n_out : double(n_out);
-    return traced(TG_K_DECODE_GEMV, 1, 0.0, rows_w * k * 2 + 2.0 * k + 2.0 * n_out, st,
-                  [&] { return launch_decode_gemv(a, epi, gamma != nullptr, st); });
-  };
-
-  struct LayerTag {
-    explicit LayerTag(int l) { t_trace.layer = l; }
-    ~LayerTag() { t_trace.layer = -1; }
-  };
-  TG_TRY(cudaMemsetAsync(P.cnt, 0, size_t(hkv) * 4, st));
-  TG_TRY(copy_rows(P.h, x, size_t(d) * 2, 1, st));
-  if (scores)
-    TG_TRY(traced(TG_K_DECODE_ATTN, k_kept, 0.0, 12.0 * k_kept, st, [&] {
-      return launch_decode_lsig(scores, n, kept_idx, k_kept, P.lsig, st);
-    }));
+  DecStepParams p{};
   for (int l = 0; l < m.n_layers; ++l) {
-    LayerTag tag(l);
     const tg_layer& L = m.layers[l];
-    const bool upper = l > gate_layer;
-    TG_TRY(gemv(L.wqkv, P.h, L.attn_norm, P.qkv, nqkv, d, DEC_EPI_STORE, 0));
-    DecAttnArgs a;
-    a.qkv = P.qkv;
-    a.q_norm = L.q_norm;
-    a.k_norm = L.k_norm;
-    a.eps = m.norm_eps;
-    a.rope_base = m.rope_base;
-    a.pos = pos;
-    a.k_cache = static_cast<__nv_bfloat16*>(kv[l].k);
-    a.v_cache = static_cast<__nv_bfloat16*>(kv[l].v);
-    a.len = lens[l];
-    a.gain = upper ? L.gain : nullptr;
-    a.tau = upper ? L.tau : nullptr;
-    a.lsig = (upper && scores) ? P.lsig : nullptr;
-    a.k_kept = scores ? k_kept : 0;
-    a.hq = hq;
-    a.hkv = hkv;
-    a.part = P.part;
-    a.counters = P.cnt;
-    a.max_split = kDecodeMaxSplits;
-    a.out = P.o;
-    const int splits = decode_splits(lens[l] + 1, hkv);
-    const double kv_bytes = (2.0 * lens[l] + 2.0) * hkv * dh * 2;
-    TG_TRY(traced(TG_K_DECODE_ATTN, lens[l] + 1, 0.0, kv_bytes, st,
-                  [&] { return launch_decode_attn(a, splits, st); }));
-    TG_TRY(gemv(L.wo, P.o, nullptr, P.h, d, hq * dh, DEC_EPI_RESIDUAL, 0));
-    if (L.w_gate_up) {
-      TG_TRY(gemv(L.w_gate_up, P.h, L.ffn_norm, P.act, m.d_ffn, d, DEC_EPI_SWIGLU, m.d_ffn));
-      TG_TRY(gemv(L.w_down, P.act, nullptr, P.h, d, m.d_ffn, DEC_EPI_RESIDUAL, 0));
-    }
+    DecLayerPtrs& q = p.layer[l];
+    q.wqkv = static_cast<const __nv_bfloat16*>(L.wqkv);
+    q.wo = static_cast<const __nv_bfloat16*>(L.wo);
+    q.w_gate_up = static_cast<const __nv_bfloat16*>(L.w_gate_up);
+    q.w_down = static_cast<const __nv_bfloat16*>(L.w_down);
+    q.attn_norm = L.attn_norm;
+    q.ffn_norm = L.ffn_norm;
+    q.q_norm = L.q_norm;
+    q.k_norm = L.k_norm;
+    q.gain = L.gain;
+    q.tau = L.tau;
+    q.k_cache = static_cast<__nv_bfloat16*>(kv[l].k);
+    q.v_cache = static_cast<__nv_bfloat16*>(kv[l].v);
+    q.len = lens[l];
   }
-  if (m.final_norm)
-    TG_TRY(rmsnorm(P.h, m.final_norm, m.norm_eps, 1, d, TG_BF16, out, st));
-  else
-    TG_TRY(copy_rows(out, P.h, size_t(d) * 2, 1, st));
+  p.n_layers = m.n_layers;
+  p.d = m.d_model;
+  p.hq = m.n_heads_q;
+  p.hkv = hkv;
+  p.dffn = m.d_ffn;
+  p.gate_layer = gate_layer;
+  p.eps = m.norm_eps;
+  p.rope_base = m.rope_base;
+  p.final_norm = m.final_norm;
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.pos = pos;
+  p.scores = scores;
+  p.n_scores = n;
+  p.kept_idx = kept_idx;
+  p.k_kept = scores ? k_kept : 0;
+  p.h = P.h;
+  p.qkv = P.qkv;
+  p.o = P.o;
+  p.act = P.act;
+  p.lsig = P.lsig;
+  p.part = P.part;
+  p.merge_cnt = P.cnt;
+  p.bar = P.cnt + hkv;
+  p.grid = decode_grid();
+  p.n_split = decode_splits(hkv);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.err = device_error_word();
+  // algorithmic bytes: every weight once, every cached k/v row once, the new rows written
+  double bytes = 0.0;
+  const double qkvw = double(m.n_heads_q + 2 * hkv) * m.head_dim * m.d_model;
+  for (int l = 0; l < m.n_layers; ++l) {
+    bytes += 2.0 * (qkvw + double(m.d_model) * m.n_heads_q * m.head_dim);
+    if (m.layers[l].w_gate_up) bytes += 2.0 * 3.0 * double(m.d_ffn) * m.d_model;
+    bytes += (2.0 * lens[l] + 2.0) * hkv * m.head_dim * 2.0;
+  }
+  TG_TRY(cudaMemsetAsync(P.cnt, 0, P.cnt_bytes, st));
+  TG_TRY(traced(TG_K_DECODE_STEP, 1, 0.0, bytes, st, [&] { return launch_decode_step(p, st); }));
   return TG_OK;
 }
 
@@ -887,7 +879,7 @@ const char* tg_kernel_name(int32_t kernel) {
   static const char* names[TG_K_COUNT] = {
       "copy", "rmsnorm", "gemm_tc_store", "gemm_tc_residual", "gemm_tc_swiglu", "gemm_tc_score",
       "rope_prep", "attention_tc", "select", "compact", "gemm_f32", "attention_f32", "f32_helper",
-      "gemm_tc_qkv", "rope_table", "decode_gemv", "decode_attention"};
+      "gemm_tc_qkv", "rope_table", "decode_step"};
   return (kernel >= 0 && kernel < TG_K_COUNT) ? names[kernel] : "unknown";
 }
 

@@ -43,7 +43,9 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
 // pdl_wait() blocks until every prerequisite grid has completed and its
 // memory is visible. A kernel runs pdl_wait() before its first global-memory
 // access (read or write), and only its prologue (barrier init, TMEM
-// allocation, tensor-map prefetch) before that. Launched without the
+// allocation, tensor-map prefetch) before that, with one exception: reads
+// of model weights, which no kernel of the library writes (the decode GEMV
+// starts its weight stream before the wait). Launched without the
 // attribute, both are no-ops.
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

@@ -152,43 +152,51 @@ bool attn_tc_supported(const AttnArgs& a);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st);      // bf16, tcgen05
 cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t st); // fp32 SIMT
 
-// ---- decode (k_decode.cu): one generated token, batch 1, bf16, head_dim 128
-enum DecEpi { DEC_EPI_STORE = 0, DEC_EPI_RESIDUAL = 1, DEC_EPI_SWIGLU = 2 };
-struct DecGemvArgs {
-  const __nv_bfloat16* w;  // [n_out, k] (SWIGLU: [2 inter, k], gate rows then up rows)
-  const __nv_bfloat16* x;  // [k]
-  const float* gamma;      // [k] RMSNorm weight when the launch normalises x
-  float eps;
-  __nv_bfloat16* y;        // [n_out]: STORE y = Wx; RESIDUAL y += Wx; SWIGLU y = SiLU(Wg x) (Wu x)
-  int n_out, k, inter;
-};
-cudaError_t launch_decode_gemv(const DecGemvArgs& a, int epi, bool norm, cudaStream_t st);
-
-constexpr int kDecodeMaxSplits = 64;
-struct DecAttnArgs {
-  const __nv_bfloat16* qkv;  // [(hq + 2 hkv) * 128]: the token's projected q | k | v
-  const float* q_norm;       // [128] or null
+// ---- decode (k_decode.cu): one generated token, batch 1, bf16, head_dim 128.
+// One cooperative launch per step runs every layer (see k_decode.cu).
+constexpr int kDecodeMaxLayers = 64;
+constexpr int kDecodeMaxSplits = 128;
+struct DecLayerPtrs {
+  const __nv_bfloat16* wqkv;       // [(hq + 2 hkv) 128, d]
+  const __nv_bfloat16* wo;         // [d, hq 128]
+  const __nv_bfloat16* w_gate_up;  // [2 I, d] or null (no FFN)
+  const __nv_bfloat16* w_down;     // [d, I]
+  const float* attn_norm;
+  const float* ffn_norm;
+  const float* q_norm;             // [128] or null
   const float* k_norm;
-  float eps, rope_base;
-  int64_t pos;               // the token's position
-  __nv_bfloat16* k_cache;    // [>= len + 1, hkv, 128], post-RoPE keys; row len is written
+  const float* gain;               // [hq] or null; used above the gate
+  const float* tau;
+  __nv_bfloat16* k_cache;          // [>= len + 1, hkv, 128] post-RoPE keys; row len is written
   __nv_bfloat16* v_cache;
-  int64_t len;               // cached rows before this token
-  const float* gain;         // [hq] or null (no gate bias)
-  const float* tau;          // [hq] or null (1)
-  const float* lsig;         // [k_kept] logsigmoid of the kept prompt tokens' scores, or null
-  int64_t k_kept;            // cache rows 0..k_kept-1 carry the bias
-  int hq, hkv;
-  float* part;               // [hkv][kDecodeMaxSplits][group][130] split softmax states
-  unsigned int* counters;    // [hkv], zero before the launch; left zero after it
-  int max_split;
-  __nv_bfloat16* out;        // [hq * 128]
+  int64_t len;                     // cached rows before this token
 };
-// Key splits per KV head for a cache of `rows` rows (plus the new one).
-int decode_splits(int64_t rows, int hkv);
-cudaError_t launch_decode_attn(const DecAttnArgs& a, int n_split, cudaStream_t st);
-cudaError_t launch_decode_lsig(const float* scores, int64_t n, const int32_t* kept_idx, int64_t k,
-                               float* lsig, cudaStream_t st);
+struct DecStepParams {
+  DecLayerPtrs layer[kDecodeMaxLayers];
+  int n_layers, d, hq, hkv, dffn, gate_layer;
+  float eps, rope_base;
+  const float* final_norm;         // [d] or null
+  const __nv_bfloat16* x;          // [d] the token's input hidden state
+  int64_t pos;                     // its position
+  const float* scores;             // [n_scores] prefill gate scores, or null (no bias)
+  int64_t n_scores;
+  const int32_t* kept_idx;         // [k_kept]: upper-cache row j < k_kept is prompt token kept_idx[j]
+  int64_t k_kept;
+  __nv_bfloat16* h;                // [d] residual stream
+  __nv_bfloat16* qkv;              // [(hq + 2 hkv) 128]
+  __nv_bfloat16* o;                // [hq 128] attention output
+  __nv_bfloat16* act;              // [I] SwiGLU product
+  float* lsig;                     // [k_kept] logsigmoid of the kept prompt tokens' scores
+  float* part;                     // [hkv][kDecodeMaxSplits][hq / hkv][130] split softmax states
+  unsigned int* merge_cnt;         // [hkv] split counters, zero at launch
+  unsigned int* bar;               // [2] grid-barrier counter and abort flag, zero at launch
+  int grid, n_split;               // CTAs (one per SM) and key splits per KV head
+  __nv_bfloat16* out;              // [d]
+  unsigned int* err;
+};
+int decode_grid();
+int decode_splits(int hkv);
+cudaError_t launch_decode_step(const DecStepParams& p, cudaStream_t st);
 
 // ---- tensor maps (tg_tmap.cu)
 // 2-D bf16 tensor map, row-major [rows, cols] with row stride ld (elements),
