@@ -19,12 +19,16 @@
 //   O          h += W_o o
 //   gate/up    a = SiLU(W_g y) * (W_u y), y = RMSNorm(h)
 //   down       h += W_d a
-// Between arriving at a barrier and waiting on it, every warp already loads
-// its first weight chunk of the next stage (weights never change), so the
-// weight stream overlaps the barrier. Separate launches cost ~9 us each at
-// this size (launch, ramp-up, tail), more than most stages' own traffic.
-// Every barrier wait is bounded; a timeout sets the error word and an abort
-// flag that makes every CTA leave at its next barrier.
+// Weights never change, so they do not wait for the barriers: a producer
+// warp in every CTA streams the CTA's share of every weight matrix of the
+// step (its contiguous rows of each layer's QKV, O, gate/up and down, in that
+// order) with bulk copies into a ring of 32 KB shared-memory slots, running
+// ahead of the seven consumer warps by up to the ring's size. A single
+// stream across stages keeps HBM busy through the barriers and avoids the
+// per-stage ramp (separate launches cost ~9 us each at this size, more than
+// most stages' own traffic). Every wait is bounded; a timed-out grid barrier
+// sets the error word and an abort flag that makes every CTA leave at its
+// next barrier.
 #include "tg_device.cuh"
 #include "tg_internal.h"
 
@@ -64,6 +68,16 @@ __device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
 // Streaming 16-byte load (read once per step; evict first from L2).
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldcs(p); }
 
+// ---------------------------------------------------------------- roles
+constexpr int kConsumers = 224;               // 7 consumer warps (8 warps in all: 255 registers)
+constexpr int kConsumerWarps = kConsumers / 32;
+constexpr int kStepThreads = kConsumers + 32;  // + the producer warp
+constexpr int kSlotBytes = 32768;             // one ring slot
+constexpr int kMaxSlots = 6;
+
+// Consumer-only CTA barrier (the producer warp never joins).
+__device__ __forceinline__ void cons_sync() { named_bar_sync(1, kConsumers); }
+
 // ---------------------------------------------------------------- barrier
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   unsigned v;
@@ -76,8 +90,9 @@ __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
   return v;
 }
 
-// Grid barrier over a monotonic counter: arrival adds 1; the n-th barrier of
-// the launch completes when the counter reaches n * gridDim.x.
+// Grid barrier over a monotonic counter among the consumer warps of every
+// CTA: arrival adds 1; the n-th barrier of the launch completes when the
+// counter reaches n * gridDim.x.
 struct GridBar {
   unsigned* count;
   unsigned* abort;
@@ -86,12 +101,10 @@ struct GridBar {
 };
 
 __device__ __forceinline__ void bar_arrive(GridBar& b) {
-  __syncthreads();  // the CTA's writes of this stage are done
+  cons_sync();  // the CTA's writes of this stage are done
   b.target += gridDim.x;
-  if (threadIdx.x == 0) {
-    __threadfence();
+  if (threadIdx.x == 0)  // release: the CTA's writes (ordered by the bar.sync above) go first
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(b.count) : "memory");
-  }
 }
 
 // false: the launch is aborting (a wait somewhere ran out); leave the kernel.
@@ -113,146 +126,203 @@ __device__ __forceinline__ bool bar_wait(GridBar& b, int* s_ok) {
         }
       }
     }
-    __threadfence();
     *s_ok = ok;
   }
-  __syncthreads();
+  cons_sync();
   return *s_ok != 0;
 }
 
-// ---------------------------------------------------------------- stages
-constexpr int kStepThreads = 256;
-constexpr int kStepWarps = kStepThreads / 32;
-
+// ---------------------------------------------------------------- x staging
 // x [k] (written by the previous stage; read past L1) into shared memory as
 // bf16, RMSNorm'd with gamma when gamma is set (rounded like the prefill's
-// normed GEMM operand).
+// normed GEMM operand). Consumers only.
 __device__ void stage_x(const __nv_bfloat16* x, int k, const float* gamma, float eps, uint4* xs,
                         float* red) {
+  constexpr int kMaxVec = 5;  // 16-byte vectors per thread: k <= 8 * 5 * kConsumers
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nv = k / 8;
   const uint4* xg = reinterpret_cast<const uint4*>(x);
+  uint4 v[kMaxVec];
+#pragma unroll
+  for (int i = 0; i < kMaxVec; ++i) {
+    const int idx = tid + i * kConsumers;
+    v[i] = idx < nv ? __ldcg(xg + idx) : make_uint4(0u, 0u, 0u, 0u);
+  }
   if (gamma != nullptr) {
     float ss = 0.f;
-    for (int v = tid; v < nv; v += kStepThreads) {
-      float f[8];
-      unpack8(__ldcg(xg + v), f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ss = fmaf(f[i], f[i], ss);
+    for (int i = 0; i < kMaxVec; ++i) {
+      float f[8];
+      unpack8(v[i], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
     }
     ss = warp_sum32(ss);
     if (lane == 0) red[warp] = ss;
-    __syncthreads();
+    cons_sync();
     float tot = 0.f;
 #pragma unroll
-    for (int w = 0; w < kStepWarps; ++w) tot += red[w];
+    for (int w = 0; w < kConsumerWarps; ++w) tot += red[w];
     const float r = rsqrtf(tot / static_cast<float>(k) + eps);
-    for (int v = tid; v < nv; v += kStepThreads) {
-      float f[8];
-      unpack8(__ldcg(xg + v), f);
-      const float4 g0 = __ldg(reinterpret_cast<const float4*>(gamma) + 2 * v);
-      const float4 g1 = __ldg(reinterpret_cast<const float4*>(gamma) + 2 * v + 1);
-      uint4 o;
-      o.x = pack_bf16x2(f[0] * r * g0.x, f[1] * r * g0.y);
-      o.y = pack_bf16x2(f[2] * r * g0.z, f[3] * r * g0.w);
-      o.z = pack_bf16x2(f[4] * r * g1.x, f[5] * r * g1.y);
-      o.w = pack_bf16x2(f[6] * r * g1.z, f[7] * r * g1.w);
-      xs[v] = o;
+#pragma unroll
+    for (int i = 0; i < kMaxVec; ++i) {
+      const int idx = tid + i * kConsumers;
+      if (idx < nv) {
+        float f[8];
+        unpack8(v[i], f);
+        const float4 g0 = __ldg(reinterpret_cast<const float4*>(gamma) + 2 * idx);
+        const float4 g1 = __ldg(reinterpret_cast<const float4*>(gamma) + 2 * idx + 1);
+        uint4 o;
+        o.x = pack_bf16x2(f[0] * r * g0.x, f[1] * r * g0.y);
+        o.y = pack_bf16x2(f[2] * r * g0.z, f[3] * r * g0.w);
+        o.z = pack_bf16x2(f[4] * r * g1.x, f[5] * r * g1.y);
+        o.w = pack_bf16x2(f[6] * r * g1.z, f[7] * r * g1.w);
+        xs[idx] = o;
+      }
     }
   } else {
-    for (int v = tid; v < nv; v += kStepThreads) xs[v] = __ldcg(xg + v);
+#pragma unroll
+    for (int i = 0; i < kMaxVec; ++i) {
+      const int idx = tid + i * kConsumers;
+      if (idx < nv) xs[idx] = v[i];
+    }
   }
-  __syncthreads();
+  cons_sync();
 }
 
-// A matrix-vector stage: item i (0 <= i < n_items) is W row i (and, for
-// SwiGLU, row inter + i); rows are nv 16-byte vectors, read in chunks of kV
-// vectors per lane. Items go to warps round-robin across CTAs. A warp's
-// (item, chunk) sequence streams through a ring of kDepth chunks held in
-// registers: the first kDepth are loaded before the barrier that precedes
-// the stage (weights never change), and each consumed slot is refilled with
-// the chunk kDepth places ahead.
-struct GemvJob {
-  const uint4* w;
-  int nv, n_items, inter;
+// ---------------------------------------------------------------- weight stream
+// A matrix-vector block: this CTA's items [i0, i1) of a stage. Item i is W
+// row i (SwiGLU: rows i and inter + i). A chunk (one ring slot) holds `per`
+// consecutive items: `per` rows, or for SwiGLU `per` gate rows followed by
+// the matching `per` up rows.
+struct Block {
+  const uint8_t* w;
+  int row_bytes, i0, i1, inter, per;
+  bool two;
+  __device__ int n_chunks() const { return (i1 - i0 + per - 1) / per; }
 };
 
-template <int kV, bool kTwo>
-struct Chunk {
-  uint4 a[kV];
-  uint4 b[kTwo ? kV : 1];
+__device__ __forceinline__ Block make_block(const void* w, int k, int n_items, bool two, int inter,
+                                            int cta, int n_cta) {
+  Block b;
+  b.w = static_cast<const uint8_t*>(w);
+  b.row_bytes = k * 2;
+  b.i0 = static_cast<int>((static_cast<int64_t>(n_items) * cta) / n_cta);
+  b.i1 = static_cast<int>((static_cast<int64_t>(n_items) * (cta + 1)) / n_cta);
+  b.inter = inter;
+  b.two = two;
+  const int rows_per_slot = kSlotBytes / b.row_bytes;  // >= 1: k <= 8192
+  b.per = two ? (rows_per_slot / 2 > 0 ? rows_per_slot / 2 : 1) : rows_per_slot;
+  if (b.per > kConsumerWarps) b.per = kConsumerWarps;
+  return b;
+}
+
+// The blocks of layer li for this CTA, in stream order (a layer without an
+// FFN has two).
+__device__ __forceinline__ int layer_blocks(const DecStepParams& p, int li, int cta, int n_cta,
+                                            Block (&b)[4]) {
+  const DecLayerPtrs& L = p.layer[li];
+  const int nqkv = (p.hq + 2 * p.hkv) * kDh, qd = p.hq * kDh;
+  b[0] = make_block(L.wqkv, p.d, nqkv, false, 0, cta, n_cta);
+  b[1] = make_block(L.wo, qd, p.d, false, 0, cta, n_cta);
+  if (L.w_gate_up == nullptr) return 2;
+  b[2] = make_block(L.w_gate_up, p.d, p.dffn, true, p.dffn, cta, n_cta);
+  b[3] = make_block(L.w_down, p.dffn, p.d, false, 0, cta, n_cta);
+  return 4;
+}
+
+struct Ring {
+  uint8_t* slots;
+  uint64_t* full;
+  uint64_t* empty;
+  int n_slots;
 };
 
-template <int kV, bool kTwo, int kDepth>
-struct GemvStream {
-  Chunk<kV, kTwo> ring[kDepth];
-};
-
-// Loads sequence element q of warp wg (nothing past the warp's last item).
-template <int kV, bool kTwo>
-__device__ __forceinline__ void gemv_load(const GemvJob& j, int wg, int tw, int n_chunks, int q,
-                                          Chunk<kV, kTwo>& ch) {
+// Producer: every chunk of the step, in order. Returns when all are issued
+// (or a wait runs out) after the last copies have landed.
+__device__ void produce(const DecStepParams& p, const Ring& r, unsigned* abort) {
   const int lane = threadIdx.x & 31;
-  const int item = wg + (q / n_chunks) * tw, c = q % n_chunks;
-  const bool live = item < j.n_items;
-  const uint4* r0 = j.w + static_cast<int64_t>(live ? item : 0) * j.nv;
-  const uint4* r1 = kTwo ? j.w + static_cast<int64_t>(j.inter + (live ? item : 0)) * j.nv : r0;
-#pragma unroll
-  for (int u = 0; u < kV; ++u) {
-    const int v = c * 32 * kV + lane + 32 * u;
-    const bool in = live && v < j.nv;
-    ch.a[u] = in ? ld_stream(r0 + v) : make_uint4(0u, 0u, 0u, 0u);
-    if (kTwo) ch.b[u] = in ? ld_stream(r1 + v) : make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-
-template <int kV, bool kTwo, int kDepth>
-__device__ __forceinline__ void gemv_prefetch(const GemvJob& j, int wg, int tw,
-                                              GemvStream<kV, kTwo, kDepth>& st) {
-  const int n_chunks = (j.nv + 32 * kV - 1) / (32 * kV);
-#pragma unroll
-  for (int r = 0; r < kDepth; ++r) gemv_load<kV, kTwo>(j, wg, tw, n_chunks, r, st.ring[r]);
-}
-
-template <int kV, bool kTwo, int kDepth, class Epi>
-__device__ __forceinline__ void gemv_run(const GemvJob& j, const uint4* xs, int wg, int tw,
-                                         GemvStream<kV, kTwo, kDepth>& st, Epi epi) {
-  const int lane = threadIdx.x & 31;
-  const int n_chunks = (j.nv + 32 * kV - 1) / (32 * kV);
-  const int my_items = wg < j.n_items ? (j.n_items - wg + tw - 1) / tw : 0;
-  const int total = my_items * n_chunks;
-  float acc0 = 0.f, acc1 = 0.f;
-  for (int q0 = 0; q0 < total; q0 += kDepth) {
-#pragma unroll
-    for (int r = 0; r < kDepth; ++r) {
-      const int q = q0 + r;
-      if (q < total) {
-        const int c = q % n_chunks;
-#pragma unroll
-        for (int u = 0; u < kV; ++u) {
-          const int v = c * 32 * kV + lane + 32 * u;
-          if (v < j.nv) {
-            const uint4 xv = xs[v];
-            acc0 += dot8(st.ring[r].a[u], xv);
-            if (kTwo) acc1 += dot8(st.ring[r].b[u], xv);
-          }
-        }
-        if (q + kDepth < total) gemv_load<kV, kTwo>(j, wg, tw, n_chunks, q + kDepth, st.ring[r]);
-        if (c == n_chunks - 1) {
-          acc0 = warp_sum32(acc0);
-          if (kTwo) acc1 = warp_sum32(acc1);
-          if (lane == 0) epi(wg + (q / n_chunks) * tw, acc0, acc1);
-          acc0 = 0.f;
-          acc1 = 0.f;
+  uint32_t seq = 0;
+  bool ok = true;
+  for (int li = 0; li < p.n_layers && ok; ++li) {
+    Block b[4];
+    const int nb = layer_blocks(p, li, blockIdx.x, gridDim.x, b);
+    for (int bi = 0; bi < nb && ok; ++bi) {
+      const int nc = b[bi].n_chunks();
+      for (int c = 0; c < nc; ++c, ++seq) {
+        const int s = static_cast<int>(seq % r.n_slots);
+        const uint32_t ph = (seq / r.n_slots) & 1u;
+        if (lane == 0) ok = mbar_wait(&r.empty[s], ph ^ 1u, p.err);
+        ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+        if (!ok || ld_relaxed_u32(abort) != 0u) { ok = false; break; }
+        if (lane == 0) {
+          const Block& B = b[bi];
+          const int first = B.i0 + c * B.per;
+          const int cnt = (B.i1 - first) < B.per ? (B.i1 - first) : B.per;
+          const uint32_t part = static_cast<uint32_t>(cnt * B.row_bytes);
+          uint8_t* dst = r.slots + static_cast<size_t>(s) * kSlotBytes;
+          mbar_arrive_expect_tx(&r.full[s], B.two ? 2 * part : part);
+          bulk_load(dst, B.w + static_cast<int64_t>(first) * B.row_bytes, part, &r.full[s]);
+          if (B.two)
+            bulk_load(dst + part, B.w + static_cast<int64_t>(B.inter + first) * B.row_bytes, part,
+                      &r.full[s]);
         }
       }
+    }
+  }
+  // Drain: the last copies land before the CTA may exit.
+  if (lane == 0) {
+    const uint32_t n = seq < static_cast<uint32_t>(r.n_slots) ? seq : static_cast<uint32_t>(r.n_slots);
+    for (uint32_t i = 0; i < n; ++i) {
+      const uint32_t q = seq - 1 - i;
+      if (!mbar_wait(&r.full[q % r.n_slots], (q / r.n_slots) & 1u, p.err)) break;
+    }
+  }
+}
+
+// Consumers: one block. Item j (local) goes to warp j % 7; its chunk is
+// waited on, the row(s) dotted with x from shared memory, and the chunk's
+// empty barrier gets this warp's share of the 7 arrivals a chunk releases
+// (the warp of the chunk's first item also arrives for the warps that have
+// no item in it).
+template <class Epi>
+__device__ void consume(const Block& B, const Ring& r, uint32_t seq0, const uint4* xs, unsigned* err,
+                        unsigned* abort, Epi epi) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n_items = B.i1 - B.i0;
+  const int nv = B.row_bytes / 16;
+  for (int j = warp; j < n_items; j += kConsumerWarps) {
+    const int c = j / B.per, jj = j % B.per;
+    const uint32_t q = seq0 + static_cast<uint32_t>(c);
+    const int s = static_cast<int>(q % r.n_slots);
+    const int first = c * B.per;
+    const int cnt = (n_items - first) < B.per ? (n_items - first) : B.per;
+    if (!mbar_wait_warp(&r.full[s], (q / r.n_slots) & 1u, err)) {
+      if (lane == 0) atomicExch(abort, 1u);  // every CTA leaves at its next grid barrier
+      return;
+    }
+    const uint4* row = reinterpret_cast<const uint4*>(r.slots + static_cast<size_t>(s) * kSlotBytes +
+                                                      static_cast<size_t>(jj) * B.row_bytes);
+    const uint4* row2 = row + static_cast<size_t>(cnt) * nv;  // SwiGLU: the matching up row
+    float a0 = 0.f, a1 = 0.f;
+    for (int v = lane; v < nv; v += 32) {
+      const uint4 xv = xs[v];
+      a0 += dot8(row[v], xv);
+      if (B.two) a1 += dot8(row2[v], xv);
+    }
+    a0 = warp_sum32(a0);
+    if (B.two) a1 = warp_sum32(a1);
+    __syncwarp();
+    if (lane == 0) {
+      epi(B.i0 + j, a0, a1);
+      mbar_arrive_n(&r.empty[s], jj == 0 ? static_cast<uint32_t>(kConsumerWarps - cnt + 1) : 1u);
     }
   }
 }
 
 // ---------------------------------------------------------------- attention
-constexpr int kHalfWarps = kStepThreads / 16;  // one key per 16-lane group
-constexpr int kKeys = 4;                       // keys in flight per group
+constexpr int kHalfWarps = kConsumers / 16;  // one key per 16-lane group
+constexpr int kKeys = 8;                       // keys in flight per group
 
 template <int kGroup>
 struct AttnSmem {
@@ -267,13 +337,13 @@ struct AttnSmem {
 // One (KV head g, key split) unit of a layer's attention.
 template <int kGroup>
 __device__ void attn_unit(const DecStepParams& p, const DecLayerPtrs& L, bool upper, int g,
-                          int split, int n_split, AttnSmem<kGroup>& sm) {
+                          int split, int n_split, const float2 (&rcs)[2], AttnSmem<kGroup>& sm) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int head0 = g * kGroup;
   const __nv_bfloat16* qkv = p.qkv;
   // 1. The token's q (this group's heads) and k: qk-norm, RoPE at pos,
   //    rounded as the prefill stores them; v as projected.
-  for (int r = warp; r <= kGroup; r += kStepWarps) {
+  for (int r = warp; r <= kGroup; r += kConsumerWarps) {
     const bool is_q = r < kGroup;
     const __nv_bfloat16* src = qkv + (is_q ? (head0 + r) : (p.hq + g)) * kDh;
     const float* nw = is_q ? L.q_norm : L.k_norm;
@@ -295,7 +365,7 @@ __device__ void attn_unit(const DecStepParams& p, const DecLayerPtrs& L, bool up
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const int i = lane + 32 * q;
-      const float2 cs = rope_cos_sin(p.pos, i, kDh, p.rope_base);
+      const float2 cs = rcs[q];
       const __nv_bfloat16 olo = __float2bfloat16_rn(lo[q] * cs.x - hi[q] * cs.y);
       const __nv_bfloat16 ohi = __float2bfloat16_rn(hi[q] * cs.x + lo[q] * cs.y);
       if (is_q) {
@@ -308,7 +378,7 @@ __device__ void attn_unit(const DecStepParams& p, const DecLayerPtrs& L, bool up
     }
   }
   if (tid < kDh) sm.kv_new[1][tid] = __ldcg(qkv + (p.hq + p.hkv + g) * kDh + tid);
-  __syncthreads();
+  cons_sync();
 
   // 2. Split 0 appends the new row (no unit reads that row from memory in
   //    this step: the split holding it takes it from shared memory).
@@ -400,7 +470,7 @@ __device__ void attn_unit(const DecStepParams& p, const DecLayerPtrs& L, bool up
 #pragma unroll
     for (int e = 0; e < 8; ++e) sm.red_o[hw][h][sub * 8 + e] = o[h][e];
   }
-  __syncthreads();
+  cons_sync();
   if (tid < kGroup) {
     float mx = -INFINITY;
     for (int w = 0; w < kHalfWarps; ++w) mx = fmaxf(mx, sm.red_m[w][tid]);
@@ -410,7 +480,7 @@ __device__ void attn_unit(const DecStepParams& p, const DecLayerPtrs& L, bool up
     sm.cta_m[tid] = mx;
     sm.cta_l[tid] = ls;
   }
-  __syncthreads();
+  cons_sync();
   float* part = p.part + (static_cast<int64_t>(g) * kDecodeMaxSplits + split) * kGroup * (kDh + 2);
   if (tid < kDh) {
 #pragma unroll
@@ -430,9 +500,9 @@ __device__ void attn_unit(const DecStepParams& p, const DecLayerPtrs& L, bool up
 
   // 5. The last split of this KV head merges every split's state.
   __threadfence();
-  __syncthreads();
+  cons_sync();
   if (tid == 0) sm.is_last = atomicAdd(p.merge_cnt + g, 1u) == static_cast<unsigned>(n_split - 1);
-  __syncthreads();
+  cons_sync();
   if (!sm.is_last) return;
   __threadfence();
   if (tid < kDh) {
@@ -457,29 +527,49 @@ __device__ void attn_unit(const DecStepParams& p, const DecLayerPtrs& L, bool up
   if (tid == 0) p.merge_cnt[g] = 0u;  // ready for the next layer
 }
 
+
 // ---------------------------------------------------------------- the step
 template <int kGroup>
 __global__ void __launch_bounds__(kStepThreads, 1) dec_step(const __grid_constant__ DecStepParams p) {
-  extern __shared__ __align__(16) uint8_t dyn_smem[];
-  uint4* xs = reinterpret_cast<uint4*>(dyn_smem);  // a stage's input vector (bf16)
-  AttnSmem<kGroup>& asm_ = *reinterpret_cast<AttnSmem<kGroup>*>(dyn_smem);
-  __shared__ float red[kStepWarps];
+  extern __shared__ __align__(1024) uint8_t dyn_smem[];
+  __shared__ __align__(8) uint64_t full[kMaxSlots], empty[kMaxSlots];
+  __shared__ float red[kConsumerWarps];
   __shared__ int s_ok;
+  Ring ring{dyn_smem, full, empty, p.n_slots};
+  uint8_t* scratch = dyn_smem + static_cast<size_t>(p.n_slots) * kSlotBytes;  // xs | attention
+  uint4* xs = reinterpret_cast<uint4*>(scratch);
+  AttnSmem<kGroup>& asm_ = *reinterpret_cast<AttnSmem<kGroup>*>(scratch);
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int wg = warp * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x);  // spread over SMs
-  const int tw = static_cast<int>(gridDim.x) * kStepWarps;
-  const int d = p.d, qd = p.hq * kDh, nqkv = (p.hq + 2 * p.hkv) * kDh;
+  if (tid == 0) {
+    for (int s = 0; s < p.n_slots; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == kConsumerWarps) {  // ------------------------------ producer warp
+    produce(p, ring, p.bar + 1);
+    return;
+  }
+  // ------------------------------------------------------------ consumers
+  const int d = p.d, qd = p.hq * kDh;
   GridBar bar{p.bar, p.bar + 1, p.err, 0u};
+  // (cos, sin) of the token's position for head-dim pairs lane and lane + 32:
+  // the same in every layer
+  float2 rcs[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) rcs[q] = rope_cos_sin(p.pos, (tid & 31) + 32 * q, kDh, p.rope_base);
 
   // Stage 0: the residual stream starts as x; the kept tokens' bias inputs.
   if (blockIdx.x == 0) {
     const uint4* x4 = reinterpret_cast<const uint4*>(p.x);
     uint4* h4 = reinterpret_cast<uint4*>(p.h);
-    for (int v = tid; v < d / 8; v += kStepThreads) h4[v] = x4[v];
+    for (int v = tid; v < d / 8; v += kConsumers) h4[v] = x4[v];
   }
   if (p.scores != nullptr) {
-    for (int64_t j = static_cast<int64_t>(blockIdx.x) * kStepThreads + tid; j < p.k_kept;
-         j += static_cast<int64_t>(gridDim.x) * kStepThreads) {
+    for (int64_t j = static_cast<int64_t>(blockIdx.x) * kConsumers + tid; j < p.k_kept;
+         j += static_cast<int64_t>(gridDim.x) * kConsumers) {
       const int32_t i = __ldg(p.kept_idx + j);
       float b = 0.f;
       if (i < 0 || i >= p.n_scores) report_error(p.err, kErrIndexRange);
@@ -493,55 +583,41 @@ __global__ void __launch_bounds__(kStepThreads, 1) dec_step(const __grid_constan
     p.h[i] = __float2bfloat16_rn(__bfloat162float(__ldcg(p.h + i)) + a0);
   };
   auto swiglu = [&](int i, float a0, float a1) { p.act[i] = __float2bfloat16_rn(silu_f(a0) * a1); };
-  // Each block: arrive (the previous stage's writes are done), load the next
-  // stage's first weight chunk, wait, run the stage.
+  uint32_t seq = 0;  // chunks of the stream consumed before the current block
   for (int li = 0; li < p.n_layers; ++li) {
     const DecLayerPtrs& L = p.layer[li];
     const bool upper = li > p.gate_layer;
-    {  // QKV
-      const GemvJob j{reinterpret_cast<const uint4*>(L.wqkv), d / 8, nqkv, 0};
-      GemvStream<8, false, 4> c;
+    Block b[4];
+    const int nb = layer_blocks(p, li, blockIdx.x, gridDim.x, b);
+    // QKV
+    bar_arrive(bar);
+    if (!bar_wait(bar, &s_ok)) return;
+    stage_x(p.h, d, L.attn_norm, p.eps, xs, red);
+    consume(b[0], ring, seq, xs, p.err, p.bar + 1, store_qkv);
+    seq += static_cast<uint32_t>(b[0].n_chunks());
+    // attention
+    bar_arrive(bar);
+    if (!bar_wait(bar, &s_ok)) return;
+    if (static_cast<int>(blockIdx.x) < n_units)
+      attn_unit<kGroup>(p, L, upper, static_cast<int>(blockIdx.x) % p.hkv,
+                        static_cast<int>(blockIdx.x) / p.hkv, p.n_split, rcs, asm_);
+    // O projection + residual
+    bar_arrive(bar);
+    if (!bar_wait(bar, &s_ok)) return;
+    stage_x(p.o, qd, nullptr, p.eps, xs, red);
+    consume(b[1], ring, seq, xs, p.err, p.bar + 1, add_h);
+    seq += static_cast<uint32_t>(b[1].n_chunks());
+    if (nb == 4) {
       bar_arrive(bar);
-      gemv_prefetch(j, wg, tw, c);
       if (!bar_wait(bar, &s_ok)) return;
-      stage_x(p.h, d, L.attn_norm, p.eps, xs, red);
-      gemv_run(j, xs, wg, tw, c, store_qkv);
-    }
-    {  // attention
+      stage_x(p.h, d, L.ffn_norm, p.eps, xs, red);
+      consume(b[2], ring, seq, xs, p.err, p.bar + 1, swiglu);
+      seq += static_cast<uint32_t>(b[2].n_chunks());
       bar_arrive(bar);
       if (!bar_wait(bar, &s_ok)) return;
-      if (static_cast<int>(blockIdx.x) < n_units)
-        attn_unit<kGroup>(p, L, upper, static_cast<int>(blockIdx.x) % p.hkv,
-                          static_cast<int>(blockIdx.x) / p.hkv, p.n_split, asm_);
-    }
-    {  // O projection + residual
-      const GemvJob j{reinterpret_cast<const uint4*>(L.wo), qd / 8, d, 0};
-      GemvStream<8, false, 4> c;
-      bar_arrive(bar);
-      gemv_prefetch(j, wg, tw, c);
-      if (!bar_wait(bar, &s_ok)) return;
-      stage_x(p.o, qd, nullptr, p.eps, xs, red);
-      gemv_run(j, xs, wg, tw, c, add_h);
-    }
-    if (L.w_gate_up != nullptr) {
-      {  // gate/up + SwiGLU
-        const GemvJob j{reinterpret_cast<const uint4*>(L.w_gate_up), d / 8, p.dffn, p.dffn};
-        GemvStream<4, true, 4> c;
-        bar_arrive(bar);
-        gemv_prefetch(j, wg, tw, c);
-        if (!bar_wait(bar, &s_ok)) return;
-        stage_x(p.h, d, L.ffn_norm, p.eps, xs, red);
-        gemv_run(j, xs, wg, tw, c, swiglu);
-      }
-      {  // down + residual
-        const GemvJob j{reinterpret_cast<const uint4*>(L.w_down), p.dffn / 8, d, 0};
-        GemvStream<8, false, 4> c;
-        bar_arrive(bar);
-        gemv_prefetch(j, wg, tw, c);
-        if (!bar_wait(bar, &s_ok)) return;
-        stage_x(p.act, p.dffn, nullptr, p.eps, xs, red);
-        gemv_run(j, xs, wg, tw, c, add_h);
-      }
+      stage_x(p.act, p.dffn, nullptr, p.eps, xs, red);
+      consume(b[3], ring, seq, xs, p.err, p.bar + 1, add_h);
+      seq += static_cast<uint32_t>(b[3].n_chunks());
     }
   }
   bar_arrive(bar);
@@ -551,27 +627,33 @@ __global__ void __launch_bounds__(kStepThreads, 1) dec_step(const __grid_constan
     if (p.final_norm != nullptr) {
       stage_x(p.h, d, p.final_norm, p.eps, xs, red);
       uint4* out4 = reinterpret_cast<uint4*>(p.out);
-      for (int v = tid; v < d / 8; v += kStepThreads) out4[v] = xs[v];
+      for (int v = tid; v < d / 8; v += kConsumers) out4[v] = xs[v];
     } else {
-      for (int v = tid; v < d / 8; v += kStepThreads)
+      for (int v = tid; v < d / 8; v += kConsumers)
         reinterpret_cast<uint4*>(p.out)[v] = __ldcg(reinterpret_cast<const uint4*>(p.h) + v);
     }
   }
 }
 
 template <int kGroup>
-size_t step_smem(const DecStepParams& p) {
+size_t step_scratch(const DecStepParams& p) {
   const int kmax = p.d > p.dffn ? p.d : p.dffn;
   const int qd = p.hq * kDh;
   const size_t xs = static_cast<size_t>(kmax > qd ? kmax : qd) * 2;
   const size_t at = sizeof(AttnSmem<kGroup>);
-  return xs > at ? xs : at;
+  return ((xs > at ? xs : at) + 127) & ~size_t(127);
 }
 
 template <int kGroup>
-cudaError_t launch_step(const DecStepParams& p, cudaStream_t st) {
+cudaError_t launch_step(DecStepParams p, cudaStream_t st) {
   auto kern = dec_step<kGroup>;
-  const size_t smem = step_smem<kGroup>(p);
+  const size_t scratch = step_scratch<kGroup>(p);
+  const size_t limit = 227 * 1024 - 1024;  // dynamic shared memory per CTA, minus static
+  int slots = static_cast<int>((limit - scratch) / kSlotBytes);
+  if (slots > kMaxSlots) slots = kMaxSlots;
+  if (slots < 2) return cudaErrorInvalidConfiguration;
+  p.n_slots = slots;
+  const size_t smem = static_cast<size_t>(slots) * kSlotBytes + scratch;
   cudaError_t e = set_smem_attr_once(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int per_sm = 0;

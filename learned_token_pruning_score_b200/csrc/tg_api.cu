@@ -468,6 +468,9 @@ tg_status validate_decode(const tg_model* m, const void* x, int64_t pos, int gat
   const int group = m->n_heads_q / m->n_heads_kv;
   TG_CHECK(group == 1 || group == 2 || group == 4 || group == 8, TG_ERR_UNSUPPORTED);
   TG_CHECK(m->d_model % 8 == 0 && (m->d_ffn <= 0 || m->d_ffn % 8 == 0), TG_ERR_UNSUPPORTED);
+  // a stage's input vector is staged in registers, 4 x 16 bytes per thread
+  TG_CHECK(m->d_model <= 8192 && m->d_ffn <= 8192 && m->n_heads_q * 128 <= 8192,
+           TG_ERR_UNSUPPORTED);
   TG_CHECK(gate_layer >= -1 && gate_layer < m->n_layers, TG_ERR_INVALID_ARG);
   TG_CHECK(pos >= 0 && pos < (int64_t(1) << 31), TG_ERR_INVALID_ARG);
   TG_CHECK(std::isfinite(m->norm_eps) && m->norm_eps >= 0.f && m->rope_base > 1.f,

@@ -191,6 +191,7 @@ struct DecStepParams {
   unsigned int* merge_cnt;         // [hkv] split counters, zero at launch
   unsigned int* bar;               // [2] grid-barrier counter and abort flag, zero at launch
   int grid, n_split;               // CTAs (one per SM) and key splits per KV head
+  int n_slots;                     // weight-stream ring slots (set by the launcher)
   __nv_bfloat16* out;              // [d]
   unsigned int* err;
 };
