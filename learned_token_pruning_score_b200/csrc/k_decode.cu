@@ -23,7 +23,7 @@
 // warp in every CTA streams the CTA's share of every weight matrix of the
 // step (its contiguous rows of each layer's QKV, O, gate/up and down, in that
 // order) with bulk copies into a ring of 32 KB shared-memory slots, running
-// ahead of the seven consumer warps by up to the ring's size. A single
+// ahead of the eleven consumer warps by up to the ring's size. A single
 // stream across stages keeps HBM busy through the barriers and avoids the
 // per-stage ramp (separate launches cost ~9 us each at this size, more than
 // most stages' own traffic). Every wait is bounded; a timed-out grid barrier
@@ -69,7 +69,7 @@ __device__ __forceinline__ float dot8(const uint4& w, const uint4& x) {
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldcs(p); }
 
 // ---------------------------------------------------------------- roles
-constexpr int kConsumers = 224;               // 7 consumer warps (8 warps in all: 255 registers)
+constexpr int kConsumers = 352;               // 11 consumer warps (12 in all: 168 registers)
 constexpr int kConsumerWarps = kConsumers / 32;
 constexpr int kStepThreads = kConsumers + 32;  // + the producer warp
 constexpr int kSlotBytes = 32768;             // one ring slot
@@ -280,9 +280,9 @@ __device__ void produce(const DecStepParams& p, const Ring& r, unsigned* abort) 
   }
 }
 
-// Consumers: one block. Item j (local) goes to warp j % 7; its chunk is
+// Consumers: one block. Item j (local) goes to warp j % 11; its chunk is
 // waited on, the row(s) dotted with x from shared memory, and the chunk's
-// empty barrier gets this warp's share of the 7 arrivals a chunk releases
+// empty barrier gets this warp's share of the 11 arrivals a chunk releases
 // (the warp of the chunk's first item also arrives for the warps that have
 // no item in it).
 template <class Epi>
@@ -322,7 +322,7 @@ __device__ void consume(const Block& B, const Ring& r, uint32_t seq0, const uint
 
 // ---------------------------------------------------------------- attention
 constexpr int kHalfWarps = kConsumers / 16;  // one key per 16-lane group
-constexpr int kKeys = 8;                       // keys in flight per group
+constexpr int kKeys = 4;                       // keys in flight per group
 
 template <int kGroup>
 struct AttnSmem {
