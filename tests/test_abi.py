@@ -146,3 +146,53 @@ def test_device_error_without_a_device_is_a_cuda_error():
     with pytest.raises(tg.TokenGateError) as ei:
         tg.tg_device_error()
     assert ei.value.status == tg.TG_ERR_CUDA
+
+
+def _decode(model, kv, lens, gate=1, pos=1000, scores=None, n=0, kept=None, k_kept=0, ws_bytes=1 << 30,
+            x=BOGUS, out=BOGUS):
+    return tg._decode(model, x, pos, gate, kv, lens, scores, n, kept, k_kept, out, BOGUS, ws_bytes,
+                      None)
+
+
+def _bogus_kv(n_layers=2, **over):
+    kv = (tg.TgKV * n_layers)()
+    for i in range(n_layers):
+        kv[i].k, kv[i].v = 4096, 8192
+    lens = (ctypes.c_int64 * n_layers)(1000, 100)
+    return kv, lens
+
+
+def test_decode_validation():
+    m, keep = _bogus_model()
+    kv, lens = _bogus_kv()
+    big = 1 << 30
+    need = tg.tg_workspace_size(tg.TG_OP_DECODE, k=100, d_model=2048, n_heads_q=16, n_heads_kv=8,
+                                head_dim=128, d_ffn=6144, dtype=tg.TG_BF16)
+    assert 0 < need < big
+    assert _decode(None, kv, lens) == tg.TG_ERR_INVALID_ARG
+    assert _decode(ctypes.byref(m), None, lens) == tg.TG_ERR_INVALID_ARG
+    assert _decode(ctypes.byref(m), kv, None) == tg.TG_ERR_INVALID_ARG
+    assert _decode(ctypes.byref(m), kv, lens, gate=2) == tg.TG_ERR_INVALID_ARG   # gate past the stack
+    assert _decode(ctypes.byref(m), kv, lens, pos=-1) == tg.TG_ERR_INVALID_ARG
+    # bias inputs: kept_idx needed, k_kept within [1, n]
+    assert _decode(ctypes.byref(m), kv, lens, scores=BOGUS, n=1000, kept=None, k_kept=100) == \
+        tg.TG_ERR_INVALID_ARG
+    assert _decode(ctypes.byref(m), kv, lens, scores=BOGUS, n=1000, kept=BOGUS, k_kept=0) == \
+        tg.TG_ERR_BUDGET
+    assert _decode(ctypes.byref(m), kv, lens, scores=BOGUS, n=1000, kept=BOGUS, k_kept=1001) == \
+        tg.TG_ERR_BUDGET
+    # an upper cache shorter than the kept prompt rows
+    assert _decode(ctypes.byref(m), kv, lens, gate=0, scores=BOGUS, n=1000, kept=BOGUS,
+                   k_kept=200) == tg.TG_ERR_INVALID_ARG
+    assert _decode(ctypes.byref(m), kv, lens, ws_bytes=16) == tg.TG_ERR_WORKSPACE
+    unaligned = ctypes.c_void_p(4096 + 2)
+    assert _decode(ctypes.byref(m), kv, lens, x=unaligned) == tg.TG_ERR_INVALID_ARG
+    kv[1].v = None
+    assert _decode(ctypes.byref(m), kv, lens) == tg.TG_ERR_INVALID_ARG
+    kv, lens = _bogus_kv()
+    m2, keep2 = _bogus_model(head_dim=64)
+    assert _decode(ctypes.byref(m2), kv, lens) == tg.TG_ERR_UNSUPPORTED
+    m3, keep3 = _bogus_model(n_heads_q=24, n_heads_kv=8)  # GQA group of 3
+    assert _decode(ctypes.byref(m3), kv, lens) == tg.TG_ERR_UNSUPPORTED
+    m4, keep4 = _bogus_model(dtype=tg.TG_F32)
+    assert _decode(ctypes.byref(m4), kv, lens) == tg.TG_ERR_UNSUPPORTED
