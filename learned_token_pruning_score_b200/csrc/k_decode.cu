@@ -322,7 +322,7 @@ __device__ void consume(const Block& B, const Ring& r, uint32_t seq0, const uint
 
 // ---------------------------------------------------------------- attention
 constexpr int kHalfWarps = kConsumers / 16;  // one key per 16-lane group
-constexpr int kKeys = 4;                       // keys in flight per group
+constexpr int kKeys = 6;                       // keys in flight per group
 
 template <int kGroup>
 struct AttnSmem {
