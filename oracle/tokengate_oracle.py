@@ -60,6 +60,12 @@ Readings where the pages are silent (each one is listed in the design notes):
       its logits over the cached keys follow R2, with the kept prompt tokens'
       scores as the bias and no bias (logsigmoid = 0) on generated tokens'
       keys; tau applies to every key.
+  R9  Backward: the gradients of the gated attention with respect to q, k,
+      v, the gate scores s, the per-head gain and the per-head temperature,
+      for an upstream gradient of its output. The pages give only the path
+      (loss -> upper attention -> gate scores -> scorer); the formulas are
+      the plain chain rule of R2. Rounding to the storage dtype passes
+      gradients straight through.
 """
 
 from __future__ import annotations
@@ -290,6 +296,97 @@ def gated_attn_prefill(q, k, v, pos, s, gain, tau, rope_base, store=round_bf16):
     qr = store(rope(q, pos, rope_base))
     kr = store(rope(k, pos, rope_base))
     return store(gated_attention(qr, kr, np.asarray(v, dtype=F64), pos, s, gain, tau))
+
+
+# ---------------------------------------------------------------------------
+# Gated-attention backward (R9). The pages' point about the gate: the top-K
+# choice itself is discrete, but the kept tokens' scores stay in the
+# differentiable graph through the upper layers' attention bias, so the task
+# loss reaches the scorer along loss -> upper attention -> gate scores ->
+# scorer, and the per-head gain and temperature are learned with it ([TC]
+# "门控机制为评分网络建立梯度路径"; [AI] "可学习剪枝的机制设计").
+# ---------------------------------------------------------------------------
+
+
+def gated_attention_grads(q, k, v, pos, s, gain, tau, dout):
+    """Gradients of o = gated_attention(q, k, v, pos, s, gain, tau) for the
+    upstream gradient dout [T, Hq, dh] (q and k as they enter the logits,
+    i.e. already rotated). Returns (dq, dk, dv, ds, dgain, dtau), float64.
+
+    With a_ij = (q_i . k_j) / (sqrt(dh) tau_h) and b_j = logsigmoid(s_j):
+      l_ij = a_ij + gain_h b_j (pos_j <= pos_i), P = softmax_j(l), o_i = sum_j P_ij v_j
+      dP_ij = dout_i . v_j
+      dl_ij = P_ij (dP_ij - sum_j' P_ij' dP_ij')          (softmax Jacobian)
+      dq_i  = sum_j dl_ij k_j / (sqrt(dh) tau_h)
+      dk_j  = sum_{h in group} sum_i dl_ij q_i / (sqrt(dh) tau_h)
+      dv_j  = sum_{h in group} sum_i P_ij dout_i
+      dgain_h = sum_ij dl_ij b_j
+      dtau_h  = -sum_ij dl_ij a_ij / tau_h                 (d a_ij / d tau_h = -a_ij / tau_h)
+      ds_j  = sigmoid(-s_j) sum_h gain_h sum_i dl_ij       (d logsigmoid(x)/dx = sigmoid(-x))
+    s None means no bias: ds is None and dgain is zero; gain/tau None mean
+    0 and 1 (dgain and dtau are still returned).
+    """
+    q = np.asarray(q, dtype=F64)
+    k = np.asarray(k, dtype=F64)
+    v = np.asarray(v, dtype=F64)
+    dout = np.asarray(dout, dtype=F64)
+    t, hq, dh = q.shape
+    hkv = k.shape[1]
+    group = hq // hkv
+    gain_v = np.zeros(hq) if gain is None else np.asarray(gain, dtype=F64)
+    tau_v = np.ones(hq) if tau is None else np.asarray(tau, dtype=F64)
+    b = np.zeros(t) if s is None else logsigmoid(s)
+    p = np.asarray(pos, dtype=np.int64)
+    allowed = p[None, :] <= p[:, None]  # [query i, key j]
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    dgain = np.zeros(hq)
+    dtau = np.zeros(hq)
+    key_sum = np.zeros(t)  # sum_h gain_h sum_i dl_ij
+    for h in range(hq):
+        g = h // group
+        c = 1.0 / (math.sqrt(dh) * tau_v[h])
+        a = (q[:, h, :] @ k[:, g, :].T) * c
+        logits = np.where(allowed, a + gain_v[h] * b[None, :], -np.inf)
+        w = np.exp(logits - logits.max(axis=1, keepdims=True))
+        w = w / w.sum(axis=1, keepdims=True)
+        dp = dout[:, h, :] @ v[:, g, :].T
+        dl = w * (dp - (w * dp).sum(axis=1, keepdims=True))
+        dq[:, h, :] = c * (dl @ k[:, g, :])
+        dk[:, g, :] += c * (dl.T @ q[:, h, :])
+        dv[:, g, :] += w.T @ dout[:, h, :]
+        col = dl.sum(axis=0)
+        dgain[h] = col @ b
+        dtau[h] = -(dl * np.where(allowed, a, 0.0)).sum() / tau_v[h]
+        key_sum += gain_v[h] * col
+    ds = None if s is None else sigmoid(-np.asarray(s, dtype=F64)) * key_sum
+    return dq, dk, dv, ds, dgain, dtau
+
+
+def gated_attn_backward(q, k, v, pos, s, gain, tau, rope_base, dout, store=round_bf16):
+    """The standalone backward call, for the inputs of gated_attn_prefill
+    (q and k un-rotated): q and k are rotated and stored as in the forward,
+    the gradients are taken there, and those of q and k are rotated back
+    (RoPE at position p is orthogonal, so its transpose is RoPE at -p; the
+    storage rounding passes gradients straight through). dq, dk, dv are
+    stored in the compute dtype; ds, dgain, dtau as float32."""
+    qr = store(rope(q, pos, rope_base))
+    kr = store(rope(k, pos, rope_base))
+    dqr, dkr, dv, ds, dgain, dtau = gated_attention_grads(
+        qr, kr, np.asarray(v, dtype=F64), pos, s, gain, tau, dout)
+    neg = -np.asarray(pos, dtype=np.int64)
+    dq = store(rope(dqr, neg, rope_base))
+    dk = store(rope(dkr, neg, rope_base))
+    return (dq, dk, store(dv), None if ds is None else round_fp32(ds), round_fp32(dgain),
+            round_fp32(dtau))
+
+
+def attention_backward_flops(t: int, hq: int, dh: int) -> float:
+    """Algorithmic FLOPs of the causal attention backward: the five
+    [t x t x dh] products (S and dP recomputed, dV, dK, dQ), 2.5 times the
+    forward's 4 * dh * hq * t (t + 1) / 2."""
+    return 2.5 * attention_flops(t, hq, dh)
 
 
 # ---------------------------------------------------------------------------

@@ -378,6 +378,97 @@ def test_gated_attention_causal_by_original_position():
                        ref.gated_attention(q, k, v, np.arange(t), None, None, None), atol=1e-13)
 
 
+# ---------------------------------------------------------------- gated attention backward
+
+
+def _bwd_case(seed, t=6, hq=4, hkv=2, dh=8):
+    rng = np.random.default_rng(seed)
+    q, k, v = _qkv(seed, t=t, hq=hq, hkv=hkv, dh=dh)
+    pos = np.sort(rng.choice(60, t, replace=False))
+    s = rng.standard_normal(t) * 2
+    gain = rng.uniform(0.2, 2.0, hq)
+    tau = rng.uniform(0.5, 1.5, hq)
+    dout = rng.standard_normal((t, hq, dh))
+    return q, k, v, pos, s, gain, tau, dout
+
+
+def test_attention_backward_matches_finite_differences():
+    # Central differences of the (separately pinned) fp64 forward, RoPE
+    # included, for every input element: a dropped term, a wrong sign or a
+    # transposed operand anywhere in the backward fails here.
+    q, k, v, pos, s, gain, tau, dout = _bwd_case(21)
+    base = 1e4
+    ident = ref.identity
+
+    def loss(q_, k_, v_, s_, g_, t_):
+        o = ref.gated_attn_prefill(q_, k_, v_, pos, s_, g_, t_, base, store=ident)
+        return float((o * dout).sum())
+
+    args = [q, k, v, s, gain, tau]
+    got = ref.gated_attn_backward(q, k, v, pos, s, gain, tau, base, dout, store=ident)
+    eps = 1e-6
+    for a_idx, g in enumerate(got):
+        fd = np.zeros_like(args[a_idx])
+        flat = fd.reshape(-1)
+        for e in range(flat.size):
+            plus = [x.copy() for x in args]
+            minus = [x.copy() for x in args]
+            plus[a_idx].reshape(-1)[e] += eps
+            minus[a_idx].reshape(-1)[e] -= eps
+            flat[e] = (loss(*plus) - loss(*minus)) / (2 * eps)
+        assert np.allclose(g, fd, rtol=1e-6, atol=1e-7), a_idx
+
+
+def test_attention_backward_matches_torch_autograd():
+    # torch autograd through SDPA with the gate bias as an additive mask and
+    # tau folded into q (fp64 on the CPU): a library derivative of the same
+    # forward, for all six gradients.
+    q, k, v, pos, s, gain, tau, dout = _bwd_case(22, t=11, hq=6, hkv=3, dh=16)
+    t, hq, dh = q.shape
+    got = ref.gated_attention_grads(q, k, v, pos, s, gain, tau, dout)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    ts, tg, tt = (torch.tensor(x, requires_grad=True) for x in (s, gain, tau))
+    causal = torch.from_numpy(pos[None, :] <= pos[:, None])
+    lsig = torch.nn.functional.logsigmoid(ts)
+    outs = []
+    for h in range(hq):
+        g = h // (hq // 3)
+        mask = torch.where(causal, tg[h] * lsig[None, :],
+                           torch.tensor(-math.inf, dtype=torch.float64))
+        qh = tq[:, h] / tt[h]  # [t, dh]
+        o = torch.nn.functional.scaled_dot_product_attention(
+            qh[None, None], tk[:, g][None, None], tv[:, g][None, None], attn_mask=mask,
+            scale=1.0 / math.sqrt(dh))
+        outs.append(o[0, 0])
+    out = torch.stack(outs, dim=1)
+    (out * torch.from_numpy(dout)).sum().backward()
+    for mine, theirs in zip(got, (tq.grad, tk.grad, tv.grad, ts.grad, tg.grad, tt.grad)):
+        assert np.allclose(mine, theirs.numpy(), rtol=1e-9, atol=1e-11)
+
+
+def test_attention_backward_invariants_and_degenerate_cases():
+    q, k, v, pos, s, gain, tau, dout = _bwd_case(23, t=9)
+    # constant scores: each head's key sums of dl vanish (softmax rows sum to
+    # one), so sum_j ds_j = 0 and dgain = 0
+    sc = np.full(len(pos), 0.7)
+    _, _, _, ds, dgain, _ = ref.gated_attention_grads(q, k, v, pos, sc, gain, tau, dout)
+    assert abs(ds.sum()) < 1e-12 and np.all(np.abs(dgain) < 1e-12)
+    # tau divides the q.k term only: dtau_h = -(1/tau_h) sum_i q_i . dq_i
+    dq, _, _, _, _, dtau = ref.gated_attention_grads(q, k, v, pos, s, gain, tau, dout)
+    assert np.allclose(dtau, -np.einsum("thd,thd->h", q, dq) / tau, atol=1e-12)
+    # no bias: nothing flows to s, and gain has no effect
+    _, _, _, ds0, dgain0, _ = ref.gated_attention_grads(q, k, v, pos, None, gain, tau, dout)
+    assert ds0 is None and np.all(dgain0 == 0.0)
+    # one token: o_0 = v_0, so dv_0 = sum over the group of dout_0 and all
+    # other gradients are zero
+    dq1, dk1, dv1, ds1, dg1, dt1 = ref.gated_attention_grads(
+        q[:1], k[:1], v[:1], pos[:1], s[:1], gain, tau, dout[:1])
+    assert np.allclose(dv1[0, 0], dout[0, 0] + dout[0, 1]) and np.allclose(dv1[0, 1],
+                                                                           dout[0, 2] + dout[0, 3])
+    for z in (dq1, dk1, ds1, dg1, dt1):
+        assert np.all(np.abs(z) < 1e-12)
+
+
 # ---------------------------------------------------------------- full stack
 
 
