@@ -575,6 +575,12 @@ def run_ours(args, rank, world, local_rank):
         dec["dense_hbm_frac"] = dec_d["hbm_frac"]
         dec["speedup_vs_dense"] = dec_d["ms_per_token"] / dec["ms_per_token"]
         extras["decode"] = {"workload": f"{w.name} + decode (K={k}, batch 1)", **dec}
+        # backward of one gated attention layer over the K kept rows (the
+        # gradient path to the scorer, gain and temperature)
+        bwd = attn_backward_bench(tg, torch, w.hq, w.hkv, w.dh, k, 20, device)
+        bwd["frac_of_sustained_bf16"] = bwd["tflops_algorithmic"] / pk["bf16_sustained"]
+        extras["attn_backward"] = {"workload": f"one gated attention layer, K={k} rows, "
+                                               f"{w.hq}/{w.hkv} heads x {w.dh}", **bwd}
 
     # ---- CPU baseline: the oracle, rank 0 only, N = 1
     cpu = None
@@ -712,6 +718,67 @@ def run_sweep(args):
           flush=True)
 
 
+# ----------------------------------------------------------------- attention backward
+
+
+def attn_backward_bench(tg, torch, hq, hkv, dh, t, steps, device, bias=True, warmup=3):
+    """tg_gated_attn_backward over t kept rows (positions spread over 8t, gate
+    bias on): median ms per call of `steps` calls (CUDA events, inputs resident),
+    algorithmic TFLOP/s (the five causal [t x t x dh] products: 2.5 times the
+    forward's FLOPs), and a traced per-kernel split."""
+    g = torch.Generator(device=device).manual_seed(5)
+    q = torch.randn(t, hq, dh, device=device, dtype=torch.bfloat16, generator=g)
+    kk = torch.randn(t, hkv, dh, device=device, dtype=torch.bfloat16, generator=g)
+    v = torch.randn(t, hkv, dh, device=device, dtype=torch.bfloat16, generator=g)
+    dout = torch.randn(t, hq, dh, device=device, dtype=torch.bfloat16, generator=g)
+    pos = torch.sort(torch.randperm(8 * t, device=device, generator=g)[:t]).values.to(torch.int32)
+    s = torch.randn(t, device=device, generator=g) * 2 if bias else None
+    gain = torch.rand(hq, device=device, generator=g) * 2 if bias else None
+    tau = torch.rand(hq, device=device, generator=g) + 0.5 if bias else None
+    out, lse, o32 = tg.tg_gated_attn_forward(q, kk, v, pos, s, gain, tau)
+    grads = [torch.empty_like(q), torch.empty_like(kk), torch.empty_like(v),
+             torch.empty(t, device=device) if bias else None,
+             torch.empty(hq, device=device), torch.empty(hq, device=device)]
+    ws = torch.empty(tg.tg_workspace_size(tg.TG_OP_GATED_ATTN_BWD, k=t, n_heads_q=hq,
+                                          n_heads_kv=hkv, head_dim=dh),
+                     dtype=torch.uint8, device=device)
+
+    def run():
+        tg.tg_gated_attn_backward(q, kk, v, pos, out, lse, dout, s, gain, tau, out_f32=o32,
+                                  dq=grads[0],
+                                  dk=grads[1], dv=grads[2], ds=grads[3], dgain=grads[4],
+                                  dtau=grads[5], want_ds=bias, ws=ws)
+
+    for _ in range(warmup):
+        run()
+    ms = []
+    for _ in range(steps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        run()
+        b.record()
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b))
+    tg.tg_trace_start()
+    for _ in range(steps):
+        run()
+    torch.cuda.synchronize()
+    tr = tg.tg_trace_stop()
+    split = {}
+    for r in tr:
+        e = split.setdefault(r["kernel"], {"ms": 0.0, "flops": 0.0})
+        e["ms"] += r["ms"] / steps
+        e["flops"] += r["flops"] / steps
+    for e in split.values():
+        e["tflops_executed"] = e["flops"] / (e["ms"] / 1e3) / 1e12 if e["flops"] else None
+        del e["flops"]
+    fwd_flops = 4.0 * dh * hq * t * (t + 1) / 2.0
+    med = statistics.median(ms)
+    return {"ms": med, "tflops_algorithmic": 2.5 * fwd_flops / (med / 1e3) / 1e12,
+            "kernels": split, "heads": [hq, hkv], "bias": bias}
+
+
 # ----------------------------------------------------------------- profiling cases
 
 
@@ -770,6 +837,12 @@ def run_case(args):
         print(json.dumps({"case": "decode", "rows": t, "steps": args.steps,
                           "ms_per_token": res["ms_per_token"], "gbs": res["gbs"]}))
         return 0
+    if args.case == "attn_bwd":
+        res = attn_backward_bench(tg, torch, w.hq, w.hkv, w.dh, t, args.steps, device,
+                                  bias=not args.no_bias)
+        assert tg.tg_device_error() == 0
+        print(json.dumps({"case": "attn_bwd", "rows": t, "steps": args.steps, **res}))
+        return 0
     if args.case == "attn":
         q = torch.randn(t, w.hq, w.dh, device=device, dtype=torch.bfloat16)
         kk = torch.randn(t, w.hkv, w.dh, device=device, dtype=torch.bfloat16)
@@ -812,7 +885,7 @@ def main():
     ap.add_argument("--quick", action="store_true", help="skip the other budgets / dense run")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--sweep", action="store_true")
-    ap.add_argument("--case", choices=["attn", "layer", "gemm", "decode"], default=None)
+    ap.add_argument("--case", choices=["attn", "attn_bwd", "layer", "gemm", "decode"], default=None)
     ap.add_argument("--rows", type=int, default=32768)
     ap.add_argument("--no-bias", action="store_true",
                     help="attn case: plain causal attention (as the layers below the gate)")

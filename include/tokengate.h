@@ -59,7 +59,8 @@ typedef enum {
   TG_OP_COMPACT = 2,
   TG_OP_GATED_ATTN = 3,
   TG_OP_PREFILL = 4,
-  TG_OP_DECODE = 5  /* shape: d_model, heads, head_dim, d_ffn, k = kept prompt tokens, dtype */
+  TG_OP_DECODE = 5,  /* shape: d_model, heads, head_dim, d_ffn, k = kept prompt tokens, dtype */
+  TG_OP_GATED_ATTN_BWD = 6  /* shape: k = rows, heads, head_dim */
 } tg_op;
 
 /* Sizes used to size a workspace; fields an op does not use are ignored. */
@@ -175,6 +176,64 @@ tg_status tg_gated_attn_prefill(const void* q, const void* kk, const void* v, co
                                 int32_t hq, int32_t hkv, int32_t dh, float rope_base,
                                 tg_dtype dtype, void* out, void* ws, size_t ws_bytes,
                                 tg_stream stream);
+
+/*
+ * tg_gated_attn_forward -- tg_gated_attn_prefill that also writes what its
+ * backward takes:
+ *   lse [hq, k] fp32: lse[h][i] = log sum_{j <= i} exp(l_ij), natural log.
+ *   out_f32 [k, hq, dh] fp32 or NULL: the output before its rounding to
+ *   bf16. The backward forms D_i = dout_i . o_i; from the bf16 output that
+ *   product carries the output's rounding (2^-9 relative) into every
+ *   gradient of row i, so pass this when exact-to-fp32 gradients matter.
+ * bf16 only (dh == 128); other arguments, workspace (TG_OP_GATED_ATTN) and
+ * errors as tg_gated_attn_prefill. lse NULL, or out_f32 not 16-byte
+ * aligned, is TG_ERR_INVALID_ARG.
+ */
+tg_status tg_gated_attn_forward(const void* q, const void* kk, const void* v, const int32_t* pos,
+                                const float* s, const float* gain, const float* tau, int64_t k,
+                                int32_t hq, int32_t hkv, int32_t dh, float rope_base,
+                                tg_dtype dtype, void* out, float* lse, float* out_f32, void* ws,
+                                size_t ws_bytes, tg_stream stream);
+
+/*
+ * tg_gated_attn_backward -- gradients of tg_gated_attn_forward for an
+ * upstream gradient dout of its output. The top-K choice is discrete, but
+ * the kept tokens' scores stay in the differentiable graph through the
+ * attention bias, so the task loss reaches the scorer along loss -> upper
+ * attention -> gate scores -> scorer, and the per-head gain and temperature
+ * are learned with it ([TC] "门控机制为评分网络建立梯度路径"; [AI]
+ * "可学习剪枝的机制设计"). The formulas are the chain rule of the forward's
+ * logits (the pages give only the path):
+ *   P_ij = exp(l_ij - lse_i), dl_ij = P_ij (dout_i . v_j - dout_i . o_i)
+ *   dq_i = R_i^T sum_j dl_ij k'_j / (sqrt(dh) tau_h)
+ *   dk_j = R_j^T sum_{h in group} sum_i dl_ij q'_i / (sqrt(dh) tau_h)
+ *   dv_j = sum_{h in group} sum_i P_ij dout_i
+ *   ds_j = sigmoid(-s_j) sum_h gain_h sum_i dl_ij
+ *   dgain_h = sum_ij dl_ij logsigmoid(s_j),  dtau_h = -(1 / tau_h) sum_i q'_i . dq'_i
+ * where q', k' are q, k rotated by RoPE R at their positions (as in the
+ * forward) and dq' the gradient before the rotation back.
+ *   q, kk, v, pos, s, gain, tau, k, hq, hkv, dh, rope_base: the forward's
+ *   inputs, unchanged since that call.
+ *   out [k, hq, dh] bf16, out_f32 [k, hq, dh] fp32 or NULL, lse [hq, k]
+ *   fp32: the forward's outputs (D_i = dout_i . o_i is taken from out_f32
+ *   when given, else from out).
+ *   dout [k, hq, dh] bf16.
+ *   dq [k, hq, dh], dk [k, hkv, dh], dv [k, hkv, dh] bf16 (w.r.t. the
+ *   un-rotated q and kk); ds [k] fp32 or NULL (needs s); dgain [hq] fp32 or
+ *   NULL (0 when s is NULL); dtau [hq] fp32 or NULL.
+ * bf16 with dh == 128 only (else TG_ERR_UNSUPPORTED). All bf16 buffers and
+ * ws 16-byte aligned (else TG_ERR_INVALID_ARG). Workspace:
+ * tg_workspace_size(TG_OP_GATED_ATTN_BWD) with k, heads, head_dim. The
+ * result is deterministic (fixed summation orders, no atomics).
+ */
+tg_status tg_gated_attn_backward(const void* q, const void* kk, const void* v, const int32_t* pos,
+                                 const float* s, const float* gain, const float* tau, int64_t k,
+                                 int32_t hq, int32_t hkv, int32_t dh, float rope_base,
+                                 tg_dtype dtype, const void* out, const float* out_f32,
+                                 const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                 float* ds,
+                                 float* dgain, float* dtau, void* ws, size_t ws_bytes,
+                                 tg_stream stream);
 
 /*
  * tg_linear -- the backbone's projection GEMM, y = x . w^T (+ residual).
@@ -309,7 +368,11 @@ typedef enum {
   TG_K_GEMM_QKV = 13,     /* tcgen05 GEMM, fused qk-norm + RoPE + V^T epilogue */
   TG_K_ROPE_TABLE = 14,   /* cos/sin table of one set of positions           */
   TG_K_DECODE_STEP = 15,  /* decode: one token through every layer (one launch) */
-  TG_K_COUNT = 16
+  TG_K_ATTN_BWD_PREP = 16,   /* backward: transposes, lse in log2 units, D = dout . o */
+  TG_K_ATTN_BWD_DKDV = 17,   /* backward: dK, dV and the per-key sums of dl (tcgen05) */
+  TG_K_ATTN_BWD_DQ = 18,     /* backward: dQ and q . dq (tcgen05)                   */
+  TG_K_ATTN_BWD_FINAL = 19,  /* backward: ds, dgain, dtau                           */
+  TG_K_COUNT = 20
 } tg_kernel;
 
 typedef struct {

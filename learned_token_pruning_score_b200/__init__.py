@@ -31,7 +31,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 TG_OK, TG_ERR_INVALID_ARG, TG_ERR_UNSUPPORTED, TG_ERR_BUDGET, TG_ERR_WORKSPACE, TG_ERR_CUDA = range(6)
 TG_F32, TG_BF16 = 0, 1
-TG_OP_SCORE, TG_OP_TOPK_SELECT, TG_OP_COMPACT, TG_OP_GATED_ATTN, TG_OP_PREFILL, TG_OP_DECODE = range(6)
+(TG_OP_SCORE, TG_OP_TOPK_SELECT, TG_OP_COMPACT, TG_OP_GATED_ATTN, TG_OP_PREFILL, TG_OP_DECODE,
+ TG_OP_GATED_ATTN_BWD) = range(7)
 
 _c_i32, _c_i64, _c_f32, _c_p, _c_sz = (ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
                                        ctypes.c_void_p, ctypes.c_size_t)
@@ -85,6 +86,11 @@ _compact = _sig("tg_compact", _ci, _c_p, _c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i3
                 _c_p, _c_p, _c_p)
 _attn = _sig("tg_gated_attn_prefill", _ci, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i64,
              _c_i32, _c_i32, _c_i32, _c_f32, _ci, _c_p, _c_p, _c_sz, _c_p)
+_attn_fwd = _sig("tg_gated_attn_forward", _ci, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i64,
+                 _c_i32, _c_i32, _c_i32, _c_f32, _ci, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p)
+_attn_bwd = _sig("tg_gated_attn_backward", _ci, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i64,
+                 _c_i32, _c_i32, _c_i32, _c_f32, _ci, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p,
+                 _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p)
 _prefill = _sig("tg_prefill", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64, _c_i64, _c_i32,
                 _c_p, _c_p, _c_p, ctypes.POINTER(TgKV), ctypes.POINTER(_c_p), _c_p, _c_sz,
                 _c_p)
@@ -275,6 +281,56 @@ def tg_gated_attn_prefill(q, k, v, pos, s=None, gain=None, tau=None, rope_base: 
     return out
 
 
+def tg_gated_attn_forward(q, k, v, pos, s=None, gain=None, tau=None, rope_base: float = 1e6,
+                          out=None, lse=None, out_f32=None, want_f32: bool = True, ws=None,
+                          stream=None):
+    """tg_gated_attn_prefill plus the per-row log-sum-exp [hq, t] and (when
+    want_f32) the output before rounding [t, hq, dh] fp32, both of which
+    tg_gated_attn_backward takes. Returns (out, lse, out_f32 or None)."""
+    t, hq, dh = q.shape
+    hkv = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(hq, t, dtype=torch.float32, device=q.device)
+    if out_f32 is None and want_f32:
+        out_f32 = torch.empty(t, hq, dh, dtype=torch.float32, device=q.device)
+    dt = _dt(q)
+    need = tg_workspace_size(TG_OP_GATED_ATTN, k=t, n_heads_q=hq, n_heads_kv=hkv, head_dim=dh,
+                             dtype=dt)
+    ws = _ws(need, q.device, ws)
+    _check(_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), _ptr(s), _ptr(gain), _ptr(tau), t, hq,
+                     hkv, dh, rope_base, dt, _ptr(out), _ptr(lse), _ptr(out_f32), _ptr(ws),
+                     ws.numel(), _stream(stream, q.device)), "tg_gated_attn_forward")
+    return out, lse, out_f32
+
+
+def tg_gated_attn_backward(q, k, v, pos, out, lse, dout, s=None, gain=None, tau=None,
+                           rope_base: float = 1e6, out_f32=None, dq=None, dk=None, dv=None,
+                           ds=None, dgain=None, dtau=None, want_ds: bool = True, ws=None,
+                           stream=None):
+    """Gradients (dq, dk, dv, ds, dgain, dtau) of tg_gated_attn_forward for dout.
+    ds is None when s is None (or want_ds is False)."""
+    t, hq, dh = q.shape
+    hkv = k.shape[1]
+    dev = q.device
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if ds is None and s is not None and want_ds:
+        ds = torch.empty(t, dtype=torch.float32, device=dev)
+    dgain = torch.empty(hq, dtype=torch.float32, device=dev) if dgain is None else dgain
+    dtau = torch.empty(hq, dtype=torch.float32, device=dev) if dtau is None else dtau
+    need = tg_workspace_size(TG_OP_GATED_ATTN_BWD, k=t, n_heads_q=hq, n_heads_kv=hkv,
+                             head_dim=dh, dtype=_dt(q))
+    ws = _ws(need, dev, ws)
+    _check(_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), _ptr(s), _ptr(gain), _ptr(tau), t, hq,
+                     hkv, dh, rope_base, _dt(q), _ptr(out), _ptr(out_f32), _ptr(lse), _ptr(dout),
+                     _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds), _ptr(dgain), _ptr(dtau), _ptr(ws),
+                     ws.numel(), _stream(stream, dev)), "tg_gated_attn_backward")
+    return dq, dk, dv, ds, dgain, dtau
+
+
 @dataclass
 class Model:
     """Device tensors of a decoder stack plus the ctypes view tg_prefill takes.
@@ -382,9 +438,10 @@ def tg_prefill(model: Model, x, protect, k: int, gate_layer: int, out=None, kept
 
 
 __all__ = [
-    "tg_score", "tg_linear", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_prefill", "tg_decode_step",
+    "tg_score", "tg_linear", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_gated_attn_forward", "tg_gated_attn_backward", "tg_prefill", "tg_decode_step",
     "tg_workspace_size", "tg_status_string", "tg_device_error", "tg_version", "Model",
     "TokenGateError", "LIB_PATH", "tg_trace_start", "tg_trace_stop", "TG_OK", "TG_ERR_INVALID_ARG", "TG_ERR_UNSUPPORTED",
     "TG_ERR_BUDGET", "TG_ERR_WORKSPACE", "TG_ERR_CUDA", "TG_F32", "TG_BF16", "TG_OP_SCORE",
     "TG_OP_TOPK_SELECT", "TG_OP_COMPACT", "TG_OP_GATED_ATTN", "TG_OP_PREFILL", "TG_OP_DECODE",
+    "TG_OP_GATED_ATTN_BWD",
 ]

@@ -1,0 +1,862 @@
+// k_attn_bwd.cu -- backward of the token-gated causal GQA attention on the
+// 5th-generation tensor cores (sm_100a): bf16 operands, fp32 accumulation.
+//
+// Forward (kept rows i, j in compacted order; positions ascend with the row):
+//   l_ij = a_ij + gain_h b_j,  a_ij = (q_i . k_j) / (sqrt(dh) tau_h),  b_j = logsigmoid(s_j)
+//   P = softmax_j(l_ij) over j <= i,  o_i = sum_j P_ij v_j
+// Backward for the upstream gradient dO, with lse_i = log sum_j exp(l_ij)
+// saved by the forward and D_i = dO_i . o_i:
+//   P_ij = exp(l_ij - lse_i),  dP_ij = dO_i . v_j,  dl_ij = P_ij (dP_ij - D_i)
+//   dq_i = sum_j dl_ij k_j / (sqrt(dh) tau_h)
+//   dk_j = sum_{h in group} sum_i dl_ij q_i / (sqrt(dh) tau_h),  dv_j = sum_{h in group} sum_i P_ij dO_i
+//   C_hj = sum_i dl_ij:  ds_j = sigmoid(-s_j) sum_h gain_h C_hj,  dgain_h = sum_j b_j C_hj
+//   dtau_h = -(1 / tau_h) sum_i q_i . dq_i
+// The top-K choice is discrete, but the kept tokens' scores stay in the
+// differentiable graph through this bias, which is how the task loss reaches
+// the scorer; the per-head gain and temperature are learned along with it
+// (Tencent Cloud article "TokenGate：端到端可训练的 Token 剪枝机制，让大模型
+// Prefill 提速 11.3 倍", section "门控机制为评分网络建立梯度路径";
+// ai.866data.com article "让大模型学会"略读"…", section "可学习剪枝的机制设计").
+// q and k are rotated (RoPE at the original positions) before the logits;
+// their gradients are rotated back with the transposed rotation.
+//
+// Kernels, in stream order:
+//   bwd_prep   Q^T, K^T, dO^T as [head, dh, t_pad] (the K-major B operands
+//              of the products that contract over rows), lse in log2 units,
+//              D (from the forward's fp32 output when given: the bf16 output
+//              carries a rounding of 2^-9 that D would pass on to every
+//              dl_ij of the row), and the zero-padded bias row logsigmoid(s).
+//   bwd_dkdv   one CTA per (128-key tile, KV head). For each query head of
+//              the group and each query tile at or after the key tile:
+//                S^T = K Q^T and dP^T = V dO^T into TMEM (128 columns each);
+//                one thread per key row forms P^T and dS^T (dS^T scaled by
+//                1 / (sqrt(dh) tau_h)) and writes them back as packed bf16
+//                over S^T and dP^T; dV += P^T dO and dK += dS^T Q with A read
+//                from TMEM. C_hj is a thread-local sum. (Keeping K and V in
+//                TMEM to double-buffer S^T and dP^T leaves room only for
+//                32-query products, whose MMA instructions are too short to
+//                keep the tensor pipe fed: measured slower.)
+//   bwd_dq     one CTA per (128-query tile, query head); Q and dO in TMEM.
+//              Keys up to the diagonal stream through a 3-stage ring (64 per
+//              stage): S = Q K^T and dP = dO V^T into one of two TMEM
+//              buffers, dS written back over S, dQ += dS K. Then dq (scaled,
+//              rotated back) and per-warp partial sums of q_i . dq_i.
+//   bwd_final  ds, dgain, dtau from C and the partial sums, in a fixed
+//              order (deterministic: no atomics anywhere).
+// Roles in both tensor-core kernels (256 threads): warp 0 TMA producer,
+// warp 1 MMA issuer, warp 2 TMEM allocation, warps 4-7 one thread per row.
+// Every wait is bounded (an expired wait sets the device error word and the
+// kernel drains and returns).
+#include "tg_device.cuh"
+#include "tg_internal.h"
+
+namespace tg {
+namespace {
+
+constexpr int kBlk = 128;        // rows per tile (queries or keys)
+constexpr int kDh = 128;
+constexpr int kThreads = 256;
+constexpr int kSub = 128 * 128;  // bytes of one [128 rows x 64 bf16] 128-byte-swizzled sub-tile
+constexpr int kTile = 2 * kSub;  // [128 x 128] bf16 tile
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct BwdParams {
+  int64_t T, t_pad;
+  int hq, hkv, n_tiles;
+  const float* bias;     // [t_pad] logsigmoid(s_j), zero past T (all zero without scores)
+  const float* gain;     // [hq], null: gain 0
+  const float* tau;      // [hq], null: tau 1
+  const float* lse2;     // [hq, t_pad] lse * log2(e), +inf past T
+  const float* dd;       // [hq, t_pad] D_i, 0 past T
+  const float2* cs;      // [dh/2, T] RoPE (cos, sin) at each row's position
+  __nv_bfloat16* dq;     // [T, hq, dh]
+  __nv_bfloat16* dk;     // [T, hkv, dh]
+  __nv_bfloat16* dv;     // [T, hkv, dh]
+  float* colsum;         // [hq, t_pad] C_hj, or null (no scores)
+  float* qdq;            // [hq, n_tiles, 4] per-warp partial sums of q_i . dq_i
+  unsigned int* err;
+};
+
+// Rotate a gradient row (dh = 128, rotate-half pairs (i, i + 64)) back
+// through RoPE: the transpose of the forward rotation.
+__device__ __forceinline__ void rope_back(float (&x)[128], const float2* cs, int64_t T,
+                                          int64_t row) {
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    const float2 c = __ldg(cs + static_cast<int64_t>(i) * T + row);
+    const float a = x[i], b = x[i + 64];
+    x[i] = a * c.x + b * c.y;
+    x[i + 64] = b * c.x - a * c.y;
+  }
+}
+
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const float (&x)[128]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int v = 0; v < 16; ++v) {
+    uint4 u;
+    u.x = pack_bf16x2(x[8 * v + 0], x[8 * v + 1]);
+    u.y = pack_bf16x2(x[8 * v + 2], x[8 * v + 3]);
+    u.z = pack_bf16x2(x[8 * v + 4], x[8 * v + 5]);
+    u.w = pack_bf16x2(x[8 * v + 6], x[8 * v + 7]);
+    d[v] = u;
+  }
+}
+
+// Four TMEM loads of 32 columns into x[128] (one wait).
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&x)[128]) {
+  uint32_t r0[32], r1[32], r2[32], r3[32];
+  tmem_ld32(taddr, r0);
+  tmem_ld32(taddr + 32, r1);
+  tmem_ld32(taddr + 64, r2);
+  tmem_ld32(taddr + 96, r3);
+  tmem_wait_ld_dep(r3);
+  tmem_ld_fence(r0);
+  tmem_ld_fence(r1);
+  tmem_ld_fence(r2);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    x[i] = __uint_as_float(r0[i]);
+    x[32 + i] = __uint_as_float(r1[i]);
+    x[64 + i] = __uint_as_float(r2[i]);
+    x[96 + i] = __uint_as_float(r3[i]);
+  }
+}
+
+// Copies this thread's row r of a [128 x 128] bf16 tile (two 128-byte-
+// swizzled [128 x 64] sub-tiles in shared memory) into 64 TMEM columns of
+// its lane, two bf16 per column: the A operand of a TS product.
+__device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int r, uint32_t taddr) {
+#pragma unroll
+  for (int hs = 0; hs < 2; ++hs) {
+    uint32_t v[32];
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      const uint4 u = *reinterpret_cast<const uint4*>(tile + hs * kSub + r * 128 + ((ch ^ (r & 7)) << 4));
+      v[4 * ch + 0] = u.x;
+      v[4 * ch + 1] = u.y;
+      v[4 * ch + 2] = u.z;
+      v[4 * ch + 3] = u.w;
+    }
+    tmem_st32(taddr + static_cast<uint32_t>(32 * hs), v);
+  }
+}
+
+// ============================================================================
+// dK, dV and C: one CTA per (key tile jt, KV head g), 128 key rows.
+// TMEM columns: S^T [0,128) (P^T packed over [0,64)), dP^T [128,256) (dS^T
+// packed over [128,192)), dV [256,384), dK [384,512). All 512 columns are in
+// use, so the products of one query tile wait for the rows of the previous
+// one; the query side is loaded in two halves (stage a: Q, dO for S^T and
+// dP^T; stage b: Q^T, dO^T, lse2, D for the rows and dV, dK) so that the
+// loads of tile n+1 overlap the work on tile n.
+namespace dkdv {
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kTile;
+constexpr int kOffQ = kOffV + kTile;     // stage a: Q_i, dO_i
+constexpr int kOffDO = kOffQ + kTile;
+constexpr int kOffQT = kOffDO + kTile;   // stage b: Q_i^T, dO_i^T, lse2 and D of tile i
+constexpr int kOffDOT = kOffQT + kTile;
+constexpr int kOffVec = kOffDOT + kTile;
+constexpr int kOffBar = kOffVec + 1024;
+constexpr size_t kSmem = 1024 + kOffBar + 256;
+}  // namespace dkdv
+
+// [128 x 128] x [128 x 128]^T over dh with both operands K-major in shared
+// memory (two 64-column swizzled sub-tiles each).
+__device__ __forceinline__ void mma_ss_128(uint32_t d, uint32_t a_addr, uint32_t b_addr) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+#pragma unroll
+  for (int kk = 0; kk < kDh / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
+    umma_f16_ss(d, sdesc_kmajor_sw128(a_addr + off), sdesc_kmajor_sw128(b_addr + off), idesc,
+                kk > 0 ? 1u : 0u);
+  }
+}
+
+// [128 x 128] x [128 x 128]^T over 128 rows with A packed in 64 TMEM columns.
+__device__ __forceinline__ void mma_ts_128(uint32_t d, uint32_t a_tmem, uint32_t b_addr,
+                                           bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+#pragma unroll
+  for (int kk = 0; kk < kBlk / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
+    umma_f16_ts(d, a_tmem + static_cast<uint32_t>(kk * 8), sdesc_kmajor_sw128(b_addr + off),
+                idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_dkdv(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ CUtensorMap tmQT,
+                  const __grid_constant__ CUtensorMap tmDOT, BwdParams p) {
+  using namespace dkdv;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* a_full = bars + 1;
+  uint64_t* a_empty = bars + 2;
+  uint64_t* b_full = bars + 3;
+  uint64_t* b_empty = bars + 4;
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 6;
+  uint64_t* acc_full = bars + 7;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int jt = static_cast<int>(blockIdx.x) / p.hkv;  // key tile 0 (the longest) first
+  const int g = static_cast<int>(blockIdx.x) % p.hkv;
+  const int group = p.hq / p.hkv;
+  const int j0 = jt * kBlk;
+  const int n_q = p.n_tiles - jt;  // query tiles jt .. n_tiles-1 see this key tile
+  const int n_it = group * n_q;
+
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(a_full, 1);
+    mbar_init(a_empty, 1);
+    mbar_init(b_full, 1);
+    mbar_init(b_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(acc_full, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmDO);
+    tma_prefetch_desc(&tmQT);
+    tma_prefetch_desc(&tmDOT);
+  }
+  if (warp == 2) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    mbar_arrive_expect_tx(kv_full, 2 * kTile);
+    tma_load_3d(&tmK, kv_full, smem + kOffK, 0, g, j0);
+    tma_load_3d(&tmK, kv_full, smem + kOffK + kSub, 64, g, j0);
+    tma_load_3d(&tmV, kv_full, smem + kOffV, 0, g, j0);
+    tma_load_3d(&tmV, kv_full, smem + kOffV + kSub, 64, g, j0);
+    for (int n = 0; n < n_it; ++n) {
+      const int h = g * group + n / n_q;
+      const int i0 = (jt + n % n_q) * kBlk;
+      const uint32_t ph = (n & 1) ^ 1;
+      if (!mbar_wait(a_empty, ph, p.err)) break;
+      mbar_arrive_expect_tx(a_full, 2 * kTile);
+      tma_load_3d(&tmQ, a_full, smem + kOffQ, 0, h, i0);
+      tma_load_3d(&tmQ, a_full, smem + kOffQ + kSub, 64, h, i0);
+      tma_load_3d(&tmDO, a_full, smem + kOffDO, 0, h, i0);
+      tma_load_3d(&tmDO, a_full, smem + kOffDO + kSub, 64, h, i0);
+      if (!mbar_wait(b_empty, ph, p.err)) break;
+      mbar_arrive_expect_tx(b_full, 2 * kTile + 1024);
+      tma_load_3d(&tmQT, b_full, smem + kOffQT, i0, 0, h);
+      tma_load_3d(&tmQT, b_full, smem + kOffQT + kSub, i0 + 64, 0, h);
+      tma_load_3d(&tmDOT, b_full, smem + kOffDOT, i0, 0, h);
+      tma_load_3d(&tmDOT, b_full, smem + kOffDOT + kSub, i0 + 64, 0, h);
+      bulk_load(smem + kOffVec, p.lse2 + static_cast<int64_t>(h) * p.t_pad + i0, 512, b_full);
+      bulk_load(smem + kOffVec + 512, p.dd + static_cast<int64_t>(h) * p.t_pad + i0, 512, b_full);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    bool ok = mbar_wait(kv_full, 0, p.err);
+    for (int n = 0; n < n_it && ok; ++n) {
+      const uint32_t ph = n & 1;
+      if (!mbar_wait(a_full, ph, p.err)) break;
+      tc_fence_after();
+      mma_ss_128(tmem + 0, smem_addr(smem + kOffK), smem_addr(smem + kOffQ));     // S^T
+      mma_ss_128(tmem + 128, smem_addr(smem + kOffV), smem_addr(smem + kOffDO));  // dP^T
+      umma_commit(s_full);
+      umma_commit(a_empty);
+      if (!mbar_wait(p_full, ph, p.err) || !mbar_wait(b_full, ph, p.err)) break;
+      tc_fence_after();
+      mma_ts_128(tmem + 256, tmem + 0, smem_addr(smem + kOffDOT), n > 0);    // dV += P^T dO
+      mma_ts_128(tmem + 384, tmem + 128, smem_addr(smem + kOffQT), n > 0);   // dK += dS^T Q
+      umma_commit(b_empty);
+    }
+    if (ok) umma_commit(acc_full);
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ one thread per key row
+    const int r = threadIdx.x - 128;
+    const int64_t j = static_cast<int64_t>(j0) + r;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float* vec_l = reinterpret_cast<const float*>(smem + kOffVec);
+    const float* vec_d = vec_l + 128;
+    const float bj = __ldg(p.bias + j);  // zero past T
+    float csum = 0.f;
+    bool ok = true;
+    for (int n = 0; n < n_it; ++n) {
+      const int h = g * group + n / n_q;
+      const int it = jt + n % n_q;
+      const uint32_t ph = n & 1;
+      const float tau = p.tau ? __ldg(p.tau + h) : 1.0f;
+      const float inv_st = 1.0f / (sqrtf(static_cast<float>(kDh)) * tau);
+      const float scale2 = kLog2e * inv_st;
+      const float b2 = (p.gain ? __ldg(p.gain + h) : 0.0f) * kLog2e * bj;
+      if (!mbar_wait_warp(s_full, ph, p.err) || !mbar_wait_warp(b_full, ph, p.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool diag = it == jt;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rs[32], rp[32];
+        tmem_ld32(tmem + lane_off + static_cast<uint32_t>(32 * c), rs);
+        tmem_ld32(tmem + lane_off + 128u + static_cast<uint32_t>(32 * c), rp);
+        tmem_wait_ld_dep(rp);
+        tmem_ld_fence(rs);
+        uint32_t pk[16], dk16[16];
+#pragma unroll
+        for (int t = 0; t < 32; t += 2) {
+          const int il = 32 * c + t;
+          float p0 = ex2_approx(fmaf(__uint_as_float(rs[t]), scale2, b2) - vec_l[il]);
+          float p1 = ex2_approx(fmaf(__uint_as_float(rs[t + 1]), scale2, b2) - vec_l[il + 1]);
+          if (diag) {  // query i0 + il sees key j0 + r only when il >= r
+            if (il < r) p0 = 0.f;
+            if (il + 1 < r) p1 = 0.f;
+          }
+          const float d0 = p0 * (__uint_as_float(rp[t]) - vec_d[il]);
+          const float d1 = p1 * (__uint_as_float(rp[t + 1]) - vec_d[il + 1]);
+          csum += d0 + d1;
+          pk[t >> 1] = pack_bf16x2(p0, p1);
+          dk16[t >> 1] = pack_bf16x2(d0 * inv_st, d1 * inv_st);
+        }
+        tmem_st16(tmem + lane_off + static_cast<uint32_t>(16 * c), pk);
+        tmem_st16(tmem + lane_off + 128u + static_cast<uint32_t>(16 * c), dk16);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
+      if (n % n_q == n_q - 1) {  // last query tile of head h: C_hj is complete
+        if (p.colsum && j < p.T) p.colsum[static_cast<int64_t>(h) * p.t_pad + j] = csum;
+        csum = 0.f;
+      }
+    }
+    if (ok && mbar_wait_warp(acc_full, 0, p.err)) {
+      tc_fence_after();
+      float x[128];
+      tmem_ld128(tmem + lane_off + 256u, x);  // dV
+      if (j < p.T) store_row_bf16(p.dv + (j * p.hkv + g) * kDh, x);
+      tmem_ld128(tmem + lane_off + 384u, x);  // dK (rotated frame)
+      if (j < p.T) {
+        rope_back(x, p.cs, p.T, j);
+        store_row_bf16(p.dk + (j * p.hkv + g) * kDh, x);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+// ============================================================================
+// dQ: one CTA per (query tile it, query head h), 128 query rows.
+// Q and dO sit in TMEM as the A operands; the key side streams through a
+// 3-stage ring of 64-key stages, with S and dP double-buffered in TMEM.
+// TMEM columns: Q [0,64), dO [64,128) (packed bf16), dQ [128,256), buffer b:
+// S [256+128b, +64), dP [320+128b, +64); dS (packed) over the first 32
+// columns of S.
+namespace dqk {
+constexpr int kHalf64 = 64 * 128;
+constexpr int kOffQ = 0;
+constexpr int kOffDO = kOffQ + kTile;
+constexpr int kOffStage = kOffDO + kTile;
+// stage: K [64 x 128], V [64 x 128] (two dh halves each), K^T [128 dh x 64], bias[64]
+constexpr int kStK = 0;
+constexpr int kStV = kStK + 2 * kHalf64;
+constexpr int kStKT = kStV + 2 * kHalf64;
+constexpr int kStBias = kStKT + 128 * 128;
+constexpr int kStageBytes = kStBias + 1024;
+constexpr uint32_t kStageTx = 3 * 16384 + 256;
+constexpr int kStages = 3;
+constexpr int kOffBar = kOffStage + kStages * kStageBytes;
+constexpr size_t kSmem = 1024 + kOffBar + 256;
+constexpr uint32_t kTmQ = 0, kTmDO = 64, kTmDQ = 128, kTmBuf = 256;
+}  // namespace dqk
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                const __grid_constant__ CUtensorMap tmKT, BwdParams p) {
+  using namespace dqk;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_ready = bars + 1;     // Q and dO copied into TMEM (128 arrivals)
+  uint64_t* st_full = bars + 2;     // [3]
+  uint64_t* st_empty = bars + 5;    // [3]
+  uint64_t* s_full = bars + 8;      // [2]
+  uint64_t* p_full = bars + 10;     // [2] (128 arrivals)
+  uint64_t* acc_full = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int it = p.n_tiles - 1 - static_cast<int>(blockIdx.x) / p.hq;  // longest first
+  const int h = static_cast<int>(blockIdx.x) % p.hq;
+  const int g = h / (p.hq / p.hkv);
+  const int i0 = it * kBlk;
+  const int n_sub = 2 * (it + 1);  // 64-key stages up to the diagonal
+
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_ready, 128);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&st_full[i], 1);
+      mbar_init(&st_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+    }
+    mbar_init(acc_full, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmDO);
+    tma_prefetch_desc(&tmKT);
+  }
+  if (warp == 2) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    mbar_arrive_expect_tx(q_full, 2 * kTile);
+    tma_load_3d(&tmQ, q_full, smem + kOffQ, 0, h, i0);
+    tma_load_3d(&tmQ, q_full, smem + kOffQ + kSub, 64, h, i0);
+    tma_load_3d(&tmDO, q_full, smem + kOffDO, 0, h, i0);
+    tma_load_3d(&tmDO, q_full, smem + kOffDO + kSub, 64, h, i0);
+    for (int m = 0; m < n_sub; ++m) {
+      const int st = m % kStages;
+      const int j0 = 64 * m;
+      if (!mbar_wait(&st_empty[st], ((m / kStages) & 1) ^ 1, p.err)) break;
+      uint8_t* sb = smem + kOffStage + st * kStageBytes;
+      mbar_arrive_expect_tx(&st_full[st], kStageTx);
+      tma_load_3d(&tmK, &st_full[st], sb + kStK, 0, g, j0);
+      tma_load_3d(&tmK, &st_full[st], sb + kStK + kHalf64, 64, g, j0);
+      tma_load_3d(&tmV, &st_full[st], sb + kStV, 0, g, j0);
+      tma_load_3d(&tmV, &st_full[st], sb + kStV + kHalf64, 64, g, j0);
+      tma_load_3d(&tmKT, &st_full[st], sb + kStKT, j0, 0, g);
+      bulk_load(sb + kStBias, p.bias + j0, 256, &st_full[st]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_n64 = idesc_bf16_f32(128, 64);
+    constexpr uint32_t idesc_n128 = idesc_bf16_f32(128, 128);
+    auto sp_products = [&](int m) {  // S_b = Q K_m^T, dP_b = dO V_m^T
+      const int b = m & 1;
+      const uint8_t* sb = smem + kOffStage + (m % kStages) * kStageBytes;
+      const uint32_t k_addr = smem_addr(sb + kStK), v_addr = smem_addr(sb + kStV);
+      const uint32_t d = tmem + kTmBuf + 128u * b;
+#pragma unroll
+      for (int kk = 0; kk < kDh / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kHalf64 + (kk & 3) * 32;
+        umma_f16_ts(d, tmem + kTmQ + kk * 8, sdesc_kmajor_sw128(k_addr + off), idesc_n64,
+                    kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < kDh / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kHalf64 + (kk & 3) * 32;
+        umma_f16_ts(d + 64u, tmem + kTmDO + kk * 8, sdesc_kmajor_sw128(v_addr + off), idesc_n64,
+                    kk > 0 ? 1u : 0u);
+      }
+      umma_commit(&s_full[b]);
+    };
+    auto dq_product = [&](int m) {  // dQ += dS_b K_m
+      const int b = m & 1, st = m % kStages;
+      const uint32_t kt_addr = smem_addr(smem + kOffStage + st * kStageBytes + kStKT);
+      const uint32_t a = tmem + kTmBuf + 128u * b;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        umma_f16_ts(tmem + kTmDQ, a + kk * 8, sdesc_kmajor_sw128(kt_addr + kk * 32), idesc_n128,
+                    (m > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(&st_empty[st]);
+    };
+    bool ok = mbar_wait(q_ready, 0, p.err);
+    for (int m = 0; m < n_sub && ok; ++m) {
+      if (!mbar_wait(&st_full[m % kStages], (m / kStages) & 1, p.err)) break;
+      tc_fence_after();
+      sp_products(m);
+      if (m > 0) {
+        if (!mbar_wait(&p_full[(m - 1) & 1], ((m - 1) >> 1) & 1, p.err)) break;
+        tc_fence_after();
+        dq_product(m - 1);
+      }
+      if (m == n_sub - 1) {
+        if (!mbar_wait(&p_full[m & 1], (m >> 1) & 1, p.err)) break;
+        tc_fence_after();
+        dq_product(m);
+        umma_commit(acc_full);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ one thread per query row
+    const int r = threadIdx.x - 128;
+    const int64_t i = static_cast<int64_t>(i0) + r;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float tau = p.tau ? __ldg(p.tau + h) : 1.0f;
+    const float inv_st = 1.0f / (sqrtf(static_cast<float>(kDh)) * tau);
+    const float scale2 = kLog2e * inv_st;
+    const float gb2 = p.gain ? __ldg(p.gain + h) * kLog2e : 0.0f;
+    const float lse2 = __ldg(p.lse2 + static_cast<int64_t>(h) * p.t_pad + i);
+    const float di = __ldg(p.dd + static_cast<int64_t>(h) * p.t_pad + i);
+    bool ok = mbar_wait_warp(q_full, 0, p.err);
+    if (ok) {
+      tile_row_to_tmem(smem + kOffQ, r, tmem + lane_off + kTmQ);
+      tile_row_to_tmem(smem + kOffDO, r, tmem + lane_off + kTmDO);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(q_ready);
+    }
+    for (int m = 0; m < n_sub && ok; ++m) {
+      const int b = m & 1, st = m % kStages;
+      if (!mbar_wait_warp(&s_full[b], (m >> 1) & 1, p.err) ||
+          !mbar_wait_warp(&st_full[st], (m / kStages) & 1, p.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* bias = reinterpret_cast<const float*>(smem + kOffStage + st * kStageBytes +
+                                                         kStBias);
+      const int lim = static_cast<int>(i - 64 * m);  // key 64m + t is visible when t <= lim
+      const uint32_t ta = tmem + lane_off + kTmBuf + 128u * b;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t rs[32], rp[32];
+        tmem_ld32(ta + 32u * c, rs);
+        tmem_ld32(ta + 64u + 32u * c, rp);
+        tmem_wait_ld_dep(rp);
+        tmem_ld_fence(rs);
+        uint32_t dk16[16];
+#pragma unroll
+        for (int t = 0; t < 32; t += 2) {
+          const int jl = 32 * c + t;
+          float p0 = ex2_approx(fmaf(__uint_as_float(rs[t]), scale2, gb2 * bias[jl]) - lse2);
+          float p1 = ex2_approx(fmaf(__uint_as_float(rs[t + 1]), scale2, gb2 * bias[jl + 1]) - lse2);
+          if (jl > lim) p0 = 0.f;
+          if (jl + 1 > lim) p1 = 0.f;
+          dk16[t >> 1] = pack_bf16x2(p0 * (__uint_as_float(rp[t]) - di),
+                                     p1 * (__uint_as_float(rp[t + 1]) - di));
+        }
+        tmem_st16(ta + 16u * c, dk16);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[b]);
+    }
+    if (ok && mbar_wait_warp(acc_full, 0, p.err)) {
+      tc_fence_after();
+      float x[128];
+      tmem_ld128(tmem + lane_off + kTmDQ, x);
+#pragma unroll
+      for (int e = 0; e < 128; ++e) x[e] *= inv_st;
+      // q_i . dq_i in the rotated frame (rows past T contribute nothing)
+      float dot = 0.f;
+      if (i < p.T) {
+        const uint8_t* qrow = smem + kOffQ + r * 128;
+#pragma unroll
+        for (int hs = 0; hs < 2; ++hs) {
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint4 u =
+                *reinterpret_cast<const uint4*>(qrow + hs * kSub + ((ch ^ (r & 7)) << 4));
+            const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+              const float2 f = __bfloat1622float2(e2[q2]);
+              const int d = hs * 64 + ch * 8 + 2 * q2;
+              dot = fmaf(f.x, x[d], fmaf(f.y, x[d + 1], dot));
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xFFFFFFFFu, dot, o);
+      if (lane == 0)
+        p.qdq[(static_cast<int64_t>(h) * p.n_tiles + it) * 4 + (warp & 3)] = dot;
+      if (i < p.T) {
+        rope_back(x, p.cs, p.T, i);
+        store_row_bf16(p.dq + (i * p.hq + h) * kDh, x);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+// ============================================================================
+// Prep: [T, H, dh] rows -> [H, dh, t_pad] (zero past T) for q_rot, k_rot and
+// dO; for dO's heads also lse2 = lse * log2(e) and D = dO . o per row.
+struct PrepArgs {
+  const __nv_bfloat16* src[3];  // q_rot, k_rot, dO
+  int heads[3];
+  __nv_bfloat16* dst[3];
+  const __nv_bfloat16* out;     // forward output [T, hq, dh]
+  const float* out_f32;         // the same before rounding, or null
+  const float* lse;             // [hq, T]
+  const float* lsig;            // [T] or null
+  float* lse2;                  // [hq, t_pad]
+  float* dd;                    // [hq, t_pad]
+  float* bias;                  // [t_pad]: lsig, zero past T (all zero without lsig)
+  int64_t T, t_pad;
+};
+
+__global__ void __launch_bounds__(256) attn_bwd_prep(PrepArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  constexpr int kRows = 64;
+  constexpr int kLd = kDh + 8;  // padded row (bf16 elements)
+  __shared__ __align__(16) __nv_bfloat16 tile[kRows * kLd];
+  int slot = blockIdx.y, which = 0;
+  while (which < 2 && slot >= a.heads[which]) slot -= a.heads[which++];
+  const int H = a.heads[which], h = slot;
+  const __nv_bfloat16* src = a.src[which];
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRows;
+  constexpr int kVec = kDh / 8;
+  for (int e = threadIdx.x; e < kRows * kVec; e += 256) {
+    const int rr = e / kVec, c = e % kVec;
+    const int64_t t = t0 + rr;
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (t < a.T) u = __ldg(reinterpret_cast<const uint4*>(src + (t * H + h) * kDh) + c);
+    *reinterpret_cast<uint4*>(&tile[rr * kLd + c * 8]) = u;
+  }
+  if (which == 1 && h == 0 && threadIdx.x < kRows) {
+    const int64_t t = t0 + threadIdx.x;
+    a.bias[t] = (a.lsig && t < a.T) ? __ldg(a.lsig + t) : 0.0f;
+  }
+  __syncthreads();
+  __nv_bfloat16* dst = a.dst[which] + static_cast<int64_t>(h) * kDh * a.t_pad;
+  for (int e = threadIdx.x; e < kDh * (kRows / 8); e += 256) {
+    const int d = e / (kRows / 8), c = e % (kRows / 8);
+    uint4 o;
+    __nv_bfloat16* oe = reinterpret_cast<__nv_bfloat16*>(&o);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) oe[q] = tile[(c * 8 + q) * kLd + d];
+    *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(d) * a.t_pad + t0 + c * 8) = o;
+  }
+  if (which == 2) {
+    // four threads per row, 32 elements each
+    const int rr = threadIdx.x >> 2, part = threadIdx.x & 3;
+    const int64_t t = t0 + rr;
+    float acc = 0.f;
+    if (t < a.T && a.out_f32) {
+      const float4* o4 = reinterpret_cast<const float4*>(a.out_f32 + (t * H + h) * kDh + part * 32);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const float4 f = __ldg(o4 + v);
+        const int d = part * 32 + v * 4;
+        acc = fmaf(f.x, __bfloat162float(tile[rr * kLd + d]), acc);
+        acc = fmaf(f.y, __bfloat162float(tile[rr * kLd + d + 1]), acc);
+        acc = fmaf(f.z, __bfloat162float(tile[rr * kLd + d + 2]), acc);
+        acc = fmaf(f.w, __bfloat162float(tile[rr * kLd + d + 3]), acc);
+      }
+    } else if (t < a.T) {
+      const uint4* o4 = reinterpret_cast<const uint4*>(a.out + (t * H + h) * kDh + part * 32);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 u = __ldg(o4 + v);
+        const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(e2[q]);
+          const int d = part * 32 + v * 8 + 2 * q;
+          acc = fmaf(f.x, __bfloat162float(tile[rr * kLd + d]),
+                     fmaf(f.y, __bfloat162float(tile[rr * kLd + d + 1]), acc));
+        }
+      }
+    }
+    acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 1);
+    acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 2);
+    if (part == 0) {
+      const int64_t k = static_cast<int64_t>(h) * a.t_pad + t;
+      a.dd[k] = t < a.T ? acc : 0.0f;
+      a.lse2[k] = t < a.T ? __ldg(a.lse + static_cast<int64_t>(h) * a.T + t) * kLog2e : INFINITY;
+    }
+  }
+}
+
+// ============================================================================
+// ds, dgain, dtau. Blocks [0, hq): one head each (dgain_h, dtau_h); the rest:
+// 256 keys each (ds_j). Fixed summation order throughout.
+struct FinalArgs {
+  const float* s;       // [T] scores (null: no scores)
+  const float* lsig;    // [T]
+  const float* gain;    // [hq] or null
+  const float* tau;     // [hq] or null
+  const float* colsum;  // [hq, t_pad]
+  const float* qdq;     // [hq, n_tiles, 4]
+  int64_t T, t_pad;
+  int hq, n_tiles;
+  float* ds;            // [T] or null
+  float* dgain;         // [hq] or null
+  float* dtau;          // [hq] or null
+};
+
+__device__ __forceinline__ float block_sum_256(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float s = 0.f;
+  if (threadIdx.x == 0)
+    for (int w = 0; w < 8; ++w) s += red[w];
+  __syncthreads();
+  return s;  // valid in thread 0
+}
+
+__global__ void __launch_bounds__(256) attn_bwd_final(FinalArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float red[8];
+  if (static_cast<int>(blockIdx.x) < a.hq) {
+    const int h = blockIdx.x;
+    float acc = 0.f;
+    if (a.lsig)
+      for (int64_t j = threadIdx.x; j < a.T; j += 256)
+        acc = fmaf(__ldg(a.lsig + j), __ldg(a.colsum + static_cast<int64_t>(h) * a.t_pad + j), acc);
+    const float dg = block_sum_256(acc, red);
+    float acc2 = 0.f;
+    for (int e = threadIdx.x; e < a.n_tiles * 4; e += 256)
+      acc2 += __ldg(a.qdq + static_cast<int64_t>(h) * a.n_tiles * 4 + e);
+    const float qd = block_sum_256(acc2, red);
+    if (threadIdx.x == 0) {
+      if (a.dgain) a.dgain[h] = dg;
+      if (a.dtau) a.dtau[h] = -qd / (a.tau ? __ldg(a.tau + h) : 1.0f);
+    }
+    return;
+  }
+  const int64_t j = static_cast<int64_t>(blockIdx.x - a.hq) * 256 + threadIdx.x;
+  if (!a.ds || j >= a.T) return;
+  float sum = 0.f;
+  if (a.gain)
+    for (int h = 0; h < a.hq; ++h)
+      sum = fmaf(__ldg(a.gain + h), __ldg(a.colsum + static_cast<int64_t>(h) * a.t_pad + j), sum);
+  a.ds[j] = sum / (1.0f + expf(__ldg(a.s + j)));  // sigmoid(-s_j) = 1 / (1 + e^s_j)
+}
+
+}  // namespace
+
+size_t attn_bwd_t_pad(int64_t T) { return align_up(static_cast<size_t>(T), kBlk); }
+
+cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t st, int stage) {
+  if (a.T <= 0) return cudaSuccess;
+  const int64_t e = 2;
+  const int n_tiles = static_cast<int>((a.T + kBlk - 1) / kBlk);
+  if (stage == 0) {
+    PrepArgs pa{};
+    pa.src[0] = static_cast<const __nv_bfloat16*>(a.q_rot);
+    pa.src[1] = static_cast<const __nv_bfloat16*>(a.k_rot);
+    pa.src[2] = static_cast<const __nv_bfloat16*>(a.dout);
+    pa.heads[0] = a.hq;
+    pa.heads[1] = a.hkv;
+    pa.heads[2] = a.hq;
+    pa.dst[0] = static_cast<__nv_bfloat16*>(a.qT);
+    pa.dst[1] = static_cast<__nv_bfloat16*>(a.kT);
+    pa.dst[2] = static_cast<__nv_bfloat16*>(a.doT);
+    pa.out = static_cast<const __nv_bfloat16*>(a.out);
+    pa.out_f32 = a.out_f32;
+    pa.lse = a.lse;
+    pa.lsig = a.lsig;
+    pa.lse2 = a.lse2;
+    pa.dd = a.dd;
+    pa.bias = a.bias;
+    pa.T = a.T;
+    pa.t_pad = a.t_pad;
+    const dim3 grid(static_cast<unsigned>(a.t_pad / 64), static_cast<unsigned>(2 * a.hq + a.hkv));
+    TG_CUDA_TRY(launch_pdl(attn_bwd_prep, grid, dim3(256), 0, st, pa));
+    return cudaGetLastError();
+  }
+  BwdParams p{};
+  p.T = a.T;
+  p.t_pad = a.t_pad;
+  p.hq = a.hq;
+  p.hkv = a.hkv;
+  p.n_tiles = n_tiles;
+  p.bias = a.bias;
+  p.gain = a.gain;
+  p.tau = a.tau;
+  p.lse2 = a.lse2;
+  p.dd = a.dd;
+  p.cs = a.cs;
+  p.dq = static_cast<__nv_bfloat16*>(a.dq);
+  p.dk = static_cast<__nv_bfloat16*>(a.dk);
+  p.dv = static_cast<__nv_bfloat16*>(a.dv);
+  p.colsum = a.lsig ? a.colsum : nullptr;
+  p.qdq = a.qdq;
+  p.err = device_error_word();
+  if (stage == 3) {
+    FinalArgs f{};
+    f.s = a.s;
+    f.lsig = a.lsig;
+    f.gain = a.gain;
+    f.tau = a.tau;
+    f.colsum = a.colsum;
+    f.qdq = a.qdq;
+    f.T = a.T;
+    f.t_pad = a.t_pad;
+    f.hq = a.hq;
+    f.n_tiles = n_tiles;
+    f.ds = a.lsig ? a.ds : nullptr;
+    f.dgain = a.dgain;
+    f.dtau = a.dtau;
+    const unsigned blocks = static_cast<unsigned>(a.hq + (a.ds && a.lsig ? (a.T + 255) / 256 : 0));
+    TG_CUDA_TRY(launch_pdl(attn_bwd_final, dim3(blocks), dim3(256), 0, st, f));
+    return cudaGetLastError();
+  }
+  // row-major [T, H, dh] operands (rows past T read as zeros), as 128-row
+  // tiles (the CTA's own rows) and 64-row stages (the streamed side)
+  auto rows_map = [&](CUtensorMap* m, const void* base, int heads, int box_rows) {
+    return make_tmap_3d_bf16(m, base, kDh, heads, a.T, kDh * e, int64_t(heads) * kDh * e, 1,
+                             box_rows);
+  };
+  // transposed [H, dh, t_pad] operands, loaded as [128 dh x 64 rows] boxes;
+  // the inner extent is T, so rows past T read as zeros
+  auto cols_map = [&](CUtensorMap* m, const void* base, int heads) {
+    return make_tmap_3d_bf16(m, base, a.T, kDh, heads, a.t_pad * e, a.t_pad * kDh * e, kDh, 1);
+  };
+  if (stage == 1) {
+    CUtensorMap tq, tk, tv, tdo, tqT, tdoT;
+    if (!rows_map(&tq, a.q_rot, a.hq, kBlk) || !rows_map(&tdo, a.dout, a.hq, kBlk) ||
+        !rows_map(&tk, a.k_rot, a.hkv, kBlk) || !rows_map(&tv, a.v, a.hkv, kBlk) ||
+        !cols_map(&tqT, a.qT, a.hq) || !cols_map(&tdoT, a.doT, a.hq))
+      return cudaErrorInvalidValue;
+    cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(attn_bwd_dkdv),
+                                         int(dkdv::kSmem));
+    if (err != cudaSuccess) return err;
+    const unsigned grid = static_cast<unsigned>(n_tiles) * static_cast<unsigned>(a.hkv);
+    return launch_pdl(attn_bwd_dkdv, dim3(grid), dim3(kThreads), dkdv::kSmem, st, tq, tk, tv, tdo,
+                      tqT, tdoT, p);
+  }
+  CUtensorMap tq, tk, tv, tdo, tkT;
+  if (!rows_map(&tq, a.q_rot, a.hq, kBlk) || !rows_map(&tdo, a.dout, a.hq, kBlk) ||
+      !rows_map(&tk, a.k_rot, a.hkv, 64) || !rows_map(&tv, a.v, a.hkv, 64) ||
+      !cols_map(&tkT, a.kT, a.hkv))
+    return cudaErrorInvalidValue;
+  cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(attn_bwd_dq), int(dqk::kSmem));
+  if (err != cudaSuccess) return err;
+  const unsigned grid = static_cast<unsigned>(n_tiles) * static_cast<unsigned>(a.hq);
+  return launch_pdl(attn_bwd_dq, dim3(grid), dim3(kThreads), dqk::kSmem, st, tq, tk, tv, tdo, tkT,
+                    p);
+}
+
+}  // namespace tg

@@ -46,6 +46,7 @@ constexpr int kOffP = kOffV + 2 * kTile;      // 2 buffers
 constexpr int kOffBar = kOffP + 2 * kTile;
 constexpr size_t kSmem = 1024 + kOffBar + 256;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThresh = 8.0f;  // log2 units
 
 struct Params {
@@ -56,6 +57,8 @@ struct Params {
   const float* gain;
   const float* tau;
   __nv_bfloat16* out;
+  float* lse;      // [hq, T] or null
+  float* out_f32;  // [T, hq, dh] or null: the output before rounding
   unsigned int* err;
 };
 
@@ -257,6 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && mbar_wait_warp(&pv_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, p.err)) {
       tc_fence_after();
       const float inv = 1.0f / l;
+      // log-sum-exp of the row's logits: m and l are in log2 units
+      if (p.lse && q_row < p.T) p.lse[head * p.T + q_row] = (m + log2f(l)) * kLn2;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         float o[32];
@@ -264,6 +269,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] *= inv;
         if (q_row < p.T) {
+          if (p.out_f32) {
+            float4* d32 = reinterpret_cast<float4*>(p.out_f32 + (q_row * p.hq + head) * kDh + c * 32);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              d32[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          }
           uint4* dst = reinterpret_cast<uint4*>(p.out + (q_row * p.hq + head) * kDh + c * 32);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
@@ -346,6 +357,8 @@ struct Params {
   const float* gain;
   const float* tau;
   __nv_bfloat16* out;
+  float* lse;      // [hq, T] or null
+  float* out_f32;  // [T, hq, dh] or null: the output before rounding
   unsigned int* err;
 };
 
@@ -644,6 +657,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && mbar_wait_warp(o_full, 0, p.err)) {
       tc_fence_after();
       const float inv = 1.0f / l;
+      // log-sum-exp of the row's logits: m and l are in log2 units
+      if (p.lse && q_row < p.T) p.lse[head * p.T + q_row] = (m + log2f(l)) * kLn2;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         float o[32];
@@ -651,6 +666,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] *= inv;
         if (q_row < p.T) {
+          if (p.out_f32) {
+            float4* d32 = reinterpret_cast<float4*>(p.out_f32 + (q_row * p.hq + head) * kDh + c * 32);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              d32[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          }
           uint4* dst = reinterpret_cast<uint4*>(p.out + (q_row * p.hq + head) * kDh + c * 32);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
@@ -703,6 +724,8 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
   p.gain = a.gain;
   p.tau = a.tau;
   p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
+  p.out_f32 = a.out_f32;
   p.err = device_error_word();
   if ((a.hq / a.hkv) % 2 == 0) {
     // paired-head kernel (the two query heads of a pair share a KV head)
@@ -717,6 +740,8 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
     pp.gain = p.gain;
     pp.tau = p.tau;
     pp.out = p.out;
+    pp.lse = p.lse;
+    pp.out_f32 = p.out_f32;
     pp.err = p.err;
     const bool bias = a.lsig != nullptr && a.gain != nullptr;
     CUtensorMap tka;

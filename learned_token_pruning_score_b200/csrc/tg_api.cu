@@ -158,6 +158,42 @@ struct AttnPlan {
   }
 };
 
+// Backward of the standalone gated attention (bf16, head_dim 128).
+struct AttnBwdPlan {
+  void* q_rot = nullptr;   // [n, hq, dh] rotated as in the forward
+  void* k_rot = nullptr;   // [n, hkv, dh]
+  float* lsig = nullptr;   // [n]
+  float2* cs = nullptr;    // [dh/2, n] RoPE table
+  void* qT = nullptr;      // [hq, dh, t_pad]
+  void* kT = nullptr;      // [hkv, dh, t_pad]
+  void* doT = nullptr;     // [hq, dh, t_pad]
+  float* lse2 = nullptr;   // [hq, t_pad]
+  float* dd = nullptr;     // [hq, t_pad]
+  float* colsum = nullptr; // [hq, t_pad]
+  float* qdq = nullptr;    // [hq, t_pad / 128, 4]
+  float* bias = nullptr;   // [t_pad] logsigmoid(s), zero-padded
+  int64_t t_pad = 0;
+  size_t bytes = 0;
+  AttnBwdPlan(void* ws, int64_t n, int hq, int hkv, int dh) {
+    Arena a(ws);
+    t_pad = static_cast<int64_t>(attn_bwd_t_pad(n));
+    const size_t tp = static_cast<size_t>(t_pad);
+    q_rot = a.carve(size_t(n) * hq * dh * 2);
+    k_rot = a.carve(size_t(n) * hkv * dh * 2);
+    lsig = static_cast<float*>(a.carve(size_t(n) * 4 + 16));
+    cs = static_cast<float2*>(a.carve(size_t(dh / 2) * n * 8));
+    qT = a.carve(size_t(hq) * dh * tp * 2);
+    kT = a.carve(size_t(hkv) * dh * tp * 2);
+    doT = a.carve(size_t(hq) * dh * tp * 2);
+    lse2 = static_cast<float*>(a.carve(size_t(hq) * tp * 4));
+    dd = static_cast<float*>(a.carve(size_t(hq) * tp * 4));
+    colsum = static_cast<float*>(a.carve(size_t(hq) * tp * 4));
+    qdq = static_cast<float*>(a.carve(size_t(hq) * (tp / 128) * 16));
+    bias = static_cast<float*>(a.carve(tp * 4));
+    bytes = a.used;
+  }
+};
+
 struct PrefillPlan {
   void* h = nullptr;       // [n, d] residual stream (all-token stage)
   void* hk = nullptr;      // [k, d] residual stream (kept rows)
@@ -292,7 +328,7 @@ cudaError_t run_score(const void* x, int64_t rows, int d, int f, const float* no
 cudaError_t attn_core(const AttnPlan& plan, const void* k_rot, const void* v, int64_t v_stride,
                       const float* lsig, const void* kaug, const float* gain, const float* tau,
                       int64_t rows, int hq, int hkv, int dh, tg_dtype dt, void* out,
-                      cudaStream_t st) {
+                      cudaStream_t st, float* lse = nullptr, float* out_f32 = nullptr) {
   const size_t es = elem_size(dt);
   const double attn_flops = 4.0 * dh * hq * double(rows) * double(rows + 1) / 2.0;
   const double attn_bytes = double(rows) * (2 * hq + 2 * hkv) * dh * es;
@@ -304,6 +340,8 @@ cudaError_t attn_core(const AttnPlan& plan, const void* k_rot, const void* v, in
   a.gain = gain; a.tau = tau;
   a.T = rows; a.hq = hq; a.hkv = hkv; a.dh = dh;
   a.out = out;
+  a.lse = lse;
+  a.out_f32 = out_f32;
   if (dt == TG_BF16) {
     a.v = plan.vT;
     a.t_pad = plan.t_pad;
@@ -324,7 +362,7 @@ cudaError_t run_attention(const void* q, int64_t q_stride, const void* kk, int64
                           const float* q_norm, const float* k_norm, float eps, int64_t rows,
                           int hq, int hkv, int dh, float rope_base, tg_dtype dt,
                           const AttnPlan& plan, void* k_out, void* v_out, void* out,
-                          cudaStream_t st) {
+                          cudaStream_t st, float* lse = nullptr, float* out_f32 = nullptr) {
   RopePrepArgs r{};
   r.q_src = q; r.k_src = kk; r.v_src = v;
   r.q_stride = q_stride; r.k_stride = k_stride; r.v_stride = v_stride;
@@ -352,7 +390,7 @@ cudaError_t run_attention(const void* q, int64_t q_stride, const void* kk, int64
     if (e != cudaSuccess) return e;
   }
   return attn_core(plan, r.k_out, v, v_stride, lsig, dt == TG_BF16 ? plan.kaug : nullptr, gain,
-                   tau, rows, hq, hkv, dh, dt, out, st);
+                   tau, rows, hq, hkv, dh, dt, out, st, lse, out_f32);
 }
 
 // ---- the decoder-layer pieces used by tg_prefill
@@ -548,6 +586,8 @@ size_t tg_workspace_size(tg_op op, const tg_shape* s) {
       return 0;
     case TG_OP_GATED_ATTN:
       return AttnPlan(nullptr, s->k, s->n_heads_q, s->n_heads_kv, s->head_dim, s->dtype, true).bytes;
+    case TG_OP_GATED_ATTN_BWD:
+      return AttnBwdPlan(nullptr, s->k, s->n_heads_q, s->n_heads_kv, s->head_dim).bytes;
     case TG_OP_PREFILL: {
       tg_model m{};
       m.dtype = s->dtype;
@@ -641,11 +681,13 @@ tg_status tg_compact(const void* x, const int32_t* pos_in, const float* scores,
                              pos_out, scores_out, nullptr, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-tg_status tg_gated_attn_prefill(const void* q, const void* kk, const void* v, const int32_t* pos,
-                                const float* s, const float* gain, const float* tau, int64_t k,
-                                int32_t hq, int32_t hkv, int32_t dh, float rope_base,
-                                tg_dtype dt, void* out, void* ws, size_t ws_bytes,
-                                tg_stream stream) {
+}  // extern "C"
+
+namespace {
+tg_status gated_attn(const void* q, const void* kk, const void* v, const int32_t* pos,
+                     const float* s, const float* gain, const float* tau, int64_t k, int32_t hq,
+                     int32_t hkv, int32_t dh, float rope_base, tg_dtype dt, void* out, float* lse,
+                     float* out_f32, void* ws, size_t ws_bytes, tg_stream stream) {
   TG_CHECK(dt == TG_BF16 || dt == TG_F32, TG_ERR_UNSUPPORTED);
   TG_CHECK(q && kk && v && pos && out && k >= 1 && hq >= 1 && hkv >= 1, TG_ERR_INVALID_ARG);
   TG_CHECK(k < (int64_t(1) << 31) - 256, TG_ERR_INVALID_ARG);
@@ -662,7 +704,92 @@ tg_status tg_gated_attn_prefill(const void* q, const void* kk, const void* v, co
   return cuda_status(run_attention(q, int64_t(hq) * dh, kk, int64_t(hkv) * dh, v,
                                    int64_t(hkv) * dh, pos, s, nullptr, gain, tau, nullptr, nullptr,
                                    0.f, k, hq, hkv, dh, rope_base, dt, plan, nullptr, nullptr, out,
-                                   reinterpret_cast<cudaStream_t>(stream)));
+                                   reinterpret_cast<cudaStream_t>(stream), lse, out_f32));
+}
+}  // namespace
+
+extern "C" {
+
+tg_status tg_gated_attn_prefill(const void* q, const void* kk, const void* v, const int32_t* pos,
+                                const float* s, const float* gain, const float* tau, int64_t k,
+                                int32_t hq, int32_t hkv, int32_t dh, float rope_base,
+                                tg_dtype dt, void* out, void* ws, size_t ws_bytes,
+                                tg_stream stream) {
+  return gated_attn(q, kk, v, pos, s, gain, tau, k, hq, hkv, dh, rope_base, dt, out, nullptr,
+                    nullptr, ws, ws_bytes, stream);
+}
+
+tg_status tg_gated_attn_forward(const void* q, const void* kk, const void* v, const int32_t* pos,
+                                const float* s, const float* gain, const float* tau, int64_t k,
+                                int32_t hq, int32_t hkv, int32_t dh, float rope_base,
+                                tg_dtype dt, void* out, float* lse, float* out_f32, void* ws,
+                                size_t ws_bytes, tg_stream stream) {
+  TG_CHECK(dt == TG_BF16 || dt == TG_F32, TG_ERR_UNSUPPORTED);
+  TG_CHECK(dt == TG_BF16, TG_ERR_UNSUPPORTED);
+  TG_CHECK(lse != nullptr && aligned16(out_f32), TG_ERR_INVALID_ARG);
+  return gated_attn(q, kk, v, pos, s, gain, tau, k, hq, hkv, dh, rope_base, dt, out, lse, out_f32,
+                    ws, ws_bytes, stream);
+}
+
+tg_status tg_gated_attn_backward(const void* q, const void* kk, const void* v, const int32_t* pos,
+                                 const float* s, const float* gain, const float* tau, int64_t k,
+                                 int32_t hq, int32_t hkv, int32_t dh, float rope_base, tg_dtype dt,
+                                 const void* out, const float* out_f32, const float* lse,
+                                 const void* dout, void* dq,
+                                 void* dk, void* dv, float* ds, float* dgain, float* dtau,
+                                 void* ws, size_t ws_bytes, tg_stream stream) {
+  TG_CHECK(dt == TG_BF16 || dt == TG_F32, TG_ERR_UNSUPPORTED);
+  TG_CHECK(dt == TG_BF16 && dh == 128, TG_ERR_UNSUPPORTED);
+  TG_CHECK(q && kk && v && pos && out && lse && dout && dq && dk && dv, TG_ERR_INVALID_ARG);
+  TG_CHECK(k >= 1 && hq >= 1 && hkv >= 1 && k < (int64_t(1) << 31) - 256, TG_ERR_INVALID_ARG);
+  TG_CHECK(hq % hkv == 0 && rope_base > 1.f, TG_ERR_INVALID_ARG);
+  TG_CHECK(ds == nullptr || s != nullptr, TG_ERR_INVALID_ARG);
+  TG_CHECK(aligned16(q) && aligned16(kk) && aligned16(v) && aligned16(out) && aligned16(dout) &&
+               aligned16(dq) && aligned16(dk) && aligned16(dv) && aligned16(ws) &&
+               aligned16(out_f32),
+           TG_ERR_INVALID_ARG);
+  AttnBwdPlan plan(nullptr, k, hq, hkv, dh);
+  TG_CHECK(ws != nullptr && ws_bytes >= plan.bytes, TG_ERR_WORKSPACE);
+  plan = AttnBwdPlan(ws, k, hq, hkv, dh);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  RopePrepArgs r{};
+  r.q_src = q; r.k_src = kk; r.v_src = v;
+  r.q_stride = int64_t(hq) * dh; r.k_stride = int64_t(hkv) * dh; r.v_stride = int64_t(hkv) * dh;
+  r.pos = pos;
+  r.T = k; r.hq = hq; r.hkv = hkv; r.dh = dh; r.rope_base = rope_base;
+  r.bf16 = true;
+  r.q_out = plan.q_rot;
+  r.k_out = plan.k_rot;
+  r.t_pad = plan.t_pad;
+  r.s = s;
+  r.lsig_out = plan.lsig;
+  const double rows = double(k);
+  TG_TRY(traced(TG_K_ROPE_PREP, k, 0.0, rows * (hq + hkv) * dh * 4.0 + (s ? 8.0 * rows : 0.0), st,
+                [&] { return launch_rope_prep(r, st); }));
+  TG_TRY(traced(TG_K_ROPE_TABLE, k, 0.0, 8.0 * (dh / 2) * rows, st,
+                [&] { return launch_rope_table(pos, k, dh, rope_base, plan.cs, st); }));
+  AttnBwdArgs a{};
+  a.q_rot = plan.q_rot; a.k_rot = plan.k_rot; a.v = v; a.out = out; a.dout = dout;
+  a.out_f32 = out_f32;
+  a.lse = lse; a.s = s; a.lsig = s ? plan.lsig : nullptr; a.gain = gain; a.tau = tau;
+  a.cs = plan.cs;
+  a.T = k; a.t_pad = plan.t_pad; a.hq = hq; a.hkv = hkv;
+  a.qT = plan.qT; a.kT = plan.kT; a.doT = plan.doT;
+  a.lse2 = plan.lse2; a.dd = plan.dd; a.colsum = plan.colsum; a.qdq = plan.qdq;
+  a.bias = plan.bias;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.ds = ds; a.dgain = dgain; a.dtau = dtau;
+  // one [T x T x dh] causal product of all query heads (half of the forward's FLOPs)
+  const double prod = 2.0 * dh * hq * rows * (rows + 1) / 2.0;
+  TG_TRY(traced(TG_K_ATTN_BWD_PREP, k, 0.0, rows * (2 * hq + hkv) * dh * 4.0 + rows * hq * dh * 2.0,
+                st, [&] { return launch_attn_bwd(a, st, 0); }));
+  TG_TRY(traced(TG_K_ATTN_BWD_DKDV, k, 4.0 * prod, 0.0, st,
+                [&] { return launch_attn_bwd(a, st, 1); }));
+  TG_TRY(traced(TG_K_ATTN_BWD_DQ, k, 3.0 * prod, 0.0, st,
+                [&] { return launch_attn_bwd(a, st, 2); }));
+  if (ds || dgain || dtau)
+    TG_TRY(traced(TG_K_ATTN_BWD_FINAL, k, 0.0, rows * hq * 4.0, st,
+                  [&] { return launch_attn_bwd(a, st, 3); }));
+  return TG_OK;
 }
 
 tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protect, int64_t n,
@@ -882,7 +1009,8 @@ const char* tg_kernel_name(int32_t kernel) {
   static const char* names[TG_K_COUNT] = {
       "copy", "rmsnorm", "gemm_tc_store", "gemm_tc_residual", "gemm_tc_swiglu", "gemm_tc_score",
       "rope_prep", "attention_tc", "select", "compact", "gemm_f32", "attention_f32", "f32_helper",
-      "gemm_tc_qkv", "rope_table", "decode_step"};
+      "gemm_tc_qkv", "rope_table", "decode_step", "attn_bwd_prep", "attn_bwd_dkdv",
+      "attn_bwd_dq", "attn_bwd_final"};
   return (kernel >= 0 && kernel < TG_K_COUNT) ? names[kernel] : "unknown";
 }
 

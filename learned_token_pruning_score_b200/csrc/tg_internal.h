@@ -147,10 +147,33 @@ struct AttnArgs {
   const void* kaug;  // bf16 [T, 16] gate-bias rows (launch_bias_aug of lsig), needed with lsig
   int64_t T; int hq, hkv, dh;
   void* out;                                    // [T, hq, dh]
+  float* lse;      // optional [hq, T]: log sum_j exp(l_ij) per row (tensor-core path only)
+  float* out_f32;  // optional [T, hq, dh]: the output before rounding (tensor-core path only)
 };
 bool attn_tc_supported(const AttnArgs& a);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st);      // bf16, tcgen05
 cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t st); // fp32 SIMT
+
+// ---- gated-attention backward (k_attn_bwd.cu): bf16, head_dim 128.
+struct AttnBwdArgs {
+  const void* q_rot; const void* k_rot;  // [T, hq|hkv, dh] rotated as in the forward
+  const void* v; const void* out; const void* dout;  // [T, hkv|hq, dh]
+  const float* out_f32;                  // [T, hq, dh] or null (then D comes from out)
+  const float* lse;                      // [hq, T]
+  const float* s; const float* lsig;     // [T] scores and logsigmoid(scores), or null
+  const float* gain; const float* tau;   // [hq] or null
+  const float2* cs;                      // [dh/2, T] RoPE (cos, sin) table
+  int64_t T, t_pad; int hq, hkv;
+  void* qT; void* kT; void* doT;         // workspace [H, dh, t_pad]
+  float* lse2; float* dd; float* colsum; // workspace [hq, t_pad]
+  float* qdq;                            // workspace [hq, n_tiles, 4]
+  float* bias;                           // workspace [t_pad]
+  void* dq; void* dk; void* dv;          // outputs [T, H, dh]
+  float* ds; float* dgain; float* dtau;  // outputs, each optional
+};
+size_t attn_bwd_t_pad(int64_t T);
+// stage 0: prep (transposes, lse2, D); 1: dK/dV/C; 2: dQ; 3: ds/dgain/dtau.
+cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t st, int stage);
 
 // ---- decode (k_decode.cu): one generated token, batch 1, bf16, head_dim 128.
 // One cooperative launch per step runs every layer (see k_decode.cu).

@@ -308,7 +308,30 @@ def gated_attn_prefill(q, k, v, pos, s, gain, tau, rope_base, store=round_bf16):
 # ---------------------------------------------------------------------------
 
 
-def gated_attention_grads(q, k, v, pos, s, gain, tau, dout):
+def gated_attention_lse(q, k, pos, s, gain, tau) -> np.ndarray:
+    """lse[h, i] = log sum_{pos_j <= pos_i} exp(l_ij) with the logits of R2
+    (q and k as they enter the logits). The forward's softmax normaliser,
+    which its backward takes instead of recomputing it."""
+    q = np.asarray(q, dtype=F64)
+    k = np.asarray(k, dtype=F64)
+    t, hq, dh = q.shape
+    group = hq // k.shape[1]
+    gain_v = np.zeros(hq) if gain is None else np.asarray(gain, dtype=F64)
+    tau_v = np.ones(hq) if tau is None else np.asarray(tau, dtype=F64)
+    b = np.zeros(t) if s is None else logsigmoid(s)
+    p = np.asarray(pos, dtype=np.int64)
+    allowed = p[None, :] <= p[:, None]
+    out = np.empty((hq, t))
+    for h in range(hq):
+        g = h // group
+        logits = (q[:, h, :] @ k[:, g, :].T) / (math.sqrt(dh) * tau_v[h]) + gain_v[h] * b[None, :]
+        logits = np.where(allowed, logits, -np.inf)
+        m = logits.max(axis=1)
+        out[h] = m + np.log(np.exp(logits - m[:, None]).sum(axis=1))
+    return out
+
+
+def gated_attention_grads(q, k, v, pos, s, gain, tau, dout, on_head=None):
     """Gradients of o = gated_attention(q, k, v, pos, s, gain, tau) for the
     upstream gradient dout [T, Hq, dh] (q and k as they enter the logits,
     i.e. already rotated). Returns (dq, dk, dv, ds, dgain, dtau), float64.
@@ -324,7 +347,9 @@ def gated_attention_grads(q, k, v, pos, s, gain, tau, dout):
       dtau_h  = -sum_ij dl_ij a_ij / tau_h                 (d a_ij / d tau_h = -a_ij / tau_h)
       ds_j  = sigmoid(-s_j) sum_h gain_h sum_i dl_ij       (d logsigmoid(x)/dx = sigmoid(-x))
     s None means no bias: ds is None and dgain is zero; gain/tau None mean
-    0 and 1 (dgain and dtau are still returned).
+    0 and 1 (dgain and dtau are still returned). on_head, if given, is called
+    as on_head(h, g, P, dl, dP) with each head's [T, T] matrices (tests use
+    them to bound the effect of storage roundings).
     """
     q = np.asarray(q, dtype=F64)
     k = np.asarray(k, dtype=F64)
@@ -353,6 +378,8 @@ def gated_attention_grads(q, k, v, pos, s, gain, tau, dout):
         w = w / w.sum(axis=1, keepdims=True)
         dp = dout[:, h, :] @ v[:, g, :].T
         dl = w * (dp - (w * dp).sum(axis=1, keepdims=True))
+        if on_head is not None:
+            on_head(h, g, w, dl, dp)
         dq[:, h, :] = c * (dl @ k[:, g, :])
         dk[:, g, :] += c * (dl.T @ q[:, h, :])
         dv[:, g, :] += w.T @ dout[:, h, :]

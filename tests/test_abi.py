@@ -106,6 +106,37 @@ def test_attention_validation():
         tg.TG_ERR_UNSUPPORTED
 
 
+def test_attention_forward_lse_and_backward_validation():
+    fwd = tg._attn_fwd
+    base = [BOGUS, BOGUS, BOGUS, BOGUS, None, None, None, 128, 4, 2, 128, 1e6]
+    assert fwd(*base, tg.TG_BF16, BOGUS, None, None, BOGUS, 1 << 30, None) == \
+        tg.TG_ERR_INVALID_ARG  # no lse
+    assert fwd(*base, tg.TG_BF16, BOGUS, BOGUS, ctypes.c_void_p(4096 + 4), BOGUS, 1 << 30,
+               None) == tg.TG_ERR_INVALID_ARG  # misaligned fp32 output
+    assert fwd(*base, tg.TG_F32, BOGUS, BOGUS, None, BOGUS, 1 << 30, None) == \
+        tg.TG_ERR_UNSUPPORTED
+    assert fwd(*base, tg.TG_BF16, BOGUS, BOGUS, None, BOGUS, 64, None) == tg.TG_ERR_WORKSPACE
+    bwd = tg._attn_bwd
+    need = tg.tg_workspace_size(tg.TG_OP_GATED_ATTN_BWD, k=128, n_heads_q=4, n_heads_kv=2,
+                                head_dim=128, dtype=tg.TG_BF16)
+    # rotated q and k, Q^T, K^T, dO^T, the RoPE table and the per-row vectors
+    assert need >= 128 * 128 * 2 * (4 + 2 + 4 + 2 + 4) + 64 * 128 * 8
+    outs = [BOGUS, BOGUS, BOGUS, BOGUS, BOGUS, BOGUS]  # dq, dk, dv, ds, dgain, dtau
+
+    def call(dt=tg.TG_BF16, dh=128, hq=4, hkv=2, s=BOGUS, out=BOGUS, o=outs, ws=BOGUS,
+             ws_bytes=1 << 30):
+        return bwd(BOGUS, BOGUS, BOGUS, BOGUS, s, None, None, 128, hq, hkv, dh, 1e6, dt, out,
+                   None, BOGUS, BOGUS, *o, ws, ws_bytes, None)
+
+    assert call(dt=tg.TG_F32) == tg.TG_ERR_UNSUPPORTED
+    assert call(dh=64) == tg.TG_ERR_UNSUPPORTED
+    assert call(hkv=3) == tg.TG_ERR_INVALID_ARG  # hq % hkv != 0
+    assert call(out=None) == tg.TG_ERR_INVALID_ARG
+    assert call(s=None) == tg.TG_ERR_INVALID_ARG  # ds asked for without scores
+    assert call(ws=ctypes.c_void_p(4096 + 8)) == tg.TG_ERR_INVALID_ARG  # misaligned workspace
+    assert call(ws_bytes=need - 1) == tg.TG_ERR_WORKSPACE
+
+
 def _bogus_model(**over):
     layers = (tg.TgLayer * 2)()
     for i in range(2):

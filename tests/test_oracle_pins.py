@@ -446,6 +446,23 @@ def test_attention_backward_matches_torch_autograd():
         assert np.allclose(mine, theirs.numpy(), rtol=1e-9, atol=1e-11)
 
 
+def test_attention_lse_closed_forms():
+    q, k, v, pos, s, gain, tau, dout = _bwd_case(24, t=10)
+    # q = 0 and no bias: every visible logit is 0, so lse_i = log(i + 1)
+    lse0 = ref.gated_attention_lse(np.zeros_like(q), k, pos, None, gain, tau)
+    assert np.allclose(lse0, np.log(np.arange(1, 11))[None, :], atol=1e-14)
+    # q = 0 with the bias: lse_i = log sum_{j <= i} sigmoid(s_j)^gain_h
+    lse1 = ref.gated_attention_lse(np.zeros_like(q), k, pos, s, gain, tau)
+    sig = 1.0 / (1.0 + np.exp(-s))
+    want = np.log(np.cumsum(sig[None, :] ** gain[:, None], axis=1))
+    assert np.allclose(lse1, want, atol=1e-13)
+    # the first row sees only itself: lse_0 = l_00
+    lse = ref.gated_attention_lse(q, k, pos, s, gain, tau)
+    for h in range(4):
+        l00 = q[0, h] @ k[0, h // 2] / (math.sqrt(8) * tau[h]) + gain[h] * math.log(sig[0])
+        assert lse[h, 0] == pytest.approx(l00, abs=1e-13)
+
+
 def test_attention_backward_invariants_and_degenerate_cases():
     q, k, v, pos, s, gain, tau, dout = _bwd_case(23, t=9)
     # constant scores: each head's key sums of dl vanish (softmax rows sum to
