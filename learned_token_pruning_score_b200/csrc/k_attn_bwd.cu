@@ -21,8 +21,9 @@
 // their gradients are rotated back with the transposed rotation.
 //
 // Kernels, in stream order:
-//   bwd_prep   Q^T, K^T, dO^T as [head, dh, t_pad] (the K-major B operands
-//              of the products that contract over rows), lse in log2 units,
+//   bwd_prep   q and k rotated (RoPE at the original positions), Q^T, K^T,
+//              dO^T as [head, dh, t_pad] (the K-major B operands of the
+//              products that contract over rows), the RoPE table, lse in log2 units,
 //              D (from the forward's fp32 output when given: the bf16 output
 //              carries a rounding of 2^-9 that D would pass on to every
 //              dl_ij of the row), and the zero-padded bias row logsigmoid(s).
@@ -174,18 +175,6 @@ __device__ __forceinline__ void mma_ss_128(uint32_t d, uint32_t a_addr, uint32_t
   }
 }
 
-// [128 x 128] x [128 x 128]^T over 128 rows with A packed in 64 TMEM columns.
-__device__ __forceinline__ void mma_ts_128(uint32_t d, uint32_t a_tmem, uint32_t b_addr,
-                                           bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
-#pragma unroll
-  for (int kk = 0; kk < kBlk / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
-    umma_f16_ts(d, a_tmem + static_cast<uint32_t>(kk * 8), sdesc_kmajor_sw128(b_addr + off),
-                idesc, (accumulate || kk > 0) ? 1u : 0u);
-  }
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -202,9 +191,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* b_full = bars + 3;
   uint64_t* b_empty = bars + 4;
   uint64_t* s_full = bars + 5;
-  uint64_t* p_full = bars + 6;
-  uint64_t* acc_full = bars + 7;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  uint64_t* p_half = bars + 6;  // [2]: P^T, dS^T of queries 0-63 / 64-127 written
+  uint64_t* acc_full = bars + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int jt = static_cast<int>(blockIdx.x) / p.hkv;  // key tile 0 (the longest) first
@@ -222,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(b_full, 1);
     mbar_init(b_empty, 1);
     mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
+    mbar_init(&p_half[0], 128);
+    mbar_init(&p_half[1], 128);
     mbar_init(acc_full, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -267,6 +257,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
+    // dV += P^T dO and dK += dS^T Q go in two halves of 64 queries each: the
+    // first half runs while the rows of the second are still being formed.
+    constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+    auto grad_half = [&](int half, bool accumulate) {
+      const uint32_t dot_addr = smem_addr(smem + kOffDOT) + half * kSub;
+      const uint32_t qt_addr = smem_addr(smem + kOffQT) + half * kSub;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t col = static_cast<uint32_t>(half * 32 + kk * 8);
+        umma_f16_ts(tmem + 256, tmem + col, sdesc_kmajor_sw128(dot_addr + kk * 32), idesc,
+                    (accumulate || kk > 0) ? 1u : 0u);
+        umma_f16_ts(tmem + 384, tmem + 128 + col, sdesc_kmajor_sw128(qt_addr + kk * 32), idesc,
+                    (accumulate || kk > 0) ? 1u : 0u);
+      }
+    };
     bool ok = mbar_wait(kv_full, 0, p.err);
     for (int n = 0; n < n_it && ok; ++n) {
       const uint32_t ph = n & 1;
@@ -276,10 +281,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_ss_128(tmem + 128, smem_addr(smem + kOffV), smem_addr(smem + kOffDO));  // dP^T
       umma_commit(s_full);
       umma_commit(a_empty);
-      if (!mbar_wait(p_full, ph, p.err) || !mbar_wait(b_full, ph, p.err)) break;
+      if (!mbar_wait(&p_half[0], ph, p.err) || !mbar_wait(b_full, ph, p.err)) break;
       tc_fence_after();
-      mma_ts_128(tmem + 256, tmem + 0, smem_addr(smem + kOffDOT), n > 0);    // dV += P^T dO
-      mma_ts_128(tmem + 384, tmem + 128, smem_addr(smem + kOffQT), n > 0);   // dK += dS^T Q
+      grad_half(0, n > 0);
+      if (!mbar_wait(&p_half[1], ph, p.err)) break;
+      tc_fence_after();
+      grad_half(1, true);
       umma_commit(b_empty);
     }
     if (ok) umma_commit(acc_full);
@@ -332,10 +339,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st16(tmem + lane_off + static_cast<uint32_t>(16 * c), pk);
         tmem_st16(tmem + lane_off + 128u + static_cast<uint32_t>(16 * c), dk16);
+        if (c & 1) {  // queries 0-63 (c = 1) or 64-127 (c = 3) done
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&p_half[c >> 1]);
+        }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full);
       if (n % n_q == n_q - 1) {  // last query tile of head h: C_hj is complete
         if (p.colsum && j < p.T) p.colsum[static_cast<int64_t>(h) * p.t_pad + j] = csum;
         csum = 0.f;
@@ -605,84 +614,124 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ============================================================================
-// Prep: [T, H, dh] rows -> [H, dh, t_pad] (zero past T) for q_rot, k_rot and
-// dO; for dO's heads also lse2 = lse * log2(e) and D = dO . o per row.
+// Prep, one CTA per (64 rows, head slot); the slots are the hq query heads,
+// the hkv key heads and the hq heads of dO. Query and key rows are rotated
+// by RoPE at their positions (the arithmetic of rope_cos_sin with theta_i
+// computed once per CTA) and written row-major for the 128-row operand
+// tiles; every slot is also written transposed, [head, dh, t_pad], for the
+// K-major operands of the products that contract over rows. The CTAs of
+// query head 0 write the (cos, sin) table that rotates the gradients back;
+// those of key head 0 the zero-padded bias row logsigmoid(s); those of dO
+// lse * log2(e) and D = dO . o per row.
+// The [64 x 128] tile sits in shared memory as 32-bit words (two bf16),
+// word w of row r at r * 64 + (w ^ (r >> 1)): the row-wise fill and the
+// column-wise reads of the transpose (two rows per lane) are both free of
+// bank conflicts.
 struct PrepArgs {
-  const __nv_bfloat16* src[3];  // q_rot, k_rot, dO
+  const __nv_bfloat16* src[3];  // q, k (un-rotated), dO: [T, H, 128]
   int heads[3];
-  __nv_bfloat16* dst[3];
+  __nv_bfloat16* rot[2];        // q_rot, k_rot [T, H, 128]
+  __nv_bfloat16* dst[3];        // [H, 128, t_pad]
+  const int32_t* pos;
+  float rope_base;
   const __nv_bfloat16* out;     // forward output [T, hq, dh]
   const float* out_f32;         // the same before rounding, or null
   const float* lse;             // [hq, T]
-  const float* lsig;            // [T] or null
+  const float* s;               // [T] or null
   float* lse2;                  // [hq, t_pad]
   float* dd;                    // [hq, t_pad]
-  float* bias;                  // [t_pad]: lsig, zero past T (all zero without lsig)
+  float* bias;                  // [t_pad]: logsigmoid(s), zero past T (all zero without s)
+  float2* cs;                   // [64, T]
   int64_t T, t_pad;
 };
+
+__device__ __forceinline__ float2 rope_cs_theta(int64_t pos, double theta) {
+  const double ang = static_cast<double>(pos) * theta;
+  const double two_pi = 6.283185307179586476925286766559;
+  const double red = ang - two_pi * rint(ang * (1.0 / two_pi));
+  float sv, cv;
+  sincosf(static_cast<float>(red), &sv, &cv);
+  return make_float2(cv, sv);
+}
 
 __global__ void __launch_bounds__(256) attn_bwd_prep(PrepArgs a) {
   pdl_trigger();
   pdl_wait();
   constexpr int kRows = 64;
-  constexpr int kLd = kDh + 8;  // padded row (bf16 elements)
-  __shared__ __align__(16) __nv_bfloat16 tile[kRows * kLd];
+  __shared__ uint32_t tile[kRows * 64];
+  __shared__ double theta[64];
   int slot = blockIdx.y, which = 0;
   while (which < 2 && slot >= a.heads[which]) slot -= a.heads[which++];
-  const int H = a.heads[which], h = slot;
-  const __nv_bfloat16* src = a.src[which];
+  const int h = slot;
+  const int H = which == 1 ? a.heads[1] : a.heads[0];
+  const __nv_bfloat16* src = which == 0 ? a.src[0] : (which == 1 ? a.src[1] : a.src[2]);
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRows;
-  constexpr int kVec = kDh / 8;
-  for (int e = threadIdx.x; e < kRows * kVec; e += 256) {
-    const int rr = e / kVec, c = e % kVec;
-    const int64_t t = t0 + rr;
-    uint4 u = make_uint4(0, 0, 0, 0);
-    if (t < a.T) u = __ldg(reinterpret_cast<const uint4*>(src + (t * H + h) * kDh) + c);
-    *reinterpret_cast<uint4*>(&tile[rr * kLd + c * 8]) = u;
+  if (which < 2 && threadIdx.x < 64)
+    theta[threadIdx.x] = exp2(-(2.0 * threadIdx.x / kDh) * log2(static_cast<double>(a.rope_base)));
+  __syncthreads();
+  __nv_bfloat16* rot = which == 0 ? a.rot[0] : a.rot[1];
+  for (int e = threadIdx.x; e < kRows * 32; e += 256) {
+    const int r = e >> 5, w = e & 31;  // words w and w + 32: elements (2w, 2w+1) and (2w+64, 2w+65)
+    const int64_t t = t0 + r;
+    uint32_t lo = 0u, hi = 0u;
+    if (t < a.T) {
+      const uint32_t* row = reinterpret_cast<const uint32_t*>(src + (t * H + h) * kDh);
+      lo = __ldg(row + w);
+      hi = __ldg(row + w + 32);
+      if (which < 2) {
+        const int64_t p = a.pos ? __ldg(a.pos + t) : t;
+        const float2 c0 = rope_cs_theta(p, theta[2 * w]);
+        const float2 c1 = rope_cs_theta(p, theta[2 * w + 1]);
+        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
+        const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
+        lo = pack_bf16x2(x.x * c0.x - y.x * c0.y, x.y * c1.x - y.y * c1.y);
+        hi = pack_bf16x2(y.x * c0.x + x.x * c0.y, y.y * c1.x + x.y * c1.y);
+        uint32_t* rrow = reinterpret_cast<uint32_t*>(rot + (t * H + h) * kDh);
+        rrow[w] = lo;
+        rrow[w + 32] = hi;
+        if (which == 0 && h == 0) {
+          a.cs[static_cast<int64_t>(2 * w) * a.T + t] = c0;
+          a.cs[static_cast<int64_t>(2 * w + 1) * a.T + t] = c1;
+        }
+      }
+    }
+    tile[r * 64 + (w ^ (r >> 1))] = lo;
+    tile[r * 64 + ((w + 32) ^ (r >> 1))] = hi;
   }
   if (which == 1 && h == 0 && threadIdx.x < kRows) {
     const int64_t t = t0 + threadIdx.x;
-    a.bias[t] = (a.lsig && t < a.T) ? __ldg(a.lsig + t) : 0.0f;
+    a.bias[t] = (a.s && t < a.T) ? logsigmoid_f(__ldg(a.s + t)) : 0.0f;
   }
   __syncthreads();
   __nv_bfloat16* dst = a.dst[which] + static_cast<int64_t>(h) * kDh * a.t_pad;
-  for (int e = threadIdx.x; e < kDh * (kRows / 8); e += 256) {
-    const int d = e / (kRows / 8), c = e % (kRows / 8);
-    uint4 o;
-    __nv_bfloat16* oe = reinterpret_cast<__nv_bfloat16*>(&o);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) oe[q] = tile[(c * 8 + q) * kLd + d];
-    *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(d) * a.t_pad + t0 + c * 8) = o;
+  for (int e = threadIdx.x; e < kDh * 32; e += 256) {
+    const int d = e >> 5, l = e & 31;  // output row d, rows 2l and 2l + 1 of the tile
+    const int w = d >> 1, sh = (d & 1) * 16;
+    const uint32_t w0 = tile[(2 * l) * 64 + (w ^ l)];
+    const uint32_t w1 = tile[(2 * l + 1) * 64 + (w ^ l)];
+    const uint32_t v = ((w0 >> sh) & 0xFFFFu) | (((w1 >> sh) & 0xFFFFu) << 16);
+    *reinterpret_cast<uint32_t*>(dst + static_cast<int64_t>(d) * a.t_pad + t0 + 2 * l) = v;
   }
   if (which == 2) {
-    // four threads per row, 32 elements each
+    // four threads per row, 16 words (32 elements) each
     const int rr = threadIdx.x >> 2, part = threadIdx.x & 3;
     const int64_t t = t0 + rr;
     float acc = 0.f;
-    if (t < a.T && a.out_f32) {
-      const float4* o4 = reinterpret_cast<const float4*>(a.out_f32 + (t * H + h) * kDh + part * 32);
-#pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        const float4 f = __ldg(o4 + v);
-        const int d = part * 32 + v * 4;
-        acc = fmaf(f.x, __bfloat162float(tile[rr * kLd + d]), acc);
-        acc = fmaf(f.y, __bfloat162float(tile[rr * kLd + d + 1]), acc);
-        acc = fmaf(f.z, __bfloat162float(tile[rr * kLd + d + 2]), acc);
-        acc = fmaf(f.w, __bfloat162float(tile[rr * kLd + d + 3]), acc);
-      }
-    } else if (t < a.T) {
-      const uint4* o4 = reinterpret_cast<const uint4*>(a.out + (t * H + h) * kDh + part * 32);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const uint4 u = __ldg(o4 + v);
-        const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(e2[q]);
-          const int d = part * 32 + v * 8 + 2 * q;
-          acc = fmaf(f.x, __bfloat162float(tile[rr * kLd + d]),
-                     fmaf(f.y, __bfloat162float(tile[rr * kLd + d + 1]), acc));
+    if (t < a.T) {
+      const int64_t base = (t * H + h) * kDh;
+#pragma unroll 4
+      for (int k = 0; k < 16; ++k) {
+        const int w = part * 16 + k;
+        const uint32_t u = tile[rr * 64 + (w ^ (rr >> 1))];
+        const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+        float2 o;
+        if (a.out_f32) {
+          o = __ldg(reinterpret_cast<const float2*>(a.out_f32 + base) + w);
+        } else {
+          const uint32_t ob = __ldg(reinterpret_cast<const uint32_t*>(a.out + base) + w);
+          o = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ob));
         }
+        acc = fmaf(g.x, o.x, fmaf(g.y, o.y, acc));
       }
     }
     acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 1);
@@ -700,7 +749,7 @@ __global__ void __launch_bounds__(256) attn_bwd_prep(PrepArgs a) {
 // 256 keys each (ds_j). Fixed summation order throughout.
 struct FinalArgs {
   const float* s;       // [T] scores (null: no scores)
-  const float* lsig;    // [T]
+  const float* bias;    // [t_pad] logsigmoid(s)
   const float* gain;    // [hq] or null
   const float* tau;     // [hq] or null
   const float* colsum;  // [hq, t_pad]
@@ -731,9 +780,9 @@ __global__ void __launch_bounds__(256) attn_bwd_final(FinalArgs a) {
   if (static_cast<int>(blockIdx.x) < a.hq) {
     const int h = blockIdx.x;
     float acc = 0.f;
-    if (a.lsig)
+    if (a.s)
       for (int64_t j = threadIdx.x; j < a.T; j += 256)
-        acc = fmaf(__ldg(a.lsig + j), __ldg(a.colsum + static_cast<int64_t>(h) * a.t_pad + j), acc);
+        acc = fmaf(__ldg(a.bias + j), __ldg(a.colsum + static_cast<int64_t>(h) * a.t_pad + j), acc);
     const float dg = block_sum_256(acc, red);
     float acc2 = 0.f;
     for (int e = threadIdx.x; e < a.n_tiles * 4; e += 256)
@@ -764,22 +813,27 @@ cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t st, int stage) {
   const int n_tiles = static_cast<int>((a.T + kBlk - 1) / kBlk);
   if (stage == 0) {
     PrepArgs pa{};
-    pa.src[0] = static_cast<const __nv_bfloat16*>(a.q_rot);
-    pa.src[1] = static_cast<const __nv_bfloat16*>(a.k_rot);
+    pa.src[0] = static_cast<const __nv_bfloat16*>(a.q);
+    pa.src[1] = static_cast<const __nv_bfloat16*>(a.k);
     pa.src[2] = static_cast<const __nv_bfloat16*>(a.dout);
     pa.heads[0] = a.hq;
     pa.heads[1] = a.hkv;
     pa.heads[2] = a.hq;
+    pa.rot[0] = static_cast<__nv_bfloat16*>(a.q_rot);
+    pa.rot[1] = static_cast<__nv_bfloat16*>(a.k_rot);
     pa.dst[0] = static_cast<__nv_bfloat16*>(a.qT);
     pa.dst[1] = static_cast<__nv_bfloat16*>(a.kT);
     pa.dst[2] = static_cast<__nv_bfloat16*>(a.doT);
+    pa.pos = a.pos;
+    pa.rope_base = a.rope_base;
     pa.out = static_cast<const __nv_bfloat16*>(a.out);
     pa.out_f32 = a.out_f32;
     pa.lse = a.lse;
-    pa.lsig = a.lsig;
+    pa.s = a.s;
     pa.lse2 = a.lse2;
     pa.dd = a.dd;
     pa.bias = a.bias;
+    pa.cs = a.cs;
     pa.T = a.T;
     pa.t_pad = a.t_pad;
     const dim3 grid(static_cast<unsigned>(a.t_pad / 64), static_cast<unsigned>(2 * a.hq + a.hkv));
@@ -801,13 +855,13 @@ cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t st, int stage) {
   p.dq = static_cast<__nv_bfloat16*>(a.dq);
   p.dk = static_cast<__nv_bfloat16*>(a.dk);
   p.dv = static_cast<__nv_bfloat16*>(a.dv);
-  p.colsum = a.lsig ? a.colsum : nullptr;
+  p.colsum = a.s ? a.colsum : nullptr;
   p.qdq = a.qdq;
   p.err = device_error_word();
   if (stage == 3) {
     FinalArgs f{};
     f.s = a.s;
-    f.lsig = a.lsig;
+    f.bias = a.bias;
     f.gain = a.gain;
     f.tau = a.tau;
     f.colsum = a.colsum;
@@ -816,10 +870,10 @@ cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t st, int stage) {
     f.t_pad = a.t_pad;
     f.hq = a.hq;
     f.n_tiles = n_tiles;
-    f.ds = a.lsig ? a.ds : nullptr;
+    f.ds = a.s ? a.ds : nullptr;
     f.dgain = a.dgain;
     f.dtau = a.dtau;
-    const unsigned blocks = static_cast<unsigned>(a.hq + (a.ds && a.lsig ? (a.T + 255) / 256 : 0));
+    const unsigned blocks = static_cast<unsigned>(a.hq + (a.ds && a.s ? (a.T + 255) / 256 : 0));
     TG_CUDA_TRY(launch_pdl(attn_bwd_final, dim3(blocks), dim3(256), 0, st, f));
     return cudaGetLastError();
   }

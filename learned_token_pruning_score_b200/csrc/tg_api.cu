@@ -162,7 +162,6 @@ struct AttnPlan {
 struct AttnBwdPlan {
   void* q_rot = nullptr;   // [n, hq, dh] rotated as in the forward
   void* k_rot = nullptr;   // [n, hkv, dh]
-  float* lsig = nullptr;   // [n]
   float2* cs = nullptr;    // [dh/2, n] RoPE table
   void* qT = nullptr;      // [hq, dh, t_pad]
   void* kT = nullptr;      // [hkv, dh, t_pad]
@@ -180,7 +179,6 @@ struct AttnBwdPlan {
     const size_t tp = static_cast<size_t>(t_pad);
     q_rot = a.carve(size_t(n) * hq * dh * 2);
     k_rot = a.carve(size_t(n) * hkv * dh * 2);
-    lsig = static_cast<float*>(a.carve(size_t(n) * 4 + 16));
     cs = static_cast<float2*>(a.carve(size_t(dh / 2) * n * 8));
     qT = a.carve(size_t(hq) * dh * tp * 2);
     kT = a.carve(size_t(hkv) * dh * tp * 2);
@@ -752,36 +750,24 @@ tg_status tg_gated_attn_backward(const void* q, const void* kk, const void* v, c
   TG_CHECK(ws != nullptr && ws_bytes >= plan.bytes, TG_ERR_WORKSPACE);
   plan = AttnBwdPlan(ws, k, hq, hkv, dh);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  RopePrepArgs r{};
-  r.q_src = q; r.k_src = kk; r.v_src = v;
-  r.q_stride = int64_t(hq) * dh; r.k_stride = int64_t(hkv) * dh; r.v_stride = int64_t(hkv) * dh;
-  r.pos = pos;
-  r.T = k; r.hq = hq; r.hkv = hkv; r.dh = dh; r.rope_base = rope_base;
-  r.bf16 = true;
-  r.q_out = plan.q_rot;
-  r.k_out = plan.k_rot;
-  r.t_pad = plan.t_pad;
-  r.s = s;
-  r.lsig_out = plan.lsig;
   const double rows = double(k);
-  TG_TRY(traced(TG_K_ROPE_PREP, k, 0.0, rows * (hq + hkv) * dh * 4.0 + (s ? 8.0 * rows : 0.0), st,
-                [&] { return launch_rope_prep(r, st); }));
-  TG_TRY(traced(TG_K_ROPE_TABLE, k, 0.0, 8.0 * (dh / 2) * rows, st,
-                [&] { return launch_rope_table(pos, k, dh, rope_base, plan.cs, st); }));
   AttnBwdArgs a{};
-  a.q_rot = plan.q_rot; a.k_rot = plan.k_rot; a.v = v; a.out = out; a.dout = dout;
-  a.out_f32 = out_f32;
-  a.lse = lse; a.s = s; a.lsig = s ? plan.lsig : nullptr; a.gain = gain; a.tau = tau;
-  a.cs = plan.cs;
+  a.q = q; a.k = kk; a.pos = pos; a.rope_base = rope_base;
+  a.v = v; a.out = out; a.dout = dout; a.out_f32 = out_f32;
+  a.lse = lse; a.s = s; a.gain = gain; a.tau = tau;
   a.T = k; a.t_pad = plan.t_pad; a.hq = hq; a.hkv = hkv;
+  a.q_rot = plan.q_rot; a.k_rot = plan.k_rot; a.cs = plan.cs;
   a.qT = plan.qT; a.kT = plan.kT; a.doT = plan.doT;
   a.lse2 = plan.lse2; a.dd = plan.dd; a.colsum = plan.colsum; a.qdq = plan.qdq;
   a.bias = plan.bias;
   a.dq = dq; a.dk = dk; a.dv = dv; a.ds = ds; a.dgain = dgain; a.dtau = dtau;
   // one [T x T x dh] causal product of all query heads (half of the forward's FLOPs)
   const double prod = 2.0 * dh * hq * rows * (rows + 1) / 2.0;
-  TG_TRY(traced(TG_K_ATTN_BWD_PREP, k, 0.0, rows * (2 * hq + hkv) * dh * 4.0 + rows * hq * dh * 2.0,
-                st, [&] { return launch_attn_bwd(a, st, 0); }));
+  // reads q, k, dO and o; writes q, k rotated and q, k, dO transposed
+  const double prep_bytes = rows * dh * 2.0 * (3.0 * (hq + hkv) + 2.0 * hq) +
+                            rows * hq * dh * (out_f32 ? 4.0 : 2.0);
+  TG_TRY(traced(TG_K_ATTN_BWD_PREP, k, 0.0, prep_bytes, st,
+                [&] { return launch_attn_bwd(a, st, 0); }));
   TG_TRY(traced(TG_K_ATTN_BWD_DKDV, k, 4.0 * prod, 0.0, st,
                 [&] { return launch_attn_bwd(a, st, 1); }));
   TG_TRY(traced(TG_K_ATTN_BWD_DQ, k, 3.0 * prod, 0.0, st,

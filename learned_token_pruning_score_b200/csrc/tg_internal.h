@@ -156,23 +156,26 @@ cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t st); // fp32 SI
 
 // ---- gated-attention backward (k_attn_bwd.cu): bf16, head_dim 128.
 struct AttnBwdArgs {
-  const void* q_rot; const void* k_rot;  // [T, hq|hkv, dh] rotated as in the forward
+  const void* q; const void* k;          // [T, hq|hkv, dh] as given to the forward (un-rotated)
+  const int32_t* pos; float rope_base;
   const void* v; const void* out; const void* dout;  // [T, hkv|hq, dh]
   const float* out_f32;                  // [T, hq, dh] or null (then D comes from out)
   const float* lse;                      // [hq, T]
-  const float* s; const float* lsig;     // [T] scores and logsigmoid(scores), or null
+  const float* s;                        // [T] scores, or null
   const float* gain; const float* tau;   // [hq] or null
-  const float2* cs;                      // [dh/2, T] RoPE (cos, sin) table
   int64_t T, t_pad; int hq, hkv;
+  void* q_rot; void* k_rot;              // workspace [T, hq|hkv, dh], rotated as in the forward
+  float2* cs;                            // workspace [dh/2, T] RoPE (cos, sin) table
   void* qT; void* kT; void* doT;         // workspace [H, dh, t_pad]
   float* lse2; float* dd; float* colsum; // workspace [hq, t_pad]
   float* qdq;                            // workspace [hq, n_tiles, 4]
-  float* bias;                           // workspace [t_pad]
+  float* bias;                           // workspace [t_pad] logsigmoid(s), zero-padded
   void* dq; void* dk; void* dv;          // outputs [T, H, dh]
   float* ds; float* dgain; float* dtau;  // outputs, each optional
 };
 size_t attn_bwd_t_pad(int64_t T);
-// stage 0: prep (transposes, lse2, D); 1: dK/dV/C; 2: dQ; 3: ds/dgain/dtau.
+// stage 0: prep (RoPE, transposes, table, lse2, D, bias); 1: dK/dV/C; 2: dQ;
+// 3: ds/dgain/dtau.
 cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t st, int stage);
 
 // ---- decode (k_decode.cu): one generated token, batch 1, bf16, head_dim 128.
