@@ -566,6 +566,41 @@ def run_ours(args, rank, world, local_rank):
             g = extras[f"gated_k{kk}"]
             g["ttft_speedup_vs_dense"] = extras["dense"]["ttft_ms"] / g["ttft_ms"]
             g["peak_mem_reduction_vs_dense"] = extras["dense"]["peak_mem_gb"] / g["peak_mem_gb"]
+        # one request at all three budgets: the below-gate pass and the scores
+        # once (tg_prefill_multi) against three single-budget prefills, both
+        # without KV outputs, L2 flushed before each timed call
+        ks = list(synth.PREFILL_32K_BUDGETS)
+        outs_m = [torch.empty(kk, w.d, dtype=torch.bfloat16, device=device) for kk in ks]
+        kept_m = [torch.empty(kk, dtype=torch.int32, device=device) for kk in ks]
+        ws_m = torch.empty(model.workspace_size(w.n, max(ks), w.gate_layer), dtype=torch.uint8,
+                           device=device)
+
+        def run_multi():
+            tg.tg_prefill_multi(model, x, prot, ks, w.gate_layer, outs=outs_m, kept_idx=kept_m,
+                                ws=ws_m)
+
+        def run_singles():
+            for kk, o, ki in zip(ks, outs_m, kept_m):
+                tg.tg_prefill(model, x, prot, kk, w.gate_layer, out=o, kept_idx=ki, ws=ws_m)
+
+        mb = {}
+        for name, fn in (("multi", run_multi), ("singles", run_singles)):
+            fn()
+            torch.cuda.synchronize()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(5)]
+            for a, b in evs:
+                flush.zero_()
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+            mb[name] = statistics.median([a.elapsed_time(b) for a, b in evs])
+        extras["multi_budget"] = {"budgets": ks, "ms": mb["multi"],
+                                  "separate_prefills_ms": mb["singles"],
+                                  "speedup_vs_separate": mb["singles"] / mb["multi"],
+                                  "tokens_per_s": w.n / (mb["multi"] / 1e3)}
+        del outs_m, kept_m, ws_m
         # decode over the pruned cache (next to the dense cache) after the prefill
         dec = decode_bench(tg, torch, model, w, k, False, 64, 8, device, stream, pk)
         dec_d = decode_bench(tg, torch, dense_model(tg, model), w, w.n, True, 64, 8, device,

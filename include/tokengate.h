@@ -310,6 +310,28 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
                      const tg_kv* kv, void* const* hidden, void* ws, size_t ws_bytes,
                      tg_stream stream);
 
+/*
+ * tg_prefill_multi -- the gated prefill at several budgets of one request
+ * (the mixed-budget use the pages describe: one trained gate serves every
+ * budget, and training averages the full-context loss with a random-budget
+ * loss each step; [AI] "可学习剪枝的机制设计"; [TC] "门控机制为评分网络建立梯度路径").
+ * The layers below the gate, the gate layer's attention and the scores do not
+ * depend on the budget, so they run once; then each budget ks[b] gets its
+ * own selection, compaction and upper layers, exactly as tg_prefill with that
+ * k (the same kernels on the same data: the results are bit-identical).
+ *   ks: HOST array of n_budgets budgets, 1 <= n_budgets <= TG_MAX_BUDGETS,
+ *       each valid for tg_prefill (any order, repeats allowed)
+ *   outs, kept_idx: HOST arrays of n_budgets device pointers; outs[b]
+ *       [ks[b], d] dtype, kept_idx[b] [ks[b]] int32
+ *   scores [n] fp32 (out) or NULL; no KV or per-layer outputs.
+ * Workspace: tg_workspace_size(TG_OP_PREFILL) with k = max(ks).
+ */
+#define TG_MAX_BUDGETS 64
+tg_status tg_prefill_multi(const tg_model* model, const void* x, const uint8_t* protect,
+                           int64_t n, const int64_t* ks, int32_t n_budgets, int32_t gate_layer,
+                           void* const* outs, int32_t* const* kept_idx, float* scores, void* ws,
+                           size_t ws_bytes, tg_stream stream);
+
 /* ---- decode over the pruned cache ---------------------------------------
  *
  * tg_decode_step -- one generated token through every layer after a gated

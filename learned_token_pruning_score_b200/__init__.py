@@ -94,6 +94,9 @@ _attn_bwd = _sig("tg_gated_attn_backward", _ci, _c_p, _c_p, _c_p, _c_p, _c_p, _c
 _prefill = _sig("tg_prefill", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64, _c_i64, _c_i32,
                 _c_p, _c_p, _c_p, ctypes.POINTER(TgKV), ctypes.POINTER(_c_p), _c_p, _c_sz,
                 _c_p)
+_prefill_multi = _sig("tg_prefill_multi", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64,
+                      ctypes.POINTER(_c_i64), _c_i32, _c_i32, ctypes.POINTER(_c_p),
+                      ctypes.POINTER(_c_p), _c_p, _c_p, _c_sz, _c_p)
 _decode = _sig("tg_decode_step", _ci, ctypes.POINTER(TgModel), _c_p, _c_i64, _c_i32,
                ctypes.POINTER(TgKV), ctypes.POINTER(_c_i64), _c_p, _c_i64, _c_p, _c_i64, _c_p, _c_p,
                _c_sz, _c_p)
@@ -437,8 +440,29 @@ def tg_prefill(model: Model, x, protect, k: int, gate_layer: int, out=None, kept
     return out, kept_idx, scores
 
 
+def tg_prefill_multi(model: Model, x, protect, ks: Sequence[int], gate_layer: int, outs=None,
+                     kept_idx=None, scores=None, ws=None, stream=None):
+    """The gated prefill at several budgets of one request: the layers below
+    the gate and the scores run once. Returns (outs, kept_idx, scores), the
+    first two lists with one tensor per budget."""
+    n, d = x.shape
+    nb = len(ks)
+    if outs is None:
+        outs = [torch.empty(k, d, dtype=x.dtype, device=x.device) for k in ks]
+    if kept_idx is None:
+        kept_idx = [torch.empty(k, dtype=torch.int32, device=x.device) for k in ks]
+    ws = _ws(model.workspace_size(n, max(ks), gate_layer), x.device, ws)
+    ks_c = (_c_i64 * nb)(*ks)
+    outs_c = (_c_p * nb)(*[_ptr(t) for t in outs])
+    kept_c = (_c_p * nb)(*[_ptr(t) for t in kept_idx])
+    _check(_prefill_multi(ctypes.byref(model.c), _ptr(x), _ptr(protect), n, ks_c, nb, gate_layer,
+                          outs_c, kept_c, _ptr(scores), _ptr(ws), ws.numel(),
+                          _stream(stream, x.device)), "tg_prefill_multi")
+    return outs, kept_idx, scores
+
+
 __all__ = [
-    "tg_score", "tg_linear", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_gated_attn_forward", "tg_gated_attn_backward", "tg_prefill", "tg_decode_step",
+    "tg_score", "tg_linear", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_gated_attn_forward", "tg_gated_attn_backward", "tg_prefill", "tg_prefill_multi", "tg_decode_step",
     "tg_workspace_size", "tg_status_string", "tg_device_error", "tg_version", "Model",
     "TokenGateError", "LIB_PATH", "tg_trace_start", "tg_trace_stop", "TG_OK", "TG_ERR_INVALID_ARG", "TG_ERR_UNSUPPORTED",
     "TG_ERR_BUDGET", "TG_ERR_WORKSPACE", "TG_ERR_CUDA", "TG_F32", "TG_BF16", "TG_OP_SCORE",

@@ -778,28 +778,26 @@ tg_status tg_gated_attn_backward(const void* q, const void* kk, const void* v, c
   return TG_OK;
 }
 
-tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protect, int64_t n,
-                     int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx, float* scores,
-                     const tg_kv* kv, void* const* hidden, void* ws, size_t ws_bytes,
-                     tg_stream stream) {
-  const tg_status vs = validate_model(model, n, k, gate_layer);
-  if (vs != TG_OK) return vs;
-  TG_CHECK(x && out && kept_idx, TG_ERR_INVALID_ARG);
-  const tg_model& m = *model;
-  if (m.dtype == TG_BF16) TG_CHECK(aligned16(x) && aligned16(out), TG_ERR_INVALID_ARG);
-  PrefillPlan P(nullptr, m, n, k);
-  TG_CHECK(ws != nullptr && ws_bytes >= P.bytes, TG_ERR_WORKSPACE);
-  P = PrefillPlan(ws, m, n, k);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t e = elem_size(m.dtype);
-  Dims D{m.d_model, m.n_heads_q, m.n_heads_kv, m.head_dim, m.d_ffn,
-         (m.n_heads_q + 2 * m.n_heads_kv) * m.head_dim};
-  float* sc = scores ? scores : P.scores;
+}  // extern "C"
 
-  struct LayerTag {  // annotates traced launches with their decoder layer
-    explicit LayerTag(int l) { t_trace.layer = l; }
-    ~LayerTag() { t_trace.layer = -1; }
-  };
+namespace {
+
+struct LayerTag {  // annotates traced launches with their decoder layer
+  explicit LayerTag(int l) { t_trace.layer = l; }
+  ~LayerTag() { t_trace.layer = -1; }
+};
+
+Dims model_dims(const tg_model& m) {
+  return Dims{m.d_model, m.n_heads_q, m.n_heads_kv, m.head_dim, m.d_ffn,
+              (m.n_heads_q + 2 * m.n_heads_kv) * m.head_dim};
+}
+
+// Stage 1 of the gated forward: the layers below the gate and the gate
+// layer's attention over all n rows (in P.h), then the scores of every row.
+tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan& P, const void* x,
+                             int64_t n, int gate_layer, const tg_kv* kv, void* const* hidden,
+                             float* sc, cudaStream_t st) {
+  const size_t e = elem_size(m.dtype);
   TG_TRY(copy_rows(P.h, x, size_t(n) * D.d * e, n, st));
   const bool tables = m.dtype == TG_BF16 && D.dh == 128;
   const double cs_bytes = 8.0 * (D.dh / 2);
@@ -807,7 +805,6 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
     TG_TRY(traced(TG_K_ROPE_TABLE, n, 0.0, cs_bytes * n, st, [&] {
       return launch_rope_table(nullptr, n, D.dh, m.rope_base, P.cs_n, st);
     }));
-  // Stage 1: layers below the gate, and the gate layer's attention, over n rows.
   for (int l = 0; l < gate_layer; ++l) {
     LayerTag tag(l);
     TG_TRY(attention_sublayer(m, m.layers[l], D, P, P.h, n, nullptr, P.cs_n, nullptr, nullptr,
@@ -820,9 +817,22 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
     TG_TRY(attention_sublayer(m, m.layers[gate_layer], D, P, P.h, n, nullptr, P.cs_n, nullptr,
                               nullptr, nullptr, nullptr, kv ? &kv[gate_layer] : nullptr, st));
   }
-  // Stage 2: score the post-attention residual, select, compact.
+  // score the post-attention residual
   TG_TRY(run_score(P.h, n, D.d, m.d_score, m.score_norm, m.norm_eps, m.score_w1, m.score_b1,
                    m.score_w2, m.score_b2, m.dtype, sc, P.y, P.hpre, st));
+  return TG_OK;
+}
+
+// Stages 2-3 for one budget k: select, compact, the gate layer's FFN and
+// the layers above over the k kept rows (in P.hk; P.h is only read), final
+// norm into out.
+tg_status prefill_above_gate(const tg_model& m, const Dims& D, const PrefillPlan& P,
+                             const uint8_t* protect, int64_t n, int64_t k, int gate_layer,
+                             const float* sc, void* out, int32_t* kept_idx, const tg_kv* kv,
+                             void* const* hidden, cudaStream_t st) {
+  const size_t e = elem_size(m.dtype);
+  const bool tables = m.dtype == TG_BF16 && D.dh == 128;
+  const double cs_bytes = 8.0 * (D.dh / 2);
   TG_TRY(select_topk(sc, protect, n, k, kept_idx, P.sel_ws, st));
   TG_TRY(compact(P.h, nullptr, sc, kept_idx, n, k, static_cast<int>(D.d * e), P.hk, P.pos_k, P.s_k,
                  P.lsig_k, st));
@@ -834,7 +844,6 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
     TG_TRY(traced(TG_K_ROPE_TABLE, k, 0.0, 36.0 * k, st,
                   [&] { return launch_bias_aug(P.lsig_k, k, P.kaug_k, st); }));
   }
-  // Stage 3: the gate layer's FFN and the layers above, over the k kept rows.
   if (gate_layer >= 0) {
     LayerTag tag(gate_layer);
     TG_TRY(ffn_sublayer(m, m.layers[gate_layer], D, P, P.hk, k, st));
@@ -853,6 +862,63 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
     TG_TRY(rmsnorm(P.hk, m.final_norm, m.norm_eps, k, D.d, m.dtype, out, st));
   else
     TG_TRY(copy_rows(out, P.hk, size_t(k) * D.d * e, k, st));
+  return TG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protect, int64_t n,
+                     int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx, float* scores,
+                     const tg_kv* kv, void* const* hidden, void* ws, size_t ws_bytes,
+                     tg_stream stream) {
+  const tg_status vs = validate_model(model, n, k, gate_layer);
+  if (vs != TG_OK) return vs;
+  TG_CHECK(x && out && kept_idx, TG_ERR_INVALID_ARG);
+  const tg_model& m = *model;
+  if (m.dtype == TG_BF16) TG_CHECK(aligned16(x) && aligned16(out), TG_ERR_INVALID_ARG);
+  PrefillPlan P(nullptr, m, n, k);
+  TG_CHECK(ws != nullptr && ws_bytes >= P.bytes, TG_ERR_WORKSPACE);
+  P = PrefillPlan(ws, m, n, k);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Dims D = model_dims(m);
+  float* sc = scores ? scores : P.scores;
+  const tg_status s1 = prefill_below_gate(m, D, P, x, n, gate_layer, kv, hidden, sc, st);
+  if (s1 != TG_OK) return s1;
+  return prefill_above_gate(m, D, P, protect, n, k, gate_layer, sc, out, kept_idx, kv, hidden, st);
+}
+
+tg_status tg_prefill_multi(const tg_model* model, const void* x, const uint8_t* protect,
+                           int64_t n, const int64_t* ks, int32_t n_budgets, int32_t gate_layer,
+                           void* const* outs, int32_t* const* kept_idx, float* scores, void* ws,
+                           size_t ws_bytes, tg_stream stream) {
+  TG_CHECK(ks != nullptr && outs != nullptr && kept_idx != nullptr, TG_ERR_INVALID_ARG);
+  TG_CHECK(n_budgets >= 1 && n_budgets <= TG_MAX_BUDGETS, TG_ERR_INVALID_ARG);
+  int64_t k_max = 0;
+  for (int b = 0; b < n_budgets; ++b) {
+    const tg_status vs = validate_model(model, n, ks[b], gate_layer);
+    if (vs != TG_OK) return vs;
+    TG_CHECK(outs[b] && kept_idx[b], TG_ERR_INVALID_ARG);
+    if (model->dtype == TG_BF16) TG_CHECK(aligned16(outs[b]), TG_ERR_INVALID_ARG);
+    k_max = ks[b] > k_max ? ks[b] : k_max;
+  }
+  TG_CHECK(x != nullptr, TG_ERR_INVALID_ARG);
+  const tg_model& m = *model;
+  if (m.dtype == TG_BF16) TG_CHECK(aligned16(x), TG_ERR_INVALID_ARG);
+  PrefillPlan P(nullptr, m, n, k_max);
+  TG_CHECK(ws != nullptr && ws_bytes >= P.bytes, TG_ERR_WORKSPACE);
+  P = PrefillPlan(ws, m, n, k_max);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Dims D = model_dims(m);
+  float* sc = scores ? scores : P.scores;
+  const tg_status s1 = prefill_below_gate(m, D, P, x, n, gate_layer, nullptr, nullptr, sc, st);
+  if (s1 != TG_OK) return s1;
+  for (int b = 0; b < n_budgets; ++b) {
+    const tg_status sb = prefill_above_gate(m, D, P, protect, n, ks[b], gate_layer, sc, outs[b],
+                                            kept_idx[b], nullptr, nullptr, st);
+    if (sb != TG_OK) return sb;
+  }
   return TG_OK;
 }
 

@@ -546,6 +546,16 @@ def prefill(x, protect, k: int, m: Model, gate_layer: int, store=round_bf16,
                          gate_residual=r if gate_layer < 0 else None)
 
 
+def prefill_budgets(x, protect, ks, m: Model, gate_layer: int, store=round_bf16,
+                    kept_sets=None) -> List[PrefillResult]:
+    """The gated forward of one request at several budgets: by definition the
+    single-budget forward at each k of ks (one trained gate serves every
+    budget, [AI] "可学习剪枝的机制设计"). kept_sets, when given, teacher-forces
+    each budget's kept set."""
+    return [prefill(x, protect, k, m, gate_layer, store,
+                    None if kept_sets is None else kept_sets[b]) for b, k in enumerate(ks)]
+
+
 def decode_step(x, pos: int, m: Model, gate_layer: int, cache, kept_scores=None,
                 store=round_bf16):
     """One generated token through every layer, after a gated prefill.

@@ -156,6 +156,30 @@ def _prefill(model, n, k, gate, ws_bytes):
                        ws_bytes, None)
 
 
+def test_prefill_multi_validation():
+    m, keep = _bogus_model()
+    big = 1 << 40
+
+    def call(ks, n=1000, outs=None, ws_bytes=big):
+        nb = len(ks)
+        ks_c = (ctypes.c_int64 * max(nb, 1))(*ks)
+        o = outs if outs is not None else [BOGUS] * max(nb, 1)
+        outs_c = (ctypes.c_void_p * max(nb, 1))(*[x.value if x is not None else None for x in o])
+        kept_c = (ctypes.c_void_p * max(nb, 1))(*([BOGUS.value] * max(nb, 1)))
+        return tg._prefill_multi(ctypes.byref(m), BOGUS, None, n, ks_c, nb, 1, outs_c, kept_c,
+                                 None, BOGUS, ws_bytes, None)
+
+    assert call([]) == tg.TG_ERR_INVALID_ARG  # no budgets
+    assert call([10] * 65) == tg.TG_ERR_INVALID_ARG  # more than TG_MAX_BUDGETS
+    assert call([100, 1001]) == tg.TG_ERR_BUDGET  # k > n
+    assert call([100, 0]) == tg.TG_ERR_BUDGET
+    assert call([100, 200], outs=[BOGUS, None]) == tg.TG_ERR_INVALID_ARG
+    p = dict(d_model=2048, n_heads_q=16, n_heads_kv=8, head_dim=128, d_score=256, d_ffn=6144,
+             n_layers=2, gate_layer=1, dtype=tg.TG_BF16)
+    need = tg.tg_workspace_size(tg.TG_OP_PREFILL, n=1000, k=500, **p)
+    assert call([100, 500], ws_bytes=need - 1) == tg.TG_ERR_WORKSPACE
+
+
 def test_prefill_validation():
     m, keep = _bogus_model()
     big = 1 << 40

@@ -601,6 +601,32 @@ def test_pruned_tokens_make_no_upper_kv_and_kept_set_drives_upper_layers():
     assert np.allclose(ref.rmsnorm(h, m.final_norm, m.eps), res.out, atol=1e-12)
 
 
+def test_budgets_nest_and_share_the_below_gate_pass():
+    # one request at several budgets: the scores do not depend on k, the kept
+    # sets nest (a larger budget keeps every token a smaller one keeps: the
+    # ranking is the same), the protected tokens are in every set, and K = N
+    # keeps everything
+    m = _tiny_model(31, qk_norm=True, n_layers=3)
+    n = 40
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((n, m.d_model))
+    prot = ref_protect(n, 4)
+    ks = [6, 13, 27, n]
+    res = ref.prefill_budgets(x, prot, ks, m, 1)
+    for r in res[1:]:
+        assert np.array_equal(r.scores, res[0].scores)
+    for a, b in zip(res, res[1:]):
+        assert set(a.kept_idx.tolist()) <= set(b.kept_idx.tolist())
+    for r in res:
+        assert set(np.nonzero(prot)[0].tolist()) <= set(r.kept_idx.tolist())
+    assert res[-1].kept_idx.tolist() == list(range(n))
+    # the budget-independent part (layers below the gate, the gate layer's
+    # attention) gives every budget the same below-gate KV
+    for r in res[1:]:
+        for (k0, v0), (k1, v1) in zip(res[0].kv[:2], r.kv[:2]):
+            assert np.array_equal(k0, k1) and np.array_equal(v0, v1)
+
+
 def test_work_counts():
     assert ref.attention_flops(2048, 16, 128) == pytest.approx(17.19e9, rel=1e-3)
     assert ref.select_compact_bytes(131072, 65536, 2048) == pytest.approx(538e6, rel=2e-3)
