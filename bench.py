@@ -601,6 +601,50 @@ def run_ours(args, rank, world, local_rank):
                                   "speedup_vs_separate": mb["singles"] / mb["multi"],
                                   "tokens_per_s": w.n / (mb["multi"] / 1e3)}
         del outs_m, kept_m, ws_m
+        # four requests of N/4 rows (budget K/4 each, the last 128 rows of
+        # each protected) in one batched call against four separate prefills
+        nb = 4
+        lens = [w.n // nb] * nb
+        ks_b = [k // nb] * nb
+        prot_b = torch.zeros(w.n, dtype=torch.uint8, device=device)
+        for b in range(nb):
+            prot_b[(b + 1) * lens[b] - w.n_protect:(b + 1) * lens[b]] = 1
+        out_b = torch.empty(sum(ks_b), w.d, dtype=torch.bfloat16, device=device)
+        kept_b = torch.empty(sum(ks_b), dtype=torch.int32, device=device)
+        ws_b = torch.empty(max(model.workspace_size(w.n + 128 * nb, k + 128 * nb, w.gate_layer),
+                               1), dtype=torch.uint8, device=device)
+
+        def run_batch():
+            tg.tg_prefill_batch(model, x, prot_b, lens, ks_b, w.gate_layer, out=out_b,
+                                kept_idx=kept_b, ws=ws_b)
+
+        def run_each():
+            r0 = k0 = 0
+            for n_r, k_r in zip(lens, ks_b):
+                tg.tg_prefill(model, x[r0:r0 + n_r], prot_b[r0:r0 + n_r], k_r, w.gate_layer,
+                              out=out_b[k0:k0 + k_r], kept_idx=kept_b[k0:k0 + k_r], ws=ws_b)
+                r0 += n_r
+                k0 += k_r
+
+        bt = {}
+        for name, fn in (("batch", run_batch), ("each", run_each)):
+            fn()
+            torch.cuda.synchronize()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(5)]
+            for a, b in evs:
+                flush.zero_()
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+            bt[name] = statistics.median([a.elapsed_time(b) for a, b in evs])
+        extras["batched"] = {"requests": nb, "rows_per_request": lens[0],
+                             "budget_per_request": ks_b[0], "ms": bt["batch"],
+                             "separate_prefills_ms": bt["each"],
+                             "speedup_vs_separate": bt["each"] / bt["batch"],
+                             "tokens_per_s": w.n / (bt["batch"] / 1e3)}
+        del out_b, kept_b, ws_b
         # decode over the pruned cache (next to the dense cache) after the prefill
         dec = decode_bench(tg, torch, model, w, k, False, 64, 8, device, stream, pk)
         dec_d = decode_bench(tg, torch, dense_model(tg, model), w, w.n, True, 64, 8, device,

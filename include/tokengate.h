@@ -332,6 +332,34 @@ tg_status tg_prefill_multi(const tg_model* model, const void* x, const uint8_t* 
                            void* const* outs, int32_t* const* kept_idx, float* scores, void* ws,
                            size_t ws_bytes, tg_stream stream);
 
+/*
+ * tg_prefill_batch -- the gated prefill of a batch of independent requests
+ * of different lengths in one call. Request b owns rows [cu_n[b], cu_n[b+1])
+ * of x and keeps ks[b] of them. The projection GEMMs, the norms and the
+ * scorer run over every request's rows at once (one GEMM per projection and
+ * layer for the whole batch); attention, selection and compaction run per
+ * request, each with its own positions 0..n_b-1, budget and protected span.
+ * Each request's result is the one tg_prefill gives for it alone (the same
+ * kernels on the same rows: bit-identical).
+ *   cu_n: HOST array [batch + 1], cu_n[0] = 0, strictly increasing;
+ *   ks: HOST array [batch], 1 <= ks[b] <= n_b; 1 <= batch <= TG_MAX_BATCH
+ *   x [cu_n[batch], d] bf16; protect [cu_n[batch]] uint8 or NULL
+ *   out [sum ks, d] bf16 and kept_idx [sum ks] int32: request b's rows at
+ *     offset ks[0] + ... + ks[b-1]; kept indices are local to the request
+ *     (0..n_b-1), ascending
+ *   scores [cu_n[batch]] fp32 (out) or NULL; no KV or per-layer outputs.
+ * bf16 with head_dim 128 only (TG_ERR_UNSUPPORTED otherwise). Internally
+ * every request's rows start on a 128-row boundary, so the workspace covers
+ * the padded counts: tg_prefill_batch_workspace_size (0 on invalid sizes).
+ */
+#define TG_MAX_BATCH 64
+size_t tg_prefill_batch_workspace_size(const tg_model* model, const int64_t* cu_n,
+                                       const int64_t* ks, int32_t batch);
+tg_status tg_prefill_batch(const tg_model* model, const void* x, const uint8_t* protect,
+                           const int64_t* cu_n, const int64_t* ks, int32_t batch,
+                           int32_t gate_layer, void* out, int32_t* kept_idx, float* scores,
+                           void* ws, size_t ws_bytes, tg_stream stream);
+
 /* ---- decode over the pruned cache ---------------------------------------
  *
  * tg_decode_step -- one generated token through every layer after a gated

@@ -97,6 +97,11 @@ _prefill = _sig("tg_prefill", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64, 
 _prefill_multi = _sig("tg_prefill_multi", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64,
                       ctypes.POINTER(_c_i64), _c_i32, _c_i32, ctypes.POINTER(_c_p),
                       ctypes.POINTER(_c_p), _c_p, _c_p, _c_sz, _c_p)
+_prefill_batch_ws = _sig("tg_prefill_batch_workspace_size", _c_sz, ctypes.POINTER(TgModel),
+                         ctypes.POINTER(_c_i64), ctypes.POINTER(_c_i64), _c_i32)
+_prefill_batch = _sig("tg_prefill_batch", _ci, ctypes.POINTER(TgModel), _c_p, _c_p,
+                      ctypes.POINTER(_c_i64), ctypes.POINTER(_c_i64), _c_i32, _c_i32, _c_p, _c_p,
+                      _c_p, _c_p, _c_sz, _c_p)
 _decode = _sig("tg_decode_step", _ci, ctypes.POINTER(TgModel), _c_p, _c_i64, _c_i32,
                ctypes.POINTER(TgKV), ctypes.POINTER(_c_i64), _c_p, _c_i64, _c_p, _c_i64, _c_p, _c_p,
                _c_sz, _c_p)
@@ -461,8 +466,38 @@ def tg_prefill_multi(model: Model, x, protect, ks: Sequence[int], gate_layer: in
     return outs, kept_idx, scores
 
 
+def tg_prefill_batch(model: Model, x, protect, lens: Sequence[int], ks: Sequence[int],
+                     gate_layer: int, out=None, kept_idx=None, scores=None, ws=None, stream=None):
+    """The gated prefill of len(lens) requests packed back to back in x
+    (request b: lens[b] rows, budget ks[b]). Returns (out [sum ks, d],
+    kept_idx [sum ks] (request-local indices), scores [sum lens] or None),
+    each request's rows after the previous ones'."""
+    d = x.shape[1]
+    nb = len(lens)
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + int(n))
+    if cu[-1] != x.shape[0]:
+        raise ValueError("sum of lens must equal x's rows")
+    cu_c = (_c_i64 * (nb + 1))(*cu)
+    ks_c = (_c_i64 * nb)(*[int(k) for k in ks])
+    tot_k = int(sum(ks))
+    if out is None:
+        out = torch.empty(tot_k, d, dtype=x.dtype, device=x.device)
+    if kept_idx is None:
+        kept_idx = torch.empty(tot_k, dtype=torch.int32, device=x.device)
+    need = _prefill_batch_ws(ctypes.byref(model.c), cu_c, ks_c, nb)
+    if need == 0:
+        raise ValueError("invalid batch sizes")
+    ws = _ws(need, x.device, ws)
+    _check(_prefill_batch(ctypes.byref(model.c), _ptr(x), _ptr(protect), cu_c, ks_c, nb,
+                          gate_layer, _ptr(out), _ptr(kept_idx), _ptr(scores), _ptr(ws),
+                          ws.numel(), _stream(stream, x.device)), "tg_prefill_batch")
+    return out, kept_idx, scores
+
+
 __all__ = [
-    "tg_score", "tg_linear", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_gated_attn_forward", "tg_gated_attn_backward", "tg_prefill", "tg_prefill_multi", "tg_decode_step",
+    "tg_score", "tg_linear", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_gated_attn_forward", "tg_gated_attn_backward", "tg_prefill", "tg_prefill_multi", "tg_prefill_batch", "tg_decode_step",
     "tg_workspace_size", "tg_status_string", "tg_device_error", "tg_version", "Model",
     "TokenGateError", "LIB_PATH", "tg_trace_start", "tg_trace_stop", "TG_OK", "TG_ERR_INVALID_ARG", "TG_ERR_UNSUPPORTED",
     "TG_ERR_BUDGET", "TG_ERR_WORKSPACE", "TG_ERR_CUDA", "TG_F32", "TG_BF16", "TG_OP_SCORE",

@@ -369,6 +369,29 @@ cudaError_t launch_rope_table(const int32_t* pos, int64_t T, int dh, float rope_
   return cudaGetLastError();
 }
 
+// Positions of packed requests (see launch_segment_positions): each thread
+// finds its request by a scan of the (at most 64) offsets.
+__global__ void segment_positions_kernel(SegRows s, int64_t total, int32_t* __restrict__ pos) {
+  pdl_trigger();
+  pdl_wait();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= total) return;
+  int32_t p = 0;
+  for (int b = 0; b < s.count; ++b) {
+    const int64_t i = t - s.off[b];
+    if (i >= 0 && i < s.len[b]) p = static_cast<int32_t>(i);
+  }
+  pos[t] = p;
+}
+
+cudaError_t launch_segment_positions(const SegRows& s, int64_t total, int32_t* pos,
+                                     cudaStream_t st) {
+  if (total <= 0) return cudaSuccess;
+  TG_CUDA_TRY(launch_pdl(segment_positions_kernel, dim3(static_cast<unsigned>((total + 255) / 256)),
+                         dim3(256), 0, st, s, total, pos));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_bias_aug(const float* lsig, int64_t T, void* kaug, cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
   TG_CUDA_TRY(launch_pdl(bias_aug_kernel, dim3(static_cast<unsigned>((T + 255) / 256)), dim3(256), 0, st, lsig, T, static_cast<uint4*>(kaug)));

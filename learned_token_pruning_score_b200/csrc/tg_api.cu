@@ -397,11 +397,42 @@ struct Dims {
   int d, hq, hkv, dh, inter, qkv;
 };
 
+// Attention of several packed requests, one launch per request over its own
+// rows (see SegRows: request b's rows start at segs.off[b], a multiple of
+// 128, so every slice of q, k, V^T and the bias rows stays 16-byte aligned).
+cudaError_t attn_segments(const AttnPlan& plan, const void* k_rot, const float* lsig,
+                          const void* kaug, const float* gain, const float* tau,
+                          const SegRows& segs, int hq, int hkv, int dh, void* out,
+                          cudaStream_t st) {
+  const size_t e = 2;
+  for (int b = 0; b < segs.count; ++b) {
+    const int64_t off = segs.off[b], rows = segs.len[b];
+    AttnArgs a{};
+    a.q = static_cast<const char*>(plan.q_rot) + size_t(off) * hq * dh * e;
+    a.k = static_cast<const char*>(k_rot) + size_t(off) * hkv * dh * e;
+    a.v = static_cast<const char*>(plan.vT) + size_t(off) * e;  // column offset in V^T rows
+    a.t_pad = plan.t_pad;
+    a.lsig = lsig ? lsig + off : nullptr;
+    a.kaug = kaug ? static_cast<const char*>(kaug) + size_t(off) * 32 : nullptr;
+    a.gain = gain;
+    a.tau = tau;
+    a.T = rows; a.hq = hq; a.hkv = hkv; a.dh = dh;
+    a.out = static_cast<char*>(out) + size_t(off) * hq * dh * e;
+    if (!attn_tc_supported(a)) return cudaErrorInvalidValue;
+    const double fl = 4.0 * dh * hq * double(rows) * double(rows + 1) / 2.0;
+    const double by = double(rows) * (2 * hq + 2 * hkv) * dh * e;
+    const cudaError_t err =
+        traced(TG_K_ATTENTION, rows, fl, by, st, [&] { return launch_attn_tc(a, st); });
+    if (err != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
 cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
                                const PrefillPlan& P, void* h, int64_t rows, const int32_t* pos,
                                const float2* cs, const float* lsig, const void* kaug,
                                const float* gain, const float* tau, const tg_kv* kv,
-                               cudaStream_t st) {
+                               cudaStream_t st, const SegRows* segs = nullptr) {
   const tg_dtype dt = m.dtype;
   const size_t e = elem_size(dt);
   cudaError_t err = rmsnorm(h, lw.attn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
@@ -415,8 +446,14 @@ cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims
     // fused: projection + qk-norm + RoPE + V^T in the GEMM epilogue
     err = gemm(gq, dt, st);
     if (err != cudaSuccess) return err;
-    err = attn_core(P.attn, k_dst, nullptr, 0, lsig, kaug, gain, tau, rows, D.hq, D.hkv, D.dh,
-                    dt, P.attn_o, st);
+    if (segs != nullptr)
+      err = attn_segments(P.attn, k_dst, lsig, kaug, gain, tau, *segs, D.hq, D.hkv, D.dh,
+                          P.attn_o, st);
+    else
+      err = attn_core(P.attn, k_dst, nullptr, 0, lsig, kaug, gain, tau, rows, D.hq, D.hkv, D.dh,
+                      dt, P.attn_o, st);
+  } else if (segs != nullptr) {
+    return cudaErrorInvalidValue;  // packed requests need the fused bf16 path
   } else {
     err = gemm(gemm_args(P.y, D.d, lw.wqkv, D.d, P.qkv, D.qkv, rows, D.qkv, D.d, EPI_STORE), dt,
                st);
@@ -865,6 +902,57 @@ tg_status prefill_above_gate(const tg_model& m, const Dims& D, const PrefillPlan
   return TG_OK;
 }
 
+// Workspace of a batch of packed requests: the prefill plan over the padded
+// row counts, plus the positions of the padded all-token rows.
+struct BatchPlan {
+  PrefillPlan P;
+  int32_t* pos_n = nullptr;
+  size_t bytes = 0;
+  BatchPlan(void* ws, const tg_model& m, int64_t n_pad, int64_t k_pad)
+      : P(ws, m, n_pad, k_pad) {
+    Arena a(ws);
+    a.used = P.bytes;
+    pos_n = static_cast<int32_t*>(a.carve(size_t(n_pad) * 4));
+    bytes = a.used;
+  }
+};
+
+constexpr int64_t kSegAlign = 128;
+
+// Validates a batch and lays it out: request b's rows at segs_n.off[b], its
+// kept rows at segs_k.off[b] (each padded to 128 rows).
+// (validate = false: sizes only, for the workspace query.)
+tg_status batch_layout(const tg_model* model, const int64_t* cu_n, const int64_t* ks,
+                       int32_t batch, int32_t gate_layer, bool validate, SegRows* segs_n,
+                       SegRows* segs_k, int64_t* n_pad, int64_t* k_pad) {
+  TG_CHECK(model && cu_n && ks, TG_ERR_INVALID_ARG);
+  TG_CHECK(batch >= 1 && batch <= TG_MAX_BATCH && batch <= kMaxSegs, TG_ERR_INVALID_ARG);
+  TG_CHECK(cu_n[0] == 0, TG_ERR_INVALID_ARG);
+  TG_CHECK(model->dtype == TG_BF16 || model->dtype == TG_F32, TG_ERR_UNSUPPORTED);
+  TG_CHECK(model->dtype == TG_BF16 && model->head_dim == 128, TG_ERR_UNSUPPORTED);
+  segs_n->count = segs_k->count = batch;
+  int64_t on = 0, ok = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t n = cu_n[b + 1] - cu_n[b];
+    TG_CHECK(n >= 1, TG_ERR_INVALID_ARG);
+    TG_CHECK(ks[b] >= 1 && ks[b] <= n, TG_ERR_BUDGET);
+    if (validate) {
+      const tg_status vs = validate_model(model, n, ks[b], gate_layer);
+      if (vs != TG_OK) return vs;
+    }
+    segs_n->off[b] = on;
+    segs_n->len[b] = n;
+    segs_k->off[b] = ok;
+    segs_k->len[b] = ks[b];
+    on += static_cast<int64_t>(align_up(static_cast<size_t>(n), kSegAlign));
+    ok += static_cast<int64_t>(align_up(static_cast<size_t>(ks[b]), kSegAlign));
+  }
+  TG_CHECK(on < (int64_t(1) << 31) - 4096, TG_ERR_INVALID_ARG);
+  *n_pad = on;
+  *k_pad = ok;
+  return TG_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -918,6 +1006,110 @@ tg_status tg_prefill_multi(const tg_model* model, const void* x, const uint8_t* 
     const tg_status sb = prefill_above_gate(m, D, P, protect, n, ks[b], gate_layer, sc, outs[b],
                                             kept_idx[b], nullptr, nullptr, st);
     if (sb != TG_OK) return sb;
+  }
+  return TG_OK;
+}
+
+size_t tg_prefill_batch_workspace_size(const tg_model* model, const int64_t* cu_n,
+                                       const int64_t* ks, int32_t batch) {
+  SegRows sn{}, sk{};
+  int64_t n_pad = 0, k_pad = 0;
+  if (batch_layout(model, cu_n, ks, batch, 0, false, &sn, &sk, &n_pad, &k_pad) != TG_OK)
+    return 0;
+  return BatchPlan(nullptr, *model, n_pad, k_pad).bytes;
+}
+
+tg_status tg_prefill_batch(const tg_model* model, const void* x, const uint8_t* protect,
+                           const int64_t* cu_n, const int64_t* ks, int32_t batch,
+                           int32_t gate_layer, void* out, int32_t* kept_idx, float* scores,
+                           void* ws, size_t ws_bytes, tg_stream stream) {
+  SegRows sn{}, sk{};
+  int64_t n_pad = 0, k_pad = 0;
+  const tg_status vs =
+      batch_layout(model, cu_n, ks, batch, gate_layer, true, &sn, &sk, &n_pad, &k_pad);
+  if (vs != TG_OK) return vs;
+  TG_CHECK(x && out && kept_idx, TG_ERR_INVALID_ARG);
+  TG_CHECK(aligned16(x) && aligned16(out), TG_ERR_INVALID_ARG);
+  const tg_model& m = *model;
+  BatchPlan B(nullptr, m, n_pad, k_pad);
+  TG_CHECK(ws != nullptr && ws_bytes >= B.bytes, TG_ERR_WORKSPACE);
+  B = BatchPlan(ws, m, n_pad, k_pad);
+  const PrefillPlan& P = B.P;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Dims D = model_dims(m);
+  const size_t e = elem_size(m.dtype);
+  const size_t row = size_t(D.d) * e;
+  char* h = static_cast<char*>(P.h);
+  char* hk = static_cast<char*>(P.hk);
+  // packed rows in, padding rows zero
+  for (int b = 0; b < batch; ++b) {
+    const int64_t n = sn.len[b], pad = static_cast<int64_t>(align_up(size_t(n), kSegAlign)) - n;
+    TG_TRY(copy_rows(h + sn.off[b] * row, static_cast<const char*>(x) + cu_n[b] * row, n * row, n,
+                     st));
+    if (pad > 0) TG_TRY(cudaMemsetAsync(h + (sn.off[b] + n) * row, 0, pad * row, st));
+  }
+  TG_TRY(launch_segment_positions(sn, n_pad, B.pos_n, st));
+  const double cs_bytes = 8.0 * (D.dh / 2);
+  TG_TRY(traced(TG_K_ROPE_TABLE, n_pad, 0.0, cs_bytes * n_pad, st, [&] {
+    return launch_rope_table(B.pos_n, n_pad, D.dh, m.rope_base, P.cs_n, st);
+  }));
+  // below the gate: projections over every request's rows, attention per request
+  for (int l = 0; l < gate_layer; ++l) {
+    LayerTag tag(l);
+    TG_TRY(attention_sublayer(m, m.layers[l], D, P, P.h, n_pad, nullptr, P.cs_n, nullptr, nullptr,
+                              nullptr, nullptr, nullptr, st, &sn));
+    TG_TRY(ffn_sublayer(m, m.layers[l], D, P, P.h, n_pad, st));
+  }
+  if (gate_layer >= 0) {
+    LayerTag tag(gate_layer);
+    TG_TRY(attention_sublayer(m, m.layers[gate_layer], D, P, P.h, n_pad, nullptr, P.cs_n, nullptr,
+                              nullptr, nullptr, nullptr, nullptr, st, &sn));
+  }
+  float* sc = P.scores;
+  TG_TRY(run_score(P.h, n_pad, D.d, m.d_score, m.score_norm, m.norm_eps, m.score_w1, m.score_b1,
+                   m.score_w2, m.score_b2, m.dtype, sc, P.y, P.hpre, st));
+  // per request: select, compact into its padded block of kept rows
+  TG_TRY(cudaMemsetAsync(P.pos_k, 0, size_t(k_pad) * 4, st));
+  int64_t ck = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t n = sn.len[b], k = sk.len[b];
+    if (scores) TG_TRY(cudaMemcpyAsync(scores + cu_n[b], sc + sn.off[b], size_t(n) * 4,
+                                       cudaMemcpyDeviceToDevice, st));
+    TG_TRY(select_topk(sc + sn.off[b], protect ? protect + cu_n[b] : nullptr, n, k, kept_idx + ck,
+                       P.sel_ws, st));
+    TG_TRY(compact(h + sn.off[b] * row, nullptr, sc + sn.off[b], kept_idx + ck, n, k,
+                   static_cast<int>(row), hk + sk.off[b] * row, P.pos_k + sk.off[b],
+                   P.s_k + sk.off[b], P.lsig_k + sk.off[b], st));
+    const int64_t pad = static_cast<int64_t>(align_up(size_t(k), kSegAlign)) - k;
+    if (pad > 0) TG_TRY(cudaMemsetAsync(hk + (sk.off[b] + k) * row, 0, pad * row, st));
+    ck += k;
+  }
+  TG_TRY(traced(TG_K_ROPE_TABLE, k_pad, 0.0, cs_bytes * k_pad + 4.0 * k_pad, st, [&] {
+    return launch_rope_table(P.pos_k, k_pad, D.dh, m.rope_base, P.cs_k, st);
+  }));
+  TG_TRY(traced(TG_K_ROPE_TABLE, k_pad, 0.0, 36.0 * k_pad, st,
+                [&] { return launch_bias_aug(P.lsig_k, k_pad, P.kaug_k, st); }));
+  // the gate layer's FFN and the layers above over every request's kept rows
+  if (gate_layer >= 0) {
+    LayerTag tag(gate_layer);
+    TG_TRY(ffn_sublayer(m, m.layers[gate_layer], D, P, P.hk, k_pad, st));
+  }
+  for (int l = gate_layer + 1; l < m.n_layers; ++l) {
+    LayerTag tag(l);
+    const tg_layer& L = m.layers[l];
+    TG_TRY(attention_sublayer(m, L, D, P, P.hk, k_pad, P.pos_k, P.cs_k, P.lsig_k, P.kaug_k, L.gain,
+                              L.tau, nullptr, st, &sk));
+    TG_TRY(ffn_sublayer(m, L, D, P, P.hk, k_pad, st));
+  }
+  ck = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t k = sk.len[b];
+    char* ob = static_cast<char*>(out) + ck * row;
+    if (m.final_norm)
+      TG_TRY(rmsnorm(hk + sk.off[b] * row, m.final_norm, m.norm_eps, k, D.d, m.dtype, ob, st));
+    else
+      TG_TRY(copy_rows(ob, hk + sk.off[b] * row, k * row, k, st));
+    ck += k;
   }
   return TG_OK;
 }

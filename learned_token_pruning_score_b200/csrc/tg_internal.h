@@ -103,6 +103,18 @@ cudaError_t launch_rope_prep(const RopePrepArgs& a, cudaStream_t st);
 cudaError_t launch_rope_table(const int32_t* pos, int64_t T, int dh, float rope_base, float2* cs,
                               cudaStream_t st);
 
+// Rows of up to kMaxSegs requests packed back to back, each starting at
+// off[b] (a multiple of 128) and len[b] rows long: pos[off[b] + i] = i for
+// i < len[b], 0 in the padding after each request, for `total` rows.
+constexpr int kMaxSegs = 64;
+struct SegRows {
+  int count;
+  int64_t off[kMaxSegs];
+  int64_t len[kMaxSegs];
+};
+cudaError_t launch_segment_positions(const SegRows& s, int64_t total, int32_t* pos,
+                                     cudaStream_t st);
+
 // Gate-bias rows for the attention's extra K-step: kaug[t] = (b_hi, b_lo,
 // b_hi, b_lo, 0 x 12) in bf16 with b = lsig[t], b_hi = bf16(b),
 // b_lo = bf16(b - b_hi).

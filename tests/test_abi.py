@@ -251,3 +251,34 @@ def test_decode_validation():
     assert _decode(ctypes.byref(m3), kv, lens) == tg.TG_ERR_UNSUPPORTED
     m4, keep4 = _bogus_model(dtype=tg.TG_F32)
     assert _decode(ctypes.byref(m4), kv, lens) == tg.TG_ERR_UNSUPPORTED
+
+
+def test_prefill_batch_validation():
+    m, keep = _bogus_model()
+    big = 1 << 40
+
+    def call(cu, ks, model=None, ws_bytes=big):
+        nb = len(ks)
+        cu_c = (ctypes.c_int64 * len(cu))(*cu)
+        ks_c = (ctypes.c_int64 * max(nb, 1))(*(ks or [0]))
+        mm = model if model is not None else m
+        return tg._prefill_batch(ctypes.byref(mm), BOGUS, None, cu_c, ks_c, nb, 1, BOGUS, BOGUS,
+                                 None, BOGUS, ws_bytes, None)
+
+    assert call([0], []) == tg.TG_ERR_INVALID_ARG  # empty batch
+    assert call([1, 300], [10]) == tg.TG_ERR_INVALID_ARG  # cu_n[0] != 0
+    assert call([0, 300, 300], [10, 10]) == tg.TG_ERR_INVALID_ARG  # an empty request
+    assert call([0, 300, 400], [10, 101]) == tg.TG_ERR_BUDGET  # k > n
+    assert call([0, 300, 400], [10, 0]) == tg.TG_ERR_BUDGET
+    m32, keep32 = _bogus_model(dtype=tg.TG_F32)
+    assert call([0, 300], [10], model=m32) == tg.TG_ERR_UNSUPPORTED
+    cu = (ctypes.c_int64 * 3)(0, 300, 429)
+    ks = (ctypes.c_int64 * 2)(100, 129)
+    need = tg._prefill_batch_ws(ctypes.byref(m), cu, ks, 2)
+    # the padded layout: 384 + 256 all-token rows, 128 + 256 kept rows
+    p = dict(d_model=2048, n_heads_q=16, n_heads_kv=8, head_dim=128, d_score=256, d_ffn=6144,
+             n_layers=2, gate_layer=1, dtype=tg.TG_BF16)
+    assert need >= tg.tg_workspace_size(tg.TG_OP_PREFILL, n=640, k=384, **p)
+    assert call([0, 300, 429], [100, 129], ws_bytes=need - 1) == tg.TG_ERR_WORKSPACE
+    bad = (ctypes.c_int64 * 2)(100, 300)
+    assert tg._prefill_batch_ws(ctypes.byref(m), cu, bad, 2) == 0
