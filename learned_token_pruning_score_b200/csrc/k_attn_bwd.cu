@@ -21,9 +21,9 @@
 // their gradients are rotated back with the transposed rotation.
 //
 // Kernels, in stream order:
-//   bwd_prep   q and k rotated (RoPE at the original positions), Q^T, K^T,
-//              dO^T as [head, dh, t_pad] (the K-major B operands of the
-//              products that contract over rows), the RoPE table, lse in log2 units,
+//   bwd_prep   q and k rotated (RoPE at the original positions), q and dO
+//              transposed to [head, dh, t_pad] (the K-major B operands of
+//              dK and dV), the RoPE table, lse in log2 units,
 //              D (from the forward's fp32 output when given: the bf16 output
 //              carries a rounding of 2^-9 that D would pass on to every
 //              dl_ij of the row), and the zero-padded bias row logsigmoid(s).
@@ -33,15 +33,20 @@
 //                one thread per key row forms P^T and dS^T (dS^T scaled by
 //                1 / (sqrt(dh) tau_h)) and writes them back as packed bf16
 //                over S^T and dP^T; dV += P^T dO and dK += dS^T Q with A read
-//                from TMEM. C_hj is a thread-local sum. (Keeping K and V in
-//                TMEM to double-buffer S^T and dP^T leaves room only for
-//                32-query products, whose MMA instructions are too short to
-//                keep the tensor pipe fed: measured slower.)
+//                from TMEM, in two 64-query halves so that the first half
+//                overlaps the row math of the second. C_hj is a
+//                thread-local sum. (Reading Q and dO MN-major instead of
+//                their transposed copies halves this kernel's operand
+//                traffic but measured 13-27% slower; keeping K and V in TMEM
+//                to double-buffer S^T and dP^T leaves room only for 32-query
+//                products, also slower.)
 //   bwd_dq     one CTA per (128-query tile, query head); Q and dO in TMEM.
-//              Keys up to the diagonal stream through a 3-stage ring (64 per
+//              Keys up to the diagonal stream through a 4-stage ring (64 per
 //              stage): S = Q K^T and dP = dO V^T into one of two TMEM
-//              buffers, dS written back over S, dQ += dS K. Then dq (scaled,
-//              rotated back) and per-warp partial sums of q_i . dq_i.
+//              buffers, dS written back over S, dQ += dS K with the same K
+//              tile read MN-major (dh contiguous; no transposed copy). Then
+//              dq (scaled, rotated back) and per-warp partial sums of
+//              q_i . dq_i.
 //   bwd_final  ds, dgain, dtau from C and the partial sums, in a fixed
 //              order (deterministic: no atomics anywhere).
 // Roles in both tensor-core kernels (256 threads): warp 0 TMA producer,
@@ -122,6 +127,27 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&x)[128]) {
     x[64 + i] = __uint_as_float(r2[i]);
     x[96 + i] = __uint_as_float(r3[i]);
   }
+}
+
+// Instruction descriptor (bf16 in, fp32 accumulate, M x N) with B read
+// MN-major (bit 16).
+constexpr uint32_t idesc_bf16_f32_bmn(int m, int n) { return idesc_bf16_f32(m, n) | (1u << 16); }
+
+// Shared-memory descriptor of an MN-major operand in the 128-byte-swizzled
+// layout: each 128-byte row holds 64 consecutive MN elements of one K index,
+// 8-row groups (8 K indices, one swizzle atom) are 1024 bytes apart (stride
+// byte offset), and 64-element MN blocks are `lbo` bytes apart (leading byte
+// offset). The row-major tiles TMA writes for the K-major products (rows =
+// tokens, 128 bytes of dh each) are exactly this layout with tokens as K and
+// dh as MN, so one copy serves both products.
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t addr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);          // start address
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;     // leading byte offset: MN blocks
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;               // stride byte offset: 8-row groups
+  d |= static_cast<uint64_t>(1u) << 46;                       // descriptor version (sm_100)
+  d |= static_cast<uint64_t>(2u) << 61;                       // layout: 128-byte swizzle
+  return d;
 }
 
 // Copies this thread's row r of a [128 x 128] bf16 tile (two 128-byte-
@@ -371,7 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ============================================================================
 // dQ: one CTA per (query tile it, query head h), 128 query rows.
 // Q and dO sit in TMEM as the A operands; the key side streams through a
-// 3-stage ring of 64-key stages, with S and dP double-buffered in TMEM.
+// 4-stage ring of 64-key stages, with S and dP double-buffered in TMEM. The
+// K tile serves both as the K-major B operand of S and as the MN-major B
+// operand of dQ.
 // TMEM columns: Q [0,64), dO [64,128) (packed bf16), dQ [128,256), buffer b:
 // S [256+128b, +64), dP [320+128b, +64); dS (packed) over the first 32
 // columns of S.
@@ -380,14 +408,13 @@ constexpr int kHalf64 = 64 * 128;
 constexpr int kOffQ = 0;
 constexpr int kOffDO = kOffQ + kTile;
 constexpr int kOffStage = kOffDO + kTile;
-// stage: K [64 x 128], V [64 x 128] (two dh halves each), K^T [128 dh x 64], bias[64]
+// stage: K [64 x 128], V [64 x 128] (two dh halves each), bias[64]
 constexpr int kStK = 0;
 constexpr int kStV = kStK + 2 * kHalf64;
-constexpr int kStKT = kStV + 2 * kHalf64;
-constexpr int kStBias = kStKT + 128 * 128;
+constexpr int kStBias = kStV + 2 * kHalf64;
 constexpr int kStageBytes = kStBias + 1024;
-constexpr uint32_t kStageTx = 3 * 16384 + 256;
-constexpr int kStages = 3;
+constexpr uint32_t kStageTx = 2 * 16384 + 256;
+constexpr int kStages = 4;
 constexpr int kOffBar = kOffStage + kStages * kStageBytes;
 constexpr size_t kSmem = 1024 + kOffBar + 256;
 constexpr uint32_t kTmQ = 0, kTmDO = 64, kTmDQ = 128, kTmBuf = 256;
@@ -396,7 +423,7 @@ constexpr uint32_t kTmQ = 0, kTmDO = 64, kTmDQ = 128, kTmBuf = 256;
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                const __grid_constant__ CUtensorMap tmKT, BwdParams p) {
+                BwdParams p) {
   using namespace dqk;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
@@ -404,12 +431,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* q_full = bars + 0;
   uint64_t* q_ready = bars + 1;     // Q and dO copied into TMEM (128 arrivals)
-  uint64_t* st_full = bars + 2;     // [3]
-  uint64_t* st_empty = bars + 5;    // [3]
-  uint64_t* s_full = bars + 8;      // [2]
-  uint64_t* p_full = bars + 10;     // [2] (128 arrivals)
-  uint64_t* acc_full = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* st_full = bars + 2;     // [kStages]
+  uint64_t* st_empty = bars + 2 + kStages;
+  uint64_t* s_full = bars + 2 + 2 * kStages;   // [2]
+  uint64_t* p_full = bars + 4 + 2 * kStages;   // [2] (128 arrivals)
+  uint64_t* acc_full = bars + 6 + 2 * kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7 + 2 * kStages);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int it = p.n_tiles - 1 - static_cast<int>(blockIdx.x) / p.hq;  // longest first
@@ -436,7 +463,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmDO);
-    tma_prefetch_desc(&tmKT);
   }
   if (warp == 2) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -462,13 +488,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(&tmK, &st_full[st], sb + kStK + kHalf64, 64, g, j0);
       tma_load_3d(&tmV, &st_full[st], sb + kStV, 0, g, j0);
       tma_load_3d(&tmV, &st_full[st], sb + kStV + kHalf64, 64, g, j0);
-      tma_load_3d(&tmKT, &st_full[st], sb + kStKT, j0, 0, g);
       bulk_load(sb + kStBias, p.bias + j0, 256, &st_full[st]);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_n64 = idesc_bf16_f32(128, 64);
-    constexpr uint32_t idesc_n128 = idesc_bf16_f32(128, 128);
+    constexpr uint32_t idesc_n128_mn = idesc_bf16_f32_bmn(128, 128);
     auto sp_products = [&](int m) {  // S_b = Q K_m^T, dP_b = dO V_m^T
       const int b = m & 1;
       const uint8_t* sb = smem + kOffStage + (m % kStages) * kStageBytes;
@@ -488,14 +513,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       umma_commit(&s_full[b]);
     };
-    auto dq_product = [&](int m) {  // dQ += dS_b K_m
+    auto dq_product = [&](int m) {  // dQ += dS_b K_m, K read MN-major (dh contiguous)
       const int b = m & 1, st = m % kStages;
-      const uint32_t kt_addr = smem_addr(smem + kOffStage + st * kStageBytes + kStKT);
+      const uint32_t k_addr = smem_addr(smem + kOffStage + st * kStageBytes + kStK);
       const uint32_t a = tmem + kTmBuf + 128u * b;
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        umma_f16_ts(tmem + kTmDQ, a + kk * 8, sdesc_kmajor_sw128(kt_addr + kk * 32), idesc_n128,
-                    (m > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < 4; ++kk) {  // 16 keys per K-step: 16 rows of 128 bytes
+        umma_f16_ts(tmem + kTmDQ, a + kk * 8, sdesc_mnmajor_sw128(k_addr + kk * 2048, kHalf64),
+                    idesc_n128_mn, (m > 0 || kk > 0) ? 1u : 0u);
       }
       umma_commit(&st_empty[st]);
     };
@@ -703,8 +728,9 @@ __global__ void __launch_bounds__(256) attn_bwd_prep(PrepArgs a) {
     a.bias[t] = (a.s && t < a.T) ? logsigmoid_f(__ldg(a.s + t)) : 0.0f;
   }
   __syncthreads();
-  __nv_bfloat16* dst = a.dst[which] + static_cast<int64_t>(h) * kDh * a.t_pad;
-  for (int e = threadIdx.x; e < kDh * 32; e += 256) {
+  __nv_bfloat16* dst = a.dst[which] ? a.dst[which] + static_cast<int64_t>(h) * kDh * a.t_pad
+                                    : nullptr;
+  for (int e = threadIdx.x; dst != nullptr && e < kDh * 32; e += 256) {
     const int d = e >> 5, l = e & 31;  // output row d, rows 2l and 2l + 1 of the tile
     const int w = d >> 1, sh = (d & 1) * 16;
     const uint32_t w0 = tile[(2 * l) * 64 + (w ^ l)];
@@ -822,7 +848,7 @@ cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t st, int stage) {
     pa.rot[0] = static_cast<__nv_bfloat16*>(a.q_rot);
     pa.rot[1] = static_cast<__nv_bfloat16*>(a.k_rot);
     pa.dst[0] = static_cast<__nv_bfloat16*>(a.qT);
-    pa.dst[1] = static_cast<__nv_bfloat16*>(a.kT);
+    pa.dst[1] = nullptr;  // K is read MN-major by dQ: no transposed copy
     pa.dst[2] = static_cast<__nv_bfloat16*>(a.doT);
     pa.pos = a.pos;
     pa.rope_base = a.rope_base;
@@ -901,16 +927,14 @@ cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t st, int stage) {
     return launch_pdl(attn_bwd_dkdv, dim3(grid), dim3(kThreads), dkdv::kSmem, st, tq, tk, tv, tdo,
                       tqT, tdoT, p);
   }
-  CUtensorMap tq, tk, tv, tdo, tkT;
+  CUtensorMap tq, tk, tv, tdo;
   if (!rows_map(&tq, a.q_rot, a.hq, kBlk) || !rows_map(&tdo, a.dout, a.hq, kBlk) ||
-      !rows_map(&tk, a.k_rot, a.hkv, 64) || !rows_map(&tv, a.v, a.hkv, 64) ||
-      !cols_map(&tkT, a.kT, a.hkv))
+      !rows_map(&tk, a.k_rot, a.hkv, 64) || !rows_map(&tv, a.v, a.hkv, 64))
     return cudaErrorInvalidValue;
   cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(attn_bwd_dq), int(dqk::kSmem));
   if (err != cudaSuccess) return err;
   const unsigned grid = static_cast<unsigned>(n_tiles) * static_cast<unsigned>(a.hq);
-  return launch_pdl(attn_bwd_dq, dim3(grid), dim3(kThreads), dqk::kSmem, st, tq, tk, tv, tdo, tkT,
-                    p);
+  return launch_pdl(attn_bwd_dq, dim3(grid), dim3(kThreads), dqk::kSmem, st, tq, tk, tv, tdo, p);
 }
 
 }  // namespace tg

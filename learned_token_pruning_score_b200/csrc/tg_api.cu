@@ -164,7 +164,6 @@ struct AttnBwdPlan {
   void* k_rot = nullptr;   // [n, hkv, dh]
   float2* cs = nullptr;    // [dh/2, n] RoPE table
   void* qT = nullptr;      // [hq, dh, t_pad]
-  void* kT = nullptr;      // [hkv, dh, t_pad]
   void* doT = nullptr;     // [hq, dh, t_pad]
   float* lse2 = nullptr;   // [hq, t_pad]
   float* dd = nullptr;     // [hq, t_pad]
@@ -181,7 +180,6 @@ struct AttnBwdPlan {
     k_rot = a.carve(size_t(n) * hkv * dh * 2);
     cs = static_cast<float2*>(a.carve(size_t(dh / 2) * n * 8));
     qT = a.carve(size_t(hq) * dh * tp * 2);
-    kT = a.carve(size_t(hkv) * dh * tp * 2);
     doT = a.carve(size_t(hq) * dh * tp * 2);
     lse2 = static_cast<float*>(a.carve(size_t(hq) * tp * 4));
     dd = static_cast<float*>(a.carve(size_t(hq) * tp * 4));
@@ -794,14 +792,14 @@ tg_status tg_gated_attn_backward(const void* q, const void* kk, const void* v, c
   a.lse = lse; a.s = s; a.gain = gain; a.tau = tau;
   a.T = k; a.t_pad = plan.t_pad; a.hq = hq; a.hkv = hkv;
   a.q_rot = plan.q_rot; a.k_rot = plan.k_rot; a.cs = plan.cs;
-  a.qT = plan.qT; a.kT = plan.kT; a.doT = plan.doT;
+  a.qT = plan.qT; a.doT = plan.doT;
   a.lse2 = plan.lse2; a.dd = plan.dd; a.colsum = plan.colsum; a.qdq = plan.qdq;
   a.bias = plan.bias;
   a.dq = dq; a.dk = dk; a.dv = dv; a.ds = ds; a.dgain = dgain; a.dtau = dtau;
   // one [T x T x dh] causal product of all query heads (half of the forward's FLOPs)
   const double prod = 2.0 * dh * hq * rows * (rows + 1) / 2.0;
-  // reads q, k, dO and o; writes q, k rotated and q, k, dO transposed
-  const double prep_bytes = rows * dh * 2.0 * (3.0 * (hq + hkv) + 2.0 * hq) +
+  // reads q, k, dO and o; writes q, k rotated and q, dO transposed
+  const double prep_bytes = rows * dh * 2.0 * (2.0 * (hq + hkv) + 3.0 * hq) +
                             rows * hq * dh * (out_f32 ? 4.0 : 2.0);
   TG_TRY(traced(TG_K_ATTN_BWD_PREP, k, 0.0, prep_bytes, st,
                 [&] { return launch_attn_bwd(a, st, 0); }));

@@ -178,7 +178,7 @@ struct AttnBwdArgs {
   int64_t T, t_pad; int hq, hkv;
   void* q_rot; void* k_rot;              // workspace [T, hq|hkv, dh], rotated as in the forward
   float2* cs;                            // workspace [dh/2, T] RoPE (cos, sin) table
-  void* qT; void* kT; void* doT;         // workspace [H, dh, t_pad]
+  void* qT; void* doT;                   // workspace [hq, dh, t_pad] (transposed q, dO)
   float* lse2; float* dd; float* colsum; // workspace [hq, t_pad]
   float* qdq;                            // workspace [hq, n_tiles, 4]
   float* bias;                           // workspace [t_pad] logsigmoid(s), zero-padded
@@ -186,8 +186,8 @@ struct AttnBwdArgs {
   float* ds; float* dgain; float* dtau;  // outputs, each optional
 };
 size_t attn_bwd_t_pad(int64_t T);
-// stage 0: prep (RoPE, transposes, table, lse2, D, bias); 1: dK/dV/C; 2: dQ;
-// 3: ds/dgain/dtau.
+// stage 0: prep (RoPE, transposes of q and dO, table, lse2, D, bias); 1: dK/dV/C;
+// 2: dQ; 3: ds/dgain/dtau.
 cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t st, int stage);
 
 // ---- decode (k_decode.cu): one generated token, batch 1, bf16, head_dim 128.

@@ -119,8 +119,8 @@ def test_attention_forward_lse_and_backward_validation():
     bwd = tg._attn_bwd
     need = tg.tg_workspace_size(tg.TG_OP_GATED_ATTN_BWD, k=128, n_heads_q=4, n_heads_kv=2,
                                 head_dim=128, dtype=tg.TG_BF16)
-    # rotated q and k, Q^T, K^T, dO^T, the RoPE table and the per-row vectors
-    assert need >= 128 * 128 * 2 * (4 + 2 + 4 + 2 + 4) + 64 * 128 * 8
+    # rotated q and k, the RoPE table and the per-row vectors
+    assert need >= 128 * 128 * 2 * (4 + 2) + 64 * 128 * 8 + 3 * 4 * 128 * 4
     outs = [BOGUS, BOGUS, BOGUS, BOGUS, BOGUS, BOGUS]  # dq, dk, dv, ds, dgain, dtau
 
     def call(dt=tg.TG_BF16, dh=128, hq=4, hkv=2, s=BOGUS, out=BOGUS, o=outs, ws=BOGUS,
