@@ -49,8 +49,9 @@
 //              q_i . dq_i.
 //   bwd_final  ds, dgain, dtau from C and the partial sums, in a fixed
 //              order (deterministic: no atomics anywhere).
-// Roles in both tensor-core kernels (256 threads): warp 0 TMA producer,
-// warp 1 MMA issuer, warp 2 TMEM allocation, warps 4-7 one thread per row.
+// Roles in both tensor-core kernels (384 threads): warp 0 TMA producer,
+// warp 1 MMA issuer, warp 2 TMEM allocation, warps 4-7 and 8-11 two
+// row-math warpgroups (one thread per row each, on half of the columns).
 // Every wait is bounded (an expired wait sets the device error word and the
 // kernel drains and returns).
 #include "tg_device.cuh"
@@ -62,6 +63,7 @@ namespace {
 constexpr int kBlk = 128;        // rows per tile (queries or keys)
 constexpr int kDh = 128;
 constexpr int kThreads = 256;
+constexpr int kThreads2 = 384;   // dK/dV and dQ: roles + two row-math warpgroups
 constexpr int kSub = 128 * 128;  // bytes of one [128 rows x 64 bf16] 128-byte-swizzled sub-tile
 constexpr int kTile = 2 * kSub;  // [128 x 128] bf16 tile
 constexpr float kLog2e = 1.4426950408889634f;
@@ -78,8 +80,8 @@ struct BwdParams {
   __nv_bfloat16* dq;     // [T, hq, dh]
   __nv_bfloat16* dk;     // [T, hkv, dh]
   __nv_bfloat16* dv;     // [T, hkv, dh]
-  float* colsum;         // [hq, t_pad] C_hj, or null (no scores)
-  float* qdq;            // [hq, n_tiles, 4] per-warp partial sums of q_i . dq_i
+  float* colsum;         // [2, hq, t_pad] C_hj over query halves 0-63 / 64-127, or null
+  float* qdq;            // [hq, n_tiles, 8] per-warp partial sums of q_i . dq_i
   unsigned int* err;
 };
 
@@ -106,6 +108,48 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const float (
     u.z = pack_bf16x2(x[8 * v + 4], x[8 * v + 5]);
     u.w = pack_bf16x2(x[8 * v + 6], x[8 * v + 7]);
     d[v] = u;
+  }
+}
+
+// Stores 32 fp32 values as bf16 (four 16-byte vectors).
+__device__ __forceinline__ void store32_bf16(__nv_bfloat16* dst, const float* x) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    uint4 u;
+    u.x = pack_bf16x2(x[8 * v + 0], x[8 * v + 1]);
+    u.y = pack_bf16x2(x[8 * v + 2], x[8 * v + 3]);
+    u.z = pack_bf16x2(x[8 * v + 4], x[8 * v + 5]);
+    u.w = pack_bf16x2(x[8 * v + 6], x[8 * v + 7]);
+    d[v] = u;
+  }
+}
+
+// Two TMEM loads of 32 columns (one wait).
+__device__ __forceinline__ void tmem_ld2x32(uint32_t ta, uint32_t tb, float (&a)[32],
+                                            float (&b)[32]) {
+  uint32_t ra[32], rb[32];
+  tmem_ld32(ta, ra);
+  tmem_ld32(tb, rb);
+  tmem_wait_ld_dep(rb);
+  tmem_ld_fence(ra);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    a[i] = __uint_as_float(ra[i]);
+    b[i] = __uint_as_float(rb[i]);
+  }
+}
+
+// Rotates the pairs (lo[i], hi[i]) = (x[i0 + i], x[i0 + 64 + i]) of a
+// rotated-frame gradient row back through RoPE (frequencies i0 .. i0+31).
+__device__ __forceinline__ void rope_back32(float (&lo)[32], float (&hi)[32], const float2* cs,
+                                            int64_t T, int64_t row, int i0) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float2 c = __ldg(cs + static_cast<int64_t>(i0 + i) * T + row);
+    const float a = lo[i], b = hi[i];
+    lo[i] = a * c.x + b * c.y;
+    hi[i] = b * c.x - a * c.y;
   }
 }
 
@@ -171,8 +215,9 @@ __device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int r, uin
 
 // ============================================================================
 // dK, dV and C: one CTA per (key tile jt, KV head g), 128 key rows.
-// TMEM columns: S^T [0,128) (P^T packed over [0,64)), dP^T [128,256) (dS^T
-// packed over [128,192)), dV [256,384), dK [384,512). All 512 columns are in
+// TMEM columns: S^T [0,128), dP^T [128,256), dV [256,384), dK [384,512).
+// P^T and dS^T are packed over the first 32 columns of each 64-query half of
+// S^T and dP^T (the half's own warpgroup has read them). All 512 columns are in
 // use, so the products of one query tile wait for the rows of the previous
 // one; the query side is loaded in two halves (stage a: Q, dO for S^T and
 // dP^T; stage b: Q^T, dO^T, lse2, D for the rows and dV, dK) so that the
@@ -201,7 +246,7 @@ __device__ __forceinline__ void mma_ss_128(uint32_t d, uint32_t a_addr, uint32_t
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads2, 1)
     attn_bwd_dkdv(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmQT,
@@ -290,8 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t dot_addr = smem_addr(smem + kOffDOT) + half * kSub;
       const uint32_t qt_addr = smem_addr(smem + kOffQT) + half * kSub;
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint32_t col = static_cast<uint32_t>(half * 32 + kk * 8);
+      for (int kk = 0; kk < 4; ++kk) {  // P^T / dS^T of queries 64 half .. + 63: 32 packed columns
+        const uint32_t col = static_cast<uint32_t>(half * 64 + kk * 8);
         umma_f16_ts(tmem + 256, tmem + col, sdesc_kmajor_sw128(dot_addr + kk * 32), idesc,
                     (accumulate || kk > 0) ? 1u : 0u);
         umma_f16_ts(tmem + 384, tmem + 128 + col, sdesc_kmajor_sw128(qt_addr + kk * 32), idesc,
@@ -317,8 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) umma_commit(acc_full);
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ one thread per key row
-    const int r = threadIdx.x - 128;
+    // ------------------------------------------------------------ row math
+    // Warpgroup wg (warps 4-7: 0, warps 8-11: 1) forms queries 64 wg .. 64 wg
+    // + 63 of every key row (one thread per key row, TMEM lane = row).
+    const int wg = (warp - 4) >> 2;
+    const int r = (threadIdx.x - 128) & 127;
     const int64_t j = static_cast<int64_t>(j0) + r;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float* vec_l = reinterpret_cast<const float*>(smem + kOffVec);
@@ -340,8 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const bool diag = it == jt;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * wg + cc;
         uint32_t rs[32], rp[32];
         tmem_ld32(tmem + lane_off + static_cast<uint32_t>(32 * c), rs);
         tmem_ld32(tmem + lane_off + 128u + static_cast<uint32_t>(32 * c), rp);
@@ -363,28 +412,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[t >> 1] = pack_bf16x2(p0, p1);
           dk16[t >> 1] = pack_bf16x2(d0 * inv_st, d1 * inv_st);
         }
-        tmem_st16(tmem + lane_off + static_cast<uint32_t>(16 * c), pk);
-        tmem_st16(tmem + lane_off + 128u + static_cast<uint32_t>(16 * c), dk16);
-        if (c & 1) {  // queries 0-63 (c = 1) or 64-127 (c = 3) done
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&p_half[c >> 1]);
-        }
+        // packed into this warpgroup's own (already read) columns: queries
+        // 64 wg + 32 cc .. + 31 at columns 64 wg + 16 cc (P^T) and 128 + the same (dS^T)
+        const uint32_t pc = static_cast<uint32_t>(64 * wg + 16 * cc);
+        tmem_st16(tmem + lane_off + pc, pk);
+        tmem_st16(tmem + lane_off + 128u + pc, dk16);
       }
-      if (n % n_q == n_q - 1) {  // last query tile of head h: C_hj is complete
-        if (p.colsum && j < p.T) p.colsum[static_cast<int64_t>(h) * p.t_pad + j] = csum;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_half[wg]);
+      if (n % n_q == n_q - 1) {  // last query tile of head h: this half's C_hj is complete
+        if (p.colsum && j < p.T)
+          p.colsum[(static_cast<int64_t>(wg) * p.hq + h) * p.t_pad + j] = csum;
         csum = 0.f;
       }
     }
     if (ok && mbar_wait_warp(acc_full, 0, p.err)) {
       tc_fence_after();
-      float x[128];
-      tmem_ld128(tmem + lane_off + 256u, x);  // dV
-      if (j < p.T) store_row_bf16(p.dv + (j * p.hkv + g) * kDh, x);
-      tmem_ld128(tmem + lane_off + 384u, x);  // dK (rotated frame)
-      if (j < p.T) {
-        rope_back(x, p.cs, p.T, j);
-        store_row_bf16(p.dk + (j * p.hkv + g) * kDh, x);
+      if (wg == 0) {  // dV
+#pragma unroll 1
+        for (int c = 0; c < 4; c += 2) {
+          float a[32], b[32];
+          tmem_ld2x32(tmem + lane_off + 256u + 32u * c, tmem + lane_off + 288u + 32u * c, a, b);
+          if (j < p.T) {
+            store32_bf16(p.dv + (j * p.hkv + g) * kDh + 32 * c, a);
+            store32_bf16(p.dv + (j * p.hkv + g) * kDh + 32 * c + 32, b);
+          }
+        }
+      } else {  // dK, rotated back pair by pair
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          float lo[32], hi[32];
+          tmem_ld2x32(tmem + lane_off + 384u + 32u * c, tmem + lane_off + 448u + 32u * c, lo, hi);
+          if (j < p.T) {
+            rope_back32(lo, hi, p.cs, p.T, j, 32 * c);
+            store32_bf16(p.dk + (j * p.hkv + g) * kDh + 32 * c, lo);
+            store32_bf16(p.dk + (j * p.hkv + g) * kDh + 64 + 32 * c, hi);
+          }
+        }
       }
     }
   }
@@ -401,8 +466,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // K tile serves both as the K-major B operand of S and as the MN-major B
 // operand of dQ.
 // TMEM columns: Q [0,64), dO [64,128) (packed bf16), dQ [128,256), buffer b:
-// S [256+128b, +64), dP [320+128b, +64); dS (packed) over the first 32
-// columns of S.
+// S [256+128b, +64), dP [320+128b, +64); dS (packed) over columns 0-15
+// (keys 0-31) and 32-47 (keys 32-63) of S, each written by the warpgroup
+// that read them.
 namespace dqk {
 constexpr int kHalf64 = 64 * 128;
 constexpr int kOffQ = 0;
@@ -420,7 +486,7 @@ constexpr size_t kSmem = 1024 + kOffBar + 256;
 constexpr uint32_t kTmQ = 0, kTmDO = 64, kTmDQ = 128, kTmBuf = 256;
 }  // namespace dqk
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads2, 1)
     attn_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                 BwdParams p) {
@@ -430,11 +496,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* q_ready = bars + 1;     // Q and dO copied into TMEM (128 arrivals)
+  uint64_t* q_ready = bars + 1;     // Q and dO copied into TMEM (256 arrivals)
   uint64_t* st_full = bars + 2;     // [kStages]
   uint64_t* st_empty = bars + 2 + kStages;
   uint64_t* s_full = bars + 2 + 2 * kStages;   // [2]
-  uint64_t* p_full = bars + 4 + 2 * kStages;   // [2] (128 arrivals)
+  uint64_t* p_full = bars + 4 + 2 * kStages;   // [2] (256 arrivals)
   uint64_t* acc_full = bars + 6 + 2 * kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7 + 2 * kStages);
 
@@ -448,14 +514,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_trigger();
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_ready, 128);
+    mbar_init(q_ready, 256);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&st_full[i], 1);
       mbar_init(&st_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 256);
     }
     mbar_init(acc_full, 1);
     fence_mbar_init();
@@ -519,7 +585,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t a = tmem + kTmBuf + 128u * b;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {  // 16 keys per K-step: 16 rows of 128 bytes
-        umma_f16_ts(tmem + kTmDQ, a + kk * 8, sdesc_mnmajor_sw128(k_addr + kk * 2048, kHalf64),
+        // dS of keys 0-31 is packed at columns 0-15, of keys 32-63 at 32-47
+        const uint32_t col = static_cast<uint32_t>((kk >> 1) * 32 + (kk & 1) * 8);
+        umma_f16_ts(tmem + kTmDQ, a + col, sdesc_mnmajor_sw128(k_addr + kk * 2048, kHalf64),
                     idesc_n128_mn, (m > 0 || kk > 0) ? 1u : 0u);
       }
       umma_commit(&st_empty[st]);
@@ -542,8 +610,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ one thread per query row
-    const int r = threadIdx.x - 128;
+    // ------------------------------------------------------------ row math
+    // Warpgroup wg (warps 4-7: 0, warps 8-11: 1) forms keys 32 wg .. 32 wg + 31
+    // of each 64-key stage for every query row (one thread per row).
+    const int wg = (warp - 4) >> 2;
+    const int r = (threadIdx.x - 128) & 127;
     const int64_t i = static_cast<int64_t>(i0) + r;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float tau = p.tau ? __ldg(p.tau + h) : 1.0f;
@@ -553,9 +624,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float lse2 = __ldg(p.lse2 + static_cast<int64_t>(h) * p.t_pad + i);
     const float di = __ldg(p.dd + static_cast<int64_t>(h) * p.t_pad + i);
     bool ok = mbar_wait_warp(q_full, 0, p.err);
-    if (ok) {
-      tile_row_to_tmem(smem + kOffQ, r, tmem + lane_off + kTmQ);
-      tile_row_to_tmem(smem + kOffDO, r, tmem + lane_off + kTmDO);
+    if (ok) {  // Q (warpgroup 0) and dO (warpgroup 1) into TMEM
+      tile_row_to_tmem(smem + (wg ? kOffDO : kOffQ), r, tmem + lane_off + (wg ? kTmDO : kTmQ));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(q_ready);
@@ -572,36 +642,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                          kStBias);
       const int lim = static_cast<int>(i - 64 * m);  // key 64m + t is visible when t <= lim
       const uint32_t ta = tmem + lane_off + kTmBuf + 128u * b;
+      const int c = wg;
+      uint32_t rs[32], rp[32];
+      tmem_ld32(ta + 32u * c, rs);
+      tmem_ld32(ta + 64u + 32u * c, rp);
+      tmem_wait_ld_dep(rp);
+      tmem_ld_fence(rs);
+      uint32_t dk16[16];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t rs[32], rp[32];
-        tmem_ld32(ta + 32u * c, rs);
-        tmem_ld32(ta + 64u + 32u * c, rp);
-        tmem_wait_ld_dep(rp);
-        tmem_ld_fence(rs);
-        uint32_t dk16[16];
-#pragma unroll
-        for (int t = 0; t < 32; t += 2) {
-          const int jl = 32 * c + t;
-          float p0 = ex2_approx(fmaf(__uint_as_float(rs[t]), scale2, gb2 * bias[jl]) - lse2);
-          float p1 = ex2_approx(fmaf(__uint_as_float(rs[t + 1]), scale2, gb2 * bias[jl + 1]) - lse2);
-          if (jl > lim) p0 = 0.f;
-          if (jl + 1 > lim) p1 = 0.f;
-          dk16[t >> 1] = pack_bf16x2(p0 * (__uint_as_float(rp[t]) - di),
-                                     p1 * (__uint_as_float(rp[t + 1]) - di));
-        }
-        tmem_st16(ta + 16u * c, dk16);
+      for (int t = 0; t < 32; t += 2) {
+        const int jl = 32 * c + t;
+        float p0 = ex2_approx(fmaf(__uint_as_float(rs[t]), scale2, gb2 * bias[jl]) - lse2);
+        float p1 = ex2_approx(fmaf(__uint_as_float(rs[t + 1]), scale2, gb2 * bias[jl + 1]) - lse2);
+        if (jl > lim) p0 = 0.f;
+        if (jl + 1 > lim) p1 = 0.f;
+        dk16[t >> 1] = pack_bf16x2(p0 * (__uint_as_float(rp[t]) - di),
+                                   p1 * (__uint_as_float(rp[t + 1]) - di));
       }
+      tmem_st16(ta + 32u * c, dk16);  // into this warpgroup's own (already read) columns
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[b]);
     }
     if (ok && mbar_wait_warp(acc_full, 0, p.err)) {
       tc_fence_after();
-      float x[128];
-      tmem_ld128(tmem + lane_off + kTmDQ, x);
+      // this warpgroup's columns: [32 wg, 32 wg + 32) and [64 + 32 wg, 96 + 32 wg)
+      float lo[32], hi[32];
+      tmem_ld2x32(tmem + lane_off + kTmDQ + 32u * wg, tmem + lane_off + kTmDQ + 64u + 32u * wg,
+                  lo, hi);
 #pragma unroll
-      for (int e = 0; e < 128; ++e) x[e] *= inv_st;
+      for (int e = 0; e < 32; ++e) {
+        lo[e] *= inv_st;
+        hi[e] *= inv_st;
+      }
       // q_i . dq_i in the rotated frame (rows past T contribute nothing)
       float dot = 0.f;
       if (i < p.T) {
@@ -609,15 +682,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int hs = 0; hs < 2; ++hs) {
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int ch = 4 * wg + k4;
             const uint4 u =
                 *reinterpret_cast<const uint4*>(qrow + hs * kSub + ((ch ^ (r & 7)) << 4));
             const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
             for (int q2 = 0; q2 < 4; ++q2) {
               const float2 f = __bfloat1622float2(e2[q2]);
-              const int d = hs * 64 + ch * 8 + 2 * q2;
-              dot = fmaf(f.x, x[d], fmaf(f.y, x[d + 1], dot));
+              const int d = k4 * 8 + 2 * q2;  // within this warpgroup's 32 columns
+              dot = hs ? fmaf(f.x, hi[d], fmaf(f.y, hi[d + 1], dot))
+                       : fmaf(f.x, lo[d], fmaf(f.y, lo[d + 1], dot));
             }
           }
         }
@@ -625,10 +700,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xFFFFFFFFu, dot, o);
       if (lane == 0)
-        p.qdq[(static_cast<int64_t>(h) * p.n_tiles + it) * 4 + (warp & 3)] = dot;
+        p.qdq[(static_cast<int64_t>(h) * p.n_tiles + it) * 8 + wg * 4 + (warp & 3)] = dot;
       if (i < p.T) {
-        rope_back(x, p.cs, p.T, i);
-        store_row_bf16(p.dq + (i * p.hq + h) * kDh, x);
+        rope_back32(lo, hi, p.cs, p.T, i, 32 * wg);
+        store32_bf16(p.dq + (i * p.hq + h) * kDh + 32 * wg, lo);
+        store32_bf16(p.dq + (i * p.hq + h) * kDh + 64 + 32 * wg, hi);
       }
     }
   }
@@ -778,8 +854,8 @@ struct FinalArgs {
   const float* bias;    // [t_pad] logsigmoid(s)
   const float* gain;    // [hq] or null
   const float* tau;     // [hq] or null
-  const float* colsum;  // [hq, t_pad]
-  const float* qdq;     // [hq, n_tiles, 4]
+  const float* colsum;  // [2, hq, t_pad] (two partial sums per entry)
+  const float* qdq;     // [hq, n_tiles, 8]
   int64_t T, t_pad;
   int hq, n_tiles;
   float* ds;            // [T] or null
@@ -808,11 +884,14 @@ __global__ void __launch_bounds__(256) attn_bwd_final(FinalArgs a) {
     float acc = 0.f;
     if (a.s)
       for (int64_t j = threadIdx.x; j < a.T; j += 256)
-        acc = fmaf(__ldg(a.bias + j), __ldg(a.colsum + static_cast<int64_t>(h) * a.t_pad + j), acc);
+        acc = fmaf(__ldg(a.bias + j),
+                   __ldg(a.colsum + static_cast<int64_t>(h) * a.t_pad + j) +
+                       __ldg(a.colsum + static_cast<int64_t>(a.hq + h) * a.t_pad + j),
+                   acc);
     const float dg = block_sum_256(acc, red);
     float acc2 = 0.f;
-    for (int e = threadIdx.x; e < a.n_tiles * 4; e += 256)
-      acc2 += __ldg(a.qdq + static_cast<int64_t>(h) * a.n_tiles * 4 + e);
+    for (int e = threadIdx.x; e < a.n_tiles * 8; e += 256)
+      acc2 += __ldg(a.qdq + static_cast<int64_t>(h) * a.n_tiles * 8 + e);
     const float qd = block_sum_256(acc2, red);
     if (threadIdx.x == 0) {
       if (a.dgain) a.dgain[h] = dg;
@@ -825,7 +904,10 @@ __global__ void __launch_bounds__(256) attn_bwd_final(FinalArgs a) {
   float sum = 0.f;
   if (a.gain)
     for (int h = 0; h < a.hq; ++h)
-      sum = fmaf(__ldg(a.gain + h), __ldg(a.colsum + static_cast<int64_t>(h) * a.t_pad + j), sum);
+      sum = fmaf(__ldg(a.gain + h),
+                 __ldg(a.colsum + static_cast<int64_t>(h) * a.t_pad + j) +
+                     __ldg(a.colsum + static_cast<int64_t>(a.hq + h) * a.t_pad + j),
+                 sum);
   a.ds[j] = sum / (1.0f + expf(__ldg(a.s + j)));  // sigmoid(-s_j) = 1 / (1 + e^s_j)
 }
 
@@ -924,8 +1006,8 @@ cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t st, int stage) {
                                          int(dkdv::kSmem));
     if (err != cudaSuccess) return err;
     const unsigned grid = static_cast<unsigned>(n_tiles) * static_cast<unsigned>(a.hkv);
-    return launch_pdl(attn_bwd_dkdv, dim3(grid), dim3(kThreads), dkdv::kSmem, st, tq, tk, tv, tdo,
-                      tqT, tdoT, p);
+    return launch_pdl(attn_bwd_dkdv, dim3(grid), dim3(kThreads2), dkdv::kSmem, st, tq, tk, tv,
+                      tdo, tqT, tdoT, p);
   }
   CUtensorMap tq, tk, tv, tdo;
   if (!rows_map(&tq, a.q_rot, a.hq, kBlk) || !rows_map(&tdo, a.dout, a.hq, kBlk) ||
@@ -934,7 +1016,8 @@ cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t st, int stage) {
   cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(attn_bwd_dq), int(dqk::kSmem));
   if (err != cudaSuccess) return err;
   const unsigned grid = static_cast<unsigned>(n_tiles) * static_cast<unsigned>(a.hq);
-  return launch_pdl(attn_bwd_dq, dim3(grid), dim3(kThreads), dqk::kSmem, st, tq, tk, tv, tdo, p);
+  return launch_pdl(attn_bwd_dq, dim3(grid), dim3(kThreads2), dqk::kSmem, st, tq, tk, tv, tdo,
+                    p);
 }
 
 }  // namespace tg

@@ -167,8 +167,8 @@ struct AttnBwdPlan {
   void* doT = nullptr;     // [hq, dh, t_pad]
   float* lse2 = nullptr;   // [hq, t_pad]
   float* dd = nullptr;     // [hq, t_pad]
-  float* colsum = nullptr; // [hq, t_pad]
-  float* qdq = nullptr;    // [hq, t_pad / 128, 4]
+  float* colsum = nullptr; // [2, hq, t_pad]
+  float* qdq = nullptr;    // [hq, t_pad / 128, 8]
   float* bias = nullptr;   // [t_pad] logsigmoid(s), zero-padded
   int64_t t_pad = 0;
   size_t bytes = 0;
@@ -183,8 +183,8 @@ struct AttnBwdPlan {
     doT = a.carve(size_t(hq) * dh * tp * 2);
     lse2 = static_cast<float*>(a.carve(size_t(hq) * tp * 4));
     dd = static_cast<float*>(a.carve(size_t(hq) * tp * 4));
-    colsum = static_cast<float*>(a.carve(size_t(hq) * tp * 4));
-    qdq = static_cast<float*>(a.carve(size_t(hq) * (tp / 128) * 16));
+    colsum = static_cast<float*>(a.carve(size_t(2) * hq * tp * 4));
+    qdq = static_cast<float*>(a.carve(size_t(hq) * (tp / 128) * 32));
     bias = static_cast<float*>(a.carve(tp * 4));
     bytes = a.used;
   }

@@ -179,8 +179,9 @@ struct AttnBwdArgs {
   void* q_rot; void* k_rot;              // workspace [T, hq|hkv, dh], rotated as in the forward
   float2* cs;                            // workspace [dh/2, T] RoPE (cos, sin) table
   void* qT; void* doT;                   // workspace [hq, dh, t_pad] (transposed q, dO)
-  float* lse2; float* dd; float* colsum; // workspace [hq, t_pad]
-  float* qdq;                            // workspace [hq, n_tiles, 4]
+  float* lse2; float* dd;                // workspace [hq, t_pad]
+  float* colsum;                         // workspace [2, hq, t_pad]
+  float* qdq;                            // workspace [hq, n_tiles, 8]
   float* bias;                           // workspace [t_pad] logsigmoid(s), zero-padded
   void* dq; void* dk; void* dv;          // outputs [T, H, dh]
   float* ds; float* dgain; float* dtau;  // outputs, each optional
