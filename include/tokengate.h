@@ -185,7 +185,8 @@ tg_status tg_gated_attn_prefill(const void* q, const void* kk, const void* v, co
  *   bf16. The backward forms D_i = dout_i . o_i; from the bf16 output that
  *   product carries the output's rounding (2^-9 relative) into every
  *   gradient of row i, so pass this when exact-to-fp32 gradients matter.
- * bf16 only (dh == 128); other arguments, workspace (TG_OP_GATED_ATTN) and
+ * bf16 (dh == 128) or fp32 (dh 64 or 128; out is then already fp32 and
+ * out_f32 must be NULL); other arguments, workspace (TG_OP_GATED_ATTN) and
  * errors as tg_gated_attn_prefill. lse NULL, or out_f32 not 16-byte
  * aligned, is TG_ERR_INVALID_ARG.
  */
@@ -214,15 +215,16 @@ tg_status tg_gated_attn_forward(const void* q, const void* kk, const void* v, co
  * forward) and dq' the gradient before the rotation back.
  *   q, kk, v, pos, s, gain, tau, k, hq, hkv, dh, rope_base: the forward's
  *   inputs, unchanged since that call.
- *   out [k, hq, dh] bf16, out_f32 [k, hq, dh] fp32 or NULL, lse [hq, k]
+ *   out [k, hq, dh] dtype, out_f32 [k, hq, dh] fp32 or NULL, lse [hq, k]
  *   fp32: the forward's outputs (D_i = dout_i . o_i is taken from out_f32
  *   when given, else from out).
- *   dout [k, hq, dh] bf16.
- *   dq [k, hq, dh], dk [k, hkv, dh], dv [k, hkv, dh] bf16 (w.r.t. the
+ *   dout [k, hq, dh] dtype.
+ *   dq [k, hq, dh], dk [k, hkv, dh], dv [k, hkv, dh] dtype (w.r.t. the
  *   un-rotated q and kk); ds [k] fp32 or NULL (needs s); dgain [hq] fp32 or
  *   NULL (0 when s is NULL); dtau [hq] fp32 or NULL.
- * bf16 with dh == 128 only (else TG_ERR_UNSUPPORTED). All bf16 buffers and
- * ws 16-byte aligned (else TG_ERR_INVALID_ARG). Workspace:
+ * bf16 with dh == 128 (tensor cores), or fp32 with dh 64 or 128 (CUDA
+ * cores; out_f32 NULL); else TG_ERR_UNSUPPORTED. All bf16 buffers and ws
+ * 16-byte aligned (else TG_ERR_INVALID_ARG). Workspace:
  * tg_workspace_size(TG_OP_GATED_ATTN_BWD) with k, heads, head_dim. The
  * result is deterministic (fixed summation orders, no atomics).
  */

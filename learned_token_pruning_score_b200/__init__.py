@@ -301,7 +301,7 @@ def tg_gated_attn_forward(q, k, v, pos, s=None, gain=None, tau=None, rope_base: 
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty(hq, t, dtype=torch.float32, device=q.device)
-    if out_f32 is None and want_f32:
+    if out_f32 is None and want_f32 and q.dtype == torch.bfloat16:
         out_f32 = torch.empty(t, hq, dh, dtype=torch.float32, device=q.device)
     dt = _dt(q)
     need = tg_workspace_size(TG_OP_GATED_ATTN, k=t, n_heads_q=hq, n_heads_kv=hkv, head_dim=dh,

@@ -855,9 +855,9 @@ struct FinalArgs {
   const float* gain;    // [hq] or null
   const float* tau;     // [hq] or null
   const float* colsum;  // [2, hq, t_pad] (two partial sums per entry)
-  const float* qdq;     // [hq, n_tiles, 8]
-  int64_t T, t_pad;
-  int hq, n_tiles;
+  const float* qdq;     // [hq, per_head] partial sums of q . dq
+  int64_t T, t_pad, per_head;
+  int hq;
   float* ds;            // [T] or null
   float* dgain;         // [hq] or null
   float* dtau;          // [hq] or null
@@ -890,8 +890,8 @@ __global__ void __launch_bounds__(256) attn_bwd_final(FinalArgs a) {
                    acc);
     const float dg = block_sum_256(acc, red);
     float acc2 = 0.f;
-    for (int e = threadIdx.x; e < a.n_tiles * 8; e += 256)
-      acc2 += __ldg(a.qdq + static_cast<int64_t>(h) * a.n_tiles * 8 + e);
+    for (int64_t e = threadIdx.x; e < a.per_head; e += 256)
+      acc2 += __ldg(a.qdq + static_cast<int64_t>(h) * a.per_head + e);
     const float qd = block_sum_256(acc2, red);
     if (threadIdx.x == 0) {
       if (a.dgain) a.dgain[h] = dg;
@@ -977,7 +977,7 @@ cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t st, int stage) {
     f.T = a.T;
     f.t_pad = a.t_pad;
     f.hq = a.hq;
-    f.n_tiles = n_tiles;
+    f.per_head = a.qdq_per_head > 0 ? a.qdq_per_head : int64_t(n_tiles) * 8;
     f.ds = a.s ? a.ds : nullptr;
     f.dgain = a.dgain;
     f.dtau = a.dtau;

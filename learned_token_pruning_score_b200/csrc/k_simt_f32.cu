@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(256) attn_f32(AttnArgs a, int64_t v_stride) {
   }
   float* out = static_cast<float*>(a.out) + (i * a.hq + h) * kDh;
   const float inv = 1.0f / l;
+  if (a.lse && lane == 0) a.lse[static_cast<int64_t>(h) * a.T + i] = m + logf(l);
 #pragma unroll
   for (int p = 0; p < kPer; ++p) out[lane + 32 * p] = o[p] * inv;
 }

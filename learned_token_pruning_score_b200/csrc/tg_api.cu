@@ -158,6 +158,27 @@ struct AttnPlan {
   }
 };
 
+// Backward of the standalone gated attention in fp32 (head_dim 64 or 128).
+struct AttnBwdF32Plan {
+  float* q_rot = nullptr;   // [n, hq, dh]
+  float* k_rot = nullptr;   // [n, hkv, dh]
+  float* lsig = nullptr;    // [n]
+  float2* cs = nullptr;     // [dh/2, n]
+  float* colsum = nullptr;  // [2, hq, n]
+  float* qdq = nullptr;     // [hq, n]
+  size_t bytes = 0;
+  AttnBwdF32Plan(void* ws, int64_t n, int hq, int hkv, int dh) {
+    Arena a(ws);
+    q_rot = static_cast<float*>(a.carve(size_t(n) * hq * dh * 4));
+    k_rot = static_cast<float*>(a.carve(size_t(n) * hkv * dh * 4));
+    lsig = static_cast<float*>(a.carve(size_t(n) * 4 + 16));
+    cs = static_cast<float2*>(a.carve(size_t(dh / 2) * n * 8));
+    colsum = static_cast<float*>(a.carve(size_t(2) * hq * n * 4));
+    qdq = static_cast<float*>(a.carve(size_t(hq) * n * 4));
+    bytes = a.used;
+  }
+};
+
 // Backward of the standalone gated attention (bf16, head_dim 128).
 struct AttnBwdPlan {
   void* q_rot = nullptr;   // [n, hq, dh] rotated as in the forward
@@ -620,6 +641,8 @@ size_t tg_workspace_size(tg_op op, const tg_shape* s) {
     case TG_OP_GATED_ATTN:
       return AttnPlan(nullptr, s->k, s->n_heads_q, s->n_heads_kv, s->head_dim, s->dtype, true).bytes;
     case TG_OP_GATED_ATTN_BWD:
+      if (s->dtype == TG_F32)
+        return AttnBwdF32Plan(nullptr, s->k, s->n_heads_q, s->n_heads_kv, s->head_dim).bytes;
       return AttnBwdPlan(nullptr, s->k, s->n_heads_q, s->n_heads_kv, s->head_dim).bytes;
     case TG_OP_PREFILL: {
       tg_model m{};
@@ -758,8 +781,8 @@ tg_status tg_gated_attn_forward(const void* q, const void* kk, const void* v, co
                                 tg_dtype dt, void* out, float* lse, float* out_f32, void* ws,
                                 size_t ws_bytes, tg_stream stream) {
   TG_CHECK(dt == TG_BF16 || dt == TG_F32, TG_ERR_UNSUPPORTED);
-  TG_CHECK(dt == TG_BF16, TG_ERR_UNSUPPORTED);
   TG_CHECK(lse != nullptr && aligned16(out_f32), TG_ERR_INVALID_ARG);
+  TG_CHECK(dt == TG_BF16 || out_f32 == nullptr, TG_ERR_INVALID_ARG);  // fp32: out is the fp32 output
   return gated_attn(q, kk, v, pos, s, gain, tau, k, hq, hkv, dh, rope_base, dt, out, lse, out_f32,
                     ws, ws_bytes, stream);
 }
@@ -772,8 +795,58 @@ tg_status tg_gated_attn_backward(const void* q, const void* kk, const void* v, c
                                  void* dk, void* dv, float* ds, float* dgain, float* dtau,
                                  void* ws, size_t ws_bytes, tg_stream stream) {
   TG_CHECK(dt == TG_BF16 || dt == TG_F32, TG_ERR_UNSUPPORTED);
-  TG_CHECK(dt == TG_BF16 && dh == 128, TG_ERR_UNSUPPORTED);
+  TG_CHECK(dt == TG_BF16 ? dh == 128 : (dh == 64 || dh == 128), TG_ERR_UNSUPPORTED);
   TG_CHECK(q && kk && v && pos && out && lse && dout && dq && dk && dv, TG_ERR_INVALID_ARG);
+  if (dt == TG_F32) {
+    TG_CHECK(k >= 1 && hq >= 1 && hkv >= 1 && k < (int64_t(1) << 31) - 256, TG_ERR_INVALID_ARG);
+    TG_CHECK(hq % hkv == 0 && rope_base > 1.f, TG_ERR_INVALID_ARG);
+    TG_CHECK(ds == nullptr || s != nullptr, TG_ERR_INVALID_ARG);
+    TG_CHECK(out_f32 == nullptr && aligned16(ws), TG_ERR_INVALID_ARG);
+    AttnBwdF32Plan fp(nullptr, k, hq, hkv, dh);
+    TG_CHECK(ws != nullptr && ws_bytes >= fp.bytes, TG_ERR_WORKSPACE);
+    fp = AttnBwdF32Plan(ws, k, hq, hkv, dh);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    RopePrepArgs r{};
+    r.q_src = q; r.k_src = kk; r.v_src = v;
+    r.q_stride = int64_t(hq) * dh; r.k_stride = int64_t(hkv) * dh; r.v_stride = int64_t(hkv) * dh;
+    r.pos = pos;
+    r.T = k; r.hq = hq; r.hkv = hkv; r.dh = dh; r.rope_base = rope_base;
+    r.bf16 = false;
+    r.q_out = fp.q_rot;
+    r.k_out = fp.k_rot;
+    r.s = s;
+    r.lsig_out = fp.lsig;
+    const double rows = double(k);
+    TG_TRY(traced(TG_K_ROPE_PREP, k, 0.0, rows * (hq + hkv) * dh * 8.0, st,
+                  [&] { return launch_rope_prep(r, st); }));
+    TG_TRY(traced(TG_K_ROPE_TABLE, k, 0.0, 8.0 * (dh / 2) * rows, st,
+                  [&] { return launch_rope_table(pos, k, dh, rope_base, fp.cs, st); }));
+    AttnBwdF32Args b{};
+    b.q_rot = fp.q_rot; b.k_rot = fp.k_rot;
+    b.v = static_cast<const float*>(v);
+    b.out = static_cast<const float*>(out);
+    b.dout = static_cast<const float*>(dout);
+    b.lse = lse;
+    b.lsig = s ? fp.lsig : nullptr;
+    b.gain = gain; b.tau = tau; b.cs = fp.cs;
+    b.T = k; b.t_pad = k; b.hq = hq; b.hkv = hkv; b.dh = dh;
+    b.colsum = s ? fp.colsum : nullptr;
+    b.qdq = fp.qdq;
+    b.dq = static_cast<float*>(dq); b.dk = static_cast<float*>(dk); b.dv = static_cast<float*>(dv);
+    const double prod = 2.0 * dh * hq * rows * (rows + 1) / 2.0;
+    TG_TRY(traced(TG_K_ATTENTION_F32, k, 4.0 * prod, 0.0, st,
+                  [&] { return launch_attn_bwd_f32(b, st); }));
+    if (ds || dgain || dtau) {
+      AttnBwdArgs f{};
+      f.s = s; f.bias = fp.lsig; f.gain = gain; f.tau = tau;
+      f.colsum = fp.colsum; f.qdq = fp.qdq; f.qdq_per_head = k;
+      f.T = k; f.t_pad = k; f.hq = hq; f.hkv = hkv;
+      f.ds = ds; f.dgain = dgain; f.dtau = dtau;
+      TG_TRY(traced(TG_K_ATTN_BWD_FINAL, k, 0.0, rows * hq * 4.0, st,
+                    [&] { return launch_attn_bwd(f, st, 3); }));
+    }
+    return TG_OK;
+  }
   TG_CHECK(k >= 1 && hq >= 1 && hkv >= 1 && k < (int64_t(1) << 31) - 256, TG_ERR_INVALID_ARG);
   TG_CHECK(hq % hkv == 0 && rope_base > 1.f, TG_ERR_INVALID_ARG);
   TG_CHECK(ds == nullptr || s != nullptr, TG_ERR_INVALID_ARG);

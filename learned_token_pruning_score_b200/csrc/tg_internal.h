@@ -185,11 +185,29 @@ struct AttnBwdArgs {
   float* bias;                           // workspace [t_pad] logsigmoid(s), zero-padded
   void* dq; void* dk; void* dv;          // outputs [T, H, dh]
   float* ds; float* dgain; float* dtau;  // outputs, each optional
+  int64_t qdq_per_head;                  // entries of qdq per head (0: n_tiles * 8)
 };
 size_t attn_bwd_t_pad(int64_t T);
 // stage 0: prep (RoPE, transposes of q and dO, table, lse2, D, bias); 1: dK/dV/C;
 // 2: dQ; 3: ds/dgain/dtau.
 cudaError_t launch_attn_bwd(const AttnBwdArgs& a, cudaStream_t st, int stage);
+
+// fp32 backward on the CUDA cores (k_attn_bwd_f32.cu), head_dim 64 or 128:
+// dq, dk, dv, the per-key sums C (colsum [2, hq, t_pad], second half zero)
+// and the per-row q . dq (qdq [hq, T]); ds/dgain/dtau then come from
+// launch_attn_bwd stage 3 with qdq_per_head = T.
+struct AttnBwdF32Args {
+  const float* q_rot; const float* k_rot;  // [T, hq|hkv, dh] rotated
+  const float* v; const float* out; const float* dout;
+  const float* lse;                        // [hq, T]
+  const float* lsig;                       // [T] or null
+  const float* gain; const float* tau;
+  const float2* cs;                        // [dh/2, T]
+  int64_t T, t_pad; int hq, hkv, dh;
+  float* colsum; float* qdq;
+  float* dq; float* dk; float* dv;
+};
+cudaError_t launch_attn_bwd_f32(const AttnBwdF32Args& a, cudaStream_t st);
 
 // ---- decode (k_decode.cu): one generated token, batch 1, bf16, head_dim 128.
 // One cooperative launch per step runs every layer (see k_decode.cu).

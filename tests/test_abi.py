@@ -113,8 +113,8 @@ def test_attention_forward_lse_and_backward_validation():
         tg.TG_ERR_INVALID_ARG  # no lse
     assert fwd(*base, tg.TG_BF16, BOGUS, BOGUS, ctypes.c_void_p(4096 + 4), BOGUS, 1 << 30,
                None) == tg.TG_ERR_INVALID_ARG  # misaligned fp32 output
-    assert fwd(*base, tg.TG_F32, BOGUS, BOGUS, None, BOGUS, 1 << 30, None) == \
-        tg.TG_ERR_UNSUPPORTED
+    assert fwd(*base, tg.TG_F32, BOGUS, BOGUS, BOGUS, BOGUS, 1 << 30, None) == \
+        tg.TG_ERR_INVALID_ARG  # fp32: the output is already fp32, no second copy
     assert fwd(*base, tg.TG_BF16, BOGUS, BOGUS, None, BOGUS, 64, None) == tg.TG_ERR_WORKSPACE
     bwd = tg._attn_bwd
     need = tg.tg_workspace_size(tg.TG_OP_GATED_ATTN_BWD, k=128, n_heads_q=4, n_heads_kv=2,
@@ -124,12 +124,17 @@ def test_attention_forward_lse_and_backward_validation():
     outs = [BOGUS, BOGUS, BOGUS, BOGUS, BOGUS, BOGUS]  # dq, dk, dv, ds, dgain, dtau
 
     def call(dt=tg.TG_BF16, dh=128, hq=4, hkv=2, s=BOGUS, out=BOGUS, o=outs, ws=BOGUS,
-             ws_bytes=1 << 30):
+             ws_bytes=1 << 30, o32=None):
         return bwd(BOGUS, BOGUS, BOGUS, BOGUS, s, None, None, 128, hq, hkv, dh, 1e6, dt, out,
-                   None, BOGUS, BOGUS, *o, ws, ws_bytes, None)
+                   o32, BOGUS, BOGUS, *o, ws, ws_bytes, None)
 
-    assert call(dt=tg.TG_F32) == tg.TG_ERR_UNSUPPORTED
-    assert call(dh=64) == tg.TG_ERR_UNSUPPORTED
+    assert call(dt=tg.TG_F32, dh=96) == tg.TG_ERR_UNSUPPORTED
+    assert call(dt=tg.TG_F32, o32=BOGUS) == tg.TG_ERR_INVALID_ARG  # fp32 takes no fp32 copy
+    assert call(dt=7) == tg.TG_ERR_UNSUPPORTED
+    assert call(dh=64) == tg.TG_ERR_UNSUPPORTED  # bf16 needs head_dim 128
+    need32 = tg.tg_workspace_size(tg.TG_OP_GATED_ATTN_BWD, k=128, n_heads_q=4, n_heads_kv=2,
+                                  head_dim=64, dtype=tg.TG_F32)
+    assert call(dt=tg.TG_F32, dh=64, ws_bytes=need32 - 1) == tg.TG_ERR_WORKSPACE
     assert call(hkv=3) == tg.TG_ERR_INVALID_ARG  # hq % hkv != 0
     assert call(out=None) == tg.TG_ERR_INVALID_ARG
     assert call(s=None) == tg.TG_ERR_INVALID_ARG  # ds asked for without scores

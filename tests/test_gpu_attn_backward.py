@@ -265,3 +265,51 @@ def test_attn_backward_constant_scores():
     assert_within_budget(ds, want[3], budget[3], "ds constant scores")
     scale = float(np.abs(want[3]).sum())
     assert np.all(np.abs(host64(dgain)) <= 1e-3 * scale)
+
+
+# ---------------------------------------------------------------- fp32 (CUDA cores)
+
+
+def _inputs_f32(t, hq, hkv, dh, seed, bias=True):
+    rng = np.random.default_rng(seed)
+    arrs = [rng.standard_normal((t, hq, dh)), rng.standard_normal((t, hkv, dh)),
+            rng.standard_normal((t, hkv, dh)), rng.standard_normal((t, hq, dh))]
+    pos = np.sort(rng.choice(max(4096, t), t, replace=False)).astype(np.int32)
+    s = (rng.standard_normal(t) * 2).astype(np.float32) if bias else None
+    gain = rng.uniform(0, 2, hq).astype(np.float32) if bias else None
+    tau = rng.uniform(0.5, 1.5, hq).astype(np.float32) if bias else None
+    dq_, dk_, dv_, do_ = (dev(x) for x in arrs)
+    d = dict(q=dq_, k=dk_, v=dv_, dout=do_, pos=torch.from_numpy(pos).cuda(),
+             s=None if s is None else dev(s), gain=None if gain is None else dev(gain),
+             tau=None if tau is None else dev(tau))
+    h = dict(q=host64(dq_), k=host64(dk_), v=host64(dv_), dout=host64(do_), pos=pos, s=s,
+             gain=gain, tau=tau)
+    return d, h
+
+
+@pytest.mark.parametrize("t,dh,bias", [(1, 64, True), (37, 64, True), (128, 128, True),
+                                       (200, 64, False), (300, 128, True)])
+def test_attn_backward_fp32(t, dh, bias):
+    # fp32 end to end: the gradients match the oracle to the fp32 tolerance
+    # (1e-4, the absolute term scaled by the tensor's RMS as in the bf16 case)
+    d, h = _inputs_f32(t, 4, 2, dh, 900 + t + dh, bias)
+    out, lse, o32 = tg.tg_gated_attn_forward(d["q"], d["k"], d["v"], d["pos"], d["s"], d["gain"],
+                                             d["tau"], rope_base=1e6)
+    assert o32 is None
+    grads = tg.tg_gated_attn_backward(d["q"], d["k"], d["v"], d["pos"], out, lse, d["dout"],
+                                      d["s"], d["gain"], d["tau"], rope_base=1e6)
+    torch.cuda.synchronize()
+    qr = ref.round_fp32(ref.rope(h["q"], h["pos"], 1e6))
+    kr = ref.round_fp32(ref.rope(h["k"], h["pos"], 1e6))
+    want_lse = ref.gated_attention_lse(qr, kr, h["pos"], h["s"], h["gain"], h["tau"])
+    assert np.max(np.abs(host64(lse) - want_lse)) <= 1e-4
+    want = ref.gated_attn_backward(h["q"], h["k"], h["v"], h["pos"], h["s"], h["gain"], h["tau"],
+                                   1e6, h["dout"], store=ref.round_fp32)
+    for name, g, r in zip(("dq", "dk", "dv", "ds", "dgain", "dtau"), grads, want):
+        if r is None:
+            assert g is None, name
+            continue
+        gg, rr = host64(g), np.asarray(r, dtype=np.float64)
+        rms = math.sqrt(float(np.mean(rr * rr))) if rr.size else 0.0
+        bad = np.abs(gg - rr) > 1e-4 * max(rms, 1e-3) + 1e-4 * np.abs(rr)
+        assert not bad.any(), (name, t, dh, float(np.abs(gg - rr).max()), rms)
