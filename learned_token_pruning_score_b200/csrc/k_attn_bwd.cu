@@ -62,7 +62,6 @@ namespace {
 
 constexpr int kBlk = 128;        // rows per tile (queries or keys)
 constexpr int kDh = 128;
-constexpr int kThreads = 256;
 constexpr int kThreads2 = 384;   // dK/dV and dQ: roles + two row-math warpgroups
 constexpr int kSub = 128 * 128;  // bytes of one [128 rows x 64 bf16] 128-byte-swizzled sub-tile
 constexpr int kTile = 2 * kSub;  // [128 x 128] bf16 tile
@@ -84,32 +83,6 @@ struct BwdParams {
   float* qdq;            // [hq, n_tiles, 8] per-warp partial sums of q_i . dq_i
   unsigned int* err;
 };
-
-// Rotate a gradient row (dh = 128, rotate-half pairs (i, i + 64)) back
-// through RoPE: the transpose of the forward rotation.
-__device__ __forceinline__ void rope_back(float (&x)[128], const float2* cs, int64_t T,
-                                          int64_t row) {
-#pragma unroll
-  for (int i = 0; i < 64; ++i) {
-    const float2 c = __ldg(cs + static_cast<int64_t>(i) * T + row);
-    const float a = x[i], b = x[i + 64];
-    x[i] = a * c.x + b * c.y;
-    x[i + 64] = b * c.x - a * c.y;
-  }
-}
-
-__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const float (&x)[128]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int v = 0; v < 16; ++v) {
-    uint4 u;
-    u.x = pack_bf16x2(x[8 * v + 0], x[8 * v + 1]);
-    u.y = pack_bf16x2(x[8 * v + 2], x[8 * v + 3]);
-    u.z = pack_bf16x2(x[8 * v + 4], x[8 * v + 5]);
-    u.w = pack_bf16x2(x[8 * v + 6], x[8 * v + 7]);
-    d[v] = u;
-  }
-}
 
 // Stores 32 fp32 values as bf16 (four 16-byte vectors).
 __device__ __forceinline__ void store32_bf16(__nv_bfloat16* dst, const float* x) {
@@ -150,26 +123,6 @@ __device__ __forceinline__ void rope_back32(float (&lo)[32], float (&hi)[32], co
     const float a = lo[i], b = hi[i];
     lo[i] = a * c.x + b * c.y;
     hi[i] = b * c.x - a * c.y;
-  }
-}
-
-// Four TMEM loads of 32 columns into x[128] (one wait).
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&x)[128]) {
-  uint32_t r0[32], r1[32], r2[32], r3[32];
-  tmem_ld32(taddr, r0);
-  tmem_ld32(taddr + 32, r1);
-  tmem_ld32(taddr + 64, r2);
-  tmem_ld32(taddr + 96, r3);
-  tmem_wait_ld_dep(r3);
-  tmem_ld_fence(r0);
-  tmem_ld_fence(r1);
-  tmem_ld_fence(r2);
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    x[i] = __uint_as_float(r0[i]);
-    x[32 + i] = __uint_as_float(r1[i]);
-    x[64 + i] = __uint_as_float(r2[i]);
-    x[96 + i] = __uint_as_float(r3[i]);
   }
 }
 
