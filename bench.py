@@ -507,9 +507,10 @@ def run_ours(args, rank, world, local_rank):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / args.steps}
 
-    # ---- other budgets, dense baseline and peak memory (not timed region)
+    # ---- other budgets, dense baseline and peak memory (not timed region;
+    # single-GPU runs only: the replicas of a multi-GPU run report the headline)
     extras = {}
-    if not args.quick:
+    if not args.quick and world == 1:
         def ttft(mdl, kk, reps=5):
             # peak memory of one prefill: weights + input + outputs (incl. KV
             # cache) + workspace, all allocated by the caller
