@@ -250,3 +250,55 @@ def decode_state(w: Workload, rng: np.random.Generator, generated: int = 0) -> D
     x = rng.standard_normal(w.d, dtype=np.float32)
     return {"lens": lens, "caches": caches, "scores": scores, "kept_idx": kept, "x": x,
             "pos": w.n + generated}
+
+
+# ---------------------------------------------------------------- hybrid models
+@dataclass(frozen=True)
+class GdnWorkload:
+    """A Gated DeltaNet layer's token mixer over T tokens (the kept tokens of
+    a gated prefill; n is what the same layer sees without the gate)."""
+    name: str
+    dtype: str
+    T: int
+    n: int
+    hk: int
+    hv: int
+    dk: int
+    dv: int
+    W: int
+    seed: int
+    eps: float = 1e-6
+
+
+# Linear-attention layer of a hybrid model at d_model 2048 (Qwen3-Next-style
+# shape: 16 key and 16 value heads of dim 128, convolution width 4); the
+# pages give the hybrid model's name but not its sizes. K = 4096 of N = 32768.
+GDN_LAYER_32K = GdnWorkload("hybrid_gdn_mixer_n32k_k4k", "bf16", T=4096, n=32768, hk=16, hv=16,
+                            dk=128, dv=128, W=4, seed=5)
+
+
+def gdn_params(w: GdnWorkload, rng: np.random.Generator) -> Dict[str, np.ndarray]:
+    """float32 mixer parameters: conv_w [C, W] ~ U(+-1/sqrt(W)); A_log =
+    log U(1, 16); dt_bias ~ U(-7, -2); norm_w ~ 1 + 0.1 N(0, 1)."""
+    C = 2 * w.hk * w.dk + w.hv * w.dv
+    lim = 1.0 / np.sqrt(w.W)
+    return {
+        "conv_w": rng.uniform(-lim, lim, (C, w.W)).astype(np.float32),
+        "A_log": np.log(rng.uniform(1.0, 16.0, w.hv)).astype(np.float32),
+        "dt_bias": rng.uniform(-7.0, -2.0, w.hv).astype(np.float32),
+        "norm_w": (1.0 + 0.1 * rng.standard_normal(w.dv)).astype(np.float32),
+    }
+
+
+def gdn_inputs(w: GdnWorkload, rng: np.random.Generator, T: Optional[int] = None
+               ) -> Dict[str, np.ndarray]:
+    """float32 projection outputs for T tokens (default w.T): qkv [T, C],
+    z [T, hv dv], a and b [T, hv], all ~ N(0, 1)."""
+    T = w.T if T is None else T
+    C = 2 * w.hk * w.dk + w.hv * w.dv
+    return {
+        "qkv": rng.standard_normal((T, C), dtype=np.float32),
+        "z": rng.standard_normal((T, w.hv * w.dv), dtype=np.float32),
+        "a": rng.standard_normal((T, w.hv), dtype=np.float32),
+        "b": rng.standard_normal((T, w.hv), dtype=np.float32),
+    }
