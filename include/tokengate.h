@@ -394,6 +394,67 @@ tg_status tg_decode_step(const tg_model* model, const void* x, int64_t pos, int3
                          const int32_t* kept_idx, int64_t k_kept, void* out, void* ws,
                          size_t ws_bytes, tg_stream stream);
 
+/* ---- hybrid models: the Gated DeltaNet mixer -----------------------------
+ *
+ * In a hybrid model most layers are Gated DeltaNet layers and only some are
+ * full attention. The scorer reads hidden states, so the gate may sit at a
+ * Gated DeltaNet layer. Above the gate the token-gated logit bias applies
+ * only in the full-attention layers (tg_gated_attn_prefill); a Gated
+ * DeltaNet layer has no logits and runs on the kept tokens as they are
+ * ([TC] "门控位置影响剪枝效果", figure 5). The layer's projections are plain
+ * GEMMs (tg_linear); this call is its token mixer over one sequence, the K
+ * kept rows in ascending original order (the pages do not spell the layer
+ * out; the mixer is the published gated delta rule of Yang, Kautz and
+ * Hatamizadeh, "Gated Delta Networks", ICLR 2025, in the Qwen3-Next shape):
+ *   c_t = SiLU(sum_{i<W} conv_w[:, i] * x_{t-W+1+i})  over the qkv channels
+ *   q = l2norm(c_q) / sqrt(dk), k = l2norm(c_k), v = c_v  (l2norm: x / sqrt(|x|^2 + 1e-6))
+ *   alpha = exp(-exp(A_log) * softplus(a_t + dt_bias)), beta = sigmoid(b_t)
+ *   S_t = alpha S_{t-1} (I - beta k k^T) + beta v k^T,  o_t = S_t q  (per value head)
+ *   y_t = o_t / sqrt(mean(o_t^2) + norm_eps) * norm_w * SiLU(z_t)    (per value head)
+ * Value head h reads key head h / (hv / hk).
+ */
+typedef struct {
+  int32_t n_heads_k;   /* hk                                               */
+  int32_t n_heads_v;   /* hv, a multiple of hk                             */
+  int32_t head_dim_k;  /* dk: 64 or 128                                    */
+  int32_t head_dim_v;  /* dv: a multiple of 32, at most 256                */
+  int32_t conv_width;  /* W: 1..8                                          */
+  const float* conv_w; /* [C, W] with C = 2 hk dk + hv dv                  */
+  const float* A_log;  /* [hv]                                             */
+  const float* dt_bias;/* [hv]                                             */
+  const float* norm_w; /* [dv]                                             */
+  float norm_eps;
+} tg_gdn_layer;
+
+/* Workspace bytes of tg_gated_deltanet for T tokens (0 for a bad layer). */
+size_t tg_gated_deltanet_workspace_size(const tg_gdn_layer* layer, int64_t T);
+
+/*
+ * tg_gated_deltanet -- the mixer above over T >= 0 tokens.
+ *   qkv [T, C] dtype: the projections before the convolution, channels
+ *     [q (hk dk) | k (hk dk) | v (hv dv)];  z [T, hv dv], a [T, hv],
+ *     b [T, hv] dtype.
+ *   conv_in [W-1, C] dtype or NULL (zeros): the rows before token 0;
+ *   conv_out [W-1, C] dtype or NULL: the last W-1 rows of [conv_in; qkv],
+ *     for a following call. Must not overlap conv_in.
+ *   state_in [hv, dv, dk] fp32 or NULL (zeros); state_out [hv, dv, dk] fp32
+ *     or NULL: S after the last token. state_out may equal state_in but not
+ *     overlap it otherwise.
+ *   y [T, hv dv] dtype.
+ * Splitting a sequence across calls that carry conv_out / state_out into the
+ * next call's conv_in / state_in gives the same result as one call, up to
+ * rounding (the carried conv rows are stored in dtype, as the inputs are).
+ * dtype bf16 or fp32; the arithmetic is fp32 throughout. ws 16-byte aligned.
+ * Errors: null pointers, T < 0, bad layer sizes or overlapping state buffers
+ * are TG_ERR_INVALID_ARG (dk other than 64/128 or dv outside the range is
+ * TG_ERR_UNSUPPORTED); a short workspace is TG_ERR_WORKSPACE.
+ */
+tg_status tg_gated_deltanet(const tg_gdn_layer* layer, const void* qkv, const void* z,
+                            const void* a, const void* b, int64_t T, tg_dtype dtype,
+                            const void* conv_in, void* conv_out, const float* state_in,
+                            float* state_out, void* y, void* ws, size_t ws_bytes,
+                            tg_stream stream);
+
 /* ---- launch tracing (optional) --------------------------------------------
  * Measurement aid with no counterpart on the pages (they report only
  * end-to-end prefill latency and memory). While tracing is on for a host
@@ -424,7 +485,10 @@ typedef enum {
   TG_K_ATTN_BWD_DKDV = 17,   /* backward: dK, dV and the per-key sums of dl (tcgen05) */
   TG_K_ATTN_BWD_DQ = 18,     /* backward: dQ and q . dq (tcgen05)                   */
   TG_K_ATTN_BWD_FINAL = 19,  /* backward: ds, dgain, dtau                           */
-  TG_K_COUNT = 20
+  TG_K_GDN_PREP = 20,        /* Gated DeltaNet: conv, norms, decay (+ conv rows)     */
+  TG_K_GDN_RECUR = 21,       /* Gated DeltaNet: the delta-rule recurrence            */
+  TG_K_GDN_OUT = 22,         /* Gated DeltaNet: gated output RMSNorm                 */
+  TG_K_COUNT = 23
 } tg_kernel;
 
 typedef struct {

@@ -63,6 +63,12 @@ class TgKV(ctypes.Structure):
     _fields_ = [("k", _c_p), ("v", _c_p)]
 
 
+class TgGdnLayer(ctypes.Structure):
+    _fields_ = [("n_heads_k", _c_i32), ("n_heads_v", _c_i32), ("head_dim_k", _c_i32),
+                ("head_dim_v", _c_i32), ("conv_width", _c_i32), ("conv_w", _c_p),
+                ("A_log", _c_p), ("dt_bias", _c_p), ("norm_w", _c_p), ("norm_eps", _c_f32)]
+
+
 class TgTraceRecord(ctypes.Structure):
     _fields_ = [("kernel", _c_i32), ("layer", _c_i32), ("rows", _c_i64), ("ms", _c_f32),
                 ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
@@ -105,6 +111,9 @@ _prefill_batch = _sig("tg_prefill_batch", _ci, ctypes.POINTER(TgModel), _c_p, _c
 _decode = _sig("tg_decode_step", _ci, ctypes.POINTER(TgModel), _c_p, _c_i64, _c_i32,
                ctypes.POINTER(TgKV), ctypes.POINTER(_c_i64), _c_p, _c_i64, _c_p, _c_i64, _c_p, _c_p,
                _c_sz, _c_p)
+_gdn_ws = _sig("tg_gated_deltanet_workspace_size", _c_sz, ctypes.POINTER(TgGdnLayer), _c_i64)
+_gdn = _sig("tg_gated_deltanet", _ci, ctypes.POINTER(TgGdnLayer), _c_p, _c_p, _c_p, _c_p, _c_i64,
+            _ci, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p)
 _status_string = _sig("tg_status_string", ctypes.c_char_p, _ci)
 _last_cuda_error = _sig("tg_last_cuda_error", _ci)
 _device_error = _sig("tg_device_error", _ci, ctypes.POINTER(ctypes.c_uint32), _ci)
@@ -340,6 +349,55 @@ def tg_gated_attn_backward(q, k, v, pos, out, lse, dout, s=None, gain=None, tau=
 
 
 @dataclass
+class GdnLayer:
+    """Parameters of a Gated DeltaNet layer's token mixer (fp32 device
+    tensors) plus the ctypes view tg_gated_deltanet takes: conv_w [C, W],
+    A_log [hv], dt_bias [hv], norm_w [dv], with C = 2 hk dk + hv dv."""
+
+    n_heads_k: int
+    n_heads_v: int
+    head_dim_k: int
+    head_dim_v: int
+    conv_w: torch.Tensor
+    A_log: torch.Tensor
+    dt_bias: torch.Tensor
+    norm_w: torch.Tensor
+    eps: float = 1e-6
+
+    def __post_init__(self):
+        self.conv_width = self.conv_w.shape[1]
+        self.channels = 2 * self.n_heads_k * self.head_dim_k + self.n_heads_v * self.head_dim_v
+        self.c = TgGdnLayer(self.n_heads_k, self.n_heads_v, self.head_dim_k, self.head_dim_v,
+                            self.conv_width, _ptr(self.conv_w), _ptr(self.A_log),
+                            _ptr(self.dt_bias), _ptr(self.norm_w), self.eps)
+
+
+def tg_gated_deltanet_workspace_size(layer: GdnLayer, T: int) -> int:
+    return int(_gdn_ws(ctypes.byref(layer.c), T))
+
+
+def tg_gated_deltanet(layer: GdnLayer, qkv, z, a, b, conv_in=None, state_in=None,
+                      want_state: bool = True, y=None, conv_out=None, state_out=None, ws=None,
+                      stream=None):
+    """The Gated DeltaNet mixer over the T rows of qkv [T, C], z [T, hv dv],
+    a, b [T, hv] (one dtype, bf16 or fp32). Returns (y, conv_out, state_out);
+    the last two are None when want_state is False and none is passed."""
+    T = qkv.shape[0]
+    dev = qkv.device
+    hv, dv, dk = layer.n_heads_v, layer.head_dim_v, layer.head_dim_k
+    y = torch.empty(T, hv * dv, dtype=qkv.dtype, device=dev) if y is None else y
+    if want_state and conv_out is None and layer.conv_width > 1:
+        conv_out = torch.empty(layer.conv_width - 1, layer.channels, dtype=qkv.dtype, device=dev)
+    if want_state and state_out is None:
+        state_out = torch.empty(hv, dv, dk, dtype=torch.float32, device=dev)
+    ws = _ws(tg_gated_deltanet_workspace_size(layer, T), dev, ws)
+    _check(_gdn(ctypes.byref(layer.c), _ptr(qkv), _ptr(z), _ptr(a), _ptr(b), T, _dt(qkv),
+                _ptr(conv_in), _ptr(conv_out), _ptr(state_in), _ptr(state_out), _ptr(y),
+                _ptr(ws), ws.numel(), _stream(stream, dev)), "tg_gated_deltanet")
+    return y, conv_out, state_out
+
+
+@dataclass
 class Model:
     """Device tensors of a decoder stack plus the ctypes view tg_prefill takes.
 
@@ -502,5 +560,5 @@ __all__ = [
     "TokenGateError", "LIB_PATH", "tg_trace_start", "tg_trace_stop", "TG_OK", "TG_ERR_INVALID_ARG", "TG_ERR_UNSUPPORTED",
     "TG_ERR_BUDGET", "TG_ERR_WORKSPACE", "TG_ERR_CUDA", "TG_F32", "TG_BF16", "TG_OP_SCORE",
     "TG_OP_TOPK_SELECT", "TG_OP_COMPACT", "TG_OP_GATED_ATTN", "TG_OP_PREFILL", "TG_OP_DECODE",
-    "TG_OP_GATED_ATTN_BWD",
+    "TG_OP_GATED_ATTN_BWD", "GdnLayer", "tg_gated_deltanet", "tg_gated_deltanet_workspace_size",
 ]

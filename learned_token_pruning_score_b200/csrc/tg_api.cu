@@ -159,6 +159,24 @@ struct AttnPlan {
 };
 
 // Backward of the standalone gated attention in fp32 (head_dim 64 or 128).
+struct GdnPlan {
+  GdnArgs a{};
+  size_t bytes = 0;
+  GdnPlan(void* ws, int64_t T, int hk, int hv, int dk, int dv) {
+    Arena ar(ws);
+    const int64_t tp = (T + 31) / 32 * 32;
+    a.t_pad = tp;
+    a.qn = static_cast<float*>(ar.carve(size_t(hk) * tp * dk * 4));
+    a.kn = static_cast<float*>(ar.carve(size_t(hk) * tp * dk * 4));
+    a.vb = static_cast<float*>(ar.carve(size_t(hv) * tp * dv * 4));
+    a.al = static_cast<float*>(ar.carve(size_t(hv) * tp * 4));
+    a.be = static_cast<float*>(ar.carve(size_t(hv) * tp * 4));
+    a.kq = static_cast<float*>(ar.carve(size_t(hk) * tp * 4));
+    a.o = static_cast<float*>(ar.carve(size_t(T) * hv * dv * 4));
+    bytes = ar.used;
+  }
+};
+
 struct AttnBwdF32Plan {
   float* q_rot = nullptr;   // [n, hq, dh]
   float* k_rot = nullptr;   // [n, hkv, dh]
@@ -1320,12 +1338,96 @@ tg_status tg_decode_step(const tg_model* model, const void* x, int64_t pos, int3
   return TG_OK;
 }
 
+// ---- Gated DeltaNet mixer
+namespace {
+tg_status validate_gdn_layer(const tg_gdn_layer* L) {
+  TG_CHECK(L != nullptr, TG_ERR_INVALID_ARG);
+  TG_CHECK(L->n_heads_k >= 1 && L->n_heads_v >= 1 && L->n_heads_v % L->n_heads_k == 0 &&
+               L->n_heads_v <= 4096,
+           TG_ERR_INVALID_ARG);
+  TG_CHECK(L->conv_width >= 1 && L->conv_width <= 8, TG_ERR_INVALID_ARG);
+  TG_CHECK(L->conv_w && L->A_log && L->dt_bias && L->norm_w, TG_ERR_INVALID_ARG);
+  TG_CHECK(std::isfinite(L->norm_eps) && L->norm_eps >= 0.f, TG_ERR_INVALID_ARG);
+  TG_CHECK(L->head_dim_k == 64 || L->head_dim_k == 128, TG_ERR_UNSUPPORTED);
+  TG_CHECK(L->head_dim_v >= 32 && L->head_dim_v <= 256 && L->head_dim_v % 32 == 0,
+           TG_ERR_UNSUPPORTED);
+  return TG_OK;
+}
+
+bool overlaps(const void* p, size_t pn, const void* q, size_t qn) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+  return a < b + qn && b < a + pn;
+}
+}  // namespace
+
+size_t tg_gated_deltanet_workspace_size(const tg_gdn_layer* L, int64_t T) {
+  if (validate_gdn_layer(L) != TG_OK || T < 0) return 0;
+  return GdnPlan(nullptr, T, L->n_heads_k, L->n_heads_v, L->head_dim_k, L->head_dim_v).bytes;
+}
+
+tg_status tg_gated_deltanet(const tg_gdn_layer* L, const void* qkv, const void* z, const void* a,
+                            const void* b, int64_t T, tg_dtype dtype, const void* conv_in,
+                            void* conv_out, const float* state_in, float* state_out, void* y,
+                            void* ws, size_t ws_bytes, tg_stream stream) {
+  const tg_status vs = validate_gdn_layer(L);
+  if (vs != TG_OK) return vs;
+  TG_CHECK(dtype == TG_BF16 || dtype == TG_F32, TG_ERR_UNSUPPORTED);
+  TG_CHECK(T >= 0 && T < (int64_t(1) << 31) - 64, TG_ERR_INVALID_ARG);
+  if (T > 0) TG_CHECK(qkv && z && a && b && y, TG_ERR_INVALID_ARG);
+  const int hk = L->n_heads_k, hv = L->n_heads_v, dk = L->head_dim_k, dv = L->head_dim_v;
+  const int W = L->conv_width;
+  const size_t C = size_t(2) * hk * dk + size_t(hv) * dv;
+  const size_t conv_bytes = size_t(W - 1) * C * elem_size(dtype);
+  const size_t state_bytes = size_t(hv) * dv * dk * 4;
+  if (conv_in && conv_out && W > 1)
+    TG_CHECK(!overlaps(conv_in, conv_bytes, conv_out, conv_bytes), TG_ERR_INVALID_ARG);
+  if (state_in && state_out && state_in != state_out)
+    TG_CHECK(!overlaps(state_in, state_bytes, state_out, state_bytes), TG_ERR_INVALID_ARG);
+  GdnPlan plan(nullptr, T, hk, hv, dk, dv);
+  TG_CHECK(ws != nullptr || plan.bytes == 0, TG_ERR_WORKSPACE);
+  TG_CHECK(ws_bytes >= plan.bytes, TG_ERR_WORKSPACE);
+  TG_CHECK(aligned16(ws), TG_ERR_INVALID_ARG);
+  plan = GdnPlan(ws, T, hk, hv, dk, dv);
+  GdnArgs g = plan.a;
+  g.qkv = qkv;
+  g.z = z;
+  g.a = a;
+  g.b = b;
+  g.T = T;
+  g.hk = hk;
+  g.hv = hv;
+  g.dk = dk;
+  g.dv = dv;
+  g.W = W;
+  g.conv_w = L->conv_w;
+  g.A_log = L->A_log;
+  g.dt_bias = L->dt_bias;
+  g.norm_w = L->norm_w;
+  g.eps = L->norm_eps;
+  g.conv_in = conv_in;
+  g.conv_out = conv_out;
+  g.state_in = state_in;
+  g.state_out = state_out;
+  g.y = y;
+  g.err = device_error_word();
+  const bool bf = dtype == TG_BF16;
+  const double e = double(elem_size(dtype)), tt = double(T);
+  const double prep_bytes = tt * (C * e + 2.0 * hv * e) + tt * 4.0 * (C + hv * 2.0 + hk);
+  const double recur_flops = tt * hv * 6.0 * dv * dk;
+  const double out_bytes = tt * hv * dv * (4.0 + 2.0 * e);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  TG_TRY(traced(TG_K_GDN_PREP, T, 0.0, prep_bytes, st, [&] { return launch_gdn(g, bf, 0, st); }));
+  TG_TRY(traced(TG_K_GDN_RECUR, T, recur_flops, 0.0, st, [&] { return launch_gdn(g, bf, 1, st); }));
+  TG_TRY(traced(TG_K_GDN_OUT, T, 0.0, out_bytes, st, [&] { return launch_gdn(g, bf, 2, st); }));
+  return TG_OK;
+}
+
 const char* tg_kernel_name(int32_t kernel) {
   static const char* names[TG_K_COUNT] = {
       "copy", "rmsnorm", "gemm_tc_store", "gemm_tc_residual", "gemm_tc_swiglu", "gemm_tc_score",
       "rope_prep", "attention_tc", "select", "compact", "gemm_f32", "attention_f32", "f32_helper",
       "gemm_tc_qkv", "rope_table", "decode_step", "attn_bwd_prep", "attn_bwd_dkdv",
-      "attn_bwd_dq", "attn_bwd_final"};
+      "attn_bwd_dq", "attn_bwd_final", "gdn_prep", "gdn_recur", "gdn_out"};
   return (kernel >= 0 && kernel < TG_K_COUNT) ? names[kernel] : "unknown";
 }
 

@@ -256,6 +256,40 @@ int decode_grid();
 int decode_splits(int hkv);
 cudaError_t launch_decode_step(const DecStepParams& p, cudaStream_t st);
 
+// ---- Gated DeltaNet mixer (k_gdn.cu)
+// One token sequence (the kept tokens of a hybrid model's gated prefill).
+// Workspace buffers are fp32, laid out for the recurrence's bulk copies; the
+// padded token count t_pad is a multiple of 32.
+struct GdnArgs {
+  const void* qkv;        // [T, 2 hk dk + hv dv] before the convolution
+  const void* z;          // [T, hv dv] output gate
+  const void* a;          // [T, hv] decay input
+  const void* b;          // [T, hv] write-strength input
+  int64_t T;
+  int64_t t_pad;
+  int hk, hv, dk, dv, W;
+  const float* conv_w;    // [C, W]
+  const float* A_log;     // [hv]
+  const float* dt_bias;   // [hv]
+  const float* norm_w;    // [dv]
+  float eps;
+  const void* conv_in;    // [W-1, C] or null (zeros)
+  void* conv_out;         // [W-1, C] or null
+  const float* state_in;  // [hv, dv, dk] or null (zeros)
+  float* state_out;       // [hv, dv, dk] or null; may equal state_in
+  void* y;                // [T, hv dv]
+  float* qn;              // [hk, t_pad, dk]  l2norm(q) / sqrt(dk)
+  float* kn;              // [hk, t_pad, dk]  l2norm(k)
+  float* vb;              // [hv, dv / 16, t_pad, 16]
+  float* al;              // [hv, t_pad] alpha
+  float* be;              // [hv, t_pad] beta
+  float* kq;              // [hk, t_pad] k . q
+  float* o;               // [T, hv, dv] S_t q_t
+  unsigned int* err;
+};
+// stage 0: prep (+ carried conv rows); 1: recurrence; 2: gated output norm.
+cudaError_t launch_gdn(const GdnArgs& a, bool bf16, int stage, cudaStream_t st);
+
 // ---- tensor maps (tg_tmap.cu)
 // 2-D bf16 tensor map, row-major [rows, cols] with row stride ld (elements),
 // box [box_rows, 64 cols], 128-byte swizzle. Returns false on failure.

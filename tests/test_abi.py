@@ -287,3 +287,46 @@ def test_prefill_batch_validation():
     assert call([0, 300, 429], [100, 129], ws_bytes=need - 1) == tg.TG_ERR_WORKSPACE
     bad = (ctypes.c_int64 * 2)(100, 300)
     assert tg._prefill_batch_ws(ctypes.byref(m), cu, bad, 2) == 0
+
+
+def _gdn_layer(hk=2, hv=4, dk=128, dv=128, W=4, eps=1e-6, ptrs=True):
+    p = BOGUS.value if ptrs else None
+    return tg.TgGdnLayer(hk, hv, dk, dv, W, p, p, p, p, eps)
+
+
+def test_gated_deltanet_validation():
+    f = tg._gdn
+    L = _gdn_layer()
+    need = tg._gdn_ws(ctypes.byref(L), 100)
+    assert need > 0
+    # the workspace holds the fp32 operands and the output before its norm
+    assert need >= 4 * 100 * (2 * 2 * 128 + 4 * 128 + 4 * 128)
+    assert tg._gdn_ws(ctypes.byref(L), 0) == 0 or tg._gdn_ws(ctypes.byref(L), 0) < need
+    ws = ctypes.c_void_p(1 << 20)
+
+    def call(layer=L, T=100, dtype=tg.TG_BF16, conv_in=None, conv_out=None, s_in=None, s_out=None,
+             ws_=ws, nbytes=need, ptr=BOGUS):
+        return f(ctypes.byref(layer) if layer is not None else None, ptr, ptr, ptr, ptr, T, dtype,
+                 conv_in, conv_out, s_in, s_out, ptr, ws_, nbytes, None)
+
+    assert call(layer=None) == tg.TG_ERR_INVALID_ARG
+    assert call(T=-1) == tg.TG_ERR_INVALID_ARG
+    assert call(ptr=None) == tg.TG_ERR_INVALID_ARG
+    assert call(dtype=7) == tg.TG_ERR_UNSUPPORTED
+    assert call(layer=_gdn_layer(hk=3, hv=4)) == tg.TG_ERR_INVALID_ARG
+    assert call(layer=_gdn_layer(W=0)) == tg.TG_ERR_INVALID_ARG
+    assert call(layer=_gdn_layer(W=9)) == tg.TG_ERR_INVALID_ARG
+    assert call(layer=_gdn_layer(eps=float("nan"))) == tg.TG_ERR_INVALID_ARG
+    assert call(layer=_gdn_layer(ptrs=False)) == tg.TG_ERR_INVALID_ARG
+    assert call(layer=_gdn_layer(dk=96)) == tg.TG_ERR_UNSUPPORTED
+    assert call(layer=_gdn_layer(dv=48)) == tg.TG_ERR_UNSUPPORTED
+    assert call(layer=_gdn_layer(dv=512)) == tg.TG_ERR_UNSUPPORTED
+    assert call(nbytes=need - 1) == tg.TG_ERR_WORKSPACE
+    assert call(ws_=None) == tg.TG_ERR_WORKSPACE
+    assert call(ws_=ctypes.c_void_p((1 << 20) + 8)) == tg.TG_ERR_INVALID_ARG
+    # overlapping carried state: conv rows always, S unless exactly in place
+    base = 1 << 24
+    assert call(conv_in=base, conv_out=base + 64) == tg.TG_ERR_INVALID_ARG
+    assert call(s_in=base, s_out=base + 4) == tg.TG_ERR_INVALID_ARG
+    names = [tg._kernel_name(i).decode() for i in (20, 21, 22, 23)]
+    assert names == ["gdn_prep", "gdn_recur", "gdn_out", "unknown"]
