@@ -661,6 +661,9 @@ def run_ours(args, rank, world, local_rank):
         bwd["frac_of_sustained_bf16"] = bwd["tflops_algorithmic"] / pk["bf16_sustained"]
         extras["attn_backward"] = {"workload": f"one gated attention layer, K={k} rows, "
                                                f"{w.hq}/{w.hkv} heads x {w.dh}", **bwd}
+        # a hybrid model's Gated DeltaNet layer above the gate runs its mixer
+        # on the kept tokens only
+        extras["gated_deltanet"] = gdn_bench(tg, torch, device, 20)
 
     # ---- CPU baseline: the oracle, rank 0 only, N = 1
     cpu = None
@@ -859,6 +862,72 @@ def attn_backward_bench(tg, torch, hq, hkv, dh, t, steps, device, bias=True, war
             "kernels": split, "heads": [hq, hkv], "bias": bias}
 
 
+# fp32 FMA rate of the CUDA cores, from the unit counts and the maximum SM
+# clock (148 SMs x 128 FP32 lanes x 2 flops x 1.965 GHz); no measured figure
+# exists for it, so fractions against it say "of nominal".
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def gdn_bench(tg, torch, device, steps, warmup=3):
+    """tg_gated_deltanet of a hybrid model's linear-attention layer over the
+    K kept tokens, next to the same mixer over all N tokens (the layer without
+    the gate): median ms per call (CUDA events, inputs resident), the
+    per-kernel split, and the recurrence's fp32 rate against the nominal
+    CUDA-core FMA rate (it runs on CUDA cores in fp32: no tensor-core path)."""
+    w = synth.GDN_LAYER_32K
+    rng = synth.rng_for(w.seed)
+    p = synth.gdn_params(w, rng)
+    layer = tg.GdnLayer(w.hk, w.hv, w.dk, w.dv, *(torch.from_numpy(p[k]).to(device)
+                                                  for k in ("conv_w", "A_log", "dt_bias",
+                                                            "norm_w")), eps=w.eps)
+    res = {"workload": f"{w.name}: {w.hk}/{w.hv} heads x {w.dk}/{w.dv}, conv {w.W}",
+           "dtype": "bf16 in/out, fp32 state"}
+    for name, T in (("gated", w.T), ("dense", w.n)):
+        g = torch.Generator(device=device).manual_seed(11)
+        C = 2 * w.hk * w.dk + w.hv * w.dv
+        x = [torch.randn(T, n, device=device, generator=g).to(torch.bfloat16)
+             for n in (C, w.hv * w.dv, w.hv, w.hv)]
+        y = torch.empty(T, w.hv * w.dv, dtype=torch.bfloat16, device=device)
+        s_out = torch.empty(w.hv, w.dv, w.dk, dtype=torch.float32, device=device)
+        ws = torch.empty(tg.tg_gated_deltanet_workspace_size(layer, T), dtype=torch.uint8,
+                         device=device)
+
+        def run():
+            tg.tg_gated_deltanet(layer, *x, y=y, state_out=s_out, want_state=False, ws=ws)
+
+        for _ in range(warmup):
+            run()
+        ms = []
+        for _ in range(steps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            run()
+            b.record()
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        tg.tg_trace_start()
+        for _ in range(steps):
+            run()
+        torch.cuda.synchronize()
+        split = {}
+        for r in tg.tg_trace_stop():
+            e = split.setdefault(r["kernel"], {"ms": 0.0, "flops": 0.0})
+            e["ms"] += r["ms"] / steps
+            e["flops"] += r["flops"] / steps
+        rec = split.get("gdn_recur", {"ms": 0.0, "flops": 0.0})
+        tf = rec["flops"] / (rec["ms"] / 1e3) / 1e12 if rec["ms"] else None
+        for e in split.values():
+            del e["flops"]
+        res[name] = {"tokens": T, "ms": statistics.median(ms),
+                     "tokens_per_s": T / (statistics.median(ms) / 1e3), "kernels": split,
+                     "recur_tflops_fp32": tf,
+                     "recur_frac_of_nominal_fp32": tf and tf / FP32_FMA_TFLOPS}
+        del x, y, ws
+    res["speedup_vs_dense"] = res["dense"]["ms"] / res["gated"]["ms"]
+    return res
+
+
 # ----------------------------------------------------------------- profiling cases
 
 
@@ -923,6 +992,22 @@ def run_case(args):
         assert tg.tg_device_error() == 0
         print(json.dumps({"case": "attn_bwd", "rows": t, "steps": args.steps, **res}))
         return 0
+    if args.case == "gdn":
+        # tg_gated_deltanet over `rows` tokens, the hybrid-layer mixer's shape
+        gw = synth.GDN_LAYER_32K
+        p = synth.gdn_params(gw, synth.rng_for(gw.seed))
+        layer = tg.GdnLayer(gw.hk, gw.hv, gw.dk, gw.dv,
+                            *(torch.from_numpy(p[k]).to(device)
+                              for k in ("conv_w", "A_log", "dt_bias", "norm_w")), eps=gw.eps)
+        C = 2 * gw.hk * gw.dk + gw.hv * gw.dv
+        x = [torch.randn(t, n, device=device).to(torch.bfloat16)
+             for n in (C, gw.hv * gw.dv, gw.hv, gw.hv)]
+        for _ in range(args.steps):
+            tg.tg_gated_deltanet(layer, *x, want_state=False)
+        torch.cuda.synchronize()
+        assert tg.tg_device_error() == 0
+        print(json.dumps({"case": "gdn", "rows": t, "reps": args.steps}))
+        return 0
     if args.case == "attn":
         q = torch.randn(t, w.hq, w.dh, device=device, dtype=torch.bfloat16)
         kk = torch.randn(t, w.hkv, w.dh, device=device, dtype=torch.bfloat16)
@@ -965,7 +1050,8 @@ def main():
     ap.add_argument("--quick", action="store_true", help="skip the other budgets / dense run")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--sweep", action="store_true")
-    ap.add_argument("--case", choices=["attn", "attn_bwd", "layer", "gemm", "decode"], default=None)
+    ap.add_argument("--case", choices=["attn", "attn_bwd", "layer", "gemm", "decode", "gdn"],
+                    default=None)
     ap.add_argument("--rows", type=int, default=32768)
     ap.add_argument("--no-bias", action="store_true",
                     help="attn case: plain causal attention (as the layers below the gate)")

@@ -418,7 +418,7 @@ typedef struct {
   int32_t n_heads_v;   /* hv, a multiple of hk                             */
   int32_t head_dim_k;  /* dk: 64 or 128                                    */
   int32_t head_dim_v;  /* dv: a multiple of 32, at most 256                */
-  int32_t conv_width;  /* W: 1..8                                          */
+  int32_t conv_width;  /* W: 1..4                                          */
   const float* conv_w; /* [C, W] with C = 2 hk dk + hv dv                  */
   const float* A_log;  /* [hv]                                             */
   const float* dt_bias;/* [hv]                                             */
@@ -486,9 +486,10 @@ typedef enum {
   TG_K_ATTN_BWD_DQ = 18,     /* backward: dQ and q . dq (tcgen05)                   */
   TG_K_ATTN_BWD_FINAL = 19,  /* backward: ds, dgain, dtau                           */
   TG_K_GDN_PREP = 20,        /* Gated DeltaNet: conv, norms, decay (+ conv rows)     */
-  TG_K_GDN_RECUR = 21,       /* Gated DeltaNet: the delta-rule recurrence            */
-  TG_K_GDN_OUT = 22,         /* Gated DeltaNet: gated output RMSNorm                 */
-  TG_K_COUNT = 23
+  TG_K_GDN_CHUNK = 21,       /* Gated DeltaNet: per-chunk solve matrices             */
+  TG_K_GDN_RECUR = 22,       /* Gated DeltaNet: the state across the chunks          */
+  TG_K_GDN_OUT = 23,         /* Gated DeltaNet: gated output RMSNorm                 */
+  TG_K_COUNT = 24
 } tg_kernel;
 
 typedef struct {

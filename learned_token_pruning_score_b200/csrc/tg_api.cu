@@ -169,9 +169,11 @@ struct GdnPlan {
     a.qn = static_cast<float*>(ar.carve(size_t(hk) * tp * dk * 4));
     a.kn = static_cast<float*>(ar.carve(size_t(hk) * tp * dk * 4));
     a.vb = static_cast<float*>(ar.carve(size_t(hv) * tp * dv * 4));
-    a.al = static_cast<float*>(ar.carve(size_t(hv) * tp * 4));
+    a.gl = static_cast<float*>(ar.carve(size_t(hv) * tp * 4));
     a.be = static_cast<float*>(ar.carve(size_t(hv) * tp * 4));
-    a.kq = static_cast<float*>(ar.carve(size_t(hk) * tp * 4));
+    a.eg = static_cast<float*>(ar.carve(size_t(hv) * tp * 4));
+    a.tt = static_cast<float*>(ar.carve(size_t(hv) * tp * 36 * 4));
+    a.mm = static_cast<float*>(ar.carve(size_t(hv) * tp * 36 * 4));
     a.o = static_cast<float*>(ar.carve(size_t(T) * hv * dv * 4));
     bytes = ar.used;
   }
@@ -1345,7 +1347,7 @@ tg_status validate_gdn_layer(const tg_gdn_layer* L) {
   TG_CHECK(L->n_heads_k >= 1 && L->n_heads_v >= 1 && L->n_heads_v % L->n_heads_k == 0 &&
                L->n_heads_v <= 4096,
            TG_ERR_INVALID_ARG);
-  TG_CHECK(L->conv_width >= 1 && L->conv_width <= 8, TG_ERR_INVALID_ARG);
+  TG_CHECK(L->conv_width >= 1 && L->conv_width <= 4, TG_ERR_INVALID_ARG);
   TG_CHECK(L->conv_w && L->A_log && L->dt_bias && L->norm_w, TG_ERR_INVALID_ARG);
   TG_CHECK(std::isfinite(L->norm_eps) && L->norm_eps >= 0.f, TG_ERR_INVALID_ARG);
   TG_CHECK(L->head_dim_k == 64 || L->head_dim_k == 128, TG_ERR_UNSUPPORTED);
@@ -1412,13 +1414,15 @@ tg_status tg_gated_deltanet(const tg_gdn_layer* L, const void* qkv, const void* 
   g.err = device_error_word();
   const bool bf = dtype == TG_BF16;
   const double e = double(elem_size(dtype)), tt = double(T);
-  const double prep_bytes = tt * (C * e + 2.0 * hv * e) + tt * 4.0 * (C + hv * 2.0 + hk);
+  const double prep_bytes = tt * (C * e + 2.0 * hv * e) + tt * 4.0 * (C + hv * 2.0);
+  const double chunk_flops = tt * hv * 2.0 * 32.0 * dk;  // the two Gram products (full square)
   const double recur_flops = tt * hv * 6.0 * dv * dk;
   const double out_bytes = tt * hv * dv * (4.0 + 2.0 * e);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   TG_TRY(traced(TG_K_GDN_PREP, T, 0.0, prep_bytes, st, [&] { return launch_gdn(g, bf, 0, st); }));
-  TG_TRY(traced(TG_K_GDN_RECUR, T, recur_flops, 0.0, st, [&] { return launch_gdn(g, bf, 1, st); }));
-  TG_TRY(traced(TG_K_GDN_OUT, T, 0.0, out_bytes, st, [&] { return launch_gdn(g, bf, 2, st); }));
+  TG_TRY(traced(TG_K_GDN_CHUNK, T, chunk_flops, 0.0, st, [&] { return launch_gdn(g, bf, 1, st); }));
+  TG_TRY(traced(TG_K_GDN_RECUR, T, recur_flops, 0.0, st, [&] { return launch_gdn(g, bf, 2, st); }));
+  TG_TRY(traced(TG_K_GDN_OUT, T, 0.0, out_bytes, st, [&] { return launch_gdn(g, bf, 3, st); }));
   return TG_OK;
 }
 
@@ -1427,7 +1431,7 @@ const char* tg_kernel_name(int32_t kernel) {
       "copy", "rmsnorm", "gemm_tc_store", "gemm_tc_residual", "gemm_tc_swiglu", "gemm_tc_score",
       "rope_prep", "attention_tc", "select", "compact", "gemm_f32", "attention_f32", "f32_helper",
       "gemm_tc_qkv", "rope_table", "decode_step", "attn_bwd_prep", "attn_bwd_dkdv",
-      "attn_bwd_dq", "attn_bwd_final", "gdn_prep", "gdn_recur", "gdn_out"};
+      "attn_bwd_dq", "attn_bwd_final", "gdn_prep", "gdn_chunk", "gdn_recur", "gdn_out"};
   return (kernel >= 0 && kernel < TG_K_COUNT) ? names[kernel] : "unknown";
 }
 

@@ -281,13 +281,16 @@ struct GdnArgs {
   float* qn;              // [hk, t_pad, dk]  l2norm(q) / sqrt(dk)
   float* kn;              // [hk, t_pad, dk]  l2norm(k)
   float* vb;              // [hv, dv / 16, t_pad, 16]
-  float* al;              // [hv, t_pad] alpha
+  float* gl;              // [hv, t_pad] log decay g
   float* be;              // [hv, t_pad] beta
-  float* kq;              // [hk, t_pad] k . q
+  float* eg;              // [hv, t_pad] exp of g summed from the chunk start
+  float* tt;              // [hv, t_pad / 32, 32, 36] per-chunk solve matrix
+  float* mm;              // [hv, t_pad / 32, 32, 36] per-chunk output matrix
   float* o;               // [T, hv, dv] S_t q_t
   unsigned int* err;
 };
-// stage 0: prep (+ carried conv rows); 1: recurrence; 2: gated output norm.
+// stage 0: prep (+ carried conv rows); 1: chunk matrices; 2: recurrence;
+// 3: gated output norm.
 cudaError_t launch_gdn(const GdnArgs& a, bool bf16, int stage, cudaStream_t st);
 
 // ---- tensor maps (tg_tmap.cu)

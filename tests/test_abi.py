@@ -300,7 +300,7 @@ def test_gated_deltanet_validation():
     need = tg._gdn_ws(ctypes.byref(L), 100)
     assert need > 0
     # the workspace holds the fp32 operands and the output before its norm
-    assert need >= 4 * 100 * (2 * 2 * 128 + 4 * 128 + 4 * 128)
+    assert need >= 4 * 100 * (2 * 2 * 128 + 4 * 128 + 4 * 128) + 2 * 4 * 4 * 128 * 36
     assert tg._gdn_ws(ctypes.byref(L), 0) == 0 or tg._gdn_ws(ctypes.byref(L), 0) < need
     ws = ctypes.c_void_p(1 << 20)
 
@@ -315,7 +315,7 @@ def test_gated_deltanet_validation():
     assert call(dtype=7) == tg.TG_ERR_UNSUPPORTED
     assert call(layer=_gdn_layer(hk=3, hv=4)) == tg.TG_ERR_INVALID_ARG
     assert call(layer=_gdn_layer(W=0)) == tg.TG_ERR_INVALID_ARG
-    assert call(layer=_gdn_layer(W=9)) == tg.TG_ERR_INVALID_ARG
+    assert call(layer=_gdn_layer(W=5)) == tg.TG_ERR_INVALID_ARG
     assert call(layer=_gdn_layer(eps=float("nan"))) == tg.TG_ERR_INVALID_ARG
     assert call(layer=_gdn_layer(ptrs=False)) == tg.TG_ERR_INVALID_ARG
     assert call(layer=_gdn_layer(dk=96)) == tg.TG_ERR_UNSUPPORTED
@@ -328,5 +328,5 @@ def test_gated_deltanet_validation():
     base = 1 << 24
     assert call(conv_in=base, conv_out=base + 64) == tg.TG_ERR_INVALID_ARG
     assert call(s_in=base, s_out=base + 4) == tg.TG_ERR_INVALID_ARG
-    names = [tg._kernel_name(i).decode() for i in (20, 21, 22, 23)]
-    assert names == ["gdn_prep", "gdn_recur", "gdn_out", "unknown"]
+    names = [tg._kernel_name(i).decode() for i in (20, 21, 22, 23, 24)]
+    assert names == ["gdn_prep", "gdn_chunk", "gdn_recur", "gdn_out", "unknown"]
