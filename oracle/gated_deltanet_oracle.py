@@ -43,6 +43,11 @@ design notes):
   G9  Rounding points: the inputs as given, the stored output y (dtype) and
       the returned states (conv state in the input dtype, S in fp32).
       Everything between is float64 here.
+  G10, G11  A Gated DeltaNet layer of a stack, and the gated forward of a
+      hybrid stack (below, with hybrid_prefill).
+
+G2-G8 agree with the Qwen3.5 Gated DeltaNet layer in the transformers
+library; the pins check the two against each other on the same weights.
 """
 
 from __future__ import annotations
@@ -218,3 +223,96 @@ def sample_mixer(qkv, z, a, b, p: MixerParams, hk: int, hv: int, dk: int, dv: in
         zz = np.asarray(z, dtype=F64).reshape(T, hv, dv)[:, h:h + 1]
         out.append(gated_rmsnorm(o, zz, p.norm_w, p.eps)[:, 0])
     return store(np.stack(out, axis=1))
+
+
+# ---------------------------------------------------------------------------
+# A hybrid stack with the gate (G10, G11)
+# ---------------------------------------------------------------------------
+#  G10 A Gated DeltaNet layer is r = x + W_out . mixer(W_in . RMSNorm(x)) (no
+#      projection biases; W_in's rows give qkv, then z, then a, then b),
+#      followed by the same SwiGLU FFN sub-layer as an attention layer.
+#      Rounding points as the attention layers': the normed rows, the
+#      projections, the mixer output and the residual are stored.
+#  G11 In a hybrid stack gated at layer L, layers below L run over all N
+#      tokens; layer L runs its token mixer (attention or Gated DeltaNet) over
+#      all N tokens and the scorer reads the post-mixer residual; the kept
+#      rows continue into layer L's FFN and every layer above. Attention
+#      layers above the gate use the token-gated logits; Gated DeltaNet
+#      layers above it run their mixer on the kept rows in order (G1).
+@dataclass
+class GdnStackLayer:
+    norm: np.ndarray                   # [d]
+    w_in: np.ndarray                   # [C + hv dv + 2 hv, d]
+    mixer: MixerParams
+    w_out: np.ndarray                  # [d, hv dv]
+    hk: int
+    hv: int
+    dk: int
+    dv: int
+    ffn_norm: Optional[np.ndarray] = None
+    w_gate_up: Optional[np.ndarray] = None
+    w_down: Optional[np.ndarray] = None
+
+
+def gdn_sublayer(x, lw: GdnStackLayer, eps: float, store=round_fp32):
+    """r = x + W_out . mixer(W_in . RMSNorm(x)) over the rows of x (one
+    sequence), and the mixer's final (conv rows, S)."""
+    from .tokengate_oracle import rmsnorm
+    x = np.asarray(x, dtype=F64)
+    T = x.shape[0]
+    C = 2 * lw.hk * lw.dk + lw.hv * lw.dv
+    y = store(rmsnorm(x, lw.norm, eps))
+    proj = store(y @ np.asarray(lw.w_in, dtype=F64).T)
+    qkv = proj[:, :C]
+    z = proj[:, C:C + lw.hv * lw.dv]
+    a = proj[:, C + lw.hv * lw.dv:C + lw.hv * lw.dv + lw.hv]
+    b = proj[:, C + lw.hv * lw.dv + lw.hv:]
+    res = gated_deltanet(qkv, z, a, b, lw.mixer, lw.hk, lw.hv, lw.dk, lw.dv, store=store)
+    r = store(x + res.y @ np.asarray(lw.w_out, dtype=F64).T)
+    assert r.shape == (T, x.shape[1])
+    return r, (res.conv_state, res.S)
+
+
+def hybrid_prefill(x, protect, k: int, m, gate_layer: int, store=round_fp32, kept_idx=None):
+    """The gated forward of a hybrid stack (G11). m is a tokengate_oracle
+    Model whose layers are attention Layers or GdnStackLayers. Returns a
+    PrefillResult; kv holds, per layer, the attention (k, v) or the Gated
+    DeltaNet (conv rows, S)."""
+    from .tokengate_oracle import (PrefillResult, attention_sublayer, compact, ffn_sublayer,
+                                   score, topk_select)
+
+    def mix(h, lw, pos, s, gated):
+        if isinstance(lw, GdnStackLayer):
+            return gdn_sublayer(h, lw, m.eps, store)
+        if gated:
+            return attention_sublayer(h, lw, m, pos, s, lw.gain, lw.tau, store)
+        return attention_sublayer(h, lw, m, pos, None, None, None, store)
+
+    x = store(np.asarray(x, dtype=F64))
+    n = x.shape[0]
+    pos = np.arange(n, dtype=np.int32)
+    kv = []
+    h = x
+    for li in range(max(gate_layer, 0)):
+        r, st = mix(h, m.layers[li], pos, None, False)
+        kv.append(st)
+        h = ffn_sublayer(r, m.layers[li], m, store)
+    if gate_layer >= 0:
+        r, st = mix(h, m.layers[gate_layer], pos, None, False)
+        kv.append(st)
+    else:
+        r = h
+    s = round_fp32(score(r, m.score_norm, m.eps, m.score_w1, m.score_b1, m.score_w2,
+                         m.score_b2, store))
+    idx = topk_select(s.astype(np.float32), protect, k) if kept_idx is None \
+        else np.asarray(kept_idx, dtype=np.int32)
+    x_k, pos_k, s_k = compact(r, idx, pos, s)
+    h = ffn_sublayer(x_k, m.layers[gate_layer], m, store) if gate_layer >= 0 else x_k
+    for li in range(gate_layer + 1, len(m.layers)):
+        r, st = mix(h, m.layers[li], pos_k, s_k, True)
+        kv.append(st)
+        h = ffn_sublayer(r, m.layers[li], m, store)
+    from .tokengate_oracle import rmsnorm
+    out = h if m.final_norm is None else store(rmsnorm(h, m.final_norm, m.eps))
+    return PrefillResult(out=out, kept_idx=idx, scores=s.astype(np.float32), kv=kv,
+                         gate_residual=r if gate_layer < 0 else None)

@@ -245,3 +245,150 @@ def test_degenerate_lengths(T):
     if T == 0:
         np.testing.assert_array_equal(r.conv_state, prev)
         np.testing.assert_allclose(r.S, S0, rtol=1e-7)
+
+
+def test_mixer_matches_the_qwen3_5_layer_in_transformers():
+    # The pages' hybrid model is Qwen3.5; transformers ships its Gated DeltaNet
+    # layer, whose portable path (no fused kernels installed) solves the
+    # recurrence in 64-token chunks in fp32. The same weights through the
+    # oracle's token-by-token recurrence must agree to fp32 rounding. This
+    # checks the readings G2-G8 (channel order, conv orientation, the L2-norm
+    # eps and q scale, the decay and strength formulas, the value-to-key head
+    # map and the gated norm) against the model's own code.
+    mq = pytest.importorskip("transformers.models.qwen3_5.modeling_qwen3_5")
+    from transformers.models.qwen3_5.configuration_qwen3_5 import Qwen3_5TextConfig
+    if mq.is_fast_path_available:
+        pytest.skip("fused kernels installed: the portable path is not the one that runs")
+    d, hk, hv, dk, dv, W, T = 48, 2, 4, 16, 8, 4, 70
+    cfg = Qwen3_5TextConfig(hidden_size=d, linear_num_key_heads=hk, linear_num_value_heads=hv,
+                            linear_key_head_dim=dk, linear_value_head_dim=dv,
+                            linear_conv_kernel_dim=W, rms_norm_eps=1e-6, hidden_act="silu",
+                            num_hidden_layers=1)
+    torch.manual_seed(0)
+    layer = mq.Qwen3_5GatedDeltaNet(cfg, layer_idx=0).double().eval()
+    with torch.no_grad():
+        for p_ in layer.parameters():
+            p_.copy_(torch.randn_like(p_) * 0.3)
+        layer.A_log.copy_(torch.log(torch.rand(hv, dtype=torch.float64) * 15 + 1))
+        layer.dt_bias.copy_(torch.randn(hv, dtype=torch.float64) - 2)
+        layer.norm.weight.copy_(1 + 0.1 * torch.randn(dv, dtype=torch.float64))
+    x = torch.randn(1, T, d, dtype=torch.float64)
+    with torch.no_grad():
+        want = layer(x)[0].numpy()
+    npw = lambda m: m.weight.detach().numpy()
+    xs = x[0].numpy()
+    p = gdn.MixerParams(conv_w=layer.conv1d.weight.detach().numpy()[:, 0, :],
+                        A_log=layer.A_log.detach().numpy(), dt_bias=layer.dt_bias.detach().numpy(),
+                        norm_w=layer.norm.weight.detach().numpy(), eps=1e-6)
+    r = gdn.gated_deltanet(xs @ npw(layer.in_proj_qkv).T, xs @ npw(layer.in_proj_z).T,
+                           xs @ npw(layer.in_proj_a).T, xs @ npw(layer.in_proj_b).T, p,
+                           hk, hv, dk, dv, store=lambda v: np.asarray(v, dtype=np.float64))
+    got = r.y @ npw(layer.out_proj).T
+    scale = np.abs(want).max()
+    np.testing.assert_allclose(got, want, rtol=1e-4, atol=1e-5 * scale)
+
+
+# ---------------------------------------------------------------- hybrid stacks
+def _gdn_stack_layer(rng, d, hk=1, hv=2, dk=8, dv=8, W=4, inter=32):
+    C = 2 * hk * dk + hv * dv
+    return gdn.GdnStackLayer(
+        norm=rng.uniform(0.5, 1.5, d), w_in=rng.standard_normal((C + hv * dv + 2 * hv, d)) * 0.2,
+        mixer=gdn.MixerParams(conv_w=rng.uniform(-0.5, 0.5, (C, W)),
+                              A_log=np.log(rng.uniform(1, 16, hv)),
+                              dt_bias=rng.uniform(-4, -1, hv), norm_w=rng.uniform(0.5, 1.5, dv)),
+        w_out=rng.standard_normal((d, hv * dv)) * 0.2, hk=hk, hv=hv, dk=dk, dv=dv,
+        ffn_norm=rng.uniform(0.5, 1.5, d), w_gate_up=rng.standard_normal((2 * inter, d)) * 0.1,
+        w_down=rng.standard_normal((d, inter)) * 0.1)
+
+
+def _hybrid_model(seed, kinds, d=64):
+    from tests.test_oracle_pins import _tiny_model
+    m = _tiny_model(seed, True, n_layers=len(kinds), d=d)
+    rng = np.random.default_rng(seed + 1000)
+    for i, kind in enumerate(kinds):
+        if kind == "gdn":
+            m.layers[i] = _gdn_stack_layer(rng, d)
+        else:
+            m.layers[i].gain = rng.uniform(0, 2, m.n_heads_q)
+            m.layers[i].tau = rng.uniform(0.5, 1.5, m.n_heads_q)
+    return m
+
+
+def test_hybrid_with_attention_layers_only_is_the_gated_prefill():
+    from oracle import tokengate_oracle as ref
+    m = _hybrid_model(50, ["attn", "attn", "attn"])
+    x = RNG.standard_normal((40, m.d_model))
+    prot = np.zeros(40, dtype=np.uint8)
+    prot[-3:] = 1
+    for gate in (-1, 0, 1):
+        a = gdn.hybrid_prefill(x, prot, 17, m, gate, store=ref.round_bf16)
+        b = ref.prefill(x, prot, 17, m, gate, store=ref.round_bf16)
+        np.testing.assert_array_equal(a.kept_idx, b.kept_idx)
+        np.testing.assert_array_equal(a.out, b.out)
+
+
+def test_gated_deltanet_layers_above_the_gate_see_only_the_kept_rows():
+    # Gate before layer 0 in a Gated DeltaNet-only stack: every layer runs on
+    # the kept rows, in order, with no positions or bias, so the result is
+    # the ungated stack applied to just those rows (reading G1).
+    from oracle import tokengate_oracle as ref
+    m = _hybrid_model(51, ["gdn", "gdn"])
+    x = RNG.standard_normal((30, m.d_model))
+    prot = np.zeros(30, dtype=np.uint8)
+    res = gdn.hybrid_prefill(x, prot, 12, m, -1)
+    h = ref.round_fp32(x)[res.kept_idx]  # the forward stores its input first
+    for lw in m.layers:
+        r, _ = gdn.gdn_sublayer(h, lw, m.eps)
+        h = ref.ffn_sublayer(r, lw, m, ref.round_fp32)
+    h = ref.round_fp32(ref.rmsnorm(h, m.final_norm, m.eps))
+    np.testing.assert_allclose(res.out, h, rtol=1e-12, atol=1e-12)
+    # and a pruned row's input changes nothing above the gate
+    pruned = np.setdiff1d(np.arange(30), res.kept_idx)[0]
+    x2 = x.copy()
+    x2[pruned] *= 3.0
+    res2 = gdn.hybrid_prefill(x2, prot, 12, m, -1, kept_idx=res.kept_idx)
+    np.testing.assert_array_equal(res2.out, res.out)
+
+
+def test_hybrid_keeping_every_token_without_bias_is_the_ungated_stack():
+    # K = N with gain 0 (and tau 1): the gate selects everything and adds
+    # nothing, so the gated hybrid forward equals the plain layer-by-layer
+    # forward, whichever layer (attention or Gated DeltaNet) holds the gate.
+    from oracle import tokengate_oracle as ref
+    m = _hybrid_model(52, ["gdn", "attn", "gdn", "attn"])
+    for lw in m.layers:
+        if not isinstance(lw, gdn.GdnStackLayer):
+            lw.gain = np.zeros(m.n_heads_q)
+            lw.tau = np.ones(m.n_heads_q)
+    n = 24
+    x = RNG.standard_normal((n, m.d_model))
+    pos = np.arange(n, dtype=np.int32)
+    h = ref.round_fp32(x)
+    for lw in m.layers:
+        if isinstance(lw, gdn.GdnStackLayer):
+            r, _ = gdn.gdn_sublayer(h, lw, m.eps)
+        else:
+            r, _ = ref.attention_sublayer(h, lw, m, pos, None, None, None, ref.round_fp32)
+        h = ref.ffn_sublayer(r, lw, m, ref.round_fp32)
+    want = ref.round_fp32(ref.rmsnorm(h, m.final_norm, m.eps))
+    for gate in (-1, 0, 1, 2):
+        res = gdn.hybrid_prefill(x, np.zeros(n, dtype=np.uint8), n, m, gate)
+        np.testing.assert_array_equal(res.kept_idx, np.arange(n))
+        np.testing.assert_allclose(res.out, want, rtol=1e-12, atol=1e-12)
+
+
+def test_gated_deltanet_sublayer_reads_its_projection_slices():
+    # Zero output-gate rows (z) make the mixer's output exactly zero, so the
+    # sub-layer is the identity; zeroing any other slice does not.
+    rng = np.random.default_rng(53)
+    d = 32
+    lw = _gdn_stack_layer(rng, d)
+    C = 2 * lw.hk * lw.dk + lw.hv * lw.dv
+    x = rng.standard_normal((9, d))
+    lw.w_in[C:C + lw.hv * lw.dv] = 0.0
+    r, _ = gdn.gdn_sublayer(x, lw, 1e-6, store=lambda v: np.asarray(v, dtype=np.float64))
+    np.testing.assert_array_equal(r, x)
+    lw2 = _gdn_stack_layer(np.random.default_rng(53), d)
+    lw2.w_in[C + lw2.hv * lw2.dv:] = 0.0  # a = b = 0 only
+    r2, _ = gdn.gdn_sublayer(x, lw2, 1e-6, store=lambda v: np.asarray(v, dtype=np.float64))
+    assert not np.allclose(r2, x)
