@@ -42,10 +42,10 @@
 namespace tg {
 namespace {
 
-constexpr int kCh = 32;      // tokens per chunk
-constexpr int kStages = 3;   // chunks in flight in the recurrence's ring
-constexpr int kRows = 16;    // state rows (value dims) per recurrence CTA
-constexpr int kLd = 36;      // row stride (floats) of the chunk matrices
+constexpr int kCh = kGdnChunk;  // tokens per chunk
+constexpr int kStages = 3;      // chunks in flight in the recurrence's ring
+constexpr int kRows = 16;       // state rows (value dims) per recurrence CTA
+constexpr int kLd = kGdnLd;     // row stride (floats) of the chunk matrices
 constexpr int kTb = 16;      // tokens per prep warp
 constexpr int kMaxW = 4;     // widest convolution
 constexpr float kL2Eps = 1e-6f;

@@ -164,7 +164,7 @@ struct GdnPlan {
   size_t bytes = 0;
   GdnPlan(void* ws, int64_t T, int hk, int hv, int dk, int dv) {
     Arena ar(ws);
-    const int64_t tp = (T + 31) / 32 * 32;
+    const int64_t tp = (T + kGdnChunk - 1) / kGdnChunk * kGdnChunk;
     a.t_pad = tp;
     a.qn = static_cast<float*>(ar.carve(size_t(hk) * tp * dk * 4));
     a.kn = static_cast<float*>(ar.carve(size_t(hk) * tp * dk * 4));
@@ -172,8 +172,8 @@ struct GdnPlan {
     a.gl = static_cast<float*>(ar.carve(size_t(hv) * tp * 4));
     a.be = static_cast<float*>(ar.carve(size_t(hv) * tp * 4));
     a.eg = static_cast<float*>(ar.carve(size_t(hv) * tp * 4));
-    a.tt = static_cast<float*>(ar.carve(size_t(hv) * tp * 36 * 4));
-    a.mm = static_cast<float*>(ar.carve(size_t(hv) * tp * 36 * 4));
+    a.tt = static_cast<float*>(ar.carve(size_t(hv) * tp * kGdnLd * 4));
+    a.mm = static_cast<float*>(ar.carve(size_t(hv) * tp * kGdnLd * 4));
     a.o = static_cast<float*>(ar.carve(size_t(T) * hv * dv * 4));
     bytes = ar.used;
   }
@@ -1415,7 +1415,7 @@ tg_status tg_gated_deltanet(const tg_gdn_layer* L, const void* qkv, const void* 
   const bool bf = dtype == TG_BF16;
   const double e = double(elem_size(dtype)), tt = double(T);
   const double prep_bytes = tt * (C * e + 2.0 * hv * e) + tt * 4.0 * (C + hv * 2.0);
-  const double chunk_flops = tt * hv * 2.0 * 32.0 * dk;  // the two Gram products (full square)
+  const double chunk_flops = tt * hv * 2.0 * kGdnChunk * dk;  // the two Gram products (full square)
   const double recur_flops = tt * hv * 6.0 * dv * dk;
   const double out_bytes = tt * hv * dv * (4.0 + 2.0 * e);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -259,7 +259,9 @@ cudaError_t launch_decode_step(const DecStepParams& p, cudaStream_t st);
 // ---- Gated DeltaNet mixer (k_gdn.cu)
 // One token sequence (the kept tokens of a hybrid model's gated prefill).
 // Workspace buffers are fp32, laid out for the recurrence's bulk copies; the
-// padded token count t_pad is a multiple of 32.
+// padded token count t_pad is a multiple of kGdnChunk.
+constexpr int kGdnChunk = 32;  // tokens per chunk of the recurrence
+constexpr int kGdnLd = 36;     // row stride (floats) of the per-chunk matrices
 struct GdnArgs {
   const void* qkv;        // [T, 2 hk dk + hv dv] before the convolution
   const void* z;          // [T, hv dv] output gate
@@ -284,8 +286,8 @@ struct GdnArgs {
   float* gl;              // [hv, t_pad] log decay g
   float* be;              // [hv, t_pad] beta
   float* eg;              // [hv, t_pad] exp of g summed from the chunk start
-  float* tt;              // [hv, t_pad / 32, 32, 36] per-chunk solve matrix
-  float* mm;              // [hv, t_pad / 32, 32, 36] per-chunk output matrix
+  float* tt;              // [hv, t_pad / kGdnChunk, kGdnChunk, kGdnLd] per-chunk solve matrix
+  float* mm;              // [hv, t_pad / kGdnChunk, kGdnChunk, kGdnLd] per-chunk output matrix
   float* o;               // [T, hv, dv] S_t q_t
   unsigned int* err;
 };
