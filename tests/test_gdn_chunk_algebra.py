@@ -15,8 +15,9 @@ leaving the chunk is e^gamma_31 s + sum_i (Tt r)_i k_i. A ragged tail is
 padded with zero tokens (k = q = v = 0, g = 0, beta = 0).
 
 This file checks that algebra, including the padding convention and the
-worst-conditioned solve (repeated keys at full strength). It runs on the CPU
-and shares no code with the CUDA path or the oracle.
+worst-conditioned solve (repeated keys at full strength). It runs on the
+CPU. The restatement shares no code with the CUDA path, and the oracle
+serves only as the reference it is compared with.
 """
 
 import numpy as np
