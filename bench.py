@@ -121,13 +121,17 @@ def kernel_source_hash(name: str) -> str:
     return h.hexdigest()[:12]
 
 
-def traffic_from_profiles(kernel: str, workload: str):
-    """dram bytes per launch of `kernel` from the committed ncu summary, or
-    None if absent or taken on another revision of the kernel source."""
+def traffic_from_profiles(kernel: str, source: str, workload: str):
+    """dram bytes per launch of `kernel` (a kernel family's launches in the
+    workload, e.g. attention_tc_gated) from the committed ncu summary, or
+    None if absent or taken on another revision of the source of the family
+    `source`."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
-    want = kernel_source_hash(kernel)
+    want = kernel_source_hash(source)
+    if not want:
+        return None
     with open(path) as fh:
         for line in fh:
             if line.startswith("#") or not line.strip():
@@ -294,25 +298,39 @@ def workload_flops(w, k):
 # ----------------------------------------------------------------- reference arm
 
 
+def config_of(w, k, args, world):
+    """The workload's config dict, the same for both arms."""
+    return {"workload": w.name, "n": w.n, "k": k, "layers": w.n_layers,
+            "gate_layer": w.gate_layer, "d_model": w.d, "heads": f"{w.hq}/{w.hkv}x{w.dh}",
+            "ffn": w.inter, "scorer": w.f, "protected": w.n_protect, "qk_norm": w.qk_norm,
+            "kv_cache_out": not args.no_kv, "parallelism": f"replicas x{world}",
+            "l2": "flushed between timed steps (256 MB write); inputs > L2"}
+
+
 def run_reference(args, rank, world):
+    """The oracle on the host cores. Each step times a bounded sample of the
+    workload (one gated upper layer over 1024 kept rows) and extrapolates the
+    whole workload's TTFT from its FLOP rate by algorithmic FLOPs: `value`
+    is that extrapolated tokens/s (mean over the steps), `ms_per_step` the
+    wall time each step's sample actually took."""
     if rank != 0:
         return 0
     w = WORKLOAD
-    per_step = []
+    per_step, step_ms = [], []
     desc = ""
     threads = 1
     for i in range(args.warmup + args.steps):
         rate, desc, threads, dt = oracle_sample(seconds=0.0, rows=1024)
         if i >= args.warmup:
             per_step.append(w.n / (workload_flops(w, HEADLINE_K) / rate))
+            step_ms.append(dt * 1e3)
     value = statistics.mean(per_step)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1000.0 * w.n / value, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": statistics.mean(step_ms),
+        "extrapolated_ttft_ms": 1000.0 * w.n / value, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "n": w.n, "k": HEADLINE_K, "layers": w.n_layers,
-                   "gate_layer": w.gate_layer, "d_model": w.d, "heads": f"{w.hq}/{w.hkv}x{w.dh}",
-                   "protected": w.n_protect},
+        "config": config_of(w, HEADLINE_K, args, world),
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": desc},
@@ -425,11 +443,13 @@ def run_ours(args, rank, world, local_rank):
         key = r["kernel"]
         if r["kernel"] == "attention_tc":
             key = "attention_tc_dense" if r["layer"] <= w.gate_layer else "attention_tc_gated"
-        e = per.setdefault(key, {"ms": 0.0, "flops": 0.0, "bytes": 0.0, "launches": 0})
+        e = per.setdefault(key, {"ms": 0.0, "flops": 0.0, "bytes": 0.0, "launches": 0,
+                                 "records": 0})
         e["ms"] += r["ms"]
         e["flops"] += r["flops"]
         e["bytes"] += r["bytes"]
         e["launches"] += LAUNCHES_PER_RECORD.get(r["kernel"], 1)
+        e["records"] += 1
     traced_ms = sum(e["ms"] for e in per.values())
     by_kernel = {}
     for key, e in sorted(per.items(), key=lambda kv: -kv[1]["ms"]):
@@ -440,32 +460,28 @@ def run_ours(args, rank, world, local_rank):
         else:
             d["gbs"] = e["bytes"] / (e["ms"] / 1e3) / 1e9
         by_kernel[key] = d
-    # dominant kernel = largest total device time among traced kernels
-    kern_tot = {}
-    for r in trace:
-        kern_tot.setdefault(r["kernel"], [0.0, 0.0, 0.0, 0])
-        kt = kern_tot[r["kernel"]]
-        kt[0] += r["ms"]
-        kt[1] += r["flops"]
-        kt[2] += r["bytes"]
-        kt[3] += 1
-    dom = max(kern_tot, key=lambda n: kern_tot[n][0])
-    dms, dfl, dby, dn = kern_tot[dom]
-    tensor_bound = dfl > 0
-    if tensor_bound:
-        achieved = dfl / (dms / 1e3) / 1e12
-        peak = pk["bf16_sustained"]
-        unit = "TFLOP/s"
-    else:
-        achieved = dby / (dms / 1e3) / 1e9
-        peak = pk["hbm"]
-        unit = "GB/s"
-    traffic = traffic_from_profiles(dom, w.name)
-    roofline = {"bound": "tensor" if tensor_bound else "hbm", "kernel": dom,
-                "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                "peak_source": f"{pk['source']} ({'bf16_tflops_sustained' if tensor_bound else 'hbm_gbs'})",
-                "traffic": traffic, "algorithmic_per_launch": (dfl if tensor_bound else dby) / dn,
-                "launches": dn}
+    # roofline of every traced kernel (the attention split into the dense
+    # launches below the gate and the gated ones above it); the dominant one
+    # (largest device time per step) is the line's `roofline`. Each launch
+    # lasts at most a few ms inside a ~24 ms step, so the denominators are
+    # the measured burst figures (bf16_tflops, hbm_gbs).
+    def roofline_of(key, e):
+        tensor = e["flops"] > 0
+        ach = (e["flops"] if tensor else e["bytes"]) / (e["ms"] / 1e3) / (1e12 if tensor else 1e9)
+        peak = pk["bf16"] if tensor else pk["hbm"]
+        n_l = max(1, e["records"])
+        base = "attention_tc" if key.startswith("attention_tc") else key
+        return {"bound": "tensor" if tensor else "hbm", "kernel": key, "achieved": ach,
+                "peak": peak, "unit": "TFLOP/s" if tensor else "GB/s", "frac": ach / peak,
+                "peak_source": f"{pk['source']} ({'bf16_tflops' if tensor else 'hbm_gbs'}, burst)",
+                "traffic": traffic_from_profiles(key, base, w.name),
+                "algorithmic_per_launch": (e["flops"] if tensor else e["bytes"]) / n_l,
+                "launches": n_l, "ms_per_step": e["ms"] / args.steps}
+
+    rooflines = {key: roofline_of(key, e) for key, e in per.items()
+                 if e["ms"] > 0 and (e["flops"] > 0 or e["bytes"] > 0)}
+    dom = max(rooflines, key=lambda kk: rooflines[kk]["ms_per_step"])
+    roofline = rooflines[dom]
     att_g = per.get("attention_tc_gated", {})
     att_d = per.get("attention_tc_dense", {})
     sel = per.get("select", {"ms": 0, "bytes": 0})
@@ -549,7 +565,7 @@ def run_ours(args, rank, world, local_rank):
                 if rs:
                     tf = sum(r["flops"] for r in rs) / (sum(r["ms"] for r in rs) / 1e3) / 1e12
                     att[f"attn_{name}_tflops"] = tf
-                    att[f"attn_{name}_frac_of_sustained_peak"] = tf / pk["bf16_sustained"]
+                    att[f"attn_{name}_frac_of_burst_peak"] = tf / pk["bf16"]
             return statistics.median(ms), mem, att
 
         del ws, kv
@@ -658,12 +674,24 @@ def run_ours(args, rank, world, local_rank):
         # backward of one gated attention layer over the K kept rows (the
         # gradient path to the scorer, gain and temperature)
         bwd = attn_backward_bench(tg, torch, w.hq, w.hkv, w.dh, k, 20, device)
-        bwd["frac_of_sustained_bf16"] = bwd["tflops_algorithmic"] / pk["bf16_sustained"]
+        bwd["frac_of_burst_bf16"] = bwd["tflops_algorithmic"] / pk["bf16"]
         extras["attn_backward"] = {"workload": f"one gated attention layer, K={k} rows, "
                                                f"{w.hq}/{w.hkv} heads x {w.dh}", **bwd}
         # a hybrid model's Gated DeltaNet layer above the gate runs its mixer
         # on the kept tokens only
         extras["gated_deltanet"] = gdn_bench(tg, torch, device, 20)
+        # the gated-attention kernel alone at each budget, with and without
+        # the gate bias
+        extras["attention_budgets"] = attention_budget_bench(
+            tg, torch, w, device, flush, pk, synth.PREFILL_32K_BUDGETS)
+        # the Qwen3-1.7B single gated layer at N=16384, K=2048 (per stage)
+        extras["layer_16k"] = single_layer_bench(tg, torch, synth.QWEN_LAYER_16K, device,
+                                                 flush, pk)
+        # select + compact over the sweep points
+        extras["select_compact_sweep"] = sweep_bench(tg, torch, device, flush, pk)
+        # the long-context gated sub-layer: N=131072 -> K=4096
+        extras["long_context_128k"] = single_layer_bench(tg, torch, synth.LONG_128K, device,
+                                                         flush, pk, reps=5)
 
     # ---- CPU baseline: the oracle, rank 0 only, N = 1
     cpu = None
@@ -679,13 +707,7 @@ def run_ours(args, rank, world, local_rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded random weights and N(0,1) hidden states)",
-            "config": {"workload": w.name, "n": w.n, "k": k, "layers": w.n_layers,
-                       "gate_layer": w.gate_layer, "d_model": w.d,
-                       "heads": f"{w.hq}/{w.hkv}x{w.dh}", "ffn": w.inter, "scorer": w.f,
-                       "protected": w.n_protect, "qk_norm": w.qk_norm,
-                       "kv_cache_out": not args.no_kv,
-                       "parallelism": f"replicas x{world}",
-                       "l2": "flushed between timed steps (256 MB write); inputs > L2"},
+            "config": config_of(w, k, args, world),
             "ttft_ms": ms_per_step,
             "traced_ms_per_step": traced_ms / args.steps,
             "tflop_per_step": workload_flops(w, k) / 1e12,
@@ -693,8 +715,9 @@ def run_ours(args, rank, world, local_rank):
             "roofline": roofline,
             "attn_gated_tflops": att_g and att_g["flops"] / (att_g["ms"] / 1e3) / 1e12,
             "attn_dense_tflops": att_d and att_d["flops"] / (att_d["ms"] / 1e3) / 1e12,
-            "attn_gated_frac_of_peak": att_g and
-            att_g["flops"] / (att_g["ms"] / 1e3) / 1e12 / pk["bf16_sustained"],
+            "attn_gated_frac_of_burst_peak": att_g and
+            att_g["flops"] / (att_g["ms"] / 1e3) / 1e12 / pk["bf16"],
+            "rooflines": rooflines,
             "select_compact_gbs": (sel["bytes"] + cmp_["bytes"]) /
             max(1e-9, (sel["ms"] + cmp_["ms"]) / 1e3) / 1e9,
             "by_kernel": by_kernel,
@@ -707,98 +730,234 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
-# ----------------------------------------------------------------- sweep mode
+# ----------------------------------------------------------------- the other workloads
 
 
-def run_sweep(args):
-    """Select+compact over the sweep points (HBM roofline) and the 128K
-    long-context gated layer; one JSON line per point."""
-    import torch
+def _events_median(torch, fn, reps, flush, stream):
+    """Median device ms of `reps` calls of fn (CUDA events on `stream`), L2
+    flushed before each call (outside the events), after one untimed call."""
+    fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for a, b in evs:
+        if flush is not None:
+            flush.zero_()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return statistics.median([a.elapsed_time(b) for a, b in evs])
 
-    import learned_token_pruning_score_b200 as tg
-    from oracle import tokengate_oracle as ref
 
-    device = torch.device("cuda", 0)
-    pk = peaks()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
-    for n, k in synth.sweep_points():
+def _traced(tg, torch, fn, reps, flush):
+    """Per-kernel totals of `reps` traced calls (each launch bracketed by its
+    own events), divided by reps: {kernel: {ms, flops, bytes, launches}}."""
+    tg.tg_trace_start(1 << 16)
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    out = {}
+    for r in tg.tg_trace_stop():
+        e = out.setdefault(r["kernel"], {"ms": 0.0, "flops": 0.0, "bytes": 0.0, "launches": 0})
+        e["ms"] += r["ms"] / reps
+        e["flops"] += r["flops"] / reps
+        e["bytes"] += r["bytes"] / reps
+        e["launches"] += LAUNCHES_PER_RECORD.get(r["kernel"], 1) / reps
+    return out
+
+
+def select_compact_bytes(n, k, d, elem=2):
+    """Algorithmic bytes of select + compact: scores (4N) and mask (N) read,
+    indices written (4K), kept rows read and written (2 K d elem), positions
+    and scores of the kept rows written (8K)."""
+    return 4 * n + n + 4 * k + 2 * k * d * elem + 8 * k
+
+
+def sweep_bench(tg, torch, device, flush, pk, reps=10, points=None):
+    """Select + compact over the sweep points (seeded fp32 N(0,1) scores with
+    exact-tie blocks and a few +-0 / +-inf, the last 128 protected, bf16 rows
+    of d 2048): median us, algorithmic GB/s and fraction of the measured HBM
+    copy bandwidth, L2 flushed before each call."""
+    res = []
+    x_all = torch.randn(max(synth.SWEEP_N), synth.SWEEP_D, device=device, dtype=torch.bfloat16)
+    for n, k in (points or synth.sweep_points()):
         rng = synth.rng_for(synth.SWEEP_SEED)
         s = torch.from_numpy(synth.sweep_scores(n, rng)).to(device)
         prot = torch.from_numpy(synth.protect_tail(n, synth.SWEEP_PROTECT)).to(device)
-        x = torch.randn(n, synth.SWEEP_D, device=device, dtype=torch.bfloat16)
+        x = x_all[:n]
         idx = torch.empty(k, dtype=torch.int32, device=device)
         xo = torch.empty(k, synth.SWEEP_D, device=device, dtype=torch.bfloat16)
         po = torch.empty(k, dtype=torch.int32, device=device)
         so = torch.empty(k, dtype=torch.float32, device=device)
         ws = torch.empty(tg.tg_workspace_size(tg.TG_OP_TOPK_SELECT, n=n), dtype=torch.uint8,
                          device=device)
+        stream = torch.cuda.current_stream(device)
 
         def once():
-            tg.tg_topk_select(s, prot, k, kept_idx=idx, ws=ws)
-            tg.tg_compact(x, idx, scores=s, x_out=xo, pos_out=po, scores_out=so)
+            tg.tg_topk_select(s, prot, k, kept_idx=idx, ws=ws, stream=stream)
+            tg.tg_compact(x, idx, scores=s, x_out=xo, pos_out=po, scores_out=so, stream=stream)
 
-        for _ in range(3):
+        for _ in range(2):
             once()
-        ms = []
-        for _ in range(args.steps):
-            flush.zero_()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record()
-            once()
-            b.record()
-            torch.cuda.synchronize()
-            ms.append(a.elapsed_time(b))
-        t = statistics.median(ms)
-        byt = ref.select_compact_bytes(n, k, synth.SWEEP_D)
+        t = _events_median(torch, once, reps, flush, stream)
+        sel_ms = _events_median(
+            torch, lambda: tg.tg_topk_select(s, prot, k, kept_idx=idx, ws=ws, stream=stream),
+            reps, flush, stream)
+        byt = select_compact_bytes(n, k, synth.SWEEP_D)
         gbs = byt / (t / 1e3) / 1e9
-        print(json.dumps({"sweep": "select+compact", "n": n, "k": k, "us": t * 1e3,
-                          "bytes": byt, "gbs": gbs, "frac_hbm": gbs / pk["hbm"]}), flush=True)
-        del s, prot, x, idx, xo, po, so, ws
+        res.append({"n": n, "k": k, "us": t * 1e3, "select_us": sel_ms * 1e3, "bytes": byt,
+                    "gbs": gbs, "frac_hbm": gbs / pk["hbm"]})
+        del s, prot, idx, xo, po, so, ws
+    del x_all
     torch.cuda.empty_cache()
+    return res
 
-    # Long-context gated attention layer: N=131072 -> K=4096, one attention-only
-    # layer (Qwen3-1.7B heads), scorer + select + compact + gated attention, vs
-    # the same layer dense over all N tokens.
-    w = synth.LONG_128K
+
+STAGE_OF = {"rmsnorm": "rmsnorm", "gemm_tc_score": "scorer", "select": "select",
+            "compact": "compact", "rope_table": "tables", "gemm_tc_qkv": "qkv_proj",
+            "attention_tc": "attention", "gemm_tc_residual": "o_proj+down_proj",
+            "gemm_tc_swiglu": "gate_up_proj", "copy": "copy"}
+
+
+def single_layer_bench(tg, torch, w, device, flush, pk, reps=10, dense_too=True):
+    """One gated layer gated before it (tg_prefill, gate_layer -1): scorer over
+    the N input rows, select, compact, then the layer over the K kept rows.
+    Reports the step's median ms, per-stage ms from a traced run, the
+    attention's TFLOP/s, the scorer's GB/s (its algorithmic bytes: the N rows
+    read once, the weights, the scores written), and the same layer dense
+    over all N rows (no gate bias)."""
     model = build_model(tg, torch, w, device)
     x = synth.torch_hidden_states(w, seed=w.seed, device=str(device))
     prot = torch.zeros(w.n, dtype=torch.uint8, device=device)
     prot[w.n - w.n_protect:] = 1
+    stream = torch.cuda.current_stream(device)
 
-    def timed(kk, dense):
-        mdl = dense_model(tg, model) if dense else model
+    def measure(mdl, kk):
         o = torch.empty(kk, w.d, dtype=torch.bfloat16, device=device)
         ki = torch.empty(kk, dtype=torch.int32, device=device)
         wsz = torch.empty(mdl.workspace_size(w.n, kk, -1), dtype=torch.uint8, device=device)
-        run = lambda: tg.tg_prefill(mdl, x, prot, kk, -1, out=o, kept_idx=ki, ws=wsz)  # noqa: E731
-        run()
-        torch.cuda.synchronize()
-        ms = []
-        tg.tg_trace_start(4096)
-        for _ in range(max(2, args.steps // 3)):
-            flush.zero_()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record()
-            run()
-            b.record()
-            torch.cuda.synchronize()
-            ms.append(a.elapsed_time(b))
-        tr = tg.tg_trace_stop()
-        att = [r for r in tr if r["kernel"] == "attention_tc"]
-        att_tf = sum(r["flops"] for r in att) / (sum(r["ms"] for r in att) / 1e3) / 1e12
+        run = lambda: tg.tg_prefill(mdl, x, prot, kk, -1, out=o, kept_idx=ki, ws=wsz,  # noqa: E731
+                                    stream=stream)
+        ms = _events_median(torch, run, reps, flush, stream)
+        tr = _traced(tg, torch, run, reps, flush)
+        stages = {}
+        for kern, e in tr.items():
+            st_ = STAGE_OF.get(kern, kern)
+            stages[st_] = stages.get(st_, 0.0) + e["ms"]
+        att = tr.get("attention_tc")
+        r = {"ms": ms, "stages_ms": stages, "launches": sum(e["launches"] for e in tr.values())}
+        if att:
+            tf = att["flops"] / (att["ms"] / 1e3) / 1e12
+            r.update(attention_tflops=tf, attention_frac_of_burst_bf16=tf / pk["bf16"])
         del o, ki, wsz
-        return statistics.median(ms), att_tf
+        return r, tr
 
-    g_ms, g_tf = timed(w.k, False)
-    d_ms, d_tf = timed(w.n, True)
-    print(json.dumps({"workload": w.name, "n": w.n, "k": w.k, "gated_ms": g_ms,
-                      "gated_attention_tflops": g_tf, "dense_ms": d_ms,
-                      "dense_attention_tflops": d_tf, "speedup_vs_dense": d_ms / g_ms,
-                      "attn_frac_of_sustained_peak": {"gated": g_tf / pk["bf16_sustained"],
-                                                      "dense": d_tf / pk["bf16_sustained"]}}),
+    g, tr = measure(model, w.k)
+    # the scorer: its RMSNorm (first rmsnorm launch of the call) and the
+    # scorer GEMM; algorithmic bytes = the rows read once + W1 + the scores
+    rows_b = w.n * w.d * 2
+    sc_bytes = rows_b + w.f * w.d * 2 + 4 * w.n
+    rms_ms = _traced_first(tg, torch, lambda: tg.tg_prefill(
+        model, x, prot, w.k, -1, stream=stream), "rmsnorm", flush)
+    sc_ms = tr.get("gemm_tc_score", {"ms": 0.0})["ms"]
+    g["scorer_ms"] = rms_ms + sc_ms
+    g["scorer_gbs"] = sc_bytes / ((rms_ms + sc_ms) / 1e3) / 1e9
+    g["scorer_frac_hbm"] = g["scorer_gbs"] / pk["hbm"]
+    sel = tr.get("select", {"ms": 0.0})["ms"] + tr.get("compact", {"ms": 0.0})["ms"]
+    g["select_compact_us"] = sel * 1e3
+    res = {"workload": w.name, "n": w.n, "k": w.k, "gated": g}
+    if dense_too:
+        d, _ = measure(dense_model(tg, model), w.n)
+        res["dense"] = d
+        res["speedup_vs_dense"] = d["ms"] / g["ms"]
+    del model, x, prot
+    torch.cuda.empty_cache()
+    return res
+
+
+def _traced_first(tg, torch, fn, kernel, flush, reps=5):
+    """Median device ms of the first launch of `kernel` in a traced call of
+    fn, over `reps` calls."""
+    ms = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        tg.tg_trace_start(1 << 12)
+        fn()
+        torch.cuda.synchronize()
+        first = [r["ms"] for r in tg.tg_trace_stop() if r["kernel"] == kernel]
+        ms.append(first[0] if first else 0.0)
+    return statistics.median(ms)
+
+
+def attention_budget_bench(tg, torch, w, device, flush, pk, budgets, reps=10):
+    """The gated-attention kernel alone at each budget: K kept rows of an
+    N-token prompt (ascending positions drawn from 0..N-1), Qwen3-1.7B heads,
+    with the gate bias (scores ~N(0, 2^2), gain U(0,2), tau U(0.5,1.5)) and
+    without it (plain causal attention over the same rows). Traced attention
+    kernel time (median launch), algorithmic TFLOP/s and fraction of the
+    measured burst bf16 peak."""
+    stream = torch.cuda.current_stream(device)
+    res = {}
+    for kk in budgets:
+        g = torch.Generator(device=device).manual_seed(100 + kk)
+        q = torch.randn(kk, w.hq, w.dh, device=device, generator=g).to(torch.bfloat16)
+        k_ = torch.randn(kk, w.hkv, w.dh, device=device, generator=g).to(torch.bfloat16)
+        v = torch.randn(kk, w.hkv, w.dh, device=device, generator=g).to(torch.bfloat16)
+        pos = torch.sort(torch.randperm(w.n, device=device, generator=g)[:kk]).values
+        pos = pos.to(torch.int32)
+        s = torch.randn(kk, device=device, generator=g) * 2
+        gain = torch.rand(w.hq, device=device, generator=g) * 2
+        tau = torch.rand(w.hq, device=device, generator=g) + 0.5
+        out = torch.empty_like(q)
+        ws = torch.empty(tg.tg_workspace_size(tg.TG_OP_GATED_ATTN, k=kk, n_heads_q=w.hq,
+                                              n_heads_kv=w.hkv, head_dim=w.dh),
+                         dtype=torch.uint8, device=device)
+        flops = 4.0 * w.dh * w.hq * kk * (kk + 1) / 2
+        r = {}
+        for name, args_ in (("bias", (s, gain, tau)), ("no_bias", (None, None, None))):
+            run = lambda a=args_: tg.tg_gated_attn_prefill(q, k_, v, pos, *a, out=out,  # noqa
+                                                           ws=ws, stream=stream)
+            run()
+            torch.cuda.synchronize()
+            tg.tg_trace_start(1 << 12)
+            for _ in range(reps):
+                flush.zero_()
+                run()
+            torch.cuda.synchronize()
+            ms = statistics.median([t["ms"] for t in tg.tg_trace_stop()
+                                    if t["kernel"] == "attention_tc"])
+            tf = flops / (ms / 1e3) / 1e12
+            r[name] = {"us": ms * 1e3, "tflops": tf, "frac_of_burst_bf16": tf / pk["bf16"]}
+        r["bias_cost"] = r["bias"]["us"] / r["no_bias"]["us"]
+        res[f"k{kk}"] = r
+        del q, k_, v, pos, s, out, ws
+    return res
+
+
+def run_sweep(args):
+    """The select+compact sweep, the 16K single layer and the 128K
+    long-context layer alone, one JSON line each."""
+    import torch
+
+    import learned_token_pruning_score_b200 as tg
+
+    device = torch.device("cuda", 0)
+    pk = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    for r in sweep_bench(tg, torch, device, flush, pk, reps=args.steps):
+        print(json.dumps({"sweep": "select+compact", **r}), flush=True)
+    print(json.dumps(single_layer_bench(tg, torch, synth.QWEN_LAYER_16K, device, flush, pk)),
           flush=True)
+    print(json.dumps(single_layer_bench(tg, torch, synth.LONG_128K, device, flush, pk, reps=5)),
+          flush=True)
+    print(json.dumps(attention_budget_bench(tg, torch, WORKLOAD, device, flush, pk,
+                                            synth.PREFILL_32K_BUDGETS)), flush=True)
+    assert tg.tg_device_error() == 0
+    return 0
 
 
 # ----------------------------------------------------------------- attention backward

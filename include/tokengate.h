@@ -126,9 +126,11 @@ tg_status tg_topk_select(const float* scores, const uint8_t* protect, int64_t n,
  * GPU loading the library holds until the process exits.
  *  - n must not exceed TG_SELECT_NOALLOC_MAX_N; larger n returns
  *    TG_ERR_UNSUPPORTED before any launch (use tg_topk_select instead).
- *  - The first call on a device looks up the array's device address (one
- *    runtime call, with that device current); make that first call before
- *    any stream capture.
+ *  - The first call in a CUDA context looks up the array's device address
+ *    (one runtime call, with the caller's device current) and caches it
+ *    under the context's unique id; make that first call before any stream
+ *    capture. After cudaDeviceReset, or in another context made current
+ *    through the driver API, the next call looks the address up again.
  *  - Every call on a device shares the one array, and each call clears what
  *    it needs. Calls whose kernels overlap on the GPU (e.g. on two streams)
  *    race on it: keep them ordered on one stream.
@@ -301,15 +303,25 @@ typedef struct {
  *   out [k, d] dtype: final-normed hidden states of the kept rows
  *   kept_idx [k] int32 (out, ascending); scores [n] fp32 (out) or NULL
  *   kv: HOST array of n_layers tg_kv, or NULL
- *   hidden: HOST array of n_layers device pointers, or NULL. hidden[l], when
- *     not NULL, receives layer l's output hidden states (after its FFN):
- *     [n, d] for layers below the gate, [k, d] (kept rows, ascending) for the
- *     gate layer and above. For inspection and per-layer checks; one copy
- *     per requested layer.
+ *   taps: HOST array of n_layers tg_layer_taps, or NULL. Each non-NULL
+ *     pointer of taps[l] receives a copy of one intermediate of layer l, for
+ *     inspection and per-layer checks (one device copy per requested tensor):
+ *       attn_out [rows, hq dh]: the attention output before the output
+ *         projection (rows = n at and below the gate, k above it);
+ *       resid [rows, d]: the residual stream after the attention sub-layer
+ *         (x + Wo . attn_out; rows as attn_out);
+ *       hidden [rows', d]: the layer's output after its FFN (rows' = n below
+ *         the gate, k for the gate layer and above; kept rows ascending).
  */
+typedef struct {
+  void* attn_out;
+  void* resid;
+  void* hidden;
+} tg_layer_taps;
+
 tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protect, int64_t n,
                      int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx, float* scores,
-                     const tg_kv* kv, void* const* hidden, void* ws, size_t ws_bytes,
+                     const tg_kv* kv, const tg_layer_taps* taps, void* ws, size_t ws_bytes,
                      tg_stream stream);
 
 /*
@@ -525,6 +537,26 @@ int tg_last_cuda_error(void);
  * This call synchronises the current device (a diagnostic, not for hot loops).
  */
 tg_status tg_device_error(uint32_t* word, int clear);
+
+/*
+ * tg_selftest_wait_timeout -- exercises the failure detection of the
+ * library's kernels without a fault. A kernel waits, with the same bounded
+ * wait the library's kernels use, for an event that never comes; after
+ * limit_ns it gives up, sets bit value 1 of the device error word (see
+ * tg_device_error) and returns, leaving the stream and the context usable.
+ * For tests and health checks; the pages have no counterpart.
+ *   mode 0: four warps wait on a shared-memory mbarrier (the wait of the
+ *           TMA / tensor-core pipelines) that nothing completes;
+ *   mode 1: the same, but the mbarrier completes: every wait succeeds;
+ *   mode 2: one CTA waits at the grid barrier of the cooperative decode
+ *           kernel, which no other CTA reaches.
+ *   limit_ns in [1000, 1e9]; result [4] int32 device (out), 16-byte aligned:
+ *   result[i] = 1 when wait i (warp i; mode 2: result[0]) completed, 0 when
+ *   it gave up. ws: mode 2 only, >= 16 bytes, 16-byte aligned (the barrier's
+ *   words, cleared by the call).
+ */
+tg_status tg_selftest_wait_timeout(int32_t mode, int64_t limit_ns, int32_t* result, void* ws,
+                                   size_t ws_bytes, tg_stream stream);
 
 /* Library version string. */
 const char* tg_version(void);

@@ -63,6 +63,10 @@ class TgKV(ctypes.Structure):
     _fields_ = [("k", _c_p), ("v", _c_p)]
 
 
+class TgLayerTaps(ctypes.Structure):
+    _fields_ = [("attn_out", _c_p), ("resid", _c_p), ("hidden", _c_p)]
+
+
 class TgGdnLayer(ctypes.Structure):
     _fields_ = [("n_heads_k", _c_i32), ("n_heads_v", _c_i32), ("head_dim_k", _c_i32),
                 ("head_dim_v", _c_i32), ("conv_width", _c_i32), ("conv_w", _c_p),
@@ -98,8 +102,8 @@ _attn_bwd = _sig("tg_gated_attn_backward", _ci, _c_p, _c_p, _c_p, _c_p, _c_p, _c
                  _c_i32, _c_i32, _c_i32, _c_f32, _ci, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p,
                  _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p)
 _prefill = _sig("tg_prefill", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64, _c_i64, _c_i32,
-                _c_p, _c_p, _c_p, ctypes.POINTER(TgKV), ctypes.POINTER(_c_p), _c_p, _c_sz,
-                _c_p)
+                _c_p, _c_p, _c_p, ctypes.POINTER(TgKV), ctypes.POINTER(TgLayerTaps), _c_p,
+                _c_sz, _c_p)
 _prefill_multi = _sig("tg_prefill_multi", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64,
                       ctypes.POINTER(_c_i64), _c_i32, _c_i32, ctypes.POINTER(_c_p),
                       ctypes.POINTER(_c_p), _c_p, _c_p, _c_sz, _c_p)
@@ -118,6 +122,7 @@ _status_string = _sig("tg_status_string", ctypes.c_char_p, _ci)
 _last_cuda_error = _sig("tg_last_cuda_error", _ci)
 _device_error = _sig("tg_device_error", _ci, ctypes.POINTER(ctypes.c_uint32), _ci)
 _version = _sig("tg_version", ctypes.c_char_p)
+_selftest_wait = _sig("tg_selftest_wait_timeout", _ci, _c_i32, _c_i64, _c_p, _c_p, _c_sz, _c_p)
 _trace_start = _sig("tg_trace_start", _ci, _c_i32)
 _trace_stop = _sig("tg_trace_stop", _c_i32, ctypes.POINTER(TgTraceRecord), _c_i32)
 _kernel_name = _sig("tg_kernel_name", ctypes.c_char_p, _c_i32)
@@ -189,6 +194,19 @@ def tg_device_error(clear: bool = False) -> int:
     w = ctypes.c_uint32(0)
     _check(_device_error(ctypes.byref(w), int(clear)), "tg_device_error")
     return int(w.value)
+
+
+def tg_selftest_wait_timeout(mode: int, limit_ns: int, device="cuda", stream=None) -> List[int]:
+    """Runs the failure-detection self-test (mode 0: an mbarrier wait that
+    never completes; 1: one that does; 2: the decode kernel's grid barrier,
+    never reached) and returns the per-wait results (1 = completed, 0 = gave
+    up after limit_ns). Synchronises the stream."""
+    res = torch.full((4,), -1, dtype=torch.int32, device=device)
+    ws = torch.zeros(16, dtype=torch.uint8, device=device)
+    _check(_selftest_wait(int(mode), int(limit_ns), _ptr(res), _ptr(ws), ws.numel(),
+                          _stream(stream, res.device)), "tg_selftest_wait_timeout")
+    torch.cuda.synchronize(res.device)
+    return res.cpu().tolist()
 
 
 def tg_trace_start(capacity: int = 65536) -> None:
@@ -473,13 +491,16 @@ def tg_decode_step(model: Model, x, pos: int, gate_layer: int, kv: Sequence, len
 
 
 def tg_prefill(model: Model, x, protect, k: int, gate_layer: int, out=None, kept_idx=None,
-               scores=None, kv: Optional[Sequence] = None, hidden: Optional[Sequence] = None,
+               scores=None, kv: Optional[Sequence] = None, taps: Optional[Sequence] = None,
                ws=None, stream=None):
     """Returns (out [k, d], kept_idx [k], scores [n] or None).
 
-    kv: per-layer (k_cache, v_cache) tensors or None entries; hidden:
-    per-layer output hidden-state tensors ([n, d] below the gate, [k, d] at
-    and above it) or None entries."""
+    kv: per-layer (k_cache, v_cache) tensors or None entries. taps: per-layer
+    dicts (or None) with any of the keys attn_out ([rows, hq*dh], the
+    attention output before the output projection), resid ([rows, d], the
+    residual stream after the attention sub-layer) and hidden (the layer's
+    output: [n, d] below the gate, [k, d] at and above it); rows = n at and
+    below the gate, k above it."""
     n, d = x.shape
     if out is None:
         out = torch.empty(k, d, dtype=x.dtype, device=x.device)
@@ -492,13 +513,16 @@ def tg_prefill(model: Model, x, protect, k: int, gate_layer: int, out=None, kept
         for i, pair in enumerate(kv):
             if pair is not None:
                 kv_c[i].k, kv_c[i].v = _ptr(pair[0]), _ptr(pair[1])
-    hid_c = None
-    if hidden is not None:
-        hid_c = (_c_p * len(model.layers))()
-        for i, t in enumerate(hidden):
-            hid_c[i] = _ptr(t)
+    taps_c = None
+    if taps is not None:
+        taps_c = (TgLayerTaps * len(model.layers))()
+        for i, t in enumerate(taps):
+            if t:
+                taps_c[i].attn_out = _ptr(t.get("attn_out"))
+                taps_c[i].resid = _ptr(t.get("resid"))
+                taps_c[i].hidden = _ptr(t.get("hidden"))
     _check(_prefill(ctypes.byref(model.c), _ptr(x), _ptr(protect), n, k, gate_layer, _ptr(out),
-                    _ptr(kept_idx), _ptr(scores), kv_c, hid_c, _ptr(ws), ws.numel(),
+                    _ptr(kept_idx), _ptr(scores), kv_c, taps_c, _ptr(ws), ws.numel(),
                     _stream(stream, x.device)), "tg_prefill")
     return out, kept_idx, scores
 
@@ -557,6 +581,7 @@ def tg_prefill_batch(model: Model, x, protect, lens: Sequence[int], ks: Sequence
 __all__ = [
     "tg_score", "tg_linear", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_gated_attn_forward", "tg_gated_attn_backward", "tg_prefill", "tg_prefill_multi", "tg_prefill_batch", "tg_decode_step",
     "tg_workspace_size", "tg_status_string", "tg_device_error", "tg_version", "Model",
+    "tg_selftest_wait_timeout",
     "TokenGateError", "LIB_PATH", "tg_trace_start", "tg_trace_stop", "TG_OK", "TG_ERR_INVALID_ARG", "TG_ERR_UNSUPPORTED",
     "TG_ERR_BUDGET", "TG_ERR_WORKSPACE", "TG_ERR_CUDA", "TG_F32", "TG_BF16", "TG_OP_SCORE",
     "TG_OP_TOPK_SELECT", "TG_OP_COMPACT", "TG_OP_GATED_ATTN", "TG_OP_PREFILL", "TG_OP_DECODE",

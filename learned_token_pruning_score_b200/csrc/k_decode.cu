@@ -98,6 +98,7 @@ struct GridBar {
   unsigned* abort;
   unsigned* err;
   unsigned target;
+  unsigned long long limit_ns = kWaitLimitNs;  // other values: the self-test only
 };
 
 __device__ __forceinline__ void bar_arrive(GridBar& b) {
@@ -117,7 +118,7 @@ __device__ __forceinline__ bool bar_wait(GridBar& b, int* s_ok) {
         if (ld_acquire_u32(b.count) >= b.target) break;
         if ((i & 63u) == 0) {
           if (ld_relaxed_u32(b.abort) != 0u) { ok = 0; break; }
-          if (global_ns() - t0 > kWaitLimitNs) {
+          if (global_ns() - t0 > b.limit_ns) {
             report_error(b.err, kErrWaitTimeout);
             atomicExch(b.abort, 1u);
             ok = 0;
@@ -673,7 +674,27 @@ cudaError_t launch_step(DecStepParams p, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
+// Self-test of the grid barrier's bounded wait: one CTA of consumers waits
+// for a barrier that no CTA arrives at (words[0] = 0 < target 1). After
+// limit_ns the wait gives up, records the timeout in err and sets the abort
+// word (words[1]); result[0] = 1 if bar_wait returned false, as it must.
+__global__ void __launch_bounds__(kConsumers, 1)
+    dec_selftest_gridbar(unsigned* words, unsigned* err, unsigned long long limit_ns,
+                         int* result) {
+  __shared__ int s_ok;
+  GridBar bar{words, words + 1, err, 1u};
+  bar.limit_ns = limit_ns;
+  const bool ok = bar_wait(bar, &s_ok);
+  if (threadIdx.x == 0) result[0] = ok ? 0 : 1;
+}
+
 }  // namespace
+
+cudaError_t launch_selftest_gridbar(unsigned* words, unsigned* err, unsigned long long limit_ns,
+                                    int* result, cudaStream_t st) {
+  dec_selftest_gridbar<<<1, kConsumers, 0, st>>>(words, err, limit_ns, result);
+  return cudaGetLastError();
+}
 
 int decode_grid() { return num_sms(); }
 

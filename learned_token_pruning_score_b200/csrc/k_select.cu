@@ -16,10 +16,14 @@
 // at the threshold key, then write the kept indices in index order: the tied
 // tokens taken are the lowest-index ones. Integer atomics only, so the
 // result is bit-reproducible.
+#include <cudaTypedefs.h>
+
 #include <mutex>
+#include <vector>
 
 #include "tg_device.cuh"
 #include "tg_internal.h"
+#include "tokengate.h"
 
 namespace tg {
 namespace {
@@ -386,36 +390,79 @@ cudaError_t run_select(const float* scores, const uint8_t* protect, int64_t n, i
 // Scratch of the allocation-free variant: one array per device, sized for
 // the largest n it accepts, shared by every call on that device.
 constexpr int64_t kNoAllocMaxN = int64_t(1) << 20;
+static_assert(kNoAllocMaxN == TG_SELECT_NOALLOC_MAX_N, "the documented limit is the built one");
 constexpr size_t kNoAllocBytes = kOffCounts + size_t(kNoAllocMaxN / kChunk) * 2 * 4;
 static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocBytes];
 
+// The array's device address, cached per CUDA context. A context is keyed by
+// its unique id (cuCtxGetId), which changes when cudaDeviceReset recreates a
+// device's primary context or when a caller makes another context current
+// through the driver API; either case makes a fresh lookup.
+struct ScratchAddr {
+  int dev;
+  unsigned long long ctx_id;
+  void* ptr;
+};
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[64] = {};
+std::vector<ScratchAddr> g_scratch_addr;
+constexpr size_t kMaxScratchAddr = 256;
+
+// Id of the current context, or 0 when none is current yet or the driver's
+// entry points cannot be fetched (then every call looks the address up).
+unsigned long long current_ctx_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 }  // namespace
 
 int64_t select_noalloc_max_n() { return kNoAllocMaxN; }
 
 // Host code cannot use g_select_scratch's name as a device address: the
-// symbol's device address is looked up once per device (with that device
-// current) and cached; kernels then get that pointer.
+// symbol's device address is looked up (cudaGetSymbolAddress, with the
+// caller's device current) on the first call in each context and cached;
+// kernels then get that pointer.
 cudaError_t launch_topk_select_noalloc(const float* scores, const uint8_t* protect, int64_t n,
                                        int64_t k, int32_t* kept_idx, cudaStream_t st) {
   if (n > kNoAllocMaxN) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
-      void* p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_select_scratch);
+    const unsigned long long id = current_ctx_id();
+    if (id != 0)
+      for (const ScratchAddr& a : g_scratch_addr)
+        if (a.dev == dev && a.ctx_id == id) scratch = a.ptr;
+    if (scratch == nullptr) {
+      e = cudaGetSymbolAddress(&scratch, g_select_scratch);
       if (e != cudaSuccess) return e;
-      g_scratch_ptr[dev] = p;
+      // the lookup makes the device's primary context current if none was
+      const unsigned long long id_now = current_ctx_id();
+      if (id_now != 0) {
+        if (g_scratch_addr.size() >= kMaxScratchAddr) g_scratch_addr.clear();
+        g_scratch_addr.push_back(ScratchAddr{dev, id_now, scratch});
+      }
     }
-    scratch = g_scratch_ptr[dev];
   }
   return launch_topk_select(scores, protect, n, k, kept_idx, scratch, st);
 }

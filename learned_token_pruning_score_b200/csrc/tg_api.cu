@@ -471,7 +471,8 @@ cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims
                                const PrefillPlan& P, void* h, int64_t rows, const int32_t* pos,
                                const float2* cs, const float* lsig, const void* kaug,
                                const float* gain, const float* tau, const tg_kv* kv,
-                               cudaStream_t st, const SegRows* segs = nullptr) {
+                               cudaStream_t st, const SegRows* segs = nullptr,
+                               const tg_layer_taps* taps = nullptr) {
   const tg_dtype dt = m.dtype;
   const size_t e = elem_size(dt);
   cudaError_t err = rmsnorm(h, lw.attn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
@@ -505,11 +506,17 @@ cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims
                         P.attn_o, st);
   }
   if (err != cudaSuccess) return err;
+  if (taps && taps->attn_out) {
+    err = copy_rows(taps->attn_out, P.attn_o, size_t(rows) * D.hq * D.dh * e, rows, st);
+    if (err != cudaSuccess) return err;
+  }
   GemmArgs g = gemm_args(P.attn_o, int64_t(D.hq) * D.dh, lw.wo, int64_t(D.hq) * D.dh, h, D.d, rows,
                          D.d, D.hq * D.dh, EPI_RESIDUAL);
   g.R = h;
   g.ldr = D.d;
-  return gemm(g, dt, st);
+  err = gemm(g, dt, st);
+  if (err != cudaSuccess || !taps || !taps->resid) return err;
+  return copy_rows(taps->resid, h, size_t(rows) * D.d * e, rows, st);
 }
 
 cudaError_t ffn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
@@ -923,8 +930,8 @@ Dims model_dims(const tg_model& m) {
 // Stage 1 of the gated forward: the layers below the gate and the gate
 // layer's attention over all n rows (in P.h), then the scores of every row.
 tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan& P, const void* x,
-                             int64_t n, int gate_layer, const tg_kv* kv, void* const* hidden,
-                             float* sc, cudaStream_t st) {
+                             int64_t n, int gate_layer, const tg_kv* kv,
+                             const tg_layer_taps* taps, float* sc, cudaStream_t st) {
   const size_t e = elem_size(m.dtype);
   TG_TRY(copy_rows(P.h, x, size_t(n) * D.d * e, n, st));
   const bool tables = m.dtype == TG_BF16 && D.dh == 128;
@@ -936,14 +943,17 @@ tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan
   for (int l = 0; l < gate_layer; ++l) {
     LayerTag tag(l);
     TG_TRY(attention_sublayer(m, m.layers[l], D, P, P.h, n, nullptr, P.cs_n, nullptr, nullptr,
-                              nullptr, nullptr, kv ? &kv[l] : nullptr, st));
+                              nullptr, nullptr, kv ? &kv[l] : nullptr, st, nullptr,
+                              taps ? &taps[l] : nullptr));
     TG_TRY(ffn_sublayer(m, m.layers[l], D, P, P.h, n, st));
-    if (hidden && hidden[l]) TG_TRY(copy_rows(hidden[l], P.h, size_t(n) * D.d * e, n, st));
+    if (taps && taps[l].hidden)
+      TG_TRY(copy_rows(taps[l].hidden, P.h, size_t(n) * D.d * e, n, st));
   }
   if (gate_layer >= 0) {
     LayerTag tag(gate_layer);
     TG_TRY(attention_sublayer(m, m.layers[gate_layer], D, P, P.h, n, nullptr, P.cs_n, nullptr,
-                              nullptr, nullptr, nullptr, kv ? &kv[gate_layer] : nullptr, st));
+                              nullptr, nullptr, nullptr, kv ? &kv[gate_layer] : nullptr, st,
+                              nullptr, taps ? &taps[gate_layer] : nullptr));
   }
   // score the post-attention residual
   TG_TRY(run_score(P.h, n, D.d, m.d_score, m.score_norm, m.norm_eps, m.score_w1, m.score_b1,
@@ -957,7 +967,7 @@ tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan
 tg_status prefill_above_gate(const tg_model& m, const Dims& D, const PrefillPlan& P,
                              const uint8_t* protect, int64_t n, int64_t k, int gate_layer,
                              const float* sc, void* out, int32_t* kept_idx, const tg_kv* kv,
-                             void* const* hidden, cudaStream_t st) {
+                             const tg_layer_taps* taps, cudaStream_t st) {
   const size_t e = elem_size(m.dtype);
   const bool tables = m.dtype == TG_BF16 && D.dh == 128;
   const double cs_bytes = 8.0 * (D.dh / 2);
@@ -975,16 +985,18 @@ tg_status prefill_above_gate(const tg_model& m, const Dims& D, const PrefillPlan
   if (gate_layer >= 0) {
     LayerTag tag(gate_layer);
     TG_TRY(ffn_sublayer(m, m.layers[gate_layer], D, P, P.hk, k, st));
-    if (hidden && hidden[gate_layer])
-      TG_TRY(copy_rows(hidden[gate_layer], P.hk, size_t(k) * D.d * e, k, st));
+    if (taps && taps[gate_layer].hidden)
+      TG_TRY(copy_rows(taps[gate_layer].hidden, P.hk, size_t(k) * D.d * e, k, st));
   }
   for (int l = gate_layer + 1; l < m.n_layers; ++l) {
     LayerTag tag(l);
     const tg_layer& L = m.layers[l];
     TG_TRY(attention_sublayer(m, L, D, P, P.hk, k, P.pos_k, P.cs_k, P.lsig_k, P.kaug_k, L.gain,
-                              L.tau, kv ? &kv[l] : nullptr, st));
+                              L.tau, kv ? &kv[l] : nullptr, st, nullptr,
+                              taps ? &taps[l] : nullptr));
     TG_TRY(ffn_sublayer(m, L, D, P, P.hk, k, st));
-    if (hidden && hidden[l]) TG_TRY(copy_rows(hidden[l], P.hk, size_t(k) * D.d * e, k, st));
+    if (taps && taps[l].hidden)
+      TG_TRY(copy_rows(taps[l].hidden, P.hk, size_t(k) * D.d * e, k, st));
   }
   if (m.final_norm)
     TG_TRY(rmsnorm(P.hk, m.final_norm, m.norm_eps, k, D.d, m.dtype, out, st));
@@ -1050,7 +1062,7 @@ extern "C" {
 
 tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protect, int64_t n,
                      int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx, float* scores,
-                     const tg_kv* kv, void* const* hidden, void* ws, size_t ws_bytes,
+                     const tg_kv* kv, const tg_layer_taps* taps, void* ws, size_t ws_bytes,
                      tg_stream stream) {
   const tg_status vs = validate_model(model, n, k, gate_layer);
   if (vs != TG_OK) return vs;
@@ -1063,9 +1075,9 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const Dims D = model_dims(m);
   float* sc = scores ? scores : P.scores;
-  const tg_status s1 = prefill_below_gate(m, D, P, x, n, gate_layer, kv, hidden, sc, st);
+  const tg_status s1 = prefill_below_gate(m, D, P, x, n, gate_layer, kv, taps, sc, st);
   if (s1 != TG_OK) return s1;
-  return prefill_above_gate(m, D, P, protect, n, k, gate_layer, sc, out, kept_idx, kv, hidden, st);
+  return prefill_above_gate(m, D, P, protect, n, k, gate_layer, sc, out, kept_idx, kv, taps, st);
 }
 
 tg_status tg_prefill_multi(const tg_model* model, const void* x, const uint8_t* protect,
@@ -1228,6 +1240,25 @@ tg_status tg_device_error(uint32_t* word, int clear) {
     const unsigned int z = 0;
     TG_TRY(cudaMemcpyToSymbol(g_tg_error_word, &z, sizeof(z)));
   }
+  return TG_OK;
+}
+
+tg_status tg_selftest_wait_timeout(int32_t mode, int64_t limit_ns, int32_t* result, void* ws,
+                                   size_t ws_bytes, tg_stream stream) {
+  TG_CHECK(mode >= 0 && mode <= 2 && result != nullptr, TG_ERR_INVALID_ARG);
+  TG_CHECK(limit_ns >= 1000 && limit_ns <= 1000000000, TG_ERR_INVALID_ARG);
+  TG_CHECK(aligned16(result), TG_ERR_INVALID_ARG);
+  if (mode == 2) TG_CHECK(ws != nullptr && ws_bytes >= 16 && aligned16(ws), TG_ERR_WORKSPACE);
+  unsigned int* err = device_error_word();
+  TG_CHECK(err != nullptr, TG_ERR_CUDA);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const auto lim = static_cast<unsigned long long>(limit_ns);
+  if (mode == 2) {
+    TG_TRY(cudaMemsetAsync(ws, 0, 16, st));
+    TG_TRY(launch_selftest_gridbar(static_cast<unsigned*>(ws), err, lim, result, st));
+    return TG_OK;
+  }
+  TG_TRY(launch_selftest_mbar(err, lim, mode == 1 ? 1 : 0, result, st));
   return TG_OK;
 }
 

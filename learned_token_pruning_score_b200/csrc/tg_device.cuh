@@ -99,13 +99,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase with the given parity of `bar` has completed.
 // Returns false (and records a timeout) when the limit is reached.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* err) {
+// (limit_ns other than kWaitLimitNs: the self-test of this path only.)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* err,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_addr(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(a, parity)) return true;
-    if ((i & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+    if ((i & 255u) == 0 && global_ns() - t0 > limit_ns) {
       report_error(err, kErrWaitTimeout);
       return false;
     }
@@ -115,8 +117,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
 // Warp-uniform bounded wait: every lane waits, and the warp proceeds only if
 // all lanes saw the phase complete (warp-collective tcgen05 loads/stores
 // follow, so the lanes must not diverge on a timeout).
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, unsigned int* err) {
-  const bool ok = mbar_wait(bar, parity, err);
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, unsigned int* err,
+                                               unsigned long long limit_ns = kWaitLimitNs) {
+  const bool ok = mbar_wait(bar, parity, err, limit_ns);
   return __all_sync(0xFFFFFFFFu, ok);
 }
 

@@ -256,6 +256,12 @@ int decode_grid();
 int decode_splits(int hkv);
 cudaError_t launch_decode_step(const DecStepParams& p, cudaStream_t st);
 
+// Self-tests of the bounded waits (tg_selftest_wait_timeout).
+cudaError_t launch_selftest_mbar(unsigned* err, unsigned long long limit_ns, int arrive,
+                                 int* result, cudaStream_t st);
+cudaError_t launch_selftest_gridbar(unsigned* words, unsigned* err, unsigned long long limit_ns,
+                                    int* result, cudaStream_t st);
+
 // ---- Gated DeltaNet mixer (k_gdn.cu)
 // One token sequence (the kept tokens of a hybrid model's gated prefill).
 // Workspace buffers are fp32, laid out for the recurrence's bulk copies; the

@@ -330,3 +330,12 @@ def test_gated_deltanet_validation():
     assert call(s_in=base, s_out=base + 4) == tg.TG_ERR_INVALID_ARG
     names = [tg._kernel_name(i).decode() for i in (20, 21, 22, 23, 24)]
     assert names == ["gdn_prep", "gdn_chunk", "gdn_recur", "gdn_out", "unknown"]
+
+
+def test_selftest_wait_validation():
+    f = tg._selftest_wait
+    assert f(3, 2_000_000, BOGUS, None, 0, None) == tg.TG_ERR_INVALID_ARG  # no such mode
+    assert f(0, 10, BOGUS, None, 0, None) == tg.TG_ERR_INVALID_ARG  # limit below 1 us
+    assert f(0, 2_000_000_000, BOGUS, None, 0, None) == tg.TG_ERR_INVALID_ARG  # above 1 s
+    assert f(0, 2_000_000, None, None, 0, None) == tg.TG_ERR_INVALID_ARG  # no result buffer
+    assert f(2, 2_000_000, BOGUS, None, 0, None) == tg.TG_ERR_WORKSPACE  # barrier words

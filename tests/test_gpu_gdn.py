@@ -55,10 +55,9 @@ def _setup(T, hk, hv, dk, dv, W, dtype, seed, carried=False):
 
 
 def _check_state(gpu, want):
-    g = host64(gpu)
-    bad = np.abs(g - want) > 1e-4 + 1e-3 * np.abs(want)
-    assert not bad.any(), f"state: {int(bad.sum())} of {bad.size} outside; max|d|=" \
-                          f"{np.abs(g - want).max():.3e}"
+    """The carried state is an fp32 output whatever the call's dtype: it is
+    held to the fp32 tolerance, |gpu - ref| <= 1e-4 + 1e-4 |ref|."""
+    assert_close(gpu, want, torch.float32, "state")
 
 
 @pytest.mark.parametrize("T", [1, 31, 32, 33, 200, 517])

@@ -1,19 +1,25 @@
 """GPU parity at the benchmark workloads' sizes.
 
 * 28-layer Qwen3-1.7B-shaped gated prefill (qk-norm, gate at layer 1),
-  checked per layer and teacher-forced (hidden states with the bulk form of
-  the tolerance, see tests/_helpers.assert_close_bulk): the oracle runs each layer on the
-  GPU's own output of the layer before (tg_prefill's per-layer hidden-state
-  outputs), so bf16 rounding differences cannot accumulate over 28 layers;
-  the kept set is checked bit-exactly on the GPU's scores.
+  checked per layer and teacher-forced at every tensor the library stores
+  between kernels. For each layer the oracle starts from the GPU's own input
+  of that layer and checks, in turn:
+    - the layer's k and v (its KV cache) from that input;
+    - the attention output (tg_prefill's attn_out tap) from the GPU's k, v;
+    - the post-attention residual (resid tap) from the GPU's attention output;
+    - at the gate layer, the scores from the GPU's residual;
+    - the layer's output (hidden tap) from the GPU's residual.
+  Each comparison thus covers one stage's arithmetic and its one rounding to
+  bf16, and every element is held to |gpu - ref| <= 2e-2 + 1e-2 |ref| with no
+  exceptions. The kept set is checked bit-exactly on the GPU's scores.
   - at a reduced N=4096, K=512 (every other shape unchanged): every row;
-  - at the full N=32768, K=4096: sampled rows, attention keys and values
-    taken from the GPU's KV cache of the layer (its rows at the sampled
-    tokens checked too).
+  - at the full N=32768 with K = 2048, 4096 and 8192, and the dense run
+    (K = N, no gate bias) the speedups are measured against: sampled rows,
+    attention keys and values taken from the GPU's KV cache of the layer.
 * long-context gated attention layer: N=131072 -> K=4096, in full.
 
 Weights are drawn on the device (seeded), so host and device see the same
-bf16 values. Tolerance: |gpu - ref| <= 2e-2 + 1e-2 |ref|.
+bf16 values.
 """
 
 from collections.abc import Sequence
@@ -24,7 +30,7 @@ import torch
 
 import synth
 from oracle import tokengate_oracle as ref
-from tests._helpers import assert_close, assert_close_bulk, boundary_flips, host64
+from tests._helpers import assert_close, boundary_flips, host64
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -62,8 +68,11 @@ class HostLayers(Sequence):
         return self.cache[1]
 
 
-def _models(w):
+def _models(w, dense=False):
     p = synth.torch_model_params(w, seed=w.seed, device="cuda")
+    if dense:  # the dense baseline: the same weights without the gate bias
+        p["layers"] = [{k: v for k, v in lp.items() if k not in ("gain", "tau")}
+                       for lp in p["layers"]]
     score = {k: p[k] for k in ("score_norm", "score_w1", "score_b1", "score_w2", "score_b2")}
     model = tg.Model(n_heads_q=w.hq, n_heads_kv=w.hkv, head_dim=w.dh, layers=p["layers"],
                      score=score, final_norm=p["final_norm"], eps=w.eps, rope_base=w.rope_base)
@@ -75,19 +84,28 @@ def _models(w):
     return model, om
 
 
-def _run_gpu(w, model, x, prot, with_hidden=False):
-    kv, hidden = [], []
+def _run_gpu(w, model, x, prot, with_taps=False):
+    kv, taps = [], []
     for li in range(w.n_layers):
         rows = w.n if li <= w.gate_layer else w.k
         kv.append((torch.empty(rows, w.hkv, w.dh, device="cuda", dtype=BF16),
                    torch.empty(rows, w.hkv, w.dh, device="cuda", dtype=BF16)))
         hrows = w.n if li < w.gate_layer else w.k
-        hidden.append(torch.empty(hrows, w.d, device="cuda", dtype=BF16))
+        taps.append({"attn_out": torch.empty(rows, w.hq * w.dh, device="cuda", dtype=BF16),
+                     "resid": torch.empty(rows, w.d, device="cuda", dtype=BF16),
+                     "hidden": torch.empty(hrows, w.d, device="cuda", dtype=BF16)})
     scores = torch.empty(w.n, device="cuda")
     out, kept, _ = tg.tg_prefill(model, x, torch.from_numpy(prot).cuda(), w.k, w.gate_layer,
-                                 scores=scores, kv=kv, hidden=hidden if with_hidden else None)
+                                 scores=scores, kv=kv, taps=taps if with_taps else None)
     torch.cuda.synchronize()
-    return out, kept.cpu().numpy(), scores.cpu().numpy(), kv, hidden
+    return out, kept.cpu().numpy(), scores.cpu().numpy(), kv, taps
+
+
+def _check_scores(r_gpu, om, scores_gpu, what):
+    s_ref = ref.round_fp32(ref.score(r_gpu, om.score_norm, om.eps, om.score_w1, om.score_b1,
+                                     om.score_w2, om.score_b2, rb))
+    assert_close(scores_gpu, s_ref, BF16, what)
+    return s_ref
 
 
 def test_prefill_28_layers_reduced_n_per_layer():
@@ -95,7 +113,7 @@ def test_prefill_28_layers_reduced_n_per_layer():
     model, om = _models(w)
     x = synth.torch_hidden_states(w, seed=w.seed + 1000, device="cuda")
     prot = synth.protect_tail(w.n, w.n_protect)
-    out, kept, scores, kv, hidden = _run_gpu(w, model, x, prot, with_hidden=True)
+    out, kept, scores, kv, taps = _run_gpu(w, model, x, prot, with_taps=True)
     assert np.array_equal(kept, ref.topk_select(scores, prot, w.k))
     pos_n = np.arange(w.n)
     s_k = scores[kept].astype(np.float64)
@@ -104,59 +122,70 @@ def test_prefill_28_layers_reduced_n_per_layer():
         lw = om.layers[li]
         dense = li <= w.gate_layer
         pos = pos_n if dense else kept
-        r, (k_o, v_o) = ref.attention_sublayer(h_in, lw, om, pos, None if dense else s_k,
-                                               None if dense else lw.gain,
-                                               None if dense else lw.tau, rb)
+        rows = pos.size
+        q, k_o, v_o = ref.project_qkv(h_in, lw, om, pos, rb)
         assert_close(kv[li][0], k_o, BF16, f"k layer {li}")
         assert_close(kv[li][1], v_o, BF16, f"v layer {li}")
+        o = rb(ref.gated_attention(q, host64(kv[li][0]), host64(kv[li][1]), pos,
+                                   None if dense else s_k, None if dense else lw.gain,
+                                   None if dense else lw.tau))
+        o_gpu = host64(taps[li]["attn_out"])
+        assert_close(o_gpu, o.reshape(rows, -1), BF16, f"attention output layer {li}")
+        r = rb(h_in + o_gpu @ lw.wo.T)
+        r_gpu = host64(taps[li]["resid"])
+        assert_close(r_gpu, r, BF16, f"post-attention residual layer {li}")
         if li == w.gate_layer:
-            s_ref = ref.round_fp32(ref.score(r, om.score_norm, om.eps, om.score_w1, om.score_b1,
-                                             om.score_w2, om.score_b2, rb))
-            assert_close(scores, s_ref, BF16, "scores")
+            s_ref = _check_scores(r_gpu, om, scores, "scores")
             flips, near = boundary_flips(s_ref.astype(np.float32), kept, prot, w.k, 2e-2, 1e-2)
             assert near, flips
-            r = r[kept]
-        h_out = ref.ffn_sublayer(r, lw, om, rb)
-        assert_close_bulk(hidden[li], h_out, BF16, f"hidden layer {li}")
-        h_in = host64(hidden[li])  # teacher forcing: the next layer reads the GPU's output
+            r_gpu = r_gpu[kept]
+        h_gpu = host64(taps[li]["hidden"])
+        assert_close(h_gpu, ref.ffn_sublayer(r_gpu, lw, om, rb), BF16, f"hidden layer {li}")
+        h_in = h_gpu  # teacher forcing: the next layer reads the GPU's output
     assert_close(out, rb(ref.rmsnorm(h_in, om.final_norm, om.eps)), BF16, "out")
 
 
-def _attn_row(h, lw, m, pos_q, k_cache, v_cache, pos_k, s_k, gain, tau, want_k, want_v, what):
-    """One token through one layer's attention sub-layer, its keys/values
-    taken from the GPU's KV cache rows [0..its own row]; checks its own k/v."""
-    hq, hkv, dh = m.n_heads_q, m.n_heads_kv, m.head_dim
-    y = rb(ref.rmsnorm(h[None], lw.attn_norm, m.eps))
-    qkv = rb(y @ lw.wqkv.T)
-    q = qkv[:, : hq * dh].reshape(1, hq, dh)
-    k = qkv[:, hq * dh: (hq + hkv) * dh].reshape(1, hkv, dh)
-    v = qkv[:, (hq + hkv) * dh:].reshape(1, hkv, dh)
-    if lw.q_norm is not None:
-        q = ref.rmsnorm(q, lw.q_norm, m.eps)
-        k = ref.rmsnorm(k, lw.k_norm, m.eps)
-    q = rb(ref.rope(q, np.array([pos_q]), m.rope_base))
-    k = rb(ref.rope(k, np.array([pos_q]), m.rope_base))
+def _attn_row(h, lw, m, pos_q, k_cache, v_cache, pos_k, s_k, gain, tau, want_k, want_v, o_gpu,
+              r_gpu, what):
+    """One token through one layer's attention sub-layer, teacher-forced:
+    its q, k, v from the GPU's input row h (k, v checked against the GPU's
+    cache row), its attention output from the GPU's cached keys/values
+    [0..its own row] (checked against o_gpu), its residual from o_gpu
+    (checked against r_gpu)."""
+    q, k, v = ref.project_qkv(h[None], lw, m, np.array([pos_q]), rb)
     assert_close(want_k, k[0], BF16, f"k {what}")
     assert_close(want_v, v[0], BF16, f"v {what}")
-    o = rb(ref.gated_attention_rows(q, np.array([pos_q]), k_cache, v_cache, pos_k, s_k, gain, tau))
-    return rb(h[None] + o.reshape(1, hq * dh) @ lw.wo.T)[0]
+    o = rb(ref.gated_attention_rows(q, np.array([pos_q]), k_cache, v_cache, pos_k, s_k, gain,
+                                    tau))
+    assert_close(o_gpu, o.reshape(-1), BF16, f"attention output {what}")
+    r = rb(h + o_gpu @ lw.wo.T)
+    assert_close(r_gpu, r, BF16, f"post-attention residual {what}")
 
 
-def test_prefill_28_layers_full_size_sampled_rows():
-    w = synth.QWEN_PREFILL_32K  # N=32768, K=4096, 28 layers, gate at layer 1
-    model, om = _models(w)
+FULL_SIZE_CASES = [pytest.param(k, False, id=f"k{k}") for k in synth.PREFILL_32K_BUDGETS] + \
+    [pytest.param(synth.QWEN_PREFILL_32K.n, True, id="dense")]
+
+
+@pytest.mark.parametrize("k,dense", FULL_SIZE_CASES)
+def test_prefill_28_layers_full_size_sampled_rows(k, dense):
+    """N=32768, 28 layers, gate at layer 1, at each budget of the workload
+    and in the dense run (K = N, no gate bias)."""
+    w = synth.shrink(synth.QWEN_PREFILL_32K, k=k)
+    model, om = _models(w, dense=dense)
     x = synth.torch_hidden_states(w, seed=w.seed + 1000, device="cuda")
     prot = synth.protect_tail(w.n, w.n_protect)
-    out, kept, scores, kv, hidden = _run_gpu(w, model, x, prot, with_hidden=True)
+    out, kept, scores, kv, taps = _run_gpu(w, model, x, prot, with_taps=True)
     # the kept set is exactly the selection of the GPU's scores
     assert np.array_equal(kept, ref.topk_select(scores, prot, w.k))
-    rng = np.random.default_rng(11)
+    if dense:
+        assert np.array_equal(kept, np.arange(w.n))
+    rng = np.random.default_rng(11 + k)
     kept_set = set(kept.tolist())
-    pruned = np.array(sorted(set(range(w.n)) - kept_set))
-    sample_kept = sorted({int(kept[-1]), int(kept[0])} |
+    pruned = np.array(sorted(set(range(w.n)) - kept_set), dtype=np.int64)
+    sample_kept = sorted({int(kept[-1]), int(kept[0]), int(kept[1])} |
                          set(rng.choice(kept[:-w.n_protect], 4, replace=False).tolist()) |
                          {int(np.nonzero(prot)[0][3])})
-    sample_pruned = sorted(rng.choice(pruned, 3, replace=False).tolist())
+    sample_pruned = sorted(rng.choice(pruned, 3, replace=False).tolist()) if pruned.size else []
     tokens = sample_kept + sample_pruned
     row_of = {int(t): r for r, t in enumerate(kept)}
     s_kept = scores[kept].astype(np.float64)
@@ -164,40 +193,47 @@ def test_prefill_28_layers_full_size_sampled_rows():
     xin = dict(zip(tokens, rows(x, tokens)))
     for li in range(w.n_layers):
         lw = om.layers[li]
+        tp = taps[li]
         if li <= w.gate_layer:  # every sampled token, keys 0..t
             kc, vc = host64(kv[li][0]), host64(kv[li][1])
-            hin = xin if li == 0 else dict(zip(tokens, rows(hidden[li - 1], tokens)))
+            hin = xin if li == 0 else dict(zip(tokens, rows(taps[li - 1]["hidden"], tokens)))
+            o_gpu = dict(zip(tokens, rows(tp["attn_out"], tokens)))
+            r_gpu = dict(zip(tokens, rows(tp["resid"], tokens)))
             for t in tokens:
-                r = _attn_row(hin[t], lw, om, t, kc[: t + 1], vc[: t + 1], np.arange(t + 1),
-                              None, None, None, kc[t], vc[t], f"layer {li} token {t}")
+                what = f"layer {li} token {t}"
+                _attn_row(hin[t], lw, om, t, kc[: t + 1], vc[: t + 1], np.arange(t + 1), None,
+                          None, None, kc[t], vc[t], o_gpu[t], r_gpu[t], what)
                 if li < w.gate_layer:
-                    want = rows(hidden[li], [t])[0]
-                    assert_close_bulk(want, ref.ffn_sublayer(r[None], lw, om, rb)[0], BF16,
-                                      f"hidden layer {li} token {t}")
+                    want = rows(tp["hidden"], [t])[0]
+                    assert_close(want, ref.ffn_sublayer(r_gpu[t][None], lw, om, rb)[0], BF16,
+                                 f"hidden {what}")
                     continue
-                # the gate layer: score of the post-attention residual, then its
-                # FFN on the kept rows
-                s_ref = ref.round_fp32(ref.score(r[None], om.score_norm, om.eps, om.score_w1,
-                                                 om.score_b1, om.score_w2, om.score_b2, rb))
-                assert_close(scores[t:t + 1], s_ref, BF16, f"score token {t}")
+                # the gate layer: score of the GPU's post-attention residual, then
+                # its FFN on the kept rows
+                _check_scores(r_gpu[t][None], om, scores[t:t + 1], f"score token {t}")
                 if t in kept_set:
-                    want = rows(hidden[li], [row_of[t]])[0]
-                    assert_close_bulk(want, ref.ffn_sublayer(r[None], lw, om, rb)[0], BF16,
-                                      f"hidden layer {li} kept row {row_of[t]}")
+                    want = rows(tp["hidden"], [row_of[t]])[0]
+                    assert_close(want, ref.ffn_sublayer(r_gpu[t][None], lw, om, rb)[0], BF16,
+                                 f"hidden layer {li} kept row {row_of[t]}")
             del kc, vc
             continue
         rk_list = [row_of[t] for t in sample_kept]
-        hin = dict(zip(sample_kept, rows(hidden[li - 1], rk_list)))
-        want_out = dict(zip(sample_kept, rows(hidden[li], rk_list)))
+        hin = dict(zip(sample_kept, rows(taps[li - 1]["hidden"], rk_list)))
+        o_gpu = dict(zip(sample_kept, rows(tp["attn_out"], rk_list)))
+        r_gpu = dict(zip(sample_kept, rows(tp["resid"], rk_list)))
+        want_out = dict(zip(sample_kept, rows(tp["hidden"], rk_list)))
         kc_all, vc_all = host64(kv[li][0]), host64(kv[li][1])
         for t in sample_kept:
             rk = row_of[t]
             kc, vc = kc_all[: rk + 1], vc_all[: rk + 1]
-            r = _attn_row(hin[t], lw, om, t, kc, vc, kept[: rk + 1], s_kept[: rk + 1], lw.gain,
-                          lw.tau, kc[rk], vc[rk], f"layer {li} kept row {rk}")
-            assert_close_bulk(want_out[t], ref.ffn_sublayer(r[None], lw, om, rb)[0], BF16,
-                              f"hidden layer {li} kept row {rk}")
-    last = rows(hidden[-1], [row_of[t] for t in sample_kept])
+            what = f"layer {li} kept row {rk}"
+            _attn_row(hin[t], lw, om, t, kc, vc, kept[: rk + 1], None if dense else
+                      s_kept[: rk + 1], lw.gain, lw.tau, kc[rk], vc[rk], o_gpu[t], r_gpu[t],
+                      what)
+            assert_close(want_out[t], ref.ffn_sublayer(r_gpu[t][None], lw, om, rb)[0], BF16,
+                         f"hidden {what}")
+        del kc_all, vc_all
+    last = rows(taps[-1]["hidden"], [row_of[t] for t in sample_kept])
     final = rb(ref.rmsnorm(last, om.final_norm, om.eps))
     assert_close(rows(out, [row_of[t] for t in sample_kept]), final, BF16, "out sampled rows")
 
