@@ -252,6 +252,38 @@ tg_status tg_gated_attn_backward(const void* q, const void* kk, const void* v, c
 tg_status tg_linear(const void* x, const void* w, const void* residual, int64_t m, int32_t n,
                     int32_t k, tg_dtype dtype, void* y, tg_stream stream);
 
+/* ---- hybrid models: the Gated DeltaNet mixer -----------------------------
+ *
+ * In a hybrid model most layers are Gated DeltaNet layers and only some are
+ * full attention. The scorer reads hidden states, so the gate may sit at a
+ * Gated DeltaNet layer. Above the gate the token-gated logit bias applies
+ * only in the full-attention layers (tg_gated_attn_prefill); a Gated
+ * DeltaNet layer has no logits and runs on the kept tokens as they are
+ * ([TC] "门控位置影响剪枝效果", figure 5). The layer's projections are plain
+ * GEMMs (tg_linear); this call is its token mixer over one sequence, the K
+ * kept rows in ascending original order (the pages do not spell the layer
+ * out; the mixer is the published gated delta rule of Yang, Kautz and
+ * Hatamizadeh, "Gated Delta Networks", ICLR 2025, in the Qwen3-Next shape):
+ *   c_t = SiLU(sum_{i<W} conv_w[:, i] * x_{t-W+1+i})  over the qkv channels
+ *   q = l2norm(c_q) / sqrt(dk), k = l2norm(c_k), v = c_v  (l2norm: x / sqrt(|x|^2 + 1e-6))
+ *   alpha = exp(-exp(A_log) * softplus(a_t + dt_bias)), beta = sigmoid(b_t)
+ *   S_t = alpha S_{t-1} (I - beta k k^T) + beta v k^T,  o_t = S_t q  (per value head)
+ *   y_t = o_t / sqrt(mean(o_t^2) + norm_eps) * norm_w * SiLU(z_t)    (per value head)
+ * Value head h reads key head h / (hv / hk).
+ */
+typedef struct {
+  int32_t n_heads_k;   /* hk                                               */
+  int32_t n_heads_v;   /* hv, a multiple of hk                             */
+  int32_t head_dim_k;  /* dk: 64 or 128                                    */
+  int32_t head_dim_v;  /* dv: a multiple of 32, at most 256                */
+  int32_t conv_width;  /* W: 1..4                                          */
+  const float* conv_w; /* [C, W] with C = 2 hk dk + hv dv                  */
+  const float* A_log;  /* [hv]                                             */
+  const float* dt_bias;/* [hv]                                             */
+  const float* norm_w; /* [dv]                                             */
+  float norm_eps;
+} tg_gdn_layer;
+
 /* ---- the full stack ---------------------------------------------------- */
 
 typedef struct {
@@ -265,6 +297,14 @@ typedef struct {
   const void* w_down;     /* [d, I]                                            */
   const float* gain;      /* [hq] gate-bias gain, layers above the gate; NULL=0 */
   const float* tau;       /* [hq] temperature, layers above the gate; NULL = 1  */
+  /* A hybrid model's Gated DeltaNet layer: gdn != NULL makes the layer's
+   * token mixer the Gated DeltaNet mixer (tg_gated_deltanet) instead of
+   * attention: r = x + W_out . mixer(W_in . RMSNorm(x; attn_norm)), then the
+   * same FFN sub-layer. wqkv, q_norm, k_norm, wo, gain and tau are unused. */
+  const tg_gdn_layer* gdn; /* HOST pointer to the mixer's parameters, or NULL   */
+  const void* w_in;       /* [C + hv dv + 2 hv, d]: rows giving qkv (C = 2 hk dk
+                             + hv dv channels), then z, then a, then b          */
+  const void* w_out;      /* [d, hv dv]                                         */
 } tg_layer;
 
 typedef struct {
@@ -302,12 +342,22 @@ typedef struct {
  *   x [n, d] dtype (input hidden states); protect [n] uint8 or NULL
  *   out [k, d] dtype: final-normed hidden states of the kept rows
  *   kept_idx [k] int32 (out, ascending); scores [n] fp32 (out) or NULL
- *   kv: HOST array of n_layers tg_kv, or NULL
+ *   kv: HOST array of n_layers tg_kv, or NULL (bf16: 16-byte aligned pointers)
+ * Hybrid stacks: a layer with gdn != NULL runs the Gated DeltaNet mixer
+ * over its rows in ascending original order (all n rows at and below the
+ * gate, the k kept rows above it); the scorer then reads the post-mixer
+ * residual when the gate sits at such a layer, and the gate bias applies
+ * only to the attention layers above the gate ([TC] "门控位置影响剪枝效果",
+ * figure 5). For such a layer kv[l].k receives the mixer's last W-1 conv
+ * input rows [W-1, C] (dtype) and kv[l].v its final state [hv, dv, dk]
+ * (fp32), which a following call continues from. bf16 only; the w_in
+ * output width C + hv dv + 2 hv must be a multiple of 32.
  *   taps: HOST array of n_layers tg_layer_taps, or NULL. Each non-NULL
  *     pointer of taps[l] receives a copy of one intermediate of layer l, for
  *     inspection and per-layer checks (one device copy per requested tensor):
  *       attn_out [rows, hq dh]: the attention output before the output
- *         projection (rows = n at and below the gate, k above it);
+ *         projection (rows = n at and below the gate, k above it); for a
+ *         Gated DeltaNet layer the mixer output [rows, hv dv];
  *       resid [rows, d]: the residual stream after the attention sub-layer
  *         (x + Wo . attn_out; rows as attn_out);
  *       hidden [rows', d]: the layer's output after its FFN (rows' = n below
@@ -318,6 +368,11 @@ typedef struct {
   void* resid;
   void* hidden;
 } tg_layer_taps;
+
+/* Workspace bytes of tg_prefill (and tg_prefill_multi with k = max(ks)) for
+ * this model: tg_workspace_size(TG_OP_PREFILL) plus the buffers of a hybrid
+ * stack's Gated DeltaNet layers (0 on invalid sizes). */
+size_t tg_prefill_workspace_size(const tg_model* model, int64_t n, int64_t k);
 
 tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protect, int64_t n,
                      int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx, float* scores,
@@ -398,7 +453,8 @@ tg_status tg_prefill_batch(const tg_model* model, const void* x, const uint8_t* 
  *     and sets bit 2 of the device error word. scores NULL: no gate bias.
  *   out [1, d] bf16: the token's final-normed hidden state.
  * bf16 and head_dim 128 only (TG_ERR_UNSUPPORTED otherwise); GQA groups of 1,
- * 2, 4 or 8 query heads. Workspace: tg_workspace_size(TG_OP_DECODE) with
+ * 2, 4 or 8 query heads; attention layers only (a Gated DeltaNet layer is
+ * TG_ERR_UNSUPPORTED). Workspace: tg_workspace_size(TG_OP_DECODE) with
  * shape.k = k_kept. Asynchronous on the stream; validates on the host first.
  */
 tg_status tg_decode_step(const tg_model* model, const void* x, int64_t pos, int32_t gate_layer,
@@ -406,37 +462,7 @@ tg_status tg_decode_step(const tg_model* model, const void* x, int64_t pos, int3
                          const int32_t* kept_idx, int64_t k_kept, void* out, void* ws,
                          size_t ws_bytes, tg_stream stream);
 
-/* ---- hybrid models: the Gated DeltaNet mixer -----------------------------
- *
- * In a hybrid model most layers are Gated DeltaNet layers and only some are
- * full attention. The scorer reads hidden states, so the gate may sit at a
- * Gated DeltaNet layer. Above the gate the token-gated logit bias applies
- * only in the full-attention layers (tg_gated_attn_prefill); a Gated
- * DeltaNet layer has no logits and runs on the kept tokens as they are
- * ([TC] "门控位置影响剪枝效果", figure 5). The layer's projections are plain
- * GEMMs (tg_linear); this call is its token mixer over one sequence, the K
- * kept rows in ascending original order (the pages do not spell the layer
- * out; the mixer is the published gated delta rule of Yang, Kautz and
- * Hatamizadeh, "Gated Delta Networks", ICLR 2025, in the Qwen3-Next shape):
- *   c_t = SiLU(sum_{i<W} conv_w[:, i] * x_{t-W+1+i})  over the qkv channels
- *   q = l2norm(c_q) / sqrt(dk), k = l2norm(c_k), v = c_v  (l2norm: x / sqrt(|x|^2 + 1e-6))
- *   alpha = exp(-exp(A_log) * softplus(a_t + dt_bias)), beta = sigmoid(b_t)
- *   S_t = alpha S_{t-1} (I - beta k k^T) + beta v k^T,  o_t = S_t q  (per value head)
- *   y_t = o_t / sqrt(mean(o_t^2) + norm_eps) * norm_w * SiLU(z_t)    (per value head)
- * Value head h reads key head h / (hv / hk).
- */
-typedef struct {
-  int32_t n_heads_k;   /* hk                                               */
-  int32_t n_heads_v;   /* hv, a multiple of hk                             */
-  int32_t head_dim_k;  /* dk: 64 or 128                                    */
-  int32_t head_dim_v;  /* dv: a multiple of 32, at most 256                */
-  int32_t conv_width;  /* W: 1..4                                          */
-  const float* conv_w; /* [C, W] with C = 2 hk dk + hv dv                  */
-  const float* A_log;  /* [hv]                                             */
-  const float* dt_bias;/* [hv]                                             */
-  const float* norm_w; /* [dv]                                             */
-  float norm_eps;
-} tg_gdn_layer;
+/* ---- the Gated DeltaNet mixer on its own (tg_gdn_layer is above) -------- */
 
 /* Workspace bytes of tg_gated_deltanet for T tokens (0 for a bad layer). */
 size_t tg_gated_deltanet_workspace_size(const tg_gdn_layer* layer, int64_t T);

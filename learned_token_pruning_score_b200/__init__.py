@@ -47,7 +47,7 @@ class TgShape(ctypes.Structure):
 
 class TgLayer(ctypes.Structure):
     _fields_ = [(n, _c_p) for n in ("attn_norm", "wqkv", "q_norm", "k_norm", "wo", "ffn_norm",
-                                    "w_gate_up", "w_down", "gain", "tau")]
+                                    "w_gate_up", "w_down", "gain", "tau", "gdn", "w_in", "w_out")]
 
 
 class TgModel(ctypes.Structure):
@@ -104,6 +104,7 @@ _attn_bwd = _sig("tg_gated_attn_backward", _ci, _c_p, _c_p, _c_p, _c_p, _c_p, _c
 _prefill = _sig("tg_prefill", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64, _c_i64, _c_i32,
                 _c_p, _c_p, _c_p, ctypes.POINTER(TgKV), ctypes.POINTER(TgLayerTaps), _c_p,
                 _c_sz, _c_p)
+_prefill_ws = _sig("tg_prefill_workspace_size", _c_sz, ctypes.POINTER(TgModel), _c_i64, _c_i64)
 _prefill_multi = _sig("tg_prefill_multi", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64,
                       ctypes.POINTER(_c_i64), _c_i32, _c_i32, ctypes.POINTER(_c_p),
                       ctypes.POINTER(_c_p), _c_p, _c_p, _c_sz, _c_p)
@@ -422,6 +423,9 @@ class Model:
     layers: one dict per layer with keys attn_norm, wqkv, wo, ffn_norm,
     w_gate_up, w_down (optional), q_norm/k_norm (optional), gain/tau
     (optional; used above the gate). Matrices in the model dtype, vectors fp32.
+    A hybrid model's Gated DeltaNet layer has instead of wqkv/wo the keys gdn
+    (a GdnLayer: the mixer's parameters), w_in [C + hv dv + 2 hv, d] and
+    w_out [d, hv dv]; attn_norm is then the norm before the mixer.
     """
 
     n_heads_q: int
@@ -434,16 +438,21 @@ class Model:
     rope_base: float = 1e6
 
     def __post_init__(self):
-        w = self.layers[0]["wqkv"]
+        w = next(lw["wqkv"] if "wqkv" in lw else lw["w_in"] for lw in self.layers)
         self.dtype = _dt(w)
         self.d_model = w.shape[1]
-        gu = self.layers[0].get("w_gate_up")
+        gu = next((lw["w_gate_up"] for lw in self.layers if lw.get("w_gate_up") is not None),
+                  None)
         self.d_ffn = 0 if gu is None else gu.shape[0] // 2
         self.d_score = self.score["score_w1"].shape[0]
         arr = (TgLayer * len(self.layers))()
         for i, lw in enumerate(self.layers):
             for name, _ in TgLayer._fields_:
-                setattr(arr[i], name, _ptr(lw.get(name)))
+                if name == "gdn":
+                    g = lw.get("gdn")
+                    arr[i].gdn = None if g is None else ctypes.addressof(g.c)
+                else:
+                    setattr(arr[i], name, _ptr(lw.get(name)))
         self._layers_c = arr
         self.c = TgModel(self.dtype, len(self.layers), self.d_model, self.n_heads_q,
                          self.n_heads_kv, self.head_dim, self.d_ffn, self.d_score, self.eps,
@@ -458,11 +467,7 @@ class Model:
                                  head_dim=self.head_dim, d_ffn=self.d_ffn, dtype=self.dtype)
 
     def workspace_size(self, n: int, k: int, gate_layer: int) -> int:
-        return tg_workspace_size(TG_OP_PREFILL, n=n, k=k, d_model=self.d_model,
-                                 n_heads_q=self.n_heads_q, n_heads_kv=self.n_heads_kv,
-                                 head_dim=self.head_dim, d_score=self.d_score, d_ffn=self.d_ffn,
-                                 n_layers=len(self.layers), gate_layer=gate_layer,
-                                 dtype=self.dtype)
+        return int(_prefill_ws(ctypes.byref(self.c), n, k))
 
 
 def tg_decode_step(model: Model, x, pos: int, gate_layer: int, kv: Sequence, lens: Sequence[int],

@@ -25,8 +25,15 @@
 //              in the 128-byte-swizzled K-major layout the MMA reads.
 //   end        O / l read from TMEM, written bf16.
 // TMEM: S0 = cols [0,128), S1 = [128,256), O = [256,384) of 512.
+#include <algorithm>
 #include <atomic>
+#include <functional>
+#include <map>
+#include <memory>
+#include <mutex>
+#include <queue>
 #include <type_traits>
+#include <vector>
 
 #include "tg_device.cuh"
 #include "tg_internal.h"
@@ -349,6 +356,16 @@ struct Layout {
   static constexpr size_t kSmem = 1024 + kOffBar + 256;
 };
 
+// Work-item table of a short sequence (see Schedule below): entry i gives
+// one part of one query tile, and the grid runs n_pairs CTAs per entry.
+//   x = qt | kv_lo << 10 | kv_hi << 20        (KV tiles kv_lo..kv_hi)
+//   y = part | (n_parts - 1) << 4 | split << 8 | slot0 << 20
+// A query tile split into n_parts parts has one counter (`split`) and
+// n_parts partial-result slots slot0 .. slot0 + n_parts - 1.
+constexpr int kMaxItems = 256;
+constexpr int kMaxSlots = 32;  // partial-result slots per head pair
+constexpr int kMaxParts = 4;
+
 struct Params {
   int64_t T;
   int hq, hkv;
@@ -360,13 +377,35 @@ struct Params {
   float* lse;      // [hq, T] or null
   float* out_f32;  // [T, hq, dh] or null: the output before rounding
   unsigned int* err;
+  // Split query tiles (n_items > 0): each part writes its unnormalised
+  // output rows and (m, l) to a slot; the part that finishes last (per-tile
+  // counter) merges every slot in slot order and writes the result.
+  int n_items;      // 0: closed-form order, no splits
+  float* part_o;    // [slots][n_pairs][2 heads][128 rows][128] fp32
+  float* part_ml;   // [slots][n_pairs][2][128][2] fp32 (m in log2 units, l)
+  unsigned* cnt;    // [splits][n_pairs], zero between launches
+  uint2 items[kMaxItems];
 };
+
+// bar.red.and over the `count` threads of named barrier `id`.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
 
 template <bool kBias>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKAug,
-                 Params p) {
+                 const __grid_constant__ Params p) {
   using Lay = Layout<kBias>;
   constexpr int kOffQAugA = Lay::kOffQAugA, kOffQAugB = Lay::kOffQAugB, kOffKAug = Lay::kOffKAug;
   constexpr int kOffQA = Lay::kOffQA, kOffQB = Lay::kOffQB, kOffK = Lay::kOffK, kOffV = Lay::kOffV;
@@ -394,7 +433,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int pairs_per_kv = (p.hq / p.hkv) / 2;
   const int n_pairs = p.hq / 2;
   int qt, head0;
-  if (p.kv_major) {
+  int kv_lo = 0;
+  if (p.n_items > 0) {
+    const uint32_t x = p.items[blockIdx.x / n_pairs].x;
+    head0 = 2 * (static_cast<int>(blockIdx.x) % n_pairs);
+    qt = static_cast<int>(x & 1023u);
+    kv_lo = static_cast<int>((x >> 10) & 1023u);
+  } else if (p.kv_major) {
     const int per_kv = p.n_qtiles * pairs_per_kv;
     const int g0 = static_cast<int>(blockIdx.x) / per_kv;
     const int rem = static_cast<int>(blockIdx.x) % per_kv;
@@ -406,8 +451,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int g = head0 / (p.hq / p.hkv);
   const int q0 = qt * kBlk;
-  const int n_kv = qt + 1;
+  // KV tiles kv_lo .. kv_hi of this item (the diagonal tile is qt)
+  const int kv_hi = p.n_items > 0 ? static_cast<int>((p.items[blockIdx.x / n_pairs].x >> 20) & 1023u)
+                                  : qt;
+  const int n_kv = kv_hi - kv_lo + 1;
   constexpr uint32_t kKBytes = kTile + (kBias ? kAugTile : 0);
+  __shared__ int s_last;
 
   pdl_trigger();
   if (threadIdx.x == 0) {
@@ -452,14 +501,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&k_empty[s], ph, p.err)) break;
         uint8_t* kd = smem + kOffK + s * kTile;
         mbar_arrive_expect_tx(&k_full[s], kKBytes);
-        tma_load_3d(&tmK, &k_full[s], kd, 0, g, j * kBlk);
-        tma_load_3d(&tmK, &k_full[s], kd + kSub, 64, g, j * kBlk);
-        if (kBias) tma_load_2d(&tmKAug, &k_full[s], smem + kOffKAug + s * kAugTile, 0, j * kBlk);
+        const int key0 = (kv_lo + j) * kBlk;
+        tma_load_3d(&tmK, &k_full[s], kd, 0, g, key0);
+        tma_load_3d(&tmK, &k_full[s], kd + kSub, 64, g, key0);
+        if (kBias) tma_load_2d(&tmKAug, &k_full[s], smem + kOffKAug + s * kAugTile, 0, key0);
         if (!mbar_wait(&v_empty[s], ph, p.err)) break;
         uint8_t* vd = smem + kOffV + s * kTile;
         mbar_arrive_expect_tx(&v_full[s], kTile);
-        tma_load_3d(&tmV, &v_full[s], vd, j * kBlk, 0, g);
-        tma_load_3d(&tmV, &v_full[s], vd + kSub, j * kBlk + 64, 0, g);
+        tma_load_3d(&tmV, &v_full[s], vd, key0, 0, g);
+        tma_load_3d(&tmV, &v_full[s], vd + kSub, key0 + 64, 0, g);
       }
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
@@ -556,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
-      const int kv0 = j * kBlk;
+      const int kv0 = (kv_lo + j) * kBlk;
       if (!mbar_wait_warp(&s_full[h], j & 1, p.err)) { ok = false; break; }
       tc_fence_after();
       // S row: four TMEM loads in flight, one wait.
@@ -580,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           x[96 + i] = __uint_as_float(r3[i]);
         }
       }
-      const bool diag = j == n_kv - 1;
+      const bool diag = kv_lo + j == qt;
       if (diag) {  // diagonal tile: causal mask
 #pragma unroll
         for (int i = 0; i < 128; ++i)
@@ -654,8 +704,83 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&p_full[h]);
     }
-    if (ok && mbar_wait_warp(o_full, 0, p.err)) {
-      tc_fence_after();
+    ok = ok && mbar_wait_warp(o_full, 0, p.err);
+    if (ok) tc_fence_after();
+    // the item's split fields (decoded here, not kept live through the loop)
+    const uint32_t iy = p.n_items > 0 ? p.items[blockIdx.x / n_pairs].y : 0u;
+    const int part = static_cast<int>(iy & 15u);
+    const int n_parts = static_cast<int>((iy >> 4) & 15u) + 1;
+    const int split = static_cast<int>((iy >> 8) & 4095u);
+    const int slot0 = static_cast<int>(iy >> 20);
+    // Output of a split query tile: this part's rows go to its slot; the
+    // part that finishes last merges every slot (slot order, so the result
+    // does not depend on which part finishes last) with weights 2^(m_s - M).
+    float wts[kMaxParts];
+    int n_merge = 1;
+    const size_t pair_idx = static_cast<size_t>(head0 / 2);
+    auto slot_row = [&](int slot) {
+      return ((static_cast<size_t>(slot) * n_pairs + pair_idx) * 2 + h) * kBlk + r;
+    };
+    if (n_parts > 1) {
+      if (ok) {
+        const size_t ri = slot_row(slot0 + part);
+        float4* po = reinterpret_cast<float4*>(p.part_o + ri * kDh);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tmem_ld32_wait(tmem + lane_off + o_col + static_cast<uint32_t>(c * 32), o);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            po[c * 8 + v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+        }
+        *reinterpret_cast<float2*>(p.part_ml + ri * 2) = make_float2(m, l);
+        __threadfence();
+      }
+      // every softmax thread of the CTA reaches both barriers, whatever ok is
+      const bool all_ok = named_bar_and(1, 256, ok);
+      if (threadIdx.x == 128) {
+        int last = 0;
+        if (all_ok) {
+          unsigned* c = p.cnt + static_cast<size_t>(split) * n_pairs + pair_idx;
+          const unsigned old = atomicAdd(c, 1u);
+          __threadfence();
+          last = old == static_cast<unsigned>(n_parts - 1);
+          if (last) *c = 0u;  // zero again for the next launch
+        }
+        s_last = last;
+      }
+      named_bar_sync(1, 256);
+      ok = s_last != 0;
+      if (ok) {
+        float ms[kMaxParts], ls[kMaxParts];
+        float M = -INFINITY;
+#pragma unroll
+        for (int s2 = 0; s2 < kMaxParts; ++s2) {
+          if (s2 < n_parts) {
+            if (s2 == part) {
+              ms[s2] = m;
+              ls[s2] = l;
+            } else {
+              const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml) +
+                                       slot_row(slot0 + s2));
+              ms[s2] = ml.x;
+              ls[s2] = ml.y;
+            }
+            M = fmaxf(M, ms[s2]);
+          }
+        }
+        float L = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < kMaxParts; ++s2) {
+          wts[s2] = s2 < n_parts ? ex2_approx(ms[s2] - M) : 0.f;
+          if (s2 < n_parts) L = fmaf(ls[s2], wts[s2], L);
+        }
+        m = M;
+        l = L;
+        n_merge = n_parts;
+      }
+    }
+    if (ok) {
       const float inv = 1.0f / l;
       // log-sum-exp of the row's logits: m and l are in log2 units
       if (p.lse && q_row < p.T) p.lse[head * p.T + q_row] = (m + log2f(l)) * kLn2;
@@ -663,6 +788,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 4; ++c) {
         float o[32];
         tmem_ld32_wait(tmem + lane_off + o_col + static_cast<uint32_t>(c * 32), o);
+        if (n_merge > 1) {
+          float acc[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+#pragma unroll
+          for (int s2 = 0; s2 < kMaxParts; ++s2) {
+            if (s2 >= n_merge) break;
+            if (s2 == part) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) acc[i] = fmaf(o[i], wts[s2], acc[i]);
+            } else {
+              const float4* src = reinterpret_cast<const float4*>(
+                  p.part_o + slot_row(slot0 + s2) * kDh + c * 32);
+#pragma unroll
+              for (int v = 0; v < 8; ++v) {
+                const float4 t = __ldcg(src + v);
+                acc[4 * v] = fmaf(t.x, wts[s2], acc[4 * v]);
+                acc[4 * v + 1] = fmaf(t.y, wts[s2], acc[4 * v + 1]);
+                acc[4 * v + 2] = fmaf(t.z, wts[s2], acc[4 * v + 2]);
+                acc[4 * v + 3] = fmaf(t.w, wts[s2], acc[4 * v + 3]);
+              }
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = acc[i];
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] *= inv;
         if (q_row < p.T) {
@@ -692,10 +843,142 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 2) tmem_dealloc(tmem, 512);
 }
 
+// ---------------------------------------------------------------------------
+// Schedule of a short sequence. With few query tiles, one CTA per (tile, head
+// pair) leaves SMs idle while the last (longest, causal) tiles finish. The
+// table instead lists query-tile parts, longest first, so that the block
+// scheduler (which starts CTAs in index order as SMs free up) runs a
+// longest-first list schedule, and splits long tiles' KV ranges into up to
+// kMaxParts parts, with the part length that gives the shortest simulated
+// makespan on the B200's 148 SMs. The schedule depends only on (T, heads), never on the device, so
+// the workspace it needs is known on the host.
+constexpr int kMaxTableQ = 64;   // query tiles (T <= 8192) eligible for a table
+constexpr int kSchedSMs = 148;
+constexpr double kItemOverhead = 1.0;  // per-CTA prologue + epilogue, in KV-tile units
+constexpr double kMergeCost = 0.5;     // writing / merging a partial
+
+struct Schedule {
+  int n_items = 0, n_split = 0, n_slots = 0;
+  uint2 items[kMaxItems];
+};
+
+double list_makespan(const std::vector<double>& jobs) {
+  std::priority_queue<double, std::vector<double>, std::greater<double>> q;
+  for (int i = 0; i < kSchedSMs; ++i) q.push(0.0);
+  double mk = 0.0;
+  for (double c : jobs) {
+    double t = q.top();
+    q.pop();
+    t += c;
+    mk = std::max(mk, t);
+    q.push(t);
+  }
+  return mk;
+}
+
+// Fills *out and returns true when a table schedule applies (n_q query tiles
+// of n_pairs head pairs); false: the closed-form order, no splits.
+bool make_schedule(int n_q, int n_pairs, Schedule* out) {
+  if (n_q < 1 || n_q > kMaxTableQ || n_pairs < 1) return false;
+  struct Part {
+    int qt, lo, hi, part, np;
+    double cost;
+  };
+  double best = 1e300;
+  std::vector<Part> best_parts;
+  // cap: the most KV tiles one part takes; longer tiles split into
+  // ceil(tiles / cap) near-equal parts
+  for (int cap = n_q; cap >= (n_q + kMaxParts - 1) / kMaxParts; --cap) {
+    std::vector<Part> parts;
+    int slots = 0;
+    for (int qt = n_q - 1; qt >= 0; --qt) {
+      const int c = qt + 1, np = (c + cap - 1) / cap;
+      for (int i = 0; i < np; ++i) {
+        const int lo = i * c / np, hi = (i + 1) * c / np - 1;
+        parts.push_back(Part{qt, lo, hi, i, np,
+                             double(hi - lo + 1) + kItemOverhead + (np > 1 ? kMergeCost : 0.0)});
+      }
+      if (np > 1) slots += np;
+    }
+    if (static_cast<int>(parts.size()) > kMaxItems || slots > kMaxSlots) continue;
+    std::stable_sort(parts.begin(), parts.end(),
+                     [](const Part& a, const Part& b) { return a.cost > b.cost; });
+    std::vector<double> jobs;
+    for (const Part& pt : parts)
+      for (int k = 0; k < n_pairs; ++k) jobs.push_back(pt.cost);
+    const double mk = list_makespan(jobs);
+    if (mk < best - 1e-9) {
+      best = mk;
+      best_parts = parts;
+    }
+  }
+  if (best_parts.empty()) return false;
+  // counters and slots of the split tiles, in query-tile order
+  std::vector<int> split_of(n_q, -1), slot_of(n_q, 0);
+  int n_split = 0, n_slots = 0;
+  for (int qt = 0; qt < n_q; ++qt)
+    for (const Part& pt : best_parts)
+      if (pt.qt == qt && pt.part == 0 && pt.np > 1) {
+        split_of[qt] = n_split++;
+        slot_of[qt] = n_slots;
+        n_slots += pt.np;
+      }
+  out->n_items = static_cast<int>(best_parts.size());
+  out->n_split = n_split;
+  out->n_slots = n_slots;
+  for (int i = 0; i < out->n_items; ++i) {
+    const Part& pt = best_parts[i];
+    const unsigned sp = pt.np > 1 ? static_cast<unsigned>(split_of[pt.qt]) : 0u;
+    const unsigned sl = pt.np > 1 ? static_cast<unsigned>(slot_of[pt.qt]) : 0u;
+    out->items[i] = make_uint2(static_cast<unsigned>(pt.qt) | static_cast<unsigned>(pt.lo) << 10 |
+                                   static_cast<unsigned>(pt.hi) << 20,
+                               static_cast<unsigned>(pt.part) |
+                                   static_cast<unsigned>(pt.np - 1) << 4 | sp << 8 | sl << 20);
+  }
+  return true;
+}
+
+// make_schedule is a host simulation (about a millisecond); its result
+// depends only on (n_q, n_pairs), so it is computed once per shape.
+const Schedule* cached_schedule(int n_q, int n_pairs) {
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, std::unique_ptr<Schedule>> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find({n_q, n_pairs});
+  if (it == cache.end()) {
+    auto sch = std::make_unique<Schedule>();
+    if (!make_schedule(n_q, n_pairs, sch.get())) sch.reset();
+    it = cache.emplace(std::make_pair(n_q, n_pairs), std::move(sch)).first;
+  }
+  return it->second.get();
+}
+
 }  // namespace pair
 
 
 }  // namespace
+
+// Byte offset of the split counters inside the split scratch.
+static size_t split_cnt_offset(int hq) {
+  const size_t rows = size_t(pair::kMaxSlots) * size_t(hq / 2) * 2 * kBlk;
+  return align_up(rows * kDh * 4, 256) + align_up(rows * 2 * 4, 256);
+}
+
+cudaError_t attn_split_clear(void* split_ws, size_t split_ws_bytes, int hq, cudaStream_t st) {
+  if (split_ws == nullptr || split_ws_bytes == 0) return cudaSuccess;
+  return cudaMemsetAsync(static_cast<char*>(split_ws) + split_cnt_offset(hq), 0,
+                         size_t(pair::kMaxSlots) * size_t(hq / 2) * 4, st);
+}
+
+size_t attn_split_bytes(int64_t T, int hq, int hkv) {
+  if (T < 1 || hkv < 1 || hq % hkv != 0 || (hq / hkv) % 2 != 0) return 0;
+  const int64_t n_q = (T + kBlk - 1) / kBlk;
+  if (n_q > pair::kMaxTableQ) return 0;
+  const size_t n_pairs = static_cast<size_t>(hq / 2);
+  const size_t rows = size_t(pair::kMaxSlots) * n_pairs * 2 * kBlk;
+  return align_up(rows * kDh * 4, 256) + align_up(rows * 2 * 4, 256) +
+         align_up(size_t(pair::kMaxSlots) * n_pairs * 4, 256);
+}
 
 bool attn_tc_supported(const AttnArgs& a) {
   auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
@@ -751,6 +1034,30 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
     } else {
       tka = tk;  // not read
     }
+    pp.n_items = 0;
+    pp.part_o = pp.part_ml = nullptr;
+    pp.cnt = nullptr;
+    unsigned grid = static_cast<unsigned>(p.n_qtiles) * static_cast<unsigned>(a.hq / 2);
+    if (a.split_ws != nullptr && a.split_ws_bytes >= attn_split_bytes(a.T, a.hq, a.hkv)) {
+      const pair::Schedule* schp = pair::cached_schedule(p.n_qtiles, a.hq / 2);
+      if (schp != nullptr) {
+        const pair::Schedule& sch = *schp;
+        const size_t n_pairs = static_cast<size_t>(a.hq / 2);
+        const size_t rows = size_t(pair::kMaxSlots) * n_pairs * 2 * kBlk;
+        char* base = static_cast<char*>(a.split_ws);
+        pp.part_o = reinterpret_cast<float*>(base);
+        pp.part_ml = reinterpret_cast<float*>(base + align_up(rows * kDh * 4, 256));
+        pp.cnt = reinterpret_cast<unsigned*>(base + split_cnt_offset(a.hq));
+        pp.n_items = sch.n_items;
+        for (int i = 0; i < sch.n_items; ++i) pp.items[i] = sch.items[i];
+        grid = static_cast<unsigned>(sch.n_items) * static_cast<unsigned>(n_pairs);
+        if (sch.n_split > 0 && !a.split_cnt_zeroed) {
+          const cudaError_t e0 =
+              cudaMemsetAsync(pp.cnt, 0, size_t(sch.n_split) * n_pairs * 4, st);
+          if (e0 != cudaSuccess) return e0;
+        }
+      }
+    }
     auto kern = bias ? pair::attn_tc_pair<true> : pair::attn_tc_pair<false>;
     const size_t smem = bias ? pair::Layout<true>::kSmem : pair::Layout<false>::kSmem;
     cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(kern), int(smem));
@@ -766,7 +1073,6 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
       ok.store(fa.numRegs == int(pair::kRegsLaunch) ? 1 : -1);
     }
     if (ok.load() < 0) return cudaErrorInvalidConfiguration;
-    const unsigned grid = static_cast<unsigned>(p.n_qtiles) * static_cast<unsigned>(a.hq / 2);
     return launch_pdl(kern, dim3(grid), dim3(pair::kThreads), smem, st, tq, tk, tv, tka, pp);
   }
   cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(attn_tc), int(kSmem));

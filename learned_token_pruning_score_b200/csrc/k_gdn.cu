@@ -92,7 +92,7 @@ __device__ __forceinline__ float softplus_f(float x) {
 // carried row W-1+r (zeros when none is carried).
 template <typename T>
 __device__ __forceinline__ float conv_src(const GdnArgs& a, int64_t r, int64_t c, int C) {
-  if (r >= 0) return ld_act(static_cast<const T*>(a.qkv) + r * C + c);
+  if (r >= 0) return ld_act(static_cast<const T*>(a.qkv) + r * a.ld_qkv + c);
   if (a.conv_in == nullptr) return 0.f;
   return ld_act(static_cast<const T*>(a.conv_in) + (r + a.W - 1) * C + c);
 }
@@ -120,7 +120,8 @@ struct ConvWindow {
                                        const bool (&on)[kPer], int64_t t, int C) {
 #pragma unroll
     for (int j = 0; j < kPer; ++j)
-      next[j] = (on[j] && t < a.T) ? ld_act(static_cast<const T*>(a.qkv) + t * C + ch[j]) : 0.f;
+      next[j] = (on[j] && t < a.T) ? ld_act(static_cast<const T*>(a.qkv) + t * a.ld_qkv + ch[j])
+                                   : 0.f;
   }
 
   __device__ __forceinline__ void init(const GdnArgs& a, const int (&ch)[kPer], bool (&on)[kPer],
@@ -241,8 +242,8 @@ __device__ __forceinline__ void prep_v(const GdnArgs& a, int h, int part, int64_
     if (lane == 0 && part == 0) {
       float g = 0.f, beta = 0.f;
       if (live) {
-        const float av = ld_act(static_cast<const T*>(a.a) + t * a.hv + h);
-        const float bv = ld_act(static_cast<const T*>(a.b) + t * a.hv + h);
+        const float av = ld_act(static_cast<const T*>(a.a) + t * a.ld_ab + h);
+        const float bv = ld_act(static_cast<const T*>(a.b) + t * a.ld_ab + h);
         g = -A * softplus_f(av + dtb);
         beta = 1.f / (1.f + expf(-bv));
       }
@@ -606,7 +607,7 @@ __global__ void __launch_bounds__(256) gdn_out(GdnArgs a) {
   if (gw >= a.T * a.hv) return;
   const int per = a.dv / 32;  // at most 8
   const float* o = a.o + gw * a.dv + lane * per;
-  const T* z = static_cast<const T*>(a.z) + gw * a.dv + lane * per;
+  const T* z = static_cast<const T*>(a.z) + (gw / a.hv) * a.ld_z + (gw % a.hv) * a.dv + lane * per;
   T* y = static_cast<T*>(a.y) + gw * a.dv + lane * per;
   float v[8];
   float ss = 0.f;

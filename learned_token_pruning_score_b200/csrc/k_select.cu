@@ -371,6 +371,263 @@ __global__ void __launch_bounds__(kThreads) sel_write(const float* __restrict__ 
   }
 }
 
+// ---------------------------------------------------------------------------
+// One-launch selection for n <= kClusterMaxN: one thread-block cluster of C
+// CTAs (C = 1, 2, 4, 8 or 16; 8192 tokens per CTA, 8 per thread) holds every
+// key in registers, so the scores are read once. Each radix pass builds a
+// per-CTA shared-memory histogram of the next digit; CTA c then sums slice c
+// of the bins over the cluster's CTAs (distributed shared memory), every CTA
+// finds the slice and then the bin where the count from the top reaches the
+// rank still needed, and the next pass refines that prefix. After the three
+// digits (11, 11, 10 bits) the threshold key and the number of tied tokens
+// to take are known; the CTAs exchange their counts of sure keeps and ties
+// and write the kept indices in index order. No global scratch besides the
+// status word; cluster barriers (hardware, all CTAs co-resident) separate
+// the steps.
+constexpr int kCThreads = 1024;
+constexpr int kCChunk = kCThreads * kPerThread;  // tokens per CTA
+constexpr int kCMaxCtas = 16;
+constexpr int64_t kClusterMaxN = int64_t(kCMaxCtas) * kCChunk;  // 131072
+
+// Exclusive prefix over the 1024 threads of a CTA (thread order); *total
+// receives the CTA sum. Uses the caller's 32-word scratch.
+__device__ __forceinline__ uint32_t cta_excl_scan_1024(uint32_t v, uint32_t* total,
+                                                       uint32_t* warp_sums) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    uint32_t w = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sums[lane] = w;  // inclusive
+  }
+  __syncthreads();
+  const uint32_t before_warp = wid ? warp_sums[wid - 1] : 0u;
+  if (total) *total = warp_sums[31];
+  const uint32_t r = before_warp + x - v;
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
+template <bool kVec>
+__global__ void __launch_bounds__(kCThreads, 1)
+    sel_cluster(const float* __restrict__ scores, const uint8_t* __restrict__ protect, int64_t n,
+                int64_t k, int32_t* __restrict__ kept_idx, int32_t* __restrict__ status) {
+  __shared__ uint32_t hist[2048];   // this CTA's counts of the current digit
+  __shared__ uint32_t red[2048];    // cluster sums of this CTA's slice of the bins
+  __shared__ uint32_t cta_val[4];   // 0: slice total, 1: sure keeps, 2: ties, 3: protected
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t s_bin, s_need;
+  pdl_trigger();
+  const int tid = threadIdx.x;
+  const uint32_t C = gridDim.x;  // the grid is one cluster
+  const uint32_t rank = cluster_ctarank();
+  pdl_wait();
+  uint32_t key[kPerThread];
+  bool prot[kPerThread];
+  const int64_t first = static_cast<int64_t>(rank) * kCChunk + static_cast<int64_t>(tid) * kPerThread;
+  const int valid = load_tokens<kVec>(scores, protect, n, first, key, prot);
+  uint32_t np_t = 0;
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j)
+    if (j < valid && prot[j]) ++np_t;
+  uint32_t np_cta;
+  cta_excl_scan_1024(np_t, &np_cta, warp_sums);
+  if (tid == 0) cta_val[3] = np_cta;
+  cluster_sync();
+  uint32_t np = 0;
+  for (uint32_t r = 0; r < C; ++r) np += ld_cluster_u32(mapa_shared(smem_addr(&cta_val[3]), r));
+  const bool over = static_cast<int64_t>(np) > k;
+  uint32_t thresh = 0xFFFFFFFFu, ties = 0u;  // np == k: no unprotected token is kept
+  uint32_t need = over ? 0u : static_cast<uint32_t>(k - static_cast<int64_t>(np));
+  if (need > 0u) {
+    uint32_t prefix = 0u;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+      const int bins = pass == 2 ? 1024 : 2048;
+      const int pbits = pass == 0 ? 0 : (pass == 1 ? 11 : 22);  // prefix bits so far
+      for (int i = tid; i < bins; i += kCThreads) hist[i] = 0u;
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < kPerThread; ++j) {
+        if (j < valid && !prot[j] &&
+            (pass == 0 || (key[j] >> (32 - pbits)) == prefix))
+          atomicAdd(&hist[(key[j] >> shift) & static_cast<uint32_t>(bins - 1)], 1u);
+      }
+      cluster_sync();
+      // this CTA's slice of the bins, summed over the cluster
+      const uint32_t S = static_cast<uint32_t>(bins) / C;
+      uint32_t part = 0u;
+      for (uint32_t t = tid; t < S; t += kCThreads) {
+        const uint32_t b = rank * S + t;
+        uint32_t sum = 0u;
+        for (uint32_t r = 0; r < C; ++r) sum += ld_cluster_u32(mapa_shared(smem_addr(&hist[b]), r));
+        red[t] = sum;
+        part += sum;
+      }
+      uint32_t slice_tot;
+      cta_excl_scan_1024(part, &slice_tot, warp_sums);
+      if (tid == 0) cta_val[0] = slice_tot;
+      cluster_sync();
+      // the slice (from the top) where the count reaches `need`, then the bin
+      if (tid == 0) {
+        uint32_t above = 0u, sl = 0u;
+        for (int r = static_cast<int>(C) - 1; r >= 0; --r) {
+          const uint32_t t = ld_cluster_u32(mapa_shared(smem_addr(&cta_val[0]), r));
+          if (above + t >= need) {
+            sl = static_cast<uint32_t>(r);
+            break;
+          }
+          above += t;
+        }
+        s_bin = sl;
+        s_need = need - above;
+      }
+      __syncthreads();
+      const uint32_t sl = s_bin, rest = s_need;
+      // slice sl's bins in descending order: thread t holds elements
+      // 2t, 2t + 1 (element e = bin S - 1 - e of the slice)
+      uint32_t v[2] = {0u, 0u};
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const uint32_t e = 2u * tid + q;
+        if (e < S) v[q] = ld_cluster_u32(mapa_shared(smem_addr(&red[S - 1 - e]), sl));
+      }
+      const uint32_t before = cta_excl_scan_1024(v[0] + v[1], nullptr, warp_sums);
+      if (before < rest && rest <= before + v[0] + v[1]) {
+        const uint32_t e = before + v[0] >= rest ? 2u * tid : 2u * tid + 1u;
+        s_bin = sl * S + (S - 1 - e);
+        s_need = rest - (e == 2u * tid ? before : before + v[0]);
+      }
+      __syncthreads();
+      prefix = pass == 0 ? s_bin : ((prefix << (pass == 1 ? 11 : 10)) | s_bin);
+      need = s_need;
+      __syncthreads();  // s_bin / s_need are rewritten by the next pass
+    }
+    thresh = prefix;
+    ties = need;
+  }
+  if (over) {
+    if (rank == 0 && tid == 0) *status = 3;
+    for (int64_t i = static_cast<int64_t>(rank) * kCThreads + tid; i < k;
+         i += static_cast<int64_t>(C) * kCThreads)
+      kept_idx[i] = -1;
+    cluster_sync();  // no CTA leaves while another may still read its shared memory
+    return;
+  }
+  // sure keeps and ties of this thread, CTA and the CTAs before it
+  uint32_t nd = 0u, nt = 0u;
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j) {
+    if (j < valid) {
+      if (prot[j] || key[j] > thresh) ++nd;
+      else if (key[j] == thresh) ++nt;
+    }
+  }
+  uint32_t nd_cta, nt_cta;
+  uint32_t sb = cta_excl_scan_1024(nd, &nd_cta, warp_sums);
+  uint32_t tb = cta_excl_scan_1024(nt, &nt_cta, warp_sums);
+  if (tid == 0) {
+    cta_val[1] = nd_cta;
+    cta_val[2] = nt_cta;
+  }
+  cluster_sync();
+  for (uint32_t r = 0; r < rank; ++r) {
+    sb += ld_cluster_u32(mapa_shared(smem_addr(&cta_val[1]), r));
+    tb += ld_cluster_u32(mapa_shared(smem_addr(&cta_val[2]), r));
+  }
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j) {
+    if (j < valid) {
+      const bool sure = prot[j] || key[j] > thresh;
+      const bool tie = !sure && key[j] == thresh;
+      if (sure) {
+        const uint32_t pos = sb + min(tb, ties);
+        if (pos < static_cast<uint64_t>(k)) kept_idx[pos] = static_cast<int32_t>(first + j);
+        ++sb;
+      } else if (tie) {
+        if (tb < ties) {
+          const uint32_t pos = sb + tb;
+          if (pos < static_cast<uint64_t>(k)) kept_idx[pos] = static_cast<int32_t>(first + j);
+        }
+        ++tb;
+      }
+    }
+  }
+  if (rank == 0 && tid == 0) *status = 0;
+  cluster_sync();  // no CTA leaves while another may still read its shared memory
+}
+
+// Cluster size for n tokens (0: n is past the one-launch path).
+int cluster_ctas(int64_t n) {
+  static int max_ctas = 0;  // 16 where the device can co-schedule it, else 8
+  static std::once_flag once;
+  std::call_once(once, [] {
+    max_ctas = 8;
+    auto kern = sel_cluster<true>;
+    if (cudaFuncSetAttribute(reinterpret_cast<const void*>(kern),
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+        cudaFuncSetAttribute(reinterpret_cast<const void*>(sel_cluster<false>),
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(16);
+      cfg.blockDim = dim3(kCThreads);
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 16;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters >= 1)
+        max_ctas = 16;
+    }
+    cudaGetLastError();  // a refused attribute is not an error of a later call
+  });
+  if (n > kClusterMaxN) return 0;
+  int c = 1;
+  while (int64_t(c) * kCChunk < n) c *= 2;
+  return c <= max_ctas ? c : 0;
+}
+
+template <bool kVec>
+cudaError_t run_select_cluster(const float* scores, const uint8_t* protect, int64_t n, int64_t k,
+                               int32_t* kept_idx, void* ws, int ctas, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  cfg.blockDim = dim3(kCThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(ctas);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, sel_cluster<kVec>, scores, protect, n, k, kept_idx,
+                            static_cast<int32_t*>(ws));
+}
+
 template <bool kVec>
 cudaError_t run_select(const float* scores, const uint8_t* protect, int64_t n, int64_t k,
                        int32_t* kept_idx, void* ws, cudaStream_t st) {
@@ -476,6 +733,10 @@ cudaError_t launch_topk_select(const float* scores, const uint8_t* protect, int6
                                int32_t* kept_idx, void* ws, cudaStream_t st) {
   const bool vec = (reinterpret_cast<uintptr_t>(scores) % 16 == 0) &&
                    (protect == nullptr || reinterpret_cast<uintptr_t>(protect) % 8 == 0);
+  const int ctas = cluster_ctas(n);
+  if (ctas > 0)
+    return vec ? run_select_cluster<true>(scores, protect, n, k, kept_idx, ws, ctas, st)
+               : run_select_cluster<false>(scores, protect, n, k, kept_idx, ws, ctas, st);
   return vec ? run_select<true>(scores, protect, n, k, kept_idx, ws, st)
              : run_select<false>(scores, protect, n, k, kept_idx, ws, st);
 }

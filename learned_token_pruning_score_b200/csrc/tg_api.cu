@@ -143,9 +143,14 @@ struct AttnPlan {
   void* vT = nullptr;     // bf16: [hkv, dh, t_pad]
   float* lsig = nullptr;  // [k]
   void* kaug = nullptr;   // bf16 [k, 16] gate-bias rows (tensor-core path)
+  void* split = nullptr;  // scratch for split query tiles of short sequences
+  size_t split_bytes = 0;
   int64_t t_pad = 0;
   size_t bytes = 0;
-  AttnPlan(void* ws, int64_t k, int hq, int hkv, int dh, tg_dtype dt, bool need_k) {
+  // split_rows: the shortest sequence this plan's attention will run (its
+  // split scratch is sized for it; 0: none)
+  AttnPlan(void* ws, int64_t k, int hq, int hkv, int dh, tg_dtype dt, bool need_k,
+           int64_t split_rows = 0) {
     Arena a(ws);
     const size_t e = elem_size(dt);
     t_pad = static_cast<int64_t>(align_up(static_cast<size_t>(k), 64));
@@ -154,6 +159,10 @@ struct AttnPlan {
     if (dt == TG_BF16) vT = a.carve(size_t(hkv) * dh * t_pad * e);
     lsig = static_cast<float*>(a.carve(size_t(k) * 4 + 16));
     if (dt == TG_BF16) kaug = a.carve(size_t(k) * 32);
+    if (dt == TG_BF16 && dh == 128 && split_rows > 0) {
+      split_bytes = attn_split_bytes(split_rows, hq, hkv);
+      if (split_bytes > 0) split = a.carve(split_bytes);
+    }
     bytes = a.used;
   }
 };
@@ -178,6 +187,12 @@ struct GdnPlan {
     bytes = ar.used;
   }
 };
+
+// The four launches of the Gated DeltaNet mixer over g.T tokens (prep with
+// the carried conv rows, per-chunk matrices, the recurrence, the gated norm).
+cudaError_t gdn_run(const GdnArgs& g, bool bf, cudaStream_t st);
+int64_t gdn_channels(const tg_gdn_layer& G);
+int64_t gdn_proj_width(const tg_gdn_layer& G);
 
 struct AttnBwdF32Plan {
   float* q_rot = nullptr;   // [n, hq, dh]
@@ -231,6 +246,9 @@ struct AttnBwdPlan {
   }
 };
 
+// Rows per block of the FFN sub-layer (its intermediate [rows, I] buffer).
+constexpr int64_t kFfnRows = 16384;
+
 struct PrefillPlan {
   void* h = nullptr;       // [n, d] residual stream (all-token stage)
   void* hk = nullptr;      // [k, d] residual stream (kept rows)
@@ -249,20 +267,30 @@ struct PrefillPlan {
   float2* cs_n = nullptr;  // [dh/2][n] cos/sin of positions 0..n-1 (dense stage)
   float2* cs_k = nullptr;  // [dh/2][k] cos/sin of the kept positions
   AttnPlan attn;           // sized for n rows, reused by every layer
+  // hybrid stacks (Gated DeltaNet layers): projections, mixer output, mixer
+  // workspace, sized for n rows and the widest such layer
+  void* gdn_proj = nullptr;
+  void* gdn_y = nullptr;
+  void* gdn_ws = nullptr;
   size_t bytes = 0;
+  // (the attention's split scratch serves any gated layer of up to 8192 rows)
   PrefillPlan(void* ws, const tg_model& m, int64_t n, int64_t k)
-      : attn(nullptr, n, m.n_heads_q, m.n_heads_kv, m.head_dim, m.dtype, true) {
+      : attn(nullptr, n, m.n_heads_q, m.n_heads_kv, m.head_dim, m.dtype, true, 1) {
     Arena a(ws);
     const size_t e = elem_size(m.dtype);
     const int d = m.d_model, hq = m.n_heads_q, hkv = m.n_heads_kv, dh = m.head_dim;
     h = a.carve(size_t(n) * d * e);
     hk = a.carve(size_t(k) * d * e);
     y = a.carve(size_t(n) * d * e);
-    qkv = a.carve(size_t(n) * (hq + 2 * hkv) * dh * e);
+    // the un-fused projection path only: bf16 attention with head_dim 128 and
+    // paired query heads projects straight into q / k / V^T (QKV epilogue)
+    if (!(m.dtype == TG_BF16 && dh == 128 && hq % 2 == 0))
+      qkv = a.carve(size_t(n) * (hq + 2 * hkv) * dh * e);
     attn_o = a.carve(size_t(n) * hq * dh * e);
-    if (m.d_ffn > 0) {
-      mlp = a.carve(size_t(n) * m.d_ffn * e);
-      if (m.dtype == TG_F32) gu = a.carve(size_t(n) * 2 * m.d_ffn * 4);
+    if (m.d_ffn > 0) {  // the FFN runs in row blocks of at most kFfnRows
+      const size_t fr = static_cast<size_t>(std::min<int64_t>(n, kFfnRows));
+      mlp = a.carve(fr * m.d_ffn * e);
+      if (m.dtype == TG_F32) gu = a.carve(fr * 2 * m.d_ffn * 4);
     }
     scores = static_cast<float*>(a.carve(size_t(n) * 4));
     if (m.dtype == TG_F32) hpre = static_cast<float*>(a.carve(size_t(n) * m.d_score * 4));
@@ -274,7 +302,21 @@ struct PrefillPlan {
     cs_n = static_cast<float2*>(a.carve(size_t(n) * (dh / 2) * sizeof(float2)));
     cs_k = static_cast<float2*>(a.carve(size_t(k) * (dh / 2) * sizeof(float2)));
     void* attn_base = a.carve(attn.bytes);
-    attn = AttnPlan(attn_base, n, hq, hkv, dh, m.dtype, true);
+    attn = AttnPlan(attn_base, n, hq, hkv, dh, m.dtype, true, 1);
+    size_t proj_w = 0, y_w = 0, gws = 0;
+    for (int l = 0; l < m.n_layers; ++l) {
+      const tg_gdn_layer* G = m.layers[l].gdn;
+      if (G == nullptr) continue;
+      proj_w = std::max(proj_w, static_cast<size_t>(gdn_proj_width(*G)));
+      y_w = std::max(y_w, static_cast<size_t>(G->n_heads_v) * G->head_dim_v);
+      gws = std::max(gws, GdnPlan(nullptr, n, G->n_heads_k, G->n_heads_v, G->head_dim_k,
+                                  G->head_dim_v).bytes);
+    }
+    if (proj_w > 0) {
+      gdn_proj = a.carve(size_t(n) * proj_w * e);
+      gdn_y = a.carve(size_t(n) * y_w * e);
+      gdn_ws = a.carve(gws);
+    }
     bytes = a.used;
   }
 };
@@ -365,7 +407,8 @@ cudaError_t run_score(const void* x, int64_t rows, int d, int f, const float* no
 cudaError_t attn_core(const AttnPlan& plan, const void* k_rot, const void* v, int64_t v_stride,
                       const float* lsig, const void* kaug, const float* gain, const float* tau,
                       int64_t rows, int hq, int hkv, int dh, tg_dtype dt, void* out,
-                      cudaStream_t st, float* lse = nullptr, float* out_f32 = nullptr) {
+                      cudaStream_t st, float* lse = nullptr, float* out_f32 = nullptr,
+                      bool split_cnt_zeroed = false) {
   const size_t es = elem_size(dt);
   const double attn_flops = 4.0 * dh * hq * double(rows) * double(rows + 1) / 2.0;
   const double attn_bytes = double(rows) * (2 * hq + 2 * hkv) * dh * es;
@@ -379,6 +422,9 @@ cudaError_t attn_core(const AttnPlan& plan, const void* k_rot, const void* v, in
   a.out = out;
   a.lse = lse;
   a.out_f32 = out_f32;
+  a.split_ws = plan.split;
+  a.split_ws_bytes = plan.split_bytes;
+  a.split_cnt_zeroed = split_cnt_zeroed;
   if (dt == TG_BF16) {
     a.v = plan.vT;
     a.t_pad = plan.t_pad;
@@ -457,6 +503,9 @@ cudaError_t attn_segments(const AttnPlan& plan, const void* k_rot, const float* 
     a.tau = tau;
     a.T = rows; a.hq = hq; a.hkv = hkv; a.dh = dh;
     a.out = static_cast<char*>(out) + size_t(off) * hq * dh * e;
+    a.split_ws = plan.split;
+    a.split_ws_bytes = plan.split_bytes;
+    a.split_cnt_zeroed = true;
     if (!attn_tc_supported(a)) return cudaErrorInvalidValue;
     const double fl = 4.0 * dh * hq * double(rows) * double(rows + 1) / 2.0;
     const double by = double(rows) * (2 * hq + 2 * hkv) * dh * e;
@@ -491,8 +540,8 @@ cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims
                           P.attn_o, st);
     else
       err = attn_core(P.attn, k_dst, nullptr, 0, lsig, kaug, gain, tau, rows, D.hq, D.hkv, D.dh,
-                      dt, P.attn_o, st);
-  } else if (segs != nullptr) {
+                      dt, P.attn_o, st, nullptr, nullptr, true);
+  } else if (segs != nullptr || P.qkv == nullptr) {
     return cudaErrorInvalidValue;  // packed requests need the fused bf16 path
   } else {
     err = gemm(gemm_args(P.y, D.d, lw.wqkv, D.d, P.qkv, D.qkv, rows, D.qkv, D.d, EPI_STORE), dt,
@@ -523,28 +572,127 @@ cudaError_t ffn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
                          const PrefillPlan& P, void* h, int64_t rows, cudaStream_t st) {
   if (lw.w_gate_up == nullptr) return cudaSuccess;
   const tg_dtype dt = m.dtype;
+  const size_t e = elem_size(dt);
   cudaError_t err = rmsnorm(h, lw.ffn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
   if (err != cudaSuccess) return err;
-  if (dt == TG_BF16) {
-    GemmArgs g = gemm_args(P.y, D.d, lw.w_gate_up, D.d, P.mlp, D.inter, rows, 2 * D.inter, D.d,
-                           EPI_SWIGLU);
-    g.inter = D.inter;
+  // row blocks of at most kFfnRows share the intermediate buffer
+  for (int64_t r0 = 0; r0 < rows; r0 += kFfnRows) {
+    const int64_t rb = std::min<int64_t>(kFfnRows, rows - r0);
+    const char* yb = static_cast<const char*>(P.y) + size_t(r0) * D.d * e;
+    void* hb = static_cast<char*>(h) + size_t(r0) * D.d * e;
+    if (dt == TG_BF16) {
+      GemmArgs g = gemm_args(yb, D.d, lw.w_gate_up, D.d, P.mlp, D.inter, rb, 2 * D.inter, D.d,
+                             EPI_SWIGLU);
+      g.inter = D.inter;
+      err = gemm(g, dt, st);
+    } else {
+      err = gemm(gemm_args(yb, D.d, lw.w_gate_up, D.d, P.gu, 2 * D.inter, rb, 2 * D.inter, D.d,
+                           EPI_STORE), dt, st);
+      if (err == cudaSuccess)
+        err = traced(TG_K_F32_HELPER, rb, 0.0, double(rb) * D.inter * 12.0, st, [&] {
+          return launch_swiglu_f32(static_cast<const float*>(P.gu), rb, D.inter,
+                                   static_cast<float*>(P.mlp), st);
+        });
+    }
+    if (err != cudaSuccess) return err;
+    GemmArgs g = gemm_args(P.mlp, D.inter, lw.w_down, D.inter, hb, D.d, rb, D.d, D.inter,
+                           EPI_RESIDUAL);
+    g.R = hb;
+    g.ldr = D.d;
     err = gemm(g, dt, st);
-  } else {
-    err = gemm(gemm_args(P.y, D.d, lw.w_gate_up, D.d, P.gu, 2 * D.inter, rows, 2 * D.inter, D.d,
-                         EPI_STORE), dt, st);
-    if (err == cudaSuccess)
-      err = traced(TG_K_F32_HELPER, rows, 0.0, double(rows) * D.inter * 12.0, st, [&] {
-        return launch_swiglu_f32(static_cast<const float*>(P.gu), rows, D.inter,
-                                 static_cast<float*>(P.mlp), st);
-      });
+    if (err != cudaSuccess) return err;
   }
+  return cudaSuccess;
+}
+
+cudaError_t gdn_run(const GdnArgs& g, bool bf, cudaStream_t st) {
+  const int64_t T = g.T;
+  const double C = double(2 * g.hk * g.dk + g.hv * g.dv);
+  const double e = bf ? 2.0 : 4.0, tt = double(T);
+  const double prep_bytes = tt * (C * e + 2.0 * g.hv * e) + tt * 4.0 * (C + g.hv * 2.0);
+  const double chunk_flops = tt * g.hv * 2.0 * kGdnChunk * g.dk;  // the two Gram products
+  const double recur_flops = tt * g.hv * 6.0 * g.dv * g.dk;
+  const double out_bytes = tt * g.hv * g.dv * (4.0 + 2.0 * e);
+  cudaError_t err =
+      traced(TG_K_GDN_PREP, T, 0.0, prep_bytes, st, [&] { return launch_gdn(g, bf, 0, st); });
+  if (err == cudaSuccess)
+    err = traced(TG_K_GDN_CHUNK, T, chunk_flops, 0.0, st, [&] { return launch_gdn(g, bf, 1, st); });
+  if (err == cudaSuccess)
+    err = traced(TG_K_GDN_RECUR, T, recur_flops, 0.0, st, [&] { return launch_gdn(g, bf, 2, st); });
+  if (err == cudaSuccess)
+    err = traced(TG_K_GDN_OUT, T, 0.0, out_bytes, st, [&] { return launch_gdn(g, bf, 3, st); });
+  return err;
+}
+
+// A hybrid model's Gated DeltaNet layer (token mixer part) over `rows` rows
+// of h: h += W_out . mixer(W_in . RMSNorm(h)), the mixer running over each
+// sequence (one, or each packed request of `segs`) in row order. kv, when
+// given, receives the last conv rows (k) and the final state (v).
+cudaError_t gdn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
+                         const PrefillPlan& P, void* h, int64_t rows, const tg_kv* kv,
+                         cudaStream_t st, const SegRows* segs, const tg_layer_taps* taps) {
+  const tg_gdn_layer& G = *lw.gdn;
+  const tg_dtype dt = m.dtype;
+  const size_t e = elem_size(dt);
+  const int64_t C = gdn_channels(G), Nt = gdn_proj_width(G);
+  const int hv = G.n_heads_v, vd = G.n_heads_v * G.head_dim_v;
+  cudaError_t err = rmsnorm(h, lw.attn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
   if (err != cudaSuccess) return err;
-  GemmArgs g = gemm_args(P.mlp, D.inter, lw.w_down, D.inter, h, D.d, rows, D.d, D.inter,
-                         EPI_RESIDUAL);
+  err = gemm(gemm_args(P.y, D.d, lw.w_in, D.d, P.gdn_proj, Nt, rows, static_cast<int>(Nt), D.d,
+                       EPI_STORE), dt, st);
+  if (err != cudaSuccess) return err;
+  const int n_seq = segs ? segs->count : 1;
+  for (int b = 0; b < n_seq; ++b) {
+    const int64_t off = segs ? segs->off[b] : 0, len = segs ? segs->len[b] : rows;
+    GdnArgs g = GdnPlan(P.gdn_ws, len, G.n_heads_k, hv, G.head_dim_k, G.head_dim_v).a;
+    const char* pr = static_cast<const char*>(P.gdn_proj) + size_t(off) * Nt * e;
+    g.qkv = pr;
+    g.z = pr + size_t(C) * e;
+    g.a = pr + size_t(C + vd) * e;
+    g.b = pr + size_t(C + vd + hv) * e;
+    g.ld_qkv = g.ld_z = g.ld_ab = Nt;
+    g.T = len;
+    g.hk = G.n_heads_k;
+    g.hv = hv;
+    g.dk = G.head_dim_k;
+    g.dv = G.head_dim_v;
+    g.W = G.conv_width;
+    g.conv_w = G.conv_w;
+    g.A_log = G.A_log;
+    g.dt_bias = G.dt_bias;
+    g.norm_w = G.norm_w;
+    g.eps = G.norm_eps;
+    g.conv_in = nullptr;
+    g.state_in = nullptr;
+    g.conv_out = (kv && !segs) ? kv->k : nullptr;
+    g.state_out = (kv && !segs) ? static_cast<float*>(kv->v) : nullptr;
+    g.y = static_cast<char*>(P.gdn_y) + size_t(off) * vd * e;
+    g.err = device_error_word();
+    err = gdn_run(g, dt == TG_BF16, st);
+    if (err != cudaSuccess) return err;
+  }
+  if (taps && taps->attn_out) {
+    err = copy_rows(taps->attn_out, P.gdn_y, size_t(rows) * vd * e, rows, st);
+    if (err != cudaSuccess) return err;
+  }
+  GemmArgs g = gemm_args(P.gdn_y, vd, lw.w_out, vd, h, D.d, rows, D.d, vd, EPI_RESIDUAL);
   g.R = h;
   g.ldr = D.d;
-  return gemm(g, dt, st);
+  err = gemm(g, dt, st);
+  if (err != cudaSuccess || !taps || !taps->resid) return err;
+  return copy_rows(taps->resid, h, size_t(rows) * D.d * e, rows, st);
+}
+
+// The token-mixer sub-layer of layer lw: attention, or the Gated DeltaNet
+// mixer of a hybrid model's linear-attention layer.
+cudaError_t mixer_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
+                           const PrefillPlan& P, void* h, int64_t rows, const int32_t* pos,
+                           const float2* cs, const float* lsig, const void* kaug,
+                           const float* gain, const float* tau, const tg_kv* kv, cudaStream_t st,
+                           const SegRows* segs = nullptr, const tg_layer_taps* taps = nullptr) {
+  if (lw.gdn != nullptr) return gdn_sublayer(m, lw, D, P, h, rows, kv, st, segs, taps);
+  return attention_sublayer(m, lw, D, P, h, rows, pos, cs, lsig, kaug, gain, tau, kv, st, segs,
+                            taps);
 }
 
 // Workspace of one decode step (batch 1, bf16).
@@ -601,6 +749,7 @@ tg_status validate_decode(const tg_model* m, const void* x, int64_t pos, int gat
   }
   for (int l = 0; l < m->n_layers; ++l) {
     const tg_layer& L = m->layers[l];
+    TG_CHECK(L.gdn == nullptr, TG_ERR_UNSUPPORTED);  // attention layers only
     TG_CHECK(L.attn_norm && L.wqkv && L.wo, TG_ERR_INVALID_ARG);
     TG_CHECK((L.q_norm == nullptr) == (L.k_norm == nullptr), TG_ERR_INVALID_ARG);
     if (L.w_gate_up) TG_CHECK(L.w_down && L.ffn_norm && m->d_ffn > 0, TG_ERR_INVALID_ARG);
@@ -614,6 +763,29 @@ tg_status validate_decode(const tg_model* m, const void* x, int64_t pos, int gat
     // above the gate the kept prompt tokens are the first k_kept cache rows
     if (l > gate_layer && scores != nullptr) TG_CHECK(lens[l] >= k_kept, TG_ERR_INVALID_ARG);
   }
+  return TG_OK;
+}
+
+// Columns of a Gated DeltaNet layer's input projection: qkv (C channels),
+// z (hv dv), a and b (hv each).
+int64_t gdn_channels(const tg_gdn_layer& G) {
+  return 2 * int64_t(G.n_heads_k) * G.head_dim_k + int64_t(G.n_heads_v) * G.head_dim_v;
+}
+int64_t gdn_proj_width(const tg_gdn_layer& G) {
+  return gdn_channels(G) + int64_t(G.n_heads_v) * G.head_dim_v + 2 * int64_t(G.n_heads_v);
+}
+
+tg_status validate_gdn_layer(const tg_gdn_layer* L) {
+  TG_CHECK(L != nullptr, TG_ERR_INVALID_ARG);
+  TG_CHECK(L->n_heads_k >= 1 && L->n_heads_v >= 1 && L->n_heads_v % L->n_heads_k == 0 &&
+               L->n_heads_v <= 4096,
+           TG_ERR_INVALID_ARG);
+  TG_CHECK(L->conv_width >= 1 && L->conv_width <= 4, TG_ERR_INVALID_ARG);
+  TG_CHECK(L->conv_w && L->A_log && L->dt_bias && L->norm_w, TG_ERR_INVALID_ARG);
+  TG_CHECK(std::isfinite(L->norm_eps) && L->norm_eps >= 0.f, TG_ERR_INVALID_ARG);
+  TG_CHECK(L->head_dim_k == 64 || L->head_dim_k == 128, TG_ERR_UNSUPPORTED);
+  TG_CHECK(L->head_dim_v >= 32 && L->head_dim_v <= 256 && L->head_dim_v % 32 == 0,
+           TG_ERR_UNSUPPORTED);
   return TG_OK;
 }
 
@@ -632,8 +804,17 @@ tg_status validate_model(const tg_model* m, int64_t n, int64_t k, int gate_layer
   const int d = m->d_model, dh = m->head_dim, qkv = (m->n_heads_q + 2 * m->n_heads_kv) * dh;
   for (int l = 0; l < m->n_layers; ++l) {
     const tg_layer& L = m->layers[l];
-    TG_CHECK(L.attn_norm && L.wqkv && L.wo, TG_ERR_INVALID_ARG);
-    TG_CHECK((L.q_norm == nullptr) == (L.k_norm == nullptr), TG_ERR_INVALID_ARG);
+    if (L.gdn != nullptr) {  // a hybrid model's Gated DeltaNet layer
+      const tg_status gs = validate_gdn_layer(L.gdn);
+      if (gs != TG_OK) return gs;
+      TG_CHECK(L.attn_norm && L.w_in && L.w_out, TG_ERR_INVALID_ARG);
+      TG_CHECK(m->dtype == TG_BF16, TG_ERR_UNSUPPORTED);
+      TG_CHECK(gdn_proj_width(*L.gdn) % 32 == 0, TG_ERR_UNSUPPORTED);
+      TG_CHECK(aligned16(L.w_in) && aligned16(L.w_out), TG_ERR_INVALID_ARG);
+    } else {
+      TG_CHECK(L.attn_norm && L.wqkv && L.wo, TG_ERR_INVALID_ARG);
+      TG_CHECK((L.q_norm == nullptr) == (L.k_norm == nullptr), TG_ERR_INVALID_ARG);
+    }
     if (L.w_gate_up) TG_CHECK(L.w_down && L.ffn_norm && m->d_ffn > 0, TG_ERR_INVALID_ARG);
   }
   bool any_ffn = false;
@@ -666,7 +847,8 @@ size_t tg_workspace_size(tg_op op, const tg_shape* s) {
     case TG_OP_COMPACT:
       return 0;
     case TG_OP_GATED_ATTN:
-      return AttnPlan(nullptr, s->k, s->n_heads_q, s->n_heads_kv, s->head_dim, s->dtype, true).bytes;
+      return AttnPlan(nullptr, s->k, s->n_heads_q, s->n_heads_kv, s->head_dim, s->dtype, true,
+                      s->k).bytes;
     case TG_OP_GATED_ATTN_BWD:
       if (s->dtype == TG_F32)
         return AttnBwdF32Plan(nullptr, s->k, s->n_heads_q, s->n_heads_kv, s->head_dim).bytes;
@@ -781,9 +963,9 @@ tg_status gated_attn(const void* q, const void* kk, const void* v, const int32_t
   } else {
     TG_CHECK(dh == 64 || dh == 128, TG_ERR_UNSUPPORTED);
   }
-  AttnPlan plan(nullptr, k, hq, hkv, dh, dt, true);
+  AttnPlan plan(nullptr, k, hq, hkv, dh, dt, true, k);
   TG_CHECK(ws != nullptr && ws_bytes >= plan.bytes, TG_ERR_WORKSPACE);
-  plan = AttnPlan(ws, k, hq, hkv, dh, dt, true);
+  plan = AttnPlan(ws, k, hq, hkv, dh, dt, true, k);
   return cuda_status(run_attention(q, int64_t(hq) * dh, kk, int64_t(hkv) * dh, v,
                                    int64_t(hkv) * dh, pos, s, nullptr, gain, tau, nullptr, nullptr,
                                    0.f, k, hq, hkv, dh, rope_base, dt, plan, nullptr, nullptr, out,
@@ -934,6 +1116,8 @@ tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan
                              const tg_layer_taps* taps, float* sc, cudaStream_t st) {
   const size_t e = elem_size(m.dtype);
   TG_TRY(copy_rows(P.h, x, size_t(n) * D.d * e, n, st));
+  // every attention launch of the call then finds its split counters zero
+  TG_TRY(attn_split_clear(P.attn.split, P.attn.split_bytes, D.hq, st));
   const bool tables = m.dtype == TG_BF16 && D.dh == 128;
   const double cs_bytes = 8.0 * (D.dh / 2);
   if (tables && gate_layer >= 0)
@@ -942,7 +1126,7 @@ tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan
     }));
   for (int l = 0; l < gate_layer; ++l) {
     LayerTag tag(l);
-    TG_TRY(attention_sublayer(m, m.layers[l], D, P, P.h, n, nullptr, P.cs_n, nullptr, nullptr,
+    TG_TRY(mixer_sublayer(m, m.layers[l], D, P, P.h, n, nullptr, P.cs_n, nullptr, nullptr,
                               nullptr, nullptr, kv ? &kv[l] : nullptr, st, nullptr,
                               taps ? &taps[l] : nullptr));
     TG_TRY(ffn_sublayer(m, m.layers[l], D, P, P.h, n, st));
@@ -951,7 +1135,7 @@ tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan
   }
   if (gate_layer >= 0) {
     LayerTag tag(gate_layer);
-    TG_TRY(attention_sublayer(m, m.layers[gate_layer], D, P, P.h, n, nullptr, P.cs_n, nullptr,
+    TG_TRY(mixer_sublayer(m, m.layers[gate_layer], D, P, P.h, n, nullptr, P.cs_n, nullptr,
                               nullptr, nullptr, nullptr, kv ? &kv[gate_layer] : nullptr, st,
                               nullptr, taps ? &taps[gate_layer] : nullptr));
   }
@@ -991,7 +1175,7 @@ tg_status prefill_above_gate(const tg_model& m, const Dims& D, const PrefillPlan
   for (int l = gate_layer + 1; l < m.n_layers; ++l) {
     LayerTag tag(l);
     const tg_layer& L = m.layers[l];
-    TG_TRY(attention_sublayer(m, L, D, P, P.hk, k, P.pos_k, P.cs_k, P.lsig_k, P.kaug_k, L.gain,
+    TG_TRY(mixer_sublayer(m, L, D, P, P.hk, k, P.pos_k, P.cs_k, P.lsig_k, P.kaug_k, L.gain,
                               L.tau, kv ? &kv[l] : nullptr, st, nullptr,
                               taps ? &taps[l] : nullptr));
     TG_TRY(ffn_sublayer(m, L, D, P, P.hk, k, st));
@@ -1060,6 +1244,11 @@ tg_status batch_layout(const tg_model* model, const int64_t* cu_n, const int64_t
 
 extern "C" {
 
+size_t tg_prefill_workspace_size(const tg_model* model, int64_t n, int64_t k) {
+  if (model == nullptr || model->layers == nullptr || n < 1 || k < 1 || k > n) return 0;
+  return PrefillPlan(nullptr, *model, n, k).bytes;
+}
+
 tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protect, int64_t n,
                      int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx, float* scores,
                      const tg_kv* kv, const tg_layer_taps* taps, void* ws, size_t ws_bytes,
@@ -1069,6 +1258,9 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
   TG_CHECK(x && out && kept_idx, TG_ERR_INVALID_ARG);
   const tg_model& m = *model;
   if (m.dtype == TG_BF16) TG_CHECK(aligned16(x) && aligned16(out), TG_ERR_INVALID_ARG);
+  if (m.dtype == TG_BF16 && kv != nullptr)  // written by the QKV GEMM's epilogue
+    for (int l = 0; l < m.n_layers; ++l)
+      TG_CHECK(aligned16(kv[l].k) && aligned16(kv[l].v), TG_ERR_INVALID_ARG);
   PrefillPlan P(nullptr, m, n, k);
   TG_CHECK(ws != nullptr && ws_bytes >= P.bytes, TG_ERR_WORKSPACE);
   P = PrefillPlan(ws, m, n, k);
@@ -1144,6 +1336,7 @@ tg_status tg_prefill_batch(const tg_model* model, const void* x, const uint8_t* 
   const size_t row = size_t(D.d) * e;
   char* h = static_cast<char*>(P.h);
   char* hk = static_cast<char*>(P.hk);
+  TG_TRY(attn_split_clear(P.attn.split, P.attn.split_bytes, D.hq, st));
   // packed rows in, padding rows zero
   for (int b = 0; b < batch; ++b) {
     const int64_t n = sn.len[b], pad = static_cast<int64_t>(align_up(size_t(n), kSegAlign)) - n;
@@ -1159,13 +1352,13 @@ tg_status tg_prefill_batch(const tg_model* model, const void* x, const uint8_t* 
   // below the gate: projections over every request's rows, attention per request
   for (int l = 0; l < gate_layer; ++l) {
     LayerTag tag(l);
-    TG_TRY(attention_sublayer(m, m.layers[l], D, P, P.h, n_pad, nullptr, P.cs_n, nullptr, nullptr,
+    TG_TRY(mixer_sublayer(m, m.layers[l], D, P, P.h, n_pad, nullptr, P.cs_n, nullptr, nullptr,
                               nullptr, nullptr, nullptr, st, &sn));
     TG_TRY(ffn_sublayer(m, m.layers[l], D, P, P.h, n_pad, st));
   }
   if (gate_layer >= 0) {
     LayerTag tag(gate_layer);
-    TG_TRY(attention_sublayer(m, m.layers[gate_layer], D, P, P.h, n_pad, nullptr, P.cs_n, nullptr,
+    TG_TRY(mixer_sublayer(m, m.layers[gate_layer], D, P, P.h, n_pad, nullptr, P.cs_n, nullptr,
                               nullptr, nullptr, nullptr, nullptr, st, &sn));
   }
   float* sc = P.scores;
@@ -1200,7 +1393,7 @@ tg_status tg_prefill_batch(const tg_model* model, const void* x, const uint8_t* 
   for (int l = gate_layer + 1; l < m.n_layers; ++l) {
     LayerTag tag(l);
     const tg_layer& L = m.layers[l];
-    TG_TRY(attention_sublayer(m, L, D, P, P.hk, k_pad, P.pos_k, P.cs_k, P.lsig_k, P.kaug_k, L.gain,
+    TG_TRY(mixer_sublayer(m, L, D, P, P.hk, k_pad, P.pos_k, P.cs_k, P.lsig_k, P.kaug_k, L.gain,
                               L.tau, nullptr, st, &sk));
     TG_TRY(ffn_sublayer(m, L, D, P, P.hk, k_pad, st));
   }
@@ -1373,20 +1566,6 @@ tg_status tg_decode_step(const tg_model* model, const void* x, int64_t pos, int3
 
 // ---- Gated DeltaNet mixer
 namespace {
-tg_status validate_gdn_layer(const tg_gdn_layer* L) {
-  TG_CHECK(L != nullptr, TG_ERR_INVALID_ARG);
-  TG_CHECK(L->n_heads_k >= 1 && L->n_heads_v >= 1 && L->n_heads_v % L->n_heads_k == 0 &&
-               L->n_heads_v <= 4096,
-           TG_ERR_INVALID_ARG);
-  TG_CHECK(L->conv_width >= 1 && L->conv_width <= 4, TG_ERR_INVALID_ARG);
-  TG_CHECK(L->conv_w && L->A_log && L->dt_bias && L->norm_w, TG_ERR_INVALID_ARG);
-  TG_CHECK(std::isfinite(L->norm_eps) && L->norm_eps >= 0.f, TG_ERR_INVALID_ARG);
-  TG_CHECK(L->head_dim_k == 64 || L->head_dim_k == 128, TG_ERR_UNSUPPORTED);
-  TG_CHECK(L->head_dim_v >= 32 && L->head_dim_v <= 256 && L->head_dim_v % 32 == 0,
-           TG_ERR_UNSUPPORTED);
-  return TG_OK;
-}
-
 bool overlaps(const void* p, size_t pn, const void* q, size_t qn) {
   const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
   return a < b + qn && b < a + pn;
@@ -1426,6 +1605,9 @@ tg_status tg_gated_deltanet(const tg_gdn_layer* L, const void* qkv, const void* 
   g.z = z;
   g.a = a;
   g.b = b;
+  g.ld_qkv = static_cast<int64_t>(C);
+  g.ld_z = int64_t(hv) * dv;
+  g.ld_ab = hv;
   g.T = T;
   g.hk = hk;
   g.hv = hv;
@@ -1443,17 +1625,7 @@ tg_status tg_gated_deltanet(const tg_gdn_layer* L, const void* qkv, const void* 
   g.state_out = state_out;
   g.y = y;
   g.err = device_error_word();
-  const bool bf = dtype == TG_BF16;
-  const double e = double(elem_size(dtype)), tt = double(T);
-  const double prep_bytes = tt * (C * e + 2.0 * hv * e) + tt * 4.0 * (C + hv * 2.0);
-  const double chunk_flops = tt * hv * 2.0 * kGdnChunk * dk;  // the two Gram products (full square)
-  const double recur_flops = tt * hv * 6.0 * dv * dk;
-  const double out_bytes = tt * hv * dv * (4.0 + 2.0 * e);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  TG_TRY(traced(TG_K_GDN_PREP, T, 0.0, prep_bytes, st, [&] { return launch_gdn(g, bf, 0, st); }));
-  TG_TRY(traced(TG_K_GDN_CHUNK, T, chunk_flops, 0.0, st, [&] { return launch_gdn(g, bf, 1, st); }));
-  TG_TRY(traced(TG_K_GDN_RECUR, T, recur_flops, 0.0, st, [&] { return launch_gdn(g, bf, 2, st); }));
-  TG_TRY(traced(TG_K_GDN_OUT, T, 0.0, out_bytes, st, [&] { return launch_gdn(g, bf, 3, st); }));
+  TG_TRY(gdn_run(g, dtype == TG_BF16, reinterpret_cast<cudaStream_t>(stream)));
   return TG_OK;
 }
 

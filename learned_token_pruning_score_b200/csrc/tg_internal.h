@@ -161,7 +161,19 @@ struct AttnArgs {
   void* out;                                    // [T, hq, dh]
   float* lse;      // optional [hq, T]: log sum_j exp(l_ij) per row (tensor-core path only)
   float* out_f32;  // optional [T, hq, dh]: the output before rounding (tensor-core path only)
+  // optional scratch for split query tiles of short sequences
+  // (attn_split_bytes); split_cnt_zeroed: its counters are already zero (the
+  // kernel leaves them zero after every launch)
+  void* split_ws = nullptr;
+  size_t split_ws_bytes = 0;
+  bool split_cnt_zeroed = false;
 };
+// Scratch the tensor-core attention over T rows can use to split long query
+// tiles across CTAs (0 when T is too long to need it).
+size_t attn_split_bytes(int64_t T, int hq, int hkv);
+// Zeroes the split counters of such scratch (before the first launch that
+// passes split_cnt_zeroed = true).
+cudaError_t attn_split_clear(void* split_ws, size_t split_ws_bytes, int hq, cudaStream_t st);
 bool attn_tc_supported(const AttnArgs& a);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st);      // bf16, tcgen05
 cudaError_t launch_attn_simt_f32(const AttnArgs& a, cudaStream_t st); // fp32 SIMT
@@ -273,6 +285,7 @@ struct GdnArgs {
   const void* z;          // [T, hv dv] output gate
   const void* a;          // [T, hv] decay input
   const void* b;          // [T, hv] write-strength input
+  int64_t ld_qkv, ld_z, ld_ab;  // row strides (elements) of qkv, z and a / b
   int64_t T;
   int64_t t_pad;
   int hk, hv, dk, dv, W;

@@ -302,3 +302,71 @@ def gdn_inputs(w: GdnWorkload, rng: np.random.Generator, T: Optional[int] = None
         "a": rng.standard_normal((T, w.hv), dtype=np.float32),
         "b": rng.standard_normal((T, w.hv), dtype=np.float32),
     }
+
+
+@dataclass(frozen=True)
+class HybridWorkload:
+    """A hybrid decoder stack: `kinds` gives each layer's token mixer
+    ("gdn": Gated DeltaNet, "attn": full attention); the attention layers
+    use `base`'s heads and every layer `base`'s FFN; the Gated DeltaNet
+    layers have hk / hv heads of dim dk / dv and convolution width W."""
+    base: Workload
+    kinds: Tuple[str, ...]
+    hk: int
+    hv: int
+    dk: int
+    dv: int
+    W: int
+
+
+# Qwen3.5-2B-like hybrid stack: three Gated DeltaNet layers to one
+# full-attention layer, d_model 2048 (the pages name the model and its gate
+# positions, layers 1 to 3, but not its sizes; the Qwen3-Next-style mixer
+# shape and Qwen3-1.7B-style attention heads stand in). N = 4096, K = 1024.
+HYBRID_4K = HybridWorkload(
+    Workload("hybrid_qwen35_like_n4k_k1k", "bf16", n=4096, k=1024, d=2048, hq=16, hkv=8, dh=128,
+             f=256, inter=6144, n_layers=8, gate_layer=1, n_protect=64, seed=6, qk_norm=True),
+    kinds=("gdn", "gdn", "gdn", "attn", "gdn", "gdn", "gdn", "attn"),
+    hk=16, hv=16, dk=128, dv=128, W=4)
+
+
+def torch_hybrid_params(w: HybridWorkload, seed: int, device: str = "cuda"):
+    """Device-side draws of a hybrid stack, like `torch_model_params`: the
+    attention layers as there; a Gated DeltaNet layer has attn_norm (the
+    norm before the mixer) = 1, w_in [C + hv dv + 2 hv, d] and w_out
+    [d, hv dv] ~ N(0, w_std), and fp32 mixer parameters conv_w [C, W] ~
+    U(+-1/sqrt(W)), A_log = log U(1, 16), dt_bias ~ U(-7, -2) and norm_w ~
+    1 + 0.1 N(0, 1) (C = 2 hk dk + hv dv)."""
+    import math
+
+    import torch
+
+    b = w.base
+    p = torch_model_params(b, seed, device)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 7919)
+    dt = torch.bfloat16 if b.dtype == "bf16" else torch.float32
+    C = 2 * w.hk * w.dk + w.hv * w.dv
+
+    def normal(*shape, std=b.w_std):
+        t = torch.empty(*shape, device=device, dtype=torch.float32)
+        return t.normal_(0.0, std, generator=g)
+
+    def unif(shape, lo, hi):
+        t = torch.empty(*shape, device=device, dtype=torch.float32)
+        return t.uniform_(lo, hi, generator=g)
+
+    for li, kind in enumerate(w.kinds):
+        if kind != "gdn":
+            continue
+        lp = p["layers"][li]
+        for key in ("wqkv", "wo", "q_norm", "k_norm", "gain", "tau"):
+            lp.pop(key, None)
+        lp["w_in"] = normal(C + w.hv * w.dv + 2 * w.hv, b.d).to(dt)
+        lp["w_out"] = normal(b.d, w.hv * w.dv).to(dt)
+        lim = 1.0 / math.sqrt(w.W)
+        lp["gdn_params"] = {"conv_w": unif((C, w.W), -lim, lim),
+                            "A_log": torch.log(unif((w.hv,), 1.0, 16.0)),
+                            "dt_bias": unif((w.hv,), -7.0, -2.0),
+                            "norm_w": 1.0 + 0.1 * normal(w.dv, std=1.0)}
+    return p

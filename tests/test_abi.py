@@ -149,6 +149,7 @@ def _bogus_model(**over):
             setattr(layers[i], name, 4096)
         layers[i].q_norm = None
         layers[i].k_norm = None
+        layers[i].gdn = None  # attention layers
     m = tg.TgModel(tg.TG_BF16, 2, 2048, 16, 8, 128, 6144, 256, 1e-6, 1e6, layers, 4096, 4096,
                    4096, None, 4096, None)
     for k, v in over.items():
@@ -339,3 +340,30 @@ def test_selftest_wait_validation():
     assert f(0, 2_000_000_000, BOGUS, None, 0, None) == tg.TG_ERR_INVALID_ARG  # above 1 s
     assert f(0, 2_000_000, None, None, 0, None) == tg.TG_ERR_INVALID_ARG  # no result buffer
     assert f(2, 2_000_000, BOGUS, None, 0, None) == tg.TG_ERR_WORKSPACE  # barrier words
+
+
+def test_prefill_validation_hybrid_layers():
+    """A Gated DeltaNet layer (hybrid stack): the mixer's sizes, the input
+    projection's width (a multiple of 32 for the tensor-core GEMM) and the
+    dtype are checked on the host."""
+    m, keep = _bogus_model()
+    big = 1 << 40
+    gdn = tg.TgGdnLayer(4, 16, 64, 32, 4, 4096, 4096, 4096, 4096, 1e-6)  # width 1568 = 49 * 32
+    keep[0].gdn = ctypes.addressof(gdn)
+    assert tg._prefill_ws(ctypes.byref(m), 1000, 100) > \
+        tg.tg_workspace_size(tg.TG_OP_PREFILL, n=1000, k=100, d_model=2048, n_heads_q=16,
+                             n_heads_kv=8, head_dim=128, d_score=256, d_ffn=6144, n_layers=2,
+                             gate_layer=1, dtype=tg.TG_BF16)
+    assert _prefill(ctypes.byref(m), 1000, 100, 1, 16) == tg.TG_ERR_WORKSPACE  # passes validation
+    bad = tg.TgGdnLayer(4, 16, 96, 32, 4, 4096, 4096, 4096, 4096, 1e-6)  # dk 96
+    keep[0].gdn = ctypes.addressof(bad)
+    assert _prefill(ctypes.byref(m), 1000, 100, 1, big) == tg.TG_ERR_UNSUPPORTED
+    odd = tg.TgGdnLayer(2, 4, 64, 64, 4, 4096, 4096, 4096, 4096, 1e-6)  # width 520
+    keep[0].gdn = ctypes.addressof(odd)
+    assert _prefill(ctypes.byref(m), 1000, 100, 1, big) == tg.TG_ERR_UNSUPPORTED
+    keep[0].gdn = ctypes.addressof(gdn)
+    keep[0].w_in = None
+    assert _prefill(ctypes.byref(m), 1000, 100, 1, big) == tg.TG_ERR_INVALID_ARG
+    m32, keep32 = _bogus_model(dtype=tg.TG_F32)
+    keep32[1].gdn = ctypes.addressof(gdn)
+    assert _prefill(ctypes.byref(m32), 1000, 100, 1, big) == tg.TG_ERR_UNSUPPORTED

@@ -103,6 +103,34 @@ def test_attn_bf16_qwen_heads_k2048():
     _attn_case(2048, 16, 8, 128, torch.bfloat16, 6, max_pos=16384)
 
 
+@pytest.mark.parametrize("t", [512, 1024, 1536])
+def test_attn_bf16_qwen_heads_short_sequences(t):
+    """Short sequences run a table schedule in which long query tiles are
+    split across CTAs (parts merged by the last one to finish): 16 / 8 heads
+    at lengths whose schedules split tiles into 2 to 4 parts."""
+    _attn_case(t, 16, 8, 128, torch.bfloat16, 20 + t, max_pos=4 * t)
+
+
+def test_attn_bf16_split_schedule_is_deterministic():
+    """Which part of a split query tile finishes last varies from run to run;
+    the merge takes the parts in a fixed order, so the bits do not."""
+    rng = np.random.default_rng(31)
+    t, hq, hkv = 2048, 16, 8
+    q = dev(rng.standard_normal((t, hq, 128)), torch.bfloat16)
+    k = dev(rng.standard_normal((t, hkv, 128)), torch.bfloat16)
+    v = dev(rng.standard_normal((t, hkv, 128)), torch.bfloat16)
+    pos = torch.from_numpy(np.sort(rng.choice(8 * t, t, replace=False)).astype(np.int32)).cuda()
+    s = dev(rng.standard_normal(t) * 2)
+    gain = dev(rng.uniform(0, 2, hq))
+    tau = dev(rng.uniform(0.5, 1.5, hq))
+    runs = [tg.tg_gated_attn_forward(q, k, v, pos, s, gain, tau) for _ in range(3)]
+    torch.cuda.synchronize()
+    for out, lse, o32 in runs[1:]:
+        assert torch.equal(out, runs[0][0])
+        assert torch.equal(lse, runs[0][1])
+        assert torch.equal(o32, runs[0][2])
+
+
 @pytest.mark.parametrize("dh", [64, 128])
 def test_attn_fp32(dh):
     _attn_case(128, 4, 2, dh, torch.float32, 7 + dh, max_pos=512)
