@@ -9,7 +9,10 @@ of the path (dense layers over N, scorer, select, compact, gated layers over
 K, final norm).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-    python bench.py --sweep      # select+compact sweep and the 128K gated layer
+    python bench.py --sweep      # select+compact sweep, the 16K and 128K layers alone
+    python bench.py --case attn|attn_bwd|layer|gemm|decode|gdn [--rows R]
+                                 # one kernel family alone: the commands the ncu
+                                 # summaries under profiles/ were captured with
 
 Prints one JSON line (rank 0). `value` = tokens/s (N / TTFT) summed over the
 ranks; ranks run independent replicas (the path has no exchange step).
@@ -41,7 +44,17 @@ HEADLINE_K = 4096
 SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-LAUNCHES_PER_RECORD = {"select": 5, "rope_prep": 2, "copy": 0}
+# library kernels behind one traced record (the rest: one each). The select
+# is one cluster launch up to 131072 tokens, else five kernels; a copy is a
+# cudaMemcpyAsync, not a kernel of the library.
+LAUNCHES_PER_RECORD = {"rope_prep": 2, "copy": 0}
+SELECT_ONE_LAUNCH_MAX_N = 131072
+
+
+def launches_of(rec) -> int:
+    if rec["kernel"] == "select":
+        return 1 if rec["rows"] <= SELECT_ONE_LAUNCH_MAX_N else 5
+    return LAUNCHES_PER_RECORD.get(rec["kernel"], 1)
 
 
 def peaks():
@@ -448,7 +461,7 @@ def run_ours(args, rank, world, local_rank):
         e["ms"] += r["ms"]
         e["flops"] += r["flops"]
         e["bytes"] += r["bytes"]
-        e["launches"] += LAUNCHES_PER_RECORD.get(r["kernel"], 1)
+        e["launches"] += launches_of(r)
         e["records"] += 1
     traced_ms = sum(e["ms"] for e in per.values())
     by_kernel = {}
@@ -765,7 +778,7 @@ def _traced(tg, torch, fn, reps, flush):
         e["ms"] += r["ms"] / reps
         e["flops"] += r["flops"] / reps
         e["bytes"] += r["bytes"] / reps
-        e["launches"] += LAUNCHES_PER_RECORD.get(r["kernel"], 1) / reps
+        e["launches"] += launches_of(r) / reps
     return out
 
 

@@ -677,7 +677,8 @@ cudaError_t launch_step(DecStepParams p, cudaStream_t st) {
 // Self-test of the grid barrier's bounded wait: one CTA of consumers waits
 // for a barrier that no CTA arrives at (words[0] = 0 < target 1). After
 // limit_ns the wait gives up, records the timeout in err and sets the abort
-// word (words[1]); result[0] = 1 if bar_wait returned false, as it must.
+// word (words[1]); result[0] = 1 if the wait completed, 0 if it gave up (as
+// it must here).
 __global__ void __launch_bounds__(kConsumers, 1)
     dec_selftest_gridbar(unsigned* words, unsigned* err, unsigned long long limit_ns,
                          int* result) {
@@ -685,7 +686,7 @@ __global__ void __launch_bounds__(kConsumers, 1)
   GridBar bar{words, words + 1, err, 1u};
   bar.limit_ns = limit_ns;
   const bool ok = bar_wait(bar, &s_ok);
-  if (threadIdx.x == 0) result[0] = ok ? 0 : 1;
+  if (threadIdx.x == 0) result[0] = ok ? 1 : 0;
 }
 
 }  // namespace

@@ -425,19 +425,36 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
   return v;
 }
 
+// Sum over the CTA's 1024 threads into *dst (zeroed by the caller before
+// the __syncthreads that precedes this call); every thread sees the sum after
+// the call's __syncthreads.
+__device__ __forceinline__ uint32_t cta_sum_1024(uint32_t v, uint32_t* dst) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  if ((threadIdx.x & 31) == 0 && v) atomicAdd(dst, v);
+  __syncthreads();
+  return *dst;
+}
+
 template <bool kVec>
 __global__ void __launch_bounds__(kCThreads, 1)
     sel_cluster(const float* __restrict__ scores, const uint8_t* __restrict__ protect, int64_t n,
                 int64_t k, int32_t* __restrict__ kept_idx, int32_t* __restrict__ status) {
   __shared__ uint32_t hist[2048];   // this CTA's counts of the current digit
   __shared__ uint32_t red[2048];    // cluster sums of this CTA's slice of the bins
-  __shared__ uint32_t cta_val[4];   // 0: slice total, 1: sure keeps, 2: ties, 3: protected
+  __shared__ uint32_t cta_val[4];   // 0 / 3: slice total of even / odd passes (another
+                                    // CTA may still read a pass's slot during the next
+                                    // pass), 1: sure keeps | ties (16 + 16 bits),
+                                    // 2: protected
+  __shared__ uint32_t tot[kCMaxCtas];
   __shared__ uint32_t warp_sums[32];
   __shared__ uint32_t s_bin, s_need;
   pdl_trigger();
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
   const uint32_t C = gridDim.x;  // the grid is one cluster
   const uint32_t rank = cluster_ctarank();
+  if (tid < 4) cta_val[tid] = 0u;
+  __syncthreads();
   pdl_wait();
   uint32_t key[kPerThread];
   bool prot[kPerThread];
@@ -447,12 +464,12 @@ __global__ void __launch_bounds__(kCThreads, 1)
 #pragma unroll
   for (int j = 0; j < kPerThread; ++j)
     if (j < valid && prot[j]) ++np_t;
-  uint32_t np_cta;
-  cta_excl_scan_1024(np_t, &np_cta, warp_sums);
-  if (tid == 0) cta_val[3] = np_cta;
+  cta_sum_1024(np_t, &cta_val[2]);
   cluster_sync();
+  if (tid < static_cast<int>(C)) tot[tid] = ld_cluster_u32(mapa_shared(smem_addr(&cta_val[2]), tid));
+  __syncthreads();
   uint32_t np = 0;
-  for (uint32_t r = 0; r < C; ++r) np += ld_cluster_u32(mapa_shared(smem_addr(&cta_val[3]), r));
+  for (uint32_t r = 0; r < C; ++r) np += tot[r];
   const bool over = static_cast<int64_t>(np) > k;
   uint32_t thresh = 0xFFFFFFFFu, ties = 0u;  // np == k: no unprotected token is kept
   uint32_t need = over ? 0u : static_cast<uint32_t>(k - static_cast<int64_t>(np));
@@ -463,13 +480,18 @@ __global__ void __launch_bounds__(kCThreads, 1)
       const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
       const int bins = pass == 2 ? 1024 : 2048;
       const int pbits = pass == 0 ? 0 : (pass == 1 ? 11 : 22);  // prefix bits so far
+      uint32_t* slice_tot = &cta_val[(pass & 1) ? 3 : 0];  // last read two passes ago
       for (int i = tid; i < bins; i += kCThreads) hist[i] = 0u;
+      if (tid == 0) *slice_tot = 0u;
       __syncthreads();
+      // warp-aggregated: one shared-memory atomic per distinct bin per warp
 #pragma unroll
       for (int j = 0; j < kPerThread; ++j) {
-        if (j < valid && !prot[j] &&
-            (pass == 0 || (key[j] >> (32 - pbits)) == prefix))
-          atomicAdd(&hist[(key[j] >> shift) & static_cast<uint32_t>(bins - 1)], 1u);
+        const bool act = j < valid && !prot[j] &&
+                         (pass == 0 || (key[j] >> (32 - pbits)) == prefix);
+        const uint32_t bin = act ? (key[j] >> shift) & static_cast<uint32_t>(bins - 1) : 0xFFFFFFFFu;
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+        if (act && (__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], __popc(peers));
       }
       cluster_sync();
       // this CTA's slice of the bins, summed over the cluster
@@ -482,26 +504,20 @@ __global__ void __launch_bounds__(kCThreads, 1)
         red[t] = sum;
         part += sum;
       }
-      uint32_t slice_tot;
-      cta_excl_scan_1024(part, &slice_tot, warp_sums);
-      if (tid == 0) cta_val[0] = slice_tot;
+      cta_sum_1024(part, slice_tot);
       cluster_sync();
       // the slice (from the top) where the count reaches `need`, then the bin
-      if (tid == 0) {
-        uint32_t above = 0u, sl = 0u;
-        for (int r = static_cast<int>(C) - 1; r >= 0; --r) {
-          const uint32_t t = ld_cluster_u32(mapa_shared(smem_addr(&cta_val[0]), r));
-          if (above + t >= need) {
-            sl = static_cast<uint32_t>(r);
-            break;
-          }
-          above += t;
-        }
-        s_bin = sl;
-        s_need = need - above;
-      }
+      if (tid < static_cast<int>(C)) tot[tid] = ld_cluster_u32(mapa_shared(smem_addr(slice_tot), tid));
       __syncthreads();
-      const uint32_t sl = s_bin, rest = s_need;
+      uint32_t above = 0u, sl = 0u;
+      for (int r = static_cast<int>(C) - 1; r >= 0; --r) {
+        if (above + tot[r] >= need) {
+          sl = static_cast<uint32_t>(r);
+          break;
+        }
+        above += tot[r];
+      }
+      const uint32_t rest = need - above;
       // slice sl's bins in descending order: thread t holds elements
       // 2t, 2t + 1 (element e = bin S - 1 - e of the slice)
       uint32_t v[2] = {0u, 0u};
@@ -519,7 +535,6 @@ __global__ void __launch_bounds__(kCThreads, 1)
       __syncthreads();
       prefix = pass == 0 ? s_bin : ((prefix << (pass == 1 ? 11 : 10)) | s_bin);
       need = s_need;
-      __syncthreads();  // s_bin / s_need are rewritten by the next pass
     }
     thresh = prefix;
     ties = need;
@@ -532,7 +547,8 @@ __global__ void __launch_bounds__(kCThreads, 1)
     cluster_sync();  // no CTA leaves while another may still read its shared memory
     return;
   }
-  // sure keeps and ties of this thread, CTA and the CTAs before it
+  // sure keeps and ties of this thread, CTA and the CTAs before it, as one
+  // packed count (sure << 16 | ties; at most 8192 of each per CTA)
   uint32_t nd = 0u, nt = 0u;
 #pragma unroll
   for (int j = 0; j < kPerThread; ++j) {
@@ -541,17 +557,16 @@ __global__ void __launch_bounds__(kCThreads, 1)
       else if (key[j] == thresh) ++nt;
     }
   }
-  uint32_t nd_cta, nt_cta;
-  uint32_t sb = cta_excl_scan_1024(nd, &nd_cta, warp_sums);
-  uint32_t tb = cta_excl_scan_1024(nt, &nt_cta, warp_sums);
-  if (tid == 0) {
-    cta_val[1] = nd_cta;
-    cta_val[2] = nt_cta;
-  }
+  uint32_t packed_cta;
+  const uint32_t packed = cta_excl_scan_1024((nd << 16) | nt, &packed_cta, warp_sums);
+  if (tid == 0) cta_val[1] = packed_cta;
   cluster_sync();
+  if (tid < static_cast<int>(rank)) tot[tid] = ld_cluster_u32(mapa_shared(smem_addr(&cta_val[1]), tid));
+  __syncthreads();
+  uint32_t sb = packed >> 16, tb = packed & 0xFFFFu;
   for (uint32_t r = 0; r < rank; ++r) {
-    sb += ld_cluster_u32(mapa_shared(smem_addr(&cta_val[1]), r));
-    tb += ld_cluster_u32(mapa_shared(smem_addr(&cta_val[2]), r));
+    sb += tot[r] >> 16;
+    tb += tot[r] & 0xFFFFu;
   }
 #pragma unroll
   for (int j = 0; j < kPerThread; ++j) {
