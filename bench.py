@@ -10,7 +10,7 @@ K, final norm).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
     python bench.py --sweep      # select+compact sweep, the 16K and 128K layers alone
-    python bench.py --case attn|attn_bwd|layer|gemm|decode|gdn [--rows R]
+    python bench.py --case attn|attn_bwd|layer|gemm|decode|gdn|score|select [--rows R]
                                  # one kernel family alone: the commands the ncu
                                  # summaries under profiles/ were captured with
 
@@ -748,7 +748,10 @@ def run_ours(args, rank, world, local_rank):
 
 def _events_median(torch, fn, reps, flush, stream):
     """Median device ms of `reps` calls of fn (CUDA events on `stream`), L2
-    flushed before each call (outside the events), after one untimed call."""
+    flushed before each call (outside the events), after one untimed call.
+    A spin kernel queued before each timed call keeps the GPU busy while the
+    host enqueues the call, so a short call's events see its device time,
+    not the host's launch latency."""
     fn()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -756,6 +759,7 @@ def _events_median(torch, fn, reps, flush, stream):
     for a, b in evs:
         if flush is not None:
             flush.zero_()
+        torch.cuda._sleep(200000)  # ~0.1 ms: longer than the host's enqueue of fn
         a.record(stream)
         fn()
         b.record(stream)
@@ -1158,6 +1162,38 @@ def run_case(args):
         print(json.dumps({"case": "decode", "rows": t, "steps": args.steps,
                           "ms_per_token": res["ms_per_token"], "gbs": res["gbs"]}))
         return 0
+    if args.case == "select":
+        # tg_topk_select then tg_compact of `rows` sweep-style scores, K = rows / 8
+        n, kk = t, max(1, t // 8)
+        rng = synth.rng_for(synth.SWEEP_SEED)
+        s = torch.from_numpy(synth.sweep_scores(n, rng)).to(device)
+        prot = torch.from_numpy(synth.protect_tail(n, synth.SWEEP_PROTECT)).to(device)
+        x = torch.randn(n, synth.SWEEP_D, device=device, dtype=torch.bfloat16)
+        idx = torch.empty(kk, dtype=torch.int32, device=device)
+        ws = torch.empty(tg.tg_workspace_size(tg.TG_OP_TOPK_SELECT, n=n), dtype=torch.uint8,
+                         device=device)
+        for _ in range(args.steps):
+            tg.tg_topk_select(s, prot, kk, kept_idx=idx, ws=ws)
+            tg.tg_compact(x, idx, scores=s)
+        torch.cuda.synchronize()
+        assert tg.tg_device_error() == 0
+        print(json.dumps({"case": "select", "rows": t, "k": kk, "reps": args.steps}))
+        return 0
+    if args.case == "score":
+        # tg_score over `rows` rows of d_model 2048 into the 256-wide scorer
+        x = torch.randn(t, w.d, device=device, dtype=torch.bfloat16)
+        nw = torch.ones(w.d, device=device)
+        w1 = (torch.randn(w.f, w.d, device=device) * 0.02).to(torch.bfloat16)
+        w2 = torch.randn(w.f, device=device) * 0.02
+        sc = torch.empty(t, device=device)
+        ws = torch.empty(tg.tg_workspace_size(tg.TG_OP_SCORE, n=t, d_model=w.d, d_score=w.f,
+                                              dtype=tg.TG_BF16), dtype=torch.uint8, device=device)
+        for _ in range(args.steps):
+            tg.tg_score(x, nw, w1, w2, scores=sc, ws=ws)
+        torch.cuda.synchronize()
+        assert tg.tg_device_error() == 0
+        print(json.dumps({"case": "score", "rows": t, "reps": args.steps}))
+        return 0
     if args.case == "attn_bwd":
         res = attn_backward_bench(tg, torch, w.hq, w.hkv, w.dh, t, args.steps, device,
                                   bias=not args.no_bias)
@@ -1222,7 +1258,8 @@ def main():
     ap.add_argument("--quick", action="store_true", help="skip the other budgets / dense run")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--sweep", action="store_true")
-    ap.add_argument("--case", choices=["attn", "attn_bwd", "layer", "gemm", "decode", "gdn"],
+    ap.add_argument("--case", choices=["attn", "attn_bwd", "layer", "gemm", "decode", "gdn", "score",
+                                       "select"],
                     default=None)
     ap.add_argument("--rows", type=int, default=32768)
     ap.add_argument("--no-bias", action="store_true",

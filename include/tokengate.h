@@ -252,6 +252,19 @@ tg_status tg_gated_attn_backward(const void* q, const void* kk, const void* v, c
 tg_status tg_linear(const void* x, const void* w, const void* residual, int64_t m, int32_t n,
                     int32_t k, tg_dtype dtype, void* y, tg_stream stream);
 
+/*
+ * tg_fold_norm_weight -- W_g[j, i] = bf16(W[j, i] * g[i]): a projection
+ * weight with the weight g of the RMSNorm in front of it folded in, for the
+ * optional wqkv_g / w_gate_up_g / score_w1_g fields (the RMSNorm of
+ * [TC] "TokenGate 提前筛选 Token"'s Qwen3 backbone and of the scorer's input
+ * is y = x / sqrt(mean(x^2) + eps) * g, so y . W^T = (x . W_g^T) / rms(x)).
+ * Device pointers: w and out [rows, cols] bf16 (out must not overlap w),
+ * g [cols] fp32. rows, cols >= 1, else TG_ERR_INVALID_ARG, as for NULL
+ * pointers. One kernel on `stream`, exact (one rounding per element).
+ */
+tg_status tg_fold_norm_weight(const void* w, const float* g, int64_t rows, int64_t cols, void* out,
+                              tg_stream stream);
+
 /* ---- hybrid models: the Gated DeltaNet mixer -----------------------------
  *
  * In a hybrid model most layers are Gated DeltaNet layers and only some are
@@ -305,6 +318,20 @@ typedef struct {
   const void* w_in;       /* [C + hv dv + 2 hv, d]: rows giving qkv (C = 2 hk dk
                              + hv dv channels), then z, then a, then b          */
   const void* w_out;      /* [d, hv dv]                                         */
+  /* Optional (bf16): the projections that read an RMSNorm-ed row, with that
+   * norm's weight folded in, W_g[j, i] = bf16(W[j, i] g[i]) (made by
+   * tg_fold_norm_weight): wqkv_g from wqkv and attn_norm, w_gate_up_g from
+   * w_gate_up and ffn_norm. RMSNorm(x; g) . W^T = (x . W_g^T) / rms(x), so
+   * with them a sub-layer whose input rows were just written by a residual
+   * GEMM runs no RMSNorm kernel: that GEMM's epilogue leaves each row's sum
+   * of squares (of the stored bf16 values) and the projection's epilogue
+   * scales its accumulator row by 1 / rms(x) = 1 / sqrt(mean(x^2) + eps).
+   * The rounding differs from the norm-then-project order only in where one
+   * bf16 rounding falls (on W g instead of on the normed row). NULL: the
+   * RMSNorm kernel and the plain weights (also used for rows that were not
+   * just written by a residual GEMM: the stack's input, the compacted rows). */
+  const void* wqkv_g;      /* [(hq + 2 hkv) dh, d] or NULL (unused with gdn)     */
+  const void* w_gate_up_g; /* [2 I, d] or NULL                                   */
 } tg_layer;
 
 typedef struct {
@@ -318,6 +345,8 @@ typedef struct {
   const float* score_b1;    /* [F] or NULL                                   */
   const float* score_w2;    /* [F]                                           */
   const float* score_b2;    /* [1] or NULL                                   */
+  const void* score_w1_g;   /* [F, d] score_w1 with score_norm folded in (as
+                               tg_layer.wqkv_g), or NULL                     */
 } tg_model;
 
 /* Per-layer KV outputs (post-RoPE keys, values), each [rows, hkv, dh] dtype.
@@ -527,7 +556,8 @@ typedef enum {
   TG_K_GDN_CHUNK = 21,       /* Gated DeltaNet: per-chunk solve matrices             */
   TG_K_GDN_RECUR = 22,       /* Gated DeltaNet: the state across the chunks          */
   TG_K_GDN_OUT = 23,         /* Gated DeltaNet: gated output RMSNorm                 */
-  TG_K_COUNT = 24
+  TG_K_FOLD_NORM = 24,       /* tg_fold_norm_weight                                  */
+  TG_K_COUNT = 25
 } tg_kernel;
 
 typedef struct {

@@ -47,7 +47,8 @@ class TgShape(ctypes.Structure):
 
 class TgLayer(ctypes.Structure):
     _fields_ = [(n, _c_p) for n in ("attn_norm", "wqkv", "q_norm", "k_norm", "wo", "ffn_norm",
-                                    "w_gate_up", "w_down", "gain", "tau", "gdn", "w_in", "w_out")]
+                                    "w_gate_up", "w_down", "gain", "tau", "gdn", "w_in", "w_out",
+                                    "wqkv_g", "w_gate_up_g")]
 
 
 class TgModel(ctypes.Structure):
@@ -56,7 +57,8 @@ class TgModel(ctypes.Structure):
                 ("d_ffn", _c_i32), ("d_score", _c_i32), ("norm_eps", _c_f32),
                 ("rope_base", _c_f32), ("layers", ctypes.POINTER(TgLayer)),
                 ("final_norm", _c_p), ("score_norm", _c_p), ("score_w1", _c_p),
-                ("score_b1", _c_p), ("score_w2", _c_p), ("score_b2", _c_p)]
+                ("score_b1", _c_p), ("score_w2", _c_p), ("score_b2", _c_p),
+                ("score_w1_g", _c_p)]
 
 
 class TgKV(ctypes.Structure):
@@ -91,6 +93,7 @@ _score = _sig("tg_score", _ci, _c_p, _c_i64, _c_i32, _c_i32, _c_p, _c_f32, _c_p,
               _ci, _c_p, _c_p, _c_sz, _c_p)
 _topk = _sig("tg_topk_select", _ci, _c_p, _c_p, _c_i64, _c_i64, _c_p, _c_p, _c_sz, _c_p)
 _linear = _sig("tg_linear", _ci, _c_p, _c_p, _c_p, _c_i64, _c_i32, _c_i32, _ci, _c_p, _c_p)
+_fold = _sig("tg_fold_norm_weight", _ci, _c_p, _c_p, _c_i64, _c_i64, _c_p, _c_p)
 _topk_noalloc = _sig("tg_topk_select_noalloc", _ci, _c_p, _c_p, _c_i64, _c_i64, _c_p, _c_p)
 _compact = _sig("tg_compact", _ci, _c_p, _c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i32, _ci, _c_p,
                 _c_p, _c_p, _c_p)
@@ -266,6 +269,17 @@ def tg_linear(x, w, residual=None, y=None, stream=None) -> torch.Tensor:
     return y
 
 
+def tg_fold_norm_weight(w, g, out=None, stream=None) -> torch.Tensor:
+    """W_g = bf16(W . diag(g)): w [rows, cols] bf16, g [cols] fp32 (the weight
+    of the RMSNorm in front of the projection w)."""
+    rows, cols = w.shape
+    if out is None:
+        out = torch.empty_like(w)
+    _check(_fold(_ptr(w), _ptr(g), rows, cols, _ptr(out), _stream(stream, w.device)),
+           "tg_fold_norm_weight")
+    return out
+
+
 SELECT_NOALLOC_MAX_N = 1 << 20
 
 
@@ -426,6 +440,11 @@ class Model:
     A hybrid model's Gated DeltaNet layer has instead of wqkv/wo the keys gdn
     (a GdnLayer: the mixer's parameters), w_in [C + hv dv + 2 hv, d] and
     w_out [d, hv dv]; attn_norm is then the norm before the mixer.
+
+    fold_norms (bf16): also keep wqkv, w_gate_up and score_w1 with the weight
+    of the RMSNorm in front of each folded in (tg_fold_norm_weight, made once
+    here), so that tg_prefill skips the norm kernels whose input rows come
+    straight from a residual GEMM.
     """
 
     n_heads_q: int
@@ -436,6 +455,7 @@ class Model:
     final_norm: Optional[torch.Tensor] = None
     eps: float = 1e-6
     rope_base: float = 1e6
+    fold_norms: bool = True
 
     def __post_init__(self):
         w = next(lw["wqkv"] if "wqkv" in lw else lw["w_in"] for lw in self.layers)
@@ -445,12 +465,28 @@ class Model:
                   None)
         self.d_ffn = 0 if gu is None else gu.shape[0] // 2
         self.d_score = self.score["score_w1"].shape[0]
+        fold = self.fold_norms and self.dtype == TG_BF16
+        self.fold_norms = fold  # what the model does (folding is bf16 only)
+        # folded-norm weights, kept beside the layer dicts (which stay as given)
+        self._folded = [{} for _ in self.layers]
+        if fold:
+            for lw, fw in zip(self.layers, self._folded):
+                if lw.get("wqkv") is not None and lw.get("gdn") is None:
+                    fw["wqkv_g"] = tg_fold_norm_weight(lw["wqkv"], lw["attn_norm"])
+                if lw.get("w_gate_up") is not None:
+                    fw["w_gate_up_g"] = tg_fold_norm_weight(lw["w_gate_up"], lw["ffn_norm"])
+            self._score_w1_g = tg_fold_norm_weight(self.score["score_w1"],
+                                                   self.score["score_norm"])
+        else:
+            self._score_w1_g = None
         arr = (TgLayer * len(self.layers))()
         for i, lw in enumerate(self.layers):
             for name, _ in TgLayer._fields_:
                 if name == "gdn":
                     g = lw.get("gdn")
                     arr[i].gdn = None if g is None else ctypes.addressof(g.c)
+                elif name in ("wqkv_g", "w_gate_up_g"):
+                    setattr(arr[i], name, _ptr(self._folded[i].get(name)))
                 else:
                     setattr(arr[i], name, _ptr(lw.get(name)))
         self._layers_c = arr
@@ -459,7 +495,7 @@ class Model:
                          self.rope_base, arr, _ptr(self.final_norm),
                          _ptr(self.score["score_norm"]), _ptr(self.score["score_w1"]),
                          _ptr(self.score.get("score_b1")), _ptr(self.score["score_w2"]),
-                         _ptr(self.score.get("score_b2")))
+                         _ptr(self.score.get("score_b2")), _ptr(self._score_w1_g))
 
     def decode_workspace_size(self, k_kept: int) -> int:
         return tg_workspace_size(TG_OP_DECODE, k=k_kept, d_model=self.d_model,

@@ -381,7 +381,7 @@ struct Params {
   // output rows and (m, l) to a slot; the part that finishes last (per-tile
   // counter) merges every slot in slot order and writes the result.
   int n_items;      // 0: closed-form order, no splits
-  float* part_o;    // [slots][n_pairs][2 heads][128 rows][128] fp32
+  float* part_o;    // [slots][n_pairs][2 heads][128 / 4 column quads][128 rows] float4
   float* part_ml;   // [slots][n_pairs][2][128][2] fp32 (m in log2 units, l)
   unsigned* cnt;    // [splits][n_pairs], zero between launches
   uint2 items[kMaxItems];
@@ -405,7 +405,7 @@ template <bool kBias>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKAug,
-                 const __grid_constant__ Params p) {
+                 const __grid_constant__ CUtensorMap tmO, const __grid_constant__ Params p) {
   using Lay = Layout<kBias>;
   constexpr int kOffQAugA = Lay::kOffQAugA, kOffQAugB = Lay::kOffQAugB, kOffKAug = Lay::kOffKAug;
   constexpr int kOffQA = Lay::kOffQA, kOffQB = Lay::kOffQB, kOffK = Lay::kOffK, kOffV = Lay::kOffV;
@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_empty = bars + 7;   // [2]
   uint64_t* s_full = bars + 9;    // [2 heads]
   uint64_t* p_full = bars + 11;   // [2 heads]
-  uint64_t* o_full = bars + 13;
+  uint64_t* o_full = bars + 13;   // head A; head B's is bars + 16
   uint64_t* qaug_full = bars + 14;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
 
@@ -470,12 +470,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[i], 128);
     }
     mbar_init(o_full, 1);
+    mbar_init(bars + 16, 1);
     mbar_init(qaug_full, 256);
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     if (kBias) tma_prefetch_desc(&tmKAug);
+    tma_prefetch_desc(&tmO);
   }
   if (warp == 2) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -557,6 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&p_full[0], j & 1, p.err)) break;
         tc_fence_after();
         issue_pv(0, j);
+        if (!more) umma_commit(o_full);  // head A's output is final
         if (more) {
           if (!mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, p.err)) break;
           tc_fence_after();
@@ -565,13 +568,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&p_full[1], j & 1, p.err)) break;
         tc_fence_after();
         issue_pv(1, j);
+        if (!more) umma_commit(bars + 16);  // head B's output is final
         umma_commit(&v_empty[s]);
         if (more) {
           issue_qk(1, j + 1);
           umma_commit(&k_empty[(j + 1) & 1]);
         }
       }
-      if (ok) umma_commit(o_full);
     }
   } else {
     setmaxnreg_inc<kRegsHigh>();
@@ -704,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&p_full[h]);
     }
-    ok = ok && mbar_wait_warp(o_full, 0, p.err);
+    ok = ok && mbar_wait_warp(h ? bars + 16 : o_full, 0, p.err);
     if (ok) tc_fence_after();
     // the item's split fields (decoded here, not kept live through the loop)
     const uint32_t iy = p.n_items > 0 ? p.items[blockIdx.x / n_pairs].y : 0u;
@@ -721,17 +724,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto slot_row = [&](int slot) {
       return ((static_cast<size_t>(slot) * n_pairs + pair_idx) * 2 + h) * kBlk + r;
     };
+    // a slot's partial output: [kDh / 4][kBlk rows] float4, so that the
+    // rows of a warp are adjacent (coalesced) for every 4 columns
+    auto slot_o = [&](int slot) {
+      return reinterpret_cast<float4*>(
+                 p.part_o + ((static_cast<size_t>(slot) * n_pairs + pair_idx) * 2 + h) * kBlk * kDh) +
+             r;
+    };
     if (n_parts > 1) {
       if (ok) {
         const size_t ri = slot_row(slot0 + part);
-        float4* po = reinterpret_cast<float4*>(p.part_o + ri * kDh);
+        float4* po = slot_o(slot0 + part);
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           float o[32];
           tmem_ld32_wait(tmem + lane_off + o_col + static_cast<uint32_t>(c * 32), o);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
-            po[c * 8 + v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+            po[(c * 8 + v) * kBlk] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
         }
         *reinterpret_cast<float2*>(p.part_ml + ri * 2) = make_float2(m, l);
         __threadfence();
@@ -799,11 +809,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int i = 0; i < 32; ++i) acc[i] = fmaf(o[i], wts[s2], acc[i]);
             } else {
-              const float4* src = reinterpret_cast<const float4*>(
-                  p.part_o + slot_row(slot0 + s2) * kDh + c * 32);
+              const float4* src = slot_o(slot0 + s2) + c * 8 * kBlk;
 #pragma unroll
               for (int v = 0; v < 8; ++v) {
-                const float4 t = __ldcg(src + v);
+                const float4 t = __ldcg(src + v * kBlk);
                 acc[4 * v] = fmaf(t.x, wts[s2], acc[4 * v]);
                 acc[4 * v + 1] = fmaf(t.y, wts[s2], acc[4 * v + 1]);
                 acc[4 * v + 2] = fmaf(t.z, wts[s2], acc[4 * v + 2]);
@@ -816,25 +825,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] *= inv;
-        if (q_row < p.T) {
-          if (p.out_f32) {
-            float4* d32 = reinterpret_cast<float4*>(p.out_f32 + (q_row * p.hq + head) * kDh + c * 32);
+        if (p.out_f32 && q_row < p.T) {
+          float4* d32 = reinterpret_cast<float4*>(p.out_f32 + (q_row * p.hq + head) * kDh + c * 32);
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-              d32[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (q_row * p.hq + head) * kDh + c * 32);
+          for (int v = 0; v < 8; ++v)
+            d32[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+        }
+        // the bf16 row into the head's (now idle) Q buffer, in the 128-byte
+        // swizzled layout of the output's TMA boxes: columns 32c .. 32c + 31
+        // are 16-byte units 4 (c & 1) .. + 3 of box c >> 1
+        uint8_t* rowp = smem + (h ? kOffQB : kOffQA) + (c >> 1) * kSub + r * 128;
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 u;
-            u.x = pack_bf16x2(o[8 * v + 0], o[8 * v + 1]);
-            u.y = pack_bf16x2(o[8 * v + 2], o[8 * v + 3]);
-            u.z = pack_bf16x2(o[8 * v + 4], o[8 * v + 5]);
-            u.w = pack_bf16x2(o[8 * v + 6], o[8 * v + 7]);
-            dst[v] = u;
-          }
+        for (int v = 0; v < 4; ++v) {
+          uint4 u;
+          u.x = pack_bf16x2(o[8 * v + 0], o[8 * v + 1]);
+          u.y = pack_bf16x2(o[8 * v + 2], o[8 * v + 3]);
+          u.z = pack_bf16x2(o[8 * v + 4], o[8 * v + 5]);
+          u.w = pack_bf16x2(o[8 * v + 6], o[8 * v + 7]);
+          const int unit = 4 * (c & 1) + v;
+          *reinterpret_cast<uint4*>(rowp + ((unit ^ (r & 7)) << 4)) = u;
         }
       }
+      fence_async_smem();
+    }
+    // The head's 128 rows leave in two TMA stores (rows past T are not
+    // written). Every thread of the warpgroup reaches the barrier.
+    const bool head_ok = named_bar_and(2 + h, 128, ok);
+    if (head_ok && r == 0) {
+      const uint8_t* ob = smem + (h ? kOffQB : kOffQA);
+      tma_store_3d(&tmO, ob, 0, head, q0);
+      tma_store_3d(&tmO, ob + kSub, 64, head, q0);
+      bulk_commit();
+      bulk_wait_read_all();  // the buffer is read before the CTA may exit
     }
   }
   tc_fence_before();
@@ -1027,7 +1049,10 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
     pp.out_f32 = p.out_f32;
     pp.err = p.err;
     const bool bias = a.lsig != nullptr && a.gain != nullptr;
-    CUtensorMap tka;
+    CUtensorMap tka, to;
+    // the output [T, hq, dh], stored by TMA in the same boxes as q is read
+    if (!make_tmap_3d_bf16(&to, a.out, kDh, a.hq, a.T, kDh * e, int64_t(a.hq) * kDh * e, 1, kBlk))
+      return cudaErrorInvalidValue;
     if (bias) {
       if (a.kaug == nullptr || !make_tmap_2d_bf16_sw32(&tka, a.kaug, a.T, 16, kBlk))
         return cudaErrorInvalidValue;
@@ -1073,7 +1098,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
       ok.store(fa.numRegs == int(pair::kRegsLaunch) ? 1 : -1);
     }
     if (ok.load() < 0) return cudaErrorInvalidConfiguration;
-    return launch_pdl(kern, dim3(grid), dim3(pair::kThreads), smem, st, tq, tk, tv, tka, pp);
+    return launch_pdl(kern, dim3(grid), dim3(pair::kThreads), smem, st, tq, tk, tv, tka, to, pp);
   }
   cudaError_t err = set_smem_attr_once(reinterpret_cast<const void*>(attn_tc), int(kSmem));
   if (err != cudaSuccess) return err;

@@ -62,7 +62,108 @@ struct EpiParams {
   __nv_bfloat16* vT_out;
   int64_t t_pad;
   __nv_bfloat16* v_out;
+  // folded RMSNorm: row sums of squares out (RESIDUAL) / in (the others)
+  float* ss_out;
+  const float* ss_in;
+  int64_t ss_ld;
+  int ss_parts;
+  float ss_inv_n, ss_eps;
+  // stream-K (sk_part != null): sk_dp_waves round-robin waves of whole
+  // tiles, then the k-blocks of the remaining tiles split evenly over the
+  // pairs (see Pieces)
+  int sk_dp_waves, sk_dp_tiles;
+  int64_t sk_units;
+  float4* sk_part;    // [pairs][2 ranks][64 column quads][128 rows]
+  unsigned* sk_flag;  // [pairs][2 ranks]
 };
+
+// One accumulator piece of a pair: k-blocks [k_lo, k_hi) of output tile `tile`.
+struct Piece {
+  int tile, k_lo, k_hi;
+};
+
+// The pieces of one CTA pair, in the same order for its producer, MMA and
+// epilogue warps. Without stream-K: tiles pair, pair + n_pairs, ... whole.
+// With it: first sk_dp_waves such waves, then the pair's contiguous share
+// [sk_units * pair / n_pairs, sk_units * (pair + 1) / n_pairs) of the
+// k-block units of tiles sk_dp_tiles.. (unit u: tile sk_dp_tiles + u / kb,
+// k-block u % kb). There are at least as many such tiles as pairs, so every
+// share spans at least one tile's k-blocks and a tile is split between at
+// most two consecutive pairs: pair q finishes its first k-blocks at the end
+// of its share (the tile's owner), pair q + 1 the rest at the start of its
+// own (it leaves them as a partial sum for the owner).
+struct Pieces {
+  int pair, n_pairs, num_tiles, num_kb, i;
+  int64_t u, u_end;
+  __device__ Pieces(const EpiParams& p, int pair_, int n_pairs_, int num_tiles_, int num_kb_)
+      : pair(pair_), n_pairs(n_pairs_), num_tiles(num_tiles_), num_kb(num_kb_), i(0), u(0),
+        u_end(0) {
+    if (p.sk_part != nullptr) {
+      u = p.sk_units * pair / n_pairs;
+      u_end = p.sk_units * (pair + 1) / n_pairs;
+    }
+  }
+  __device__ bool next(const EpiParams& p, Piece& pc) {
+    if (p.sk_part == nullptr || i < p.sk_dp_waves) {
+      const int tile = pair + i * n_pairs;
+      if (tile >= num_tiles) return false;
+      ++i;
+      pc = Piece{tile, 0, num_kb};
+      return true;
+    }
+    if (u >= u_end) return false;
+    const int k_lo = static_cast<int>(u % num_kb);
+    const int64_t left = u_end - u;
+    const int k_hi = left < num_kb - k_lo ? k_lo + static_cast<int>(left) : num_kb;
+    pc = Piece{p.sk_dp_tiles + static_cast<int>(u / num_kb), k_lo, k_hi};
+    u += k_hi - k_lo;
+    return true;
+  }
+};
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* f) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned* f, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+// Warp-uniform bounded wait for a partial-sum flag (lane 0 polls).
+__device__ __forceinline__ bool wait_flag_warp(const unsigned* f, unsigned int* err) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) {
+    if (ld_acquire_gpu(f) == 0u) {
+      const unsigned long long t0 = global_ns();
+      for (uint32_t i = 1;; ++i) {
+        if (ld_acquire_gpu(f) != 0u) break;
+        if ((i & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+          report_error(err, kErrWaitTimeout);
+          ok = 0;
+          break;
+        }
+      }
+    }
+  }
+  return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+
+// Accumulator columns [col, col + 32) of this thread's row, plus another
+// pair's partial sums of the same row and columns when the tile was split.
+__device__ __forceinline__ void acc_ld(uint32_t t_row, int col, const float4* part,
+                                       float (&v)[32]) {
+  tmem_ld32_wait(t_row + static_cast<uint32_t>(col), v);
+  if (part != nullptr) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 x = __ldcg(part + (col / 4 + q) * 128);
+      v[4 * q] += x.x;
+      v[4 * q + 1] += x.y;
+      v[4 * q + 2] += x.z;
+      v[4 * q + 3] += x.w;
+    }
+  }
+}
 
 __device__ __forceinline__ float round_bf16_f(float x) {
   return __bfloat162float(__float2bfloat16_rn(x));
@@ -95,32 +196,53 @@ __device__ __forceinline__ void add32_bf16(const __nv_bfloat16* src, float (&v)[
 // The fused epilogue of one accumulator tile, run by one epilogue warp for
 // its 32 rows: this thread owns accumulator row `row` (global index), whose
 // kBN fp32 columns start at TMEM address `t_row`; `nb` is the tile's column
-// block.
+// block; `part` (or null): the row's partial sums from the pair that did the
+// tile's last k-blocks.
 template <int kBN, int kEpi>
 __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, uint32_t t_row,
-                                              int nb) {
+                                              int nb, const float4* part) {
   const bool row_ok = row < p.M;
+  // Folded RMSNorm of the input row: B holds W . diag(g), and the row's
+  // accumulator is scaled by rs = 1 / sqrt(mean(x^2) + eps), the mean from the
+  // producing residual GEMM's per-column-block sums (added in block order).
+  float rs = 1.0f;
+  if (kEpi != EPI_RESIDUAL && p.ss_in != nullptr && row_ok) {
+    float ss = 0.f;
+    for (int q = 0; q < p.ss_parts; ++q) ss += __ldcg(p.ss_in + q * p.ss_ld + row);
+    rs = rsqrtf(ss * p.ss_inv_n + p.ss_eps);
+  }
   if constexpr (kEpi == EPI_STORE || kEpi == EPI_RESIDUAL) {
+    float ss = 0.f;  // RESIDUAL: sum of squares of the stored values
 #pragma unroll 1
     for (int c = 0; c < kBN / 32; ++c) {
       float v[32];
-      tmem_ld32_wait(t_row + c * 32, v);
+      acc_ld(t_row, c * 32, part, v);
       const int col = nb * kBN + c * 32;
       if (row_ok && col < p.N) {
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) + row * p.ldc + col;
-        if (kEpi == EPI_RESIDUAL)
+        if (kEpi == EPI_RESIDUAL) {
           add32_bf16(static_cast<const __nv_bfloat16*>(p.R) + row * p.ldr + col, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float f = round_bf16_f(v[j]);
+            ss = fmaf(f, f, ss);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] *= rs;
+        }
         store32_bf16(dst, v);
       }
     }
+    if (kEpi == EPI_RESIDUAL && p.ss_out != nullptr && row_ok) p.ss_out[nb * p.ss_ld + row] = ss;
   } else if constexpr (kEpi == EPI_SWIGLU) {
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       float g[32], u[32];
-      tmem_ld32_wait(t_row + c * 32, g);
-      tmem_ld32_wait(t_row + 128 + c * 32, u);
+      acc_ld(t_row, c * 32, part, g);
+      acc_ld(t_row, 128 + c * 32, part, u);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) g[j] = silu_f(g[j]) * u[j];
+      for (int j = 0; j < 32; ++j) g[j] = silu_f(g[j] * rs) * (u[j] * rs);
       if (row_ok)
         store32_bf16(static_cast<__nv_bfloat16*>(p.C) + row * p.ldc + nb * 128 + c * 32, g);
     }
@@ -131,7 +253,6 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
 #pragma unroll 1
     for (int hh = 0; hh < 2; ++hh) {
       const int hg = nb * 2 + hh;  // head index across the q | k | v columns
-      const uint32_t t_head = t_row + static_cast<uint32_t>(hh * 128);
       if (hg < p.hq + p.hkv) {
         const bool is_q = hg < p.hq;
         const float* nw = is_q ? p.q_norm : p.k_norm;
@@ -141,10 +262,10 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             float v[32];
-            tmem_ld32_wait(t_head + c * 32, v);
+            acc_ld(t_row, hh * 128 + c * 32, part, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float f = round_bf16_f(v[i]);
+              const float f = round_bf16_f(v[i] * rs);
               ss = fmaf(f, f, ss);
             }
           }
@@ -157,14 +278,14 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           float lo[32], hi[32];
-          tmem_ld32_wait(t_head + c * 32, lo);
-          tmem_ld32_wait(t_head + 64 + c * 32, hi);
+          acc_ld(t_row, hh * 128 + c * 32, part, lo);
+          acc_ld(t_row, hh * 128 + 64 + c * 32, part, hi);
           if (row_ok) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int pi = c * 32 + i;
-              float a = round_bf16_f(lo[i]) * rstd;
-              float b = round_bf16_f(hi[i]) * rstd;
+              float a = round_bf16_f(lo[i] * rs) * rstd;
+              float b = round_bf16_f(hi[i] * rs) * rstd;
               if (nw != nullptr) {
                 a *= __ldg(nw + pi);
                 b *= __ldg(nw + pi + 64);
@@ -182,7 +303,9 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           float v[32];
-          tmem_ld32_wait(t_head + c * 32, v);
+          acc_ld(t_row, hh * 128 + c * 32, part, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= rs;
           if (row_ok) {
             if (p.v_out) store32_bf16(p.v_out + (row * p.hkv + g) * 128 + c * 32, v);
             __nv_bfloat16* vt = p.vT_out + (static_cast<int64_t>(g) * 128 + c * 32) * p.t_pad + row;
@@ -197,12 +320,12 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
 #pragma unroll 1
     for (int c = 0; c < kBN / 32; ++c) {
       float v[32];
-      tmem_ld32_wait(t_row + c * 32, v);
+      acc_ld(t_row, c * 32, part, v);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int f = c * 32 + j;
         if (f < p.N) {
-          const float h = v[j] + (p.b1 ? __ldg(p.b1 + f) : 0.f);
+          const float h = v[j] * rs + (p.b1 ? __ldg(p.b1 + f) : 0.f);
           acc = fmaf(__ldg(p.w2 + f), silu_f(h), acc);
         }
       }
@@ -228,6 +351,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                  EpiParams p) {
   using C = PairCfg;
   constexpr int kBN = 256;
+  static_assert(kBN == kSsBlockCols, "row sums of squares are per 256-column block");
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base for the swizzled tiles; the offset is the same in
   // both CTAs (same kernel, same static layout).
@@ -273,12 +397,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
-      const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
+    Pieces pieces(p, pair, n_pairs, num_tiles, num_kb);
+    Piece pc;
+    while (ok && pieces.next(p, pc)) {
+      const int mb = pc.tile / p.tiles_n, nb = pc.tile % p.tiles_n;
       const int a_row = mb * 256 + static_cast<int>(rank) * 128;
       const int b_row = kEpi == EPI_SWIGLU ? (rank ? p.inter : 0) + nb * 128
                                            : nb * 256 + static_cast<int>(rank) * 128;
-      for (int kb = 0; kb < num_kb; ++kb) {
+      for (int kb = pc.k_lo; kb < pc.k_hi; ++kb) {
         if (!mbar_wait(&empty[s], ph ^ 1u, p.err)) { ok = false; break; }
         uint8_t* a_dst = tiles + size_t(s) * C::kStageBytes;
         uint8_t* b_dst = a_dst + C::kHalfBytes;
@@ -302,13 +428,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t ph = 0;
     bool ok = true;
     int it = 0;
-    for (int tile = pair; tile < num_tiles && ok; tile += n_pairs, ++it) {
+    Pieces pieces(p, pair, n_pairs, num_tiles, num_kb);
+    Piece pc;
+    for (; ok && pieces.next(p, pc); ++it) {
       const int a = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       if (!mbar_wait(&acc_empty[a], (use & 1u) ^ 1u, p.err)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * kBN);
-      for (int kb = 0; kb < num_kb; ++kb) {
+      for (int kb = pc.k_lo; kb < pc.k_hi; ++kb) {
         if (!mbar_wait(&full[s], ph, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_addr = smem_addr(tiles + size_t(s) * C::kStageBytes);
@@ -316,7 +444,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
           umma_f16_ss_pair(d_tmem, sdesc_kmajor_sw128(a_addr + k * 32),
-                           sdesc_kmajor_sw128(b_addr + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+                           sdesc_kmajor_sw128(b_addr + k * 32), idesc,
+                           (kb > pc.k_lo || k != 0) ? 1u : 0u);
         }
         const uint32_t e = smem_addr(&empty[s]);
         umma_commit_pair(e);
@@ -339,18 +468,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp >= 4) {
     // ---------------------------------------------------------- epilogue
     const int quarter = warp & 3;
+    const int rl = quarter * 32 + lane;  // row within this CTA's 128 accumulator rows
     int it = 0;
-    for (int tile = pair; tile < num_tiles; tile += n_pairs, ++it) {
-      const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
+    Pieces pieces(p, pair, n_pairs, num_tiles, num_kb);
+    Piece pc;
+    for (; pieces.next(p, pc); ++it) {
+      const int mb = pc.tile / p.tiles_n, nb = pc.tile % p.tiles_n;
       const int a = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       if (!mbar_wait_warp(&acc_full[a], use & 1u, p.err)) break;
       tc_fence_after();
-      const int64_t row =
-          static_cast<int64_t>(mb) * 256 + static_cast<int64_t>(rank) * 128 + quarter * 32 + lane;
+      const int64_t row = static_cast<int64_t>(mb) * 256 + static_cast<int64_t>(rank) * 128 + rl;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(a * kBN);
-      epilogue_tile<kBN, kEpi>(p, row, t_row, nb);
+      if (pc.k_lo > 0) {
+        // the tile's last k-blocks: a partial sum for the pair that owns it
+        float4* dst = p.sk_part + static_cast<size_t>(pair * 2 + rank) * (64 * 128) + rl;
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+          float v[32];
+          tmem_ld32_wait(t_row + c * 32, v);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[(c * 8 + q) * 128] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+        __threadfence();
+        named_bar_sync(1, 128);  // the four epilogue warps' rows are written
+        if (threadIdx.x == 128) st_release_gpu(p.sk_flag + pair * 2 + rank, 1u);
+      } else if (pc.k_hi < num_kb) {
+        // the tile's first k-blocks: add pair + 1's partial sums
+        const unsigned* f = p.sk_flag + (pair + 1) * 2 + rank;
+        const bool ready = wait_flag_warp(f, p.err);
+        __threadfence();  // every lane's partial-sum loads follow the flag
+        if (ready)
+          epilogue_tile<kBN, kEpi>(
+              p, row, t_row, nb, p.sk_part + static_cast<size_t>((pair + 1) * 2 + rank) * (64 * 128) + rl);
+        named_bar_sync(1, 128);  // every warp has seen the flag
+        if (threadIdx.x == 128) p.sk_flag[(pair + 1) * 2 + rank] = 0u;  // for the next launch
+      } else {
+        epilogue_tile<kBN, kEpi>(p, row, t_row, nb, nullptr);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&acc_empty[a]), 0));
@@ -393,6 +550,16 @@ cudaError_t run(const GemmArgs& g, cudaStream_t st) {
   p.vT_out = static_cast<__nv_bfloat16*>(g.vT_out);
   p.t_pad = g.t_pad;
   p.v_out = static_cast<__nv_bfloat16*>(g.v_out);
+  p.ss_out = g.ss_out;
+  p.ss_in = g.ss_in;
+  p.ss_ld = g.ss_ld;
+  p.ss_parts = g.ss_parts;
+  p.ss_inv_n = g.ss_inv_n;
+  p.ss_eps = g.ss_eps;
+  p.sk_dp_waves = p.sk_dp_tiles = 0;
+  p.sk_units = 0;
+  p.sk_part = nullptr;
+  p.sk_flag = nullptr;
   p.tiles_m = static_cast<int>((g.M + 255) / 256);
   p.tiles_n = kEpi == EPI_SWIGLU ? g.inter / 128 : (g.N + 255) / 256;
   p.err = device_error_word();
@@ -421,6 +588,17 @@ cudaError_t run(const GemmArgs& g, cudaStream_t st) {
     if (dev >= 0 && dev < kMaxDevices) resident[dev].store(max_pairs);
   }
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
+  // Stream-K when the tiles are more than one wave but not a whole number of
+  // waves: the last one to two waves' k-blocks are shared evenly by all pairs.
+  const int num_kb = (p.K + kBK - 1) / kBK;
+  if (g.sk_ws != nullptr && g.sk_ws_bytes >= gemm_sk_bytes() && pairs <= kSkMaxPairs &&
+      tiles > pairs && tiles % pairs != 0 && num_kb >= 4) {
+    p.sk_dp_waves = tiles / pairs - 1;
+    p.sk_dp_tiles = p.sk_dp_waves * pairs;
+    p.sk_units = static_cast<int64_t>(tiles - p.sk_dp_tiles) * num_kb;
+    p.sk_part = static_cast<float4*>(g.sk_ws);
+    p.sk_flag = reinterpret_cast<unsigned*>(static_cast<char*>(g.sk_ws) + gemm_sk_flag_offset());
+  }
   return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), C::kSmem, st, ta, tb, p);
 }
 

@@ -314,6 +314,49 @@ __global__ void score_dot_f32(const float* __restrict__ hpre, int64_t rows, int 
 
 }  // namespace
 
+// W_g[j, i] = bf16(W[j, i] * g[i]), eight elements per thread (cols % 8 == 0,
+// 16-byte aligned) or one.
+template <int kVec>
+__global__ void __launch_bounds__(256) fold_norm_weight(const __nv_bfloat16* __restrict__ w,
+                                                        const float* __restrict__ g, int64_t rows,
+                                                        int64_t cols, __nv_bfloat16* __restrict__ out) {
+  const int64_t n = rows * cols / kVec;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t c = (i * kVec) % cols;
+    if constexpr (kVec == 8) {
+      const uint4 u = __ldcs(reinterpret_cast<const uint4*>(w) + i);
+      const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&u);
+      uint4 o;
+      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(e[j]);
+        ow[j] = pack_bf16x2(f.x * __ldg(g + c + 2 * j), f.y * __ldg(g + c + 2 * j + 1));
+      }
+      __stcs(reinterpret_cast<uint4*>(out) + i, o);
+    } else {
+      out[i] = __float2bfloat16_rn(__bfloat162float(w[i]) * __ldg(g + c));
+    }
+  }
+}
+
+cudaError_t launch_fold_norm_weight(const void* w, const float* g, int64_t rows, int64_t cols,
+                                    void* out, cudaStream_t st) {
+  if (rows <= 0 || cols <= 0) return cudaSuccess;
+  const bool vec = cols % 8 == 0 &&
+                   ((reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(out)) & 15u) == 0;
+  const int64_t work = rows * cols / (vec ? 8 : 1);
+  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((work + 255) / 256, 148 * 16));
+  const auto* wb = static_cast<const __nv_bfloat16*>(w);
+  auto* ob = static_cast<__nv_bfloat16*>(out);
+  if (vec)
+    fold_norm_weight<8><<<blocks, 256, 0, st>>>(wb, g, rows, cols, ob);
+  else
+    fold_norm_weight<1><<<blocks, 256, 0, st>>>(wb, g, rows, cols, ob);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_rmsnorm(const void* x, const float* gamma, float eps, int64_t rows, int d,
                            bool bf16, void* y, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;

@@ -436,7 +436,21 @@ __device__ __forceinline__ uint32_t cta_sum_1024(uint32_t v, uint32_t* dst) {
   return *dst;
 }
 
-template <bool kVec>
+// kPer tokens per thread (a multiple of 8); kOne: a single CTA (no
+// cluster), whose barriers are plain __syncthreads and whose "remote" shared
+// memory is its own.
+template <bool kOne>
+__device__ __forceinline__ void sel_sync() {
+  if (kOne) __syncthreads();
+  else cluster_sync();
+}
+template <bool kOne>
+__device__ __forceinline__ uint32_t ld_rank(const uint32_t* p, uint32_t rank) {
+  if (kOne) return *reinterpret_cast<const volatile uint32_t*>(p);
+  return ld_cluster_u32(mapa_shared(smem_addr(p), rank));
+}
+
+template <bool kVec, int kPer, bool kOne>
 __global__ void __launch_bounds__(kCThreads, 1)
     sel_cluster(const float* __restrict__ scores, const uint8_t* __restrict__ protect, int64_t n,
                 int64_t k, int32_t* __restrict__ kept_idx, int32_t* __restrict__ status) {
@@ -452,21 +466,33 @@ __global__ void __launch_bounds__(kCThreads, 1)
   pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31;
   const uint32_t C = gridDim.x;  // the grid is one cluster
-  const uint32_t rank = cluster_ctarank();
+  const uint32_t rank = kOne ? 0u : cluster_ctarank();
   if (tid < 4) cta_val[tid] = 0u;
   __syncthreads();
   pdl_wait();
-  uint32_t key[kPerThread];
-  bool prot[kPerThread];
-  const int64_t first = static_cast<int64_t>(rank) * kCChunk + static_cast<int64_t>(tid) * kPerThread;
-  const int valid = load_tokens<kVec>(scores, protect, n, first, key, prot);
+  static_assert(kPer % kPerThread == 0 && kPer <= 16, "tokens per thread");
+  uint32_t key[kPer];
+  uint32_t pmask = 0u;  // bit j: token j of this thread is protected
+  const int64_t first = static_cast<int64_t>(rank) * kCThreads * kPer + static_cast<int64_t>(tid) * kPer;
+  int valid = 0;  // tokens of this thread that exist (a prefix of its kPer)
+#pragma unroll
+  for (int q = 0; q < kPer / kPerThread; ++q) {
+    uint32_t kq[kPerThread];
+    bool pq[kPerThread];
+    valid += load_tokens<kVec>(scores, protect, n, first + q * kPerThread, kq, pq);
+#pragma unroll
+    for (int j = 0; j < kPerThread; ++j) {
+      key[q * kPerThread + j] = kq[j];
+      if (pq[j]) pmask |= 1u << (q * kPerThread + j);
+    }
+  }
   uint32_t np_t = 0;
 #pragma unroll
-  for (int j = 0; j < kPerThread; ++j)
-    if (j < valid && prot[j]) ++np_t;
+  for (int j = 0; j < kPer; ++j)
+    if (j < valid && ((pmask >> j) & 1u)) ++np_t;
   cta_sum_1024(np_t, &cta_val[2]);
-  cluster_sync();
-  if (tid < static_cast<int>(C)) tot[tid] = ld_cluster_u32(mapa_shared(smem_addr(&cta_val[2]), tid));
+  sel_sync<kOne>();
+  if (tid < static_cast<int>(C)) tot[tid] = ld_rank<kOne>(&cta_val[2], tid);
   __syncthreads();
   uint32_t np = 0;
   for (uint32_t r = 0; r < C; ++r) np += tot[r];
@@ -484,30 +510,35 @@ __global__ void __launch_bounds__(kCThreads, 1)
       for (int i = tid; i < bins; i += kCThreads) hist[i] = 0u;
       if (tid == 0) *slice_tot = 0u;
       __syncthreads();
-      // warp-aggregated: one shared-memory atomic per distinct bin per warp
+      // A warp whose 32 keys fall in one bin (tied scores) adds once;
+      // otherwise one shared-memory atomic per active key.
 #pragma unroll
-      for (int j = 0; j < kPerThread; ++j) {
-        const bool act = j < valid && !prot[j] &&
+      for (int j = 0; j < kPer; ++j) {
+        const bool act = j < valid && !((pmask >> j) & 1u) &&
                          (pass == 0 || (key[j] >> (32 - pbits)) == prefix);
         const uint32_t bin = act ? (key[j] >> shift) & static_cast<uint32_t>(bins - 1) : 0xFFFFFFFFu;
-        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
-        if (act && (__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], __popc(peers));
+        const uint32_t bin0 = __shfl_sync(0xFFFFFFFFu, bin, 0);
+        if (__all_sync(0xFFFFFFFFu, bin == bin0)) {
+          if (lane == 0 && bin0 != 0xFFFFFFFFu) atomicAdd(&hist[bin0], 32u);
+        } else if (act) {
+          atomicAdd(&hist[bin], 1u);
+        }
       }
-      cluster_sync();
+      sel_sync<kOne>();
       // this CTA's slice of the bins, summed over the cluster
       const uint32_t S = static_cast<uint32_t>(bins) / C;
       uint32_t part = 0u;
       for (uint32_t t = tid; t < S; t += kCThreads) {
         const uint32_t b = rank * S + t;
         uint32_t sum = 0u;
-        for (uint32_t r = 0; r < C; ++r) sum += ld_cluster_u32(mapa_shared(smem_addr(&hist[b]), r));
+        for (uint32_t r = 0; r < C; ++r) sum += ld_rank<kOne>(&hist[b], r);
         red[t] = sum;
         part += sum;
       }
       cta_sum_1024(part, slice_tot);
-      cluster_sync();
+      sel_sync<kOne>();
       // the slice (from the top) where the count reaches `need`, then the bin
-      if (tid < static_cast<int>(C)) tot[tid] = ld_cluster_u32(mapa_shared(smem_addr(slice_tot), tid));
+      if (tid < static_cast<int>(C)) tot[tid] = ld_rank<kOne>(slice_tot, tid);
       __syncthreads();
       uint32_t above = 0u, sl = 0u;
       for (int r = static_cast<int>(C) - 1; r >= 0; --r) {
@@ -524,7 +555,7 @@ __global__ void __launch_bounds__(kCThreads, 1)
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         const uint32_t e = 2u * tid + q;
-        if (e < S) v[q] = ld_cluster_u32(mapa_shared(smem_addr(&red[S - 1 - e]), sl));
+        if (e < S) v[q] = ld_rank<kOne>(&red[S - 1 - e], sl);
       }
       const uint32_t before = cta_excl_scan_1024(v[0] + v[1], nullptr, warp_sums);
       if (before < rest && rest <= before + v[0] + v[1]) {
@@ -544,24 +575,24 @@ __global__ void __launch_bounds__(kCThreads, 1)
     for (int64_t i = static_cast<int64_t>(rank) * kCThreads + tid; i < k;
          i += static_cast<int64_t>(C) * kCThreads)
       kept_idx[i] = -1;
-    cluster_sync();  // no CTA leaves while another may still read its shared memory
+    sel_sync<kOne>();  // no CTA leaves while another may still read its shared memory
     return;
   }
   // sure keeps and ties of this thread, CTA and the CTAs before it, as one
   // packed count (sure << 16 | ties; at most 8192 of each per CTA)
   uint32_t nd = 0u, nt = 0u;
 #pragma unroll
-  for (int j = 0; j < kPerThread; ++j) {
+  for (int j = 0; j < kPer; ++j) {
     if (j < valid) {
-      if (prot[j] || key[j] > thresh) ++nd;
+      if (((pmask >> j) & 1u) || key[j] > thresh) ++nd;
       else if (key[j] == thresh) ++nt;
     }
   }
   uint32_t packed_cta;
   const uint32_t packed = cta_excl_scan_1024((nd << 16) | nt, &packed_cta, warp_sums);
   if (tid == 0) cta_val[1] = packed_cta;
-  cluster_sync();
-  if (tid < static_cast<int>(rank)) tot[tid] = ld_cluster_u32(mapa_shared(smem_addr(&cta_val[1]), tid));
+  sel_sync<kOne>();
+  if (tid < static_cast<int>(rank)) tot[tid] = ld_rank<kOne>(&cta_val[1], tid);
   __syncthreads();
   uint32_t sb = packed >> 16, tb = packed & 0xFFFFu;
   for (uint32_t r = 0; r < rank; ++r) {
@@ -569,9 +600,9 @@ __global__ void __launch_bounds__(kCThreads, 1)
     tb += tot[r] & 0xFFFFu;
   }
 #pragma unroll
-  for (int j = 0; j < kPerThread; ++j) {
+  for (int j = 0; j < kPer; ++j) {
     if (j < valid) {
-      const bool sure = prot[j] || key[j] > thresh;
+      const bool sure = ((pmask >> j) & 1u) || key[j] > thresh;
       const bool tie = !sure && key[j] == thresh;
       if (sure) {
         const uint32_t pos = sb + min(tb, ties);
@@ -587,7 +618,7 @@ __global__ void __launch_bounds__(kCThreads, 1)
     }
   }
   if (rank == 0 && tid == 0) *status = 0;
-  cluster_sync();  // no CTA leaves while another may still read its shared memory
+  sel_sync<kOne>();  // no CTA leaves while another may still read its shared memory
 }
 
 // Cluster size for n tokens (0: n is past the one-launch path).
@@ -596,10 +627,10 @@ int cluster_ctas(int64_t n) {
   static std::once_flag once;
   std::call_once(once, [] {
     max_ctas = 8;
-    auto kern = sel_cluster<true>;
+    auto kern = sel_cluster<true, kPerThread, false>;
     if (cudaFuncSetAttribute(reinterpret_cast<const void*>(kern),
                              cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
-        cudaFuncSetAttribute(reinterpret_cast<const void*>(sel_cluster<false>),
+        cudaFuncSetAttribute(reinterpret_cast<const void*>(sel_cluster<false, kPerThread, false>),
                              cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(16);
@@ -623,24 +654,36 @@ int cluster_ctas(int64_t n) {
   return c <= max_ctas ? c : 0;
 }
 
+// One CTA (n <= 2 x 8192: up to 16 tokens per thread, no cluster barriers),
+// else one cluster of `ctas` CTAs with 8 tokens per thread.
 template <bool kVec>
 cudaError_t run_select_cluster(const float* scores, const uint8_t* protect, int64_t n, int64_t k,
                                int32_t* kept_idx, void* ws, int ctas, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
   cfg.blockDim = dim3(kCThreads);
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(ctas);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
+  int32_t* status = static_cast<int32_t*>(ws);
+  if (n <= 2 * kCChunk) {
+    cfg.gridDim = dim3(1);
+    cfg.numAttrs = 1;
+    if (n <= kCChunk)
+      return cudaLaunchKernelEx(&cfg, sel_cluster<kVec, 8, true>, scores, protect, n, k, kept_idx,
+                                status);
+    return cudaLaunchKernelEx(&cfg, sel_cluster<kVec, 16, true>, scores, protect, n, k,
+                              kept_idx, status);
+  }
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(ctas);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, sel_cluster<kVec>, scores, protect, n, k, kept_idx,
-                            static_cast<int32_t*>(ws));
+  return cudaLaunchKernelEx(&cfg, sel_cluster<kVec, kPerThread, false>, scores, protect, n, k,
+                            kept_idx, status);
 }
 
 template <bool kVec>

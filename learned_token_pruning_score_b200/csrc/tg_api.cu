@@ -259,6 +259,17 @@ struct PrefillPlan {
   void* gu = nullptr;
   float* scores = nullptr; // [n]
   float* hpre = nullptr;   // fp32 scorer pre-activation [n, F]
+  // Folded RMSNorm (bf16): the row sums of squares the last residual GEMM
+  // left, [ss_parts][ss_ld] (one per 256-column block), and which residual
+  // stream (rows [0, ss_rows) of buffer ss_for) they describe. Anything
+  // other than a residual GEMM that writes a stream resets ss_for.
+  void* gemm_sk = nullptr;  // stream-K scratch of the tensor-core GEMMs
+  float* ss = nullptr;    // rows of h: [ss_parts][n]
+  float* ss_k = nullptr;  // rows of hk: [ss_parts][k]
+  int64_t ss_ld = 0, ss_ld_k = 0;
+  int ss_parts = 0;
+  mutable const void* ss_for = nullptr;
+  mutable int64_t ss_rows = 0;
   int32_t* pos_k = nullptr;
   float* s_k = nullptr;
   float* lsig_k = nullptr;
@@ -293,6 +304,14 @@ struct PrefillPlan {
       if (m.dtype == TG_F32) gu = a.carve(fr * 2 * m.d_ffn * 4);
     }
     scores = static_cast<float*>(a.carve(size_t(n) * 4));
+    if (m.dtype == TG_BF16) {
+      ss_parts = ss_parts_of(d);
+      ss_ld = n;
+      ss_ld_k = k;
+      ss = static_cast<float*>(a.carve(size_t(ss_parts) * n * 4));
+      ss_k = static_cast<float*>(a.carve(size_t(ss_parts) * k * 4));
+      gemm_sk = a.carve(gemm_sk_bytes());
+    }
     if (m.dtype == TG_F32) hpre = static_cast<float*>(a.carve(size_t(n) * m.d_score * 4));
     pos_k = static_cast<int32_t*>(a.carve(size_t(k) * 4));
     s_k = static_cast<float*>(a.carve(size_t(k) * 4));
@@ -366,13 +385,13 @@ cudaError_t select_topk(const float* scores, const uint8_t* protect, int64_t n, 
 
 cudaError_t compact(const void* x, const int32_t* pos_in, const float* scores, const int32_t* idx,
                     int64_t n, int64_t k, int row_bytes, void* x_out, int32_t* pos_out,
-                    float* s_out, float* lsig_out, cudaStream_t st) {
+                    float* s_out, float* lsig_out, cudaStream_t st, const SsGather& ss = {}) {
   const double bytes = 2.0 * double(k) * row_bytes + 4.0 * k /*idx*/ + 4.0 * k /*pos*/ +
                        (scores ? 4.0 * k : 0.0) + (s_out ? 4.0 * k : 0.0) +
                        (lsig_out ? 4.0 * k : 0.0);
   return traced(TG_K_COMPACT, k, 0.0, bytes, st, [&] {
     return launch_compact(x, pos_in, scores, idx, n, k, row_bytes, x_out, pos_out, s_out,
-                          lsig_out, st);
+                          lsig_out, ss, st);
   });
 }
 
@@ -384,15 +403,66 @@ GemmArgs gemm_args(const void* A, int64_t lda, const void* B, int64_t ldb, void*
   return g;
 }
 
-// Scorer over `rows` rows of x (dtype dt) into scores[rows].
+// Stream-K scratch of the plan for a tensor-core GEMM (its flags are zeroed
+// once per call by sk_clear, and every launch leaves them zero).
+GemmArgs& with_sk(GemmArgs& g, const PrefillPlan& P) {
+  if (P.gemm_sk != nullptr) {
+    g.sk_ws = P.gemm_sk;
+    g.sk_ws_bytes = gemm_sk_bytes();
+  }
+  return g;
+}
+cudaError_t sk_clear(const PrefillPlan& P, cudaStream_t st) {
+  if (P.gemm_sk == nullptr) return cudaSuccess;
+  return cudaMemsetAsync(static_cast<char*>(P.gemm_sk) + gemm_sk_flag_offset(), 0,
+                         gemm_sk_bytes() - gemm_sk_flag_offset(), st);
+}
+
+// Folded RMSNorm: rows [0, rows) of the stream h carry the row sums of
+// squares their last residual GEMM left in P.ss.
+bool ss_ready(const PrefillPlan& P, const void* h, int64_t rows) {
+  return P.ss != nullptr && P.ss_for == h && P.ss_rows == rows;
+}
+// The row sums of the stream h (the all-token buffer or the kept-row one).
+float* ss_of(const PrefillPlan& P, const void* h) { return h == P.hk ? P.ss_k : P.ss; }
+int64_t ss_ld_of(const PrefillPlan& P, const void* h) { return h == P.hk ? P.ss_ld_k : P.ss_ld; }
+// The projection of rows [row0, row0 + M) of h scales its accumulator rows by 1 / rms.
+void ss_consume(GemmArgs& g, const PrefillPlan& P, const void* h, float eps, int d, int64_t row0) {
+  g.ss_in = ss_of(P, h) + row0;
+  g.ss_ld = ss_ld_of(P, h);
+  g.ss_parts = P.ss_parts;
+  g.ss_inv_n = 1.0f / static_cast<float>(d);
+  g.ss_eps = eps;
+}
+// The residual GEMM of rows [row0, row0 + M) of h leaves their sums of squares.
+void ss_produce(GemmArgs& g, const PrefillPlan& P, const void* h, int64_t row0) {
+  if (P.ss == nullptr) return;
+  g.ss_out = ss_of(P, h) + row0;
+  g.ss_ld = ss_ld_of(P, h);
+}
+void ss_mark(const PrefillPlan& P, const void* h, int64_t rows) {
+  if (P.ss == nullptr) return;
+  P.ss_for = h;
+  P.ss_rows = rows;
+}
+
+// Scorer over `rows` rows of x (dtype dt) into scores[rows]. With a plan
+// whose row sums describe x and the folded w1_g, no RMSNorm kernel runs.
 cudaError_t run_score(const void* x, int64_t rows, int d, int f, const float* norm_w, float eps,
                       const void* w1, const float* b1, const float* w2, const float* b2,
-                      tg_dtype dt, float* scores, void* y, float* hpre, cudaStream_t st) {
-  cudaError_t e = rmsnorm(x, norm_w, eps, rows, d, dt, y, st);
-  if (e != cudaSuccess) return e;
+                      tg_dtype dt, float* scores, void* y, float* hpre, cudaStream_t st,
+                      const PrefillPlan* P = nullptr, const void* w1_g = nullptr) {
+  const bool fold = P != nullptr && w1_g != nullptr && ss_ready(*P, x, rows);
+  cudaError_t e = cudaSuccess;
+  if (!fold) {
+    e = rmsnorm(x, norm_w, eps, rows, d, dt, y, st);
+    if (e != cudaSuccess) return e;
+  }
   if (dt == TG_BF16) {
-    GemmArgs g = gemm_args(y, d, w1, d, nullptr, 0, rows, f, d, EPI_SCORE);
+    GemmArgs g = gemm_args(fold ? x : y, d, fold ? w1_g : w1, d, nullptr, 0, rows, f, d, EPI_SCORE);
     g.b1 = b1; g.w2 = w2; g.b2 = b2; g.scores = scores;
+    if (fold) ss_consume(g, *P, x, eps, d, 0);
+    if (P != nullptr) with_sk(g, *P);
     return gemm(g, dt, st);
   }
   GemmArgs g = gemm_args(y, d, w1, d, hpre, f, rows, f, d, EPI_STORE);
@@ -524,10 +594,19 @@ cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims
                                const tg_layer_taps* taps = nullptr) {
   const tg_dtype dt = m.dtype;
   const size_t e = elem_size(dt);
-  cudaError_t err = rmsnorm(h, lw.attn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
-  if (err != cudaSuccess) return err;
+  // folded RMSNorm (h's rows fresh from a residual GEMM), else the norm kernel
+  const bool fold = lw.wqkv_g != nullptr && ss_ready(P, h, rows);
+  cudaError_t err = cudaSuccess;
+  if (!fold) {
+    err = rmsnorm(h, lw.attn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
+    if (err != cudaSuccess) return err;
+  }
+  const void* xin = fold ? h : P.y;
+  const void* wqkv = fold ? lw.wqkv_g : lw.wqkv;
   void* k_dst = (kv && kv->k) ? kv->k : P.attn.k_rot;
-  GemmArgs gq = gemm_args(P.y, D.d, lw.wqkv, D.d, nullptr, 0, rows, D.qkv, D.d, EPI_QKV);
+  GemmArgs gq = gemm_args(xin, D.d, wqkv, D.d, nullptr, 0, rows, D.qkv, D.d, EPI_QKV);
+  if (fold) ss_consume(gq, P, h, m.norm_eps, D.d, 0);
+  with_sk(gq, P);
   gq.hq = D.hq; gq.hkv = D.hkv; gq.rope_cs = cs; gq.q_norm = lw.q_norm; gq.k_norm = lw.k_norm;
   gq.eps = m.norm_eps; gq.q_out = P.attn.q_rot; gq.k_out = k_dst; gq.vT_out = P.attn.vT;
   gq.t_pad = P.attn.t_pad; gq.v_out = kv ? kv->v : nullptr;
@@ -544,8 +623,9 @@ cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims
   } else if (segs != nullptr || P.qkv == nullptr) {
     return cudaErrorInvalidValue;  // packed requests need the fused bf16 path
   } else {
-    err = gemm(gemm_args(P.y, D.d, lw.wqkv, D.d, P.qkv, D.qkv, rows, D.qkv, D.d, EPI_STORE), dt,
-               st);
+    GemmArgs gs = gemm_args(xin, D.d, wqkv, D.d, P.qkv, D.qkv, rows, D.qkv, D.d, EPI_STORE);
+    if (fold) ss_consume(gs, P, h, m.norm_eps, D.d, 0);
+    err = gemm(gs, dt, st);
     if (err != cudaSuccess) return err;
     const char* qkv = static_cast<const char*>(P.qkv);
     err = run_attention(qkv, D.qkv, qkv + size_t(D.hq) * D.dh * e, D.qkv,
@@ -563,8 +643,12 @@ cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims
                          D.d, D.hq * D.dh, EPI_RESIDUAL);
   g.R = h;
   g.ldr = D.d;
+  ss_produce(g, P, h, 0);
+  with_sk(g, P);
   err = gemm(g, dt, st);
-  if (err != cudaSuccess || !taps || !taps->resid) return err;
+  if (err != cudaSuccess) return err;
+  ss_mark(P, h, rows);
+  if (!taps || !taps->resid) return err;
   return copy_rows(taps->resid, h, size_t(rows) * D.d * e, rows, st);
 }
 
@@ -573,17 +657,24 @@ cudaError_t ffn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
   if (lw.w_gate_up == nullptr) return cudaSuccess;
   const tg_dtype dt = m.dtype;
   const size_t e = elem_size(dt);
-  cudaError_t err = rmsnorm(h, lw.ffn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
-  if (err != cudaSuccess) return err;
+  // folded RMSNorm (h's rows fresh from a residual GEMM), else the norm kernel
+  const bool fold = lw.w_gate_up_g != nullptr && ss_ready(P, h, rows);
+  cudaError_t err = cudaSuccess;
+  if (!fold) {
+    err = rmsnorm(h, lw.ffn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
+    if (err != cudaSuccess) return err;
+  }
   // row blocks of at most kFfnRows share the intermediate buffer
   for (int64_t r0 = 0; r0 < rows; r0 += kFfnRows) {
     const int64_t rb = std::min<int64_t>(kFfnRows, rows - r0);
-    const char* yb = static_cast<const char*>(P.y) + size_t(r0) * D.d * e;
+    const char* yb = static_cast<const char*>(fold ? h : P.y) + size_t(r0) * D.d * e;
     void* hb = static_cast<char*>(h) + size_t(r0) * D.d * e;
     if (dt == TG_BF16) {
-      GemmArgs g = gemm_args(yb, D.d, lw.w_gate_up, D.d, P.mlp, D.inter, rb, 2 * D.inter, D.d,
-                             EPI_SWIGLU);
+      GemmArgs g = gemm_args(yb, D.d, fold ? lw.w_gate_up_g : lw.w_gate_up, D.d, P.mlp, D.inter, rb,
+                             2 * D.inter, D.d, EPI_SWIGLU);
       g.inter = D.inter;
+      if (fold) ss_consume(g, P, h, m.norm_eps, D.d, r0);
+      with_sk(g, P);
       err = gemm(g, dt, st);
     } else {
       err = gemm(gemm_args(yb, D.d, lw.w_gate_up, D.d, P.gu, 2 * D.inter, rb, 2 * D.inter, D.d,
@@ -599,9 +690,12 @@ cudaError_t ffn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
                            EPI_RESIDUAL);
     g.R = hb;
     g.ldr = D.d;
+    ss_produce(g, P, h, r0);
+    with_sk(g, P);
     err = gemm(g, dt, st);
     if (err != cudaSuccess) return err;
   }
+  ss_mark(P, h, rows);
   return cudaSuccess;
 }
 
@@ -678,8 +772,12 @@ cudaError_t gdn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
   GemmArgs g = gemm_args(P.gdn_y, vd, lw.w_out, vd, h, D.d, rows, D.d, vd, EPI_RESIDUAL);
   g.R = h;
   g.ldr = D.d;
+  ss_produce(g, P, h, 0);
+  with_sk(g, P);
   err = gemm(g, dt, st);
-  if (err != cudaSuccess || !taps || !taps->resid) return err;
+  if (err != cudaSuccess) return err;
+  ss_mark(P, h, rows);
+  if (!taps || !taps->resid) return err;
   return copy_rows(taps->resid, h, size_t(rows) * D.d * e, rows, st);
 }
 
@@ -816,6 +914,15 @@ tg_status validate_model(const tg_model* m, int64_t n, int64_t k, int gate_layer
       TG_CHECK((L.q_norm == nullptr) == (L.k_norm == nullptr), TG_ERR_INVALID_ARG);
     }
     if (L.w_gate_up) TG_CHECK(L.w_down && L.ffn_norm && m->d_ffn > 0, TG_ERR_INVALID_ARG);
+    // folded-norm weights: bf16 only, TMA-aligned, beside the weights they fold
+    const void* wqkv_g = L.gdn == nullptr ? L.wqkv_g : nullptr;  // unused by a mixer layer
+    if (wqkv_g || L.w_gate_up_g) TG_CHECK(m->dtype == TG_BF16, TG_ERR_UNSUPPORTED);
+    if (wqkv_g) TG_CHECK(aligned16(wqkv_g), TG_ERR_INVALID_ARG);
+    if (L.w_gate_up_g) TG_CHECK(L.w_gate_up && aligned16(L.w_gate_up_g), TG_ERR_INVALID_ARG);
+  }
+  if (m->score_w1_g) {
+    TG_CHECK(m->dtype == TG_BF16, TG_ERR_UNSUPPORTED);
+    TG_CHECK(aligned16(m->score_w1_g), TG_ERR_INVALID_ARG);
   }
   bool any_ffn = false;
   for (int l = 0; l < m->n_layers; ++l) any_ffn |= m->layers[l].w_gate_up != nullptr;
@@ -918,6 +1025,19 @@ tg_status tg_linear(const void* x, const void* w, const void* residual, int64_t 
     TG_CHECK(gemm_tc_supported(g), TG_ERR_INVALID_ARG);
   }
   return cuda_status(gemm(g, dt, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tg_status tg_fold_norm_weight(const void* w, const float* g, int64_t rows, int64_t cols, void* out,
+                              tg_stream stream) {
+  TG_CHECK(w && g && out && rows >= 1 && cols >= 1, TG_ERR_INVALID_ARG);
+  TG_CHECK(rows <= (int64_t(1) << 40) / cols, TG_ERR_INVALID_ARG);
+  const uintptr_t wa = reinterpret_cast<uintptr_t>(w), oa = reinterpret_cast<uintptr_t>(out);
+  const uintptr_t nb = static_cast<uintptr_t>(rows * cols * 2);
+  TG_CHECK(oa + nb <= wa || wa + nb <= oa, TG_ERR_INVALID_ARG);  // no overlap
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return cuda_status(traced(TG_K_FOLD_NORM, rows, 0.0, 4.0 * rows * cols + 4.0 * cols, st, [&] {
+    return launch_fold_norm_weight(w, g, rows, cols, out, st);
+  }));
 }
 
 tg_status tg_topk_select_noalloc(const float* scores, const uint8_t* protect, int64_t n,
@@ -1116,8 +1236,10 @@ tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan
                              const tg_layer_taps* taps, float* sc, cudaStream_t st) {
   const size_t e = elem_size(m.dtype);
   TG_TRY(copy_rows(P.h, x, size_t(n) * D.d * e, n, st));
+  P.ss_for = nullptr;  // the input rows carry no row sums
   // every attention launch of the call then finds its split counters zero
   TG_TRY(attn_split_clear(P.attn.split, P.attn.split_bytes, D.hq, st));
+  TG_TRY(sk_clear(P, st));
   const bool tables = m.dtype == TG_BF16 && D.dh == 128;
   const double cs_bytes = 8.0 * (D.dh / 2);
   if (tables && gate_layer >= 0)
@@ -1141,7 +1263,7 @@ tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan
   }
   // score the post-attention residual
   TG_TRY(run_score(P.h, n, D.d, m.d_score, m.score_norm, m.norm_eps, m.score_w1, m.score_b1,
-                   m.score_w2, m.score_b2, m.dtype, sc, P.y, P.hpre, st));
+                   m.score_w2, m.score_b2, m.dtype, sc, P.y, P.hpre, st, &P, m.score_w1_g));
   return TG_OK;
 }
 
@@ -1156,8 +1278,14 @@ tg_status prefill_above_gate(const tg_model& m, const Dims& D, const PrefillPlan
   const bool tables = m.dtype == TG_BF16 && D.dh == 128;
   const double cs_bytes = 8.0 * (D.dh / 2);
   TG_TRY(select_topk(sc, protect, n, k, kept_idx, P.sel_ws, st));
+  // the kept rows take their row sums along when h's are current
+  SsGather sg;
+  const bool carry = ss_ready(P, P.h, n) && P.ss_parts <= 32;
+  if (carry) sg = SsGather{P.ss, P.ss_ld, P.ss_k, P.ss_ld_k, P.ss_parts};
   TG_TRY(compact(P.h, nullptr, sc, kept_idx, n, k, static_cast<int>(D.d * e), P.hk, P.pos_k, P.s_k,
-                 P.lsig_k, st));
+                 P.lsig_k, st, sg));
+  if (carry) ss_mark(P, P.hk, k);
+  else if (P.ss_for == P.hk) P.ss_for = nullptr;
   if (tables) {
     TG_TRY(traced(TG_K_ROPE_TABLE, k, 0.0, cs_bytes * k + 4.0 * k, st, [&] {
       return launch_rope_table(P.pos_k, k, D.dh, m.rope_base, P.cs_k, st);
@@ -1337,6 +1465,7 @@ tg_status tg_prefill_batch(const tg_model* model, const void* x, const uint8_t* 
   char* h = static_cast<char*>(P.h);
   char* hk = static_cast<char*>(P.hk);
   TG_TRY(attn_split_clear(P.attn.split, P.attn.split_bytes, D.hq, st));
+  TG_TRY(sk_clear(P, st));
   // packed rows in, padding rows zero
   for (int b = 0; b < batch; ++b) {
     const int64_t n = sn.len[b], pad = static_cast<int64_t>(align_up(size_t(n), kSegAlign)) - n;
@@ -1363,9 +1492,12 @@ tg_status tg_prefill_batch(const tg_model* model, const void* x, const uint8_t* 
   }
   float* sc = P.scores;
   TG_TRY(run_score(P.h, n_pad, D.d, m.d_score, m.score_norm, m.norm_eps, m.score_w1, m.score_b1,
-                   m.score_w2, m.score_b2, m.dtype, sc, P.y, P.hpre, st));
-  // per request: select, compact into its padded block of kept rows
+                   m.score_w2, m.score_b2, m.dtype, sc, P.y, P.hpre, st, &P, m.score_w1_g));
+  // per request: select, compact into its padded block of kept rows (with
+  // the rows' sums of squares when h's are current; padding rows get 0)
   TG_TRY(cudaMemsetAsync(P.pos_k, 0, size_t(k_pad) * 4, st));
+  const bool carry = ss_ready(P, P.h, n_pad) && P.ss_parts <= 32;
+  if (carry) TG_TRY(cudaMemsetAsync(P.ss_k, 0, size_t(P.ss_parts) * P.ss_ld_k * 4, st));
   int64_t ck = 0;
   for (int b = 0; b < batch; ++b) {
     const int64_t n = sn.len[b], k = sk.len[b];
@@ -1373,13 +1505,18 @@ tg_status tg_prefill_batch(const tg_model* model, const void* x, const uint8_t* 
                                        cudaMemcpyDeviceToDevice, st));
     TG_TRY(select_topk(sc + sn.off[b], protect ? protect + cu_n[b] : nullptr, n, k, kept_idx + ck,
                        P.sel_ws, st));
+    SsGather sg;
+    if (carry)
+      sg = SsGather{P.ss + sn.off[b], P.ss_ld, P.ss_k + sk.off[b], P.ss_ld_k, P.ss_parts};
     TG_TRY(compact(h + sn.off[b] * row, nullptr, sc + sn.off[b], kept_idx + ck, n, k,
                    static_cast<int>(row), hk + sk.off[b] * row, P.pos_k + sk.off[b],
-                   P.s_k + sk.off[b], P.lsig_k + sk.off[b], st));
+                   P.s_k + sk.off[b], P.lsig_k + sk.off[b], st, sg));
     const int64_t pad = static_cast<int64_t>(align_up(size_t(k), kSegAlign)) - k;
     if (pad > 0) TG_TRY(cudaMemsetAsync(hk + (sk.off[b] + k) * row, 0, pad * row, st));
     ck += k;
   }
+  if (carry) ss_mark(P, P.hk, k_pad);
+  else if (P.ss_for == P.hk) P.ss_for = nullptr;
   TG_TRY(traced(TG_K_ROPE_TABLE, k_pad, 0.0, cs_bytes * k_pad + 4.0 * k_pad, st, [&] {
     return launch_rope_table(P.pos_k, k_pad, D.dh, m.rope_base, P.cs_k, st);
   }));
@@ -1634,7 +1771,8 @@ const char* tg_kernel_name(int32_t kernel) {
       "copy", "rmsnorm", "gemm_tc_store", "gemm_tc_residual", "gemm_tc_swiglu", "gemm_tc_score",
       "rope_prep", "attention_tc", "select", "compact", "gemm_f32", "attention_f32", "f32_helper",
       "gemm_tc_qkv", "rope_table", "decode_step", "attn_bwd_prep", "attn_bwd_dkdv",
-      "attn_bwd_dq", "attn_bwd_final", "gdn_prep", "gdn_chunk", "gdn_recur", "gdn_out"};
+      "attn_bwd_dq", "attn_bwd_final", "gdn_prep", "gdn_chunk", "gdn_recur", "gdn_out",
+      "fold_norm"};
   return (kernel >= 0 && kernel < TG_K_COUNT) ? names[kernel] : "unknown";
 }
 

@@ -71,12 +71,24 @@ cudaError_t launch_topk_select_noalloc(const float* scores, const uint8_t* prote
                                        int64_t k, int32_t* kept_idx, cudaStream_t st);
 
 // ---- compaction (k_compact.cu). Optional lsig_out[r] = logsigmoid(scores[idx[r]]).
+// Optional row sums of squares (folded RMSNorm): ss_out[p * ss_ld_out + r] =
+// ss_in[p * ss_ld_in + idx[r]] for p < ss_parts.
+struct SsGather {
+  const float* in = nullptr;
+  int64_t ld_in = 0;
+  float* out = nullptr;
+  int64_t ld_out = 0;
+  int parts = 0;
+};
 cudaError_t launch_compact(const void* x, const int32_t* pos_in, const float* scores,
                            const int32_t* kept_idx, int64_t n, int64_t k, int row_bytes,
                            void* x_out, int32_t* pos_out, float* scores_out, float* lsig_out,
-                           cudaStream_t st);
+                           const SsGather& ss, cudaStream_t st);
 
 // ---- row-wise kernels (k_rowwise.cu)
+// W_g = bf16(W . diag(g)) for bf16 W [rows, cols] (tg_fold_norm_weight)
+cudaError_t launch_fold_norm_weight(const void* w, const float* g, int64_t rows, int64_t cols,
+                                    void* out, cudaStream_t st);
 cudaError_t launch_rmsnorm(const void* x, const float* gamma, float eps, int64_t rows, int d,
                            bool bf16, void* y, cudaStream_t st);
 
@@ -143,7 +155,29 @@ struct GemmArgs {
   int hq, hkv;
   const float2* rope_cs; const float* q_norm; const float* k_norm; float eps;
   void* q_out; void* k_out; void* vT_out; int64_t t_pad; void* v_out;
+  // Folded RMSNorm (tensor-core path only). RESIDUAL: ss_out[nb * ss_ld + m]
+  // = sum of squares of the stored bf16 row m over the tile column block nb
+  // (256 columns; ceil(N / 256) blocks). STORE / SWIGLU / SCORE / QKV: when
+  // ss_in is set, row m of the accumulator is scaled by
+  // 1 / sqrt(ss_inv_n * sum_{p < ss_parts} ss_in[p * ss_ld + m] + ss_eps)
+  // before the epilogue's own math (B holding W . diag(g)).
+  float* ss_out = nullptr;
+  const float* ss_in = nullptr;
+  int64_t ss_ld = 0;
+  int ss_parts = 0;
+  float ss_inv_n = 0.f, ss_eps = 0.f;
+  // Optional stream-K scratch (tensor-core path): partial sums and flags,
+  // gemm_sk_bytes(); the flags must be zero before the first launch that
+  // uses it (launches leave them zero).
+  void* sk_ws = nullptr;
+  size_t sk_ws_bytes = 0;
 };
+constexpr int kSkMaxPairs = 96;
+constexpr size_t gemm_sk_flag_offset() { return size_t(kSkMaxPairs) * 2 * 64 * 128 * 16; }
+constexpr size_t gemm_sk_bytes() { return gemm_sk_flag_offset() + size_t(kSkMaxPairs) * 2 * 4; }
+// tile column blocks of a residual GEMM's row sums of squares
+constexpr int kSsBlockCols = 256;
+inline int ss_parts_of(int n) { return (n + kSsBlockCols - 1) / kSsBlockCols; }
 // bf16 on the 5th-generation tensor cores (k_gemm_tc.cu)
 bool gemm_tc_supported(const GemmArgs& g);
 cudaError_t launch_gemm_tc(const GemmArgs& g, cudaStream_t st);

@@ -273,45 +273,56 @@ def gdn_sublayer(x, lw: GdnStackLayer, eps: float, store=round_fp32):
     return r, (res.conv_state, res.S)
 
 
-def hybrid_prefill(x, protect, k: int, m, gate_layer: int, store=round_fp32, kept_idx=None):
+def hybrid_prefill(x, protect, k: int, m, gate_layer: int, store=round_fp32, kept_idx=None,
+                   fold_norms: bool = False):
     """The gated forward of a hybrid stack (G11). m is a tokengate_oracle
     Model whose layers are attention Layers or GdnStackLayers. Returns a
     PrefillResult; kv holds, per layer, the attention (k, v) or the Gated
-    DeltaNet (conv rows, S)."""
+    DeltaNet (conv rows, S). fold_norms: as in tokengate_oracle.prefill (R7b);
+    a Gated DeltaNet layer's input projection is never folded."""
     from .tokengate_oracle import (PrefillResult, attention_sublayer, compact, ffn_sublayer,
                                    score, topk_select)
 
-    def mix(h, lw, pos, s, gated):
+    def mix(h, lw, pos, s, gated, fresh):
         if isinstance(lw, GdnStackLayer):
             return gdn_sublayer(h, lw, m.eps, store)
+        fold = fold_norms and fresh
         if gated:
-            return attention_sublayer(h, lw, m, pos, s, lw.gain, lw.tau, store)
-        return attention_sublayer(h, lw, m, pos, None, None, None, store)
+            return attention_sublayer(h, lw, m, pos, s, lw.gain, lw.tau, store, fold)
+        return attention_sublayer(h, lw, m, pos, None, None, None, store, fold)
 
     x = store(np.asarray(x, dtype=F64))
     n = x.shape[0]
     pos = np.arange(n, dtype=np.int32)
     kv = []
     h = x
+    fresh = False  # rows just written by a residual GEMM (R7b)
     for li in range(max(gate_layer, 0)):
-        r, st = mix(h, m.layers[li], pos, None, False)
+        r, st = mix(h, m.layers[li], pos, None, False, fresh)
         kv.append(st)
-        h = ffn_sublayer(r, m.layers[li], m, store)
+        h = ffn_sublayer(r, m.layers[li], m, store, fold_norms)
+        fresh = True
     if gate_layer >= 0:
-        r, st = mix(h, m.layers[gate_layer], pos, None, False)
+        r, st = mix(h, m.layers[gate_layer], pos, None, False, fresh)
         kv.append(st)
+        fresh = True
     else:
         r = h
     s = round_fp32(score(r, m.score_norm, m.eps, m.score_w1, m.score_b1, m.score_w2,
-                         m.score_b2, store))
+                         m.score_b2, store, fold_norms and fresh))
     idx = topk_select(s.astype(np.float32), protect, k) if kept_idx is None \
         else np.asarray(kept_idx, dtype=np.int32)
-    x_k, pos_k, s_k = compact(r, idx, pos, s)
-    h = ffn_sublayer(x_k, m.layers[gate_layer], m, store) if gate_layer >= 0 else x_k
+    x_k, pos_k, s_k = compact(r, idx, pos, s)  # rows keep their freshness
+    if gate_layer >= 0:
+        h = ffn_sublayer(x_k, m.layers[gate_layer], m, store, fold_norms and fresh)
+        fresh = fresh or m.layers[gate_layer].w_gate_up is not None
+    else:
+        h = x_k
     for li in range(gate_layer + 1, len(m.layers)):
-        r, st = mix(h, m.layers[li], pos_k, s_k, True)
+        r, st = mix(h, m.layers[li], pos_k, s_k, True, fresh)
         kv.append(st)
-        h = ffn_sublayer(r, m.layers[li], m, store)
+        h = ffn_sublayer(r, m.layers[li], m, store, fold_norms)
+        fresh = True
     from .tokengate_oracle import rmsnorm
     out = h if m.final_norm is None else store(rmsnorm(h, m.final_norm, m.eps))
     return PrefillResult(out=out, kept_idx=idx, scores=s.astype(np.float32), kv=kv,

@@ -60,6 +60,15 @@ Readings where the pages are silent (each one is listed in the design notes):
       its logits over the cached keys follow R2, with the kept prompt tokens'
       scores as the bias and no bias (logsigmoid = 0) on generated tokens'
       keys; tau applies to every key.
+  R7b Folded RMSNorm (an implementation form of R6, not from the pages):
+      RMSNorm(x; g) . W^T = (x / rms(x)) . (W diag g)^T in real arithmetic.
+      When the library runs a projection with the folded weight
+      W_g = W diag(g) (stored once, in the compute dtype), the normed row is
+      never stored, so by R7 the rounding point moves from the normed row
+      to W_g. It does so where the norm's input rows were just written by a
+      residual GEMM (`fresh` below; the compaction gathers the rows' sums of
+      squares with them): every norm but the stack's input and a Gated
+      DeltaNet layer's input projection.
   R9  Backward: the gradients of the gated attention with respect to q, k,
       v, the gate scores s, the per-head gain and the per-head temperature,
       for an upstream gradient of its output. The pages give only the path
@@ -125,6 +134,18 @@ def rmsnorm(x, gamma, eps: float) -> np.ndarray:
     return x / np.sqrt(ms + eps) * np.asarray(gamma, dtype=F64)
 
 
+def norm_project(x, gamma, w, eps: float, store, fold: bool = False) -> np.ndarray:
+    """RMSNorm(x; gamma) . w^T, unrounded. fold=False: the normed rows are a
+    stored GEMM operand (R7): store(RMSNorm(x)) . w^T. fold=True (R7b): the
+    folded weight is the stored operand: (x / rms(x)) . store(w diag gamma)^T."""
+    w = np.asarray(w, dtype=F64)
+    if not fold:
+        return store(rmsnorm(x, gamma, eps)) @ w.T
+    x = np.asarray(x, dtype=F64)
+    inv_rms = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return (x * inv_rms) @ store(w * np.asarray(gamma, dtype=F64)).T
+
+
 def sigmoid(x) -> np.ndarray:
     """1 / (1 + exp(-x)), written as exp(x) / (1 + exp(x)) for x < 0 so
     that no exponential overflows and small values keep full precision."""
@@ -149,18 +170,18 @@ def logsigmoid(x) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 
-def score(r, norm_w, eps, w1, b1, w2, b2, store: Callable = round_bf16) -> np.ndarray:
+def score(r, norm_w, eps, w1, b1, w2, b2, store: Callable = round_bf16,
+          fold: bool = False) -> np.ndarray:
     """Importance score of each token from its post-attention residual.
 
     s_t = w2 . SiLU(W1 . RMSNorm(r_t) + b1) + b2   (R1)
 
     r: [N, d]; w1: [F, d]; b1: [F] or None; w2: [F]; b2: scalar or None.
-    The normalised rows are rounded by `store` (they are a GEMM operand).
-    Returns float64 scores; a caller that needs the stored value rounds them
-    to float32.
+    The normalised rows are rounded by `store` (they are a GEMM operand), or
+    with fold the folded weight is (R7b). Returns float64 scores; a caller
+    that needs the stored value rounds them to float32.
     """
-    y = store(rmsnorm(r, norm_w, eps))
-    h = y @ np.asarray(w1, dtype=F64).T
+    h = norm_project(r, norm_w, w1, eps, store, fold)
     if b1 is not None:
         h = h + np.asarray(b1, dtype=F64)
     s = silu(h) @ np.asarray(w2, dtype=F64).reshape(-1)
@@ -452,13 +473,12 @@ class Model:
     rope_base: float = 1e6
 
 
-def project_qkv(x, lw: Layer, m: Model, pos, store):
+def project_qkv(x, lw: Layer, m: Model, pos, store, fold: bool = False):
     """Rows x [t, d] -> q [t, Hq, dh] and k [t, Hkv, dh] (qk-norm, then RoPE at
-    pos, stored) and v [t, Hkv, dh] (stored) (R4, R6, R7)."""
+    pos, stored) and v [t, Hkv, dh] (stored) (R4, R6, R7; fold: R7b)."""
     t = x.shape[0]
     hq, hkv, dh = m.n_heads_q, m.n_heads_kv, m.head_dim
-    y = store(rmsnorm(x, lw.attn_norm, m.eps))
-    qkv = store(y @ np.asarray(lw.wqkv, dtype=F64).T)
+    qkv = store(norm_project(x, lw.attn_norm, lw.wqkv, m.eps, store, fold))
     q = qkv[:, : hq * dh].reshape(t, hq, dh)
     k = qkv[:, hq * dh : (hq + hkv) * dh].reshape(t, hkv, dh)
     v = qkv[:, (hq + hkv) * dh :].reshape(t, hkv, dh)
@@ -468,22 +488,21 @@ def project_qkv(x, lw: Layer, m: Model, pos, store):
     return store(rope(q, pos, m.rope_base)), store(rope(k, pos, m.rope_base)), v
 
 
-def attention_sublayer(x, lw: Layer, m: Model, pos, s, gain, tau, store):
+def attention_sublayer(x, lw: Layer, m: Model, pos, s, gain, tau, store, fold: bool = False):
     """r = x + Wo . attn(RoPE(qk-norm(W_qkv . RMSNorm(x)))) and the layer's KV."""
     t = x.shape[0]
-    q, k, v = project_qkv(x, lw, m, pos, store)
+    q, k, v = project_qkv(x, lw, m, pos, store, fold)
     o = store(gated_attention(q, k, v, pos, s, gain, tau))
     r = store(x + o.reshape(t, m.n_heads_q * m.head_dim) @ np.asarray(lw.wo, dtype=F64).T)
     return r, (k, v)
 
 
-def ffn_sublayer(x, lw: Layer, m: Model, store):
+def ffn_sublayer(x, lw: Layer, m: Model, store, fold: bool = False):
     """x + W_down . (SiLU(W_gate . y) * (W_up . y)), y = RMSNorm(x)."""
     if lw.w_gate_up is None:
         return x
     inter = lw.w_gate_up.shape[0] // 2
-    y = store(rmsnorm(x, lw.ffn_norm, m.eps))
-    gu = y @ np.asarray(lw.w_gate_up, dtype=F64).T
+    gu = norm_project(x, lw.ffn_norm, lw.w_gate_up, m.eps, store, fold)
     h = store(silu(gu[:, :inter]) * gu[:, inter:])
     return store(x + h @ np.asarray(lw.w_down, dtype=F64).T)
 
@@ -498,7 +517,7 @@ class PrefillResult:
 
 
 def prefill(x, protect, k: int, m: Model, gate_layer: int, store=round_bf16,
-            kept_idx=None) -> PrefillResult:
+            kept_idx=None, fold_norms: bool = False) -> PrefillResult:
     """The three-stage gated forward ([TC] "TokenGate 提前筛选 Token";
     [FW] "论文的方法"; [AI] "可学习剪枝的机制设计").
 
@@ -511,49 +530,61 @@ def prefill(x, protect, k: int, m: Model, gate_layer: int, store=round_bf16,
 
     kept_idx, when given, replaces the oracle's own selection (teacher
     forcing): the later stages then consume exactly that kept set.
+
+    fold_norms (R7b): a norm whose input rows come straight from a residual
+    GEMM (`fresh`) rounds the folded weight instead of the normed rows.
     """
     x = store(np.asarray(x, dtype=F64))
     n = x.shape[0]
     pos = np.arange(n, dtype=np.int32)
     kv = []
     h = x
+    fresh = False  # the input rows were not written by a residual GEMM
     for li in range(max(gate_layer, 0)):
-        r, kvl = attention_sublayer(h, m.layers[li], m, pos, None, None, None, store)
+        r, kvl = attention_sublayer(h, m.layers[li], m, pos, None, None, None, store,
+                                    fold_norms and fresh)
         kv.append(kvl)
-        h = ffn_sublayer(r, m.layers[li], m, store)
+        h = ffn_sublayer(r, m.layers[li], m, store, fold_norms)
+        fresh = True
     if gate_layer >= 0:
         lw = m.layers[gate_layer]
-        r, kvl = attention_sublayer(h, lw, m, pos, None, None, None, store)
+        r, kvl = attention_sublayer(h, lw, m, pos, None, None, None, store, fold_norms and fresh)
         kv.append(kvl)
+        fresh = True
     else:
         r = h
     s = round_fp32(score(r, m.score_norm, m.eps, m.score_w1, m.score_b1, m.score_w2,
-                         m.score_b2, store))
+                         m.score_b2, store, fold_norms and fresh))
     idx = topk_select(s.astype(np.float32), protect, k) if kept_idx is None \
         else np.asarray(kept_idx, dtype=np.int32)
-    x_k, pos_k, s_k = compact(r, idx, pos, s)
+    x_k, pos_k, s_k = compact(r, idx, pos, s)  # rows keep their freshness (R7b)
     if gate_layer >= 0:
-        h = ffn_sublayer(x_k, m.layers[gate_layer], m, store)
+        lw = m.layers[gate_layer]
+        h = ffn_sublayer(x_k, lw, m, store, fold_norms and fresh)
+        fresh = fresh or lw.w_gate_up is not None
     else:
         h = x_k
     for li in range(gate_layer + 1, len(m.layers)):
         lw = m.layers[li]
-        r, kvl = attention_sublayer(h, lw, m, pos_k, s_k, lw.gain, lw.tau, store)
+        r, kvl = attention_sublayer(h, lw, m, pos_k, s_k, lw.gain, lw.tau, store,
+                                    fold_norms and fresh)
         kv.append(kvl)
-        h = ffn_sublayer(r, lw, m, store)
+        h = ffn_sublayer(r, lw, m, store, fold_norms)
+        fresh = True
     out = h if m.final_norm is None else store(rmsnorm(h, m.final_norm, m.eps))
     return PrefillResult(out=out, kept_idx=idx, scores=s.astype(np.float32), kv=kv,
                          gate_residual=r if gate_layer < 0 else None)
 
 
 def prefill_budgets(x, protect, ks, m: Model, gate_layer: int, store=round_bf16,
-                    kept_sets=None) -> List[PrefillResult]:
+                    kept_sets=None, fold_norms: bool = False) -> List[PrefillResult]:
     """The gated forward of one request at several budgets: by definition the
     single-budget forward at each k of ks (one trained gate serves every
     budget, [AI] "可学习剪枝的机制设计"). kept_sets, when given, teacher-forces
     each budget's kept set."""
     return [prefill(x, protect, k, m, gate_layer, store,
-                    None if kept_sets is None else kept_sets[b]) for b, k in enumerate(ks)]
+                    None if kept_sets is None else kept_sets[b], fold_norms)
+            for b, k in enumerate(ks)]
 
 
 def decode_step(x, pos: int, m: Model, gate_layer: int, cache, kept_scores=None,
@@ -613,11 +644,13 @@ def decode_bytes(m: Model, lens, elem: int = 2) -> int:
     return total
 
 
-def gated_layer_forward(x_k, pos_k, s_k, lw: Layer, m: Model, store=round_bf16):
-    """One upper (gated) layer over already-compacted rows: attention + FFN."""
+def gated_layer_forward(x_k, pos_k, s_k, lw: Layer, m: Model, store=round_bf16,
+                        fold_norms: bool = False):
+    """One upper (gated) layer over already-compacted rows: attention + FFN
+    (the FFN's input rows come from the attention's residual GEMM, R7b)."""
     r, kv = attention_sublayer(np.asarray(x_k, dtype=F64), lw, m, pos_k, s_k,
                                lw.gain, lw.tau, store)
-    return ffn_sublayer(r, lw, m, store), kv
+    return ffn_sublayer(r, lw, m, store, fold_norms), kv
 
 
 # ---------------------------------------------------------------------------

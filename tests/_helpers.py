@@ -46,7 +46,7 @@ def device_params(params: dict, dtype):
     return out
 
 
-def build_models(w, rng, dtype):
+def build_models(w, rng, dtype, fold_norms=True):
     """(library Model, oracle Model) holding identical values."""
     import learned_token_pruning_score_b200 as tg
     import synth
@@ -57,7 +57,7 @@ def build_models(w, rng, dtype):
                                                "score_b2")}, dtype)
     final_d = dev(p["final_norm"])
     m = tg.Model(n_heads_q=w.hq, n_heads_kv=w.hkv, head_dim=w.dh, layers=layers_d, score=score_d,
-                 final_norm=final_d, eps=w.eps, rope_base=w.rope_base)
+                 final_norm=final_d, eps=w.eps, rope_base=w.rope_base, fold_norms=fold_norms)
     o_layers = []
     for ld in layers_d:
         g = lambda k: host64(ld[k]) if k in ld else None  # noqa: E731

@@ -202,6 +202,38 @@ def test_prefill_validation():
     assert _prefill(ctypes.byref(m), 1000, 100, 1, big) == tg.TG_ERR_INVALID_ARG
 
 
+def test_prefill_validation_folded_norm_weights():
+    """The optional folded-norm weights: bf16 models only, 16-byte aligned
+    (they are TMA operands), and the FFN one only beside an FFN."""
+    big = 1 << 40
+    m, keep = _bogus_model()
+    keep[1].wqkv_g = 4096 + 8
+    assert _prefill(ctypes.byref(m), 1000, 100, 1, big) == tg.TG_ERR_INVALID_ARG
+    m, keep = _bogus_model()
+    keep[0].w_gate_up_g = 4096 + 2
+    assert _prefill(ctypes.byref(m), 1000, 100, 1, big) == tg.TG_ERR_INVALID_ARG
+    m, keep = _bogus_model(score_w1_g=4096 + 4)
+    assert _prefill(ctypes.byref(m), 1000, 100, 1, big) == tg.TG_ERR_INVALID_ARG
+    m, keep = _bogus_model(dtype=tg.TG_F32)
+    assert _prefill(ctypes.byref(m), 1000, 100, 1, big) == tg.TG_ERR_UNSUPPORTED
+    m, keep = _bogus_model(dtype=tg.TG_F32)
+    for i in range(2):
+        keep[i].wqkv_g = keep[i].w_gate_up_g = None
+    assert _prefill(ctypes.byref(m), 1000, 100, 1, 16) == tg.TG_ERR_WORKSPACE  # valid otherwise
+
+
+def test_fold_norm_weight_validation():
+    f = tg._fold
+    w, g, out = 4096, 1 << 20, 1 << 24
+    assert f(None, g, 2, 8, out, None) == tg.TG_ERR_INVALID_ARG
+    assert f(w, None, 2, 8, out, None) == tg.TG_ERR_INVALID_ARG
+    assert f(w, g, 2, 8, None, None) == tg.TG_ERR_INVALID_ARG
+    assert f(w, g, 0, 8, out, None) == tg.TG_ERR_INVALID_ARG
+    assert f(w, g, 2, 0, out, None) == tg.TG_ERR_INVALID_ARG
+    assert f(w, g, 2, 8, w + 16, None) == tg.TG_ERR_INVALID_ARG  # out overlaps w (32 bytes)
+    assert f(w, g, 2, 8, w, None) == tg.TG_ERR_INVALID_ARG
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="exercises the no-device error path")
 def test_device_error_without_a_device_is_a_cuda_error():
     with pytest.raises(tg.TokenGateError) as ei:
@@ -329,8 +361,8 @@ def test_gated_deltanet_validation():
     base = 1 << 24
     assert call(conv_in=base, conv_out=base + 64) == tg.TG_ERR_INVALID_ARG
     assert call(s_in=base, s_out=base + 4) == tg.TG_ERR_INVALID_ARG
-    names = [tg._kernel_name(i).decode() for i in (20, 21, 22, 23, 24)]
-    assert names == ["gdn_prep", "gdn_chunk", "gdn_recur", "gdn_out", "unknown"]
+    names = [tg._kernel_name(i).decode() for i in (20, 21, 22, 23, 24, 25)]
+    assert names == ["gdn_prep", "gdn_chunk", "gdn_recur", "gdn_out", "fold_norm", "unknown"]
 
 
 def test_selftest_wait_validation():

@@ -136,6 +136,8 @@ def assert_within_budget(gpu, want, budget, what):
         i = np.unravel_index(np.argmax(np.where(bad, d / lim, -1)), d.shape)
         raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} outside the budget; worst at "
                              f"{i}: gpu={g[i]!r} ref={w[i]!r} budget={lim[i]:.3e}")
+    if d.size <= 64:  # per-head scalars (dgain, dtau): the budget per element only
+        return
     rms_err = math.sqrt(float(np.mean(d * d))) if d.size else 0.0
     assert rms_err <= 1e-2 * max(rms, 1e-3), f"{what}: rms error {rms_err:.3e} vs rms {rms:.3e}"
 

@@ -73,7 +73,7 @@ def test_batch_against_the_oracle():
         kb = kept_np[k0:k0 + k]
         assert np.array_equal(kb, ref.topk_select(scores[r0:r0 + n], prots[b], k))
         res = ref.prefill(xh[r0:r0 + n], prots[b], k, om, 1, store=STORE[torch.bfloat16],
-                          kept_idx=kb)
+                          kept_idx=kb, fold_norms=model.fold_norms)
         assert_close(scores[r0:r0 + n], res.scores, torch.bfloat16, f"scores request {b}")
         assert_close(out[k0:k0 + k], res.out, torch.bfloat16, f"out request {b}")
         r0 += n

@@ -128,6 +128,11 @@ def _check_stack(w, gate):
     assert np.array_equal(kept, ref.topk_select(scores, prot, b.k))
     s_k = scores[kept].astype(np.float64)
     h_in = host64(x)
+    # folded norms (the model's default): a norm whose rows a residual GEMM
+    # just wrote runs on the folded weight; a Gated DeltaNet input projection
+    # never does
+    fold = model.fold_norms
+    fresh = False
     if gate < 0:  # the gate before the stack: the scorer reads x, the layers see x[kept]
         s_ref = ref.round_fp32(ref.score(h_in, om.score_norm, om.eps, om.score_w1, om.score_b1,
                                          om.score_w2, om.score_b2, rb))
@@ -152,7 +157,7 @@ def _check_stack(w, gate):
             assert_close(kv[li][1], res.S, BF16, f"state {what}")
             r = rb(h_in + mix_gpu @ lw.w_out.T)
         else:
-            q, k_o, v_o = ref.project_qkv(h_in, lw, om, pos, rb)
+            q, k_o, v_o = ref.project_qkv(h_in, lw, om, pos, rb, fold and fresh)
             assert_close(kv[li][0], k_o, BF16, f"k {what}")
             assert_close(kv[li][1], v_o, BF16, f"v {what}")
             o = rb(ref.gated_attention(q, host64(kv[li][0]), host64(kv[li][1]), pos,
@@ -162,15 +167,18 @@ def _check_stack(w, gate):
             r = rb(h_in + mix_gpu @ lw.wo.T)
         r_gpu = host64(taps[li]["resid"])
         assert_close(r_gpu, r, BF16, f"post-mixer residual {what}")
+        fresh = True
         if li == gate:
             s_ref = ref.round_fp32(ref.score(r_gpu, om.score_norm, om.eps, om.score_w1,
-                                             om.score_b1, om.score_w2, om.score_b2, rb))
+                                             om.score_b1, om.score_w2, om.score_b2, rb, fold))
             assert_close(scores, s_ref, BF16, "scores")
             flips, near = boundary_flips(s_ref.astype(np.float32), kept, prot, b.k, 2e-2, 1e-2)
             assert near, flips
-            r_gpu = r_gpu[kept]
+            r_gpu = r_gpu[kept]  # the compacted rows keep their row sums
         h_gpu = host64(taps[li]["hidden"])
-        assert_close(h_gpu, ref.ffn_sublayer(r_gpu, lw, om, rb), BF16, f"hidden {what}")
+        assert_close(h_gpu, ref.ffn_sublayer(r_gpu, lw, om, rb, fold and fresh), BF16,
+                     f"hidden {what}")
+        fresh = True
         h_in = h_gpu
     assert_close(out, rb(ref.rmsnorm(h_in, om.final_norm, om.eps)), BF16, "out")
 

@@ -71,7 +71,7 @@ def test_multi_budget_against_the_oracle():
     for b, k in enumerate(ks):
         assert np.array_equal(kept_np[b], ref.topk_select(scores, prot_np, k))
     res = ref.prefill_budgets(host64(x), prot_np, ks, om, 1, store=STORE[torch.bfloat16],
-                              kept_sets=kept_np)
+                              kept_sets=kept_np, fold_norms=model.fold_norms)
     for b, r in enumerate(res):
         assert_close(scores, r.scores, torch.bfloat16, "scores")
         assert_close(outs[b], r.out, torch.bfloat16, f"out k={ks[b]}")

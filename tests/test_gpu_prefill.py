@@ -28,10 +28,10 @@ def _no_device_errors():
     assert tg.tg_device_error() == 0
 
 
-def _run(w, want_kv=True, seed=None):
+def _run(w, want_kv=True, seed=None, fold_norms=True):
     dtype = DT[w.dtype]
     rng = synth.rng_for(w.seed if seed is None else seed)
-    model, om = build_models(w, rng, dtype)
+    model, om = build_models(w, rng, dtype, fold_norms)
     x_np = synth.hidden_states(w, rng)
     x = torch.from_numpy(x_np).to("cuda", dtype)
     prot_np = synth.protect_tail(w.n, w.n_protect)
@@ -56,7 +56,7 @@ def _check_against_oracle(w, r):
     assert np.array_equal(r["kept"], ref.topk_select(r["scores"], r["prot"], w.k))
     # 2. teacher-forced oracle run
     res = ref.prefill(host64(r["x"]), r["prot"], w.k, r["om"], w.gate_layer,
-                      store=STORE[dtype], kept_idx=r["kept"])
+                      store=STORE[dtype], kept_idx=r["kept"], fold_norms=r["model"].fold_norms)
     assert_close(r["scores"], res.scores, dtype, "scores")
     assert_close(r["out"], res.out, dtype, "out")
     if r["kv"] is not None:
@@ -79,13 +79,29 @@ def test_tiny_fp32_gated_block():
     _check_against_oracle(synth.TINY_F32, _run(synth.TINY_F32))
 
 
+@pytest.mark.parametrize("fold_norms", [True, False])
 @pytest.mark.parametrize("qk_norm", [False, True])
 @pytest.mark.parametrize("gate_layer", [-1, 0, 1])
-def test_small_bf16_stack(qk_norm, gate_layer):
+def test_small_bf16_stack(qk_norm, gate_layer, fold_norms):
+    """fold_norms: the RMSNorms after a residual GEMM folded into the next
+    projection (its weight times the norm weight, its accumulator rows over
+    the rms), or the norm kernel before every projection."""
     w = synth.shrink(synth.QWEN_LAYER_16K, name="small", n=300, k=100, d=256, hq=4, hkv=2, dh=128,
                      f=64, inter=256, n_layers=3, gate_layer=gate_layer, n_protect=10,
                      qk_norm=qk_norm, seed=40 + gate_layer, salient_frac=0.02)
-    _check_against_oracle(w, _run(w))
+    _check_against_oracle(w, _run(w, fold_norms=fold_norms))
+
+
+@pytest.mark.parametrize("rows,cols", [(3, 8), (17, 2048), (5, 13), (1, 1)])
+def test_fold_norm_weight_is_exact(rows, cols):
+    """W_g = bf16(W . diag(g)): one product and one round-to-nearest-even per
+    element (the vector path for cols % 8 == 0, the scalar one otherwise)."""
+    gen = torch.Generator(device="cuda").manual_seed(rows * 1000 + cols)
+    w = (torch.randn(rows, cols, device="cuda", generator=gen) * 3).to(torch.bfloat16)
+    g = torch.rand(cols, device="cuda", generator=gen) * 2 - 0.5
+    out = tg.tg_fold_norm_weight(w, g)
+    torch.cuda.synchronize()
+    assert torch.equal(out, (w.float() * g).to(torch.bfloat16))
 
 
 def test_small_fp32_stack():

@@ -101,9 +101,9 @@ def _run_gpu(w, model, x, prot, with_taps=False):
     return out, kept.cpu().numpy(), scores.cpu().numpy(), kv, taps
 
 
-def _check_scores(r_gpu, om, scores_gpu, what):
+def _check_scores(r_gpu, om, scores_gpu, what, fold):
     s_ref = ref.round_fp32(ref.score(r_gpu, om.score_norm, om.eps, om.score_w1, om.score_b1,
-                                     om.score_w2, om.score_b2, rb))
+                                     om.score_w2, om.score_b2, rb, fold))
     assert_close(scores_gpu, s_ref, BF16, what)
     return s_ref
 
@@ -118,12 +118,16 @@ def test_prefill_28_layers_reduced_n_per_layer():
     pos_n = np.arange(w.n)
     s_k = scores[kept].astype(np.float64)
     h_in = host64(x)
+    # folded norms (the default): every norm whose rows a residual GEMM just
+    # wrote (the compacted rows keep their row sums), i.e. all but layer 0's
+    # attention norm
+    fold = model.fold_norms
     for li in range(w.n_layers):
         lw = om.layers[li]
         dense = li <= w.gate_layer
         pos = pos_n if dense else kept
         rows = pos.size
-        q, k_o, v_o = ref.project_qkv(h_in, lw, om, pos, rb)
+        q, k_o, v_o = ref.project_qkv(h_in, lw, om, pos, rb, fold and li > 0)
         assert_close(kv[li][0], k_o, BF16, f"k layer {li}")
         assert_close(kv[li][1], v_o, BF16, f"v layer {li}")
         o = rb(ref.gated_attention(q, host64(kv[li][0]), host64(kv[li][1]), pos,
@@ -135,24 +139,25 @@ def test_prefill_28_layers_reduced_n_per_layer():
         r_gpu = host64(taps[li]["resid"])
         assert_close(r_gpu, r, BF16, f"post-attention residual layer {li}")
         if li == w.gate_layer:
-            s_ref = _check_scores(r_gpu, om, scores, "scores")
+            s_ref = _check_scores(r_gpu, om, scores, "scores", fold)
             flips, near = boundary_flips(s_ref.astype(np.float32), kept, prot, w.k, 2e-2, 1e-2)
             assert near, flips
             r_gpu = r_gpu[kept]
         h_gpu = host64(taps[li]["hidden"])
-        assert_close(h_gpu, ref.ffn_sublayer(r_gpu, lw, om, rb), BF16, f"hidden layer {li}")
+        assert_close(h_gpu, ref.ffn_sublayer(r_gpu, lw, om, rb, fold), BF16,
+                     f"hidden layer {li}")
         h_in = h_gpu  # teacher forcing: the next layer reads the GPU's output
     assert_close(out, rb(ref.rmsnorm(h_in, om.final_norm, om.eps)), BF16, "out")
 
 
 def _attn_row(h, lw, m, pos_q, k_cache, v_cache, pos_k, s_k, gain, tau, want_k, want_v, o_gpu,
-              r_gpu, what):
+              r_gpu, what, fold):
     """One token through one layer's attention sub-layer, teacher-forced:
     its q, k, v from the GPU's input row h (k, v checked against the GPU's
     cache row), its attention output from the GPU's cached keys/values
     [0..its own row] (checked against o_gpu), its residual from o_gpu
     (checked against r_gpu)."""
-    q, k, v = ref.project_qkv(h[None], lw, m, np.array([pos_q]), rb)
+    q, k, v = ref.project_qkv(h[None], lw, m, np.array([pos_q]), rb, fold)
     assert_close(want_k, k[0], BF16, f"k {what}")
     assert_close(want_v, v[0], BF16, f"v {what}")
     o = rb(ref.gated_attention_rows(q, np.array([pos_q]), k_cache, v_cache, pos_k, s_k, gain,
@@ -189,6 +194,7 @@ def test_prefill_28_layers_full_size_sampled_rows(k, dense):
     tokens = sample_kept + sample_pruned
     row_of = {int(t): r for r, t in enumerate(kept)}
     s_kept = scores[kept].astype(np.float64)
+    fold = model.fold_norms  # all norms but layer 0's attention
     rows = lambda t_, idx: host64(t_[torch.as_tensor(idx, device="cuda")])  # noqa: E731
     xin = dict(zip(tokens, rows(x, tokens)))
     for li in range(w.n_layers):
@@ -202,19 +208,19 @@ def test_prefill_28_layers_full_size_sampled_rows(k, dense):
             for t in tokens:
                 what = f"layer {li} token {t}"
                 _attn_row(hin[t], lw, om, t, kc[: t + 1], vc[: t + 1], np.arange(t + 1), None,
-                          None, None, kc[t], vc[t], o_gpu[t], r_gpu[t], what)
+                          None, None, kc[t], vc[t], o_gpu[t], r_gpu[t], what, fold and li > 0)
                 if li < w.gate_layer:
                     want = rows(tp["hidden"], [t])[0]
-                    assert_close(want, ref.ffn_sublayer(r_gpu[t][None], lw, om, rb)[0], BF16,
-                                 f"hidden {what}")
+                    assert_close(want, ref.ffn_sublayer(r_gpu[t][None], lw, om, rb, fold)[0],
+                                 BF16, f"hidden {what}")
                     continue
                 # the gate layer: score of the GPU's post-attention residual, then
                 # its FFN on the kept rows
-                _check_scores(r_gpu[t][None], om, scores[t:t + 1], f"score token {t}")
+                _check_scores(r_gpu[t][None], om, scores[t:t + 1], f"score token {t}", fold)
                 if t in kept_set:
                     want = rows(tp["hidden"], [row_of[t]])[0]
-                    assert_close(want, ref.ffn_sublayer(r_gpu[t][None], lw, om, rb)[0], BF16,
-                                 f"hidden layer {li} kept row {row_of[t]}")
+                    assert_close(want, ref.ffn_sublayer(r_gpu[t][None], lw, om, rb, fold)[0],
+                                 BF16, f"hidden layer {li} kept row {row_of[t]}")
             del kc, vc
             continue
         rk_list = [row_of[t] for t in sample_kept]
@@ -229,9 +235,9 @@ def test_prefill_28_layers_full_size_sampled_rows(k, dense):
             what = f"layer {li} kept row {rk}"
             _attn_row(hin[t], lw, om, t, kc, vc, kept[: rk + 1], None if dense else
                       s_kept[: rk + 1], lw.gain, lw.tau, kc[rk], vc[rk], o_gpu[t], r_gpu[t],
-                      what)
-            assert_close(want_out[t], ref.ffn_sublayer(r_gpu[t][None], lw, om, rb)[0], BF16,
-                         f"hidden {what}")
+                      what, fold)
+            assert_close(want_out[t], ref.ffn_sublayer(r_gpu[t][None], lw, om, rb, fold)[0],
+                         BF16, f"hidden {what}")
         del kc_all, vc_all
     last = rows(taps[-1]["hidden"], [row_of[t] for t in sample_kept])
     final = rb(ref.rmsnorm(last, om.final_norm, om.eps))
@@ -264,7 +270,8 @@ def test_long_context_gated_layer_128k():
     prot = synth.protect_tail(w.n, w.n_protect)
     out, kept, scores, kv, _ = _run_gpu(w, model, x, prot)
     assert np.array_equal(kept, ref.topk_select(scores, prot, w.k))
-    res = ref.prefill(host64(x), prot, w.k, om, -1, store=rb, kept_idx=kept)
+    res = ref.prefill(host64(x), prot, w.k, om, -1, store=rb, kept_idx=kept,
+                      fold_norms=model.fold_norms)
     assert_close(scores, res.scores, BF16, "scores")
     assert_close(kv[0][0], res.kv[0][0], BF16, "k")
     assert_close(kv[0][1], res.kv[0][1], BF16, "v")

@@ -573,6 +573,52 @@ def ref_protect(n, p):
     return m
 
 
+def test_folded_norm_projection():
+    """R7b: (x / rms(x)) . (W diag g)^T is RMSNorm(x; g) . W^T. In exact
+    arithmetic the two forms agree to rounding; with bf16 storage the folded
+    form rounds W g instead of the normed rows, so the two differ by at most
+    one bf16 rounding of either operand, and the folded form keeps RMSNorm's
+    scale invariance."""
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((9, 64)) * rng.uniform(0.1, 10, (9, 1))
+    g = rng.uniform(0.2, 3.0, 64)
+    w = rng.standard_normal((24, 64)) * 0.1
+    a = ref.norm_project(x, g, w, 1e-6, ref.identity, fold=True)
+    b = ref.norm_project(x, g, w, 1e-6, ref.identity, fold=False)
+    assert np.allclose(a, b, rtol=1e-12, atol=1e-13)
+    assert np.allclose(b, ref.rmsnorm(x, g, 1e-6) @ w.T, rtol=1e-12, atol=1e-13)
+    af = ref.norm_project(x, g, w, 0.0, ref.round_bf16, fold=True)
+    bf = ref.norm_project(x, g, w, 0.0, ref.round_bf16, fold=False)
+    mag = np.abs(ref.rmsnorm(x, g, 0.0)) @ np.abs(w).T
+    assert np.all(np.abs(af - a) <= 2.0 ** -8 * mag + 1e-12)
+    assert np.all(np.abs(bf - a) <= 2.0 ** -8 * mag + 1e-12)
+    assert np.allclose(ref.norm_project(7.0 * x, g, w, 0.0, ref.round_bf16, fold=True), af,
+                       rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("gate_layer", [1, -1])
+def test_prefill_with_folded_norms_is_the_same_map(gate_layer):
+    """R7b only moves rounding points: with exact storage the folded-norm
+    forward equals the plain one, for an attention stack and a hybrid one."""
+    from oracle import gated_deltanet_oracle as gdn
+    m = _tiny_model(33, True, n_layers=3)
+    rng = np.random.default_rng(8)
+    for lw in m.layers:
+        lw.gain = rng.uniform(0, 2, m.n_heads_q)
+        lw.tau = rng.uniform(0.5, 1.5, m.n_heads_q)
+    n, k = 30, 11
+    x = rng.standard_normal((n, m.d_model))
+    prot = ref_protect(n, 3)
+    a = ref.prefill(x, prot, k, m, gate_layer, store=ref.identity, fold_norms=True)
+    b = ref.prefill(x, prot, k, m, gate_layer, store=ref.identity)
+    assert np.array_equal(a.kept_idx, b.kept_idx)
+    assert np.allclose(a.out, b.out, rtol=0, atol=1e-10)
+    assert np.allclose(a.scores, b.scores, rtol=0, atol=1e-6)
+    c = gdn.hybrid_prefill(x, prot, k, m, gate_layer, store=ref.identity, fold_norms=True)
+    assert np.array_equal(c.kept_idx, b.kept_idx)
+    assert np.allclose(c.out, b.out, rtol=0, atol=1e-10)
+
+
 def test_pruned_tokens_make_no_upper_kv_and_kept_set_drives_upper_layers():
     m = _tiny_model(30, True, n_layers=4)
     rng = np.random.default_rng(6)
