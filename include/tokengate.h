@@ -390,12 +390,16 @@ typedef struct {
  *       resid [rows, d]: the residual stream after the attention sub-layer
  *         (x + Wo . attn_out; rows as attn_out);
  *       hidden [rows', d]: the layer's output after its FFN (rows' = n below
- *         the gate, k for the gate layer and above; kept rows ascending).
+ *         the gate, k for the gate layer and above; kept rows ascending);
+ *       mixer_in [rows, C + hv dv + 2 hv]: a Gated DeltaNet layer's input
+ *         projection (qkv | z | a | b, the mixer's input); unused for
+ *         attention layers.
  */
 typedef struct {
   void* attn_out;
   void* resid;
   void* hidden;
+  void* mixer_in;
 } tg_layer_taps;
 
 /* Workspace bytes of tg_prefill (and tg_prefill_multi with k = max(ks)) for

@@ -66,7 +66,7 @@ class TgKV(ctypes.Structure):
 
 
 class TgLayerTaps(ctypes.Structure):
-    _fields_ = [("attn_out", _c_p), ("resid", _c_p), ("hidden", _c_p)]
+    _fields_ = [("attn_out", _c_p), ("resid", _c_p), ("hidden", _c_p), ("mixer_in", _c_p)]
 
 
 class TgGdnLayer(ctypes.Structure):
@@ -562,6 +562,7 @@ def tg_prefill(model: Model, x, protect, k: int, gate_layer: int, out=None, kept
                 taps_c[i].attn_out = _ptr(t.get("attn_out"))
                 taps_c[i].resid = _ptr(t.get("resid"))
                 taps_c[i].hidden = _ptr(t.get("hidden"))
+                taps_c[i].mixer_in = _ptr(t.get("mixer_in"))
     _check(_prefill(ctypes.byref(model.c), _ptr(x), _ptr(protect), n, k, gate_layer, _ptr(out),
                     _ptr(kept_idx), _ptr(scores), kv_c, taps_c, _ptr(ws), ws.numel(),
                     _stream(stream, x.device)), "tg_prefill")

@@ -68,102 +68,7 @@ struct EpiParams {
   int64_t ss_ld;
   int ss_parts;
   float ss_inv_n, ss_eps;
-  // stream-K (sk_part != null): sk_dp_waves round-robin waves of whole
-  // tiles, then the k-blocks of the remaining tiles split evenly over the
-  // pairs (see Pieces)
-  int sk_dp_waves, sk_dp_tiles;
-  int64_t sk_units;
-  float4* sk_part;    // [pairs][2 ranks][64 column quads][128 rows]
-  unsigned* sk_flag;  // [pairs][2 ranks]
 };
-
-// One accumulator piece of a pair: k-blocks [k_lo, k_hi) of output tile `tile`.
-struct Piece {
-  int tile, k_lo, k_hi;
-};
-
-// The pieces of one CTA pair, in the same order for its producer, MMA and
-// epilogue warps. Without stream-K: tiles pair, pair + n_pairs, ... whole.
-// With it: first sk_dp_waves such waves, then the pair's contiguous share
-// [sk_units * pair / n_pairs, sk_units * (pair + 1) / n_pairs) of the
-// k-block units of tiles sk_dp_tiles.. (unit u: tile sk_dp_tiles + u / kb,
-// k-block u % kb). There are at least as many such tiles as pairs, so every
-// share spans at least one tile's k-blocks and a tile is split between at
-// most two consecutive pairs: pair q finishes its first k-blocks at the end
-// of its share (the tile's owner), pair q + 1 the rest at the start of its
-// own (it leaves them as a partial sum for the owner).
-struct Pieces {
-  int pair, n_pairs, num_tiles, num_kb, i;
-  int64_t u, u_end;
-  __device__ Pieces(const EpiParams& p, int pair_, int n_pairs_, int num_tiles_, int num_kb_)
-      : pair(pair_), n_pairs(n_pairs_), num_tiles(num_tiles_), num_kb(num_kb_), i(0), u(0),
-        u_end(0) {
-    if (p.sk_part != nullptr) {
-      u = p.sk_units * pair / n_pairs;
-      u_end = p.sk_units * (pair + 1) / n_pairs;
-    }
-  }
-  __device__ bool next(const EpiParams& p, Piece& pc) {
-    if (p.sk_part == nullptr || i < p.sk_dp_waves) {
-      const int tile = pair + i * n_pairs;
-      if (tile >= num_tiles) return false;
-      ++i;
-      pc = Piece{tile, 0, num_kb};
-      return true;
-    }
-    if (u >= u_end) return false;
-    const int k_lo = static_cast<int>(u % num_kb);
-    const int64_t left = u_end - u;
-    const int k_hi = left < num_kb - k_lo ? k_lo + static_cast<int>(left) : num_kb;
-    pc = Piece{p.sk_dp_tiles + static_cast<int>(u / num_kb), k_lo, k_hi};
-    u += k_hi - k_lo;
-    return true;
-  }
-};
-
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* f) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_gpu(unsigned* f, unsigned v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
-}
-// Warp-uniform bounded wait for a partial-sum flag (lane 0 polls).
-__device__ __forceinline__ bool wait_flag_warp(const unsigned* f, unsigned int* err) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) {
-    if (ld_acquire_gpu(f) == 0u) {
-      const unsigned long long t0 = global_ns();
-      for (uint32_t i = 1;; ++i) {
-        if (ld_acquire_gpu(f) != 0u) break;
-        if ((i & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
-          report_error(err, kErrWaitTimeout);
-          ok = 0;
-          break;
-        }
-      }
-    }
-  }
-  return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
-}
-
-// Accumulator columns [col, col + 32) of this thread's row, plus another
-// pair's partial sums of the same row and columns when the tile was split.
-__device__ __forceinline__ void acc_ld(uint32_t t_row, int col, const float4* part,
-                                       float (&v)[32]) {
-  tmem_ld32_wait(t_row + static_cast<uint32_t>(col), v);
-  if (part != nullptr) {
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float4 x = __ldcg(part + (col / 4 + q) * 128);
-      v[4 * q] += x.x;
-      v[4 * q + 1] += x.y;
-      v[4 * q + 2] += x.z;
-      v[4 * q + 3] += x.w;
-    }
-  }
-}
 
 __device__ __forceinline__ float round_bf16_f(float x) {
   return __bfloat162float(__float2bfloat16_rn(x));
@@ -196,11 +101,10 @@ __device__ __forceinline__ void add32_bf16(const __nv_bfloat16* src, float (&v)[
 // The fused epilogue of one accumulator tile, run by one epilogue warp for
 // its 32 rows: this thread owns accumulator row `row` (global index), whose
 // kBN fp32 columns start at TMEM address `t_row`; `nb` is the tile's column
-// block; `part` (or null): the row's partial sums from the pair that did the
-// tile's last k-blocks.
+// block.
 template <int kBN, int kEpi>
 __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, uint32_t t_row,
-                                              int nb, const float4* part) {
+                                              int nb) {
   const bool row_ok = row < p.M;
   // Folded RMSNorm of the input row: B holds W . diag(g), and the row's
   // accumulator is scaled by rs = 1 / sqrt(mean(x^2) + eps), the mean from the
@@ -216,7 +120,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
 #pragma unroll 1
     for (int c = 0; c < kBN / 32; ++c) {
       float v[32];
-      acc_ld(t_row, c * 32, part, v);
+      tmem_ld32_wait(t_row + c * 32, v);
       const int col = nb * kBN + c * 32;
       if (row_ok && col < p.N) {
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) + row * p.ldc + col;
@@ -239,8 +143,8 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       float g[32], u[32];
-      acc_ld(t_row, c * 32, part, g);
-      acc_ld(t_row, 128 + c * 32, part, u);
+      tmem_ld32_wait(t_row + c * 32, g);
+      tmem_ld32_wait(t_row + 128 + c * 32, u);
 #pragma unroll
       for (int j = 0; j < 32; ++j) g[j] = silu_f(g[j] * rs) * (u[j] * rs);
       if (row_ok)
@@ -253,6 +157,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
 #pragma unroll 1
     for (int hh = 0; hh < 2; ++hh) {
       const int hg = nb * 2 + hh;  // head index across the q | k | v columns
+      const uint32_t t_head = t_row + static_cast<uint32_t>(hh * 128);
       if (hg < p.hq + p.hkv) {
         const bool is_q = hg < p.hq;
         const float* nw = is_q ? p.q_norm : p.k_norm;
@@ -262,7 +167,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             float v[32];
-            acc_ld(t_row, hh * 128 + c * 32, part, v);
+            tmem_ld32_wait(t_head + c * 32, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const float f = round_bf16_f(v[i] * rs);
@@ -278,8 +183,8 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           float lo[32], hi[32];
-          acc_ld(t_row, hh * 128 + c * 32, part, lo);
-          acc_ld(t_row, hh * 128 + 64 + c * 32, part, hi);
+          tmem_ld32_wait(t_head + c * 32, lo);
+          tmem_ld32_wait(t_head + 64 + c * 32, hi);
           if (row_ok) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -303,7 +208,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           float v[32];
-          acc_ld(t_row, hh * 128 + c * 32, part, v);
+          tmem_ld32_wait(t_head + c * 32, v);
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] *= rs;
           if (row_ok) {
@@ -320,7 +225,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
 #pragma unroll 1
     for (int c = 0; c < kBN / 32; ++c) {
       float v[32];
-      acc_ld(t_row, c * 32, part, v);
+      tmem_ld32_wait(t_row + c * 32, v);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int f = c * 32 + j;
@@ -397,14 +302,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    Pieces pieces(p, pair, n_pairs, num_tiles, num_kb);
-    Piece pc;
-    while (ok && pieces.next(p, pc)) {
-      const int mb = pc.tile / p.tiles_n, nb = pc.tile % p.tiles_n;
+    for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
+      const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
       const int a_row = mb * 256 + static_cast<int>(rank) * 128;
       const int b_row = kEpi == EPI_SWIGLU ? (rank ? p.inter : 0) + nb * 128
                                            : nb * 256 + static_cast<int>(rank) * 128;
-      for (int kb = pc.k_lo; kb < pc.k_hi; ++kb) {
+      for (int kb = 0; kb < num_kb; ++kb) {
         if (!mbar_wait(&empty[s], ph ^ 1u, p.err)) { ok = false; break; }
         uint8_t* a_dst = tiles + size_t(s) * C::kStageBytes;
         uint8_t* b_dst = a_dst + C::kHalfBytes;
@@ -428,15 +331,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t ph = 0;
     bool ok = true;
     int it = 0;
-    Pieces pieces(p, pair, n_pairs, num_tiles, num_kb);
-    Piece pc;
-    for (; ok && pieces.next(p, pc); ++it) {
+    for (int tile = pair; tile < num_tiles && ok; tile += n_pairs, ++it) {
       const int a = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       if (!mbar_wait(&acc_empty[a], (use & 1u) ^ 1u, p.err)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * kBN);
-      for (int kb = pc.k_lo; kb < pc.k_hi; ++kb) {
+      for (int kb = 0; kb < num_kb; ++kb) {
         if (!mbar_wait(&full[s], ph, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_addr = smem_addr(tiles + size_t(s) * C::kStageBytes);
@@ -444,8 +345,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
           umma_f16_ss_pair(d_tmem, sdesc_kmajor_sw128(a_addr + k * 32),
-                           sdesc_kmajor_sw128(b_addr + k * 32), idesc,
-                           (kb > pc.k_lo || k != 0) ? 1u : 0u);
+                           sdesc_kmajor_sw128(b_addr + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
         }
         const uint32_t e = smem_addr(&empty[s]);
         umma_commit_pair(e);
@@ -468,46 +368,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp >= 4) {
     // ---------------------------------------------------------- epilogue
     const int quarter = warp & 3;
-    const int rl = quarter * 32 + lane;  // row within this CTA's 128 accumulator rows
     int it = 0;
-    Pieces pieces(p, pair, n_pairs, num_tiles, num_kb);
-    Piece pc;
-    for (; pieces.next(p, pc); ++it) {
-      const int mb = pc.tile / p.tiles_n, nb = pc.tile % p.tiles_n;
+    for (int tile = pair; tile < num_tiles; tile += n_pairs, ++it) {
+      const int mb = tile / p.tiles_n, nb = tile % p.tiles_n;
       const int a = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       if (!mbar_wait_warp(&acc_full[a], use & 1u, p.err)) break;
       tc_fence_after();
-      const int64_t row = static_cast<int64_t>(mb) * 256 + static_cast<int64_t>(rank) * 128 + rl;
+      const int64_t row =
+          static_cast<int64_t>(mb) * 256 + static_cast<int64_t>(rank) * 128 + quarter * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(a * kBN);
-      if (pc.k_lo > 0) {
-        // the tile's last k-blocks: a partial sum for the pair that owns it
-        float4* dst = p.sk_part + static_cast<size_t>(pair * 2 + rank) * (64 * 128) + rl;
-#pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
-          float v[32];
-          tmem_ld32_wait(t_row + c * 32, v);
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[(c * 8 + q) * 128] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-        }
-        __threadfence();
-        named_bar_sync(1, 128);  // the four epilogue warps' rows are written
-        if (threadIdx.x == 128) st_release_gpu(p.sk_flag + pair * 2 + rank, 1u);
-      } else if (pc.k_hi < num_kb) {
-        // the tile's first k-blocks: add pair + 1's partial sums
-        const unsigned* f = p.sk_flag + (pair + 1) * 2 + rank;
-        const bool ready = wait_flag_warp(f, p.err);
-        __threadfence();  // every lane's partial-sum loads follow the flag
-        if (ready)
-          epilogue_tile<kBN, kEpi>(
-              p, row, t_row, nb, p.sk_part + static_cast<size_t>((pair + 1) * 2 + rank) * (64 * 128) + rl);
-        named_bar_sync(1, 128);  // every warp has seen the flag
-        if (threadIdx.x == 128) p.sk_flag[(pair + 1) * 2 + rank] = 0u;  // for the next launch
-      } else {
-        epilogue_tile<kBN, kEpi>(p, row, t_row, nb, nullptr);
-      }
+      epilogue_tile<kBN, kEpi>(p, row, t_row, nb);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&acc_empty[a]), 0));
@@ -556,10 +428,6 @@ cudaError_t run(const GemmArgs& g, cudaStream_t st) {
   p.ss_parts = g.ss_parts;
   p.ss_inv_n = g.ss_inv_n;
   p.ss_eps = g.ss_eps;
-  p.sk_dp_waves = p.sk_dp_tiles = 0;
-  p.sk_units = 0;
-  p.sk_part = nullptr;
-  p.sk_flag = nullptr;
   p.tiles_m = static_cast<int>((g.M + 255) / 256);
   p.tiles_n = kEpi == EPI_SWIGLU ? g.inter / 128 : (g.N + 255) / 256;
   p.err = device_error_word();
@@ -588,17 +456,6 @@ cudaError_t run(const GemmArgs& g, cudaStream_t st) {
     if (dev >= 0 && dev < kMaxDevices) resident[dev].store(max_pairs);
   }
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
-  // Stream-K when the tiles are more than one wave but not a whole number of
-  // waves: the last one to two waves' k-blocks are shared evenly by all pairs.
-  const int num_kb = (p.K + kBK - 1) / kBK;
-  if (g.sk_ws != nullptr && g.sk_ws_bytes >= gemm_sk_bytes() && pairs <= kSkMaxPairs &&
-      tiles > pairs && tiles % pairs != 0 && num_kb >= 4) {
-    p.sk_dp_waves = tiles / pairs - 1;
-    p.sk_dp_tiles = p.sk_dp_waves * pairs;
-    p.sk_units = static_cast<int64_t>(tiles - p.sk_dp_tiles) * num_kb;
-    p.sk_part = static_cast<float4*>(g.sk_ws);
-    p.sk_flag = reinterpret_cast<unsigned*>(static_cast<char*>(g.sk_ws) + gemm_sk_flag_offset());
-  }
   return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), C::kSmem, st, ta, tb, p);
 }
 

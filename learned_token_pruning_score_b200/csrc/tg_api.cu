@@ -259,17 +259,15 @@ struct PrefillPlan {
   void* gu = nullptr;
   float* scores = nullptr; // [n]
   float* hpre = nullptr;   // fp32 scorer pre-activation [n, F]
-  // Folded RMSNorm (bf16): the row sums of squares the last residual GEMM
-  // left, [ss_parts][ss_ld] (one per 256-column block), and which residual
-  // stream (rows [0, ss_rows) of buffer ss_for) they describe. Anything
-  // other than a residual GEMM that writes a stream resets ss_for.
-  void* gemm_sk = nullptr;  // stream-K scratch of the tensor-core GEMMs
+  // Folded RMSNorm (bf16): per residual stream (h, hk) the row sums of
+  // squares its last residual GEMM left, [ss_parts][ld] (one per
+  // 256-column block), and how many leading rows they describe (-1: none).
+  // Anything other than a residual GEMM that writes a stream resets it.
   float* ss = nullptr;    // rows of h: [ss_parts][n]
   float* ss_k = nullptr;  // rows of hk: [ss_parts][k]
   int64_t ss_ld = 0, ss_ld_k = 0;
   int ss_parts = 0;
-  mutable const void* ss_for = nullptr;
-  mutable int64_t ss_rows = 0;
+  mutable int64_t ss_rows_h = -1, ss_rows_hk = -1;
   int32_t* pos_k = nullptr;
   float* s_k = nullptr;
   float* lsig_k = nullptr;
@@ -310,7 +308,6 @@ struct PrefillPlan {
       ss_ld_k = k;
       ss = static_cast<float*>(a.carve(size_t(ss_parts) * n * 4));
       ss_k = static_cast<float*>(a.carve(size_t(ss_parts) * k * 4));
-      gemm_sk = a.carve(gemm_sk_bytes());
     }
     if (m.dtype == TG_F32) hpre = static_cast<float*>(a.carve(size_t(n) * m.d_score * 4));
     pos_k = static_cast<int32_t*>(a.carve(size_t(k) * 4));
@@ -403,25 +400,12 @@ GemmArgs gemm_args(const void* A, int64_t lda, const void* B, int64_t ldb, void*
   return g;
 }
 
-// Stream-K scratch of the plan for a tensor-core GEMM (its flags are zeroed
-// once per call by sk_clear, and every launch leaves them zero).
-GemmArgs& with_sk(GemmArgs& g, const PrefillPlan& P) {
-  if (P.gemm_sk != nullptr) {
-    g.sk_ws = P.gemm_sk;
-    g.sk_ws_bytes = gemm_sk_bytes();
-  }
-  return g;
-}
-cudaError_t sk_clear(const PrefillPlan& P, cudaStream_t st) {
-  if (P.gemm_sk == nullptr) return cudaSuccess;
-  return cudaMemsetAsync(static_cast<char*>(P.gemm_sk) + gemm_sk_flag_offset(), 0,
-                         gemm_sk_bytes() - gemm_sk_flag_offset(), st);
-}
-
 // Folded RMSNorm: rows [0, rows) of the stream h carry the row sums of
 // squares their last residual GEMM left in P.ss.
 bool ss_ready(const PrefillPlan& P, const void* h, int64_t rows) {
-  return P.ss != nullptr && P.ss_for == h && P.ss_rows == rows;
+  if (P.ss == nullptr) return false;
+  if (h == P.h) return P.ss_rows_h == rows;
+  return h == P.hk && P.ss_rows_hk == rows;
 }
 // The row sums of the stream h (the all-token buffer or the kept-row one).
 float* ss_of(const PrefillPlan& P, const void* h) { return h == P.hk ? P.ss_k : P.ss; }
@@ -442,8 +426,8 @@ void ss_produce(GemmArgs& g, const PrefillPlan& P, const void* h, int64_t row0) 
 }
 void ss_mark(const PrefillPlan& P, const void* h, int64_t rows) {
   if (P.ss == nullptr) return;
-  P.ss_for = h;
-  P.ss_rows = rows;
+  if (h == P.h) P.ss_rows_h = rows;
+  if (h == P.hk) P.ss_rows_hk = rows;
 }
 
 // Scorer over `rows` rows of x (dtype dt) into scores[rows]. With a plan
@@ -462,7 +446,6 @@ cudaError_t run_score(const void* x, int64_t rows, int d, int f, const float* no
     GemmArgs g = gemm_args(fold ? x : y, d, fold ? w1_g : w1, d, nullptr, 0, rows, f, d, EPI_SCORE);
     g.b1 = b1; g.w2 = w2; g.b2 = b2; g.scores = scores;
     if (fold) ss_consume(g, *P, x, eps, d, 0);
-    if (P != nullptr) with_sk(g, *P);
     return gemm(g, dt, st);
   }
   GemmArgs g = gemm_args(y, d, w1, d, hpre, f, rows, f, d, EPI_STORE);
@@ -606,7 +589,6 @@ cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims
   void* k_dst = (kv && kv->k) ? kv->k : P.attn.k_rot;
   GemmArgs gq = gemm_args(xin, D.d, wqkv, D.d, nullptr, 0, rows, D.qkv, D.d, EPI_QKV);
   if (fold) ss_consume(gq, P, h, m.norm_eps, D.d, 0);
-  with_sk(gq, P);
   gq.hq = D.hq; gq.hkv = D.hkv; gq.rope_cs = cs; gq.q_norm = lw.q_norm; gq.k_norm = lw.k_norm;
   gq.eps = m.norm_eps; gq.q_out = P.attn.q_rot; gq.k_out = k_dst; gq.vT_out = P.attn.vT;
   gq.t_pad = P.attn.t_pad; gq.v_out = kv ? kv->v : nullptr;
@@ -644,7 +626,6 @@ cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims
   g.R = h;
   g.ldr = D.d;
   ss_produce(g, P, h, 0);
-  with_sk(g, P);
   err = gemm(g, dt, st);
   if (err != cudaSuccess) return err;
   ss_mark(P, h, rows);
@@ -674,7 +655,6 @@ cudaError_t ffn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
                              2 * D.inter, D.d, EPI_SWIGLU);
       g.inter = D.inter;
       if (fold) ss_consume(g, P, h, m.norm_eps, D.d, r0);
-      with_sk(g, P);
       err = gemm(g, dt, st);
     } else {
       err = gemm(gemm_args(yb, D.d, lw.w_gate_up, D.d, P.gu, 2 * D.inter, rb, 2 * D.inter, D.d,
@@ -691,7 +671,6 @@ cudaError_t ffn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
     g.R = hb;
     g.ldr = D.d;
     ss_produce(g, P, h, r0);
-    with_sk(g, P);
     err = gemm(g, dt, st);
     if (err != cudaSuccess) return err;
   }
@@ -735,6 +714,10 @@ cudaError_t gdn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
   err = gemm(gemm_args(P.y, D.d, lw.w_in, D.d, P.gdn_proj, Nt, rows, static_cast<int>(Nt), D.d,
                        EPI_STORE), dt, st);
   if (err != cudaSuccess) return err;
+  if (taps && taps->mixer_in) {
+    err = copy_rows(taps->mixer_in, P.gdn_proj, size_t(rows) * Nt * e, rows, st);
+    if (err != cudaSuccess) return err;
+  }
   const int n_seq = segs ? segs->count : 1;
   for (int b = 0; b < n_seq; ++b) {
     const int64_t off = segs ? segs->off[b] : 0, len = segs ? segs->len[b] : rows;
@@ -773,7 +756,6 @@ cudaError_t gdn_sublayer(const tg_model& m, const tg_layer& lw, const Dims& D,
   g.R = h;
   g.ldr = D.d;
   ss_produce(g, P, h, 0);
-  with_sk(g, P);
   err = gemm(g, dt, st);
   if (err != cudaSuccess) return err;
   ss_mark(P, h, rows);
@@ -1236,10 +1218,9 @@ tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan
                              const tg_layer_taps* taps, float* sc, cudaStream_t st) {
   const size_t e = elem_size(m.dtype);
   TG_TRY(copy_rows(P.h, x, size_t(n) * D.d * e, n, st));
-  P.ss_for = nullptr;  // the input rows carry no row sums
+  P.ss_rows_h = -1;  // the input rows carry no row sums
   // every attention launch of the call then finds its split counters zero
   TG_TRY(attn_split_clear(P.attn.split, P.attn.split_bytes, D.hq, st));
-  TG_TRY(sk_clear(P, st));
   const bool tables = m.dtype == TG_BF16 && D.dh == 128;
   const double cs_bytes = 8.0 * (D.dh / 2);
   if (tables && gate_layer >= 0)
@@ -1284,8 +1265,7 @@ tg_status prefill_above_gate(const tg_model& m, const Dims& D, const PrefillPlan
   if (carry) sg = SsGather{P.ss, P.ss_ld, P.ss_k, P.ss_ld_k, P.ss_parts};
   TG_TRY(compact(P.h, nullptr, sc, kept_idx, n, k, static_cast<int>(D.d * e), P.hk, P.pos_k, P.s_k,
                  P.lsig_k, st, sg));
-  if (carry) ss_mark(P, P.hk, k);
-  else if (P.ss_for == P.hk) P.ss_for = nullptr;
+  P.ss_rows_hk = carry ? k : -1;
   if (tables) {
     TG_TRY(traced(TG_K_ROPE_TABLE, k, 0.0, cs_bytes * k + 4.0 * k, st, [&] {
       return launch_rope_table(P.pos_k, k, D.dh, m.rope_base, P.cs_k, st);
@@ -1465,7 +1445,6 @@ tg_status tg_prefill_batch(const tg_model* model, const void* x, const uint8_t* 
   char* h = static_cast<char*>(P.h);
   char* hk = static_cast<char*>(P.hk);
   TG_TRY(attn_split_clear(P.attn.split, P.attn.split_bytes, D.hq, st));
-  TG_TRY(sk_clear(P, st));
   // packed rows in, padding rows zero
   for (int b = 0; b < batch; ++b) {
     const int64_t n = sn.len[b], pad = static_cast<int64_t>(align_up(size_t(n), kSegAlign)) - n;
@@ -1515,8 +1494,7 @@ tg_status tg_prefill_batch(const tg_model* model, const void* x, const uint8_t* 
     if (pad > 0) TG_TRY(cudaMemsetAsync(hk + (sk.off[b] + k) * row, 0, pad * row, st));
     ck += k;
   }
-  if (carry) ss_mark(P, P.hk, k_pad);
-  else if (P.ss_for == P.hk) P.ss_for = nullptr;
+  P.ss_rows_hk = carry ? k_pad : -1;
   TG_TRY(traced(TG_K_ROPE_TABLE, k_pad, 0.0, cs_bytes * k_pad + 4.0 * k_pad, st, [&] {
     return launch_rope_table(P.pos_k, k_pad, D.dh, m.rope_base, P.cs_k, st);
   }));

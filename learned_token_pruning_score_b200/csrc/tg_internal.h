@@ -166,15 +166,7 @@ struct GemmArgs {
   int64_t ss_ld = 0;
   int ss_parts = 0;
   float ss_inv_n = 0.f, ss_eps = 0.f;
-  // Optional stream-K scratch (tensor-core path): partial sums and flags,
-  // gemm_sk_bytes(); the flags must be zero before the first launch that
-  // uses it (launches leave them zero).
-  void* sk_ws = nullptr;
-  size_t sk_ws_bytes = 0;
 };
-constexpr int kSkMaxPairs = 96;
-constexpr size_t gemm_sk_flag_offset() { return size_t(kSkMaxPairs) * 2 * 64 * 128 * 16; }
-constexpr size_t gemm_sk_bytes() { return gemm_sk_flag_offset() + size_t(kSkMaxPairs) * 2 * 4; }
 // tile column blocks of a residual GEMM's row sums of squares
 constexpr int kSsBlockCols = 256;
 inline int ss_parts_of(int n) { return (n + kSsBlockCols - 1) / kSsBlockCols; }

@@ -10,12 +10,13 @@ Cloud article on TokenGate, section "门控位置影响剪枝效果", figure 5).
 tg_prefill is compared with the oracle's hybrid_prefill layer by layer,
 teacher-forced at every tensor the library stores between kernels (the
 layer taps): each layer starts from the GPU's own input; a Gated DeltaNet
-layer's mixer output, then its residual (from the GPU's mixer output), an
-attention layer's k/v, output and residual likewise, then the FFN output from
-the GPU's residual. Every element is held to 2e-2 + 1e-2 |ref| (bf16). The
-mixer's carried conv rows and final state (the layer's KV outputs) are
-compared at the same bound: the oracle derives them from its own bf16
-projection of the layer input, one rounding away from the GPU's.
+layer's input projection, its mixer output (from the GPU's stored
+projection: the recurrence can amplify a one-ulp difference of its input
+where a head's output is small before the gated norm), then its residual
+(from the GPU's mixer output), an attention layer's k/v, output and residual
+likewise, then the FFN output from the GPU's residual. Every element is held
+to 2e-2 + 1e-2 |ref| (bf16). The mixer's carried conv rows and final state
+(the layer's KV outputs) are compared at the same bound.
 """
 
 from collections.abc import Sequence
@@ -109,9 +110,13 @@ def _run(w, model, x, prot, gate):
                        torch.empty(rows, b.hkv, b.dh, device="cuda", dtype=BF16)))
             width = b.hq * b.dh
         hrows = b.n if li < gate else b.k
-        taps.append({"attn_out": torch.empty(rows, width, device="cuda", dtype=BF16),
-                     "resid": torch.empty(rows, b.d, device="cuda", dtype=BF16),
-                     "hidden": torch.empty(hrows, b.d, device="cuda", dtype=BF16)})
+        t = {"attn_out": torch.empty(rows, width, device="cuda", dtype=BF16),
+             "resid": torch.empty(rows, b.d, device="cuda", dtype=BF16),
+             "hidden": torch.empty(hrows, b.d, device="cuda", dtype=BF16)}
+        if kind == "gdn":
+            t["mixer_in"] = torch.empty(rows, C + w.hv * w.dv + 2 * w.hv, device="cuda",
+                                        dtype=BF16)
+        taps.append(t)
     scores = torch.empty(b.n, device="cuda")
     out, kept, _ = tg.tg_prefill(model, x, torch.from_numpy(prot).cuda(), b.k, gate,
                                  scores=scores, kv=kv, taps=taps)
@@ -147,7 +152,9 @@ def _check_stack(w, gate):
         if kind == "gdn":
             C = 2 * w.hk * w.dk + w.hv * w.dv
             y = rb(ref.rmsnorm(h_in, lw.norm, b.eps))
-            proj = rb(y @ lw.w_in.T)
+            proj_gpu = host64(taps[li]["mixer_in"])
+            assert_close(proj_gpu, rb(y @ lw.w_in.T), BF16, f"input projection {what}")
+            proj = proj_gpu  # the mixer from the GPU's stored projection
             res = gdn.gated_deltanet(proj[:, :C], proj[:, C:C + w.hv * w.dv],
                                      proj[:, C + w.hv * w.dv:C + w.hv * w.dv + w.hv],
                                      proj[:, C + w.hv * w.dv + w.hv:], lw.mixer, w.hk, w.hv,
