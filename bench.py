@@ -507,14 +507,14 @@ def run_ours(args, rank, world, local_rank):
         prot_host = prot.cpu().pin_memory()
         out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         kept_host = torch.empty(kept.shape, dtype=kept.dtype).pin_memory()
-        x_dev = torch.empty_like(x)
         prot_dev = torch.empty_like(prot)
 
+        # the input stays in pinned host memory: tg_prefill_host copies it in
+        # chunks that overlap layer 0's projection and attention
         def e2e_step():
-            x_dev.copy_(x_host, non_blocking=True)
             prot_dev.copy_(prot_host, non_blocking=True)
-            tg.tg_prefill(model, x_dev, prot_dev, k, w.gate_layer, out=out, kept_idx=kept,
-                          scores=scores, kv=kv, ws=ws, stream=stream)
+            tg.tg_prefill_host(model, x_host, prot_dev, k, w.gate_layer, out=out, kept_idx=kept,
+                               scores=scores, kv=kv, ws=ws, stream=stream)
             out_host.copy_(out, non_blocking=True)
             kept_host.copy_(kept, non_blocking=True)
 

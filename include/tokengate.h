@@ -402,6 +402,26 @@ typedef struct {
   void* mixer_in;
 } tg_layer_taps;
 
+/*
+ * tg_prefill_host -- tg_prefill with the input hidden states in HOST memory
+ * (page-locked for the copies to be asynchronous): what a serving stack
+ * calls when the prompt's hidden states come from the host. Same arguments,
+ * results and workspace as tg_prefill (no taps), except that x is a host
+ * pointer [n, d] dtype; protect, out, kept_idx, scores and kv stay device
+ * pointers. The call copies x into its workspace; when the model runs bf16
+ * paired-head attention at layer 0, the gate is at or above layer 0 and n >
+ * 8192, the copy goes in 4096-row chunks on a library-owned stream, and the
+ * RMSNorm, the fused QKV projection and the causal attention of each chunk's
+ * rows run on `stream` as soon as the chunk has landed, so that the copy
+ * overlaps layer 0 (the results are the same as tg_prefill's bit for bit).
+ * Returns when the work is queued on `stream`; x must stay valid until the
+ * stream reaches the end of the call's work.
+ */
+tg_status tg_prefill_host(const tg_model* model, const void* x_host, const uint8_t* protect,
+                          int64_t n, int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx,
+                          float* scores, const tg_kv* kv, void* ws, size_t ws_bytes,
+                          tg_stream stream);
+
 /* Workspace bytes of tg_prefill (and tg_prefill_multi with k = max(ks)) for
  * this model: tg_workspace_size(TG_OP_PREFILL) plus the buffers of a hybrid
  * stack's Gated DeltaNet layers (0 on invalid sizes). */

@@ -108,6 +108,8 @@ _prefill = _sig("tg_prefill", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64, 
                 _c_p, _c_p, _c_p, ctypes.POINTER(TgKV), ctypes.POINTER(TgLayerTaps), _c_p,
                 _c_sz, _c_p)
 _prefill_ws = _sig("tg_prefill_workspace_size", _c_sz, ctypes.POINTER(TgModel), _c_i64, _c_i64)
+_prefill_host = _sig("tg_prefill_host", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64, _c_i64,
+                     _c_i32, _c_p, _c_p, _c_p, ctypes.POINTER(TgKV), _c_p, _c_sz, _c_p)
 _prefill_multi = _sig("tg_prefill_multi", _ci, ctypes.POINTER(TgModel), _c_p, _c_p, _c_i64,
                       ctypes.POINTER(_c_i64), _c_i32, _c_i32, ctypes.POINTER(_c_p),
                       ctypes.POINTER(_c_p), _c_p, _c_p, _c_sz, _c_p)
@@ -531,6 +533,34 @@ def tg_decode_step(model: Model, x, pos: int, gate_layer: int, kv: Sequence, len
     return out
 
 
+def tg_prefill_host(model: Model, x_host, protect, k: int, gate_layer: int, device=None,
+                    out=None, kept_idx=None, scores=None, kv: Optional[Sequence] = None, ws=None,
+                    stream=None):
+    """tg_prefill with x_host [n, d] a CPU tensor (pinned for the copy to
+    overlap layer 0); protect, out, kept_idx, scores and kv on the device.
+    Returns (out [k, d], kept_idx [k], scores [n] or None)."""
+    if x_host.is_cuda:
+        raise ValueError("x_host must be a host (CPU) tensor; use tg_prefill for device input")
+    n, d = x_host.shape
+    dev = torch.device(device) if device is not None else (
+        protect.device if protect is not None else torch.device("cuda", torch.cuda.current_device()))
+    if out is None:
+        out = torch.empty(k, d, dtype=x_host.dtype, device=dev)
+    if kept_idx is None:
+        kept_idx = torch.empty(k, dtype=torch.int32, device=dev)
+    ws = _ws(model.workspace_size(n, k, gate_layer), dev, ws)
+    kv_c = None
+    if kv is not None:
+        kv_c = (TgKV * len(model.layers))()
+        for i, pair in enumerate(kv):
+            if pair is not None:
+                kv_c[i].k, kv_c[i].v = _ptr(pair[0]), _ptr(pair[1])
+    _check(_prefill_host(ctypes.byref(model.c), _ptr(x_host), _ptr(protect), n, k,
+                         gate_layer, _ptr(out), _ptr(kept_idx), _ptr(scores), kv_c, _ptr(ws),
+                         ws.numel(), _stream(stream, dev)), "tg_prefill_host")
+    return out, kept_idx, scores
+
+
 def tg_prefill(model: Model, x, protect, k: int, gate_layer: int, out=None, kept_idx=None,
                scores=None, kv: Optional[Sequence] = None, taps: Optional[Sequence] = None,
                ws=None, stream=None):
@@ -621,7 +651,7 @@ def tg_prefill_batch(model: Model, x, protect, lens: Sequence[int], ks: Sequence
 
 
 __all__ = [
-    "tg_score", "tg_linear", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_gated_attn_forward", "tg_gated_attn_backward", "tg_prefill", "tg_prefill_multi", "tg_prefill_batch", "tg_decode_step",
+    "tg_score", "tg_linear", "tg_fold_norm_weight", "tg_prefill_host", "tg_topk_select", "tg_topk_select_noalloc", "SELECT_NOALLOC_MAX_N", "tg_compact", "tg_gated_attn_prefill", "tg_gated_attn_forward", "tg_gated_attn_backward", "tg_prefill", "tg_prefill_multi", "tg_prefill_batch", "tg_decode_step",
     "tg_workspace_size", "tg_status_string", "tg_device_error", "tg_version", "Model",
     "tg_selftest_wait_timeout",
     "TokenGateError", "LIB_PATH", "tg_trace_start", "tg_trace_stop", "TG_OK", "TG_ERR_INVALID_ARG", "TG_ERR_UNSUPPORTED",

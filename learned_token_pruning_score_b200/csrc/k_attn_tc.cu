@@ -370,6 +370,7 @@ struct Params {
   int64_t T;
   int hq, hkv;
   int n_qtiles;
+  int qt_lo;     // first query tile of the launch (tiles qt_lo .. n_qtiles - 1)
   int kv_major;  // 1: CTAs ordered KV-head-major (large T), 0: heaviest tiles first
   const float* gain;
   const float* tau;
@@ -440,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     qt = static_cast<int>(x & 1023u);
     kv_lo = static_cast<int>((x >> 10) & 1023u);
   } else if (p.kv_major) {
-    const int per_kv = p.n_qtiles * pairs_per_kv;
+    const int per_kv = (p.n_qtiles - p.qt_lo) * pairs_per_kv;
     const int g0 = static_cast<int>(blockIdx.x) / per_kv;
     const int rem = static_cast<int>(blockIdx.x) % per_kv;
     qt = p.n_qtiles - 1 - rem / pairs_per_kv;
@@ -1008,7 +1009,9 @@ size_t attn_split_bytes(int64_t T, int hq, int hkv) {
 bool attn_tc_supported(const AttnArgs& a) {
   auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
   return a.dh == kDh && a.hq % a.hkv == 0 && a.t_pad % 64 == 0 && a.t_pad >= a.T && al16(a.q) &&
-         al16(a.k) && al16(a.v) && al16(a.out) && a.T < (int64_t(1) << 31) - kBlk;
+         al16(a.k) && al16(a.v) && al16(a.out) && a.T < (int64_t(1) << 31) - kBlk &&
+         a.q_lo >= 0 && a.q_lo % kBlk == 0 && a.q_lo < a.T &&
+         (a.q_lo == 0 || (a.hq / a.hkv) % 2 == 0);
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
@@ -1042,6 +1045,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
     pp.hq = p.hq;
     pp.hkv = p.hkv;
     pp.n_qtiles = p.n_qtiles;
+    pp.qt_lo = static_cast<int>(a.q_lo / kBlk);
     // K and V of all KV heads: above ~48 MB the working set would not stay
     // in the 126 MB L2 across a wave of CTAs spread over every head.
     pp.kv_major = (double(a.T) * a.hkv * kDh * 4.0 > 48.0e6) ? 1 : 0;
@@ -1065,8 +1069,9 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t st) {
     pp.n_items = 0;
     pp.part_o = pp.part_ml = nullptr;
     pp.cnt = nullptr;
-    unsigned grid = static_cast<unsigned>(p.n_qtiles) * static_cast<unsigned>(a.hq / 2);
-    if (a.split_ws != nullptr && a.split_ws_bytes >= attn_split_bytes(a.T, a.hq, a.hkv)) {
+    unsigned grid = static_cast<unsigned>(p.n_qtiles - pp.qt_lo) * static_cast<unsigned>(a.hq / 2);
+    if (pp.qt_lo == 0 && a.split_ws != nullptr &&
+        a.split_ws_bytes >= attn_split_bytes(a.T, a.hq, a.hkv)) {
       const pair::Schedule* schp = pair::cached_schedule(p.n_qtiles, a.hq / 2);
       if (schp != nullptr) {
         const pair::Schedule& sch = *schp;

@@ -62,6 +62,7 @@ struct EpiParams {
   __nv_bfloat16* vT_out;
   int64_t t_pad;
   __nv_bfloat16* v_out;
+  int64_t rope_ld;
   // folded RMSNorm: row sums of squares out (RESIDUAL) / in (the others)
   float* ss_out;
   const float* ss_in;
@@ -179,7 +180,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
         __nv_bfloat16* dst =
             is_q ? p.q_out + (row * p.hq + hg) * 128
                  : p.k_out + (row * p.hkv + (hg - p.hq)) * 128;
-        const float2* cs = p.rope_cs + row;  // frequency-major: entry i at cs[i * M]
+        const float2* cs = p.rope_cs + row;  // frequency-major: entry i at cs[i * rope_ld]
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           float lo[32], hi[32];
@@ -195,7 +196,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
                 a *= __ldg(nw + pi);
                 b *= __ldg(nw + pi + 64);
               }
-              const float2 t = __ldg(cs + static_cast<int64_t>(pi) * p.M);
+              const float2 t = __ldg(cs + static_cast<int64_t>(pi) * p.rope_ld);
               lo[i] = a * t.x - b * t.y;
               hi[i] = b * t.x + a * t.y;
             }
@@ -422,6 +423,7 @@ cudaError_t run(const GemmArgs& g, cudaStream_t st) {
   p.vT_out = static_cast<__nv_bfloat16*>(g.vT_out);
   p.t_pad = g.t_pad;
   p.v_out = static_cast<__nv_bfloat16*>(g.v_out);
+  p.rope_ld = g.rope_ld > 0 ? g.rope_ld : g.M;
   p.ss_out = g.ss_out;
   p.ss_in = g.ss_in;
   p.ss_ld = g.ss_ld;

@@ -15,6 +15,7 @@
 #include <cuda_bf16.h>
 
 #include <cmath>
+#include <map>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -461,10 +462,12 @@ cudaError_t attn_core(const AttnPlan& plan, const void* k_rot, const void* v, in
                       const float* lsig, const void* kaug, const float* gain, const float* tau,
                       int64_t rows, int hq, int hkv, int dh, tg_dtype dt, void* out,
                       cudaStream_t st, float* lse = nullptr, float* out_f32 = nullptr,
-                      bool split_cnt_zeroed = false) {
+                      bool split_cnt_zeroed = false, int64_t q_lo = 0, bool whole_tiles = false) {
   const size_t es = elem_size(dt);
-  const double attn_flops = 4.0 * dh * hq * double(rows) * double(rows + 1) / 2.0;
-  const double attn_bytes = double(rows) * (2 * hq + 2 * hkv) * dh * es;
+  // causal work of query rows [q_lo, rows) over keys [0, rows)
+  const double attn_flops = 4.0 * dh * hq *
+                            (double(rows) * double(rows + 1) - double(q_lo) * double(q_lo + 1)) / 2.0;
+  const double attn_bytes = double(rows - q_lo) * 2 * hq * dh * es + double(rows) * 2 * hkv * dh * es;
   AttnArgs a{};
   a.q = plan.q_rot;
   a.k = k_rot;
@@ -475,9 +478,12 @@ cudaError_t attn_core(const AttnPlan& plan, const void* k_rot, const void* v, in
   a.out = out;
   a.lse = lse;
   a.out_f32 = out_f32;
-  a.split_ws = plan.split;
-  a.split_ws_bytes = plan.split_bytes;
+  // whole_tiles: one CTA per query tile (no split tiles), as in a launch over
+  // more rows than the split schedule covers
+  a.split_ws = whole_tiles ? nullptr : plan.split;
+  a.split_ws_bytes = whole_tiles ? 0 : plan.split_bytes;
   a.split_cnt_zeroed = split_cnt_zeroed;
+  a.q_lo = q_lo;
   if (dt == TG_BF16) {
     a.v = plan.vT;
     a.t_pad = plan.t_pad;
@@ -1211,13 +1217,108 @@ Dims model_dims(const tg_model& m) {
               (m.n_heads_q + 2 * m.n_heads_kv) * m.head_dim};
 }
 
+// Rows per chunk of a prefill whose input arrives from host memory (small
+// chunks expose less of the first copy; every later copy hides behind the
+// growing attention work of the chunk before it).
+constexpr int64_t kHostChunkRows = 4096;
+
+// Whether tg_prefill_host can overlap the input copy with layer 0: the
+// paired-head tensor-core attention, layer 0 an attention layer at or below
+// the gate, and n above the 8192 rows up to which the one-shot attention may
+// split query tiles (the chunks run whole tiles, so the results stay equal).
+bool host_chunks_apply(const tg_model& m, const Dims& D, int64_t n, int gate_layer) {
+  return m.dtype == TG_BF16 && D.dh == 128 && (D.hq / D.hkv) % 2 == 0 && gate_layer >= 0 &&
+         m.layers[0].gdn == nullptr && n > 8192;
+}
+
+// Layer 0's attention sub-layer while its input rows arrive from host
+// memory: the rows are copied into P.h in chunks on `copy_st`; as each chunk
+// lands, its RMSNorm, its fused QKV projection and the attention of its
+// query rows (over every key up to the chunk's end) run on `st`, so that the
+// copies of the later chunks overlap the work of the earlier ones. Then the
+// output projection over all n rows. Each query tile and each GEMM tile is
+// computed exactly as by the one-shot launches (chunk bounds are multiples of
+// the 256-row GEMM tile).
+tg_status attn_layer0_from_host(const tg_model& m, const Dims& D, const PrefillPlan& P,
+                                const void* x_host, int64_t n, const tg_kv* kv,
+                                cudaStream_t st, cudaStream_t copy_st) {
+  const tg_layer& lw = m.layers[0];
+  const size_t e = elem_size(m.dtype), row = size_t(D.d) * e;
+  const int64_t n_chunks = (n + kHostChunkRows - 1) / kHostChunkRows;
+  std::vector<cudaEvent_t> landed(static_cast<size_t>(n_chunks), nullptr);
+  cudaEvent_t start = nullptr;
+  auto release = [&] {
+    for (cudaEvent_t ev : landed)
+      if (ev) cudaEventDestroy(ev);
+    if (start) cudaEventDestroy(start);
+  };
+  cudaError_t err = cudaEventCreateWithFlags(&start, cudaEventDisableTiming);
+  for (int64_t c = 0; c < n_chunks && err == cudaSuccess; ++c)
+    err = cudaEventCreateWithFlags(&landed[size_t(c)], cudaEventDisableTiming);
+  // the copies start after the work already queued on st (it may still read P.h)
+  if (err == cudaSuccess) err = cudaEventRecord(start, st);
+  if (err == cudaSuccess) err = cudaStreamWaitEvent(copy_st, start, 0);
+  for (int64_t c = 0; c < n_chunks && err == cudaSuccess; ++c) {
+    const int64_t r0 = c * kHostChunkRows, rc = std::min(kHostChunkRows, n - r0);
+    err = traced(TG_K_COPY, rc, 0.0, double(rc) * row, copy_st, [&] {
+      return cudaMemcpyAsync(static_cast<char*>(P.h) + size_t(r0) * row,
+                             static_cast<const char*>(x_host) + size_t(r0) * row,
+                             size_t(rc) * row, cudaMemcpyHostToDevice, copy_st);
+    });
+    if (err == cudaSuccess) err = cudaEventRecord(landed[size_t(c)], copy_st);
+  }
+  void* k_dst = (kv && kv->k) ? kv->k : P.attn.k_rot;
+  for (int64_t c = 0; c < n_chunks && err == cudaSuccess; ++c) {
+    const int64_t r0 = c * kHostChunkRows, r1 = std::min(n, r0 + kHostChunkRows), rc = r1 - r0;
+    err = cudaStreamWaitEvent(st, landed[size_t(c)], 0);
+    if (err != cudaSuccess) break;
+    char* yc = static_cast<char*>(P.y) + size_t(r0) * row;
+    err = rmsnorm(static_cast<char*>(P.h) + size_t(r0) * row, lw.attn_norm, m.norm_eps, rc, D.d,
+                  m.dtype, yc, st);
+    if (err != cudaSuccess) break;
+    GemmArgs gq = gemm_args(yc, D.d, lw.wqkv, D.d, nullptr, 0, rc, D.qkv, D.d, EPI_QKV);
+    gq.hq = D.hq; gq.hkv = D.hkv; gq.q_norm = lw.q_norm; gq.k_norm = lw.k_norm;
+    gq.eps = m.norm_eps;
+    gq.rope_cs = P.cs_n + r0;
+    gq.rope_ld = n;
+    gq.q_out = static_cast<char*>(P.attn.q_rot) + size_t(r0) * D.hq * D.dh * e;
+    gq.k_out = static_cast<char*>(k_dst) + size_t(r0) * D.hkv * D.dh * e;
+    gq.vT_out = static_cast<__nv_bfloat16*>(P.attn.vT) + r0;
+    gq.t_pad = P.attn.t_pad;
+    gq.v_out = (kv && kv->v) ? static_cast<char*>(kv->v) + size_t(r0) * D.hkv * D.dh * e : nullptr;
+    if (!gemm_tc_supported(gq)) {
+      err = cudaErrorInvalidValue;
+      break;
+    }
+    err = gemm(gq, m.dtype, st);
+    if (err != cudaSuccess) break;
+    // whole query tiles, as the one-shot launch over n > 8192 rows runs them
+    err = attn_core(P.attn, k_dst, nullptr, 0, nullptr, nullptr, nullptr, nullptr, r1, D.hq,
+                    D.hkv, D.dh, m.dtype, P.attn_o, st, nullptr, nullptr, true, r0, true);
+  }
+  release();  // events may still be pending; their resources go when they complete
+  if (err != cudaSuccess) return cuda_status(err);
+  GemmArgs g = gemm_args(P.attn_o, int64_t(D.hq) * D.dh, lw.wo, int64_t(D.hq) * D.dh, P.h, D.d, n,
+                         D.d, D.hq * D.dh, EPI_RESIDUAL);
+  g.R = P.h;
+  g.ldr = D.d;
+  ss_produce(g, P, P.h, 0);
+  TG_TRY(gemm(g, m.dtype, st));
+  ss_mark(P, P.h, n);
+  return TG_OK;
+}
+
 // Stage 1 of the gated forward: the layers below the gate and the gate
 // layer's attention over all n rows (in P.h), then the scores of every row.
+// x_in_h: the input rows are already in P.h. With copy_st, x is a host
+// pointer and layer 0's attention overlaps its copy (attn_layer0_from_host).
 tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan& P, const void* x,
                              int64_t n, int gate_layer, const tg_kv* kv,
-                             const tg_layer_taps* taps, float* sc, cudaStream_t st) {
+                             const tg_layer_taps* taps, float* sc, cudaStream_t st,
+                             bool x_in_h = false, cudaStream_t copy_st = nullptr) {
   const size_t e = elem_size(m.dtype);
-  TG_TRY(copy_rows(P.h, x, size_t(n) * D.d * e, n, st));
+  const bool x_host = copy_st != nullptr;
+  if (!x_in_h && !x_host) TG_TRY(copy_rows(P.h, x, size_t(n) * D.d * e, n, st));
   P.ss_rows_h = -1;  // the input rows carry no row sums
   // every attention launch of the call then finds its split counters zero
   TG_TRY(attn_split_clear(P.attn.split, P.attn.split_bytes, D.hq, st));
@@ -1227,20 +1328,25 @@ tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan
     TG_TRY(traced(TG_K_ROPE_TABLE, n, 0.0, cs_bytes * n, st, [&] {
       return launch_rope_table(nullptr, n, D.dh, m.rope_base, P.cs_n, st);
     }));
-  for (int l = 0; l < gate_layer; ++l) {
+  auto mixer = [&](int l) -> tg_status {
     LayerTag tag(l);
-    TG_TRY(mixer_sublayer(m, m.layers[l], D, P, P.h, n, nullptr, P.cs_n, nullptr, nullptr,
-                              nullptr, nullptr, kv ? &kv[l] : nullptr, st, nullptr,
-                              taps ? &taps[l] : nullptr));
+    if (l == 0 && x_host) return attn_layer0_from_host(m, D, P, x, n, kv ? &kv[0] : nullptr, st,
+                                                       copy_st);
+    return cuda_status(mixer_sublayer(m, m.layers[l], D, P, P.h, n, nullptr, P.cs_n, nullptr,
+                                      nullptr, nullptr, nullptr, kv ? &kv[l] : nullptr, st,
+                                      nullptr, taps ? &taps[l] : nullptr));
+  };
+  for (int l = 0; l < gate_layer; ++l) {
+    const tg_status ms = mixer(l);
+    if (ms != TG_OK) return ms;
+    LayerTag tag(l);
     TG_TRY(ffn_sublayer(m, m.layers[l], D, P, P.h, n, st));
     if (taps && taps[l].hidden)
       TG_TRY(copy_rows(taps[l].hidden, P.h, size_t(n) * D.d * e, n, st));
   }
   if (gate_layer >= 0) {
-    LayerTag tag(gate_layer);
-    TG_TRY(mixer_sublayer(m, m.layers[gate_layer], D, P, P.h, n, nullptr, P.cs_n, nullptr,
-                              nullptr, nullptr, nullptr, kv ? &kv[gate_layer] : nullptr, st,
-                              nullptr, taps ? &taps[gate_layer] : nullptr));
+    const tg_status ms = mixer(gate_layer);
+    if (ms != TG_OK) return ms;
   }
   // score the post-attention residual
   TG_TRY(run_score(P.h, n, D.d, m.d_score, m.score_norm, m.norm_eps, m.score_w1, m.score_b1,
@@ -1378,6 +1484,59 @@ tg_status tg_prefill(const tg_model* model, const void* x, const uint8_t* protec
   const tg_status s1 = prefill_below_gate(m, D, P, x, n, gate_layer, kv, taps, sc, st);
   if (s1 != TG_OK) return s1;
   return prefill_above_gate(m, D, P, protect, n, k, gate_layer, sc, out, kept_idx, kv, taps, st);
+}
+
+// A non-blocking stream per device for the host-input copies of
+// tg_prefill_host (created on first use, kept for the process).
+static cudaStream_t host_copy_stream(cudaError_t* err) {
+  static std::mutex mu;
+  static std::map<int, cudaStream_t> streams;
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = streams.find(dev);
+  if (it != streams.end()) return it->second;
+  cudaStream_t s = nullptr;
+  *err = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
+  if (*err != cudaSuccess) return nullptr;
+  streams[dev] = s;
+  return s;
+}
+
+tg_status tg_prefill_host(const tg_model* model, const void* x_host, const uint8_t* protect,
+                          int64_t n, int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx,
+                          float* scores, const tg_kv* kv, void* ws, size_t ws_bytes,
+                          tg_stream stream) {
+  const tg_status vs = validate_model(model, n, k, gate_layer);
+  if (vs != TG_OK) return vs;
+  TG_CHECK(x_host && out && kept_idx, TG_ERR_INVALID_ARG);
+  const tg_model& m = *model;
+  if (m.dtype == TG_BF16) TG_CHECK(aligned16(out), TG_ERR_INVALID_ARG);
+  if (m.dtype == TG_BF16 && kv != nullptr)
+    for (int l = 0; l < m.n_layers; ++l)
+      TG_CHECK(aligned16(kv[l].k) && aligned16(kv[l].v), TG_ERR_INVALID_ARG);
+  PrefillPlan P(nullptr, m, n, k);
+  TG_CHECK(ws != nullptr && ws_bytes >= P.bytes, TG_ERR_WORKSPACE);
+  P = PrefillPlan(ws, m, n, k);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Dims D = model_dims(m);
+  float* sc = scores ? scores : P.scores;
+  tg_status s1 = TG_OK;
+  if (host_chunks_apply(m, D, n, gate_layer)) {
+    cudaError_t e = cudaSuccess;
+    cudaStream_t cs = host_copy_stream(&e);
+    if (e != cudaSuccess) return cuda_status(e);
+    s1 = prefill_below_gate(m, D, P, x_host, n, gate_layer, kv, nullptr, sc, st, false, cs);
+  } else {
+    const size_t bytes = size_t(n) * D.d * elem_size(m.dtype);
+    TG_TRY(traced(TG_K_COPY, n, 0.0, double(bytes), st, [&] {
+      return cudaMemcpyAsync(P.h, x_host, bytes, cudaMemcpyHostToDevice, st);
+    }));
+    s1 = prefill_below_gate(m, D, P, P.h, n, gate_layer, kv, nullptr, sc, st, true);
+  }
+  if (s1 != TG_OK) return s1;
+  return prefill_above_gate(m, D, P, protect, n, k, gate_layer, sc, out, kept_idx, kv, nullptr, st);
 }
 
 tg_status tg_prefill_multi(const tg_model* model, const void* x, const uint8_t* protect,

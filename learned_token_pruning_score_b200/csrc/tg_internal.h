@@ -155,6 +155,7 @@ struct GemmArgs {
   int hq, hkv;
   const float2* rope_cs; const float* q_norm; const float* k_norm; float eps;
   void* q_out; void* k_out; void* vT_out; int64_t t_pad; void* v_out;
+  int64_t rope_ld = 0;  // stride of rope_cs between frequencies (0: M)
   // Folded RMSNorm (tensor-core path only). RESIDUAL: ss_out[nb * ss_ld + m]
   // = sum of squares of the stored bf16 row m over the tile column block nb
   // (256 columns; ceil(N / 256) blocks). STORE / SWIGLU / SCORE / QKV: when
@@ -193,6 +194,10 @@ struct AttnArgs {
   void* split_ws = nullptr;
   size_t split_ws_bytes = 0;
   bool split_cnt_zeroed = false;
+  // First query row of this launch (a multiple of 128; paired-head bf16
+  // kernel only): rows [q_lo, T) attend to keys [0, T). Rows below q_lo are
+  // neither read as queries nor written.
+  int64_t q_lo = 0;
 };
 // Scratch the tensor-core attention over T rows can use to split long query
 // tiles across CTAs (0 when T is too long to need it).

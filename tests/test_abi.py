@@ -222,6 +222,23 @@ def test_prefill_validation_folded_norm_weights():
     assert _prefill(ctypes.byref(m), 1000, 100, 1, 16) == tg.TG_ERR_WORKSPACE  # valid otherwise
 
 
+def test_prefill_host_validation():
+    m, keep = _bogus_model()
+    big = 1 << 40
+    f = tg._prefill_host
+
+    def call(x=BOGUS, n=1000, k=100, gate=1, ws_bytes=big, out=BOGUS):
+        return f(ctypes.byref(m), x, None, n, k, gate, out, BOGUS, None, None, BOGUS, ws_bytes,
+                 None)
+
+    assert call(x=None) == tg.TG_ERR_INVALID_ARG
+    assert call(out=None) == tg.TG_ERR_INVALID_ARG
+    assert call(out=ctypes.c_void_p(4096 + 2)) == tg.TG_ERR_INVALID_ARG
+    assert call(k=0) == tg.TG_ERR_BUDGET
+    assert call(gate=2) == tg.TG_ERR_INVALID_ARG
+    assert call(ws_bytes=16) == tg.TG_ERR_WORKSPACE
+
+
 def test_fold_norm_weight_validation():
     f = tg._fold
     w, g, out = 4096, 1 << 20, 1 << 24

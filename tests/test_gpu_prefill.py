@@ -130,6 +130,41 @@ def test_gated_equals_dense_when_all_kept():
     assert torch.equal(out_g, out_d)
 
 
+@pytest.mark.parametrize("n", [16684, 700])
+def test_prefill_from_host_memory_equals_device_input(n):
+    """tg_prefill_host (x in pinned host memory) gives tg_prefill's results
+    bit for bit: above 8192 rows the copy is chunked and layer 0's norm, QKV
+    projection and attention run per chunk as the rows land (n = 16684: four
+    whole 4096-row chunks and a ragged one); below, one copy then the same
+    path."""
+    w = synth.shrink(synth.QWEN_LAYER_16K, name="host_in", n=n, k=n // 5, d=256, hq=4, hkv=2,
+                     dh=128, f=64, inter=256, n_layers=3, gate_layer=1, n_protect=16, seed=81,
+                     qk_norm=True)
+    rng = synth.rng_for(w.seed)
+    model, _ = build_models(w, rng, torch.bfloat16)
+    x = torch.from_numpy(synth.hidden_states(w, rng)).to("cuda", torch.bfloat16)
+    prot = torch.from_numpy(synth.protect_tail(w.n, w.n_protect)).cuda()
+
+    def kvs():
+        return [(torch.zeros(w.n if li <= w.gate_layer else w.k, w.hkv, w.dh, device="cuda",
+                             dtype=torch.bfloat16),
+                 torch.zeros(w.n if li <= w.gate_layer else w.k, w.hkv, w.dh, device="cuda",
+                             dtype=torch.bfloat16)) for li in range(w.n_layers)]
+    kv_d, kv_h = kvs(), kvs()
+    sc_d = torch.empty(w.n, device="cuda")
+    sc_h = torch.empty(w.n, device="cuda")
+    out_d, kept_d, _ = tg.tg_prefill(model, x, prot, w.k, w.gate_layer, scores=sc_d, kv=kv_d)
+    x_host = x.cpu().pin_memory()
+    out_h, kept_h, _ = tg.tg_prefill_host(model, x_host, prot, w.k, w.gate_layer, scores=sc_h,
+                                          kv=kv_h)
+    torch.cuda.synchronize()
+    assert torch.equal(kept_h, kept_d)
+    assert torch.equal(sc_h, sc_d)
+    assert torch.equal(out_h, out_d)
+    for (kd, vd), (kh, vh) in zip(kv_d, kv_h):
+        assert torch.equal(kh, kd) and torch.equal(vh, vd)
+
+
 def test_pruned_tokens_make_no_upper_kv():
     w = synth.shrink(synth.QWEN_LAYER_16K, name="kvrows", n=300, k=60, d=256, hq=4, hkv=2, dh=128,
                      f=64, inter=256, n_layers=3, gate_layer=0, n_protect=6, seed=9)
