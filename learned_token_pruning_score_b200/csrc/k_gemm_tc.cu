@@ -102,10 +102,13 @@ __device__ __forceinline__ void add32_bf16(const __nv_bfloat16* src, float (&v)[
 // The fused epilogue of one accumulator tile, run by one epilogue warp for
 // its 32 rows: this thread owns accumulator row `row` (global index), whose
 // kBN fp32 columns start at TMEM address `t_row`; `nb` is the tile's column
-// block.
+// block; `stage` (QKV only): the warp's 8 KB of shared memory (1024-byte
+// aligned) through which its 32 rows of a q/k head leave in two TMA stores
+// (tm_q / tm_k: q_out [M, hq, 128] and k_out [M, hkv, 128], boxes of 64 x 1 x 32).
 template <int kBN, int kEpi>
 __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, uint32_t t_row,
-                                              int nb) {
+                                              int nb, uint8_t* stage, const CUtensorMap* tm_q,
+                                              const CUtensorMap* tm_k) {
   const bool row_ok = row < p.M;
   // Folded RMSNorm of the input row: B holds W . diag(g), and the row's
   // accumulator is scaled by rs = 1 / sqrt(mean(x^2) + eps), the mean from the
@@ -177,10 +180,14 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
           }
           rstd = rsqrtf(ss * (1.0f / 128.0f) + p.eps);
         }
-        __nv_bfloat16* dst =
-            is_q ? p.q_out + (row * p.hq + hg) * 128
-                 : p.k_out + (row * p.hkv + (hg - p.hq)) * 128;
         const float2* cs = p.rope_cs + row;  // frequency-major: entry i at cs[i * rope_ld]
+        const int lane = static_cast<int>(threadIdx.x & 31);
+        // The stage is free once this warp's previous stores have read it.
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+        // this thread's row in the stage: two 64-column boxes of 32 rows x 128
+        // bytes, 128-byte swizzle (16-byte unit u of row r at u ^ (r & 7))
+        uint8_t* srow = stage + lane * 128;
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           float lo[32], hi[32];
@@ -200,9 +207,33 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, int64_t row, u
               lo[i] = a * t.x - b * t.y;
               hi[i] = b * t.x + a * t.y;
             }
-            store32_bf16(dst + c * 32, lo);
-            store32_bf16(dst + 64 + c * 32, hi);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 ul, uh;
+              ul.x = pack_bf16x2(lo[8 * q + 0], lo[8 * q + 1]);
+              ul.y = pack_bf16x2(lo[8 * q + 2], lo[8 * q + 3]);
+              ul.z = pack_bf16x2(lo[8 * q + 4], lo[8 * q + 5]);
+              ul.w = pack_bf16x2(lo[8 * q + 6], lo[8 * q + 7]);
+              uh.x = pack_bf16x2(hi[8 * q + 0], hi[8 * q + 1]);
+              uh.y = pack_bf16x2(hi[8 * q + 2], hi[8 * q + 3]);
+              uh.z = pack_bf16x2(hi[8 * q + 4], hi[8 * q + 5]);
+              uh.w = pack_bf16x2(hi[8 * q + 6], hi[8 * q + 7]);
+              // dims 32c + 8q (box 0) and 64 + 32c + 8q (box 1): unit 4c + q
+              const int u = (4 * c + q) ^ (lane & 7);
+              *reinterpret_cast<uint4*>(srow + (u << 4)) = ul;
+              *reinterpret_cast<uint4*>(srow + 4096 + (u << 4)) = uh;
+            }
           }
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {  // rows past M are not written
+          const int64_t row0 = row - lane;
+          const CUtensorMap* tm = is_q ? tm_q : tm_k;
+          const int head = is_q ? hg : hg - p.hq;
+          tma_store_3d(tm, stage, 0, head, static_cast<int>(row0));
+          tma_store_3d(tm, stage + 4096, 64, head, static_cast<int>(row0));
+          bulk_commit();
         }
       } else {
         const int g = hg - p.hq - p.hkv;
@@ -249,12 +280,20 @@ struct PairCfg {
   static constexpr int kStages = 6;
   static constexpr int kTmemCols = 512;                  // 2 x 256 fp32 accumulators
   static constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes + 256;
+  // QKV: 8 KB per epilogue warp (after the barriers, 1024-aligned) through
+  // which its q/k rows leave by TMA
+  static constexpr size_t kStageQkv = 1024 - 256 + 4 * 8192;
 };
+template <int kEpi>
+constexpr size_t gemm_smem() {
+  return PairCfg::kSmem + (kEpi == EPI_QKV ? PairCfg::kStageQkv : 0);
+}
 
 template <int kEpi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 EpiParams p) {
+            const __grid_constant__ CUtensorMap tmQo, const __grid_constant__ CUtensorMap tmKo,
+            EpiParams p) {
   using C = PairCfg;
   constexpr int kBN = 256;
   static_assert(kBN == kSsBlockCols, "row sums of squares are per 256-column block");
@@ -380,11 +419,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           static_cast<int64_t>(mb) * 256 + static_cast<int64_t>(rank) * 128 + quarter * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(a * kBN);
-      epilogue_tile<kBN, kEpi>(p, row, t_row, nb);
+      uint8_t* stage = kEpi == EPI_QKV
+                           ? tiles + size_t(C::kStages) * C::kStageBytes + 1024 + quarter * 8192
+                           : nullptr;
+      epilogue_tile<kBN, kEpi>(p, row, t_row, nb, stage, &tmQo, &tmKo);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&acc_empty[a]), 0));
     }
+    // the last TMA stores have read this warp's stage before the CTA exits
+    if (kEpi == EPI_QKV && lane == 0) bulk_wait_read_all();
   }
   tc_fence_before();
   cluster_sync();
@@ -396,9 +440,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 template <int kEpi>
 cudaError_t run(const GemmArgs& g, cudaStream_t st) {
   using C = PairCfg;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tqo, tko;
   if (!make_tmap_2d_bf16(&ta, g.A, g.M, g.K, g.lda, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d_bf16(&tb, g.B, g.N, g.K, g.ldb, 128)) return cudaErrorInvalidValue;
+  if (kEpi == EPI_QKV) {  // q_out [M, hq, 128] and k_out [M, hkv, 128], 32-row boxes
+    if (!make_tmap_3d_bf16(&tqo, g.q_out, 128, g.hq, g.M, 256, int64_t(g.hq) * 256, 1, 32) ||
+        !make_tmap_3d_bf16(&tko, g.k_out, 128, g.hkv, g.M, 256, int64_t(g.hkv) * 256, 1, 32))
+      return cudaErrorInvalidValue;
+  } else {
+    tqo = ta;  // not read
+    tko = ta;
+  }
   EpiParams p;
   p.M = g.M;
   p.N = kEpi == EPI_SWIGLU ? g.inter : g.N;
@@ -436,7 +488,9 @@ cudaError_t run(const GemmArgs& g, cudaStream_t st) {
   const int tiles = p.tiles_m * p.tiles_n;
   if (tiles == 0) return cudaSuccess;
   auto kern = gemm_tc<kEpi>;
-  cudaError_t e = set_smem_attr_once(reinterpret_cast<const void*>(kern), static_cast<int>(C::kSmem));
+  constexpr size_t kSmemBytes = gemm_smem<kEpi>();
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+  cudaError_t e = set_smem_attr_once(reinterpret_cast<const void*>(kern), static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   // Persistent grid: as many pairs as can be resident at once (the SMs of a
   // pair must share a TPC, so this can be below num_sms() / 2).
@@ -449,7 +503,7 @@ cudaError_t run(const GemmArgs& g, cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(num_sms() & ~1), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = st;
     if (cudaOccupancyMaxActiveClusters(&max_pairs, kern, &cfg) != cudaSuccess || max_pairs <= 0) {
       cudaGetLastError();
@@ -458,7 +512,7 @@ cudaError_t run(const GemmArgs& g, cudaStream_t st) {
     if (dev >= 0 && dev < kMaxDevices) resident[dev].store(max_pairs);
   }
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
-  return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), C::kSmem, st, ta, tb, p);
+  return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), kSmemBytes, st, ta, tb, tqo, tko, p);
 }
 
 }  // namespace
