@@ -415,7 +415,10 @@ typedef struct {
  * rows run on `stream` as soon as the chunk has landed, so that the copy
  * overlaps layer 0 (the results are the same as tg_prefill's bit for bit).
  * Returns when the work is queued on `stream`; x must stay valid until the
- * stream reaches the end of the call's work.
+ * stream reaches the end of the call's work. The chunked copy uses one
+ * non-blocking stream per device (created on the first such call, kept for
+ * the process) and a few CUDA events per call; no device memory is
+ * allocated.
  */
 tg_status tg_prefill_host(const tg_model* model, const void* x_host, const uint8_t* protect,
                           int64_t n, int64_t k, int32_t gate_layer, void* out, int32_t* kept_idx,
