@@ -592,12 +592,14 @@ __global__ void __launch_bounds__(kCThreads, 1)
   const uint32_t packed = cta_excl_scan_1024((nd << 16) | nt, &packed_cta, warp_sums);
   if (tid == 0) cta_val[1] = packed_cta;
   sel_sync<kOne>();
-  if (tid < static_cast<int>(rank)) tot[tid] = ld_rank<kOne>(&cta_val[1], tid);
-  __syncthreads();
   uint32_t sb = packed >> 16, tb = packed & 0xFFFFu;
-  for (uint32_t r = 0; r < rank; ++r) {
-    sb += tot[r] >> 16;
-    tb += tot[r] & 0xFFFFu;
+  if constexpr (!kOne) {  // the counts of the CTAs before this one
+    if (tid < static_cast<int>(rank)) tot[tid] = ld_rank<kOne>(&cta_val[1], tid);
+    __syncthreads();
+    for (uint32_t r = 0; r < rank; ++r) {
+      sb += tot[r] >> 16;
+      tb += tot[r] & 0xFFFFu;
+    }
   }
 #pragma unroll
   for (int j = 0; j < kPer; ++j) {
