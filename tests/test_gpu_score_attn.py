@@ -161,11 +161,14 @@ def test_attn_reduces_to_causal_attention_when_gain_zero_tau_one():
 
 
 @pytest.mark.parametrize("m,n,k", [(1, 256, 64), (127, 2048, 2048), (1000, 4096, 2048),
-                                   (300, 2048, 6144), (4096, 288, 520)])
+                                   (300, 2048, 6144), (4096, 288, 520),
+                                   (4000, 1824, 520), (8192, 2048, 2048)])
 @pytest.mark.parametrize("residual", [False, True])
 def test_linear_bf16(m, n, k, residual):
     """The tcgen05 GEMM against a float64 product of the same bf16 values
-    (ragged m, k not a multiple of 64, n not a multiple of 256)."""
+    (ragged m, k not a multiple of 64, n not a multiple of 256). The last two
+    shapes fill more than one wave of pair tiles, the first of them with a
+    ragged last column block."""
     rng = np.random.default_rng(m + n + k)
     x = dev(rng.standard_normal((m, k)), torch.bfloat16)
     w = dev(rng.standard_normal((n, k)) * 0.02, torch.bfloat16)
