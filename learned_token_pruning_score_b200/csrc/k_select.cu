@@ -8,14 +8,17 @@
 // with -0.0 == +0.0 and NaN lowest.
 //
 // Method: radix select over the 32-bit order-preserving key of each fp32
-// score, in three digits (11, 11, 10 bits). Each pass histograms the next
-// digit of the keys that still match the prefix found so far; every CTA
-// finds the threshold bin from the finished histogram of the previous pass
-// (identical work, identical result), so no CTA waits on another. The last
-// two kernels count, per chunk, the tokens kept for sure and the tokens tied
-// at the threshold key, then write the kept indices in index order: the tied
-// tokens taken are the lowest-index ones. Integer atomics only, so the
-// result is bit-reproducible.
+// score. Up to 131072 tokens (sel_cluster): one launch of one CTA or one
+// thread-block cluster, keys in registers, four 8-bit digits with one
+// cluster barrier each. Above that (sel_hist0 ... sel_write): five kernels
+// over the key stream in three digits (11, 11, 10 bits). Each pass
+// histograms the next digit of the keys that still match the prefix found
+// so far; every CTA finds the threshold bin from the finished histogram of
+// the previous pass (identical work, identical result), so no CTA waits on
+// another. The last step counts, per chunk, the tokens kept for sure and the
+// tokens tied at the threshold key, then writes the kept indices in index
+// order: the tied tokens taken are the lowest-index ones. Integer atomics
+// only, so the result is bit-reproducible.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -425,17 +428,6 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
   return v;
 }
 
-// Sum over the CTA's 1024 threads into *dst (zeroed by the caller before
-// the __syncthreads that precedes this call); every thread sees the sum after
-// the call's __syncthreads.
-__device__ __forceinline__ uint32_t cta_sum_1024(uint32_t v, uint32_t* dst) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-  if ((threadIdx.x & 31) == 0 && v) atomicAdd(dst, v);
-  __syncthreads();
-  return *dst;
-}
-
 // kPer tokens per thread (a multiple of 8); kOne: a single CTA (no
 // cluster), whose barriers are plain __syncthreads and whose "remote" shared
 // memory is its own.
@@ -450,24 +442,30 @@ __device__ __forceinline__ uint32_t ld_rank(const uint32_t* p, uint32_t rank) {
   return ld_cluster_u32(mapa_shared(smem_addr(p), rank));
 }
 
+// One launch, four 8-bit digits, most significant first. Pass p histograms
+// digit p of the unprotected keys that match the digits found so far into
+// hist[p & 1] (pass 0 also counts the CTA's protected tokens, in bin 256).
+// One barrier over the cluster per pass; then every CTA sums the cluster's
+// counts itself and its warp 0 scans the 256 bins from the top for the bin
+// where the count reaches `need`, so no second exchange is needed. A buffer
+// is zeroed again in the pass after its use, once every CTA has passed that
+// pass's barrier and so has finished reading it.
+constexpr int kRBins = 260;  // 256 digit bins + the protected count, padded
 template <bool kVec, int kPer, bool kOne>
 __global__ void __launch_bounds__(kCThreads, 1)
     sel_cluster(const float* __restrict__ scores, const uint8_t* __restrict__ protect, int64_t n,
                 int64_t k, int32_t* __restrict__ kept_idx, int32_t* __restrict__ status) {
-  __shared__ uint32_t hist[2048];   // this CTA's counts of the current digit
-  __shared__ uint32_t red[2048];    // cluster sums of this CTA's slice of the bins
-  __shared__ uint32_t cta_val[4];   // 0 / 3: slice total of even / odd passes (another
-                                    // CTA may still read a pass's slot during the next
-                                    // pass), 1: sure keeps | ties (16 + 16 bits),
-                                    // 2: protected
+  __shared__ uint32_t hist[2 * kRBins];  // this CTA's counts, even / odd passes
+  __shared__ uint32_t red[kRBins];       // the cluster's counts of the current pass
+  __shared__ uint32_t cta_val[2];        // 1: sure keeps | ties (16 + 16 bits)
   __shared__ uint32_t tot[kCMaxCtas];
   __shared__ uint32_t warp_sums[32];
-  __shared__ uint32_t s_bin, s_need;
+  __shared__ uint32_t s_bin, s_need, s_stop;
   pdl_trigger();
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t C = gridDim.x;  // the grid is one cluster
   const uint32_t rank = kOne ? 0u : cluster_ctarank();
-  if (tid < 4) cta_val[tid] = 0u;
+  for (int i = tid; i < 2 * kRBins; i += kCThreads) hist[i] = 0u;
   __syncthreads();
   pdl_wait();
   static_assert(kPer % kPerThread == 0 && kPer <= 16, "tokens per thread");
@@ -486,89 +484,98 @@ __global__ void __launch_bounds__(kCThreads, 1)
       if (pq[j]) pmask |= 1u << (q * kPerThread + j);
     }
   }
-  uint32_t np_t = 0;
+  uint32_t np_w = 0;
 #pragma unroll
   for (int j = 0; j < kPer; ++j)
-    if (j < valid && ((pmask >> j) & 1u)) ++np_t;
-  cta_sum_1024(np_t, &cta_val[2]);
-  sel_sync<kOne>();
-  if (tid < static_cast<int>(C)) tot[tid] = ld_rank<kOne>(&cta_val[2], tid);
-  __syncthreads();
-  uint32_t np = 0;
-  for (uint32_t r = 0; r < C; ++r) np += tot[r];
-  const bool over = static_cast<int64_t>(np) > k;
-  uint32_t thresh = 0xFFFFFFFFu, ties = 0u;  // np == k: no unprotected token is kept
-  uint32_t need = over ? 0u : static_cast<uint32_t>(k - static_cast<int64_t>(np));
-  if (need > 0u) {
-    uint32_t prefix = 0u;
+    if (j < valid && ((pmask >> j) & 1u)) ++np_w;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) np_w += __shfl_xor_sync(0xFFFFFFFFu, np_w, o);
+  bool over = false;
+  uint32_t prefix = 0u, need = 0u;
+  uint32_t thresh = 0xFFFFFFFFu, ties = 0u;  // no unprotected token kept
 #pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-      const int bins = pass == 2 ? 1024 : 2048;
-      const int pbits = pass == 0 ? 0 : (pass == 1 ? 11 : 22);  // prefix bits so far
-      uint32_t* slice_tot = &cta_val[(pass & 1) ? 3 : 0];  // last read two passes ago
-      for (int i = tid; i < bins; i += kCThreads) hist[i] = 0u;
-      if (tid == 0) *slice_tot = 0u;
-      __syncthreads();
-      // A warp whose 32 keys fall in one bin (tied scores) adds once;
-      // otherwise one shared-memory atomic per active key.
+  for (int pass = 0; pass < 4; ++pass) {
+    uint32_t* h = hist + (pass & 1) * kRBins;
+    const int shift = 24 - 8 * pass;
+    if (pass == 0 && lane == 0 && np_w) atomicAdd(&h[256], np_w);
+    // A warp whose keys are all active and in one bin (a run of tied
+    // scores) adds once, a warp with no active key skips the pass; otherwise
+    // one shared-memory atomic per active key. One vote per warp and pass.
+    uint32_t bin[kPer];
+    bool same = true;
 #pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        const bool act = j < valid && !((pmask >> j) & 1u) &&
-                         (pass == 0 || (key[j] >> (32 - pbits)) == prefix);
-        const uint32_t bin = act ? (key[j] >> shift) & static_cast<uint32_t>(bins - 1) : 0xFFFFFFFFu;
-        const uint32_t bin0 = __shfl_sync(0xFFFFFFFFu, bin, 0);
-        if (__all_sync(0xFFFFFFFFu, bin == bin0)) {
-          if (lane == 0 && bin0 != 0xFFFFFFFFu) atomicAdd(&hist[bin0], 32u);
-        } else if (act) {
-          atomicAdd(&hist[bin], 1u);
-        }
-      }
-      sel_sync<kOne>();
-      // this CTA's slice of the bins, summed over the cluster
-      const uint32_t S = static_cast<uint32_t>(bins) / C;
-      uint32_t part = 0u;
-      for (uint32_t t = tid; t < S; t += kCThreads) {
-        const uint32_t b = rank * S + t;
-        uint32_t sum = 0u;
-        for (uint32_t r = 0; r < C; ++r) sum += ld_rank<kOne>(&hist[b], r);
-        red[t] = sum;
-        part += sum;
-      }
-      cta_sum_1024(part, slice_tot);
-      sel_sync<kOne>();
-      // the slice (from the top) where the count reaches `need`, then the bin
-      if (tid < static_cast<int>(C)) tot[tid] = ld_rank<kOne>(slice_tot, tid);
-      __syncthreads();
-      uint32_t above = 0u, sl = 0u;
-      for (int r = static_cast<int>(C) - 1; r >= 0; --r) {
-        if (above + tot[r] >= need) {
-          sl = static_cast<uint32_t>(r);
-          break;
-        }
-        above += tot[r];
-      }
-      const uint32_t rest = need - above;
-      // slice sl's bins in descending order: thread t holds elements
-      // 2t, 2t + 1 (element e = bin S - 1 - e of the slice)
-      uint32_t v[2] = {0u, 0u};
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const uint32_t e = 2u * tid + q;
-        if (e < S) v[q] = ld_rank<kOne>(&red[S - 1 - e], sl);
-      }
-      const uint32_t before = cta_excl_scan_1024(v[0] + v[1], nullptr, warp_sums);
-      if (before < rest && rest <= before + v[0] + v[1]) {
-        const uint32_t e = before + v[0] >= rest ? 2u * tid : 2u * tid + 1u;
-        s_bin = sl * S + (S - 1 - e);
-        s_need = rest - (e == 2u * tid ? before : before + v[0]);
-      }
-      __syncthreads();
-      prefix = pass == 0 ? s_bin : ((prefix << (pass == 1 ? 11 : 10)) | s_bin);
-      need = s_need;
+    for (int j = 0; j < kPer; ++j) {
+      const bool act = j < valid && !((pmask >> j) & 1u) &&
+                       (pass == 0 || (key[j] >> (32 - 8 * pass)) == prefix);
+      bin[j] = act ? (key[j] >> shift) & 0xFFu : 0xFFFFFFFFu;
+      same = same && bin[j] == bin[0];
     }
-    thresh = prefix;
-    ties = need;
+    const uint32_t wbin = __shfl_sync(0xFFFFFFFFu, bin[0], 0);
+    if (__all_sync(0xFFFFFFFFu, same && bin[0] == wbin)) {
+      if (lane == 0 && wbin != 0xFFFFFFFFu) atomicAdd(&h[wbin], 32u * kPer);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kPer; ++j)
+        if (bin[j] != 0xFFFFFFFFu) atomicAdd(&h[bin[j]], 1u);
+    }
+    sel_sync<kOne>();  // every CTA's counts of this pass are complete
+    if (tid <= 256) {
+      uint32_t sum = 0u;
+      for (uint32_t r = 0; r < C; ++r) sum += ld_rank<kOne>(&h[tid], r);
+      red[tid] = sum;
+    } else if (tid >= 512 && tid < 512 + kRBins) {
+      hist[((pass + 1) & 1) * kRBins + (tid - 512)] = 0u;  // read last in the pass before
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t nd = need, stop = 0u;
+      if (pass == 0) {
+        const uint32_t np = red[256];
+        if (static_cast<int64_t>(np) > k) stop = 2u;
+        else nd = static_cast<uint32_t>(k - static_cast<int64_t>(np));
+        if (nd == 0u && stop == 0u) stop = 1u;
+      }
+      if (stop == 0u) {
+        // lane l holds bins 255 - 8l ... 248 - 8l (descending)
+        uint32_t c[8], sum = 0u;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          c[q] = red[255 - 8 * lane - q];
+          sum += c[q];
+        }
+        uint32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        uint32_t run = incl - sum;
+        if (run < nd && nd <= incl) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            if (run + c[q] >= nd) {
+              s_bin = static_cast<uint32_t>(255 - 8 * lane - q);
+              s_need = nd - run;
+              break;
+            }
+            run += c[q];
+          }
+        }
+      }
+      if (lane == 0) s_stop = stop;
+    }
+    __syncthreads();
+    const uint32_t stop = s_stop;
+    if (stop != 0u) {
+      over = stop == 2u;
+      break;
+    }
+    prefix = (prefix << 8) | s_bin;
+    need = s_need;
+    if (pass == 3) {
+      thresh = prefix;
+      ties = need;
+    }
   }
   if (over) {
     if (rank == 0 && tid == 0) *status = 3;
@@ -656,8 +663,9 @@ int cluster_ctas(int64_t n) {
   return c <= max_ctas ? c : 0;
 }
 
-// One CTA (n <= 2 x 8192: up to 16 tokens per thread, no cluster barriers),
-// else one cluster of `ctas` CTAs with 8 tokens per thread.
+// One CTA (n <= 8192, no cluster barriers), else one cluster of `ctas`
+// CTAs; 8 tokens per thread. (One CTA with 16 tokens per thread at
+// n <= 16384 measured as slow as a 4-CTA cluster at 32768.)
 template <bool kVec>
 cudaError_t run_select_cluster(const float* scores, const uint8_t* protect, int64_t n, int64_t k,
                                int32_t* kept_idx, void* ws, int ctas, cudaStream_t st) {
@@ -669,13 +677,10 @@ cudaError_t run_select_cluster(const float* scores, const uint8_t* protect, int6
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   int32_t* status = static_cast<int32_t*>(ws);
-  if (n <= 2 * kCChunk) {
+  if (n <= kCChunk) {
     cfg.gridDim = dim3(1);
     cfg.numAttrs = 1;
-    if (n <= kCChunk)
-      return cudaLaunchKernelEx(&cfg, sel_cluster<kVec, 8, true>, scores, protect, n, k, kept_idx,
-                                status);
-    return cudaLaunchKernelEx(&cfg, sel_cluster<kVec, 16, true>, scores, protect, n, k,
+    return cudaLaunchKernelEx(&cfg, sel_cluster<kVec, kPerThread, true>, scores, protect, n, k,
                               kept_idx, status);
   }
   cfg.gridDim = dim3(static_cast<unsigned>(ctas));
