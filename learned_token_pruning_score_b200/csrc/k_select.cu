@@ -428,9 +428,8 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
   return v;
 }
 
-// kPer tokens per thread (a multiple of 8); kOne: a single CTA (no
-// cluster), whose barriers are plain __syncthreads and whose "remote" shared
-// memory is its own.
+// kOne: a single CTA (no cluster), whose barriers are plain __syncthreads
+// and whose "remote" shared memory is its own.
 template <bool kOne>
 __device__ __forceinline__ void sel_sync() {
   if (kOne) __syncthreads();
@@ -449,7 +448,8 @@ __device__ __forceinline__ uint32_t ld_rank(const uint32_t* p, uint32_t rank) {
 // counts itself and its warp 0 scans the 256 bins from the top for the bin
 // where the count reaches `need`, so no second exchange is needed. A buffer
 // is zeroed again in the pass after its use, once every CTA has passed that
-// pass's barrier and so has finished reading it.
+// pass's barrier and so has finished reading it. kPer tokens per thread (a
+// multiple of 8).
 constexpr int kRBins = 260;  // 256 digit bins + the protected count, padded
 template <bool kVec, int kPer, bool kOne>
 __global__ void __launch_bounds__(kCThreads, 1)
@@ -457,7 +457,7 @@ __global__ void __launch_bounds__(kCThreads, 1)
                 int64_t k, int32_t* __restrict__ kept_idx, int32_t* __restrict__ status) {
   __shared__ uint32_t hist[2 * kRBins];  // this CTA's counts, even / odd passes
   __shared__ uint32_t red[kRBins];       // the cluster's counts of the current pass
-  __shared__ uint32_t cta_val[2];        // 1: sure keeps | ties (16 + 16 bits)
+  __shared__ uint32_t cta_val[2];        // [1]: the CTA's sure keeps | ties (16 + 16 bits)
   __shared__ uint32_t tot[kCMaxCtas];
   __shared__ uint32_t warp_sums[32];
   __shared__ uint32_t s_bin, s_need, s_stop;
