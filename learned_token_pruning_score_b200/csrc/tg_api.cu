@@ -580,14 +580,18 @@ cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims
                                const float2* cs, const float* lsig, const void* kaug,
                                const float* gain, const float* tau, const tg_kv* kv,
                                cudaStream_t st, const SegRows* segs = nullptr,
-                               const tg_layer_taps* taps = nullptr) {
+                               const tg_layer_taps* taps = nullptr,
+                               const void* h_in = nullptr) {
   const tg_dtype dt = m.dtype;
   const size_t e = elem_size(dt);
+  // h_in: the sub-layer's input rows when they are not in h yet (the
+  // stack's input, read in place); the output rows h = h_in + attention go to h
+  const void* hsrc = h_in ? h_in : h;
   // folded RMSNorm (h's rows fresh from a residual GEMM), else the norm kernel
-  const bool fold = lw.wqkv_g != nullptr && ss_ready(P, h, rows);
+  const bool fold = lw.wqkv_g != nullptr && h_in == nullptr && ss_ready(P, h, rows);
   cudaError_t err = cudaSuccess;
   if (!fold) {
-    err = rmsnorm(h, lw.attn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
+    err = rmsnorm(hsrc, lw.attn_norm, m.norm_eps, rows, D.d, dt, P.y, st);
     if (err != cudaSuccess) return err;
   }
   const void* xin = fold ? h : P.y;
@@ -629,7 +633,7 @@ cudaError_t attention_sublayer(const tg_model& m, const tg_layer& lw, const Dims
   }
   GemmArgs g = gemm_args(P.attn_o, int64_t(D.hq) * D.dh, lw.wo, int64_t(D.hq) * D.dh, h, D.d, rows,
                          D.d, D.hq * D.dh, EPI_RESIDUAL);
-  g.R = h;
+  g.R = hsrc;
   g.ldr = D.d;
   ss_produce(g, P, h, 0);
   err = gemm(g, dt, st);
@@ -1318,7 +1322,11 @@ tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan
                              bool x_in_h = false, cudaStream_t copy_st = nullptr) {
   const size_t e = elem_size(m.dtype);
   const bool x_host = copy_st != nullptr;
-  if (!x_in_h && !x_host) TG_TRY(copy_rows(P.h, x, size_t(n) * D.d * e, n, st));
+  // Device input and an attention layer 0 below or at the gate: layer 0
+  // reads x in place and writes its residual output into P.h, so x is never
+  // copied. (Scores of the input itself, gate_layer < 0, need x in P.h.)
+  const bool x_direct = !x_in_h && !x_host && gate_layer >= 0 && m.layers[0].gdn == nullptr;
+  if (!x_in_h && !x_host && !x_direct) TG_TRY(copy_rows(P.h, x, size_t(n) * D.d * e, n, st));
   P.ss_rows_h = -1;  // the input rows carry no row sums
   // every attention launch of the call then finds its split counters zero
   TG_TRY(attn_split_clear(P.attn.split, P.attn.split_bytes, D.hq, st));
@@ -1332,6 +1340,10 @@ tg_status prefill_below_gate(const tg_model& m, const Dims& D, const PrefillPlan
     LayerTag tag(l);
     if (l == 0 && x_host) return attn_layer0_from_host(m, D, P, x, n, kv ? &kv[0] : nullptr, st,
                                                        copy_st);
+    if (l == 0 && x_direct)
+      return cuda_status(attention_sublayer(m, m.layers[0], D, P, P.h, n, nullptr, P.cs_n, nullptr,
+                                            nullptr, nullptr, nullptr, kv ? &kv[0] : nullptr, st,
+                                            nullptr, taps ? &taps[0] : nullptr, x));
     return cuda_status(mixer_sublayer(m, m.layers[l], D, P, P.h, n, nullptr, P.cs_n, nullptr,
                                       nullptr, nullptr, nullptr, kv ? &kv[l] : nullptr, st,
                                       nullptr, taps ? &taps[l] : nullptr));
