@@ -1108,12 +1108,23 @@ def gdn_bench(tg, torch, device, steps, warmup=3):
 
 
 def run_case(args):
-    """Small, repeatable invocations of one kernel family for ncu captures.
+    """Small, repeatable invocations of one kernel family: the commands that
+    the ncu summaries under profiles/ were captured with, and the timings
+    they quote. Not part of the default bench line.
 
-    attn:  tg_gated_attn_prefill over `rows` rows, Qwen3-1.7B heads (16/8 x 128),
-           gate bias on -- the attention kernel (plus its RoPE prep).
-    layer: tg_prefill of a 2-layer Qwen3-1.7B-shaped model, gate at layer 0,
-           N = rows, K = rows / 8 -- every GEMM epilogue, select and compact.
+    attn:     tg_gated_attn_prefill over `rows` rows, Qwen3-1.7B heads
+              (16/8 x 128), gate bias on (--no-bias: plain causal) -- the
+              attention kernel (plus its RoPE prep).
+    attn_bwd: tg_gated_attn_forward + tg_gated_attn_backward at those heads.
+    layer:    tg_prefill of a 2-layer Qwen3-1.7B-shaped model, gate at layer 0,
+              N = rows, K = rows / 8 -- every GEMM epilogue, select and compact.
+    gemm:     the prefill's projection shapes through tg_linear, next to
+              torch.matmul (cuBLAS) on the same operands, timed interleaved.
+    decode:   a 2-layer Qwen3-1.7B-shaped model gated at layer 0 (N = rows,
+              K = rows / 8, at least 128): prefill, then `steps` decode steps.
+    gdn:      the Gated DeltaNet mixer over `rows` kept tokens.
+    score:    tg_score over `rows` rows (d_model 2048, 256 hidden).
+    select:   tg_topk_select then tg_compact of `rows` sweep-style scores.
     """
     import torch
 
@@ -1260,7 +1271,9 @@ def main():
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--case", choices=["attn", "attn_bwd", "layer", "gemm", "decode", "gdn", "score",
                                        "select"],
-                    default=None)
+                    default=None,
+                    help="run one kernel family's small case (the profiles/ captures) instead "
+                         "of the bench line")
     ap.add_argument("--rows", type=int, default=32768)
     ap.add_argument("--no-bias", action="store_true",
                     help="attn case: plain causal attention (as the layers below the gate)")
