@@ -329,7 +329,8 @@ typedef struct {
    * The rounding differs from the norm-then-project order only in where one
    * bf16 rounding falls (on W g instead of on the normed row). NULL: the
    * RMSNorm kernel and the plain weights (also used for rows that were not
-   * just written by a residual GEMM: the stack's input, the compacted rows). */
+   * just written by a residual GEMM: the stack's input; the compaction
+   * carries the kept rows' sums of squares along, so they stay folded). */
   const void* wqkv_g;      /* [(hq + 2 hkv) dh, d] or NULL (unused with gdn)     */
   const void* w_gate_up_g; /* [2 I, d] or NULL                                   */
 } tg_layer;
@@ -368,7 +369,9 @@ typedef struct {
  * gate_layer = -1 puts the gate before layer 0 (the scorer reads x itself).
  * With k == n and every gain NULL/0 and tau NULL/1 the call is a dense
  * prefill.
- *   x [n, d] dtype (input hidden states); protect [n] uint8 or NULL
+ *   x [n, d] dtype (input hidden states, only read: layer 0 reads them in
+ *     place, so x must stay valid until the stream reaches the end of the
+ *     call's work); protect [n] uint8 or NULL
  *   out [k, d] dtype: final-normed hidden states of the kept rows
  *   kept_idx [k] int32 (out, ascending); scores [n] fp32 (out) or NULL
  *   kv: HOST array of n_layers tg_kv, or NULL (bf16: 16-byte aligned pointers)
